@@ -1,0 +1,489 @@
+"""Benchmark of the CSA / HCA attention forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload csa_prefill|hca_prefill|decode128k|decode1m]
+    python bench.py --impl reference ...   # the fp64 CPU oracle, timed on this host's cores
+
+A step is one full pass of the layer forward over one batch of synthetic inputs already resident
+in HBM: compress -> lightning indexer + top-k -> sparse + window attention for CSA prefill
+(the V4-Flash layer, S=8192), compress -> dense attention for HCA prefill (S=65536), and
+indexer + top-k -> attention for decode. Per-step CUDA events on the launching stream time
+every kernel phase; L2 is flushed (a 256 MiB write) between steps, outside the timed events.
+Multi-GPU runs are independent replicas (the path has no exchange step): every rank runs the same
+workload and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
+
+WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---- algorithmic work (flops / bytes the method needs, not what a kernel happens to do) ----------
+
+def csa_attention_flops(wl):
+    """4*D flops per (query, head, key): QK^T and PV over the full head dim."""
+    t = np.arange(wl.S, dtype=np.int64)
+    n_win = np.minimum(wl.W, t + 1)
+    vis = np.minimum((t + 1) // wl.m, wl.T)
+    n_sel = np.minimum(wl.topk, vis) if wl.kind == "csa_prefill" else vis
+    return float((n_win + n_sel).sum()) * wl.H * 4.0 * wl.D
+
+
+def index_flops(wl):
+    t = np.arange(wl.S, dtype=np.int64)
+    vis = np.minimum((t + 1) // wl.m, wl.T)
+    return float(vis.sum()) * 2.0 * wl.HI * wl.dI
+
+
+def attention_bytes(wl):
+    """Each tensor once: q in, o out (fp32), entries and window rows once."""
+    return wl.S * wl.H * wl.D * 2 + wl.S * wl.H * wl.D * 4 + wl.T * wl.D * 2 + wl.S * wl.D * 2
+
+
+def decode_bytes(wl, B):
+    """k^I stream + selected entries + window rows + q + o per step."""
+    T, D, r = wl.T, wl.D, wl.r
+    ent = (D - r) + 4 + 2 * r if wl.cache == "fp8" else 2 * D
+    per_seq = T * wl.dI * 2 + wl.topk * ent + wl.W * D * 2 + wl.H * D * 2 + wl.H * D * 4 + wl.HI * (wl.dI * 2 + 4)
+    return float(B * per_seq)
+
+
+# ---- clocks sampled during the timed region ------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, f in enumerate(fl) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "samples": len(rows), "reasons": reasons}
+
+
+# ---- the GPU arm ---------------------------------------------------------------------------------
+
+class Step:
+    """One workload's step, split into its kernel phases with events between them."""
+
+    def __init__(self, name, wl, csa, dev):
+        self.name, self.wl, self.csa, self.dev = name, wl, csa, dev
+        self.stream = torch.cuda.current_stream()
+        if wl.kind == "csa_decode":
+            self.B = wl.B
+            self.x = decode_inputs(wl, device=dev)
+            self.P = wl.ctx - 1
+            self.o = torch.empty(self.B, wl.H, wl.D, dtype=torch.float32, device=dev)
+            self.idx = torch.empty(self.B, wl.topk, dtype=torch.int32, device=dev)
+            self.ws = torch.empty(csa.workspace_size("decode", B=self.B, T=wl.T, k=wl.topk), dtype=torch.uint8,
+                                  device=dev)
+            self.phases = ["decode"]
+            self.units = self.B
+        else:
+            self.x = prefill_inputs(wl, device=dev)
+            S, T = wl.S, wl.T
+            self.C = torch.empty(T, wl.D, dtype=torch.bfloat16, device=dev)
+            self.kv_rot = torch.empty(S, wl.D, dtype=torch.bfloat16, device=dev)
+            self.o = torch.empty(S, wl.H, wl.D, dtype=torch.float32, device=dev)
+            if wl.kind == "csa_prefill":
+                self.idx = torch.empty(S, wl.topk, dtype=torch.int32, device=dev)
+                self.ws = torch.empty(csa.workspace_size("csa_forward", S=S, T=T), dtype=torch.uint8, device=dev)
+                self.phases = ["compress", "index_topk", "attend"]
+            else:
+                self.ws = torch.empty(csa.workspace_size("hca_forward"), dtype=torch.uint8, device=dev)
+                self.phases = ["compress", "attend"]
+            self.units = S
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
+
+    def launches_per_step(self):
+        # compress_entries + rotate_rows, index_scores + topk, attention
+        return {"csa_prefill": 5, "hca_prefill": 3, "csa_decode": 3}[self.wl.kind]
+
+    def run(self, timed: bool):
+        wl, x, csa = self.wl, self.x, self.csa
+        ev = self.events
+        if timed:
+            ev[0].record(self.stream)
+        if wl.kind == "csa_decode":
+            kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
+            csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], self.P, wl.topk, wl.r, wl.theta_tok,
+                       wl.theta_cmp, o=self.o, idx=self.idx, workspace=self.ws, **kw)
+            if timed:
+                ev[1].record(self.stream)
+            return
+        csa.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok, C=self.C,
+                     kv_rot=self.kv_rot)
+        if timed:
+            ev[1].record(self.stream)
+        if wl.kind == "csa_prefill":
+            csa.index_topk(x["qI"], x["kI"], x["w"], wl.m, wl.topk, idx=self.idx, workspace=self.ws)
+            if timed:
+                ev[2].record(self.stream)
+            csa.attend(x["q"], self.C, self.kv_rot, self.idx, x["sinks"], wl.m, wl.W, wl.r, wl.theta_tok,
+                       wl.theta_cmp, o=self.o, workspace=self.ws)
+            if timed:
+                ev[3].record(self.stream)
+        else:
+            csa.hca_attend(x["q"], self.C, self.kv_rot, x["sinks"], wl.m, wl.W, wl.r, wl.theta_tok, wl.theta_cmp,
+                           o=self.o, workspace=self.ws)
+            if timed:
+                ev[2].record(self.stream)
+
+    def phase_ms(self):
+        return [self.events[i].elapsed_time(self.events[i + 1]) for i in range(len(self.phases))]
+
+
+def e2e_run(step, steps, warmup):
+    """Same metric through the public fused call with host buffers: each step copies its inputs
+    from pinned host memory, runs the forward, and reads the output back."""
+    csa, wl, dev = step.csa, step.wl, step.dev
+    host = {k: v.cpu().pin_memory() for k, v in step.x.items()}
+    devbuf = {k: torch.empty_like(v) for k, v in step.x.items()}
+    o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o_host.numel() * o_host.element_size()
+    s = torch.cuda.current_stream()
+
+    def one():
+        for k in host:
+            devbuf[k].copy_(host[k], non_blocking=True)
+        x = devbuf
+        if wl.kind == "csa_prefill":
+            o, _, _, _ = csa.csa_forward(x["q"], x["kv"], x["gate"], x["pos_bias"], x["qI"], x["kI"], x["w"],
+                                         x["sinks"], wl.m, wl.L, wl.topk, wl.W, wl.r, wl.theta_tok, wl.theta_cmp,
+                                         out=(step.o, step.C, step.kv_rot, step.idx), workspace=step.ws)
+        elif wl.kind == "hca_prefill":
+            o, _, _ = csa.hca_forward(x["q"], x["kv"], x["gate"], x["pos_bias"], x["sinks"], wl.m, wl.L, wl.W, wl.r,
+                                      wl.theta_tok, wl.theta_cmp, out=(step.o, step.C, step.kv_rot), workspace=step.ws)
+        else:
+            kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
+            o, _ = csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], step.P, wl.topk, wl.r,
+                              wl.theta_tok, wl.theta_cmp, o=step.o, idx=step.idx, workspace=step.ws, **kw)
+        o_host.copy_(o, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        one()
+    e1.record(s)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del devbuf
+    return ms, h2d, d2h
+
+
+# ---- the oracle (CPU baseline and reference arm) -----------------------------------------------------
+
+def oracle_sample_rows(wl, n, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(wl.S, size=n, replace=False)).astype(np.int64)
+
+
+class OracleStep:
+    """The fp64 oracle on a bounded sample of the workload: prefill rows are independent once the
+    entries are pooled, so a sample of query rows (plus the pooling, amortised per token) measures
+    the oracle's per-token rate; decode samples whole sequences."""
+
+    def __init__(self, wl, target_s=4.0):
+        import oracle
+        self.oracle, self.wl = oracle, wl
+        if wl.kind == "csa_decode":
+            self.x = decode_inputs(wl, device="cpu", batch=1)
+            self.P = wl.ctx - 1
+        else:
+            self.x = prefill_inputs(wl, device="cpu")
+            t0 = time.perf_counter()
+            self.C, self.kvr = oracle.compress(self.x["kv"], self.x["gate"], self.x["pos_bias"], wl.m, wl.L, wl.r,
+                                               wl.theta_cmp, wl.theta_tok)
+            self.compress_s = time.perf_counter() - t0
+            t0 = time.perf_counter()
+            self._rows(oracle_sample_rows(wl, 2, seed=99))
+            per_row = (time.perf_counter() - t0) / 2
+            self.n = int(max(2, min(256, target_s / max(per_row, 1e-6))))
+        self.calls = 0
+
+    def _rows(self, rows):
+        wl, x, o = self.wl, self.x, self.oracle
+        if wl.kind == "csa_prefill":
+            ridx, _ = o.index_topk(x["qI"], x["kI"], x["w"], wl.m, wl.topk, rows=rows)
+            idx = np.full((wl.S, wl.topk), -1, np.int32)
+            idx[rows] = ridx
+        else:
+            idx = None
+        o.attend(x["q"], self.C, self.kvr, idx, x["sinks"], wl.m, wl.W, wl.r, wl.theta_tok, wl.theta_cmp, rows=rows)
+
+    def run(self):
+        """Returns (units, seconds) of one sampled step."""
+        wl, o, x = self.wl, self.oracle, self.x
+        self.calls += 1
+        t0 = time.perf_counter()
+        if wl.kind == "csa_decode":
+            ridx, _ = o.decode_index_topk(x["qI"], x["w"], x["kI"], wl.topk)
+            kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
+            o.decode_attend(x["q"], x["win"], ridx, x["sinks"], self.P, wl.r, wl.theta_tok, wl.theta_cmp, **kw)
+            return 1, time.perf_counter() - t0
+        rows = oracle_sample_rows(wl, self.n, seed=self.calls)
+        self._rows(rows)
+        dt = time.perf_counter() - t0 + self.compress_s * self.n / wl.S    # pooling amortised per token
+        return self.n, dt
+
+    def sample_desc(self):
+        if self.wl.kind == "csa_decode":
+            return f"1 of {self.wl.B} sequences per step (full index scan over T={self.wl.T} + attention)"
+        return (f"{self.n} random query rows of S={self.wl.S} per step (index + top-k + attention per row) "
+                f"plus the full pooling amortised per token")
+
+
+def unit_name(wl):
+    return "queries/s" if wl.kind == "csa_decode" else "tokens/s"
+
+
+def metric_name(wl):
+    return {"csa_prefill": "csa_prefill_tokens_per_s", "hca_prefill": "hca_prefill_tokens_per_s",
+            "csa_decode": "csa_decode_queries_per_s"}[wl.kind]
+
+
+def config_of(wl, n_gpus):
+    c = {"workload": wl.name, "S": wl.S, "H": wl.H, "D": wl.D, "m": wl.m, "window_L": wl.L, "W": wl.W,
+         "rope_dim": wl.r, "theta_tok": wl.theta_tok, "theta_cmp": wl.theta_cmp, "parallelism": f"replicas{n_gpus}",
+         "l2": "flushed between steps (256 MiB write outside the timed events)"}
+    if wl.kind == "csa_decode":
+        c.update({"B": wl.B, "ctx": wl.ctx, "T": wl.T, "topk": wl.topk, "index": f"{wl.HI}x{wl.dI}",
+                  "cache": wl.cache})
+        del c["S"]
+    elif wl.kind == "csa_prefill":
+        c.update({"topk": wl.topk, "index": f"{wl.HI}x{wl.dI}", "T": wl.T})
+    else:
+        c.update({"T": wl.T})
+    return c
+
+
+def reference_arm(args, wl, rank, world):
+    if rank != 0:
+        return 0
+    threads = None
+    try:
+        import oracle
+        threads = oracle.num_threads()
+        st = OracleStep(wl)
+        for _ in range(args.warmup):
+            st.run()
+        units = secs = 0.0
+        for _ in range(args.steps):
+            u, s = st.run()
+            units += u
+            secs += s
+    except Exception as e:  # the oracle is plain C; a failure here is a build problem
+        print(json.dumps({"impl": "reference", "unavailable": f"oracle failed: {e}"}))
+        return 0
+    v = units / secs
+    line = {"impl": "reference", "metric": metric_name(wl), "value": v, "unit": unit_name(wl), "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(wl, world),
+            "cpu_baseline": {"value": v, "unit": unit_name(wl), "cores": threads, "kind": "oracle",
+                             "sample": st.sample_desc()},
+            "e2e": {"value": v, "unit": unit_name(wl), "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def cpu_baseline(wl):
+    import oracle
+    st = OracleStep(wl, target_s=6.0)
+    units = secs = 0.0
+    t_end = time.perf_counter() + 15.0
+    while True:
+        u, s = st.run()
+        units += u
+        secs += s
+        if time.perf_counter() > t_end:
+            break
+    return {"value": units / secs, "unit": unit_name(wl), "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": st.sample_desc() + f"; {st.calls} steps"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="csa_prefill", choices=sorted(WORKLOAD_IDS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[WORKLOAD_IDS[args.workload]]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, wl, rank, world)
+
+    import long_context_sparse_fwd_b200 as csa
+    csa.lib()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    step = Step(args.workload, wl, csa, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(max(3, args.warmup)):
+        step.run(False)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    phase_ms = []
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1)
+            step.run(True)
+            torch.cuda.synchronize()
+            phase_ms.append(step.phase_ms())
+    torch.cuda.synchronize()
+    barrier()
+    phase_ms = np.array(phase_ms)                        # [steps, phases]
+    total_ms = float(phase_ms.sum())
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    units = step.units * args.steps * world
+    value = units / (total_ms / 1e3)
+
+    peaks, peak_src = load_peaks()
+    mean_phase = phase_ms.mean(0)
+    dom = int(np.argmax(mean_phase))
+    dom_name = step.phases[dom]
+    if wl.kind == "csa_decode":
+        alg = decode_bytes(wl, step.B)
+        roof = {"bound": "hbm", "kernel": "csa_decode (index scan + top-k + attention)",
+                "achieved": alg / (mean_phase[dom] / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    elif dom_name == "attend":
+        alg = csa_attention_flops(wl)
+        roof = {"bound": "tensor", "kernel": "attention", "achieved": alg / (mean_phase[dom] / 1e3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    elif dom_name == "index_topk":
+        alg = index_flops(wl)
+        roof = {"bound": "tensor", "kernel": "index_topk", "achieved": alg / (mean_phase[dom] / 1e3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        alg = float(wl.S * wl.D * 2 * 3 + wl.T * wl.D * 2)
+        roof = {"bound": "hbm", "kernel": "compress", "achieved": alg / (mean_phase[dom] / 1e3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling fallback'})"
+    roof["traffic"] = None
+    roof["ms_per_launch"] = float(mean_phase[dom])
+
+    e2e = None
+    if not args.no_e2e:
+        ms, h2d, d2h = e2e_run(step, max(2, args.steps // 2), 1)
+        te = torch.tensor([ms], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        n_e2e = max(2, args.steps // 2)
+        e2e = {"value": step.units * n_e2e * world / (float(te.item()) / 1e3), "unit": unit_name(wl),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    line = {
+        "metric": metric_name(wl), "value": value, "unit": unit_name(wl), "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate/out", "data": "synthetic",
+        "config": config_of(wl, world),
+        "phases_ms": {n: float(v) for n, v in zip(step.phases, mean_phase)},
+        "roofline": roof, "e2e": e2e, "gpu_launches": step.launches_per_step() * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

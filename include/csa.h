@@ -1,0 +1,174 @@
+/*
+ * csa.h -- C ABI of the B200 (sm_100a) DeepSeek-V4 hybrid-attention forward: Compressed Sparse
+ * Attention (CSA) and Heavily Compressed Attention (HCA), prefill and decode.
+ *
+ * Sources for what each call computes:
+ *   [HF-V4]   Hugging Face Transformers docs, "DeepSeek-V4", sections "Hybrid attention (§2.3)"
+ *             and "Attention mask layout";
+ *   [digest]  insight.ai.kr digest of the Hugging Face DeepSeek-V4 blog post (softmax-gated
+ *             pooling with a learned position bias; ReLU multi-head lightning indexer; FP8 KV
+ *             with BF16 RoPE dims);
+ *   [atlas]   llm-atlas "DeepSeek-V4-Flash", table "config.json full fields" (head_dim 512,
+ *             64 heads, 1 KV head, qk_rope_head_dim 64, index 64 x 128, index_topk 512,
+ *             sliding_window 128, rope_theta 10000, compress_rope_theta 160000).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates and
+ *     frees nothing. Layouts are dense row-major with the shapes given. bf16 tensors are passed
+ *     as void* (IEEE bfloat16 bit patterns), FP8 as uint8 E4M3 codes (OCP definition).
+ *   - Base pointers must be 16-byte aligned; D, d_I and rope_dim as documented per call.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Argument checks run on the host
+ *     before anything is launched; a failed check returns its status and launches nothing.
+ *     Kernels run asynchronously in stream order; launch failures return CSA_ERR_CUDA.
+ *   - `workspace` (device, caller-owned, size from csa_workspace_size) starts with a status word.
+ *     Each call that takes a workspace zeroes it in stream order, then kernels record data errors
+ *     found on the device (for example an index that is out of range or not yet visible; such a
+ *     key is skipped). Read it with csa_get_device_status after the call.
+ *   - Calls on the same workspace must not overlap on the GPU.
+ *   - Nothing here aborts, traps or asserts on the device.
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum csa_status {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, misalignment, bad index data found on device */
+    CSA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement (e.g. D % 8 != 0) */
+    CSA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    CSA_ERR_TIMEOUT = 4,      /* a bounded device-side wait expired */
+    CSA_ERR_WORKSPACE = 5     /* workspace missing or smaller than csa_workspace_size() */
+} csa_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+CSA_API const char *csa_status_str(csa_status s);
+
+/* Library version string. */
+CSA_API const char *csa_version(void);
+
+/* ---- workspace sizing ------------------------------------------------------------------------ */
+
+typedef enum csa_op {
+    CSA_OP_INDEX_TOPK = 1,
+    CSA_OP_ATTEND = 2,        /* csa_attend and hca_attend */
+    CSA_OP_CSA_FORWARD = 3,
+    CSA_OP_HCA_FORWARD = 4,
+    CSA_OP_DECODE = 5
+} csa_op;
+
+typedef struct csa_dims {
+    int64_t S;      /* prefill tokens */
+    int64_t T;      /* compressed entries (prefill: floor(S/m); decode: per sequence) */
+    int32_t B;      /* decode sequences */
+    int32_t H, D;   /* query heads, head dim */
+    int32_t HI, dI; /* index heads, index head dim */
+    int32_t k;      /* top-k */
+    int32_t W;      /* sliding window */
+} csa_dims;
+
+/* Bytes of device workspace `op` needs for `dims` (>= 256; the first 256 bytes hold the status word). */
+CSA_API size_t csa_workspace_size(csa_op op, const csa_dims *dims);
+
+/* Copies the status word of `workspace` to *status after synchronizing `stream`. */
+CSA_API csa_status csa_get_device_status(const void *workspace, int32_t *status, void *stream);
+
+/* ---- 1. compressor ------------------------------------------------------------------------------
+ * [HF-V4 "Hybrid attention"; digest]. Entry w (0 <= w < T = floor(S/m)) pools the window
+ * [(w+1)m - L, (w+1)m) clipped to [0,S): per channel d, softmax over positions j of
+ * gate[j,d] + pos_bias[j - ((w+1)m - L)], weights applied to kv[j,d]. CSA: L = 2m (overlapping),
+ * HCA: L = m. The entry is then RoPE-rotated at position w*m with theta_cmp on its last rope_dim
+ * channels (interleaved pairs). kv_rot[j] = kv[j] rotated at position j with theta_tok.
+ *   kv, gate   [S, D] bf16            pos_bias [L] fp32
+ *   C          [T, D] bf16 (out)      kv_rot   [S, D] bf16 (out, may be NULL)
+ * Requires D % 8 == 0, rope_dim even, rope_dim % 8 == 0, rope_dim <= D, 1 <= m <= L <= 4096. */
+CSA_API csa_status csa_compress(const void *kv, const void *gate, const float *pos_bias,
+                        int64_t S, int32_t D, int32_t m, int32_t L, int32_t rope_dim,
+                        double theta_cmp, double theta_tok,
+                        void *C, void *kv_rot, void *stream);
+
+/* ---- 2. lightning indexer + top-k (prefill) ----------------------------------------------------
+ * [HF-V4 "Hybrid attention", CSA; "Attention mask layout", CSA layer; digest].
+ * I[t,s] = sum_h w[t,h] * ReLU(qI[t,h,:] . kI[s,:]) for visible entries s < floor((t+1)/m);
+ * idx[t] = the min(k, vis) largest, ties to the smaller s, written in ascending index order,
+ * remaining slots -1.
+ *   qI [S, HI, dI] bf16   kI [T, dI] bf16   w [S, HI] fp32   idx [S, k] int32 (out)
+ * Requires dI % 8 == 0, 1 <= k. */
+CSA_API csa_status csa_index_topk(const void *qI, const void *kI, const float *w,
+                          int64_t S, int64_t T, int32_t HI, int32_t dI, int32_t m, int32_t k,
+                          int32_t *idx, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---- 3. sparse + window attention (CSA prefill) ---------------------------------------------
+ * [HF-V4 "Hybrid attention": shared K=V MQA, partial interleaved RoPE, output rope slice rotated
+ * at -i (eq. 26), per-head sink (eq. 27), sliding-window branch; "Attention mask layout"].
+ * For query t, head h: keys = kv_rot[j] for j in [t-W+1, t] (window) plus C[s] for s in idx[t]
+ * (s != -1). Logits lambda*(R_tok(t) q).kv_rot[j] and lambda*(R_cmp(t) q).C[s]; one softmax over
+ * all keys plus exp(sinks[h]); K = V; each branch's rope slice rotated back by -t with its theta.
+ *   q [S, H, D] bf16 (un-rotated)   C [T, D] bf16 (post-RoPE)   kv_rot [S, D] bf16 (post-RoPE)
+ *   idx [S, k] int32                sinks [H] fp32               o [S, H, D] fp32 (out)
+ * softmax_scale <= 0 selects 1/sqrt(D). Index values >= floor((t+1)/m) are skipped and reported
+ * as CSA_ERR_INVALID_ARG in the workspace status. */
+CSA_API csa_status csa_attend(const void *q, const void *C, const void *kv_rot, const int32_t *idx,
+                      const float *sinks, int64_t S, int32_t H, int32_t D, int64_t T, int32_t k,
+                      int32_t W, int32_t rope_dim, int32_t m, double theta_tok, double theta_cmp,
+                      float softmax_scale, float *o, void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+/* ---- 4. dense compressed + window attention (HCA prefill) --------------------------------------
+ * [HF-V4 "Hybrid attention", HCA; "Attention mask layout", HCA layer]. As csa_attend with the
+ * entry branch = every visible entry C[w], w < floor((t+1)/m). */
+CSA_API csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const float *sinks,
+                      int64_t S, int32_t H, int32_t D, int64_t T, int32_t W, int32_t rope_dim,
+                      int32_t m, double theta_tok, double theta_cmp, float softmax_scale, float *o,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---- 5. fused layer forward ----------------------------------------------------------------------
+ * csa_forward = csa_compress (L = 2m) -> csa_index_topk -> csa_attend, in stream order.
+ * hca_forward = csa_compress (L = m)  -> hca_attend. Intermediates C, kv_rot, idx are
+ * caller-provided outputs (kv_rot and C are needed by later decode steps as cache). */
+CSA_API csa_status csa_forward(const void *q, const void *kv, const void *gate, const float *pos_bias,
+                       const void *qI, const void *kI, const float *w, const float *sinks,
+                       int64_t S, int32_t H, int32_t D, int32_t HI, int32_t dI, int32_t m, int32_t L,
+                       int32_t k, int32_t W, int32_t rope_dim, double theta_tok, double theta_cmp,
+                       float softmax_scale, void *C, void *kv_rot, int32_t *idx, float *o,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+CSA_API csa_status hca_forward(const void *q, const void *kv, const void *gate, const float *pos_bias,
+                       const float *sinks, int64_t S, int32_t H, int32_t D, int32_t m, int32_t L,
+                       int32_t W, int32_t rope_dim, double theta_tok, double theta_cmp,
+                       float softmax_scale, void *C, void *kv_rot, float *o,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---- 6. CSA decode ---------------------------------------------------------------------------------
+ * One new query per sequence at position P against post-RoPE caches; every one of the T entries
+ * is visible. Indexer + top-k over all T entries, then the attention of csa_attend for row P.
+ *   q [B, H, D] bf16 (un-rotated)   qI [B, HI, dI] bf16   w [B, HI] fp32   kI [B, T, dI] bf16
+ *   entries: C [B, T, D] bf16, or (C == NULL) the FP8 cache of [digest] as three arrays:
+ *            c8 [B, T, D-rope_dim] E4M3 codes, c8_scale [B, T] fp32, c_rope [B, T, rope_dim] bf16;
+ *            value = e4m3(c8) * scale on channels [0, D-rope_dim), c_rope on the rest
+ *   win [B, W, D] bf16: window rows for positions P-W+1 .. P (rows at negative positions ignored)
+ *   sinks [H] fp32    idx_out [B, k] int32 (out, may be NULL)    o [B, H, D] fp32 (out) */
+CSA_API csa_status csa_decode(const void *q, const void *qI, const float *w, const void *kI,
+                      const void *C, const uint8_t *c8, const float *c8_scale, const void *c_rope,
+                      const void *win, const float *sinks, int32_t B, int32_t H, int32_t D,
+                      int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W, int32_t rope_dim,
+                      int64_t P, double theta_tok, double theta_cmp, float softmax_scale,
+                      int32_t *idx_out, float *o, void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_B200_H */

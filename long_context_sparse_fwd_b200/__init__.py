@@ -1,0 +1,268 @@
+"""Python binding of the sm_100a CSA / HCA attention library (libcsa.so, C ABI in include/csa.h).
+
+Argument marshalling only: every step of the forward runs in the library's CUDA kernels. PyTorch
+provides device memory and the current stream. There is no CPU path: if the library is missing
+or the tensors are not on a CUDA device the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "CSAError", "lib", "library_path", "compress", "index_topk", "attend", "hca_attend", "csa_forward",
+    "hca_forward", "decode", "workspace_size", "get_device_status", "OP",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libcsa.so")
+_lib = None
+
+OP = {"index_topk": 1, "attend": 2, "csa_forward": 3, "hca_forward": 4, "decode": 5}
+_STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
+           4: "CSA_ERR_TIMEOUT", 5: "CSA_ERR_WORKSPACE"}
+
+
+class CSAError(RuntimeError):
+    def __init__(self, call: str, code: int):
+        super().__init__(f"{call} failed: {_STATUS.get(code, code)}")
+        self.code = code
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("S", ctypes.c_int64), ("T", ctypes.c_int64), ("B", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("D", ctypes.c_int32), ("HI", ctypes.c_int32), ("dI", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("W", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libcsa.so (built by ``build.build()``); raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {_LIB_PATH} is missing (run __graft_entry__.build())")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I64, I32, F64, F32, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_double,
+                                     ctypes.c_float, ctypes.c_size_t)
+        sig = {
+            "csa_status_str": (ctypes.c_char_p, [I32]),
+            "csa_version": (ctypes.c_char_p, []),
+            "csa_workspace_size": (SZ, [I32, ctypes.POINTER(_Dims)]),
+            "csa_get_device_status": (I32, [P, ctypes.POINTER(ctypes.c_int32), P]),
+            "csa_compress": (I32, [P, P, P, I64, I32, I32, I32, I32, F64, F64, P, P, P]),
+            "csa_index_topk": (I32, [P, P, P, I64, I64, I32, I32, I32, I32, P, P, SZ, P]),
+            "csa_attend": (I32, [P, P, P, P, P, I64, I32, I32, I64, I32, I32, I32, I32, F64, F64, F32, P, P,
+                                 SZ, P]),
+            "hca_attend": (I32, [P, P, P, P, I64, I32, I32, I64, I32, I32, I32, F64, F64, F32, P, P, SZ, P]),
+            "csa_forward": (I32, [P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, I32, I32, I32, I32, F64,
+                                  F64, F32, P, P, P, P, P, SZ, P]),
+            "hca_forward": (I32, [P, P, P, P, P, I64, I32, I32, I32, I32, I32, I32, F64, F64, F32, P, P, P, P,
+                                  SZ, P]),
+            "csa_decode": (I32, [P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, I32, I64,
+                                 F64, F64, F32, P, P, P, SZ, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ---- marshalling ----------------------------------------------------------------------------------
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: Optional[torch.Tensor], dtype, name: str, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(call: str, code: int):
+    if code != 0:
+        raise CSAError(call, code)
+
+
+def workspace_size(op: str, S=0, T=0, B=0, H=0, D=0, HI=0, dI=0, k=0, W=0) -> int:
+    d = _Dims(S, T, B, H, D, HI, dI, k, W)
+    return int(lib().csa_workspace_size(OP[op], ctypes.byref(d)))
+
+
+def _workspace(op: str, device, ws: Optional[torch.Tensor], **dims) -> torch.Tensor:
+    need = workspace_size(op, **dims)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    elif ws.numel() < need:
+        raise ValueError(f"workspace of {ws.numel()} bytes is smaller than the {need} bytes needed")
+    return ws
+
+
+def get_device_status(ws: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_int32(0)
+    _check("csa_get_device_status", lib().csa_get_device_status(_ptr(ws), ctypes.byref(v), _stream(stream)))
+    return int(v.value)
+
+
+# ---- the calls ----------------------------------------------------------------------------------------
+
+def compress(kv, gate, pos_bias, m: int, L: int, rope_dim: int, theta_cmp: float, theta_tok: float,
+             C=None, kv_rot=None, want_kv_rot: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    S, D = kv.shape
+    T = S // m
+    _dev(kv, torch.bfloat16, "kv", (S, D))
+    _dev(gate, torch.bfloat16, "gate", (S, D))
+    _dev(pos_bias, torch.float32, "pos_bias", (L,))
+    C = torch.empty(T, D, dtype=torch.bfloat16, device=kv.device) if C is None else _dev(C, torch.bfloat16, "C", (T, D))
+    if want_kv_rot:
+        kv_rot = torch.empty_like(kv) if kv_rot is None else _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+    else:
+        kv_rot = None
+    _check("csa_compress", lib().csa_compress(_ptr(kv), _ptr(gate), _ptr(pos_bias), S, D, m, L, rope_dim,
+                                              float(theta_cmp), float(theta_tok), _ptr(C), _ptr(kv_rot),
+                                              _stream(stream)))
+    return C, kv_rot
+
+
+def index_topk(qI, kI, w, m: int, k: int, idx=None, workspace=None, stream=None) -> torch.Tensor:
+    S, HI, dI = qI.shape
+    T = kI.shape[0]
+    _dev(qI, torch.bfloat16, "qI")
+    _dev(kI, torch.bfloat16, "kI", (T, dI))
+    _dev(w, torch.float32, "w", (S, HI))
+    idx = torch.empty(S, k, dtype=torch.int32, device=qI.device) if idx is None else _dev(idx, torch.int32, "idx", (S, k))
+    ws = _workspace("index_topk", qI.device, workspace, S=S, T=T)
+    _check("csa_index_topk", lib().csa_index_topk(_ptr(qI), _ptr(kI), _ptr(w), S, T, HI, dI, m, k, _ptr(idx),
+                                                  _ptr(ws), ws.numel(), _stream(stream)))
+    return idx
+
+
+def attend(q, C, kv_rot, idx, sinks, m: int, W: int, rope_dim: int, theta_tok: float, theta_cmp: float,
+           softmax_scale: float = 0.0, o=None, workspace=None, stream=None) -> torch.Tensor:
+    S, H, D = q.shape
+    T = C.shape[0]
+    k = idx.shape[1]
+    _dev(q, torch.bfloat16, "q")
+    _dev(C, torch.bfloat16, "C", (T, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+    _dev(idx, torch.int32, "idx", (S, k))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
+    ws = _workspace("attend", q.device, workspace)
+    _check("csa_attend", lib().csa_attend(_ptr(q), _ptr(C), _ptr(kv_rot), _ptr(idx), _ptr(sinks), S, H, D, T, k, W,
+                                          rope_dim, m, float(theta_tok), float(theta_cmp), float(softmax_scale),
+                                          _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def hca_attend(q, C, kv_rot, sinks, m: int, W: int, rope_dim: int, theta_tok: float, theta_cmp: float,
+               softmax_scale: float = 0.0, o=None, workspace=None, stream=None) -> torch.Tensor:
+    S, H, D = q.shape
+    T = C.shape[0]
+    _dev(q, torch.bfloat16, "q")
+    _dev(C, torch.bfloat16, "C", (T, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
+    ws = _workspace("attend", q.device, workspace)
+    _check("hca_attend", lib().hca_attend(_ptr(q), _ptr(C), _ptr(kv_rot), _ptr(sinks), S, H, D, T, W, rope_dim, m,
+                                          float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(o),
+                                          _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def csa_forward(q, kv, gate, pos_bias, qI, kI, w, sinks, m: int, L: int, k: int, W: int, rope_dim: int,
+                theta_tok: float, theta_cmp: float, softmax_scale: float = 0.0, out=None, workspace=None,
+                stream=None):
+    """Returns (o, C, kv_rot, idx). `out` may pass preallocated (o, C, kv_rot, idx)."""
+    S, H, D = q.shape
+    HI, dI = qI.shape[1], qI.shape[2]
+    T = S // m
+    for t, n, dt in ((q, "q", torch.bfloat16), (kv, "kv", torch.bfloat16), (gate, "gate", torch.bfloat16),
+                     (pos_bias, "pos_bias", torch.float32), (qI, "qI", torch.bfloat16), (kI, "kI", torch.bfloat16),
+                     (w, "w", torch.float32), (sinks, "sinks", torch.float32)):
+        _dev(t, dt, n)
+    if out is None:
+        dev = q.device
+        out = (torch.empty(S, H, D, dtype=torch.float32, device=dev), torch.empty(T, D, dtype=torch.bfloat16, device=dev),
+               torch.empty(S, D, dtype=torch.bfloat16, device=dev), torch.empty(S, k, dtype=torch.int32, device=dev))
+    o, C, kv_rot, idx = out
+    ws = _workspace("csa_forward", q.device, workspace, S=S, T=T)
+    _check("csa_forward", lib().csa_forward(_ptr(q), _ptr(kv), _ptr(gate), _ptr(pos_bias), _ptr(qI), _ptr(kI), _ptr(w),
+                                            _ptr(sinks), S, H, D, HI, dI, m, L, k, W, rope_dim, float(theta_tok),
+                                            float(theta_cmp), float(softmax_scale), _ptr(C), _ptr(kv_rot), _ptr(idx),
+                                            _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, C, kv_rot, idx
+
+
+def hca_forward(q, kv, gate, pos_bias, sinks, m: int, L: int, W: int, rope_dim: int, theta_tok: float,
+                theta_cmp: float, softmax_scale: float = 0.0, out=None, workspace=None, stream=None):
+    """Returns (o, C, kv_rot)."""
+    S, H, D = q.shape
+    T = S // m
+    for t, n, dt in ((q, "q", torch.bfloat16), (kv, "kv", torch.bfloat16), (gate, "gate", torch.bfloat16),
+                     (pos_bias, "pos_bias", torch.float32), (sinks, "sinks", torch.float32)):
+        _dev(t, dt, n)
+    if out is None:
+        dev = q.device
+        out = (torch.empty(S, H, D, dtype=torch.float32, device=dev), torch.empty(T, D, dtype=torch.bfloat16, device=dev),
+               torch.empty(S, D, dtype=torch.bfloat16, device=dev))
+    o, C, kv_rot = out
+    ws = _workspace("hca_forward", q.device, workspace)
+    _check("hca_forward", lib().hca_forward(_ptr(q), _ptr(kv), _ptr(gate), _ptr(pos_bias), _ptr(sinks), S, H, D, m, L,
+                                            W, rope_dim, float(theta_tok), float(theta_cmp), float(softmax_scale),
+                                            _ptr(C), _ptr(kv_rot), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, C, kv_rot
+
+
+def decode(q, qI, w, kI, win, sinks, P: int, k: int, rope_dim: int, theta_tok: float, theta_cmp: float,
+           C=None, c8=None, c8_scale=None, c_rope=None, softmax_scale: float = 0.0, o=None, idx=None,
+           workspace=None, stream=None):
+    """Returns (o [B,H,D] fp32, idx [B,k] int32)."""
+    B, H, D = q.shape
+    HI, dI = qI.shape[1], qI.shape[2]
+    T = kI.shape[1]
+    W = win.shape[1]
+    _dev(q, torch.bfloat16, "q")
+    _dev(qI, torch.bfloat16, "qI")
+    _dev(w, torch.float32, "w", (B, HI))
+    _dev(kI, torch.bfloat16, "kI", (B, T, dI))
+    _dev(win, torch.bfloat16, "win", (B, W, D))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    if C is not None:
+        _dev(C, torch.bfloat16, "C", (B, T, D))
+    else:
+        _dev(c8, torch.uint8, "c8", (B, T, D - rope_dim))
+        _dev(c8_scale, torch.float32, "c8_scale", (B, T))
+        _dev(c_rope, torch.bfloat16, "c_rope", (B, T, rope_dim))
+    o = torch.empty(B, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (B, H, D))
+    idx = torch.empty(B, k, dtype=torch.int32, device=q.device) if idx is None else _dev(idx, torch.int32, "idx", (B, k))
+    ws = _workspace("decode", q.device, workspace, B=B, T=T, k=k)
+    _check("csa_decode", lib().csa_decode(_ptr(q), _ptr(qI), _ptr(w), _ptr(kI), _ptr(C), _ptr(c8), _ptr(c8_scale),
+                                          _ptr(c_rope), _ptr(win), _ptr(sinks), B, H, D, T, HI, dI, k, W, rope_dim,
+                                          int(P), float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(idx),
+                                          _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, idx

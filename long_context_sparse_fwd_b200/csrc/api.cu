@@ -1,0 +1,345 @@
+// api.cu -- the C ABI declared in include/csa.h: host-side argument checks, workspace layout and
+// launch sequencing. Nothing here allocates device memory; every buffer is the caller's.
+#include <math.h>
+#include <string.h>
+
+#include "kernels.cuh"
+
+
+using namespace csa;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline csa_status from_cuda(cudaError_t e)
+{
+    return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
+#define CSA_CHECK_ARG(cond)                \
+    do {                                   \
+        if (!(cond)) return CSA_ERR_INVALID_ARG; \
+    } while (0)
+#define CSA_CHECK_SUP(cond)                \
+    do {                                   \
+        if (!(cond)) return CSA_ERR_UNSUPPORTED; \
+    } while (0)
+#define CSA_TRY(expr)                                   \
+    do {                                                \
+        csa_status _s = (expr);                         \
+        if (_s != CSA_OK) return _s;                    \
+    } while (0)
+#define CSA_CUDA(expr)                                  \
+    do {                                                \
+        if ((expr) != cudaSuccess) return CSA_ERR_CUDA; \
+    } while (0)
+
+inline bool theta_ok(double th) { return isfinite(th) && th > 1.0; }
+
+size_t scores_bytes(int64_t R, int64_t T) { return align256(sizeof(float) * (size_t)R * (size_t)T); }
+
+csa_status check_workspace(void *ws, size_t bytes, size_t need)
+{
+    if (ws == nullptr || bytes < need) return CSA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return CSA_ERR_INVALID_ARG;
+    return CSA_OK;
+}
+
+csa_status reset_status(void *ws, cudaStream_t stream)
+{
+    CSA_CUDA(cudaMemsetAsync(ws, 0, sizeof(int32_t), stream));
+    return CSA_OK;
+}
+
+csa_status check_compress(const void *kv, const void *gate, const float *pos_bias, int64_t S, int32_t D, int32_t m,
+                          int32_t L, int32_t r, double theta_cmp, double theta_tok, const void *C)
+{
+    CSA_CHECK_ARG(S >= 0 && D > 0 && m >= 1 && L >= m && r >= 0 && r <= D && (r % 2) == 0);
+    CSA_CHECK_ARG(S == 0 || (kv != nullptr && gate != nullptr && pos_bias != nullptr));
+    CSA_CHECK_ARG(S / m == 0 || C != nullptr);
+    CSA_CHECK_ARG(r == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_SUP(D % 8 == 0 && r % 8 == 0 && L <= 4096);
+    CSA_CHECK_ARG(aligned16(kv) && aligned16(gate) && aligned16(C));
+    return CSA_OK;
+}
+
+csa_status check_attend_common(const void *q, const void *C, const void *kv_rot, const float *sinks, int64_t S,
+                               int32_t H, int32_t D, int64_t T, int32_t W, int32_t r, int32_t m, double theta_tok,
+                               double theta_cmp, const float *o)
+{
+    CSA_CHECK_ARG(S >= 0 && H > 0 && D > 0 && T >= 0 && W >= 0 && m >= 1 && r >= 0 && r <= D && (r % 2) == 0);
+    CSA_CHECK_ARG(T <= S / m);
+    CSA_CHECK_ARG(S == 0 || (q != nullptr && sinks != nullptr && o != nullptr));
+    CSA_CHECK_ARG(S == 0 || W == 0 || kv_rot != nullptr);
+    CSA_CHECK_ARG(T == 0 || C != nullptr);
+    CSA_CHECK_ARG(r == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_SUP(D == 64 || D == 128 || D == 256 || D == 512);
+    CSA_CHECK_SUP(r % 8 == 0);
+    CSA_CHECK_ARG(aligned16(q) && aligned16(C) && aligned16(kv_rot) && aligned16(o));
+    return CSA_OK;
+}
+
+AttnArgs prefill_args(const void *q, const void *C, const void *kv_rot, const int32_t *idx, const float *sinks,
+                      int64_t S, int32_t H, int32_t D, int64_t T, int32_t k, int32_t W, int32_t r, int32_t m,
+                      double theta_tok, double theta_cmp, float scale, float *o, void *ws)
+{
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = static_cast<const uint16_t *>(q);
+    a.win = static_cast<const uint16_t *>(kv_rot);
+    a.C = static_cast<const uint16_t *>(C);
+    a.idx = idx;
+    a.sinks = sinks;
+    a.o = o;
+    a.status = static_cast<int32_t *>(ws);
+    a.R = S;
+    a.T = T;
+    a.H = H;
+    a.D = D;
+    a.k = k;
+    a.W = W;
+    a.r = r;
+    a.m = m;
+    a.scale = scale > 0.f ? scale : (float)(1.0 / sqrt((double)D));
+    a.log2_theta_tok = r > 0 ? log2(theta_tok) : 0.0;
+    a.log2_theta_cmp = r > 0 ? log2(theta_cmp) : 0.0;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *csa_status_str(csa_status s)
+{
+    switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT";
+    case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
+    }
+    return "CSA_ERR_UNKNOWN";
+}
+
+const char *csa_version(void) { return "csa-b200 0.1 (sm_100a)"; }
+
+size_t csa_workspace_size(csa_op op, const csa_dims *d)
+{
+    if (d == nullptr) return 0;
+    switch (op) {
+    case CSA_OP_INDEX_TOPK:
+    case CSA_OP_CSA_FORWARD:
+        return kStatusBytes + scores_bytes(d->S, d->T);
+    case CSA_OP_ATTEND:
+    case CSA_OP_HCA_FORWARD:
+        return kStatusBytes;
+    case CSA_OP_DECODE:
+        return kStatusBytes + scores_bytes(d->B, d->T) + align256(sizeof(int32_t) * (size_t)d->B * (size_t)d->k);
+    }
+    return 0;
+}
+
+csa_status csa_get_device_status(const void *workspace, int32_t *status, void *stream)
+{
+    CSA_CHECK_ARG(workspace != nullptr && status != nullptr);
+    int32_t v = 0;
+    CSA_CUDA(cudaMemcpyAsync(&v, workspace, sizeof v, cudaMemcpyDeviceToHost, as_stream(stream)));
+    CSA_CUDA(cudaStreamSynchronize(as_stream(stream)));
+    *status = v;
+    return CSA_OK;
+}
+
+csa_status csa_compress(const void *kv, const void *gate, const float *pos_bias, int64_t S, int32_t D, int32_t m,
+                        int32_t L, int32_t rope_dim, double theta_cmp, double theta_tok, void *C, void *kv_rot,
+                        void *stream)
+{
+    CSA_TRY(check_compress(kv, gate, pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    CSA_CHECK_ARG(aligned16(kv_rot));
+    return from_cuda(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate),
+                                     pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok,
+                                     static_cast<uint16_t *>(C), static_cast<uint16_t *>(kv_rot), as_stream(stream)));
+}
+
+csa_status csa_index_topk(const void *qI, const void *kI, const float *w, int64_t S, int64_t T, int32_t HI,
+                          int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace, size_t workspace_bytes,
+                          void *stream)
+{
+    CSA_CHECK_ARG(S >= 0 && T >= 0 && HI > 0 && dI > 0 && m >= 1 && k >= 1);
+    CSA_CHECK_ARG(T <= S / m);
+    CSA_CHECK_ARG(S == 0 || (qI != nullptr && w != nullptr && idx != nullptr));
+    CSA_CHECK_ARG(T == 0 || kI != nullptr);
+    CSA_CHECK_SUP(dI == 32 || dI == 64 || dI == 128 || dI == 256);
+    CSA_CHECK_SUP(HI <= 128 && (size_t)HI * dI * 4 <= 160 * 1024);
+    CSA_CHECK_ARG(aligned16(qI) && aligned16(kI));
+    csa_dims dims;
+    memset(&dims, 0, sizeof dims);
+    dims.S = S;
+    dims.T = T;
+    CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_INDEX_TOPK, &dims)));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    float *scores = reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes);
+    CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), S, T, HI,
+                                 dI, m, 0, scores, st));
+    CSA_CUDA(launch_topk_rows(scores, S, T, m, 0, k, idx, st));
+    return CSA_OK;
+}
+
+csa_status csa_attend(const void *q, const void *C, const void *kv_rot, const int32_t *idx, const float *sinks,
+                      int64_t S, int32_t H, int32_t D, int64_t T, int32_t k, int32_t W, int32_t rope_dim, int32_t m,
+                      double theta_tok, double theta_cmp, float softmax_scale, float *o, void *workspace,
+                      size_t workspace_bytes, void *stream)
+{
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_CHECK_ARG(k >= 1 && (S == 0 || idx != nullptr));
+    CSA_CHECK_SUP(k <= 4096);
+    CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
+                              softmax_scale, o, workspace);
+    return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const float *sinks, int64_t S, int32_t H,
+                      int32_t D, int64_t T, int32_t W, int32_t rope_dim, int32_t m, double theta_tok,
+                      double theta_cmp, float softmax_scale, float *o, void *workspace, size_t workspace_bytes,
+                      void *stream)
+{
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
+                              softmax_scale, o, workspace);
+    return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status csa_forward(const void *q, const void *kv, const void *gate, const float *pos_bias, const void *qI,
+                       const void *kI, const float *w, const float *sinks, int64_t S, int32_t H, int32_t D,
+                       int32_t HI, int32_t dI, int32_t m, int32_t L, int32_t k, int32_t W, int32_t rope_dim,
+                       double theta_tok, double theta_cmp, float softmax_scale, void *C, void *kv_rot, int32_t *idx,
+                       float *o, void *workspace, size_t workspace_bytes, void *stream)
+{
+    const int64_t T = m >= 1 ? S / m : 0;
+    CSA_TRY(check_compress(kv, gate, pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    CSA_CHECK_ARG(kv_rot != nullptr || S == 0);
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_CHECK_ARG(k >= 1 && (S == 0 || idx != nullptr));
+    CSA_CHECK_SUP(k <= 4096);
+    CSA_CHECK_ARG(HI > 0 && dI > 0 && (S == 0 || (qI != nullptr && w != nullptr)) && (T == 0 || kI != nullptr));
+    CSA_CHECK_SUP(dI == 32 || dI == 64 || dI == 128 || dI == 256);
+    CSA_CHECK_SUP(HI <= 128 && (size_t)HI * dI * 4 <= 160 * 1024);
+    CSA_CHECK_ARG(aligned16(qI) && aligned16(kI) && aligned16(kv_rot));
+    csa_dims dims;
+    memset(&dims, 0, sizeof dims);
+    dims.S = S;
+    dims.T = T;
+    CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_CSA_FORWARD, &dims)));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, D,
+                             m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
+                             static_cast<uint16_t *>(kv_rot), st));
+    float *scores = reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes);
+    CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), S, T, HI,
+                                 dI, m, 0, scores, st));
+    CSA_CUDA(launch_topk_rows(scores, S, T, m, 0, k, idx, st));
+    AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
+                              softmax_scale, o, workspace);
+    return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status hca_forward(const void *q, const void *kv, const void *gate, const float *pos_bias, const float *sinks,
+                       int64_t S, int32_t H, int32_t D, int32_t m, int32_t L, int32_t W, int32_t rope_dim,
+                       double theta_tok, double theta_cmp, float softmax_scale, void *C, void *kv_rot, float *o,
+                       void *workspace, size_t workspace_bytes, void *stream)
+{
+    const int64_t T = m >= 1 ? S / m : 0;
+    CSA_TRY(check_compress(kv, gate, pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    CSA_CHECK_ARG(kv_rot != nullptr || S == 0);
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_CHECK_ARG(aligned16(kv_rot));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, D,
+                             m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
+                             static_cast<uint16_t *>(kv_rot), st));
+    AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
+                              softmax_scale, o, workspace);
+    return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status csa_decode(const void *q, const void *qI, const float *w, const void *kI, const void *C, const uint8_t *c8,
+                      const float *c8_scale, const void *c_rope, const void *win, const float *sinks, int32_t B,
+                      int32_t H, int32_t D, int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W, int32_t rope_dim,
+                      int64_t P, double theta_tok, double theta_cmp, float softmax_scale, int32_t *idx_out, float *o,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && HI > 0 && dI > 0 && k >= 1 && W >= 0 && P >= 0);
+    CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
+    CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_ARG(B == 0 || (q != nullptr && qI != nullptr && w != nullptr && sinks != nullptr && o != nullptr));
+    CSA_CHECK_ARG(B == 0 || T == 0 || kI != nullptr);
+    CSA_CHECK_ARG(B == 0 || W == 0 || win != nullptr);
+    const bool fp8 = C == nullptr;
+    CSA_CHECK_ARG(B == 0 || T == 0 || !fp8 || (c8 != nullptr && c8_scale != nullptr && c_rope != nullptr));
+    CSA_CHECK_SUP(D == 64 || D == 128 || D == 256 || D == 512);
+    CSA_CHECK_SUP(rope_dim % 8 == 0 && k <= 4096);
+    CSA_CHECK_SUP(dI == 32 || dI == 64 || dI == 128 || dI == 256);
+    CSA_CHECK_SUP(HI <= 128 && (size_t)HI * dI * 4 <= 160 * 1024);
+    CSA_CHECK_ARG(aligned16(q) && aligned16(qI) && aligned16(kI) && aligned16(C) && aligned16(c8) &&
+                  aligned16(c_rope) && aligned16(win) && aligned16(o));
+    csa_dims dims;
+    memset(&dims, 0, sizeof dims);
+    dims.B = B;
+    dims.T = T;
+    dims.k = k;
+    CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_DECODE, &dims)));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    char *base = static_cast<char *>(workspace);
+    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
+    int32_t *idx = idx_out != nullptr ? idx_out
+                                      : reinterpret_cast<int32_t *>(base + kStatusBytes + scores_bytes(B, T));
+    CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T, HI,
+                                 dI, 1, 1, scores, st));
+    CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = static_cast<const uint16_t *>(q);
+    a.win = static_cast<const uint16_t *>(win);
+    a.C = static_cast<const uint16_t *>(C);
+    a.c8 = c8;
+    a.c8_scale = c8_scale;
+    a.c_rope = static_cast<const uint16_t *>(c_rope);
+    a.idx = idx;
+    a.sinks = sinks;
+    a.o = o;
+    a.status = static_cast<int32_t *>(workspace);
+    a.R = B;
+    a.T = T;
+    a.P = P;
+    a.H = H;
+    a.D = D;
+    a.k = k;
+    a.W = W;
+    a.r = rope_dim;
+    a.m = 1;
+    a.decode = 1;
+    a.scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / sqrt((double)D));
+    a.log2_theta_tok = rope_dim > 0 ? log2(theta_tok) : 0.0;
+    a.log2_theta_cmp = rope_dim > 0 ? log2(theta_cmp) : 0.0;
+    return from_cuda(launch_attend_simt(a, st));
+}
+
+}  // extern "C"

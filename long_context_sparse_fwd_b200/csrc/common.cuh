@@ -1,0 +1,59 @@
+// common.cuh -- small device helpers shared by the CSA / HCA kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+// Status word at the start of every workspace. Kernels record the first data error they find.
+__device__ __forceinline__ void report(int32_t *status, int32_t code)
+{
+    if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(((uint32_t)b) << 16); }
+__device__ __forceinline__ float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+__device__ __forceinline__ uint16_t f2bf(float f)
+{
+    __nv_bfloat16 h = __float2bfloat16_rn(f);
+    return *reinterpret_cast<uint16_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi)
+{
+    return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
+}
+
+// Interleaved-pair RoPE angle: pair p of r rope channels at position pos has angle
+// pos * theta^(-2p/r) (Hugging Face Transformers docs "DeepSeek-V4", "Hybrid attention":
+// partial RoPE on the last qk_rope_head_dim channels, interleaved pairs). The angle is formed
+// and reduced in double precision so positions up to 2^20 keep fp32-accurate sines.
+__device__ __forceinline__ void rope_cos_sin(double pos, int p, int r, double log2_theta, float *c, float *s)
+{
+    double freq = exp2(-(2.0 * p / (double)r) * log2_theta);
+    double sd, cd;
+    sincos(pos * freq, &sd, &cd);
+    *c = (float)cd;
+    *s = (float)sd;
+}
+
+// Order-preserving map of an fp32 score to uint32 (larger score -> larger key); -0 maps like +0.
+__device__ __forceinline__ uint32_t score_key(float x)
+{
+    uint32_t u = __float_as_uint(x + 0.0f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ int64_t visible_entries(int64_t t, int m, int64_t T)
+{
+    int64_t v = (t + 1) / m;
+    return v < T ? v : T;
+}
+
+}  // namespace csa

@@ -1,0 +1,35 @@
+// kernels.cuh -- launchers shared between the C-ABI layer and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace csa {
+
+// Arguments of the attention kernels (prefill rows or decode sequences).
+struct AttnArgs {
+    const uint16_t *q;         // [R, H, D] bf16, un-rotated
+    const uint16_t *win;       // prefill: kv_rot [S, D]; decode: win [R, W, D] (post-RoPE)
+    const uint16_t *C;         // bf16 entries: prefill [T, D]; decode [R, T, D] (or null = fp8 cache)
+    const uint8_t *c8;         // fp8 entries [R, T, D-r]
+    const float *c8_scale;     // [R, T]
+    const uint16_t *c_rope;    // [R, T, r]
+    const int32_t *idx;        // [R, k] or null (all visible entries: HCA)
+    const float *sinks;        // [H]
+    float *o;                  // [R, H, D] fp32
+    int32_t *status;           // workspace status word
+    int64_t R, T, P;           // rows, entries (per row for decode), decode position
+    int H, D, k, W, r, m, decode;
+    float scale;
+    double log2_theta_tok, log2_theta_cmp;
+};
+
+cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const float *bias, int64_t S, int D, int m,
+                            int L, int r, double theta_cmp, double theta_tok, uint16_t *C, uint16_t *kv_rot,
+                            cudaStream_t stream);
+cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t R, int64_t T,
+                                int HI, int dI, int m, int decode, float *scores, cudaStream_t stream);
+cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t T, int m, int decode, int k, int32_t *idx,
+                             cudaStream_t stream);
+cudaError_t launch_attend_simt(const AttnArgs &a, cudaStream_t stream);
+
+}  // namespace csa

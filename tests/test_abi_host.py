@@ -1,0 +1,135 @@
+"""CPU-only checks of the C ABI: the library loads, exports every call include/csa.h declares,
+and rejects bad arguments on the host with the documented status before launching anything.
+
+Every call below fails a host-side check, so no kernel is launched and no pointer is touched
+(the fake pointers are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_sparse_fwd_b200 as csa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+INVALID, UNSUP, WS = 1, 2, 5
+
+
+def declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"CSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_library_exports_every_declared_call():
+    names = declared_functions()
+    assert len(names) >= 11
+    L = ctypes.CDLL(csa.library_path())
+    for n in names:
+        assert hasattr(L, n), n
+    assert csa.lib().csa_version().decode().startswith("csa-b200")
+
+
+def test_status_strings():
+    L = csa.lib()
+    for code, name in [(0, "CSA_OK"), (1, "CSA_ERR_INVALID_ARG"), (2, "CSA_ERR_UNSUPPORTED"), (3, "CSA_ERR_CUDA"),
+                       (4, "CSA_ERR_TIMEOUT"), (5, "CSA_ERR_WORKSPACE")]:
+        assert L.csa_status_str(code).decode() == name
+
+
+def test_workspace_sizes():
+    assert csa.workspace_size("attend") == 256
+    assert csa.workspace_size("hca_forward") == 256
+    assert csa.workspace_size("index_topk", S=8192, T=2048) == 256 + 8192 * 2048 * 4
+    assert csa.workspace_size("decode", B=64, T=32768, k=1024) >= 256 + 64 * 32768 * 4 + 64 * 1024 * 4
+
+
+# The fake pointers below are only safe because every call fails a host check first; they are
+# never handed to a machine with a GPU, where a check that regressed would launch a kernel on them.
+no_gpu = pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="fake-pointer checks run on CPU hosts only")
+
+FAKE = ctypes.c_void_p(0x10000)      # 16-byte aligned, never dereferenced
+MIS = ctypes.c_void_p(0x10002)       # misaligned
+
+
+def compress(**kw):
+    a = dict(kv=FAKE, gate=FAKE, b=FAKE, S=64, D=64, m=4, L=8, r=16, tc=160000.0, tt=10000.0, C=FAKE, kvr=FAKE)
+    a.update(kw)
+    return csa.lib().csa_compress(a["kv"], a["gate"], a["b"], a["S"], a["D"], a["m"], a["L"], a["r"], a["tc"],
+                                  a["tt"], a["C"], a["kvr"], None)
+
+
+@no_gpu
+def test_compress_rejects_bad_arguments():
+    assert compress(S=-1) == INVALID
+    assert compress(m=0) == INVALID
+    assert compress(L=2) == INVALID            # window shorter than the stride
+    assert compress(r=3) == INVALID            # odd rope dims
+    assert compress(r=128) == INVALID          # rope dims beyond D
+    assert compress(kv=None) == INVALID
+    assert compress(C=None) == INVALID
+    assert compress(tc=0.5) == INVALID
+    assert compress(kv=MIS) == INVALID
+    assert compress(D=60) == UNSUP
+    assert compress(r=12) == UNSUP
+    assert compress(L=8192, m=4096) == UNSUP
+
+
+def attend(**kw):
+    a = dict(q=FAKE, C=FAKE, kvr=FAKE, idx=FAKE, sinks=FAKE, S=64, H=8, D=128, T=16, k=4, W=8, r=32, m=4,
+             tt=1e4, tc=1.6e5, sc=0.0, o=FAKE, ws=FAKE, wsb=256)
+    a.update(kw)
+    return csa.lib().csa_attend(a["q"], a["C"], a["kvr"], a["idx"], a["sinks"], a["S"], a["H"], a["D"], a["T"],
+                                a["k"], a["W"], a["r"], a["m"], a["tt"], a["tc"], a["sc"], a["o"], a["ws"],
+                                a["wsb"], None)
+
+
+@no_gpu
+def test_attend_rejects_bad_arguments():
+    assert attend(T=17) == INVALID             # more entries than floor(S/m)
+    assert attend(H=0) == INVALID
+    assert attend(W=-1) == INVALID
+    assert attend(k=0) == INVALID
+    assert attend(idx=None) == INVALID
+    assert attend(q=MIS) == INVALID
+    assert attend(D=96) == UNSUP
+    assert attend(k=5000) == UNSUP
+    assert attend(ws=None) == WS
+    assert attend(wsb=16) == WS
+    assert attend(ws=ctypes.c_void_p(0x10010)) == INVALID   # workspace must be 256-byte aligned
+
+
+@no_gpu
+def test_index_topk_rejects_bad_arguments():
+    L = csa.lib()
+    f = lambda S=64, T=16, HI=4, dI=64, m=4, k=8, ws=FAKE, wsb=1 << 20, q=FAKE: L.csa_index_topk(
+        q, FAKE, FAKE, S, T, HI, dI, m, k, FAKE, ws, wsb, None)
+    assert f(T=17) == INVALID
+    assert f(k=0) == INVALID
+    assert f(q=None) == INVALID
+    assert f(dI=48) == UNSUP
+    assert f(wsb=100) == WS
+
+
+@no_gpu
+def test_decode_rejects_bad_arguments():
+    L = csa.lib()
+
+    def f(C=FAKE, c8=None, B=2, D=512, k=64, P=100, dI=128, wsb=1 << 24):
+        return L.csa_decode(FAKE, FAKE, FAKE, FAKE, C, c8, None, None, FAKE, FAKE, B, 8, D, 256, 4, dI, k, 8, 64,
+                            P, 1e4, 1.6e5, 0.0, None, FAKE, FAKE, wsb, None)
+    assert f(C=None) == INVALID                 # neither bf16 entries nor an FP8 cache
+    assert f(P=-1) == INVALID
+    assert f(D=96) == UNSUP
+    assert f(dI=40) == UNSUP
+    assert f(wsb=64) == WS
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        csa.compress(torch.zeros(8, 8, dtype=torch.bfloat16), torch.zeros(8, 8, dtype=torch.bfloat16),
+                     torch.zeros(8), 4, 8, 0, 1e4, 1e4)

@@ -92,17 +92,19 @@ def _uniform(shape, seed, tid, device):
 _Q, _KV, _GATE, _BIAS, _QI, _KI, _WI, _SINK, _C, _KVROT, _WIN = range(11)
 
 
-def prefill_inputs(wl: Workload, device="cpu", need_index: Optional[bool] = None) -> Dict[str, torch.Tensor]:
+def prefill_inputs(wl: Workload, device="cpu", need_index: Optional[bool] = None,
+                   need_q: bool = True) -> Dict[str, torch.Tensor]:
     """q [S,H,D] bf16, kv/gate [S,D] bf16, pos_bias [L] f32, sinks [H] f32 and, for CSA,
     q^I [S,HI,dI] bf16, k^I [T,dI] bf16 (one index key per entry), w [S,HI] f32."""
     S, H, D, T = wl.S, wl.H, wl.D, wl.T
     out = {
-        "q": _normal((S, H, D), wl.q_std, wl.seed, _Q, device),
         "kv": _normal((S, D), 1.0, wl.seed, _KV, device),
         "gate": _normal((S, D), 1.0, wl.seed, _GATE, device),
         "pos_bias": _normal((wl.L,), 0.02, wl.seed, _BIAS, device, torch.float32),
         "sinks": _normal((H,), 1.0, wl.seed, _SINK, device, torch.float32),
     }
+    if need_q:
+        out["q"] = _normal((S, H, D), wl.q_std, wl.seed, _Q, device)
     if need_index is None:
         need_index = wl.kind == "csa_prefill"
     if need_index:
