@@ -167,6 +167,32 @@ CSA_API csa_status csa_decode(const void *q, const void *qI, const float *w, con
                       int32_t *idx_out, float *o, void *workspace, size_t workspace_bytes,
                       void *stream);
 
+/* ---- 7. CSA decode without caller-provided scratch ---------------------------------------------
+ * No counterpart on the source pages: this is a convenience of this library.
+ * For callers that cannot allocate device memory (a runtime without its own CUDA allocator, or a
+ * serving loop that must not call cudaMalloc while other work is in flight), this is csa_decode
+ * with its scratch taken from a fixed 16 MiB array inside the library; every GPU that loads the
+ * library holds that array until the process exits. Arguments and results are those of
+ * csa_decode, without workspace and workspace_bytes. It allocates nothing.
+ *   - Returns CSA_ERR_WORKSPACE, launching nothing, when the problem needs more scratch than the
+ *     array holds, i.e. when csa_workspace_size(CSA_OP_DECODE, dims) exceeds
+ *     csa_decode_noalloc_max_scratch() (B*T*4 + B*k*4 bytes plus alignment, e.g. B=64 sequences
+ *     of T=32768 entries, or B=8 of T=262144, fit).
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the last call's contents: calls that
+ *     overlap on the GPU (different streams, or different host threads) race and must be
+ *     serialised by the caller. The device status word of the last call is not readable through
+ *     csa_get_device_status (there is no workspace pointer to pass). */
+CSA_API size_t csa_decode_noalloc_max_scratch(void);
+
+CSA_API csa_status csa_decode_noalloc(const void *q, const void *qI, const float *w, const void *kI,
+                      const void *C, const uint8_t *c8, const float *c8_scale, const void *c_rope,
+                      const void *win, const float *sinks, int32_t B, int32_t H, int32_t D,
+                      int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W, int32_t rope_dim,
+                      int64_t P, double theta_tok, double theta_cmp, float softmax_scale,
+                      int32_t *idx_out, float *o, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

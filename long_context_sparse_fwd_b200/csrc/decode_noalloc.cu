@@ -1,0 +1,72 @@
+// decode_noalloc.cu -- csa_decode for callers that cannot allocate device memory.
+//
+// csa_decode needs device scratch (the per-entry index scores and the selected indices) and asks
+// the caller for it. Some callers have no way to provide it: a host runtime that owns no CUDA
+// allocator (all device memory was partitioned up front by someone else), or a serving loop that
+// must not call cudaMalloc while other work is in flight because the call can synchronise the
+// device and stall every stream. This entry point takes the scratch from a fixed array that lives
+// inside the library instead, so the caller passes only its inputs and outputs.
+//
+// The array is a file-scope __device__ variable: each GPU that loads the library holds one copy
+// of it until the process exits. Host code cannot use the array's name as a device address (it is
+// a host-side stand-in), so the device address is looked up once per device with
+// cudaGetSymbolAddress, with that device current, and cached.
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)16 << 20;   // 16 MiB per GPU that loads the library
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+void *g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mutex;
+
+// Device address of the scratch array on the current device (looked up on first use per device).
+csa_status scratch_on_current_device(void **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return CSA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return CSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess || p == nullptr) return CSA_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return CSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t csa_decode_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+csa_status csa_decode_noalloc(const void *q, const void *qI, const float *w, const void *kI, const void *C,
+                              const uint8_t *c8, const float *c8_scale, const void *c_rope, const void *win,
+                              const float *sinks, int32_t B, int32_t H, int32_t D, int64_t T, int32_t HI, int32_t dI,
+                              int32_t k, int32_t W, int32_t rope_dim, int64_t P, double theta_tok, double theta_cmp,
+                              float softmax_scale, int32_t *idx_out, float *o, void *stream)
+{
+    if (B < 0 || T < 0 || k < 1) return CSA_ERR_INVALID_ARG;
+    csa_dims dims = {};
+    dims.B = B;
+    dims.T = T;
+    dims.k = k;
+    if (csa_workspace_size(CSA_OP_DECODE, &dims) > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    const csa_status s = scratch_on_current_device(&scratch);
+    if (s != CSA_OK) return s;
+    // csa_decode zeroes the status word at the start of the scratch and writes every score and
+    // index it later reads, so nothing left over from an earlier call is used.
+    return csa_decode(q, qI, w, kI, C, c8, c8_scale, c_rope, win, sinks, B, H, D, T, HI, dI, k, W, rope_dim, P,
+                      theta_tok, theta_cmp, softmax_scale, idx_out, o, scratch, kNoAllocScratchBytes, stream);
+}
+
+}  // extern "C"
