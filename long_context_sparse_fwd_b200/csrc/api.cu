@@ -112,6 +112,20 @@ AttnArgs prefill_args(const void *q, const void *C, const void *kv_rot, const in
     return a;
 }
 
+// Prefill indexer + top-k: the tcgen05 kernel with on-chip scores where it applies, else the
+// general path (scores through the workspace, then a radix select per row).
+cudaError_t index_topk_any(const void *qI, const void *kI, const float *w, int64_t S, int64_t T, int32_t HI,
+                           int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace, cudaStream_t st)
+{
+    const uint16_t *q16 = static_cast<const uint16_t *>(qI), *k16 = static_cast<const uint16_t *>(kI);
+    if (T > 0 && index_topk_tc_supported(T, HI, dI, k))
+        return launch_index_topk_tc(q16, k16, w, S, T, HI, dI, m, k, idx, static_cast<int32_t *>(workspace), st);
+    float *scores = reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes);
+    cudaError_t e = launch_index_scores(q16, w, k16, S, T, HI, dI, m, 0, scores, st);
+    if (e != cudaSuccess) return e;
+    return launch_topk_rows(scores, S, T, m, 0, k, idx, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -186,10 +200,7 @@ csa_status csa_index_topk(const void *qI, const void *kI, const float *w, int64_
     CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_INDEX_TOPK, &dims)));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
-    float *scores = reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes);
-    CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), S, T, HI,
-                                 dI, m, 0, scores, st));
-    CSA_CUDA(launch_topk_rows(scores, S, T, m, 0, k, idx, st));
+    CSA_CUDA(index_topk_any(qI, kI, w, S, T, HI, dI, m, k, idx, workspace, st));
     return CSA_OK;
 }
 
@@ -249,10 +260,7 @@ csa_status csa_forward(const void *q, const void *kv, const void *gate, const fl
     CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, D,
                              m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
                              static_cast<uint16_t *>(kv_rot), st));
-    float *scores = reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes);
-    CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), S, T, HI,
-                                 dI, m, 0, scores, st));
-    CSA_CUDA(launch_topk_rows(scores, S, T, m, 0, k, idx, st));
+    CSA_CUDA(index_topk_any(qI, kI, w, S, T, HI, dI, m, k, idx, workspace, st));
     AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
     return from_cuda(launch_attend_simt(a, st));

@@ -1,0 +1,343 @@
+// index_tc.cu -- lightning indexer on the 5th-generation tensor cores with the top-k fused in.
+//
+// Scores (Hugging Face Transformers docs "DeepSeek-V4", section "Hybrid attention", CSA; the
+// insight.ai.kr digest of the HF blog: a ReLU multi-head dot product):
+//     I[t,s] = sum_h w[t,h] * ReLU(qI[t,h,:] . kI[s,:]),   s < vis(t) = floor((t+1)/m)
+// then the top-k per query with ties to the smaller entry index ("Attention mask layout":
+// unfilled slots are -1).
+//
+// Mapping: the GEMM is transposed so an entry sits on a TMEM lane and the (query, head) pairs of
+// Q = 256/HI consecutive queries run along the N = 256 columns:
+//     D[s, (q,h)] = kI[s,:] . qI[q,h,:]          M = 128 entries, N = 256, K = dI
+// Each epilogue thread then owns one entry and reduces a query's HI columns in registers
+// (w-weighted ReLU sum): no cross-lane reduction. The scores of the Q queries for every visible
+// entry stay in shared memory; after the last entry tile each epilogue warp runs an exact radix
+// select for one query and writes the kept indices in ascending order.
+//
+// Roles (6 warps): warp 0 issues TMA loads (q^I block once, k^I tiles through a ring of stages),
+// warp 1 owns TMEM (2 x 256 columns, double-buffered accumulators) and issues tcgen05.mma, warps
+// 2-5 read TMEM, score, and select. Every wait is bounded; a timeout sets CSA_ERR_TIMEOUT.
+#include <algorithm>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;          // entries per tile = TMEM lanes
+constexpr int BN = 256;          // (query, head) columns
+constexpr int NUM_THREADS = 192;
+constexpr int EPI_THREADS = 128;
+constexpr uint32_t TMEM_COLS = 512;
+
+struct IdxParams {
+    const float *w;      // [S, HI]
+    int32_t *idx;        // [S, k]
+    int32_t *status;
+    int64_t S, T;
+    int HI, dI, m, k, Q, stages, T_cap;
+};
+
+__device__ __forceinline__ void topk_warp(const float *sc, int n, int k, uint32_t *hist, int32_t *out)
+{
+    const int lane = threadIdx.x & 31;
+    if (n <= k) {
+        for (int i = lane; i < k; i += 32) out[i] = i < n ? i : -1;
+        return;
+    }
+    uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
+        __syncwarp();
+        for (int s = lane; s < n; s += 32) {
+            const uint32_t key = score_key(sc[s]);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        uint32_t c[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { c[j] = hist[lane * 8 + j]; tot += c[j]; }
+        // counts held by lanes above this one (higher digits)
+        uint32_t above = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_down_sync(0xffffffffu, above, o);
+            if (lane + o < 32) above += v;
+        }
+        above -= tot;
+        // the digit d with count(> d) < remaining <= count(>= d)
+        int found = -1;
+        uint32_t above_d = 0, cnt_d = 0;
+        uint32_t run = above;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+            if (found < 0 && run + c[j] >= remaining) { found = lane * 8 + j; above_d = run; cnt_d = c[j]; }
+            run += c[j];
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, found >= 0 && (above < remaining));
+        const int src = __ffs(who) - 1;
+        const int d = __shfl_sync(0xffffffffu, found, src);
+        above_d = __shfl_sync(0xffffffffu, above_d, src);
+        cnt_d = __shfl_sync(0xffffffffu, cnt_d, src);
+        prefix |= (uint32_t)d << shift;
+        mask |= 255u << shift;
+        remaining -= above_d;
+        __syncwarp();
+        if (cnt_d == remaining) break;   // the whole bucket is taken
+    }
+    int written = 0, eq_seen = 0;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < n && written < k; base += 32) {
+        const int s = base + lane;
+        uint32_t key = 0;
+        if (s < n) key = score_key(sc[s]) & mask;
+        const bool gt = s < n && key > prefix;
+        const bool eq = s < n && key == prefix;
+        const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+        const int rank = eq_seen + __popc(eqb & lt);
+        const bool sel = gt || (eq && rank < (int)remaining);
+        const unsigned sb = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(sb & lt)] = s;
+        written += __popc(sb);
+        eq_seen += __popc(eqb);
+    }
+    for (int i = written + lane; i < k; i += 32) out[i] = -1;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     IdxParams p)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int kchunks = p.dI / 64;                      // 128-byte swizzle atoms along K
+    const uint32_t b_bytes = (uint32_t)kchunks * BN * 128;
+    const uint32_t a_bytes = (uint32_t)kchunks * BM * 128;
+    uint8_t *sB = smem;
+    uint8_t *sA = sB + b_bytes;
+    float *scores = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [Q][T_cap]
+    float *sw = scores + (size_t)p.Q * p.T_cap;                                  // [BN]
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                      // [4][256]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 4 * 256);
+    uint64_t *full = bars;                   // [stages]
+    uint64_t *empty = bars + 8;              // [stages]
+    uint64_t *tfull = bars + 16;             // [2]
+    uint64_t *tempty = bars + 18;            // [2]
+    uint64_t *qfull = bars + 20;
+    uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(bars + 21);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 22);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t0 = (int64_t)blockIdx.x * p.Q;
+    const int64_t t_last = min(t0 + p.Q - 1, p.S - 1);
+    const int64_t vis_max = visible_entries(t_last, p.m, p.T);
+    const int ntiles = (int)((vis_max + BM - 1) / BM);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < p.stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], EPI_THREADS); }
+        mbar_init(qfull, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_base_ptr, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp >= 2) {   // index weights of this block's queries
+        for (int i = threadIdx.x - 64; i < p.Q * p.HI; i += EPI_THREADS) {
+            const int64_t t = t0 + i / p.HI;
+            sw[i] = t < p.S ? p.w[t * p.HI + (i % p.HI)] : 0.f;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_ptr;
+
+    if (warp == 0 && ntiles > 0) {
+        // ---------------- TMA producer ----------------
+        if (elect_one()) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            mbar_arrive_expect_tx(qfull, b_bytes);
+            for (int c = 0; c < kchunks; ++c)
+                tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
+            int issued = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int st = i % p.stages;
+                if (!mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status)) break;
+                mbar_arrive_expect_tx(&full[st], a_bytes);
+                for (int c = 0; c < kchunks; ++c)
+                    tma_load_2d(sA + (size_t)st * a_bytes + (size_t)c * BM * 128, &tm_k, &full[st], c * 64, i * BM);
+                issued = i + 1;
+            }
+            // never leave with copies in flight into this CTA's shared memory
+            mbar_wait(qfull, 0, abort, p.status, 100000000ull);
+            for (int i = max(0, issued - p.stages); i < issued; ++i)
+                mbar_wait(&full[i % p.stages], (i / p.stages) & 1, abort, p.status, 100000000ull);
+        }
+    } else if (warp == 1 && ntiles > 0) {
+        // ---------------- MMA issuer ----------------
+        const uint32_t idesc = idesc_bf16(BM, BN);
+        bool ok = mbar_wait(qfull, 0, abort, p.status);
+        int issued = 0;
+        for (int i = 0; ok && i < ntiles; ++i) {
+            const int st = i % p.stages, buf = i & 1;
+            if (!mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1, abort, p.status)) break;
+            if (!mbar_wait(&full[st], (i / p.stages) & 1, abort, p.status)) break;
+            tc_fence_after();
+            if (elect_one()) {
+                const uint32_t a0 = smem_u32(sA + (size_t)st * a_bytes), b0 = smem_u32(sB);
+                for (int c = 0; c < kchunks; ++c) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = sdesc_sw128(a0 + c * BM * 128 + ks * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(b0 + c * BN * 128 + ks * 32, 16, 1024);
+                        mma_bf16(tmem_base + buf * BN, ad, bd, idesc, (c | ks) != 0);
+                    }
+                }
+                mma_commit(&empty[st]);
+                mma_commit(&tfull[buf]);
+            }
+            __syncwarp();
+            issued = i + 1;
+        }
+        if (issued > 0) {   // the last accumulator must be complete before TMEM is released
+            const int i = issued - 1;
+            mbar_wait(&tfull[i & 1], (i >> 1) & 1, abort, p.status, 100000000ull);
+        }
+    } else if (warp >= 2) {
+        // ---------------- epilogue: scores into shared memory ----------------
+        const int quarter = warp & 3;              // TMEM lanes this warp may read
+        for (int i = 0; i < ntiles; ++i) {
+            const int buf = i & 1;
+            if (!mbar_wait(&tfull[buf], (i >> 1) & 1, abort, p.status)) break;
+            tc_fence_after();
+            const int s = i * BM + quarter * 32 + lane;
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+            for (int q = 0; q < p.Q; ++q) {
+                float acc = 0.f;
+                // columns [q*HI, (q+1)*HI) of this buffer; never read past them (HI = 16 uses x16 loads)
+                for (int h0 = 0; h0 < p.HI; h0 += 16) {
+                    const float *wq = sw + q * p.HI + h0;
+                    if (h0 + 32 <= p.HI) {
+                        float v[32];
+                        tmem_ld32(taddr + q * p.HI + h0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) acc = fmaf(wq[j], fmaxf(v[j], 0.f), acc);
+                        h0 += 16;
+                    } else {
+                        float v[16];
+                        tmem_ld16(taddr + q * p.HI + h0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) acc = fmaf(wq[j], fmaxf(v[j], 0.f), acc);
+                    }
+                }
+                if (s < p.T_cap) scores[q * p.T_cap + s] = acc + 0.0f;
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+        }
+        named_barrier_sync(1, EPI_THREADS);
+        // ---------------- exact top-k, one query per warp ----------------
+        if (!*abort) {
+            for (int q = warp - 2; q < p.Q; q += 4) {
+                const int64_t t = t0 + q;
+                if (t >= p.S) continue;
+                const int n = (int)visible_entries(t, p.m, p.T);
+                topk_warp(scores + (size_t)q * p.T_cap, n, p.k, hist + (warp - 2) * 256, p.idx + t * (int64_t)p.k);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+// ---- host: tensor maps ------------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (fn == nullptr) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128-byte swizzle.
+bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)
+{
+    (void)k;
+    return (dI == 64 || dI == 128) && (HI == 16 || HI == 32 || HI == 64 || HI == 128) && T <= 4096 && T >= 1 &&
+           encode_fn() != nullptr;
+}
+
+cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t T, int HI,
+                                 int dI, int m, int k, int32_t *idx, int32_t *status, cudaStream_t stream)
+{
+    if (S == 0) return cudaSuccess;
+    IdxParams p;
+    p.w = w;
+    p.idx = idx;
+    p.status = status;
+    p.S = S;
+    p.T = T;
+    p.HI = HI;
+    p.dI = dI;
+    p.m = m;
+    p.k = k;
+    p.Q = BN / HI;
+    p.T_cap = (int)((T + BM - 1) / BM * BM);
+    const size_t a_bytes = (size_t)(dI / 64) * BM * 128, b_bytes = (size_t)(dI / 64) * BN * 128;
+    const size_t fixed = 1024 + b_bytes + (size_t)p.Q * p.T_cap * 4 + BN * 4 + 4 * 256 * 4 + 256;
+    const size_t budget = 227 * 1024;
+    p.stages = (int)std::min<size_t>(4, (budget - fixed) / a_bytes);
+    if (p.stages < 2) return cudaErrorInvalidValue;
+    const size_t smem = fixed + (size_t)p.stages * a_bytes;
+    CUtensorMap tq, tk;
+    if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)S * HI, dI, BN)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)T, dI, BM)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(index_topk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((S + p.Q - 1) / p.Q);
+    index_topk_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tk, p);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -32,4 +32,9 @@ cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t T, int m, i
                              cudaStream_t stream);
 cudaError_t launch_attend_simt(const AttnArgs &a, cudaStream_t stream);
 
+// index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
+bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
+cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t T, int HI,
+                                 int dI, int m, int k, int32_t *idx, int32_t *status, cudaStream_t stream);
+
 }  // namespace csa

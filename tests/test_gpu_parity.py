@@ -80,6 +80,22 @@ def test_index_topk(wid, S, nrows):
         assert (np.diff(kept) > 0).all()
 
 
+@pytest.mark.parametrize("HI,dI,S,k", [(64, 128, 1030, 16), (32, 64, 777, 40), (128, 128, 600, 8),
+                                        (16, 64, 5000, 300), (64, 128, 16384, 512), (64, 128, 20000, 512)])
+def test_index_topk_shapes(HI, dI, S, k):
+    """Tensor-core path shapes (N = 256 query-head columns, T up to 4096 on chip), ragged query
+    blocks and entry tiles, k above and below vis(t); S=20000 (T > 4096) takes the general path."""
+    wl = WORKLOADS[1].with_(S=S, HI=HI, dI=dI, topk=k)
+    g, x = gen(prefill_inputs, wl, need_q=False)
+    idx = csa.index_topk(g["qI"], g["kI"], g["w"], wl.m, wl.topk)
+    torch.cuda.synchronize()
+    rows = sample_rows(S, 96, 13, must=list(range(0, 9)) + [255, 256, 511, S - 2, S - 1])
+    ridx, sc = oracle.index_topk(x["qI"], x["kI"], x["w"], wl.m, wl.topk, rows=rows)
+    vis = [oracle.visible(t, wl.m, wl.T) for t in rows]
+    exc = check_topk_sets(idx.cpu().numpy()[rows], ridx, sc, vis, wl.topk)
+    assert len(exc) <= max(2, len(rows) // 50), f"too many near-tie exceptions: {exc[:5]}"
+
+
 def test_index_topk_all_zero_ties():
     """Weights 0 make every score exactly 0: the k smallest visible indices win."""
     wl = WORKLOADS[0].with_(S=200)
