@@ -112,6 +112,14 @@ AttnArgs prefill_args(const void *q, const void *C, const void *kv_rot, const in
     return a;
 }
 
+// Prefill attention: the tcgen05 kernel for the V4 head shape (64 heads x 512, rope 64), else the
+// general CUDA-core kernel.
+cudaError_t attend_any(const AttnArgs &a, cudaStream_t st)
+{
+    if (!a.decode && attend_tc_supported(a.H, a.D, a.r, a.idx != nullptr ? a.k : 0)) return launch_attend_tc(a, st);
+    return launch_attend_simt(a, st);
+}
+
 // Prefill indexer + top-k: the tcgen05 kernel with on-chip scores where it applies, else the
 // general path (scores through the workspace, then a radix select per row).
 cudaError_t index_topk_any(const void *qI, const void *kI, const float *w, int64_t S, int64_t T, int32_t HI,
@@ -217,7 +225,7 @@ csa_status csa_attend(const void *q, const void *C, const void *kv_rot, const in
     CSA_TRY(reset_status(workspace, st));
     AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
-    return from_cuda(launch_attend_simt(a, st));
+    return from_cuda(attend_any(a, st));
 }
 
 csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const float *sinks, int64_t S, int32_t H,
@@ -231,7 +239,7 @@ csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const fl
     CSA_TRY(reset_status(workspace, st));
     AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
-    return from_cuda(launch_attend_simt(a, st));
+    return from_cuda(attend_any(a, st));
 }
 
 csa_status csa_forward(const void *q, const void *kv, const void *gate, const float *pos_bias, const void *qI,
@@ -263,7 +271,7 @@ csa_status csa_forward(const void *q, const void *kv, const void *gate, const fl
     CSA_CUDA(index_topk_any(qI, kI, w, S, T, HI, dI, m, k, idx, workspace, st));
     AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
-    return from_cuda(launch_attend_simt(a, st));
+    return from_cuda(attend_any(a, st));
 }
 
 csa_status hca_forward(const void *q, const void *kv, const void *gate, const float *pos_bias, const float *sinks,
@@ -284,7 +292,7 @@ csa_status hca_forward(const void *q, const void *kv, const void *gate, const fl
                              static_cast<uint16_t *>(kv_rot), st));
     AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
-    return from_cuda(launch_attend_simt(a, st));
+    return from_cuda(attend_any(a, st));
 }
 
 csa_status csa_decode(const void *q, const void *qI, const float *w, const void *kI, const void *C, const uint8_t *c8,

@@ -1,0 +1,466 @@
+// attend_tc.cu -- CSA / HCA prefill attention on the 5th-generation tensor cores (H=64, D=512,
+// rope 64), one query per CTA.
+//
+// What it computes (Hugging Face Transformers docs "DeepSeek-V4", section "Hybrid attention":
+// shared K=V MQA, partial interleaved RoPE with the output rope slice rotated at -i (eq. 26), a
+// per-head sink (eq. 27), the sliding-window branch concatenated with the compressed entries;
+// section "Attention mask layout": window (i - W, i], CSA picks from the indexer, HCA every
+// entry w < (i+1)//m): for query t and head h, one softmax over the window rows kv_rot[j]
+// (scored with q rotated by theta_tok) and the entry rows C[s] (scored with q rotated by
+// theta_cmp) plus exp(sink_h); K = V; each branch's rope slice rotated back by -t with its theta.
+//
+// Design. A query's 64 heads form an M=64 tile; its keys (window rows first, then the entries)
+// are gathered 64 at a time with 16-byte cp.async into 128-byte-swizzled shared memory, where the
+// same tile is the K-major B operand of S = Q K^T and the MN-major B operand of O += P V:
+// the selected rows are read from L2/HBM once and shared by all 64 heads.
+//   TMEM (M=64 uses 16 lanes of each 32-lane quarter; a second tile sits at lane offset 16):
+//     lanes +0 : O_lo  cols [0,256)   output dims 0..255
+//     lanes +16: O_hi  cols [0,192)   dims 256..447, cols [192,256) entry-branch rope dims 448..511
+//     lanes +16: O_rw  cols [256,320) window-branch rope dims 448..511
+//     S_b      cols [320,384) at lanes +16*(b&1)    (double-buffered logits)
+//   The rope slice of each branch accumulates separately so each can be rotated back by -t
+//   with its own theta in the epilogue.
+// Softmax runs in the exp2 domain with a reference max per head that is only raised when a block
+// exceeds it by more than 2^8 (then O is rescaled in TMEM after the previous P V completes),
+// so almost every block needs no rescale. The sink seeds the reference and the running sum.
+// Roles: warps 0-3 softmax + epilogue, warps 4-5 gather keys, warp 6 owns TMEM and issues MMAs.
+// Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
+#include <algorithm>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace csa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int HH = 64, DD = 512, RR = 64;
+constexpr int KB = 64;                          // keys per block
+constexpr int NCH = DD / 64;                    // 64-element chunks per row
+constexpr int QCH = 9;                          // Q chunks: 7 un-rotated, rope(theta_cmp), rope(theta_tok)
+constexpr int QCHUNK = HH * 128;                // 8 KB
+constexpr int KCHUNK = KB * 128;                // 8 KB
+constexpr int STAGE = NCH * KCHUNK;             // 64 KB
+constexpr int PBUF = HH * 128;                  // 8 KB
+constexpr int NUM_THREADS = 224;
+constexpr int SM_THREADS = 128;
+constexpr int PROD_THREADS = 64;
+constexpr int MMA_WARP = 6;
+constexpr float TAU = 8.f;
+constexpr uint32_t COL_RW = 256, COL_S = 320;
+constexpr uint32_t LANE16 = 16u << 16;
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr size_t OFF_Q = 0;
+constexpr size_t OFF_KV = OFF_Q + (size_t)QCH * QCHUNK;       // 72 KB
+constexpr size_t OFF_P = OFF_KV + 2 * (size_t)STAGE;          // 200 KB
+constexpr size_t OFF_ROPE = OFF_P + 2 * (size_t)PBUF;         // 216 KB: cos/sin [2 thetas][32 pairs][2]
+constexpr size_t OFF_BAR = OFF_ROPE + 2 * 32 * 2 * 4;
+constexpr size_t OFF_LIST = OFF_BAR + 256;
+
+struct TcArgs {
+    const uint16_t *q;        // [S, 64, 512]
+    const uint16_t *kv_rot;   // [S, 512]
+    const uint16_t *C;        // [T, 512]
+    const int32_t *idx;       // [S, k] or null (HCA)
+    const float *sinks;       // [64]
+    float *o;                 // [S, 64, 512]
+    int32_t *status;
+    int64_t S, T;
+    int k, W, m;
+    float scale_log2;         // softmax scale * log2(e)
+    double log2_theta_tok, log2_theta_cmp;
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// byte offset of 16-byte unit `u` (0..7) of row `row` inside a 128-byte-swizzled [rows x 128 B] chunk
+__device__ __forceinline__ uint32_t sw128(int row, int u) { return (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4)); }
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sQ = smem + OFF_Q;
+    uint8_t *sKV = smem + OFF_KV;
+    uint8_t *sP = smem + OFF_P;
+    float *rope_cs = reinterpret_cast<float *>(smem + OFF_ROPE);     // [theta: 0 tok, 1 cmp][pair][cos, sin]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *kv_full = bars + 0;     // [2] 64 producer arrivals
+    uint64_t *kv_empty = bars + 2;    // [2] MMA commit
+    uint64_t *s_full = bars + 4;      // [2] MMA commit
+    uint64_t *p_ready = bars + 6;     // [2] 128 softmax arrivals
+    uint64_t *o_done = bars + 8;      // MMA commit after each P V
+    uint64_t *q_ready = bars + 9;     // 128 softmax arrivals
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 10);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 11);
+    int *nlist = reinterpret_cast<int *>(bars + 12);
+    int *elist = reinterpret_cast<int *>(smem + OFF_LIST);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = a.S - 1 - (int64_t)blockIdx.x;          // longest key lists first
+    const int64_t vis = visible_entries(t, a.m, a.T);
+    const int64_t wpos0 = max((int64_t)0, t - a.W + 1);
+    const int nw = (int)(t - wpos0 + 1);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&kv_full[i], PROD_THREADS);
+            mbar_init(&kv_empty[i], 1);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_ready[i], SM_THREADS);
+        }
+        mbar_init(o_done, 1);
+        mbar_init(q_ready, SM_THREADS);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(tmem_ptr, TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (threadIdx.x < 64) {   // rope table: angle t * theta^(-2p/64) for both thetas
+        const int p = threadIdx.x & 31, th = threadIdx.x >> 5;
+        float c, s;
+        rope_cos_sin((double)t, p, RR, th ? a.log2_theta_cmp : a.log2_theta_tok, &c, &s);
+        rope_cs[(th * 32 + p) * 2] = c;
+        rope_cs[(th * 32 + p) * 2 + 1] = s;
+    }
+    if (warp == 4) {          // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
+        if (a.idx != nullptr) {
+            const int32_t *ir = a.idx + t * (int64_t)a.k;
+            int cnt = 0;
+            for (int base = 0; base < a.k; base += 32) {
+                const int j = base + lane;
+                const int s = j < a.k ? ir[j] : -1;
+                const bool ok = s >= 0 && (int64_t)s < vis;
+                if (s >= 0 && !ok) report(a.status, CSA_ERR_INVALID_ARG);
+                const unsigned mk = __ballot_sync(0xffffffffu, ok);
+                if (ok) elist[cnt + __popc(mk & ((1u << lane) - 1u))] = s;
+                cnt += __popc(mk);
+            }
+            if (lane == 0) *nlist = cnt;
+        } else if (lane == 0) {
+            *nlist = (int)vis;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    const int ne = *nlist;
+    const int nbw = (nw + KB - 1) / KB, nbe = (ne + KB - 1) / KB, nb = nbw + nbe;
+
+    if (warp < 4) {
+        // =============== softmax + epilogue (warp w owns TMEM lane quarter w) ===============
+        const int tid = threadIdx.x;
+        // Q tile: 7 un-rotated chunks, rope chunk rotated with theta_cmp (7) and theta_tok (8)
+        for (int i = tid; i < HH * 64; i += SM_THREADS) {
+            const int h = i >> 6, u = i & 63, dc = u >> 3, uu = u & 7;
+            const uint4 v = *reinterpret_cast<const uint4 *>(a.q + ((t * HH + h) * (int64_t)DD) + u * 8);
+            if (dc < 7) {
+                *reinterpret_cast<uint4 *>(sQ + dc * QCHUNK + sw128(h, uu)) = v;
+            } else {
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint32_t oc[4], ot[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int p = uu * 4 + e;
+                    const float x0 = bf_lo(w4[e]), x1 = bf_hi(w4[e]);
+                    const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
+                    const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
+                    oc[e] = pack_bf2(x0 * cc - x1 * sc, x0 * sc + x1 * cc);
+                    ot[e] = pack_bf2(x0 * ct - x1 * st, x0 * st + x1 * ct);
+                }
+                *reinterpret_cast<uint4 *>(sQ + 7 * QCHUNK + sw128(h, uu)) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
+                *reinterpret_cast<uint4 *>(sQ + 8 * QCHUNK + sw128(h, uu)) = make_uint4(ot[0], ot[1], ot[2], ot[3]);
+            }
+        }
+        fence_async_smem();
+        mbar_arrive(q_ready);
+
+        const int h = warp * 16 + (lane & 15);
+        const int half = lane >> 4;
+        const float zl = a.sinks[h] * 1.4426950408889634f;
+        float m_ref = zl, l = (zl == -INFINITY) ? 0.f : 1.f;
+        const uint32_t tq = tmem + ((uint32_t)(warp * 32) << 16);
+        bool ok = true;
+        for (int b = 0; b < nb && ok; ++b) {
+            const int buf = b & 1;
+            const int nk = b < nbw ? min(KB, nw - b * KB) : min(KB, ne - (b - nbw) * KB);
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (b >> 1) & 1, abort, a.status));
+            if (!ok) break;
+            tc_fence_after();
+            float s0[32], s1[32];
+            tmem_ld32(tq + COL_S, s0);
+            tmem_ld32(tq + COL_S + 32, s1);
+            tmem_wait_ld();
+            const bool active = half == buf;
+            float corr = 1.f;
+            bool need = false;
+            if (active) {
+                float mb = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    s0[j] = j < nk ? s0[j] * a.scale_log2 : -INFINITY;
+                    s1[j] = j + 32 < nk ? s1[j] * a.scale_log2 : -INFINITY;
+                    mb = fmaxf(mb, fmaxf(s0[j], s1[j]));
+                }
+                if (mb > m_ref + TAU) {
+                    corr = exp2f(m_ref - mb);
+                    m_ref = mb;
+                    l *= corr;
+                    need = b > 0;
+                }
+                float sum = 0.f;
+                uint32_t pk[32];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const uint32_t w0 = pack_bf2(exp2f(s0[j] - m_ref), exp2f(s0[j + 1] - m_ref));
+                    const uint32_t w1 = pack_bf2(exp2f(s1[j] - m_ref), exp2f(s1[j + 1] - m_ref));
+                    pk[j >> 1] = w0;
+                    pk[16 + (j >> 1)] = w1;
+                    sum += bf_lo(w0) + bf_hi(w0) + bf_lo(w1) + bf_hi(w1);
+                }
+                l += sum;
+                uint8_t *prow = sP + buf * PBUF;
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu)
+                    *reinterpret_cast<uint4 *>(prow + sw128(h, uu)) =
+                        make_uint4(pk[uu * 4], pk[uu * 4 + 1], pk[uu * 4 + 2], pk[uu * 4 + 3]);
+            }
+            // keep both halves of the warp in step: the partner lane holds the same head
+            const float pm = __shfl_xor_sync(0xffffffffu, m_ref, 16);
+            const float pl = __shfl_xor_sync(0xffffffffu, l, 16);
+            const float pc = __shfl_xor_sync(0xffffffffu, corr, 16);
+            const int pn = __shfl_xor_sync(0xffffffffu, (int)need, 16);
+            if (!active) { m_ref = pm; l = pl; corr = pc; need = pn != 0; }
+            if (__any_sync(0xffffffffu, need)) {
+                // O must hold every earlier P V before it is rescaled
+                ok = __all_sync(0xffffffffu, mbar_wait(o_done, (b - 1) & 1, abort, a.status));
+                tc_fence_after();
+                if (ok) {
+                    for (uint32_t c = 0; c < COL_S; c += 32) {
+                        float v[32];
+                        tmem_ld32(tq + c, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) v[j] *= corr;
+                        tmem_st32(tq + c, v);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&p_ready[buf]);
+        }
+        // ---------------- epilogue ----------------
+        if (ok && nb > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (nb - 1) & 1, abort, a.status));
+        if (ok && nb > 0) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
+            const bool has_win = nbw > 0, has_ent = nbe > 0;
+            for (int c = 0; c < 256; c += 32) {
+                float v[32], rw[32];
+                tmem_ld32(tq + c, v);
+                if (c >= 192) tmem_ld32(tq + COL_RW + (c - 192), rw);   // warp-uniform collective loads
+                tmem_wait_ld();
+                if (half == 1 && c >= 192) {
+                    // rope slice: entry branch (here) + window branch (O_rw), each rotated by -t
+#pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        const int p = (c - 192 + j) >> 1;
+                        const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
+                        const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
+                        float e0 = has_ent ? v[j] : 0.f, e1 = has_ent ? v[j + 1] : 0.f;
+                        float w0 = has_win ? rw[j] : 0.f, w1 = has_win ? rw[j + 1] : 0.f;
+                        v[j] = (e0 * cc + e1 * sc) + (w0 * ct + w1 * st);
+                        v[j + 1] = (-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4 *>(orow + c + j) =
+                        make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv);
+            }
+        } else if (nb == 0) {
+            float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
+            for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else if (warp < 6) {
+        // =============== key gather: cp.async into 128-byte-swizzled stages ===============
+        const int ptid = threadIdx.x - 128;
+        for (int b = 0; b < nb; ++b) {
+            const int st = b & 1;
+            if (!mbar_wait(&kv_empty[st], ((b >> 1) & 1) ^ 1, abort, a.status)) break;
+            const bool win = b < nbw;
+            const int kbase = win ? b * KB : (b - nbw) * KB;
+            const int nk = win ? min(KB, nw - kbase) : min(KB, ne - kbase);
+            const uint32_t sbase = smem_u32(sKV + st * STAGE);
+            for (int i = ptid; i < KB * 64; i += PROD_THREADS) {
+                const int key = i >> 6, u = i & 63;
+                const bool valid = key < nk;
+                const uint16_t *row = a.q;        // any mapped address when not valid (0 bytes read)
+                if (valid) {
+                    if (win) {
+                        row = a.kv_rot + (wpos0 + kbase + key) * (int64_t)DD;
+                    } else {
+                        const int64_t s = a.idx != nullptr ? (int64_t)elist[kbase + key] : (int64_t)(kbase + key);
+                        row = a.C + s * DD;
+                    }
+                }
+                cp_async16(sbase + (u >> 3) * KCHUNK + sw128(key, u & 7), row + (valid ? u * 8 : 0), valid ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(&kv_full[st]);
+        }
+        cp_async_wait_all();
+    } else if (warp == MMA_WARP) {
+        // =============== MMA issuer ===============
+        const uint32_t idS = idesc_bf16(64, 64);
+        const uint32_t idPV256 = idesc_bf16(64, 256, true);
+        const uint32_t idPV192 = idesc_bf16(64, 192, true);
+        const uint32_t idPV64 = idesc_bf16(64, 64, true);
+        const uint32_t q0 = smem_u32(sQ), kv0 = smem_u32(sKV), p0 = smem_u32(sP);
+        int s_issued = 0, pv_issued = 0;
+        bool ok = nb == 0 || mbar_wait(q_ready, 0, abort, a.status);
+        auto issue_S = [&](int b) -> bool {
+            const int st = b & 1;
+            if (!mbar_wait(&kv_full[st], (b >> 1) & 1, abort, a.status)) return false;
+            fence_async_smem();
+            tc_fence_after();
+            if (elect_one()) {
+                const uint32_t d = tmem + COL_S + (b & 1) * LANE16;
+                const int rope_chunk = b < nbw ? 8 : 7;
+                for (int dc = 0; dc < NCH; ++dc) {
+                    const uint32_t qa = q0 + (dc < 7 ? dc : rope_chunk) * QCHUNK;
+                    const uint32_t kb = kv0 + st * STAGE + dc * KCHUNK;
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(d, sdesc_sw128(qa + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 32, 16, 1024), idS,
+                                 (dc | ks) != 0);
+                }
+                mma_commit(&s_full[b & 1]);
+            }
+            __syncwarp();
+            return true;
+        };
+        if (ok && nb > 0) { ok = issue_S(0); s_issued = ok ? 1 : 0; }
+        for (int b = 0; ok && b < nb; ++b) {
+            if (b + 1 < nb) {
+                if (!issue_S(b + 1)) { ok = false; break; }
+                s_issued = b + 2;
+            }
+            if (!mbar_wait(&p_ready[b & 1], (b >> 1) & 1, abort, a.status)) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) {
+                const int st = b & 1;
+                const bool win = b < nbw;
+                const uint32_t pa = p0 + (b & 1) * PBUF;
+                const uint32_t vb = kv0 + st * STAGE;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const uint64_t ad = sdesc_sw128(pa + ks * 32, 16, 1024);
+                    const uint32_t koff = ks * 2 * 1024;
+                    // dims 0..255 -> O_lo
+                    mma_bf16(tmem, ad, sdesc_sw128(vb + koff, KCHUNK, 1024), idPV256, b > 0 || ks > 0);
+                    // dims 256..447 -> O_hi cols 0..191
+                    mma_bf16(tmem + LANE16, ad, sdesc_sw128(vb + 4 * KCHUNK + koff, KCHUNK, 1024), idPV192,
+                             b > 0 || ks > 0);
+                    // dims 448..511 -> the rope accumulator of this block's branch
+                    const uint32_t drope = win ? tmem + LANE16 + COL_RW : tmem + LANE16 + 192;
+                    const bool first = win ? (b == 0) : (b == nbw);
+                    mma_bf16(drope, ad, sdesc_sw128(vb + 7 * KCHUNK + koff, KCHUNK, 1024), idPV64, !first || ks > 0);
+                }
+                mma_commit(&kv_empty[st]);
+                mma_commit(o_done);
+            }
+            __syncwarp();
+            pv_issued = b + 1;
+        }
+        // leave only when every issued MMA has completed
+        if (pv_issued > 0) mbar_wait(o_done, (pv_issued - 1) & 1, abort, a.status, 100000000ull);
+        if (s_issued > pv_issued) {
+            const int b = s_issued - 1;
+            mbar_wait(&s_full[b & 1], (b >> 1) & 1, abort, a.status, 100000000ull);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+bool attend_tc_supported(int H, int D, int r, int k)
+{
+    return H == HH && D == DD && r == RR && k <= 1024;
+}
+
+cudaError_t launch_attend_tc(const AttnArgs &x, cudaStream_t stream)
+{
+    if (x.R == 0) return cudaSuccess;
+    TcArgs a;
+    a.q = x.q;
+    a.kv_rot = x.win;
+    a.C = x.C;
+    a.idx = x.idx;
+    a.sinks = x.sinks;
+    a.o = x.o;
+    a.status = x.status;
+    a.S = x.R;
+    a.T = x.T;
+    a.k = x.idx != nullptr ? x.k : 0;
+    a.W = x.W;
+    a.m = x.m;
+    a.scale_log2 = x.scale * 1.4426950408889634f;
+    a.log2_theta_tok = x.log2_theta_tok;
+    a.log2_theta_cmp = x.log2_theta_cmp;
+    const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

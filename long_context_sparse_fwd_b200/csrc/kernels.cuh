@@ -32,6 +32,10 @@ cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t T, int m, i
                              cudaStream_t stream);
 cudaError_t launch_attend_simt(const AttnArgs &a, cudaStream_t stream);
 
+// attend_tc.cu: tcgen05 prefill attention for H=64, D=512, rope 64 (CSA when idx != null, else HCA)
+bool attend_tc_supported(int H, int D, int r, int k);
+cudaError_t launch_attend_tc(const AttnArgs &a, cudaStream_t stream);
+
 // index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
 cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t T, int HI,
