@@ -23,7 +23,10 @@
 // Softmax runs in the exp2 domain with a reference max per head that is only raised when a block
 // exceeds it by more than 2^8 (then O is rescaled in TMEM after the previous P V completes),
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
-// Roles: warps 0-3 softmax + epilogue, warps 4-5 gather keys, warp 6 owns TMEM and issues MMAs.
+// Keys arrive by TMA: window rows as 64-row tiles, entry rows by tile::gather4 (4 rows per
+// instruction) straight into the swizzled layout.
+// Roles: warps 0-3 softmax + epilogue, warp 4 issues the key TMAs, warp 5 owns TMEM and issues MMAs
+// from an event loop (a P V never waits for the next block's keys).
 // Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
 #include <algorithm>
 
@@ -44,10 +47,10 @@ constexpr int QCHUNK = HH * 128;                // 8 KB
 constexpr int KCHUNK = KB * 128;                // 8 KB
 constexpr int STAGE = NCH * KCHUNK;             // 64 KB
 constexpr int PBUF = HH * 128;                  // 8 KB
-constexpr int NUM_THREADS = 224;
+constexpr int NUM_THREADS = 192;
 constexpr int SM_THREADS = 128;
-constexpr int PROD_THREADS = 64;
-constexpr int MMA_WARP = 6;
+constexpr int PROD_WARP = 4;
+constexpr int MMA_WARP = 5;
 constexpr float TAU = 8.f;
 constexpr uint32_t COL_RW = 256, COL_S = 320;
 constexpr uint32_t LANE16 = 16u << 16;
@@ -73,18 +76,6 @@ struct TcArgs {
     float scale_log2;         // softmax scale * log2(e)
     double log2_theta_tok, log2_theta_cmp;
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -113,7 +104,9 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 // byte offset of 16-byte unit `u` (0..7) of row `row` inside a 128-byte-swizzled [rows x 128 B] chunk
 __device__ __forceinline__ uint32_t sw128(int row, int u) { return (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4)); }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                 const __grid_constant__ CUtensorMap tm_c, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -122,7 +115,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
     uint8_t *sP = smem + OFF_P;
     float *rope_cs = reinterpret_cast<float *>(smem + OFF_ROPE);     // [theta: 0 tok, 1 cmp][pair][cos, sin]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *kv_full = bars + 0;     // [2] 64 producer arrivals
+    uint64_t *kv_full = bars + 0;     // [2] TMA transaction count
     uint64_t *kv_empty = bars + 2;    // [2] MMA commit
     uint64_t *s_full = bars + 4;      // [2] MMA commit
     uint64_t *p_ready = bars + 6;     // [2] 128 softmax arrivals
@@ -131,6 +124,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 10);
     volatile int *abort = reinterpret_cast<volatile int *>(bars + 11);
     int *nlist = reinterpret_cast<int *>(bars + 12);
+    uint64_t *q_tma = bars + 13;      // TMA of the 7 un-rotated Q chunks
     int *elist = reinterpret_cast<int *>(smem + OFF_LIST);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -141,15 +135,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&kv_full[i], PROD_THREADS);
+            mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_ready[i], SM_THREADS);
         }
         mbar_init(o_done, 1);
         mbar_init(q_ready, SM_THREADS);
+        mbar_init(q_tma, 1);
         *abort = 0;
         fence_barrier_init();
+        mbar_arrive_expect_tx(q_tma, 7 * QCHUNK);
+        for (int dc = 0; dc < 7; ++dc) tma_load_2d(sQ + dc * QCHUNK, &tm_q, q_tma, dc * 64, (int)(t * HH));
     }
     if (warp == MMA_WARP) {
         tmem_alloc(tmem_ptr, TMEM_COLS);
@@ -165,10 +162,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
     if (warp == 4) {          // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
         if (a.idx != nullptr) {
             const int32_t *ir = a.idx + t * (int64_t)a.k;
+            int vals[32];   // k <= 1024: all loads in flight at once
+#pragma unroll
+            for (int i = 0; i < 32; ++i) vals[i] = i * 32 + lane < a.k ? __ldg(ir + i * 32 + lane) : -1;
             int cnt = 0;
-            for (int base = 0; base < a.k; base += 32) {
-                const int j = base + lane;
-                const int s = j < a.k ? ir[j] : -1;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int s = vals[i];
                 const bool ok = s >= 0 && (int64_t)s < vis;
                 if (s >= 0 && !ok) report(a.status, CSA_ERR_INVALID_ARG);
                 const unsigned mk = __ballot_sync(0xffffffffu, ok);
@@ -191,12 +191,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
         // =============== softmax + epilogue (warp w owns TMEM lane quarter w) ===============
         const int tid = threadIdx.x;
         // Q tile: 7 un-rotated chunks, rope chunk rotated with theta_cmp (7) and theta_tok (8)
-        for (int i = tid; i < HH * 64; i += SM_THREADS) {
-            const int h = i >> 6, u = i & 63, dc = u >> 3, uu = u & 7;
-            const uint4 v = *reinterpret_cast<const uint4 *>(a.q + ((t * HH + h) * (int64_t)DD) + u * 8);
-            if (dc < 7) {
-                *reinterpret_cast<uint4 *>(sQ + dc * QCHUNK + sw128(h, uu)) = v;
-            } else {
+        uint4 qv[4];   // rope chunk: 64 heads x 8 units, 4 per thread, all loads in flight
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+            const int i = tid + r4 * SM_THREADS, h = i >> 3, uu = i & 7;
+            qv[r4] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((t * HH + h) * (int64_t)DD) + 448 + uu * 8));
+        }
+#pragma unroll
+        for (int r4 = 0; r4 < 4; ++r4) {
+            const int i = tid + r4 * SM_THREADS, h = i >> 3, uu = i & 7;
+            const uint4 v = qv[r4];
+            {
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
                 uint32_t oc[4], ot[4];
 #pragma unroll
@@ -325,102 +330,110 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) attend_tc_kernel(TcArgs a)
             float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
             for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-    } else if (warp < 6) {
-        // =============== key gather: cp.async into 128-byte-swizzled stages ===============
-        const int ptid = threadIdx.x - 128;
+    } else if (warp == PROD_WARP) {
+        // =============== key loads: TMA tiles (window) and TMA gather4 (entries) ===============
         for (int b = 0; b < nb; ++b) {
             const int st = b & 1;
-            if (!mbar_wait(&kv_empty[st], ((b >> 1) & 1) ^ 1, abort, a.status)) break;
-            const bool win = b < nbw;
-            const int kbase = win ? b * KB : (b - nbw) * KB;
-            const int nk = win ? min(KB, nw - kbase) : min(KB, ne - kbase);
-            const uint32_t sbase = smem_u32(sKV + st * STAGE);
-            for (int i = ptid; i < KB * 64; i += PROD_THREADS) {
-                const int key = i >> 6, u = i & 63;
-                const bool valid = key < nk;
-                const uint16_t *row = a.q;        // any mapped address when not valid (0 bytes read)
-                if (valid) {
-                    if (win) {
-                        row = a.kv_rot + (wpos0 + kbase + key) * (int64_t)DD;
-                    } else {
-                        const int64_t s = a.idx != nullptr ? (int64_t)elist[kbase + key] : (int64_t)(kbase + key);
-                        row = a.C + s * DD;
-                    }
+            if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], ((b >> 1) & 1) ^ 1, abort, a.status))) break;
+            uint8_t *stage = sKV + st * STAGE;
+            if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], STAGE);
+            __syncwarp();
+            if (b < nbw) {
+                // 64 consecutive rows from wpos0 + b*64; rows past t are masked in the softmax,
+                // rows past S are zero-filled by the TMA unit
+                if (lane < NCH)
+                    tma_load_2d(stage + lane * KCHUNK, &tm_kv, &kv_full[st], lane * 64, (int)(wpos0 + b * KB));
+            } else {
+                const int kbase = (b - nbw) * KB;
+                const int nk = min(KB, ne - kbase);
+                const int g = lane >> 1;                 // rows 4g .. 4g+3
+                int r[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int key = min(4 * g + i, nk - 1);   // padding rows repeat a valid row (masked)
+                    r[i] = a.idx != nullptr ? elist[kbase + key] : kbase + key;
                 }
-                cp_async16(sbase + (u >> 3) * KCHUNK + sw128(key, u & 7), row + (valid ? u * 8 : 0), valid ? 16u : 0u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int dc = (lane & 1) * 4 + j;
+                    tma_gather4(stage + dc * KCHUNK + 4 * g * 128, &tm_c, &kv_full[st], dc * 64, r[0], r[1], r[2], r[3]);
+                }
             }
-            cp_async_arrive_noinc(&kv_full[st]);
         }
-        cp_async_wait_all();
-    } else if (warp == MMA_WARP) {
-        // =============== MMA issuer ===============
+        // never leave with copies in flight into this CTA's shared memory
+        if (lane == 0 && nb > 0) {
+            const int last = nb - 1;
+            for (int b = max(0, last - 1); b <= last; ++b)
+                mbar_wait(&kv_full[b & 1], (b >> 1) & 1, abort, a.status, 100000000ull);
+        }
+    } else if (warp == MMA_WARP && lane == 0) {
+        // =============== MMA issuer: one thread, event loop ===============
         const uint32_t idS = idesc_bf16(64, 64);
         const uint32_t idPV256 = idesc_bf16(64, 256, true);
         const uint32_t idPV192 = idesc_bf16(64, 192, true);
         const uint32_t idPV64 = idesc_bf16(64, 64, true);
-        const uint32_t q0 = smem_u32(sQ), kv0 = smem_u32(sKV), p0 = smem_u32(sP);
-        int s_issued = 0, pv_issued = 0;
-        bool ok = nb == 0 || mbar_wait(q_ready, 0, abort, a.status);
-        auto issue_S = [&](int b) -> bool {
-            const int st = b & 1;
-            if (!mbar_wait(&kv_full[st], (b >> 1) & 1, abort, a.status)) return false;
-            fence_async_smem();
-            tc_fence_after();
-            if (elect_one()) {
-                const uint32_t d = tmem + COL_S + (b & 1) * LANE16;
-                const int rope_chunk = b < nbw ? 8 : 7;
+        // descriptors are formed once; a tile / k-step offset is added to the start-address field
+        const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t dK = sdesc_sw128(smem_u32(sKV), 16, 1024);
+        const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
+        const uint64_t dV = sdesc_sw128(smem_u32(sKV), KCHUNK, 1024);
+        int nS = 0, nPV = 0;
+        bool ok = nb == 0 || (mbar_wait(q_ready, 0, abort, a.status) && mbar_wait(q_tma, 0, abort, a.status));
+        uint64_t t_progress = globaltimer();
+        uint32_t polls = 0;
+        while (ok && nPV < nb) {
+            bool progressed = false;
+            // S(nS) needs its keys and a free logits buffer (softmax of nS-2 finished, i.e. PV(nS-2) issued)
+            if (nS < nb && nS <= nPV + 1 && mbar_try_wait(&kv_full[nS & 1], (nS >> 1) & 1)) {
+                tc_fence_after();
+                const int st = nS & 1;
+                const uint32_t d = tmem + COL_S + (uint32_t)st * LANE16;
+                const int rope_chunk = nS < nbw ? 8 : 7;
                 for (int dc = 0; dc < NCH; ++dc) {
-                    const uint32_t qa = q0 + (dc < 7 ? dc : rope_chunk) * QCHUNK;
-                    const uint32_t kb = kv0 + st * STAGE + dc * KCHUNK;
+                    const uint64_t qa = dQ + (((dc < 7 ? dc : rope_chunk) * QCHUNK) >> 4);
+                    const uint64_t kb = dK + ((st * STAGE + dc * KCHUNK) >> 4);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(d, sdesc_sw128(qa + ks * 32, 16, 1024), sdesc_sw128(kb + ks * 32, 16, 1024), idS,
-                                 (dc | ks) != 0);
+                    for (int ks = 0; ks < 4; ++ks) mma_bf16(d, qa + 2 * ks, kb + 2 * ks, idS, (dc | ks) != 0);
                 }
-                mma_commit(&s_full[b & 1]);
+                mma_commit(&s_full[st]);
+                ++nS;
+                progressed = true;
             }
-            __syncwarp();
-            return true;
-        };
-        if (ok && nb > 0) { ok = issue_S(0); s_issued = ok ? 1 : 0; }
-        for (int b = 0; ok && b < nb; ++b) {
-            if (b + 1 < nb) {
-                if (!issue_S(b + 1)) { ok = false; break; }
-                s_issued = b + 2;
-            }
-            if (!mbar_wait(&p_ready[b & 1], (b >> 1) & 1, abort, a.status)) { ok = false; break; }
-            tc_fence_after();
-            if (elect_one()) {
-                const int st = b & 1;
+            // PV(nPV) needs the softmax of block nPV
+            if (nPV < nS && mbar_try_wait(&p_ready[nPV & 1], (nPV >> 1) & 1)) {
+                tc_fence_after();
+                const int b = nPV, st = b & 1;
                 const bool win = b < nbw;
-                const uint32_t pa = p0 + (b & 1) * PBUF;
-                const uint32_t vb = kv0 + st * STAGE;
+                const uint32_t drope = win ? tmem + LANE16 + COL_RW : tmem + LANE16 + 192;
+                const bool rope_first = win ? (b == 0) : (b == nbw);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = sdesc_sw128(pa + ks * 32, 16, 1024);
-                    const uint32_t koff = ks * 2 * 1024;
-                    // dims 0..255 -> O_lo
-                    mma_bf16(tmem, ad, sdesc_sw128(vb + koff, KCHUNK, 1024), idPV256, b > 0 || ks > 0);
-                    // dims 256..447 -> O_hi cols 0..191
-                    mma_bf16(tmem + LANE16, ad, sdesc_sw128(vb + 4 * KCHUNK + koff, KCHUNK, 1024), idPV192,
-                             b > 0 || ks > 0);
-                    // dims 448..511 -> the rope accumulator of this block's branch
-                    const uint32_t drope = win ? tmem + LANE16 + COL_RW : tmem + LANE16 + 192;
-                    const bool first = win ? (b == 0) : (b == nbw);
-                    mma_bf16(drope, ad, sdesc_sw128(vb + 7 * KCHUNK + koff, KCHUNK, 1024), idPV64, !first || ks > 0);
+                    const uint64_t ad = dP + ((st * PBUF + ks * 32) >> 4);
+                    const uint64_t vb = dV + ((st * STAGE + ks * 2048) >> 4);
+                    mma_bf16(tmem, ad, vb, idPV256, b > 0 || ks > 0);                                  // dims 0..255
+                    mma_bf16(tmem + LANE16, ad, vb + ((4 * KCHUNK) >> 4), idPV192, b > 0 || ks > 0);   // 256..447
+                    mma_bf16(drope, ad, vb + ((7 * KCHUNK) >> 4), idPV64, !rope_first || ks > 0);     // 448..511
                 }
                 mma_commit(&kv_empty[st]);
                 mma_commit(o_done);
+                ++nPV;
+                progressed = true;
             }
-            __syncwarp();
-            pv_issued = b + 1;
+            if (progressed) {
+                t_progress = globaltimer();
+            } else if ((++polls & 255u) == 0) {
+                if (*abort) { ok = false; break; }
+                if (globaltimer() - t_progress > 2000000000ull) {
+                    *abort = 1;
+                    report(a.status, CSA_ERR_TIMEOUT);
+                    ok = false;
+                }
+            }
         }
         // leave only when every issued MMA has completed
-        if (pv_issued > 0) mbar_wait(o_done, (pv_issued - 1) & 1, abort, a.status, 100000000ull);
-        if (s_issued > pv_issued) {
-            const int b = s_issued - 1;
-            mbar_wait(&s_full[b & 1], (b >> 1) & 1, abort, a.status, 100000000ull);
-        }
+        mbar_wait(q_tma, 0, abort, a.status, 100000000ull);
+        if (nPV > 0) mbar_wait(o_done, (nPV - 1) & 1, abort, a.status, 100000000ull);
+        if (nS > nPV) mbar_wait(&s_full[(nS - 1) & 1], ((nS - 1) >> 1) & 1, abort, a.status, 100000000ull);
     }
     tc_fence_before();
     __syncthreads();
@@ -457,9 +470,14 @@ cudaError_t launch_attend_tc(const AttnArgs &x, cudaStream_t stream)
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
     const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
+    CUtensorMap tq, tkv, tc;
+    if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_sw128(&tkv, x.W > 0 ? x.win : x.q, x.W > 0 ? (uint64_t)x.R : (uint64_t)x.R * HH, DD, 64))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_sw128(&tc, x.T > 0 ? x.C : x.q, x.T > 0 ? (uint64_t)x.T : 1, DD, 1)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(a);
+    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(tq, tkv, tc, a);
     return cudaGetLastError();
 }
 

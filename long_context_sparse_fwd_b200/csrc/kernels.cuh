@@ -1,6 +1,8 @@
 // kernels.cuh -- launchers shared between the C-ABI layer and the kernel files.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace csa {
@@ -35,6 +37,9 @@ cudaError_t launch_attend_simt(const AttnArgs &a, cudaStream_t stream);
 // attend_tc.cu: tcgen05 prefill attention for H=64, D=512, rope 64 (CSA when idx != null, else HCA)
 bool attend_tc_supported(int H, int D, int r, int k);
 cudaError_t launch_attend_tc(const AttnArgs &a, cudaStream_t stream);
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128-byte swizzle
+bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
