@@ -23,9 +23,10 @@
 // Softmax runs in the exp2 domain with a reference max per head that is only raised when a block
 // exceeds it by more than 2^8 (then O is rescaled in TMEM after the previous P V completes),
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
-// Keys arrive by TMA: window rows as 64-row tiles, entry rows by tile::gather4 (4 rows per
-// instruction) straight into the swizzled layout.
-// Roles: warps 0-3 softmax + epilogue, warp 4 issues the key TMAs, warp 5 owns TMEM and issues MMAs
+// Keys arrive by 16-byte cp.async from four loader warps (each row 1 KB, two 512-byte coalesced
+// halves per warp instruction), written straight into the swizzled layout; with four warps in
+// flight a 64-key block of random rows lands in about a microsecond.
+// Roles: warps 0-3 softmax + epilogue, warps 4-7 load keys, warp 8 owns TMEM and issues MMAs
 // from an event loop (a P V never waits for the next block's keys).
 // Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
 #include <algorithm>
@@ -47,10 +48,11 @@ constexpr int QCHUNK = HH * 128;                // 8 KB
 constexpr int KCHUNK = KB * 128;                // 8 KB
 constexpr int STAGE = NCH * KCHUNK;             // 64 KB
 constexpr int PBUF = HH * 128;                  // 8 KB
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 288;
 constexpr int SM_THREADS = 128;
-constexpr int PROD_WARP = 4;
-constexpr int MMA_WARP = 5;
+constexpr int LOAD_WARP0 = 4;                   // warps 4..7 load keys
+constexpr int LOAD_THREADS = 128;
+constexpr int MMA_WARP = 8;
 constexpr float TAU = 8.f;
 constexpr uint32_t COL_RW = 256, COL_S = 320;
 constexpr uint32_t LANE16 = 16u << 16;
@@ -76,6 +78,18 @@ struct TcArgs {
     float scale_log2;         // softmax scale * log2(e)
     double log2_theta_tok, log2_theta_cmp;
 };
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -105,8 +119,7 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ uint32_t sw128(int row, int u) { return (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4)); }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
-                 const __grid_constant__ CUtensorMap tm_c, TcArgs a)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -115,7 +128,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint8_t *sP = smem + OFF_P;
     float *rope_cs = reinterpret_cast<float *>(smem + OFF_ROPE);     // [theta: 0 tok, 1 cmp][pair][cos, sin]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *kv_full = bars + 0;     // [2] TMA transaction count
+    uint64_t *kv_full = bars + 0;     // [2] one cp.async arrival per loader thread
     uint64_t *kv_empty = bars + 2;    // [2] MMA commit
     uint64_t *s_full = bars + 4;      // [2] MMA commit
     uint64_t *p_ready = bars + 6;     // [2] 128 softmax arrivals
@@ -135,7 +148,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&kv_full[i], 1);
+            mbar_init(&kv_full[i], LOAD_THREADS);
             mbar_init(&kv_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_ready[i], SM_THREADS);
@@ -146,7 +159,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         *abort = 0;
         fence_barrier_init();
         mbar_arrive_expect_tx(q_tma, 7 * QCHUNK);
-        for (int dc = 0; dc < 7; ++dc) tma_load_2d(sQ + dc * QCHUNK, &tm_q, q_tma, dc * 64, (int)(t * HH));
+        const uint64_t pol_q = policy_evict_first();     // q is read once
+        for (int dc = 0; dc < 7; ++dc) tma_load_2d_hint(sQ + dc * QCHUNK, &tm_q, q_tma, dc * 64, (int)(t * HH), pol_q);
     }
     if (warp == MMA_WARP) {
         tmem_alloc(tmem_ptr, TMEM_COLS);
@@ -159,7 +173,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         rope_cs[(th * 32 + p) * 2] = c;
         rope_cs[(th * 32 + p) * 2 + 1] = s;
     }
-    if (warp == 4) {          // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
+    if (warp == LOAD_WARP0) { // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
         if (a.idx != nullptr) {
             const int32_t *ir = a.idx + t * (int64_t)a.k;
             int vals[32];   // k <= 1024: all loads in flight at once
@@ -322,50 +336,42 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 }
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4 *>(orow + c + j) =
-                        make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv);
+                for (int j = 0; j < 32; j += 4)   // streaming stores: the output is not re-read here
+                    __stcs(reinterpret_cast<float4 *>(orow + c + j),
+                           make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv));
             }
         } else if (nb == 0) {
             float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
             for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-    } else if (warp == PROD_WARP) {
-        // =============== key loads: TMA tiles (window) and TMA gather4 (entries) ===============
+    } else if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
+        // =============== key loads: 16-byte cp.async into the swizzled stages ===============
+        const int lw = warp - LOAD_WARP0;        // rows 16*lw .. 16*lw+15 of each block
         for (int b = 0; b < nb; ++b) {
             const int st = b & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], ((b >> 1) & 1) ^ 1, abort, a.status))) break;
-            uint8_t *stage = sKV + st * STAGE;
-            if (lane == 0) mbar_arrive_expect_tx(&kv_full[st], STAGE);
-            __syncwarp();
-            if (b < nbw) {
-                // 64 consecutive rows from wpos0 + b*64; rows past t are masked in the softmax,
-                // rows past S are zero-filled by the TMA unit
-                if (lane < NCH)
-                    tma_load_2d(stage + lane * KCHUNK, &tm_kv, &kv_full[st], lane * 64, (int)(wpos0 + b * KB));
-            } else {
-                const int kbase = (b - nbw) * KB;
-                const int nk = min(KB, ne - kbase);
-                const int g = lane >> 1;                 // rows 4g .. 4g+3
-                int r[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int key = min(4 * g + i, nk - 1);   // padding rows repeat a valid row (masked)
-                    r[i] = a.idx != nullptr ? elist[kbase + key] : kbase + key;
+            const bool win = b < nbw;
+            const int kbase = win ? b * KB : (b - nbw) * KB;
+            const int nk = win ? min(KB, nw - kbase) : min(KB, ne - kbase);
+            const uint32_t sbase = smem_u32(sKV + st * STAGE);
+#pragma unroll 4
+            for (int r = 0; r < 16; ++r) {
+                const int key = lw * 16 + r;
+                const bool valid = key < nk;
+                const uint16_t *row = a.q;       // any mapped address for padding rows (zero-filled, 0 bytes read)
+                if (valid) {
+                    if (win) row = a.kv_rot + (wpos0 + kbase + key) * (int64_t)DD;
+                    else row = a.C + (int64_t)(a.idx != nullptr ? elist[kbase + key] : kbase + key) * DD;
                 }
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int dc = (lane & 1) * 4 + j;
-                    tma_gather4(stage + dc * KCHUNK + 4 * g * 128, &tm_c, &kv_full[st], dc * 64, r[0], r[1], r[2], r[3]);
+                for (int hlf = 0; hlf < 2; ++hlf) {
+                    const int u = lane + 32 * hlf;
+                    cp_async16(sbase + (u >> 3) * KCHUNK + sw128(key, u & 7), row + (valid ? u * 8 : 0), valid ? 16u : 0u);
                 }
             }
+            cp_async_arrive_noinc(&kv_full[st]);
         }
-        // never leave with copies in flight into this CTA's shared memory
-        if (lane == 0 && nb > 0) {
-            const int last = nb - 1;
-            for (int b = max(0, last - 1); b <= last; ++b)
-                mbar_wait(&kv_full[b & 1], (b >> 1) & 1, abort, a.status, 100000000ull);
-        }
+        cp_async_wait_all();   // never leave with copies in flight into this CTA's shared memory
     } else if (warp == MMA_WARP && lane == 0) {
         // =============== MMA issuer: one thread, event loop ===============
         const uint32_t idS = idesc_bf16(64, 64);
@@ -385,6 +391,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             bool progressed = false;
             // S(nS) needs its keys and a free logits buffer (softmax of nS-2 finished, i.e. PV(nS-2) issued)
             if (nS < nb && nS <= nPV + 1 && mbar_try_wait(&kv_full[nS & 1], (nS >> 1) & 1)) {
+                fence_async_smem();   // keys were written by cp.async (generic proxy); the MMA reads via the async proxy
                 tc_fence_after();
                 const int st = nS & 1;
                 const uint32_t d = tmem + COL_S + (uint32_t)st * LANE16;
@@ -470,14 +477,11 @@ cudaError_t launch_attend_tc(const AttnArgs &x, cudaStream_t stream)
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
     const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
-    CUtensorMap tq, tkv, tc;
+    CUtensorMap tq;
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_sw128(&tkv, x.W > 0 ? x.win : x.q, x.W > 0 ? (uint64_t)x.R : (uint64_t)x.R * HH, DD, 64))
-        return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_sw128(&tc, x.T > 0 ? x.C : x.q, x.T > 0 ? (uint64_t)x.T : 1, DD, 1)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(tq, tkv, tc, a);
+    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(tq, a);
     return cudaGetLastError();
 }
 
