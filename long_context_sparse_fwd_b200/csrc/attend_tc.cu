@@ -24,8 +24,8 @@
 // exceeds it by more than 2^8 (then O is rescaled in TMEM after the previous P V completes),
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
 // Keys arrive by 16-byte cp.async from four loader warps (each row 1 KB, two 512-byte coalesced
-// halves per warp instruction), written straight into the swizzled layout; with four warps in
-// flight a 64-key block of random rows lands in about a microsecond.
+// halves per warp instruction), written straight into the swizzled layout.
+// The output is staged through the idle key buffers and written by TMA tensor stores.
 // Roles: warps 0-3 softmax + epilogue, warps 4-7 load keys, warp 8 owns TMEM and issues MMAs
 // from an event loop (a P V never waits for the next block's keys).
 // Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
@@ -58,6 +58,8 @@ constexpr uint32_t COL_RW = 256, COL_S = 320;
 constexpr uint32_t LANE16 = 16u << 16;
 constexpr uint32_t TMEM_COLS = 512;
 
+constexpr int OBOX = HH * 128;                  // output staging box: 64 rows x 32 fp32 (8 KB)
+
 constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_KV = OFF_Q + (size_t)QCH * QCHUNK;       // 72 KB
 constexpr size_t OFF_P = OFF_KV + 2 * (size_t)STAGE;          // 200 KB
@@ -84,6 +86,7 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
+// arrive on `bar` when this thread's earlier cp.async copies have landed (no pending-count increment)
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
 {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -119,7 +122,7 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ uint32_t sw128(int row, int u) { return (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4)); }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -128,7 +131,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
     uint8_t *sP = smem + OFF_P;
     float *rope_cs = reinterpret_cast<float *>(smem + OFF_ROPE);     // [theta: 0 tok, 1 cmp][pair][cos, sin]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *kv_full = bars + 0;     // [2] one cp.async arrival per loader thread
+    uint64_t *kv_full = bars + 0;     // [2] loader arrivals
     uint64_t *kv_empty = bars + 2;    // [2] MMA commit
     uint64_t *s_full = bars + 4;      // [2] MMA commit
     uint64_t *p_ready = bars + 6;     // [2] 128 softmax arrivals
@@ -148,7 +151,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&kv_full[i], LOAD_THREADS);
+            mbar_init(&kv_full[i], LOAD_THREADS);   // one cp.async arrival per loader thread
             mbar_init(&kv_empty[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_ready[i], SM_THREADS);
@@ -315,8 +318,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
         if (ok && nb > 0) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
             const bool has_win = nbw > 0, has_ent = nbe > 0;
+            // Every MMA has completed, so the key stages are idle: stage this query's output there as
+            // 16 boxes of [64 heads x 32 floats] (128-byte swizzled) for TMA tensor stores.
             for (int c = 0; c < 256; c += 32) {
                 float v[32], rw[32];
                 tmem_ld32(tq + c, v);
@@ -335,10 +339,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                         v[j + 1] = (-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct);
                     }
                 }
+                uint8_t *box = sKV + (half * 8 + (c >> 5)) * OBOX;
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)   // streaming stores: the output is not re-read here
-                    __stcs(reinterpret_cast<float4 *>(orow + c + j),
-                           make_float4(v[j] * inv, v[j + 1] * inv, v[j + 2] * inv, v[j + 3] * inv));
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4 *>(box + sw128(h, u)) =
+                        make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
+            }
+            fence_async_smem();
+            named_barrier_sync(1, SM_THREADS);
+            if (tid == 0) {
+                for (int bx = 0; bx < DD / 32; ++bx) tma_store_2d(&tm_o, sKV + bx * OBOX, bx * 32, (int)(t * HH));
+                bulk_commit();
+                bulk_wait_read_all();   // the staging buffer must be read out before the CTA exits
             }
         } else if (nb == 0) {
             float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
@@ -477,11 +489,12 @@ cudaError_t launch_attend_tc(const AttnArgs &x, cudaStream_t stream)
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
     const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
-    CUtensorMap tq;
+    CUtensorMap tq, to;
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_f32_sw128(&to, x.o, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(tq, a);
+    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(tq, to, a);
     return cudaGetLastError();
 }
 

@@ -287,18 +287,30 @@ EncodeTiledFn encode_fn()
 
 }  // namespace
 
-// 2-D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128-byte swizzle.
-bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+static bool make_tmap_sw128(CUtensorMap *map, const void *base, CUtensorMapDataType dt, uint32_t esize, uint64_t rows,
+                            uint64_t cols, uint32_t box_rows)
 {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {64, box_rows};
+    cuuint64_t strides[1] = {cols * esize};
+    cuuint32_t box[2] = {128 / esize, box_rows};   // one 128-byte swizzle span per box row
     cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128-byte swizzle.
+bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    return make_tmap_sw128(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, cols, box_rows);
+}
+
+// 2-D fp32 tensor map over a row-major [rows, cols] matrix, box [box_rows, 32], 128-byte swizzle.
+bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    return make_tmap_sw128(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols, box_rows);
 }
 
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)

@@ -40,6 +40,8 @@ cudaError_t launch_attend_tc(const AttnArgs &a, cudaStream_t stream);
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128-byte swizzle
 bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// 2-D fp32 tensor map, box [box_rows, 32], 128-byte swizzle
+bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
