@@ -1,6 +1,7 @@
 // api.cu -- the C ABI declared in include/csa.h: host-side argument checks, workspace layout and
 // launch sequencing. Nothing here allocates device memory; every buffer is the caller's.
 #include <math.h>
+#include <algorithm>
 #include <string.h>
 
 #include "kernels.cuh"
@@ -164,7 +165,8 @@ size_t csa_workspace_size(csa_op op, const csa_dims *d)
     case CSA_OP_HCA_FORWARD:
         return kStatusBytes;
     case CSA_OP_DECODE:
-        return kStatusBytes + scores_bytes(d->B, d->T) + align256(sizeof(int32_t) * (size_t)d->B * (size_t)d->k);
+        return kStatusBytes + align256(std::max(scores_bytes(d->B, d->T), decode_index_workspace(d->B, d->T, d->k))) +
+               align256(sizeof(int32_t) * (size_t)d->B * (size_t)d->k);
     }
     return 0;
 }
@@ -325,11 +327,16 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
     CSA_TRY(reset_status(workspace, st));
     char *base = static_cast<char *>(workspace);
     float *scores = reinterpret_cast<float *>(base + kStatusBytes);
-    int32_t *idx = idx_out != nullptr ? idx_out
-                                      : reinterpret_cast<int32_t *>(base + kStatusBytes + scores_bytes(B, T));
-    CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T, HI,
-                                 dI, 1, 1, scores, st));
-    CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
+    const size_t index_ws = align256(std::max(scores_bytes(B, T), decode_index_workspace(B, T, k)));
+    int32_t *idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t *>(base + kStatusBytes + index_ws);
+    if (T > 0 && decode_index_tc_supported(T, HI, dI, k)) {
+        CSA_CUDA(launch_decode_index_tc(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
+                                        HI, dI, k, idx, scores, static_cast<int32_t *>(workspace), st));
+    } else {
+        CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
+                                     HI, dI, 1, 1, scores, st));
+        CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
+    }
     AttnArgs a;
     memset(&a, 0, sizeof a);
     a.q = static_cast<const uint16_t *>(q);

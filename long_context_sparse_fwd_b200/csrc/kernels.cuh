@@ -43,6 +43,12 @@ bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uin
 // 2-D fp32 tensor map, box [box_rows, 32], 128-byte swizzle
 bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
+// decode_tc.cu: decode index scan (tcgen05, HBM streaming) + two-stage exact top-k
+size_t decode_index_workspace(int64_t B, int64_t T, int k);
+bool decode_index_tc_supported(int64_t T, int HI, int dI, int k);
+cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t B, int64_t T, int HI,
+                                   int dI, int k, int32_t *idx, void *ws, int32_t *status, cudaStream_t stream);
+
 // index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
 cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t T, int HI,
