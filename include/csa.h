@@ -158,7 +158,9 @@ CSA_API csa_status hca_forward(const void *q, const void *kv, const void *gate, 
  *            c8 [B, T, D-rope_dim] E4M3 codes, c8_scale [B, T] fp32, c_rope [B, T, rope_dim] bf16;
  *            value = e4m3(c8) * scale on channels [0, D-rope_dim), c_rope on the rest
  *   win [B, W, D] bf16: window rows for positions P-W+1 .. P (rows at negative positions ignored)
- *   sinks [H] fp32    idx_out [B, k] int32 (out, may be NULL)    o [B, H, D] fp32 (out) */
+ *   sinks [H] fp32    idx_out [B, k] int32 (out, may be NULL)    o [B, H, D] fp32 (out)
+ * csa_workspace_size(CSA_OP_DECODE) is the recommended workspace; any workspace down to the index
+ * scores, candidates and indices is accepted and uses fewer attention splits per sequence. */
 CSA_API csa_status csa_decode(const void *q, const void *qI, const float *w, const void *kI,
                       const void *C, const uint8_t *c8, const float *c8_scale, const void *c_rope,
                       const void *win, const float *sinks, int32_t B, int32_t H, int32_t D,
@@ -175,9 +177,9 @@ CSA_API csa_status csa_decode(const void *q, const void *qI, const float *w, con
  * library holds that array until the process exits. Arguments and results are those of
  * csa_decode, without workspace and workspace_bytes. It allocates nothing.
  *   - Returns CSA_ERR_WORKSPACE, launching nothing, when the problem needs more scratch than the
- *     array holds, i.e. when csa_workspace_size(CSA_OP_DECODE, dims) exceeds
- *     csa_decode_noalloc_max_scratch() (B*T*4 + B*k*4 bytes plus alignment, e.g. B=64 sequences
- *     of T=32768 entries, or B=8 of T=262144, fit).
+ *     array holds: the index scores and candidates plus the selected indices, about
+ *     B*T*4 + 2*B*ceil(T/8192)*k*4 + B*k*4 bytes (e.g. B=64 sequences of T=32768 entries, or
+ *     B=8 of T=262144, fit). Whatever the array has left is used for attention splits.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  *     that device current; make that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's contents: calls that

@@ -113,6 +113,29 @@ AttnArgs prefill_args(const void *q, const void *C, const void *kv_rot, const in
     return a;
 }
 
+// Decode workspace: status word, index scores/candidates, selected indices, then the attention
+// split partials (optional: fewer splits when the workspace is smaller).
+size_t decode_index_bytes(int64_t B, int64_t T, int32_t k)
+{
+    return align256(std::max(scores_bytes(B, T), decode_index_workspace(B, T, k)));
+}
+
+int decode_splits_preferred(int64_t B)
+{
+    return (int)std::min<int64_t>(8, std::max<int64_t>(1, (2 * 148 + B - 1) / std::max<int64_t>(B, 1)));
+}
+
+}  // namespace
+
+namespace csa {
+size_t decode_workspace_min(int64_t B, int64_t T, int32_t k)
+{
+    return kStatusBytes + decode_index_bytes(B, T, k) + align256(sizeof(int32_t) * (size_t)B * (size_t)k);
+}
+}  // namespace csa
+
+namespace {
+
 // Prefill attention: the tcgen05 kernel for the V4 head shape (64 heads x 512, rope 64), else the
 // general CUDA-core kernel.
 cudaError_t attend_any(const AttnArgs &a, cudaStream_t st)
@@ -165,8 +188,8 @@ size_t csa_workspace_size(csa_op op, const csa_dims *d)
     case CSA_OP_HCA_FORWARD:
         return kStatusBytes;
     case CSA_OP_DECODE:
-        return kStatusBytes + align256(std::max(scores_bytes(d->B, d->T), decode_index_workspace(d->B, d->T, d->k))) +
-               align256(sizeof(int32_t) * (size_t)d->B * (size_t)d->k);
+        return decode_workspace_min(d->B, d->T, d->k) +
+               align256(attend_tc_decode_partials(d->B, decode_splits_preferred(d->B)));
     }
     return 0;
 }
@@ -322,13 +345,14 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
     dims.B = B;
     dims.T = T;
     dims.k = k;
-    CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_DECODE, &dims)));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, decode_workspace_min(B, T, k)));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
     char *base = static_cast<char *>(workspace);
     float *scores = reinterpret_cast<float *>(base + kStatusBytes);
-    const size_t index_ws = align256(std::max(scores_bytes(B, T), decode_index_workspace(B, T, k)));
+    const size_t index_ws = decode_index_bytes(B, T, k);
     int32_t *idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t *>(base + kStatusBytes + index_ws);
+    const size_t used = decode_workspace_min(B, T, k);
     if (T > 0 && decode_index_tc_supported(T, HI, dI, k)) {
         CSA_CUDA(launch_decode_index_tc(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
                                         HI, dI, k, idx, scores, static_cast<int32_t *>(workspace), st));
@@ -362,6 +386,12 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
     a.scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / sqrt((double)D));
     a.log2_theta_tok = rope_dim > 0 ? log2(theta_tok) : 0.0;
     a.log2_theta_cmp = rope_dim > 0 ? log2(theta_cmp) : 0.0;
+    if (attend_tc_supported(H, D, rope_dim, k)) {
+        // as many attention splits per sequence as the workspace holds (up to the preferred count)
+        int nsplit = decode_splits_preferred(B);
+        while (nsplit > 1 && used + align256(attend_tc_decode_partials(B, nsplit)) > workspace_bytes) --nsplit;
+        return from_cuda(launch_attend_tc_decode(a, nsplit, reinterpret_cast<float *>(base + used), st));
+    }
     return from_cuda(launch_attend_simt(a, st));
 }
 

@@ -31,6 +31,9 @@
 // Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
 #include <algorithm>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -68,15 +71,19 @@ constexpr size_t OFF_BAR = OFF_ROPE + 2 * 32 * 2 * 4;
 constexpr size_t OFF_LIST = OFF_BAR + 256;
 
 struct TcArgs {
-    const uint16_t *q;        // [S, 64, 512]
-    const uint16_t *kv_rot;   // [S, 512]
-    const uint16_t *C;        // [T, 512]
-    const int32_t *idx;       // [S, k] or null (HCA)
+    const uint16_t *q;        // [R, 64, 512] (R = S prefill rows or B decode sequences)
+    const uint16_t *kv_rot;   // prefill: [S, 512] window rows; decode: [B, W, 512] (positions P-W+1..P)
+    const uint16_t *C;        // prefill: [T, 512]; decode: [B, T, 512] bf16 (or null: FP8 cache)
+    const uint8_t *c8;        // decode FP8 cache: [B, T, 448] E4M3 codes
+    const float *c8_scale;    //                   [B, T]
+    const uint16_t *c_rope;   //                   [B, T, 64] bf16
+    const int32_t *idx;       // [R, k] or null (HCA: every visible entry)
     const float *sinks;       // [64]
-    float *o;                 // [S, 64, 512]
+    float *o;                 // [R, 64, 512]
+    float *part_ml;           // split partials: [R*nsplit, 64, 2] (log2-domain reference max, sum)
     int32_t *status;
-    int64_t S, T;
-    int k, W, m;
+    int64_t S, T, P;          // S: prefill rows; P: decode position
+    int k, W, m, decode, nsplit;
     float scale_log2;         // softmax scale * log2(e)
     double log2_theta_tok, log2_theta_cmp;
 };
@@ -135,19 +142,30 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint64_t *kv_empty = bars + 2;    // [2] MMA commit
     uint64_t *s_full = bars + 4;      // [2] MMA commit
     uint64_t *p_ready = bars + 6;     // [2] 128 softmax arrivals
-    uint64_t *o_done = bars + 8;      // MMA commit after each P V
-    uint64_t *q_ready = bars + 9;     // 128 softmax arrivals
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 10);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 11);
-    int *nlist = reinterpret_cast<int *>(bars + 12);
-    uint64_t *q_tma = bars + 13;      // TMA of the 7 un-rotated Q chunks
+    // P V completion: block b commits o_done[b & 1]. When the softmax of block b waits for P V of
+    // block b-1, every earlier completion of that barrier (block b-3) is already known to be done
+    // (it preceded S of block b), so a parity wait cannot mistake an older phase for the one wanted.
+    uint64_t *o_done = bars + 8;      // [2]
+    uint64_t *o_final = bars + 10;    // single use: every MMA of this CTA has completed
+    uint64_t *q_ready = bars + 11;    // 128 softmax arrivals
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 12);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 13);
+    int *nlist = reinterpret_cast<int *>(bars + 14);
+    uint64_t *q_tma = bars + 15;      // TMA of the 7 un-rotated Q chunks
     int *elist = reinterpret_cast<int *>(smem + OFF_LIST);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = a.S - 1 - (int64_t)blockIdx.x;          // longest key lists first
-    const int64_t vis = visible_entries(t, a.m, a.T);
+    // prefill: one CTA per query row, longest key lists first; decode: nsplit CTAs per sequence
+    const int64_t row = a.decode ? (int64_t)(blockIdx.x / a.nsplit) : a.S - 1 - (int64_t)blockIdx.x;
+    const int split = a.decode ? (int)(blockIdx.x % a.nsplit) : 0;
+    const bool partial = a.nsplit > 1;
+    const int64_t t = a.decode ? a.P : row;                   // position of the query
+    const int64_t vis = a.decode ? a.T : visible_entries(t, a.m, a.T);
     const int64_t wpos0 = max((int64_t)0, t - a.W + 1);
     const int nw = (int)(t - wpos0 + 1);
+    const uint16_t *win0 = a.decode ? a.kv_rot + (row * a.W + (a.W - nw)) * (int64_t)DD
+                                    : a.kv_rot + wpos0 * (int64_t)DD;   // first window row
+    const uint16_t *ent0 = a.decode && a.C != nullptr ? a.C + row * a.T * DD : a.C;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -156,14 +174,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(&s_full[i], 1);
             mbar_init(&p_ready[i], SM_THREADS);
         }
-        mbar_init(o_done, 1);
+        mbar_init(&o_done[0], 1);
+        mbar_init(&o_done[1], 1);
+        mbar_init(o_final, 1);
         mbar_init(q_ready, SM_THREADS);
         mbar_init(q_tma, 1);
         *abort = 0;
         fence_barrier_init();
         mbar_arrive_expect_tx(q_tma, 7 * QCHUNK);
         const uint64_t pol_q = policy_evict_first();     // q is read once
-        for (int dc = 0; dc < 7; ++dc) tma_load_2d_hint(sQ + dc * QCHUNK, &tm_q, q_tma, dc * 64, (int)(t * HH), pol_q);
+        for (int dc = 0; dc < 7; ++dc) tma_load_2d_hint(sQ + dc * QCHUNK, &tm_q, q_tma, dc * 64, (int)(row * HH), pol_q);
     }
     if (warp == MMA_WARP) {
         tmem_alloc(tmem_ptr, TMEM_COLS);
@@ -178,7 +198,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     if (warp == LOAD_WARP0) { // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
         if (a.idx != nullptr) {
-            const int32_t *ir = a.idx + t * (int64_t)a.k;
+            const int32_t *ir = a.idx + row * (int64_t)a.k;
             int vals[32];   // k <= 1024: all loads in flight at once
 #pragma unroll
             for (int i = 0; i < 32; ++i) vals[i] = i * 32 + lane < a.k ? __ldg(ir + i * 32 + lane) : -1;
@@ -202,7 +222,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
     const int ne = *nlist;
-    const int nbw = (nw + KB - 1) / KB, nbe = (ne + KB - 1) / KB, nb = nbw + nbe;
+    const int nbw = (nw + KB - 1) / KB, nbe = (ne + KB - 1) / KB, nb_all = nbw + nbe;
+    // this CTA's share of the key blocks (window blocks first, then entry blocks)
+    const int gb0 = (int)((int64_t)split * nb_all / a.nsplit);
+    const int nb = (int)((int64_t)(split + 1) * nb_all / a.nsplit) - gb0;
+    const bool has_win = gb0 < nbw && nb > 0, has_ent = gb0 + nb > nbw;
 
     if (warp < 4) {
         // =============== softmax + epilogue (warp w owns TMEM lane quarter w) ===============
@@ -212,7 +236,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
             const int i = tid + r4 * SM_THREADS, h = i >> 3, uu = i & 7;
-            qv[r4] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((t * HH + h) * (int64_t)DD) + 448 + uu * 8));
+            qv[r4] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((row * HH + h) * (int64_t)DD) + 448 + uu * 8));
         }
 #pragma unroll
         for (int r4 = 0; r4 < 4; ++r4) {
@@ -239,13 +263,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
         const int h = warp * 16 + (lane & 15);
         const int half = lane >> 4;
-        const float zl = a.sinks[h] * 1.4426950408889634f;
+        // the sink seeds the running max and sum; split partials leave it to the combine step
+        const float zl = partial ? -INFINITY : a.sinks[h] * 1.4426950408889634f;
         float m_ref = zl, l = (zl == -INFINITY) ? 0.f : 1.f;
         const uint32_t tq = tmem + ((uint32_t)(warp * 32) << 16);
         bool ok = true;
         for (int b = 0; b < nb && ok; ++b) {
             const int buf = b & 1;
-            const int nk = b < nbw ? min(KB, nw - b * KB) : min(KB, ne - (b - nbw) * KB);
+            const int gb = gb0 + b;
+            const int nk = gb < nbw ? min(KB, nw - gb * KB) : min(KB, ne - (gb - nbw) * KB);
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (b >> 1) & 1, abort, a.status));
             if (!ok) break;
             tc_fence_after();
@@ -295,7 +321,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!active) { m_ref = pm; l = pl; corr = pc; need = pn != 0; }
             if (__any_sync(0xffffffffu, need)) {
                 // O must hold every earlier P V before it is rescaled
-                ok = __all_sync(0xffffffffu, mbar_wait(o_done, (b - 1) & 1, abort, a.status));
+                ok = __all_sync(0xffffffffu, mbar_wait(&o_done[(b - 1) & 1], ((b - 1) >> 1) & 1, abort, a.status));
                 tc_fence_after();
                 if (ok) {
                     for (uint32_t c = 0; c < COL_S; c += 32) {
@@ -314,11 +340,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_arrive(&p_ready[buf]);
         }
         // ---------------- epilogue ----------------
-        if (ok && nb > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (nb - 1) & 1, abort, a.status));
+        if (ok && nb > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, abort, a.status));
         if (ok && nb > 0) {
             tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const bool has_win = nbw > 0, has_ent = nbe > 0;
+            const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
             // Every MMA has completed, so the key stages are idle: stage this query's output there as
             // 16 boxes of [64 heads x 32 floats] (128-byte swizzled) for TMA tensor stores.
             for (int c = 0; c < 256; c += 32) {
@@ -348,37 +373,83 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_async_smem();
             named_barrier_sync(1, SM_THREADS);
             if (tid == 0) {
-                for (int bx = 0; bx < DD / 32; ++bx) tma_store_2d(&tm_o, sKV + bx * OBOX, bx * 32, (int)(t * HH));
+                const int y = (int)((row * a.nsplit + split) * HH);
+                for (int bx = 0; bx < DD / 32; ++bx) tma_store_2d(&tm_o, sKV + bx * OBOX, bx * 32, y);
                 bulk_commit();
                 bulk_wait_read_all();   // the staging buffer must be read out before the CTA exits
             }
-        } else if (nb == 0) {
-            float *orow = a.o + ((t * HH + h) * (int64_t)DD) + half * 256;
+        } else if (nb == 0 && !partial) {
+            float *orow = a.o + ((row * HH + h) * (int64_t)DD) + half * 256;
             for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        if (partial && lane < 16) {   // reference max (log2 domain) and sum of this split; an empty split has l = 0
+            float *ml = a.part_ml + ((row * a.nsplit + split) * HH + h) * 2;
+            ml[0] = ok && nb > 0 ? m_ref : -INFINITY;
+            ml[1] = ok && nb > 0 ? l : 0.f;
         }
     } else if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
         // =============== key loads: 16-byte cp.async into the swizzled stages ===============
         const int lw = warp - LOAD_WARP0;        // rows 16*lw .. 16*lw+15 of each block
         for (int b = 0; b < nb; ++b) {
-            const int st = b & 1;
+            const int st = b & 1, gb = gb0 + b;
             if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], ((b >> 1) & 1) ^ 1, abort, a.status))) break;
-            const bool win = b < nbw;
-            const int kbase = win ? b * KB : (b - nbw) * KB;
+            const bool win = gb < nbw;
+            const int kbase = win ? gb * KB : (gb - nbw) * KB;
             const int nk = win ? min(KB, nw - kbase) : min(KB, ne - kbase);
+            if (!win && a.C == nullptr) {
+                // FP8 entry cache: codes * per-entry scale on channels [0,448), bf16 rope on [448,512),
+                // converted to bf16 here and stored into the swizzled stage
+                uint8_t *stage = sKV + st * STAGE;
+#pragma unroll 2
+                for (int r = 0; r < 16; ++r) {
+                    const int key = lw * 16 + r;
+                    uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
+                    if (key < nk) {
+                        const int64_t e = row * a.T + (a.idx != nullptr ? elist[kbase + key] : kbase + key);
+                        if (lane < 28) {
+                            const float sc = __ldg(a.c8_scale + e);
+                            const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(a.c8 + e * 448) + lane);
+                            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+                            uint32_t ow[8];
+#pragma unroll
+                            for (int q2 = 0; q2 < 8; ++q2) {
+                                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                                    (__nv_fp8x2_storage_t)((cw[q2 >> 1] >> ((q2 & 1) * 16)) & 0xffffu), __NV_E4M3);
+                                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+                                ow[q2] = pack_bf2(f.x * sc, f.y * sc);
+                            }
+                            o0 = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                            o1 = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                        } else {
+                            const uint4 *rr = reinterpret_cast<const uint4 *>(a.c_rope + e * 64);
+                            o0 = __ldg(rr + 2 * (lane - 28));
+                            o1 = __ldg(rr + 2 * (lane - 28) + 1);
+                        }
+                    }
+                    // lane < 28: dims [16*lane, 16*lane+16); lanes 28..31: rope dims 448 + 16*(lane-28)
+                    const int d0 = lane < 28 ? 16 * lane : 448 + 16 * (lane - 28);
+                    const int dc = d0 >> 6, u0 = (d0 & 63) >> 3;
+                    *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0)) = o0;
+                    *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0 + 1)) = o1;
+                }
+                fence_async_smem();
+                mbar_arrive(&kv_full[st]);
+                continue;
+            }
             const uint32_t sbase = smem_u32(sKV + st * STAGE);
 #pragma unroll 4
             for (int r = 0; r < 16; ++r) {
                 const int key = lw * 16 + r;
                 const bool valid = key < nk;
-                const uint16_t *row = a.q;       // any mapped address for padding rows (zero-filled, 0 bytes read)
+                const uint16_t *rowp = a.q;      // any mapped address for padding rows (zero-filled, 0 bytes read)
                 if (valid) {
-                    if (win) row = a.kv_rot + (wpos0 + kbase + key) * (int64_t)DD;
-                    else row = a.C + (int64_t)(a.idx != nullptr ? elist[kbase + key] : kbase + key) * DD;
+                    if (win) rowp = win0 + (int64_t)(kbase + key) * DD;
+                    else rowp = ent0 + (int64_t)(a.idx != nullptr ? elist[kbase + key] : kbase + key) * DD;
                 }
 #pragma unroll
                 for (int hlf = 0; hlf < 2; ++hlf) {
                     const int u = lane + 32 * hlf;
-                    cp_async16(sbase + (u >> 3) * KCHUNK + sw128(key, u & 7), row + (valid ? u * 8 : 0), valid ? 16u : 0u);
+                    cp_async16(sbase + (u >> 3) * KCHUNK + sw128(key, u & 7), rowp + (valid ? u * 8 : 0), valid ? 16u : 0u);
                 }
             }
             cp_async_arrive_noinc(&kv_full[st]);
@@ -407,7 +478,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tc_fence_after();
                 const int st = nS & 1;
                 const uint32_t d = tmem + COL_S + (uint32_t)st * LANE16;
-                const int rope_chunk = nS < nbw ? 8 : 7;
+                const int rope_chunk = gb0 + nS < nbw ? 8 : 7;
                 for (int dc = 0; dc < NCH; ++dc) {
                     const uint64_t qa = dQ + (((dc < 7 ? dc : rope_chunk) * QCHUNK) >> 4);
                     const uint64_t kb = dK + ((st * STAGE + dc * KCHUNK) >> 4);
@@ -421,10 +492,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // PV(nPV) needs the softmax of block nPV
             if (nPV < nS && mbar_try_wait(&p_ready[nPV & 1], (nPV >> 1) & 1)) {
                 tc_fence_after();
-                const int b = nPV, st = b & 1;
-                const bool win = b < nbw;
+                const int b = nPV, st = b & 1, gb = gb0 + b;
+                const bool win = gb < nbw;
                 const uint32_t drope = win ? tmem + LANE16 + COL_RW : tmem + LANE16 + 192;
-                const bool rope_first = win ? (b == 0) : (b == nbw);
+                // the first block of each branch handled by this CTA starts that branch's rope accumulator
+                const bool rope_first = win ? (b == 0) : (gb == max(nbw, gb0));
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     const uint64_t ad = dP + ((st * PBUF + ks * 32) >> 4);
@@ -434,7 +506,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     mma_bf16(drope, ad, vb + ((7 * KCHUNK) >> 4), idPV64, !rope_first || ks > 0);     // 448..511
                 }
                 mma_commit(&kv_empty[st]);
-                mma_commit(o_done);
+                mma_commit(&o_done[b & 1]);
+                if (b + 1 == nb) mma_commit(o_final);
                 ++nPV;
                 progressed = true;
             }
@@ -451,8 +524,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         // leave only when every issued MMA has completed
         mbar_wait(q_tma, 0, abort, a.status, 100000000ull);
-        if (nPV > 0) mbar_wait(o_done, (nPV - 1) & 1, abort, a.status, 100000000ull);
-        if (nS > nPV) mbar_wait(&s_full[(nS - 1) & 1], ((nS - 1) >> 1) & 1, abort, a.status, 100000000ull);
+        if (nPV == nb && nb > 0) {
+            mbar_wait(o_final, 0, abort, a.status, 100000000ull);
+        } else if (nS > 0 || nPV > 0) {
+            // stopped early: commit once more and wait for that (covers every MMA issued so far)
+            mma_commit(o_final);
+            mbar_wait(o_final, 0, abort, a.status, 100000000ull);
+        }
     }
     tc_fence_before();
     __syncthreads();
@@ -469,32 +547,97 @@ bool attend_tc_supported(int H, int D, int r, int k)
     return H == HH && D == DD && r == RR && k <= 1024;
 }
 
-cudaError_t launch_attend_tc(const AttnArgs &x, cudaStream_t stream)
+// Combine the split partials of decode: per (sequence, head), o = sum_i 2^(m_i - M) O_i / L with
+// L = 2^(z - M) + sum_i 2^(m_i - M) l_i and M the largest of the split maxima and the sink z (all in
+// the log2 domain). The sink enters here exactly once.
+__global__ void __launch_bounds__(128)
+combine_splits_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml, const float *__restrict__ sinks,
+                      int nsplit, float *__restrict__ o)
 {
-    if (x.R == 0) return cudaSuccess;
+    const int64_t b = blockIdx.x / HH;
+    const int h = blockIdx.x % HH;
+    const float z = sinks[h] * 1.4426950408889634f;
+    float M = z;
+    for (int i = 0; i < nsplit; ++i) {
+        const float mi = part_ml[((b * nsplit + i) * HH + h) * 2];
+        M = fmaxf(M, mi);
+    }
+    float L = (z == -INFINITY) ? 0.f : exp2f(z - M);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < nsplit; ++i) {
+        const float mi = part_ml[((b * nsplit + i) * HH + h) * 2];
+        const float li = part_ml[((b * nsplit + i) * HH + h) * 2 + 1];
+        if (mi == -INFINITY || li == 0.f) continue;   // empty split: its O was never written
+        const float wgt = exp2f(mi - M);
+        L += wgt * li;
+        const float4 v = reinterpret_cast<const float4 *>(part_o + ((b * nsplit + i) * HH + h) * (int64_t)DD)[threadIdx.x];
+        acc.x += wgt * v.x;
+        acc.y += wgt * v.y;
+        acc.z += wgt * v.z;
+        acc.w += wgt * v.w;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    reinterpret_cast<float4 *>(o + (b * HH + h) * (int64_t)DD)[threadIdx.x] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
+static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, float *part_ml, cudaStream_t stream)
+{
     TcArgs a;
     a.q = x.q;
     a.kv_rot = x.win;
     a.C = x.C;
+    a.c8 = x.c8;
+    a.c8_scale = x.c8_scale;
+    a.c_rope = x.c_rope;
     a.idx = x.idx;
     a.sinks = x.sinks;
     a.o = x.o;
+    a.part_ml = part_ml;
     a.status = x.status;
     a.S = x.R;
     a.T = x.T;
+    a.P = x.P;
     a.k = x.idx != nullptr ? x.k : 0;
     a.W = x.W;
     a.m = x.m;
+    a.decode = x.decode;
+    a.nsplit = nsplit;
     a.scale_log2 = x.scale * 1.4426950408889634f;
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
     const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
     CUtensorMap tq, to;
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap_f32_sw128(&to, x.o, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
+    if (!make_tmap_f32_sw128(&to, out_rows, (uint64_t)x.R * nsplit * HH, DD, 64)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<(unsigned)x.R, NUM_THREADS, smem, stream>>>(tq, to, a);
+    attend_tc_kernel<<<(unsigned)(x.R * nsplit), NUM_THREADS, smem, stream>>>(tq, to, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_attend_tc(const AttnArgs &x, cudaStream_t stream)
+{
+    if (x.R == 0) return cudaSuccess;
+    return launch_tc(x, 1, x.o, nullptr, stream);
+}
+
+size_t attend_tc_decode_partials(int64_t B, int nsplit)
+{
+    return nsplit <= 1 ? 0 : (size_t)B * nsplit * HH * (DD + 2) * sizeof(float);
+}
+
+// Decode: nsplit CTAs per sequence write partials into `part` (attend_tc_decode_partials bytes),
+// then one combine launch produces o. nsplit == 1 writes o directly.
+cudaError_t launch_attend_tc_decode(const AttnArgs &x, int nsplit, float *part, cudaStream_t stream)
+{
+    if (x.R == 0) return cudaSuccess;
+    if (nsplit <= 1) return launch_tc(x, 1, x.o, nullptr, stream);
+    float *part_o = part;
+    float *part_ml = part + (size_t)x.R * nsplit * HH * DD;
+    cudaError_t e = launch_tc(x, nsplit, part_o, part_ml, stream);
+    if (e != cudaSuccess) return e;
+    combine_splits_kernel<<<(unsigned)(x.R * HH), 128, 0, stream>>>(part_o, part_ml, x.sinks, nsplit, x.o);
     return cudaGetLastError();
 }
 

@@ -55,16 +55,13 @@ csa_status csa_decode_noalloc(const void *q, const void *qI, const float *w, con
                               float softmax_scale, int32_t *idx_out, float *o, void *stream)
 {
     if (B < 0 || T < 0 || k < 1) return CSA_ERR_INVALID_ARG;
-    csa_dims dims = {};
-    dims.B = B;
-    dims.T = T;
-    dims.k = k;
-    if (csa_workspace_size(CSA_OP_DECODE, &dims) > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;
+    if (csa::decode_workspace_min(B, T, k) > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;
     void *scratch = nullptr;
     const csa_status s = scratch_on_current_device(&scratch);
     if (s != CSA_OK) return s;
-    // csa_decode zeroes the status word at the start of the scratch and writes every score and
-    // index it later reads, so nothing left over from an earlier call is used.
+    // csa_decode zeroes the status word at the start of the scratch and writes every score, index
+    // and attention partial it later reads, so nothing left over from an earlier call is used. It
+    // takes as many attention splits per sequence as the rest of the array holds.
     return csa_decode(q, qI, w, kI, C, c8, c8_scale, c_rope, win, sinks, B, H, D, T, HI, dI, k, W, rope_dim, P,
                       theta_tok, theta_cmp, softmax_scale, idx_out, o, scratch, kNoAllocScratchBytes, stream);
 }

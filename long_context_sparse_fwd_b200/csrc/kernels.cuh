@@ -37,11 +37,17 @@ cudaError_t launch_attend_simt(const AttnArgs &a, cudaStream_t stream);
 // attend_tc.cu: tcgen05 prefill attention for H=64, D=512, rope 64 (CSA when idx != null, else HCA)
 bool attend_tc_supported(int H, int D, int r, int k);
 cudaError_t launch_attend_tc(const AttnArgs &a, cudaStream_t stream);
+// decode: nsplit CTAs per sequence with partials in `part` (attend_tc_decode_partials bytes) + combine
+size_t attend_tc_decode_partials(int64_t B, int nsplit);
+cudaError_t launch_attend_tc_decode(const AttnArgs &a, int nsplit, float *part, cudaStream_t stream);
 
 // 2-D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, 64], 128-byte swizzle
 bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // 2-D fp32 tensor map, box [box_rows, 32], 128-byte swizzle
 bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+// api.cu: smallest workspace csa_decode accepts (no attention split partials)
+size_t decode_workspace_min(int64_t B, int64_t T, int32_t k);
 
 // decode_tc.cu: decode index scan (tcgen05, HBM streaming) + two-stage exact top-k
 size_t decode_index_workspace(int64_t B, int64_t T, int k);
