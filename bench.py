@@ -164,8 +164,10 @@ class Step:
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.phases) + 1)]
 
     def launches_per_step(self):
-        # compress_entries + rotate_rows, index_scores + topk, attention
-        return {"csa_prefill": 5, "hca_prefill": 3, "csa_decode": 3}[self.wl.kind]
+        # library kernels per step on the tensor-core paths these workloads take:
+        # prefill: compress_entries + rotate_rows, fused index/top-k (CSA), attention;
+        # decode: index scan, chunk top-k, merge, split attention, combine
+        return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 5}[self.wl.kind]
 
     def run(self, timed: bool):
         wl, x, csa = self.wl, self.x, self.csa
