@@ -120,9 +120,10 @@ size_t decode_index_bytes(int64_t B, int64_t T, int32_t k)
     return align256(std::max(scores_bytes(B, T), decode_index_workspace(B, T, k)));
 }
 
+// attention CTAs per sequence: about one wave of CTAs over the SMs (one CTA fits per SM)
 int decode_splits_preferred(int64_t B)
 {
-    return (int)std::min<int64_t>(8, std::max<int64_t>(1, (2 * 148 + B - 1) / std::max<int64_t>(B, 1)));
+    return (int)std::min<int64_t>(8, std::max<int64_t>(1, 148 / std::max<int64_t>(B, 1)));
 }
 
 }  // namespace

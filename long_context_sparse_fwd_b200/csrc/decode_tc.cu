@@ -5,8 +5,8 @@
 //     I[b,s] = sum_h w[b,h] * ReLU(qI[b,h,:] . kI[b,s,:])
 //
 // The k^I stream (T x d_I bf16 per sequence: 8 MiB at 128K context, 64 MiB at 1M) dominates the
-// step, so the score kernel is built to run at HBM speed: each CTA streams a contiguous chunk of
-// one sequence's k^I through a 6-deep TMA ring (128-byte swizzle), the tensor cores form
+// step, so the score kernel is built to run at HBM speed: one persistent CTA per SM streams a
+// contiguous range of k^I tiles through a 6-deep TMA ring (128-byte swizzle), the tensor cores form
 // D[s,h] = kI[s,:] . qI[b,h,:] (entries on TMEM lanes, M=128 x N=HI), and each epilogue thread
 // reduces its entry's HI heads in registers and writes one fp32 score.
 //
@@ -29,7 +29,6 @@ constexpr int BM = 128;
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_THREADS = 128;
 constexpr int MAX_STAGES = 6;
-constexpr int SCORE_CHUNK = 4096;      // entries per score CTA
 constexpr int SEL_CHUNK = 8192;        // scores per first-stage select CTA
 constexpr int SEL_THREADS = 512;
 constexpr int MERGE_THREADS = 1024;
@@ -38,10 +37,13 @@ struct ScoreParams {
     const float *w;      // [B, HI]
     float *scores;       // [B, T]
     int32_t *status;
-    int64_t T;
-    int HI, dI, stages;
+    int64_t T, G;        // entries per sequence; total tiles (B * tiles per sequence)
+    int HI, dI, stages, tps;
 };
 
+// Persistent: CTA c takes the contiguous tile range [c*G/n, (c+1)*G/n) of the flat list
+// (sequence-major, 128 entries per tile), so the HBM stream never idles on a wave tail. q^I of the
+// current sequence is double-buffered; a range crosses at most a few sequence boundaries.
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         ScoreParams p)
@@ -51,25 +53,30 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const int kchunks = p.dI / 64;
     const uint32_t b_bytes = (uint32_t)kchunks * p.HI * 128;
     const uint32_t a_bytes = (uint32_t)kchunks * BM * 128;
-    uint8_t *sB = smem;
-    uint8_t *sA = sB + b_bytes;
-    float *sw = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [HI]
+    uint8_t *sB = smem;                                   // [2][b_bytes]
+    uint8_t *sA = sB + 2 * b_bytes;
+    float *sw = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [HI] of the current sequence
     uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 256);
-    uint64_t *full = bars, *empty = bars + 8, *tfull = bars + 16, *tempty = bars + 18, *qfull = bars + 20;
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 21);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 22);
+    uint64_t *full = bars, *empty = bars + 8, *tfull = bars + 16, *tempty = bars + 18;
+    uint64_t *qfull = bars + 20, *qempty = bars + 22;     // [2] each
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 24);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 25);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = blockIdx.y;
-    const int64_t s_begin = (int64_t)blockIdx.x * SCORE_CHUNK;
-    const int64_t s_end = min(p.T, s_begin + SCORE_CHUNK);
-    const int ntiles = (int)((s_end - s_begin + BM - 1) / BM);
+    const int64_t g_lo = (int64_t)blockIdx.x * p.G / gridDim.x;
+    const int64_t g_hi = (int64_t)(blockIdx.x + 1) * p.G / gridDim.x;
+    const int ntiles = (int)(g_hi - g_lo);
+    const int64_t b_first = g_lo / p.tps;
     const uint32_t tcols = p.HI * 2 <= 32 ? 32 : (p.HI * 2 <= 64 ? 64 : (p.HI * 2 <= 128 ? 128 : 256));
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], EPI_THREADS); }
-        mbar_init(qfull, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], EPI_THREADS);
+            mbar_init(&qfull[i], 1);
+            mbar_init(&qempty[i], 1);
+        }
         *abort = 0;
         fence_barrier_init();
     }
@@ -77,8 +84,6 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         tmem_alloc(tmem_ptr, tcols);
         tmem_relinquish();
     }
-    if (warp >= 2)
-        for (int i = threadIdx.x - 64; i < p.HI; i += EPI_THREADS) sw[i] = p.w[(int64_t)b * p.HI + i];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -87,19 +92,29 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     if (warp == 0) {
         if (elect_one() && ntiles > 0) {
             const uint64_t pol_stream = policy_evict_first();   // k^I is read once per step
-            mbar_arrive_expect_tx(qfull, b_bytes);
-            for (int c = 0; c < kchunks; ++c) tma_load_2d(sB + c * p.HI * 128, &tm_q, qfull, c * 64, b * p.HI);
-            int issued = 0;
+            int issued = 0, nseg = 0;
             for (int i = 0; i < ntiles; ++i) {
+                const int64_t g = g_lo + i, b = g / p.tps;
+                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+                if (i == 0 || it == 0) {   // a new sequence: its q^I into buffer j & 1
+                    if (!mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status)) break;
+                    mbar_arrive_expect_tx(&qfull[j & 1], b_bytes);
+                    for (int c = 0; c < kchunks; ++c)
+                        tma_load_2d(sB + (j & 1) * b_bytes + c * p.HI * 128, &tm_q, &qfull[j & 1], c * 64,
+                                    (int)(b * p.HI));
+                    nseg = j + 1;
+                }
                 const int st = i % p.stages;
                 if (!mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status)) break;
                 mbar_arrive_expect_tx(&full[st], a_bytes);
-                const int y = (int)((int64_t)b * p.T + s_begin + (int64_t)i * BM);
+                const int y = (int)(b * p.T + (int64_t)it * BM);
                 for (int c = 0; c < kchunks; ++c)
                     tma_load_2d_hint(sA + st * a_bytes + c * BM * 128, &tm_k, &full[st], c * 64, y, pol_stream);
                 issued = i + 1;
             }
-            mbar_wait(qfull, 0, abort, p.status, 100000000ull);
+            // never leave with copies in flight into this CTA's shared memory
+            for (int j = max(0, nseg - 2); j < nseg; ++j)
+                mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status, 100000000ull);
             for (int i = max(0, issued - p.stages); i < issued; ++i)
                 mbar_wait(&full[i % p.stages], (i / p.stages) & 1, abort, p.status, 100000000ull);
         }
@@ -107,28 +122,40 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (lane == 0 && ntiles > 0) {
             const uint32_t idesc = idesc_bf16(BM, p.HI);
             const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
-            bool ok = mbar_wait(qfull, 0, abort, p.status);
             int issued = 0;
-            for (int i = 0; ok && i < ntiles; ++i) {
+            for (int i = 0; i < ntiles; ++i) {
+                const int64_t g = g_lo + i, b = g / p.tps;
+                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+                if (i == 0 || it == 0)
+                    if (!mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status)) break;
                 const int st = i % p.stages, buf = i & 1;
                 if (!mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1, abort, p.status)) break;
                 if (!mbar_wait(&full[st], (i / p.stages) & 1, abort, p.status)) break;
                 tc_fence_after();
+                const uint64_t dBj = dB + (((j & 1) * b_bytes) >> 4);
                 for (int c = 0; c < kchunks; ++c)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
                         mma_bf16(tmem + buf * p.HI, dA + ((st * a_bytes + c * BM * 128 + ks * 32) >> 4),
-                                 dB + ((c * p.HI * 128 + ks * 32) >> 4), idesc, (c | ks) != 0);
+                                 dBj + ((c * p.HI * 128 + ks * 32) >> 4), idesc, (c | ks) != 0);
                 mma_commit(&empty[st]);
                 mma_commit(&tfull[buf]);
+                if (i + 1 == ntiles || it + 1 == p.tps) mma_commit(&qempty[j & 1]);   // done with this q^I
                 issued = i + 1;
             }
             if (issued > 0) mbar_wait(&tfull[(issued - 1) & 1], ((issued - 1) >> 1) & 1, abort, p.status, 100000000ull);
         }
     } else {
-        const int quarter = warp & 3;
+        const int quarter = warp & 3, etid = threadIdx.x - 64;
         const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
         for (int i = 0; i < ntiles; ++i) {
+            const int64_t g = g_lo + i, b = g / p.tps;
+            const int it = (int)(g - b * p.tps);
+            if (i == 0 || it == 0) {   // index weights of the new sequence
+                named_barrier_sync(1, EPI_THREADS);
+                for (int h = etid; h < p.HI; h += EPI_THREADS) sw[h] = p.w[b * p.HI + h];
+                named_barrier_sync(1, EPI_THREADS);
+            }
             const int buf = i & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i >> 1) & 1, abort, p.status))) break;
             tc_fence_after();
@@ -139,20 +166,20 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                     tmem_ld32(taddr0 + buf * p.HI + h0, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc = fmaf(sw[h0 + j], fmaxf(v[j], 0.f), acc);
+                    for (int jj = 0; jj < 32; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
                     h0 += 16;
                 } else {
                     float v[16];
                     tmem_ld16(taddr0 + buf * p.HI + h0, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc = fmaf(sw[h0 + j], fmaxf(v[j], 0.f), acc);
+                    for (int jj = 0; jj < 16; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
                 }
             }
             tc_fence_before();
             mbar_arrive(&tempty[buf]);
-            const int64_t s = s_begin + (int64_t)i * BM + quarter * 32 + lane;
-            if (s < s_end) p.scores[(int64_t)b * p.T + s] = acc + 0.0f;
+            const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
+            if (s < p.T) p.scores[b * p.T + s] = acc + 0.0f;
         }
     }
     tc_fence_before();
@@ -194,6 +221,8 @@ __device__ __forceinline__ int block_incl_scan(int v, int *wsum, int *total)
 
 // Keep the k largest of keys[0..n) (ties: smaller position first). Writes the kept positions in
 // ascending order to pos[0..min(k,n)) and returns that count. hist: 256 words; sh: 40 words.
+// The radix digits start at the highest bit where the keys differ (scores of one query usually
+// share sign and leading exponent bits, which would put every key into one or two bins).
 __device__ int block_select(const uint32_t *keys, int n, int k, int *pos, uint32_t *hist, int *sh)
 {
     if (n <= k) {
@@ -201,14 +230,61 @@ __device__ int block_select(const uint32_t *keys, int n, int k, int *pos, uint32
         __syncthreads();
         return n;
     }
-    uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
+    // smallest and largest key
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        lo = min(lo, keys[i]);
+        hi = max(hi, keys[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    uint32_t *red = reinterpret_cast<uint32_t *>(hist);   // 2 x 32 words of scratch before the passes
+    if ((threadIdx.x & 31) == 0) {
+        red[threadIdx.x >> 5] = lo;
+        red[32 + (threadIdx.x >> 5)] = hi;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int nw = blockDim.x >> 5;
+        uint32_t l2 = threadIdx.x < nw ? red[threadIdx.x] : 0xffffffffu;
+        uint32_t h2 = threadIdx.x < nw ? red[32 + threadIdx.x] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            l2 = min(l2, __shfl_xor_sync(0xffffffffu, l2, o));
+            h2 = max(h2, __shfl_xor_sync(0xffffffffu, h2, o));
+        }
+        if (threadIdx.x == 0) {
+            sh[35] = (int)l2;
+            sh[36] = (int)h2;
+        }
+    }
+    __syncthreads();
+    lo = (uint32_t)sh[35];
+    hi = (uint32_t)sh[36];
+    __syncthreads();
+    uint32_t prefix, mask, remaining = (uint32_t)k;
+    int lowbit;   // bits [0, lowbit) are still undecided
+    if (lo == hi) {
+        prefix = hi;
+        mask = 0xffffffffu;
+        lowbit = 0;
+    } else {
+        const int top = 31 - __clz(lo ^ hi);   // highest differing bit; bits above it are common
+        mask = top == 31 ? 0u : ~((2u << top) - 1u);
+        prefix = hi & mask;
+        lowbit = top + 1;
+    }
+    while (lowbit > 0) {
+        const int width = min(8, lowbit), shift = lowbit - width;
+        const uint32_t dm = (1u << width) - 1u;
         for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const uint32_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dm], 1u);
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -238,9 +314,10 @@ __device__ int block_select(const uint32_t *keys, int n, int k, int *pos, uint32
         }
         __syncthreads();
         prefix |= (uint32_t)sh[32] << shift;
-        mask |= 255u << shift;
+        mask |= dm << shift;
         remaining -= (uint32_t)sh[33];
         const bool whole_bucket = (uint32_t)sh[34] == remaining;
+        lowbit = shift;
         __syncthreads();
         if (whole_bucket) break;
     }
@@ -361,13 +438,18 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     sp.T = T;
     sp.HI = HI;
     sp.dI = dI;
+    sp.tps = (int)((T + BM - 1) / BM);
+    sp.G = (int64_t)B * sp.tps;
     const size_t a_bytes = (size_t)(dI / 64) * BM * 128;
-    const size_t fixed = 1024 + (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
+    const size_t fixed = 1024 + 2 * (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
     sp.stages = (int)std::min<size_t>(MAX_STAGES, (227 * 1024 - fixed) / a_bytes);
     const size_t smem = fixed + (size_t)sp.stages * a_bytes;
     cudaError_t e = cudaFuncSetAttribute(decode_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 g1((unsigned)((T + SCORE_CHUNK - 1) / SCORE_CHUNK), (unsigned)B);
+    int dev = 0, nsm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
     decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     dim3 g2((unsigned)nchunks, (unsigned)B);

@@ -42,6 +42,9 @@ struct IdxParams {
     int HI, dI, m, k, Q, stages, T_cap;
 };
 
+// Exact top-k of one query's scores by one warp: radix select over order-preserving keys, starting
+// at the highest bit where the keys differ (one query's scores usually share their leading bits), then
+// one ordered pass that keeps the selected indices in ascending order (ties to the smaller index).
 __device__ __forceinline__ void topk_warp(const float *sc, int n, int k, uint32_t *hist, int32_t *out)
 {
     const int lane = threadIdx.x & 31;
@@ -49,32 +52,52 @@ __device__ __forceinline__ void topk_warp(const float *sc, int n, int k, uint32_
         for (int i = lane; i < k; i += 32) out[i] = i < n ? i : -1;
         return;
     }
-    uint32_t prefix = 0, mask = 0, remaining = (uint32_t)k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int s = lane; s < n; s += 32) {
+        const uint32_t key = score_key(sc[s]);
+        lo = min(lo, key);
+        hi = max(hi, key);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    uint32_t prefix, mask, remaining = (uint32_t)k;
+    int lowbit;
+    if (lo == hi) {
+        prefix = hi;
+        mask = 0xffffffffu;
+        lowbit = 0;
+    } else {
+        const int top = 31 - __clz(lo ^ hi);
+        mask = top == 31 ? 0u : ~((2u << top) - 1u);
+        prefix = hi & mask;
+        lowbit = top + 1;
+    }
+    while (lowbit > 0) {
+        const int width = min(8, lowbit), shift = lowbit - width;
+        const uint32_t dm = (1u << width) - 1u;
 #pragma unroll
         for (int j = 0; j < 8; ++j) hist[lane * 8 + j] = 0;
         __syncwarp();
         for (int s = lane; s < n; s += 32) {
             const uint32_t key = score_key(sc[s]);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dm], 1u);
         }
         __syncwarp();
         uint32_t c[8], tot = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) { c[j] = hist[lane * 8 + j]; tot += c[j]; }
-        // counts held by lanes above this one (higher digits)
-        uint32_t above = tot;
+        uint32_t above = tot;   // counts held by higher lanes (higher digits)
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t v = __shfl_down_sync(0xffffffffu, above, o);
             if (lane + o < 32) above += v;
         }
         above -= tot;
-        // the digit d with count(> d) < remaining <= count(>= d)
         int found = -1;
-        uint32_t above_d = 0, cnt_d = 0;
-        uint32_t run = above;
+        uint32_t above_d = 0, cnt_d = 0, run = above;
 #pragma unroll
         for (int j = 7; j >= 0; --j) {
             if (found < 0 && run + c[j] >= remaining) { found = lane * 8 + j; above_d = run; cnt_d = c[j]; }
@@ -86,8 +109,9 @@ __device__ __forceinline__ void topk_warp(const float *sc, int n, int k, uint32_
         above_d = __shfl_sync(0xffffffffu, above_d, src);
         cnt_d = __shfl_sync(0xffffffffu, cnt_d, src);
         prefix |= (uint32_t)d << shift;
-        mask |= 255u << shift;
+        mask |= dm << shift;
         remaining -= above_d;
+        lowbit = shift;
         __syncwarp();
         if (cnt_d == remaining) break;   // the whole bucket is taken
     }
