@@ -29,6 +29,7 @@ constexpr int BM = 128;
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_THREADS = 128;
 constexpr int MAX_STAGES = 6;
+constexpr int NACC = 4;                // TMEM accumulators (each HI columns) in flight
 constexpr int SEL_CHUNK = 8192;        // scores per first-stage select CTA
 constexpr int SEL_THREADS = 512;
 constexpr int MERGE_THREADS = 1024;
@@ -57,23 +58,25 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     uint8_t *sA = sB + 2 * b_bytes;
     float *sw = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [HI] of the current sequence
     uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 256);
-    uint64_t *full = bars, *empty = bars + 8, *tfull = bars + 16, *tempty = bars + 18;
-    uint64_t *qfull = bars + 20, *qempty = bars + 22;     // [2] each
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 24);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 25);
+    uint64_t *full = bars, *empty = bars + 8, *tfull = bars + 16, *tempty = bars + 20;   // tfull/tempty: [NACC]
+    uint64_t *qfull = bars + 24, *qempty = bars + 26;     // [2] each
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 28);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 29);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t g_lo = (int64_t)blockIdx.x * p.G / gridDim.x;
     const int64_t g_hi = (int64_t)(blockIdx.x + 1) * p.G / gridDim.x;
     const int ntiles = (int)(g_hi - g_lo);
     const int64_t b_first = g_lo / p.tps;
-    const uint32_t tcols = p.HI * 2 <= 32 ? 32 : (p.HI * 2 <= 64 ? 64 : (p.HI * 2 <= 128 ? 128 : 256));
+    const uint32_t tcols = p.HI * NACC <= 32 ? 32 : (p.HI * NACC <= 64 ? 64 : (p.HI * NACC <= 128 ? 128 : (p.HI * NACC <= 256 ? 256 : 512)));
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NACC; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], EPI_THREADS);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&qfull[i], 1);
             mbar_init(&qempty[i], 1);
         }
@@ -128,8 +131,8 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
                 if (i == 0 || it == 0)
                     if (!mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status)) break;
-                const int st = i % p.stages, buf = i & 1;
-                if (!mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1, abort, p.status)) break;
+                const int st = i % p.stages, buf = i % NACC;
+                if (!mbar_wait(&tempty[buf], ((i / NACC) & 1) ^ 1, abort, p.status)) break;
                 if (!mbar_wait(&full[st], (i / p.stages) & 1, abort, p.status)) break;
                 tc_fence_after();
                 const uint64_t dBj = dB + (((j & 1) * b_bytes) >> 4);
@@ -143,11 +146,13 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 if (i + 1 == ntiles || it + 1 == p.tps) mma_commit(&qempty[j & 1]);   // done with this q^I
                 issued = i + 1;
             }
-            if (issued > 0) mbar_wait(&tfull[(issued - 1) & 1], ((issued - 1) >> 1) & 1, abort, p.status, 100000000ull);
+            if (issued > 0)
+                mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
         }
     } else {
         const int quarter = warp & 3, etid = threadIdx.x - 64;
         const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
+        float wr[64];   // index weights of the current sequence (HI == 64 keeps them in registers)
         for (int i = 0; i < ntiles; ++i) {
             const int64_t g = g_lo + i, b = g / p.tps;
             const int it = (int)(g - b * p.tps);
@@ -155,29 +160,47 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 named_barrier_sync(1, EPI_THREADS);
                 for (int h = etid; h < p.HI; h += EPI_THREADS) sw[h] = p.w[b * p.HI + h];
                 named_barrier_sync(1, EPI_THREADS);
-            }
-            const int buf = i & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i >> 1) & 1, abort, p.status))) break;
-            tc_fence_after();
-            float acc = 0.f;
-            for (int h0 = 0; h0 < p.HI; h0 += 16) {
-                if (h0 + 32 <= p.HI) {
-                    float v[32];
-                    tmem_ld32(taddr0 + buf * p.HI + h0, v);
-                    tmem_wait_ld();
+                if (p.HI == 64) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
-                    h0 += 16;
-                } else {
-                    float v[16];
-                    tmem_ld16(taddr0 + buf * p.HI + h0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
+                    for (int h = 0; h < 64; ++h) wr[h] = sw[h];
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[buf]);
+            const int buf = i % NACC;
+            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i / NACC) & 1, abort, p.status))) break;
+            tc_fence_after();
+            float acc = 0.f;
+            if (p.HI == 64) {
+                float v0[32], v1[32];
+                tmem_ld32(taddr0 + buf * 64, v0);        // both loads in flight, one wait
+                tmem_ld32(taddr0 + buf * 64 + 32, v1);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&tempty[buf]);               // the accumulator may be reused from here
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    acc = fmaf(wr[jj], fmaxf(v0[jj], 0.f), acc);
+                    acc = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), acc);
+                }
+            } else {
+                for (int h0 = 0; h0 < p.HI; h0 += 16) {
+                    if (h0 + 32 <= p.HI) {
+                        float v[32];
+                        tmem_ld32(taddr0 + buf * p.HI + h0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 32; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
+                        h0 += 16;
+                    } else {
+                        float v[16];
+                        tmem_ld16(taddr0 + buf * p.HI + h0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&tempty[buf]);
+            }
             const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
             if (s < p.T) p.scores[b * p.T + s] = acc + 0.0f;
         }
@@ -321,24 +344,28 @@ __device__ int block_select(const uint32_t *keys, int n, int k, int *pos, uint32
         __syncthreads();
         if (whole_bucket) break;
     }
-    int written = 0, eq_seen = 0;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const uint32_t key = i < n ? (keys[i] & mask) : 0u;
-        const int is_eq = (i < n && key == prefix) ? 1 : 0;
-        int eq_tot;
-        const int eq_incl = block_incl_scan(is_eq, sh, &eq_tot);
-        const int rank = eq_seen + eq_incl - is_eq;
-        const int sel = (i < n && (key > prefix || (is_eq && rank < (int)remaining))) ? 1 : 0;
-        int sel_tot;
-        const int sel_incl = block_incl_scan(sel, sh, &sel_tot);
-        if (sel) pos[written + sel_incl - 1] = i;
-        written += sel_tot;
-        eq_seen += eq_tot;
-        if (written >= k) break;
+    // ordered compaction: each thread owns a contiguous run of positions; two block scans place the
+    // kept positions (keys above the threshold, and the first `remaining` equal ones) in order
+    const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int b0 = min(n, (int)threadIdx.x * per), b1 = min(n, b0 + per);
+    int ngt = 0, neq = 0;
+    for (int i = b0; i < b1; ++i) {
+        const uint32_t key = keys[i] & mask;
+        ngt += key > prefix;
+        neq += key == prefix;
+    }
+    int eq_tot;
+    const int eq_before = block_incl_scan(neq, sh, &eq_tot) - neq;
+    int take_eq = min(max((int)remaining - eq_before, 0), neq);
+    const int cnt = ngt + take_eq;
+    int total;
+    int off = block_incl_scan(cnt, sh, &total) - cnt;
+    for (int i = b0; i < b1; ++i) {
+        const uint32_t key = keys[i] & mask;
+        if (key > prefix || (key == prefix && take_eq-- > 0)) pos[off++] = i;
     }
     __syncthreads();
-    return written;
+    return min(total, k);
 }
 
 // Stage 1: per (chunk of SEL_CHUNK scores, sequence) keep the chunk's top-k.
