@@ -36,6 +36,25 @@ WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m":
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu record, or None when the
+    kernel source changed since the counters were taken (or nothing was recorded)."""
+    import hashlib
+    try:
+        for line in open(os.path.join(ROOT, "profiles", "traffic.txt")):
+            if line.startswith("#") or not line.strip():
+                continue
+            wl, src, sha, nbytes = line.split()
+            if wl != workload:
+                continue
+            path = os.path.join(ROOT, "long_context_sparse_fwd_b200", "csrc", src)
+            if hashlib.sha256(open(path, "rb").read()).hexdigest()[:16] == sha:
+                return int(nbytes)
+    except Exception:
+        return None
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -455,7 +474,7 @@ def main():
                 "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'profiling fallback'})"
-    roof["traffic"] = None
+    roof["traffic"] = recorded_traffic(args.workload)   # ncu DRAM bytes per launch (profiles/traffic.txt)
     roof["ms_per_launch"] = float(mean_phase[dom])
 
     e2e = None
