@@ -25,7 +25,7 @@
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
 // Keys arrive by 16-byte cp.async from four loader warps (each row 1 KB, two 512-byte coalesced
 // halves per warp instruction), written straight into the swizzled layout.
-// The output is staged through the idle key buffers and written by TMA tensor stores.
+// The epilogue transposes each warp's output tile through shared memory into 128-byte row segments.
 // Roles: warps 0-3 softmax + epilogue, warps 4-7 load keys, warp 8 owns TMEM and issues MMAs
 // from an event loop (a P V never waits for the next block's keys).
 // Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
@@ -61,7 +61,6 @@ constexpr uint32_t COL_RW = 256, COL_S = 320;
 constexpr uint32_t LANE16 = 16u << 16;
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr int OBOX = HH * 128;                  // output staging box: 64 rows x 32 fp32 (8 KB)
 
 constexpr size_t OFF_Q = 0;
 constexpr size_t OFF_KV = OFF_Q + (size_t)QCH * QCHUNK;       // 72 KB
@@ -129,7 +128,7 @@ __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.
 __device__ __forceinline__ uint32_t sw128(int row, int u) { return (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4)); }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, TcArgs a)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -344,8 +343,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (ok && nb > 0) {
             tc_fence_after();
             const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
-            // Every MMA has completed, so the key stages are idle: stage this query's output there as
-            // 16 boxes of [64 heads x 32 floats] (128-byte swizzled) for TMA tensor stores.
+            // Every MMA has completed, so the P buffers are idle: each warp transposes its 32 rows x 32
+            // columns (16 heads x two dim halves) through its own 4 KB slice and writes whole 128-byte
+            // row segments (8 lanes per segment) to the output.
+            uint8_t *wbuf = sP + warp * 4096;
+            float *obase = partial ? a.o + ((row * a.nsplit + split) * HH) * (int64_t)DD   // o = partial rows
+                                   : a.o + (row * HH) * (int64_t)DD;
             for (int c = 0; c < 256; c += 32) {
                 float v[32], rw[32];
                 tmem_ld32(tq + c, v);
@@ -364,19 +367,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         v[j + 1] = (-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct);
                     }
                 }
-                uint8_t *box = sKV + (half * 8 + (c >> 5)) * OBOX;
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<float4 *>(box + sw128(h, u)) =
+                    *reinterpret_cast<float4 *>(wbuf + sw128(lane, u)) =
                         make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
-            }
-            fence_async_smem();
-            named_barrier_sync(1, SM_THREADS);
-            if (tid == 0) {
-                const int y = (int)((row * a.nsplit + split) * HH);
-                for (int bx = 0; bx < DD / 32; ++bx) tma_store_2d(&tm_o, sKV + bx * OBOX, bx * 32, y);
-                bulk_commit();
-                bulk_wait_read_all();   // the staging buffer must be read out before the CTA exits
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int pr = i * 4 + (lane >> 3), u = lane & 7;   // row pr of this warp's tile
+                    const float4 x = *reinterpret_cast<const float4 *>(wbuf + sw128(pr, u));
+                    const int hh = warp * 16 + (pr & 15);
+                    __stcs(reinterpret_cast<float4 *>(obase + hh * (int64_t)DD + (pr >> 4) * 256 + c + u * 4), x);
+                }
+                __syncwarp();
             }
         } else if (nb == 0 && !partial) {
             float *orow = a.o + ((row * HH + h) * (int64_t)DD) + half * 256;
@@ -592,7 +595,6 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     a.c_rope = x.c_rope;
     a.idx = x.idx;
     a.sinks = x.sinks;
-    a.o = x.o;
     a.part_ml = part_ml;
     a.status = x.status;
     a.S = x.R;
@@ -607,12 +609,12 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
     const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
-    CUtensorMap tq, to;
+    CUtensorMap tq;
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
-    if (!make_tmap_f32_sw128(&to, out_rows, (uint64_t)x.R * nsplit * HH, DD, 64)) return cudaErrorInvalidValue;
+    a.o = out_rows;   // final rows, or the split partials
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<(unsigned)(x.R * nsplit), NUM_THREADS, smem, stream>>>(tq, to, a);
+    attend_tc_kernel<<<(unsigned)(x.R * nsplit), NUM_THREADS, smem, stream>>>(tq, a);
     return cudaGetLastError();
 }
 
