@@ -1,5 +1,5 @@
-// attend_tc.cu -- CSA / HCA prefill attention on the 5th-generation tensor cores (H=64, D=512,
-// rope 64), one query per CTA.
+// attend_tc.cu -- CSA / HCA attention on the 5th-generation tensor cores (H=64, D=512, rope 64):
+// a persistent kernel, one CTA per SM walking the queries (prefill rows, or decode sequence splits).
 //
 // What it computes (Hugging Face Transformers docs "DeepSeek-V4", section "Hybrid attention":
 // shared K=V MQA, partial interleaved RoPE with the output rope slice rotated at -i (eq. 26), a
@@ -12,22 +12,32 @@
 // Design. A query's 64 heads form an M=64 tile; its keys (window rows first, then the entries)
 // are gathered 64 at a time with 16-byte cp.async into 128-byte-swizzled shared memory, where the
 // same tile is the K-major B operand of S = Q K^T and the MN-major B operand of O += P V:
-// the selected rows are read from L2/HBM once and shared by all 64 heads.
-//   TMEM (M=64 uses 16 lanes of each 32-lane quarter; a second tile sits at lane offset 16):
-//     lanes +0 : O_lo  cols [0,256)   output dims 0..255
-//     lanes +16: O_hi  cols [0,192)   dims 256..447, cols [192,256) entry-branch rope dims 448..511
-//     lanes +16: O_rw  cols [256,320) window-branch rope dims 448..511
-//     S_b      cols [320,384) at lanes +16*(b&1)    (double-buffered logits)
+// the selected rows are read from L2/HBM once and shared by all 64 heads. Three key stages.
+// Q lives in TMEM as the A operand of S, so shared memory holds only keys and P, and the S
+// MMA reads only the key tile from shared memory.
+//   TMEM (M=64 uses 16 lanes of each 32-lane quarter, "half 0" = lanes +0..15, "half 1" = +16..31):
+//     half 0: S_b   cols [0,64), [64,128)   double-buffered logits (on the lanes of Q, as the
+//                                  A-from-TMEM MMA requires)
+//             O_rw  cols [128,192) window-branch rope dims 448..511
+//             Q     cols [192,480) 9 chunks of 64 dims (32 columns, 2 bf16 each): 7 un-rotated,
+//                                  rope rotated with theta_cmp (chunk 7) and theta_tok (chunk 8)
+//     half 1: O     cols [0,448)   output dims 0..447, cols [448,512) entry-branch rope dims
+//   (accumulator column ranges start on multiples of 64)
 //   The rope slice of each branch accumulates separately so each can be rotated back by -t
 //   with its own theta in the epilogue.
 // Softmax runs in the exp2 domain with a reference max per head that is only raised when a block
 // exceeds it by more than 2^8 (then O is rescaled in TMEM after the previous P V completes),
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
-// Keys arrive by 16-byte cp.async from four loader warps (each row 1 KB, two 512-byte coalesced
-// halves per warp instruction), written straight into the swizzled layout.
-// The epilogue transposes each warp's output tile through shared memory into 128-byte row segments.
-// Roles: warps 0-3 softmax + epilogue, warps 4-7 load keys, warp 8 owns TMEM and issues MMAs
-// from an event loop (a P V never waits for the next block's keys).
+// TMEM is read and written with the 16-lane x2 access shape, so both halves of a warp work on the
+// 16 heads of its quarter (each thread one head, half of the columns).
+// Roles: warps 0-3 softmax + epilogue; warps 4-7 load keys (16-byte cp.async, each row 1 KB in
+// two 512-byte coalesced halves per warp instruction) and write each query's Q into their TMEM
+// quarter; warp 8 owns TMEM and issues MMAs from an event loop (a P V never waits for the next
+// block's keys); warp 9 plans: it builds the next query's entry list, block range and rope table
+// in a second slot and prefetches its Q into L2. Key blocks are counted over all of a CTA's
+// queries, so the loaders run into the next query while the current one finishes; the next
+// query's Q is written as soon as the last S of the current one has completed, and its first
+// P V waits only until the epilogue has read O out of TMEM.
 // Every wait is bounded (CSA_ERR_TIMEOUT on expiry).
 #include <algorithm>
 
@@ -46,28 +56,29 @@ namespace {
 constexpr int HH = 64, DD = 512, RR = 64;
 constexpr int KB = 64;                          // keys per block
 constexpr int NCH = DD / 64;                    // 64-element chunks per row
-constexpr int QCH = 9;                          // Q chunks: 7 un-rotated, rope(theta_cmp), rope(theta_tok)
-constexpr int QCHUNK = HH * 128;                // 8 KB
+constexpr int NSTAGE = 3;                       // key stages
 constexpr int KCHUNK = KB * 128;                // 8 KB
 constexpr int STAGE = NCH * KCHUNK;             // 64 KB
 constexpr int PBUF = HH * 128;                  // 8 KB
-constexpr int NUM_THREADS = 288;
+constexpr int NUM_THREADS = 320;
 constexpr int SM_THREADS = 128;
-constexpr int LOAD_WARP0 = 4;                   // warps 4..7 load keys
+constexpr int LOAD_WARP0 = 4;                   // warps 4..7 load keys and write Q
 constexpr int LOAD_THREADS = 128;
 constexpr int MMA_WARP = 8;
+constexpr int PLAN_WARP = 9;
+constexpr int PLAN_CONSUMERS = 4 + 1 + 4;       // loader warps, MMA thread, softmax warps
 constexpr float TAU = 8.f;
-constexpr uint32_t COL_RW = 256, COL_S = 320;
 constexpr uint32_t LANE16 = 16u << 16;
+constexpr uint32_t COL_S = 0, COL_RW = 128, COL_Q = 192;   // half 0
+constexpr uint32_t COL_OHI = 256, COL_OER = 448;          // half 1 (O_lo at column 0)
 constexpr uint32_t TMEM_COLS = 512;
 
-
-constexpr size_t OFF_Q = 0;
-constexpr size_t OFF_KV = OFF_Q + (size_t)QCH * QCHUNK;       // 72 KB
-constexpr size_t OFF_P = OFF_KV + 2 * (size_t)STAGE;          // 200 KB
-constexpr size_t OFF_ROPE = OFF_P + 2 * (size_t)PBUF;         // 216 KB: cos/sin [2 thetas][32 pairs][2]
-constexpr size_t OFF_BAR = OFF_ROPE + 2 * 32 * 2 * 4;
-constexpr size_t OFF_LIST = OFF_BAR + 256;
+constexpr size_t OFF_KV = 0;
+constexpr size_t OFF_P = OFF_KV + (size_t)NSTAGE * STAGE;     // 192 KB
+constexpr size_t OFF_ROPE = OFF_P + 2 * (size_t)PBUF;         // 208 KB: cos/sin [2 slots][2 thetas][32 pairs][2]
+constexpr size_t OFF_PLAN = OFF_ROPE + 2 * 2 * 32 * 2 * 4;
+constexpr size_t OFF_BAR = OFF_PLAN + 128;
+constexpr size_t OFF_LIST = OFF_BAR + 256;                    // entry lists [2 slots][k rounded up to 4]
 
 struct TcArgs {
     const uint16_t *q;        // [R, 64, 512] (R = S prefill rows or B decode sequences)
@@ -78,7 +89,7 @@ struct TcArgs {
     const uint16_t *c_rope;   //                   [B, T, 64] bf16
     const int32_t *idx;       // [R, k] or null (HCA: every visible entry)
     const float *sinks;       // [64]
-    float *o;                 // [R, 64, 512]
+    float *o;                 // [R, 64, 512] (or split partials [R*nsplit, 64, 512])
     float *part_ml;           // split partials: [R*nsplit, 64, 2] (log2-domain reference max, sum)
     int32_t *status;
     int64_t S, T, P;          // S: prefill rows; P: decode position
@@ -86,6 +97,20 @@ struct TcArgs {
     float scale_log2;         // softmax scale * log2(e)
     double log2_theta_tok, log2_theta_cmp;
 };
+
+// What the planner hands to the other roles for one query (double-buffered with its entry list
+// and rope table).
+struct Plan {
+    int64_t row;       // prefill query row, or decode sequence
+    int64_t win_row;   // kv_rot row holding the first window key
+    int32_t nw, ne;    // window keys, selected (valid) entries
+    int32_t nbw;       // window blocks of the whole key list
+    int32_t gb0, nb;   // this unit's key blocks: [gb0, gb0 + nb) of (window blocks, entry blocks)
+    int32_t split;
+    int32_t pad[2];
+};
+static_assert(sizeof(Plan) == 48, "plan layout");
+static_assert(2 * sizeof(Plan) <= 128, "plan slots");
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
@@ -98,197 +123,204 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Wait (at most 100 ms) for a phase regardless of the abort flag: used before exit so that no
+// copy or MMA is still writing this CTA's shared memory or TMEM.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > 100000000ull) return;
+}
+
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-        "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-        "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-        "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-        "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-        "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
 // byte offset of 16-byte unit `u` (0..7) of row `row` inside a 128-byte-swizzled [rows x 128 B] chunk
 __device__ __forceinline__ uint32_t sw128(int row, int u) { return (uint32_t)(row * 128 + ((u ^ (row & 7)) << 4)); }
+
+// Rotate the 16 bf16 pairs in w (interleaved RoPE pairs p0 .. p0+15) by the angles of table `cs`
+// ([pair][cos, sin]); result packed as bf16 pairs.
+__device__ __forceinline__ void rotate16(const uint32_t (&w)[16], const float *cs, int p0, uint32_t (&out)[16])
+{
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float x0 = bf_lo(w[i]), x1 = bf_hi(w[i]);
+        const float c = cs[(p0 + i) * 2], s = cs[(p0 + i) * 2 + 1];
+        out[i] = pack_bf2(x0 * c - x1 * s, x0 * s + x1 * c);
+    }
+}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    uint8_t *sQ = smem + OFF_Q;
     uint8_t *sKV = smem + OFF_KV;
     uint8_t *sP = smem + OFF_P;
-    float *rope_cs = reinterpret_cast<float *>(smem + OFF_ROPE);     // [theta: 0 tok, 1 cmp][pair][cos, sin]
+    float *rope_tab = reinterpret_cast<float *>(smem + OFF_ROPE);   // [slot][theta: 0 tok, 1 cmp][pair][cos, sin]
+    Plan *plans = reinterpret_cast<Plan *>(smem + OFF_PLAN);         // [slot]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *kv_full = bars + 0;     // [2] loader arrivals
-    uint64_t *kv_empty = bars + 2;    // [2] MMA commit
-    uint64_t *s_full = bars + 4;      // [2] MMA commit
-    uint64_t *p_ready = bars + 6;     // [2] 128 softmax arrivals
-    // P V completion: block b commits o_done[b & 1]. When the softmax of block b waits for P V of
-    // block b-1, every earlier completion of that barrier (block b-3) is already known to be done
-    // (it preceded S of block b), so a parity wait cannot mistake an older phase for the one wanted.
-    uint64_t *o_done = bars + 8;      // [2]
-    uint64_t *o_final = bars + 10;    // single use: every MMA of this CTA has completed
-    uint64_t *q_ready = bars + 11;    // 128 softmax arrivals
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 12);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 13);
-    int *nlist = reinterpret_cast<int *>(bars + 14);
-    uint64_t *q_tma = bars + 15;      // TMA of the 7 un-rotated Q chunks
-    int *elist = reinterpret_cast<int *>(smem + OFF_LIST);
+    uint64_t *kv_full = bars + 0;      // [stage] loader arrivals
+    uint64_t *kv_empty = bars + 3;     // [stage] MMA commit
+    uint64_t *s_full = bars + 6;       // [2] MMA commit
+    uint64_t *p_ready = bars + 8;      // [2] 128 softmax arrivals
+    // P V completion: block g (counted over all of this CTA's queries) commits o_done[g & 1]. When
+    // the softmax of block g waits for P V of block g-1, the previous completion of that barrier
+    // (block g-3) is already known to be done (it preceded S of block g), so a parity wait cannot
+    // mistake an older phase for the one wanted.
+    uint64_t *o_done = bars + 10;      // [2]
+    uint64_t *o_final = bars + 12;     // [query & 1] every MMA of the query has completed
+    uint64_t *o_free = bars + 14;      // 128 epilogue arrivals: O of the query has been read from TMEM
+    uint64_t *q_free = bars + 15;      // MMA commit after the last S of a query
+    uint64_t *q_ready = bars + 16;     // 128 loader arrivals: Q of the query is in TMEM
+    uint64_t *plan_ready = bars + 17;  // [slot] planner
+    uint64_t *plan_free = bars + 19;   // [slot] 4 loader warps + MMA + 4 softmax warps
+    uint64_t *drain = bars + 21;       // single use: every MMA issued has completed
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 22);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 23);
+    int *elist_all = reinterpret_cast<int *>(smem + OFF_LIST);    // [slot][kcap]
+    const int kcap = (max(a.k, 1) + 3) & ~3;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // prefill: one CTA per query row, longest key lists first; decode: nsplit CTAs per sequence
-    const int64_t row = a.decode ? (int64_t)(blockIdx.x / a.nsplit) : a.S - 1 - (int64_t)blockIdx.x;
-    const int split = a.decode ? (int)(blockIdx.x % a.nsplit) : 0;
     const bool partial = a.nsplit > 1;
-    const int64_t t = a.decode ? a.P : row;                   // position of the query
-    const int64_t vis = a.decode ? a.T : visible_entries(t, a.m, a.T);
-    const int64_t wpos0 = max((int64_t)0, t - a.W + 1);
-    const int nw = (int)(t - wpos0 + 1);
-    const uint16_t *win0 = a.decode ? a.kv_rot + (row * a.W + (a.W - nw)) * (int64_t)DD
-                                    : a.kv_rot + wpos0 * (int64_t)DD;   // first window row
-    const uint16_t *ent0 = a.decode && a.C != nullptr ? a.C + row * a.T * DD : a.C;
+    const int64_t units = a.S * a.nsplit;   // prefill: one query row each; decode: (sequence, split)
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NSTAGE; ++i) {
             mbar_init(&kv_full[i], LOAD_THREADS);   // one cp.async arrival per loader thread
             mbar_init(&kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
             mbar_init(&p_ready[i], SM_THREADS);
+            mbar_init(&o_done[i], 1);
+            mbar_init(&o_final[i], 1);
+            mbar_init(&plan_ready[i], 1);
+            mbar_init(&plan_free[i], PLAN_CONSUMERS);
         }
-        mbar_init(&o_done[0], 1);
-        mbar_init(&o_done[1], 1);
-        mbar_init(o_final, 1);
-        mbar_init(q_ready, SM_THREADS);
-        mbar_init(q_tma, 1);
+        mbar_init(o_free, SM_THREADS);
+        mbar_init(q_free, 1);
+        mbar_init(q_ready, LOAD_THREADS);
+        mbar_init(drain, 1);
         *abort = 0;
         fence_barrier_init();
-        mbar_arrive_expect_tx(q_tma, 7 * QCHUNK);
-        const uint64_t pol_q = policy_evict_first();     // q is read once
-        for (int dc = 0; dc < 7; ++dc) tma_load_2d_hint(sQ + dc * QCHUNK, &tm_q, q_tma, dc * 64, (int)(row * HH), pol_q);
     }
     if (warp == MMA_WARP) {
         tmem_alloc(tmem_ptr, TMEM_COLS);
         tmem_relinquish();
     }
-    if (threadIdx.x < 64) {   // rope table: angle t * theta^(-2p/64) for both thetas
-        const int p = threadIdx.x & 31, th = threadIdx.x >> 5;
-        float c, s;
-        rope_cos_sin((double)t, p, RR, th ? a.log2_theta_cmp : a.log2_theta_tok, &c, &s);
-        rope_cs[(th * 32 + p) * 2] = c;
-        rope_cs[(th * 32 + p) * 2 + 1] = s;
-    }
-    if (warp == LOAD_WARP0) { // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
-        if (a.idx != nullptr) {
-            const int32_t *ir = a.idx + row * (int64_t)a.k;
-            int vals[32];   // k <= 1024: all loads in flight at once
-#pragma unroll
-            for (int i = 0; i < 32; ++i) vals[i] = i * 32 + lane < a.k ? __ldg(ir + i * 32 + lane) : -1;
-            int cnt = 0;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int s = vals[i];
-                const bool ok = s >= 0 && (int64_t)s < vis;
-                if (s >= 0 && !ok) report(a.status, CSA_ERR_INVALID_ARG);
-                const unsigned mk = __ballot_sync(0xffffffffu, ok);
-                if (ok) elist[cnt + __popc(mk & ((1u << lane) - 1u))] = s;
-                cnt += __popc(mk);
-            }
-            if (lane == 0) *nlist = cnt;
-        } else if (lane == 0) {
-            *nlist = (int)vis;
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
-    const int ne = *nlist;
-    const int nbw = (nw + KB - 1) / KB, nbe = (ne + KB - 1) / KB, nb_all = nbw + nbe;
-    // this CTA's share of the key blocks (window blocks first, then entry blocks)
-    const int gb0 = (int)((int64_t)split * nb_all / a.nsplit);
-    const int nb = (int)((int64_t)(split + 1) * nb_all / a.nsplit) - gb0;
-    const bool has_win = gb0 < nbw && nb > 0, has_ent = gb0 + nb > nbw;
 
-    if (warp < 4) {
-        // =============== softmax + epilogue (warp w owns TMEM lane quarter w) ===============
-        const int tid = threadIdx.x;
-        // Q tile: 7 un-rotated chunks, rope chunk rotated with theta_cmp (7) and theta_tok (8)
-        uint4 qv[4];   // rope chunk: 64 heads x 8 units, 4 per thread, all loads in flight
+    if (warp == PLAN_WARP) {
+        // =============== planner: index list, block split and rope table of each query ===============
+        for (int64_t n = 0;; ++n) {
+            const int64_t u = blockIdx.x + n * gridDim.x;
+            if (u >= units) break;
+            const int s = (int)(n & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&plan_free[s], (uint32_t)((n >> 1) & 1) ^ 1u, abort, a.status)))
+                break;
+            // prefill: rows longest-first over the grid; decode: nsplit units per sequence
+            const int64_t row = a.decode ? u / a.nsplit : a.S - 1 - u;
+            const int split = a.decode ? (int)(u % a.nsplit) : 0;
+            if (lane == 0 && (!a.decode || split == 0))   // bring this query's Q into L2 ahead of its use
+                for (int dc = 0; dc < NCH; ++dc) tma_prefetch_2d(&tm_q, dc * 64, (int)(row * HH));
+            const int64_t t = a.decode ? a.P : row;                   // position of the query
+            const int64_t vis = a.decode ? a.T : visible_entries(t, a.m, a.T);
+            const int64_t wpos0 = max((int64_t)0, t - a.W + 1);
+            const int nw = (int)(t - wpos0 + 1);
+            int *elist = elist_all + s * kcap;
+            int ne;
+            if (a.idx != nullptr) {   // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
+                const int32_t *ir = a.idx + row * (int64_t)a.k;
+                int vals[32];   // k <= 1024: all loads in flight at once
 #pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-            const int i = tid + r4 * SM_THREADS, h = i >> 3, uu = i & 7;
-            qv[r4] = __ldg(reinterpret_cast<const uint4 *>(a.q + ((row * HH + h) * (int64_t)DD) + 448 + uu * 8));
-        }
+                for (int i = 0; i < 32; ++i) vals[i] = i * 32 + lane < a.k ? __ldg(ir + i * 32 + lane) : -1;
+                int cnt = 0;
 #pragma unroll
-        for (int r4 = 0; r4 < 4; ++r4) {
-            const int i = tid + r4 * SM_THREADS, h = i >> 3, uu = i & 7;
-            const uint4 v = qv[r4];
-            {
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-                uint32_t oc[4], ot[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int p = uu * 4 + e;
-                    const float x0 = bf_lo(w4[e]), x1 = bf_hi(w4[e]);
-                    const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
-                    const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
-                    oc[e] = pack_bf2(x0 * cc - x1 * sc, x0 * sc + x1 * cc);
-                    ot[e] = pack_bf2(x0 * ct - x1 * st, x0 * st + x1 * ct);
+                for (int i = 0; i < 32; ++i) {
+                    const int e = vals[i];
+                    const bool valid = e >= 0 && (int64_t)e < vis;
+                    if (e >= 0 && !valid) report(a.status, CSA_ERR_INVALID_ARG);
+                    const unsigned mk = __ballot_sync(0xffffffffu, valid);
+                    if (valid) elist[cnt + __popc(mk & ((1u << lane) - 1u))] = e;
+                    cnt += __popc(mk);
                 }
-                *reinterpret_cast<uint4 *>(sQ + 7 * QCHUNK + sw128(h, uu)) = make_uint4(oc[0], oc[1], oc[2], oc[3]);
-                *reinterpret_cast<uint4 *>(sQ + 8 * QCHUNK + sw128(h, uu)) = make_uint4(ot[0], ot[1], ot[2], ot[3]);
+                ne = cnt;
+            } else {
+                ne = (int)vis;
             }
+            {   // rope table: angle t * theta^(-2p/64) for both thetas
+                float c, sn;
+                rope_cos_sin((double)t, lane, RR, a.log2_theta_tok, &c, &sn);
+                rope_tab[s * 128 + lane * 2] = c;
+                rope_tab[s * 128 + lane * 2 + 1] = sn;
+                rope_cos_sin((double)t, lane, RR, a.log2_theta_cmp, &c, &sn);
+                rope_tab[s * 128 + (32 + lane) * 2] = c;
+                rope_tab[s * 128 + (32 + lane) * 2 + 1] = sn;
+            }
+            if (lane == 0) {
+                const int nbw = (nw + KB - 1) / KB, nb_all = nbw + (ne + KB - 1) / KB;
+                Plan p;
+                p.row = row;
+                p.win_row = a.decode ? row * a.W + (a.W - nw) : wpos0;
+                p.nw = nw;
+                p.ne = ne;
+                p.nbw = nbw;
+                // this unit's share of the key blocks (window blocks first, then the entry blocks)
+                p.gb0 = (int)((int64_t)split * nb_all / a.nsplit);
+                p.nb = (int)((int64_t)(split + 1) * nb_all / a.nsplit) - p.gb0;
+                p.split = split;
+                plans[s] = p;
+            }
+            __threadfence_block();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&plan_ready[s]);
         }
-        fence_async_smem();
-        mbar_arrive(q_ready);
-
-        const int h = warp * 16 + (lane & 15);
-        const int half = lane >> 4;
+    } else if (warp < 4) {
+        // =============== softmax + epilogue (warp w owns TMEM quarter w: heads 16w..16w+15) ===============
+        const int hl = lane & 15, hf = lane >> 4;   // head of this thread, which half of the columns
+        const int h = warp * 16 + hl;
+        const uint32_t tq0 = tmem + ((uint32_t)(warp * 32) << 16);   // half 0 of the quarter
+        const uint32_t tq1 = tq0 + LANE16;                            // half 1
         // the sink seeds the running max and sum; split partials leave it to the combine step
         const float zl = partial ? -INFINITY : a.sinks[h] * 1.4426950408889634f;
-        float m_ref = zl, l = (zl == -INFINITY) ? 0.f : 1.f;
-        const uint32_t tq = tmem + ((uint32_t)(warp * 32) << 16);
+        int g = 0;   // key blocks of this CTA's earlier queries
         bool ok = true;
-        for (int b = 0; b < nb && ok; ++b) {
-            const int buf = b & 1;
-            const int gb = gb0 + b;
-            const int nk = gb < nbw ? min(KB, nw - gb * KB) : min(KB, ne - (gb - nbw) * KB);
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (b >> 1) & 1, abort, a.status));
+        for (int64_t n = 0;; ++n) {
+            const int64_t u = blockIdx.x + n * gridDim.x;
+            if (u >= units) break;
+            const int s = (int)(n & 1);
+            ok = __all_sync(0xffffffffu, mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status));
             if (!ok) break;
-            tc_fence_after();
-            float s0[32], s1[32];
-            tmem_ld32(tq + COL_S, s0);
-            tmem_ld32(tq + COL_S + 32, s1);
-            tmem_wait_ld();
-            const bool active = half == buf;
-            float corr = 1.f;
-            bool need = false;
-            if (active) {
+            const Plan pl = plans[s];
+            const float *rope_cs = rope_tab + s * 128;
+            const int nb = pl.nb, gb0 = pl.gb0, nbw = pl.nbw;
+            const bool has_win = gb0 < nbw && nb > 0, has_ent = gb0 + nb > nbw;
+            float m_ref = zl, l = (zl == -INFINITY) ? 0.f : 1.f;
+            for (int b = 0; b < nb && ok; ++b) {
+                const int gg = g + b;
+                const int buf = gg & 1;
+                const int gb = gb0 + b;
+                const int nk = gb < nbw ? min(KB, pl.nw - gb * KB) : min(KB, pl.ne - (gb - nbw) * KB);
+                ok = __all_sync(0xffffffffu, mbar_wait(&s_full[buf], (uint32_t)((gg >> 1) & 1), abort, a.status));
+                if (!ok) break;
+                tc_fence_after();
+                float sv[32];   // logits of keys 32*hf .. 32*hf+31 for head h
+                tmem_ld_half32(tq0 + COL_S + (uint32_t)buf * 64, sv);
+                tmem_wait_ld();
                 float mb = -INFINITY;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    s0[j] = j < nk ? s0[j] * a.scale_log2 : -INFINITY;
-                    s1[j] = j + 32 < nk ? s1[j] * a.scale_log2 : -INFINITY;
-                    mb = fmaxf(mb, fmaxf(s0[j], s1[j]));
+                    sv[j] = hf * 32 + j < nk ? sv[j] * a.scale_log2 : -INFINITY;
+                    mb = fmaxf(mb, sv[j]);
                 }
+                mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 16));   // the partner thread holds the same head
+                float corr = 1.f;
+                bool need = false;
                 if (mb > m_ref + TAU) {
                     corr = exp2f(m_ref - mb);
                     m_ref = mb;
@@ -296,244 +328,313 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                     need = b > 0;
                 }
                 float sum = 0.f;
-                uint32_t pk[32];
+                uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 32; j += 2) {
-                    const uint32_t w0 = pack_bf2(exp2f(s0[j] - m_ref), exp2f(s0[j + 1] - m_ref));
-                    const uint32_t w1 = pack_bf2(exp2f(s1[j] - m_ref), exp2f(s1[j + 1] - m_ref));
-                    pk[j >> 1] = w0;
-                    pk[16 + (j >> 1)] = w1;
-                    sum += bf_lo(w0) + bf_hi(w0) + bf_lo(w1) + bf_hi(w1);
+                    const uint32_t w = pack_bf2(exp2f(sv[j] - m_ref), exp2f(sv[j + 1] - m_ref));
+                    pk[j >> 1] = w;
+                    sum += bf_lo(w) + bf_hi(w);
                 }
-                l += sum;
+                l += sum + __shfl_xor_sync(0xffffffffu, sum, 16);
                 uint8_t *prow = sP + buf * PBUF;
 #pragma unroll
-                for (int uu = 0; uu < 8; ++uu)
-                    *reinterpret_cast<uint4 *>(prow + sw128(h, uu)) =
+                for (int uu = 0; uu < 4; ++uu)
+                    *reinterpret_cast<uint4 *>(prow + sw128(h, hf * 4 + uu)) =
                         make_uint4(pk[uu * 4], pk[uu * 4 + 1], pk[uu * 4 + 2], pk[uu * 4 + 3]);
-            }
-            // keep both halves of the warp in step: the partner lane holds the same head
-            const float pm = __shfl_xor_sync(0xffffffffu, m_ref, 16);
-            const float pl = __shfl_xor_sync(0xffffffffu, l, 16);
-            const float pc = __shfl_xor_sync(0xffffffffu, corr, 16);
-            const int pn = __shfl_xor_sync(0xffffffffu, (int)need, 16);
-            if (!active) { m_ref = pm; l = pl; corr = pc; need = pn != 0; }
-            if (__any_sync(0xffffffffu, need)) {
-                // O must hold every earlier P V before it is rescaled
-                ok = __all_sync(0xffffffffu, mbar_wait(&o_done[(b - 1) & 1], ((b - 1) >> 1) & 1, abort, a.status));
-                tc_fence_after();
-                if (ok) {
-                    for (uint32_t c = 0; c < COL_S; c += 32) {
-                        float v[32];
-                        tmem_ld32(tq + c, v);
-                        tmem_wait_ld();
+                if (__any_sync(0xffffffffu, need)) {
+                    // O must hold every earlier P V of this query before it is rescaled
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(&o_done[(gg - 1) & 1], (uint32_t)(((gg - 1) >> 1) & 1), abort, a.status));
+                    tc_fence_after();
+                    if (ok) {
+#pragma unroll 1
+                        for (uint32_t c = 0; c <= DD; c += 64) {   // O (half 1) then O_rw (half 0)
+                            const uint32_t ta = c < DD ? tq1 + c : tq0 + COL_RW;
+                            float v[32];
+                            tmem_ld_half32(ta, v);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] *= corr;
-                        tmem_st32(tq + c, v);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&p_ready[buf]);
-        }
-        // ---------------- epilogue ----------------
-        if (ok && nb > 0) ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, abort, a.status));
-        if (ok && nb > 0) {
-            tc_fence_after();
-            const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
-            // Every MMA has completed, so the P buffers are idle: each warp transposes its 32 rows x 32
-            // columns (16 heads x two dim halves) through its own 4 KB slice and writes whole 128-byte
-            // row segments (8 lanes per segment) to the output.
-            uint8_t *wbuf = sP + warp * 4096;
-            float *obase = partial ? a.o + ((row * a.nsplit + split) * HH) * (int64_t)DD   // o = partial rows
-                                   : a.o + (row * HH) * (int64_t)DD;
-            for (int c = 0; c < 256; c += 32) {
-                float v[32], rw[32];
-                tmem_ld32(tq + c, v);
-                if (c >= 192) tmem_ld32(tq + COL_RW + (c - 192), rw);   // warp-uniform collective loads
-                tmem_wait_ld();
-                if (half == 1 && c >= 192) {
-                    // rope slice: entry branch (here) + window branch (O_rw), each rotated by -t
-#pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        const int p = (c - 192 + j) >> 1;
-                        const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
-                        const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
-                        float e0 = has_ent ? v[j] : 0.f, e1 = has_ent ? v[j + 1] : 0.f;
-                        float w0 = has_win ? rw[j] : 0.f, w1 = has_win ? rw[j + 1] : 0.f;
-                        v[j] = (e0 * cc + e1 * sc) + (w0 * ct + w1 * st);
-                        v[j + 1] = (-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct);
-                    }
-                }
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    *reinterpret_cast<float4 *>(wbuf + sw128(lane, u)) =
-                        make_float4(v[4 * u] * inv, v[4 * u + 1] * inv, v[4 * u + 2] * inv, v[4 * u + 3] * inv);
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int pr = i * 4 + (lane >> 3), u = lane & 7;   // row pr of this warp's tile
-                    const float4 x = *reinterpret_cast<const float4 *>(wbuf + sw128(pr, u));
-                    const int hh = warp * 16 + (pr & 15);
-                    __stcs(reinterpret_cast<float4 *>(obase + hh * (int64_t)DD + (pr >> 4) * 256 + c + u * 4), x);
-                }
-                __syncwarp();
-            }
-        } else if (nb == 0 && !partial) {
-            float *orow = a.o + ((row * HH + h) * (int64_t)DD) + half * 256;
-            for (int c = 0; c < 256; c += 4) *reinterpret_cast<float4 *>(orow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        if (partial && lane < 16) {   // reference max (log2 domain) and sum of this split; an empty split has l = 0
-            float *ml = a.part_ml + ((row * a.nsplit + split) * HH + h) * 2;
-            ml[0] = ok && nb > 0 ? m_ref : -INFINITY;
-            ml[1] = ok && nb > 0 ? l : 0.f;
-        }
-    } else if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
-        // =============== key loads: 16-byte cp.async into the swizzled stages ===============
-        const int lw = warp - LOAD_WARP0;        // rows 16*lw .. 16*lw+15 of each block
-        for (int b = 0; b < nb; ++b) {
-            const int st = b & 1, gb = gb0 + b;
-            if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], ((b >> 1) & 1) ^ 1, abort, a.status))) break;
-            const bool win = gb < nbw;
-            const int kbase = win ? gb * KB : (gb - nbw) * KB;
-            const int nk = win ? min(KB, nw - kbase) : min(KB, ne - kbase);
-            if (!win && a.C == nullptr) {
-                // FP8 entry cache: codes * per-entry scale on channels [0,448), bf16 rope on [448,512),
-                // converted to bf16 here and stored into the swizzled stage
-                uint8_t *stage = sKV + st * STAGE;
-#pragma unroll 2
-                for (int r = 0; r < 16; ++r) {
-                    const int key = lw * 16 + r;
-                    uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
-                    if (key < nk) {
-                        const int64_t e = row * a.T + (a.idx != nullptr ? elist[kbase + key] : kbase + key);
-                        if (lane < 28) {
-                            const float sc = __ldg(a.c8_scale + e);
-                            const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(a.c8 + e * 448) + lane);
-                            const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-                            uint32_t ow[8];
-#pragma unroll
-                            for (int q2 = 0; q2 < 8; ++q2) {
-                                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
-                                    (__nv_fp8x2_storage_t)((cw[q2 >> 1] >> ((q2 & 1) * 16)) & 0xffffu), __NV_E4M3);
-                                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
-                                ow[q2] = pack_bf2(f.x * sc, f.y * sc);
-                            }
-                            o0 = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                            o1 = make_uint4(ow[4], ow[5], ow[6], ow[7]);
-                        } else {
-                            const uint4 *rr = reinterpret_cast<const uint4 *>(a.c_rope + e * 64);
-                            o0 = __ldg(rr + 2 * (lane - 28));
-                            o1 = __ldg(rr + 2 * (lane - 28) + 1);
+                            for (int j = 0; j < 32; ++j) v[j] *= corr;
+                            tmem_st_half32(ta, v);
                         }
+                        tmem_wait_st();
                     }
-                    // lane < 28: dims [16*lane, 16*lane+16); lanes 28..31: rope dims 448 + 16*(lane-28)
-                    const int d0 = lane < 28 ? 16 * lane : 448 + 16 * (lane - 28);
-                    const int dc = d0 >> 6, u0 = (d0 & 63) >> 3;
-                    *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0)) = o0;
-                    *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0 + 1)) = o1;
                 }
                 fence_async_smem();
-                mbar_arrive(&kv_full[st]);
-                continue;
+                tc_fence_before();
+                mbar_arrive(&p_ready[buf]);
             }
-            const uint32_t sbase = smem_u32(sKV + st * STAGE);
-#pragma unroll 4
-            for (int r = 0; r < 16; ++r) {
-                const int key = lw * 16 + r;
-                const bool valid = key < nk;
-                const uint16_t *rowp = a.q;      // any mapped address for padding rows (zero-filled, 0 bytes read)
-                if (valid) {
-                    if (win) rowp = win0 + (int64_t)(kbase + key) * DD;
-                    else rowp = ent0 + (int64_t)(a.idx != nullptr ? elist[kbase + key] : kbase + key) * DD;
-                }
+            // ---------------- epilogue ----------------
+            if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[s], (uint32_t)((n >> 1) & 1), abort, a.status));
+            if (!ok) break;
+            tc_fence_after();
+            const int64_t orow = partial ? pl.row * a.nsplit + pl.split : pl.row;   // o holds partial rows
+            float *orp = a.o + (orow * HH + h) * (int64_t)DD;
+            if (nb > 0) {
+                const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
+#pragma unroll 1
+                for (int c = 0; c < 448; c += 64) {   // dims c + 32*hf .. +31
+                    float v[32];
+                    tmem_ld_half32(tq1 + (uint32_t)c, v);
+                    tmem_wait_ld();
+                    float4 *dst = reinterpret_cast<float4 *>(orp + c + hf * 32);
 #pragma unroll
-                for (int hlf = 0; hlf < 2; ++hlf) {
-                    const int u = lane + 32 * hlf;
-                    cp_async16(sbase + (u >> 3) * KCHUNK + sw128(key, u & 7), rowp + (valid ? u * 8 : 0), valid ? 16u : 0u);
+                    for (int i = 0; i < 8; ++i)
+                        __stcs(dst + i, make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv, v[4 * i + 3] * inv));
+                }
+                // rope dims 448..511: entry branch + window branch, each rotated back by -t with its theta
+                float e[32], w[32];
+                tmem_ld_half32(tq1 + COL_OER, e);
+                tmem_ld_half32(tq0 + COL_RW, w);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(o_free);   // O has been read: the next query's P V may overwrite it
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const int p = hf * 16 + (j >> 1);
+                    const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
+                    const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
+                    const float e0 = has_ent ? e[j] : 0.f, e1 = has_ent ? e[j + 1] : 0.f;
+                    const float w0 = has_win ? w[j] : 0.f, w1 = has_win ? w[j + 1] : 0.f;
+                    e[j] = ((e0 * cc + e1 * sc) + (w0 * ct + w1 * st)) * inv;
+                    e[j + 1] = ((-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct)) * inv;
+                }
+                float4 *dst = reinterpret_cast<float4 *>(orp + 448 + hf * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) __stcs(dst + i, make_float4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]));
+            } else {
+                tc_fence_before();
+                mbar_arrive(o_free);
+                if (!partial) {
+                    float4 *dst = reinterpret_cast<float4 *>(orp + hf * 256);
+                    for (int i = 0; i < 64; ++i) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            cp_async_arrive_noinc(&kv_full[st]);
+            if (partial && hf == 0) {   // reference max (log2 domain) and sum of this split; an empty split has l = 0
+                float *ml = a.part_ml + (orow * HH + h) * 2;
+                ml[0] = nb > 0 ? m_ref : -INFINITY;
+                ml[1] = nb > 0 ? l : 0.f;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&plan_free[s]);
+            g += nb;
+        }
+    } else if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
+        // ===== key loads (16-byte cp.async into the swizzled stages) and Q into TMEM quarter lw =====
+        const int lw = warp - LOAD_WARP0;        // key rows 16*lw .. 16*lw+15 of each block; heads 16*lw..
+        const int hl = lane & 15, hf = lane >> 4;
+        const uint32_t tqq = tmem + ((uint32_t)(lw * 32) << 16) + COL_Q;   // Q chunks, half 0 of quarter lw
+        int g = 0;
+        for (int64_t n = 0;; ++n) {
+            const int64_t u = blockIdx.x + n * gridDim.x;
+            if (u >= units) break;
+            const int s = (int)(n & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status))) break;
+            const Plan pl = plans[s];
+            const int *elist = elist_all + s * kcap;
+            const float *rope_cs = rope_tab + s * 128;
+            const uint16_t *win0 = a.kv_rot + pl.win_row * DD;
+            const uint16_t *ent0 = a.decode && a.C != nullptr ? a.C + pl.row * a.T * DD : a.C;
+            bool ok = true;
+            for (int b = 0; b <= pl.nb; ++b) {
+                if (b == min(1, pl.nb)) {
+                    // Q of this query into TMEM, once every S of the previous query has completed:
+                    // thread (hl, hf) writes head 16*lw+hl, dims 64c + 32hf .. +31 of each chunk c
+                    if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(q_free, (uint32_t)((n - 1) & 1), abort, a.status))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint4 *qsrc = reinterpret_cast<const uint4 *>(a.q + (pl.row * HH + lw * 16 + hl) * (int64_t)DD + hf * 32);
+#pragma unroll 2
+                    for (int c = 0; c < NCH; ++c) {
+                        uint4 x[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) x[i] = __ldg(qsrc + c * 8 + i);
+                        const uint32_t wq[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
+                                                 x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
+                        if (c < NCH - 1) {
+                            tmem_st_half16u(tqq + c * 32, wq);
+                        } else {   // rope dims: rotated with theta_cmp (chunk 7) and theta_tok (chunk 8)
+                            uint32_t r[16];
+                            rotate16(wq, rope_cs + 64, hf * 16, r);
+                            tmem_st_half16u(tqq + 7 * 32, r);
+                            rotate16(wq, rope_cs, hf * 16, r);
+                            tmem_st_half16u(tqq + 8 * 32, r);
+                        }
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(q_ready);
+                }
+                if (b == pl.nb) break;
+                const int gg = g + b;
+                const int st = gg % NSTAGE, gb = pl.gb0 + b;
+                if (!__all_sync(0xffffffffu, mbar_wait(&kv_empty[st], (uint32_t)((gg / NSTAGE) & 1) ^ 1u, abort, a.status))) {
+                    ok = false;
+                    break;
+                }
+                const bool win = gb < pl.nbw;
+                const int kbase = win ? gb * KB : (gb - pl.nbw) * KB;
+                const int nk = win ? min(KB, pl.nw - kbase) : min(KB, pl.ne - kbase);
+                if (!win && a.C == nullptr) {
+                    // FP8 entry cache: codes * per-entry scale on channels [0,448), bf16 rope on [448,512),
+                    // converted to bf16 here and stored into the swizzled stage
+                    uint8_t *stage = sKV + st * STAGE;
+#pragma unroll 2
+                    for (int r = 0; r < 16; ++r) {
+                        const int key = lw * 16 + r;
+                        uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
+                        if (key < nk) {
+                            const int64_t e = pl.row * a.T + (a.idx != nullptr ? elist[kbase + key] : kbase + key);
+                            if (lane < 28) {
+                                const float sc = __ldg(a.c8_scale + e);
+                                const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(a.c8 + e * 448) + lane);
+                                const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+                                uint32_t ow[8];
+#pragma unroll
+                                for (int q2 = 0; q2 < 8; ++q2) {
+                                    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
+                                        (__nv_fp8x2_storage_t)((cw[q2 >> 1] >> ((q2 & 1) * 16)) & 0xffffu), __NV_E4M3);
+                                    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
+                                    ow[q2] = pack_bf2(f.x * sc, f.y * sc);
+                                }
+                                o0 = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                                o1 = make_uint4(ow[4], ow[5], ow[6], ow[7]);
+                            } else {
+                                const uint4 *rr = reinterpret_cast<const uint4 *>(a.c_rope + e * 64);
+                                o0 = __ldg(rr + 2 * (lane - 28));
+                                o1 = __ldg(rr + 2 * (lane - 28) + 1);
+                            }
+                        }
+                        // lane < 28: dims [16*lane, 16*lane+16); lanes 28..31: rope dims 448 + 16*(lane-28)
+                        const int d0 = lane < 28 ? 16 * lane : 448 + 16 * (lane - 28);
+                        const int dc = d0 >> 6, u0 = (d0 & 63) >> 3;
+                        *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0)) = o0;
+                        *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0 + 1)) = o1;
+                    }
+                    fence_async_smem();
+                    mbar_arrive(&kv_full[st]);
+                    continue;
+                }
+                const uint32_t sbase = smem_u32(sKV + st * STAGE);
+#pragma unroll 4
+                for (int r = 0; r < 16; ++r) {
+                    const int key = lw * 16 + r;
+                    const bool valid = key < nk;
+                    const uint16_t *rowp = a.q;      // any mapped address for padding rows (zero-filled, 0 bytes read)
+                    if (valid) {
+                        if (win) rowp = win0 + (int64_t)(kbase + key) * DD;
+                        else rowp = ent0 + (int64_t)(a.idx != nullptr ? elist[kbase + key] : kbase + key) * DD;
+                    }
+#pragma unroll
+                    for (int hlf = 0; hlf < 2; ++hlf) {
+                        const int uo = lane + 32 * hlf;
+                        cp_async16(sbase + (uo >> 3) * KCHUNK + sw128(key, uo & 7), rowp + (valid ? uo * 8 : 0),
+                                   valid ? 16u : 0u);
+                    }
+                }
+                cp_async_arrive_noinc(&kv_full[st]);
+            }
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&plan_free[s]);
+            g += pl.nb;
         }
         cp_async_wait_all();   // never leave with copies in flight into this CTA's shared memory
     } else if (warp == MMA_WARP && lane == 0) {
-        // =============== MMA issuer: one thread, event loop ===============
+        // =============== MMA issuer: one thread, event loop per query ===============
         const uint32_t idS = idesc_bf16(64, 64);
         const uint32_t idPV256 = idesc_bf16(64, 256, true);
         const uint32_t idPV192 = idesc_bf16(64, 192, true);
         const uint32_t idPV64 = idesc_bf16(64, 64, true);
         // descriptors are formed once; a tile / k-step offset is added to the start-address field
-        const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
         const uint64_t dK = sdesc_sw128(smem_u32(sKV), 16, 1024);
         const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
         const uint64_t dV = sdesc_sw128(smem_u32(sKV), KCHUNK, 1024);
-        int nS = 0, nPV = 0;
-        bool ok = nb == 0 || (mbar_wait(q_ready, 0, abort, a.status) && mbar_wait(q_tma, 0, abort, a.status));
-        uint64_t t_progress = globaltimer();
-        uint32_t polls = 0;
-        while (ok && nPV < nb) {
-            bool progressed = false;
-            // S(nS) needs its keys and a free logits buffer (softmax of nS-2 finished, i.e. PV(nS-2) issued)
-            if (nS < nb && nS <= nPV + 1 && mbar_try_wait(&kv_full[nS & 1], (nS >> 1) & 1)) {
-                fence_async_smem();   // keys were written by cp.async (generic proxy); the MMA reads via the async proxy
-                tc_fence_after();
-                const int st = nS & 1;
-                const uint32_t d = tmem + COL_S + (uint32_t)st * LANE16;
-                const int rope_chunk = gb0 + nS < nbw ? 8 : 7;
-                for (int dc = 0; dc < NCH; ++dc) {
-                    const uint64_t qa = dQ + (((dc < 7 ? dc : rope_chunk) * QCHUNK) >> 4);
-                    const uint64_t kb = dK + ((st * STAGE + dc * KCHUNK) >> 4);
+        int g = 0;
+        for (int64_t n = 0;; ++n) {
+            const int64_t u = blockIdx.x + n * gridDim.x;
+            if (u >= units) break;
+            const int s = (int)(n & 1);
+            if (!mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status)) break;
+            const int nb = plans[s].nb, gb0 = plans[s].gb0, nbw = plans[s].nbw;
+            if (!mbar_wait(q_ready, (uint32_t)(n & 1), abort, a.status)) break;
+            tc_fence_after();
+            int nS = 0, nPV = 0;
+            bool ofree = n == 0;      // O of the previous query has been read out
+            bool ok = true;
+            uint64_t t_progress = globaltimer();
+            uint32_t polls = 0;
+            while (nPV < nb) {
+                bool progressed = false;
+                // S(nS) needs its keys and a free logits buffer (softmax of nS-2 finished, i.e. PV(nS-2) issued)
+                const int gs = g + nS;
+                if (nS < nb && nS <= nPV + 1 &&
+                    mbar_try_wait(&kv_full[gs % NSTAGE], (uint32_t)((gs / NSTAGE) & 1))) {
+                    fence_async_smem();   // keys were written by cp.async (generic proxy); the MMA reads via the async proxy
+                    tc_fence_after();
+                    const int st = gs % NSTAGE;
+                    const uint32_t d = tmem + COL_S + (uint32_t)(gs & 1) * 64;
+                    const int rope_chunk = gb0 + nS < nbw ? 8 : 7;
+                    for (int dc = 0; dc < NCH; ++dc) {
+                        const uint32_t qa = tmem + COL_Q + (uint32_t)(dc < 7 ? dc : rope_chunk) * 32;
+                        const uint64_t kb = dK + ((st * STAGE + dc * KCHUNK) >> 4);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) mma_bf16(d, qa + 2 * ks, kb + 2 * ks, idS, (dc | ks) != 0);
+                        for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(d, qa + ks * 8, kb + 2 * ks, idS, (dc | ks) != 0);
+                    }
+                    mma_commit(&s_full[gs & 1]);
+                    if (nS + 1 == nb) mma_commit(q_free);
+                    ++nS;
+                    progressed = true;
                 }
-                mma_commit(&s_full[st]);
-                ++nS;
-                progressed = true;
-            }
-            // PV(nPV) needs the softmax of block nPV
-            if (nPV < nS && mbar_try_wait(&p_ready[nPV & 1], (nPV >> 1) & 1)) {
-                tc_fence_after();
-                const int b = nPV, st = b & 1, gb = gb0 + b;
-                const bool win = gb < nbw;
-                const uint32_t drope = win ? tmem + LANE16 + COL_RW : tmem + LANE16 + 192;
-                // the first block of each branch handled by this CTA starts that branch's rope accumulator
-                const bool rope_first = win ? (b == 0) : (gb == max(nbw, gb0));
+                if (!ofree && nPV < nS) ofree = mbar_try_wait(o_free, (uint32_t)((n - 1) & 1));
+                // PV(nPV) needs the softmax of block nPV (and, for the first, O of the previous query read out)
+                const int gp = g + nPV;
+                if (ofree && nPV < nS && mbar_try_wait(&p_ready[gp & 1], (uint32_t)((gp >> 1) & 1))) {
+                    tc_fence_after();
+                    const int b = nPV, st = gp % NSTAGE, gb = gb0 + b;
+                    const bool win = gb < nbw;
+                    const uint32_t drope = win ? tmem + COL_RW : tmem + LANE16 + COL_OER;
+                    // the first block of each branch handled by this unit starts that branch's rope accumulator
+                    const bool rope_first = win ? (b == 0) : (gb == max(nbw, gb0));
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = dP + ((st * PBUF + ks * 32) >> 4);
-                    const uint64_t vb = dV + ((st * STAGE + ks * 2048) >> 4);
-                    mma_bf16(tmem, ad, vb, idPV256, b > 0 || ks > 0);                                  // dims 0..255
-                    mma_bf16(tmem + LANE16, ad, vb + ((4 * KCHUNK) >> 4), idPV192, b > 0 || ks > 0);   // 256..447
-                    mma_bf16(drope, ad, vb + ((7 * KCHUNK) >> 4), idPV64, !rope_first || ks > 0);     // 448..511
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = dP + (((gp & 1) * PBUF + ks * 32) >> 4);
+                        const uint64_t vb = dV + ((st * STAGE + ks * 2048) >> 4);
+                        mma_bf16(tmem + LANE16, ad, vb, idPV256, b > 0 || ks > 0);                                  // dims 0..255
+                        mma_bf16(tmem + LANE16 + COL_OHI, ad, vb + ((4 * KCHUNK) >> 4), idPV192, b > 0 || ks > 0);   // 256..447
+                        mma_bf16(drope, ad, vb + ((7 * KCHUNK) >> 4), idPV64, !rope_first || ks > 0);              // 448..511
+                    }
+                    mma_commit(&kv_empty[st]);
+                    mma_commit(&o_done[gp & 1]);
+                    if (b + 1 == nb) mma_commit(&o_final[s]);
+                    ++nPV;
+                    progressed = true;
                 }
-                mma_commit(&kv_empty[st]);
-                mma_commit(&o_done[b & 1]);
-                if (b + 1 == nb) mma_commit(o_final);
-                ++nPV;
-                progressed = true;
-            }
-            if (progressed) {
-                t_progress = globaltimer();
-            } else if ((++polls & 255u) == 0) {
-                if (*abort) { ok = false; break; }
-                if (globaltimer() - t_progress > 2000000000ull) {
-                    *abort = 1;
-                    report(a.status, CSA_ERR_TIMEOUT);
-                    ok = false;
+                if (progressed) {
+                    t_progress = globaltimer();
+                } else if ((++polls & 255u) == 0) {
+                    if (*abort) { ok = false; break; }
+                    if (globaltimer() - t_progress > 2000000000ull) {
+                        *abort = 1;
+                        report(a.status, CSA_ERR_TIMEOUT);
+                        ok = false;
+                        break;
+                    }
                 }
             }
+            if (!ok) break;
+            if (nb == 0) {   // nothing to compute: release Q and complete the query's phases
+                mma_commit(q_free);
+                mma_commit(&o_final[s]);
+            }
+            mbar_arrive(&plan_free[s]);
+            g += nb;
         }
-        // leave only when every issued MMA has completed
-        mbar_wait(q_tma, 0, abort, a.status, 100000000ull);
-        if (nPV == nb && nb > 0) {
-            mbar_wait(o_final, 0, abort, a.status, 100000000ull);
-        } else if (nS > 0 || nPV > 0) {
-            // stopped early: commit once more and wait for that (covers every MMA issued so far)
-            mma_commit(o_final);
-            mbar_wait(o_final, 0, abort, a.status, 100000000ull);
-        }
+        // leave only when every MMA and commit issued has completed
+        mma_commit(drain);
+        mbar_drain(drain, 0);
     }
     tc_fence_before();
     __syncthreads();
@@ -608,13 +709,19 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     a.scale_log2 = x.scale * 1.4426950408889634f;
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
-    const size_t smem = 1024 + OFF_LIST + sizeof(int) * (size_t)std::max(a.k, 1);
+    const size_t smem = 1024 + OFF_LIST + 2 * sizeof(int) * (size_t)((std::max(a.k, 1) + 3) & ~3);
     CUtensorMap tq;
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
     a.o = out_rows;   // final rows, or the split partials
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<(unsigned)(x.R * nsplit), NUM_THREADS, smem, stream>>>(tq, a);
+    // persistent: one CTA per SM walks the units (query rows, or sequence splits) with stride grid
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int64_t units = x.R * nsplit;
+    const unsigned grid = (unsigned)std::min<int64_t>(units, std::max(sms, 1));
+    attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, a);
     return cudaGetLastError();
 }
 
