@@ -372,36 +372,52 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             float *orp = a.o + (orow * HH + h) * (int64_t)DD;
             if (nb > 0) {
                 const float inv = partial ? 1.f : (l > 0.f ? 1.f / l : 0.f);
+                // Each 64-column piece goes through this warp's own rows of the two P buffers
+                // (32 rows of 128 B: row 16*hf + hl holds head 16w+hl, dims c + 32hf .. +31) and
+                // leaves as whole 128-byte row segments, 8 lanes per segment.
+                uint8_t *stage0 = sP + warp * 2048, *stage1 = sP + PBUF + warp * 2048;
+                uint8_t *mine = (hf ? stage1 : stage0) + hl * 128;
+                float *obase = a.o + (orow * HH + warp * 16) * (int64_t)DD;
 #pragma unroll 1
-                for (int c = 0; c < 448; c += 64) {   // dims c + 32*hf .. +31
+                for (int c = 0; c < DD; c += 64) {
                     float v[32];
-                    tmem_ld_half32(tq1 + (uint32_t)c, v);
-                    tmem_wait_ld();
-                    float4 *dst = reinterpret_cast<float4 *>(orp + c + hf * 32);
+                    if (c < COL_OER) {
+                        tmem_ld_half32(tq1 + (uint32_t)c, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        __stcs(dst + i, make_float4(v[4 * i] * inv, v[4 * i + 1] * inv, v[4 * i + 2] * inv, v[4 * i + 3] * inv));
+                        for (int j = 0; j < 32; ++j) v[j] *= inv;
+                    } else {
+                        // rope dims 448..511: entry branch + window branch, each rotated back by -t with its theta
+                        float w[32];
+                        tmem_ld_half32(tq1 + COL_OER, v);
+                        tmem_ld_half32(tq0 + COL_RW, w);
+                        tmem_wait_ld();
+                        tc_fence_before();
+                        mbar_arrive(o_free);   // O has been read: the next query's P V may overwrite it
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            const int p = hf * 16 + (j >> 1);
+                            const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
+                            const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
+                            const float e0 = has_ent ? v[j] : 0.f, e1 = has_ent ? v[j + 1] : 0.f;
+                            const float w0 = has_win ? w[j] : 0.f, w1 = has_win ? w[j + 1] : 0.f;
+                            v[j] = ((e0 * cc + e1 * sc) + (w0 * ct + w1 * st)) * inv;
+                            v[j + 1] = ((-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct)) * inv;
+                        }
+                    }
+#pragma unroll
+                    for (int uq = 0; uq < 8; ++uq)
+                        *reinterpret_cast<float4 *>(mine + ((uq ^ (hl & 7)) << 4)) =
+                            make_float4(v[4 * uq], v[4 * uq + 1], v[4 * uq + 2], v[4 * uq + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = i * 4 + (lane >> 3), uq = lane & 7;   // staged row rr
+                        const float4 x = *reinterpret_cast<const float4 *>((rr >= 16 ? stage1 : stage0) + sw128(rr & 15, uq));
+                        __stcs(reinterpret_cast<float4 *>(obase + (rr & 15) * (int64_t)DD + c + (rr >> 4) * 32 + uq * 4), x);
+                    }
+                    __syncwarp();
                 }
-                // rope dims 448..511: entry branch + window branch, each rotated back by -t with its theta
-                float e[32], w[32];
-                tmem_ld_half32(tq1 + COL_OER, e);
-                tmem_ld_half32(tq0 + COL_RW, w);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(o_free);   // O has been read: the next query's P V may overwrite it
-#pragma unroll
-                for (int j = 0; j < 32; j += 2) {
-                    const int p = hf * 16 + (j >> 1);
-                    const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
-                    const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
-                    const float e0 = has_ent ? e[j] : 0.f, e1 = has_ent ? e[j + 1] : 0.f;
-                    const float w0 = has_win ? w[j] : 0.f, w1 = has_win ? w[j + 1] : 0.f;
-                    e[j] = ((e0 * cc + e1 * sc) + (w0 * ct + w1 * st)) * inv;
-                    e[j + 1] = ((-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct)) * inv;
-                }
-                float4 *dst = reinterpret_cast<float4 *>(orp + 448 + hf * 32);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) __stcs(dst + i, make_float4(e[4 * i], e[4 * i + 1], e[4 * i + 2], e[4 * i + 3]));
             } else {
                 tc_fence_before();
                 mbar_arrive(o_free);
@@ -440,27 +456,39 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                 if (b == min(1, pl.nb)) {
                     // Q of this query into TMEM, once every S of the previous query has completed:
                     // thread (hl, hf) writes head 16*lw+hl, dims 64c + 32hf .. +31 of each chunk c
+                    const uint4 *qsrc = reinterpret_cast<const uint4 *>(a.q + (pl.row * HH + lw * 16 + hl) * (int64_t)DD + hf * 32);
+                    // chunks 0-3 are loaded before the wait, 4-7 (L2 hits after the planner's
+                    // prefetch) once the first half is in TMEM
+                    uint4 x[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] = __ldg(qsrc + (i >> 2) * 8 + (i & 3));
                     if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(q_free, (uint32_t)((n - 1) & 1), abort, a.status))) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint4 *qsrc = reinterpret_cast<const uint4 *>(a.q + (pl.row * HH + lw * 16 + hl) * (int64_t)DD + hf * 32);
-#pragma unroll 2
-                    for (int c = 0; c < NCH; ++c) {
-                        uint4 x[4];
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        if (half == 1) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) x[i] = __ldg(qsrc + c * 8 + i);
-                        const uint32_t wq[16] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w,
-                                                 x[2].x, x[2].y, x[2].z, x[2].w, x[3].x, x[3].y, x[3].z, x[3].w};
-                        if (c < NCH - 1) {
-                            tmem_st_half16u(tqq + c * 32, wq);
-                        } else {   // rope dims: rotated with theta_cmp (chunk 7) and theta_tok (chunk 8)
-                            uint32_t r[16];
-                            rotate16(wq, rope_cs + 64, hf * 16, r);
-                            tmem_st_half16u(tqq + 7 * 32, r);
-                            rotate16(wq, rope_cs, hf * 16, r);
-                            tmem_st_half16u(tqq + 8 * 32, r);
+                            for (int i = 0; i < 16; ++i) x[i] = __ldg(qsrc + 32 + (i >> 2) * 8 + (i & 3));
+                        }
+#pragma unroll
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int c = half * 4 + cc;
+                            const uint32_t wq[16] = {x[4 * cc].x,     x[4 * cc].y,     x[4 * cc].z,     x[4 * cc].w,
+                                                     x[4 * cc + 1].x, x[4 * cc + 1].y, x[4 * cc + 1].z, x[4 * cc + 1].w,
+                                                     x[4 * cc + 2].x, x[4 * cc + 2].y, x[4 * cc + 2].z, x[4 * cc + 2].w,
+                                                     x[4 * cc + 3].x, x[4 * cc + 3].y, x[4 * cc + 3].z, x[4 * cc + 3].w};
+                            if (c < NCH - 1) {
+                                tmem_st_half16u(tqq + c * 32, wq);
+                            } else {   // rope dims: rotated with theta_cmp (chunk 7) and theta_tok (chunk 8)
+                                uint32_t r[16];
+                                rotate16(wq, rope_cs + 64, hf * 16, r);
+                                tmem_st_half16u(tqq + 7 * 32, r);
+                                rotate16(wq, rope_cs, hf * 16, r);
+                                tmem_st_half16u(tqq + 8 * 32, r);
+                            }
                         }
                     }
                     tmem_wait_st();
