@@ -18,13 +18,15 @@
 //   TMEM (M=64 uses 16 lanes of each 32-lane quarter, "half 0" = lanes +0..15, "half 1" = +16..31):
 //     half 0: S_b   cols [0,64), [64,128)   double-buffered logits (on the lanes of Q, as the
 //                                  A-from-TMEM MMA requires)
-//             O_rw  cols [128,192) window-branch rope dims 448..511
-//             Q     cols [192,480) 9 chunks of 64 dims (32 columns, 2 bf16 each): 7 un-rotated,
-//                                  rope rotated with theta_cmp (chunk 7) and theta_tok (chunk 8)
-//     half 1: O     cols [0,448)   output dims 0..447, cols [448,512) entry-branch rope dims
-//   (accumulator column ranges start on multiples of 64)
-//   The rope slice of each branch accumulates separately so each can be rotated back by -t
-//   with its own theta in the epilogue.
+//             Q     cols [128,384) 8 chunks of 64 dims (32 columns, 2 bf16 each), the rope chunk
+//                                  rotated with theta_cmp
+//     half 1: O     cols [0,512)   output dims 0..511
+// The two branches rotate their rope slices with different thetas. Once a window block has
+// landed, the planner turns the rope slice of each window key by t * (f_cmp - f_tok) per pair
+// (f = theta^(-2p/64)): a window key then scores against the theta_cmp-rotated q exactly as it
+// did against the theta_tok-rotated one (rotations preserve dot products), and its value, rotated
+// back by -t * f_cmp at the end, comes out rotated by -t * f_tok as required. So one rope chunk
+// of q, one rope accumulator and one rotation back serve both branches.
 // Softmax runs in the exp2 domain with a reference max per head that is only raised when a block
 // exceeds it by more than 2^8 (then O is rescaled in TMEM after the previous P V completes),
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
@@ -69,14 +71,15 @@ constexpr int PLAN_WARP = 9;
 constexpr int PLAN_CONSUMERS = 4 + 1 + 4;       // loader warps, MMA thread, softmax warps
 constexpr float TAU = 8.f;
 constexpr uint32_t LANE16 = 16u << 16;
-constexpr uint32_t COL_S = 0, COL_RW = 128, COL_Q = 192;   // half 0
-constexpr uint32_t COL_OHI = 256, COL_OER = 448;          // half 1 (O_lo at column 0)
+constexpr uint32_t COL_S = 0, COL_Q = 128;   // half 0
+constexpr uint32_t COL_O2 = 256;             // half 1: O dims 256..511 (dims 0..255 at column 0)
+constexpr int ROPE_TAB = 3 * 32 * 2;         // floats per slot: [tok, cmp, cmp - tok][pair][cos, sin]
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr size_t OFF_KV = 0;
 constexpr size_t OFF_P = OFF_KV + (size_t)NSTAGE * STAGE;     // 192 KB
-constexpr size_t OFF_ROPE = OFF_P + 2 * (size_t)PBUF;         // 208 KB: cos/sin [2 slots][2 thetas][32 pairs][2]
-constexpr size_t OFF_PLAN = OFF_ROPE + 2 * 2 * 32 * 2 * 4;
+constexpr size_t OFF_ROPE = OFF_P + 2 * (size_t)PBUF;         // 208 KB: rope tables [2 slots][ROPE_TAB]
+constexpr size_t OFF_PLAN = OFF_ROPE + 2 * ROPE_TAB * 4;
 constexpr size_t OFF_BAR = OFF_PLAN + 128;
 constexpr size_t OFF_LIST = OFF_BAR + 256;                    // entry lists [2 slots][k rounded up to 4]
 
@@ -112,9 +115,20 @@ struct Plan {
 static_assert(sizeof(Plan) == 48, "plan layout");
 static_assert(2 * sizeof(Plan) <= 128, "plan slots");
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
+__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void *src, uint32_t src_bytes, uint64_t policy)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src), "r"(src_bytes),
+                 "l"(policy)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint4 ldg_hint(const uint4 *p, uint64_t policy)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p), "l"(policy));
+    return v;
 }
 
 // arrive on `bar` when this thread's earlier cp.async copies have landed (no pending-count increment)
@@ -158,10 +172,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t *sKV = smem + OFF_KV;
     uint8_t *sP = smem + OFF_P;
-    float *rope_tab = reinterpret_cast<float *>(smem + OFF_ROPE);   // [slot][theta: 0 tok, 1 cmp][pair][cos, sin]
+    float *rope_tab = reinterpret_cast<float *>(smem + OFF_ROPE);   // [slot][tok, cmp, cmp - tok][pair][cos, sin]
     Plan *plans = reinterpret_cast<Plan *>(smem + OFF_PLAN);         // [slot]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    uint64_t *kv_full = bars + 0;      // [stage] loader arrivals
+    // A stage's loads complete on kv_full (entry blocks) or kv_wfull (window blocks): each barrier
+    // then counts the uses of one kind in order, so every waiter waits exactly one phase ahead.
+    uint64_t *kv_full = bars + 0;      // [stage] loader arrivals, entry blocks
     uint64_t *kv_empty = bars + 3;     // [stage] MMA commit
     uint64_t *s_full = bars + 6;       // [2] MMA commit
     uint64_t *p_ready = bars + 8;      // [2] 128 softmax arrivals
@@ -177,8 +193,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
     uint64_t *plan_ready = bars + 17;  // [slot] planner
     uint64_t *plan_free = bars + 19;   // [slot] 4 loader warps + MMA + 4 softmax warps
     uint64_t *drain = bars + 21;       // single use: every MMA issued has completed
-    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 22);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 23);
+    uint64_t *kv_rdy = bars + 22;      // [stage] planner: a window block's rope slice has been turned
+    uint64_t *kv_wfull = bars + 25;    // [stage] loader arrivals, window blocks
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 28);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 29);
     int *elist_all = reinterpret_cast<int *>(smem + OFF_LIST);    // [slot][kcap]
     const int kcap = (max(a.k, 1) + 3) & ~3;
 
@@ -190,6 +208,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
         for (int i = 0; i < NSTAGE; ++i) {
             mbar_init(&kv_full[i], LOAD_THREADS);   // one cp.async arrival per loader thread
             mbar_init(&kv_empty[i], 1);
+            mbar_init(&kv_rdy[i], 1);
+            mbar_init(&kv_wfull[i], LOAD_THREADS);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
@@ -216,7 +236,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
     const uint32_t tmem = *tmem_ptr;
 
     if (warp == PLAN_WARP) {
-        // =============== planner: index list, block split and rope table of each query ===============
+        // ====== planner: index list, block split and rope tables of each query; window rope turn ======
+        int g = 0;           // key blocks of this CTA's earlier queries
+        uint32_t wpar = 0;   // per stage: parity of the next kv_wfull completion
         for (int64_t n = 0;; ++n) {
             const int64_t u = blockIdx.x + n * gridDim.x;
             if (u >= units) break;
@@ -253,14 +275,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             } else {
                 ne = (int)vis;
             }
-            {   // rope table: angle t * theta^(-2p/64) for both thetas
+            {   // rope tables: angle t * f_p (f_p = theta^(-2p/64)) for both thetas, and their difference
+                float *rt = rope_tab + s * ROPE_TAB;
                 float c, sn;
                 rope_cos_sin((double)t, lane, RR, a.log2_theta_tok, &c, &sn);
-                rope_tab[s * 128 + lane * 2] = c;
-                rope_tab[s * 128 + lane * 2 + 1] = sn;
+                rt[lane * 2] = c;
+                rt[lane * 2 + 1] = sn;
                 rope_cos_sin((double)t, lane, RR, a.log2_theta_cmp, &c, &sn);
-                rope_tab[s * 128 + (32 + lane) * 2] = c;
-                rope_tab[s * 128 + (32 + lane) * 2 + 1] = sn;
+                rt[64 + lane * 2] = c;
+                rt[64 + lane * 2 + 1] = sn;
+                const double e = -(2.0 * lane / (double)RR);
+                const double dang = (double)t * (exp2(e * a.log2_theta_cmp) - exp2(e * a.log2_theta_tok));
+                double sd, cd;
+                sincos(dang, &sd, &cd);
+                rt[128 + lane * 2] = (float)cd;
+                rt[128 + lane * 2 + 1] = (float)sd;
             }
             if (lane == 0) {
                 const int nbw = (nw + KB - 1) / KB, nb_all = nbw + (ne + KB - 1) / KB;
@@ -279,6 +308,42 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             __threadfence_block();
             __syncwarp();
             if (lane == 0) mbar_arrive(&plan_ready[s]);
+
+            // Turn the rope slice of this unit's window keys (see the header) once each window
+            // block has landed; the MMA waits for kv_rdy on window blocks.
+            const Plan pl = plans[s];
+            const float *dt = rope_tab + s * ROPE_TAB + 128;
+            bool ok = true;
+            for (int b = 0; b < pl.nb && pl.gb0 + b < pl.nbw; ++b) {
+                const int gg = g + b, st = gg % NSTAGE;
+                if (!__all_sync(0xffffffffu, mbar_wait(&kv_wfull[st], (wpar >> st) & 1u, abort, a.status))) {
+                    ok = false;
+                    break;
+                }
+                wpar ^= 1u << st;
+                uint8_t *rope_rows = sKV + st * STAGE + (NCH - 1) * KCHUNK;   // dims 448..511 of each key
+#pragma unroll 4
+                for (int i = lane; i < KB * 8; i += 32) {
+                    const int key = i >> 3, uu = i & 7;   // 16-byte unit uu: pairs 4uu .. 4uu+3
+                    uint4 *ptr = reinterpret_cast<uint4 *>(rope_rows + sw128(key, uu));
+                    const uint4 v = *ptr;
+                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int pp = uu * 4 + e;
+                        const float x0 = bf_lo(w4[e]), x1 = bf_hi(w4[e]);
+                        const float c = dt[pp * 2], sn = dt[pp * 2 + 1];
+                        o4[e] = pack_bf2(x0 * c - x1 * sn, x0 * sn + x1 * c);
+                    }
+                    *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&kv_rdy[st]);
+            }
+            if (!ok) break;
+            g += pl.nb;
         }
     } else if (warp < 4) {
         // =============== softmax + epilogue (warp w owns TMEM quarter w: heads 16w..16w+15) ===============
@@ -297,9 +362,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             ok = __all_sync(0xffffffffu, mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status));
             if (!ok) break;
             const Plan pl = plans[s];
-            const float *rope_cs = rope_tab + s * 128;
+            const float *rope_cmp = rope_tab + s * ROPE_TAB + 64;
             const int nb = pl.nb, gb0 = pl.gb0, nbw = pl.nbw;
-            const bool has_win = gb0 < nbw && nb > 0, has_ent = gb0 + nb > nbw;
             float m_ref = zl, l = (zl == -INFINITY) ? 0.f : 1.f;
             for (int b = 0; b < nb && ok; ++b) {
                 const int gg = g + b;
@@ -348,8 +412,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                     tc_fence_after();
                     if (ok) {
 #pragma unroll 1
-                        for (uint32_t c = 0; c <= DD; c += 64) {   // O (half 1) then O_rw (half 0)
-                            const uint32_t ta = c < DD ? tq1 + c : tq0 + COL_RW;
+                        for (uint32_t c = 0; c < DD; c += 64) {   // O (half 1)
+                            const uint32_t ta = tq1 + c;
                             float v[32];
                             tmem_ld_half32(ta, v);
                             tmem_wait_ld();
@@ -381,30 +445,23 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
 #pragma unroll 1
                 for (int c = 0; c < DD; c += 64) {
                     float v[32];
-                    if (c < COL_OER) {
-                        tmem_ld_half32(tq1 + (uint32_t)c, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) v[j] *= inv;
-                    } else {
-                        // rope dims 448..511: entry branch + window branch, each rotated back by -t with its theta
-                        float w[32];
-                        tmem_ld_half32(tq1 + COL_OER, v);
-                        tmem_ld_half32(tq0 + COL_RW, w);
-                        tmem_wait_ld();
+                    tmem_ld_half32(tq1 + (uint32_t)c, v);
+                    tmem_wait_ld();
+                    if (c == DD - 64) {
                         tc_fence_before();
                         mbar_arrive(o_free);   // O has been read: the next query's P V may overwrite it
+                        // rope dims 448..511: rotated back by -t * f_cmp (window keys were turned to match)
 #pragma unroll
                         for (int j = 0; j < 32; j += 2) {
                             const int p = hf * 16 + (j >> 1);
-                            const float ct = rope_cs[p * 2], st = rope_cs[p * 2 + 1];
-                            const float cc = rope_cs[(32 + p) * 2], sc = rope_cs[(32 + p) * 2 + 1];
-                            const float e0 = has_ent ? v[j] : 0.f, e1 = has_ent ? v[j + 1] : 0.f;
-                            const float w0 = has_win ? w[j] : 0.f, w1 = has_win ? w[j + 1] : 0.f;
-                            v[j] = ((e0 * cc + e1 * sc) + (w0 * ct + w1 * st)) * inv;
-                            v[j + 1] = ((-e0 * sc + e1 * cc) + (-w0 * st + w1 * ct)) * inv;
+                            const float cc = rope_cmp[p * 2], sc = rope_cmp[p * 2 + 1];
+                            const float e0 = v[j], e1 = v[j + 1];
+                            v[j] = e0 * cc + e1 * sc;
+                            v[j + 1] = -e0 * sc + e1 * cc;
                         }
                     }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= inv;
 #pragma unroll
                     for (int uq = 0; uq < 8; ++uq)
                         *reinterpret_cast<float4 *>(mine + ((uq ^ (hl & 7)) << 4)) =
@@ -440,6 +497,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
         const int lw = warp - LOAD_WARP0;        // key rows 16*lw .. 16*lw+15 of each block; heads 16*lw..
         const int hl = lane & 15, hf = lane >> 4;
         const uint32_t tqq = tmem + ((uint32_t)(lw * 32) << 16) + COL_Q;   // Q chunks, half 0 of quarter lw
+        // L2 policies: q is read once; prefill entries are shared by many queries (kept), decode
+        // caches are read once per step; prefill window rows serve ~W consecutive queries (default)
+        const uint64_t pol_once = policy_evict_first();
+        const uint64_t pol_ent = a.decode ? pol_once : policy_evict_last();
+        const uint64_t pol_win = a.decode ? pol_once : policy_evict_normal();
         int g = 0;
         for (int64_t n = 0;; ++n) {
             const int64_t u = blockIdx.x + n * gridDim.x;
@@ -448,7 +510,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             if (!__all_sync(0xffffffffu, mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status))) break;
             const Plan pl = plans[s];
             const int *elist = elist_all + s * kcap;
-            const float *rope_cs = rope_tab + s * 128;
+            const float *rope_cs = rope_tab + s * ROPE_TAB;
             const uint16_t *win0 = a.kv_rot + pl.win_row * DD;
             const uint16_t *ent0 = a.decode && a.C != nullptr ? a.C + pl.row * a.T * DD : a.C;
             bool ok = true;
@@ -461,7 +523,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                     // prefetch) once the first half is in TMEM
                     uint4 x[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) x[i] = __ldg(qsrc + (i >> 2) * 8 + (i & 3));
+                    for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + (i >> 2) * 8 + (i & 3), pol_once);
                     if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(q_free, (uint32_t)((n - 1) & 1), abort, a.status))) {
                         ok = false;
                         break;
@@ -471,7 +533,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                     for (int half = 0; half < 2; ++half) {
                         if (half == 1) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) x[i] = __ldg(qsrc + 32 + (i >> 2) * 8 + (i & 3));
+                            for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + 32 + (i >> 2) * 8 + (i & 3), pol_once);
                         }
 #pragma unroll
                         for (int cc = 0; cc < 4; ++cc) {
@@ -482,12 +544,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                                                      x[4 * cc + 3].x, x[4 * cc + 3].y, x[4 * cc + 3].z, x[4 * cc + 3].w};
                             if (c < NCH - 1) {
                                 tmem_st_half16u(tqq + c * 32, wq);
-                            } else {   // rope dims: rotated with theta_cmp (chunk 7) and theta_tok (chunk 8)
+                            } else {   // rope dims: rotated with theta_cmp
                                 uint32_t r[16];
                                 rotate16(wq, rope_cs + 64, hf * 16, r);
                                 tmem_st_half16u(tqq + 7 * 32, r);
-                                rotate16(wq, rope_cs, hf * 16, r);
-                                tmem_st_half16u(tqq + 8 * 32, r);
                             }
                         }
                     }
@@ -545,24 +605,28 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                     mbar_arrive(&kv_full[st]);
                     continue;
                 }
-                const uint32_t sbase = smem_u32(sKV + st * STAGE);
-#pragma unroll 4
+                // lane j < 16 resolves the source row of key 16*lw + j once; the issue loop below
+                // takes it by shuffle, so no copy waits on a shared-memory lookup
+                const uint16_t *base = win ? win0 : ent0;
+                int my_row = -1;
+                if (lane < 16 && lw * 16 + lane < nk) {
+                    const int kk = kbase + lw * 16 + lane;
+                    my_row = (win || a.idx == nullptr) ? kk : elist[kk];
+                }
+                const uint64_t pol = win ? pol_win : pol_ent;
+                const uint32_t sdst = smem_u32(sKV + st * STAGE) + (lane >> 3) * KCHUNK;   // unit lane (chunk lane/8)
+#pragma unroll
                 for (int r = 0; r < 16; ++r) {
                     const int key = lw * 16 + r;
-                    const bool valid = key < nk;
-                    const uint16_t *rowp = a.q;      // any mapped address for padding rows (zero-filled, 0 bytes read)
-                    if (valid) {
-                        if (win) rowp = win0 + (int64_t)(kbase + key) * DD;
-                        else rowp = ent0 + (int64_t)(a.idx != nullptr ? elist[kbase + key] : kbase + key) * DD;
-                    }
-#pragma unroll
-                    for (int hlf = 0; hlf < 2; ++hlf) {
-                        const int uo = lane + 32 * hlf;
-                        cp_async16(sbase + (uo >> 3) * KCHUNK + sw128(key, uo & 7), rowp + (valid ? uo * 8 : 0),
-                                   valid ? 16u : 0u);
-                    }
+                    const int row = __shfl_sync(0xffffffffu, my_row, r);
+                    const bool valid = row >= 0;
+                    // padding rows: zero-filled, 0 bytes read from any mapped address
+                    const uint16_t *rowp = valid ? base + (int64_t)row * DD + lane * 8 : a.q;
+                    const uint32_t d = sdst + sw128(key, lane & 7);
+                    cp_async16_hint(d, rowp, valid ? 16u : 0u, pol);                        // dims 8*lane ..
+                    cp_async16_hint(d + 4 * KCHUNK, valid ? rowp + 256 : a.q, valid ? 16u : 0u, pol);   // 256 + 8*lane ..
                 }
-                cp_async_arrive_noinc(&kv_full[st]);
+                cp_async_arrive_noinc(win ? &kv_wfull[st] : &kv_full[st]);
             }
             if (!ok) break;
             __syncwarp();
@@ -573,14 +637,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
     } else if (warp == MMA_WARP && lane == 0) {
         // =============== MMA issuer: one thread, event loop per query ===============
         const uint32_t idS = idesc_bf16(64, 64);
-        const uint32_t idPV256 = idesc_bf16(64, 256, true);
-        const uint32_t idPV192 = idesc_bf16(64, 192, true);
-        const uint32_t idPV64 = idesc_bf16(64, 64, true);
+        const uint32_t idPV = idesc_bf16(64, 256, true);
         // descriptors are formed once; a tile / k-step offset is added to the start-address field
         const uint64_t dK = sdesc_sw128(smem_u32(sKV), 16, 1024);
         const uint64_t dP = sdesc_sw128(smem_u32(sP), 16, 1024);
         const uint64_t dV = sdesc_sw128(smem_u32(sKV), KCHUNK, 1024);
         int g = 0;
+        uint32_t wpar = 0;   // per stage: parity of the next kv_rdy completion (window blocks)
+        uint32_t epar = 0;   // per stage: parity of the next kv_full completion (entry blocks)
         for (int64_t n = 0;; ++n) {
             const int64_t u = blockIdx.x + n * gridDim.x;
             if (u >= units) break;
@@ -598,16 +662,19 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                 bool progressed = false;
                 // S(nS) needs its keys and a free logits buffer (softmax of nS-2 finished, i.e. PV(nS-2) issued)
                 const int gs = g + nS;
+                const int sst = gs % NSTAGE;
+                const bool swin = gb0 + nS < nbw;   // window block: wait until its rope slice is turned
                 if (nS < nb && nS <= nPV + 1 &&
-                    mbar_try_wait(&kv_full[gs % NSTAGE], (uint32_t)((gs / NSTAGE) & 1))) {
+                    (swin ? mbar_try_wait(&kv_rdy[sst], (wpar >> sst) & 1u)
+                          : mbar_try_wait(&kv_full[sst], (epar >> sst) & 1u))) {
+                    if (swin) wpar ^= 1u << sst;
+                    else epar ^= 1u << sst;
                     fence_async_smem();   // keys were written by cp.async (generic proxy); the MMA reads via the async proxy
                     tc_fence_after();
-                    const int st = gs % NSTAGE;
                     const uint32_t d = tmem + COL_S + (uint32_t)(gs & 1) * 64;
-                    const int rope_chunk = gb0 + nS < nbw ? 8 : 7;
                     for (int dc = 0; dc < NCH; ++dc) {
-                        const uint32_t qa = tmem + COL_Q + (uint32_t)(dc < 7 ? dc : rope_chunk) * 32;
-                        const uint64_t kb = dK + ((st * STAGE + dc * KCHUNK) >> 4);
+                        const uint32_t qa = tmem + COL_Q + (uint32_t)dc * 32;
+                        const uint64_t kb = dK + ((sst * STAGE + dc * KCHUNK) >> 4);
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(d, qa + ks * 8, kb + 2 * ks, idS, (dc | ks) != 0);
                     }
@@ -621,18 +688,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                 const int gp = g + nPV;
                 if (ofree && nPV < nS && mbar_try_wait(&p_ready[gp & 1], (uint32_t)((gp >> 1) & 1))) {
                     tc_fence_after();
-                    const int b = nPV, st = gp % NSTAGE, gb = gb0 + b;
-                    const bool win = gb < nbw;
-                    const uint32_t drope = win ? tmem + COL_RW : tmem + LANE16 + COL_OER;
-                    // the first block of each branch handled by this unit starts that branch's rope accumulator
-                    const bool rope_first = win ? (b == 0) : (gb == max(nbw, gb0));
+                    const int b = nPV, st = gp % NSTAGE;
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
                         const uint64_t ad = dP + (((gp & 1) * PBUF + ks * 32) >> 4);
                         const uint64_t vb = dV + ((st * STAGE + ks * 2048) >> 4);
-                        mma_bf16(tmem + LANE16, ad, vb, idPV256, b > 0 || ks > 0);                                  // dims 0..255
-                        mma_bf16(tmem + LANE16 + COL_OHI, ad, vb + ((4 * KCHUNK) >> 4), idPV192, b > 0 || ks > 0);   // 256..447
-                        mma_bf16(drope, ad, vb + ((7 * KCHUNK) >> 4), idPV64, !rope_first || ks > 0);              // 448..511
+                        mma_bf16(tmem + LANE16, ad, vb, idPV, b > 0 || ks > 0);                                 // dims 0..255
+                        mma_bf16(tmem + LANE16 + COL_O2, ad, vb + ((4 * KCHUNK) >> 4), idPV, b > 0 || ks > 0);   // 256..511
                     }
                     mma_commit(&kv_empty[st]);
                     mma_commit(&o_done[gp & 1]);
