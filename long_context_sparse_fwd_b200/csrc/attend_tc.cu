@@ -68,7 +68,7 @@ constexpr int LOAD_WARP0 = 4;                   // warps 4..7 load keys and writ
 constexpr int LOAD_THREADS = 128;
 constexpr int MMA_WARP = 8;
 constexpr int PLAN_WARP = 9;
-constexpr int PLAN_CONSUMERS = 4 + 1 + 4;       // loader warps, MMA thread, softmax warps
+constexpr int PLAN_CONSUMERS = 4 + 1 + 4;       // loader warps, MMA warp (one arrival), softmax warps
 constexpr float TAU = 8.f;
 constexpr uint32_t LANE16 = 16u << 16;
 constexpr uint32_t COL_S = 0, COL_Q = 128;   // half 0
@@ -634,8 +634,11 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             g += pl.nb;
         }
         cp_async_wait_all();   // never leave with copies in flight into this CTA's shared memory
-    } else if (warp == MMA_WARP && lane == 0) {
-        // =============== MMA issuer: one thread, event loop per query ===============
+    } else if (warp == MMA_WARP) {
+        // =============== MMA issuer: event loop per query ===============
+        // The whole warp runs the loop (every decision is made warp-uniform with a vote) and one
+        // elected lane issues the MMAs and commits: with warp-uniform control flow the descriptors
+        // stay in uniform registers and each tcgen05.mma issues without per-instruction overhead.
         const uint32_t idS = idesc_bf16(64, 64);
         const uint32_t idPV = idesc_bf16(64, 256, true);
         // descriptors are formed once; a tile / k-step offset is added to the start-address field
@@ -649,14 +652,14 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             const int64_t u = blockIdx.x + n * gridDim.x;
             if (u >= units) break;
             const int s = (int)(n & 1);
-            if (!mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&plan_ready[s], (uint32_t)((n >> 1) & 1), abort, a.status))) break;
             const int nb = plans[s].nb, gb0 = plans[s].gb0, nbw = plans[s].nbw;
-            if (!mbar_wait(q_ready, (uint32_t)(n & 1), abort, a.status)) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(q_ready, (uint32_t)(n & 1), abort, a.status))) break;
             tc_fence_after();
             int nS = 0, nPV = 0;
             bool ofree = n == 0;      // O of the previous query has been read out
             bool ok = true;
-            uint64_t t_progress = globaltimer();
+            uint64_t t_progress = __shfl_sync(0xffffffffu, globaltimer(), 0);
             uint32_t polls = 0;
             while (nPV < nb) {
                 bool progressed = false;
@@ -665,65 +668,78 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                 const int sst = gs % NSTAGE;
                 const bool swin = gb0 + nS < nbw;   // window block: wait until its rope slice is turned
                 if (nS < nb && nS <= nPV + 1 &&
-                    (swin ? mbar_try_wait(&kv_rdy[sst], (wpar >> sst) & 1u)
-                          : mbar_try_wait(&kv_full[sst], (epar >> sst) & 1u))) {
+                    __all_sync(0xffffffffu, swin ? mbar_try_wait(&kv_rdy[sst], (wpar >> sst) & 1u)
+                                                 : mbar_try_wait(&kv_full[sst], (epar >> sst) & 1u))) {
                     if (swin) wpar ^= 1u << sst;
                     else epar ^= 1u << sst;
                     fence_async_smem();   // keys were written by cp.async (generic proxy); the MMA reads via the async proxy
                     tc_fence_after();
-                    const uint32_t d = tmem + COL_S + (uint32_t)(gs & 1) * 64;
-                    for (int dc = 0; dc < NCH; ++dc) {
-                        const uint32_t qa = tmem + COL_Q + (uint32_t)dc * 32;
-                        const uint64_t kb = dK + ((sst * STAGE + dc * KCHUNK) >> 4);
+                    if (elect_one()) {
+                        const uint32_t d = tmem + COL_S + (uint32_t)(gs & 1) * 64;
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(d, qa + ks * 8, kb + 2 * ks, idS, (dc | ks) != 0);
+                        for (int dc = 0; dc < NCH; ++dc) {
+                            const uint32_t qa = tmem + COL_Q + (uint32_t)dc * 32;
+                            const uint64_t kb = dK + ((sst * STAGE + dc * KCHUNK) >> 4);
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(d, qa + ks * 8, kb + 2 * ks, idS, (dc | ks) != 0);
+                        }
+                        mma_commit(&s_full[gs & 1]);
+                        if (nS + 1 == nb) mma_commit(q_free);
                     }
-                    mma_commit(&s_full[gs & 1]);
-                    if (nS + 1 == nb) mma_commit(q_free);
+                    __syncwarp();
                     ++nS;
                     progressed = true;
                 }
-                if (!ofree && nPV < nS) ofree = mbar_try_wait(o_free, (uint32_t)((n - 1) & 1));
+                if (!ofree && nPV < nS) ofree = __all_sync(0xffffffffu, mbar_try_wait(o_free, (uint32_t)((n - 1) & 1)));
                 // PV(nPV) needs the softmax of block nPV (and, for the first, O of the previous query read out)
                 const int gp = g + nPV;
-                if (ofree && nPV < nS && mbar_try_wait(&p_ready[gp & 1], (uint32_t)((gp >> 1) & 1))) {
+                if (ofree && nPV < nS && __all_sync(0xffffffffu, mbar_try_wait(&p_ready[gp & 1], (uint32_t)((gp >> 1) & 1)))) {
                     tc_fence_after();
                     const int b = nPV, st = gp % NSTAGE;
+                    if (elect_one()) {
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = dP + (((gp & 1) * PBUF + ks * 32) >> 4);
-                        const uint64_t vb = dV + ((st * STAGE + ks * 2048) >> 4);
-                        mma_bf16(tmem + LANE16, ad, vb, idPV, b > 0 || ks > 0);                                 // dims 0..255
-                        mma_bf16(tmem + LANE16 + COL_O2, ad, vb + ((4 * KCHUNK) >> 4), idPV, b > 0 || ks > 0);   // 256..511
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad = dP + (((gp & 1) * PBUF + ks * 32) >> 4);
+                            const uint64_t vb = dV + ((st * STAGE + ks * 2048) >> 4);
+                            mma_bf16(tmem + LANE16, ad, vb, idPV, b > 0 || ks > 0);                                 // dims 0..255
+                            mma_bf16(tmem + LANE16 + COL_O2, ad, vb + ((4 * KCHUNK) >> 4), idPV, b > 0 || ks > 0);   // 256..511
+                        }
+                        mma_commit(&kv_empty[st]);
+                        mma_commit(&o_done[gp & 1]);
+                        if (b + 1 == nb) mma_commit(&o_final[s]);
                     }
-                    mma_commit(&kv_empty[st]);
-                    mma_commit(&o_done[gp & 1]);
-                    if (b + 1 == nb) mma_commit(&o_final[s]);
+                    __syncwarp();
                     ++nPV;
                     progressed = true;
                 }
                 if (progressed) {
-                    t_progress = globaltimer();
+                    t_progress = __shfl_sync(0xffffffffu, globaltimer(), 0);
                 } else if ((++polls & 255u) == 0) {
-                    if (*abort) { ok = false; break; }
-                    if (globaltimer() - t_progress > 2000000000ull) {
-                        *abort = 1;
-                        report(a.status, CSA_ERR_TIMEOUT);
+                    if (__any_sync(0xffffffffu, *abort != 0)) { ok = false; break; }
+                    if (__shfl_sync(0xffffffffu, globaltimer(), 0) - t_progress > 2000000000ull) {
+                        if (lane == 0) {
+                            *abort = 1;
+                            report(a.status, CSA_ERR_TIMEOUT);
+                        }
                         ok = false;
                         break;
                     }
                 }
             }
             if (!ok) break;
-            if (nb == 0) {   // nothing to compute: release Q and complete the query's phases
-                mma_commit(q_free);
-                mma_commit(&o_final[s]);
+            if (elect_one()) {
+                if (nb == 0) {   // nothing to compute: release Q and complete the query's phases
+                    mma_commit(q_free);
+                    mma_commit(&o_final[s]);
+                }
+                mbar_arrive(&plan_free[s]);
             }
-            mbar_arrive(&plan_free[s]);
+            __syncwarp();
             g += nb;
         }
         // leave only when every MMA and commit issued has completed
-        mma_commit(drain);
+        if (elect_one()) mma_commit(drain);
+        __syncwarp();
         mbar_drain(drain, 0);
     }
     tc_fence_before();

@@ -93,26 +93,32 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     const uint32_t tmem = *tmem_ptr;
 
     if (warp == 0) {
-        if (elect_one() && ntiles > 0) {
+        if (ntiles > 0) {
             const uint64_t pol_stream = policy_evict_first();   // k^I is read once per step
             int issued = 0, nseg = 0;
             for (int i = 0; i < ntiles; ++i) {
                 const int64_t g = g_lo + i, b = g / p.tps;
                 const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
                 if (i == 0 || it == 0) {   // a new sequence: its q^I into buffer j & 1
-                    if (!mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status)) break;
-                    mbar_arrive_expect_tx(&qfull[j & 1], b_bytes);
-                    for (int c = 0; c < kchunks; ++c)
-                        tma_load_2d(sB + (j & 1) * b_bytes + c * p.HI * 128, &tm_q, &qfull[j & 1], c * 64,
-                                    (int)(b * p.HI));
+                    if (!__all_sync(0xffffffffu, mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status))) break;
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&qfull[j & 1], b_bytes);
+                        for (int c = 0; c < kchunks; ++c)
+                            tma_load_2d(sB + (j & 1) * b_bytes + c * p.HI * 128, &tm_q, &qfull[j & 1], c * 64,
+                                        (int)(b * p.HI));
+                    }
+                    __syncwarp();
                     nseg = j + 1;
                 }
                 const int st = i % p.stages;
-                if (!mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status)) break;
-                mbar_arrive_expect_tx(&full[st], a_bytes);
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status))) break;
                 const int y = (int)(b * p.T + (int64_t)it * BM);
-                for (int c = 0; c < kchunks; ++c)
-                    tma_load_2d_hint(sA + st * a_bytes + c * BM * 128, &tm_k, &full[st], c * 64, y, pol_stream);
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[st], a_bytes);
+                    for (int c = 0; c < kchunks; ++c)
+                        tma_load_2d_hint(sA + st * a_bytes + c * BM * 128, &tm_k, &full[st], c * 64, y, pol_stream);
+                }
+                __syncwarp();
                 issued = i + 1;
             }
             // never leave with copies in flight into this CTA's shared memory
@@ -122,7 +128,7 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 mbar_wait(&full[i % p.stages], (i / p.stages) & 1, abort, p.status, 100000000ull);
         }
     } else if (warp == 1) {
-        if (lane == 0 && ntiles > 0) {
+        if (ntiles > 0) {
             const uint32_t idesc = idesc_bf16(BM, p.HI);
             const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
             int issued = 0;
@@ -130,20 +136,23 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 const int64_t g = g_lo + i, b = g / p.tps;
                 const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
                 if (i == 0 || it == 0)
-                    if (!mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status)) break;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status))) break;
                 const int st = i % p.stages, buf = i % NACC;
-                if (!mbar_wait(&tempty[buf], ((i / NACC) & 1) ^ 1, abort, p.status)) break;
-                if (!mbar_wait(&full[st], (i / p.stages) & 1, abort, p.status)) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((i / NACC) & 1) ^ 1, abort, p.status))) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / p.stages) & 1, abort, p.status))) break;
                 tc_fence_after();
                 const uint64_t dBj = dB + (((j & 1) * b_bytes) >> 4);
-                for (int c = 0; c < kchunks; ++c)
+                if (elect_one()) {   // one lane issues; the loop itself runs warp-wide (uniform operands)
+                    for (int c = 0; c < kchunks; ++c)
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(tmem + buf * p.HI, dA + ((st * a_bytes + c * BM * 128 + ks * 32) >> 4),
-                                 dBj + ((c * p.HI * 128 + ks * 32) >> 4), idesc, (c | ks) != 0);
-                mma_commit(&empty[st]);
-                mma_commit(&tfull[buf]);
-                if (i + 1 == ntiles || it + 1 == p.tps) mma_commit(&qempty[j & 1]);   // done with this q^I
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tmem + buf * p.HI, dA + ((st * a_bytes + c * BM * 128 + ks * 32) >> 4),
+                                     dBj + ((c * p.HI * 128 + ks * 32) >> 4), idesc, (c | ks) != 0);
+                    mma_commit(&empty[st]);
+                    mma_commit(&tfull[buf]);
+                    if (i + 1 == ntiles || it + 1 == p.tps) mma_commit(&qempty[j & 1]);   // done with this q^I
+                }
+                __syncwarp();
                 issued = i + 1;
             }
             if (issued > 0)

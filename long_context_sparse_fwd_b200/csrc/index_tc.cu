@@ -186,27 +186,31 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tmem_base = *tmem_base_ptr;
 
     if (warp == 0 && ntiles > 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer (warp-wide loop, one elected lane issues) ----------------
         if (elect_one()) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             mbar_arrive_expect_tx(qfull, b_bytes);
             for (int c = 0; c < kchunks; ++c)
                 tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
-            int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int st = i % p.stages;
-                if (!mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status)) break;
+        }
+        __syncwarp();
+        int issued = 0;
+        for (int i = 0; i < ntiles; ++i) {
+            const int st = i % p.stages;
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status))) break;
+            if (elect_one()) {
                 mbar_arrive_expect_tx(&full[st], a_bytes);
                 for (int c = 0; c < kchunks; ++c)
                     tma_load_2d(sA + (size_t)st * a_bytes + (size_t)c * BM * 128, &tm_k, &full[st], c * 64, i * BM);
-                issued = i + 1;
             }
-            // never leave with copies in flight into this CTA's shared memory
-            mbar_wait(qfull, 0, abort, p.status, 100000000ull);
-            for (int i = max(0, issued - p.stages); i < issued; ++i)
-                mbar_wait(&full[i % p.stages], (i / p.stages) & 1, abort, p.status, 100000000ull);
+            __syncwarp();
+            issued = i + 1;
         }
+        // never leave with copies in flight into this CTA's shared memory
+        mbar_wait(qfull, 0, abort, p.status, 100000000ull);
+        for (int i = max(0, issued - p.stages); i < issued; ++i)
+            mbar_wait(&full[i % p.stages], (i / p.stages) & 1, abort, p.status, 100000000ull);
     } else if (warp == 1 && ntiles > 0) {
         // ---------------- MMA issuer ----------------
         const uint32_t idesc = idesc_bf16(BM, BN);
