@@ -10,9 +10,10 @@
 // theta_cmp) plus exp(sink_h); K = V; each branch's rope slice rotated back by -t with its theta.
 //
 // Design. A query's 64 heads form an M=64 tile; its keys (window rows first, then the entries)
-// are gathered 64 at a time with 16-byte cp.async into 128-byte-swizzled shared memory, where the
-// same tile is the K-major B operand of S = Q K^T and the MN-major B operand of O += P V:
-// the selected rows are read from L2/HBM once and shared by all 64 heads. Three key stages.
+// are brought 64 at a time by TMA into 128-byte-swizzled shared memory (window rows as 2-D tiles,
+// entries by four-row gathers), where the same tile is the K-major B operand of S = Q K^T and the
+// MN-major B operand of O += P V: the selected rows are read from L2/HBM once and shared by all
+// 64 heads. Three key stages.
 // Q lives in TMEM as the A operand of S, so shared memory holds only keys and P, and the S
 // MMA reads only the key tile from shared memory.
 //   TMEM (M=64 uses 16 lanes of each 32-lane quarter, "half 0" = lanes +0..15, "half 1" = +16..31):
@@ -32,9 +33,9 @@
 // so almost every block needs no rescale. The sink seeds the reference and the running sum.
 // TMEM is read and written with the 16-lane x2 access shape, so both halves of a warp work on the
 // 16 heads of its quarter (each thread one head, half of the columns).
-// Roles: warps 0-3 softmax + epilogue; warps 4-7 load keys (16-byte cp.async, each row 1 KB in
-// two 512-byte coalesced halves per warp instruction) and write each query's Q into their TMEM
-// quarter; warp 8 owns TMEM and issues MMAs from an event loop (a P V never waits for the next
+// Roles: warps 0-3 softmax + epilogue; warps 4-7 load keys (each warp a quarter of the block's
+// rows, TMA issued by one elected lane; FP8 decode entries are converted by the whole warp) and
+// write each query's Q into their TMEM quarter; warp 8 owns TMEM and issues MMAs from an event loop (a P V never waits for the next
 // block's keys); warp 9 plans: it builds the next query's entry list, block range and rope table
 // in a second slot and prefetches its Q into L2. Key blocks are counted over all of a CTA's
 // queries, so the loaders run into the next query while the current one finishes; the next
@@ -115,13 +116,6 @@ struct Plan {
 static_assert(sizeof(Plan) == 48, "plan layout");
 static_assert(2 * sizeof(Plan) <= 128, "plan slots");
 
-__device__ __forceinline__ void cp_async16_hint(uint32_t dst, const void *src, uint32_t src_bytes, uint64_t policy)
-{
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst), "l"(src), "r"(src_bytes),
-                 "l"(policy)
-                 : "memory");
-}
-
 __device__ __forceinline__ uint4 ldg_hint(const uint4 *p, uint64_t policy)
 {
     uint4 v;
@@ -129,12 +123,6 @@ __device__ __forceinline__ uint4 ldg_hint(const uint4 *p, uint64_t policy)
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p), "l"(policy));
     return v;
-}
-
-// arrive on `bar` when this thread's earlier cp.async copies have landed (no pending-count increment)
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
-{
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Wait (at most 100 ms) for a phase regardless of the abort flag: used before exit so that no
@@ -145,8 +133,6 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
     while (!mbar_try_wait(bar, parity))
         if (globaltimer() - t0 > 100000000ull) return;
 }
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -166,7 +152,8 @@ __device__ __forceinline__ void rotate16(const uint32_t (&w)[16], const float *c
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
+attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
+                 const __grid_constant__ CUtensorMap tm_w, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -206,10 +193,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NSTAGE; ++i) {
-            mbar_init(&kv_full[i], LOAD_THREADS);   // one cp.async arrival per loader thread
+            mbar_init(&kv_full[i], 4);   // one arrival (expect_tx, or after FP8 stores) per loader warp
             mbar_init(&kv_empty[i], 1);
             mbar_init(&kv_rdy[i], 1);
-            mbar_init(&kv_wfull[i], LOAD_THREADS);
+            mbar_init(&kv_wfull[i], 4);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s_full[i], 1);
@@ -493,15 +480,18 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             g += nb;
         }
     } else if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
-        // ===== key loads (16-byte cp.async into the swizzled stages) and Q into TMEM quarter lw =====
+        // ===== key loads (TMA into the swizzled stages) and Q into TMEM quarter lw =====
         const int lw = warp - LOAD_WARP0;        // key rows 16*lw .. 16*lw+15 of each block; heads 16*lw..
         const int hl = lane & 15, hf = lane >> 4;
         const uint32_t tqq = tmem + ((uint32_t)(lw * 32) << 16) + COL_Q;   // Q chunks, half 0 of quarter lw
-        // L2 policies: q is read once; prefill entries are shared by many queries (kept), decode
-        // caches are read once per step; prefill window rows serve ~W consecutive queries (default)
-        const uint64_t pol_once = policy_evict_first();
-        const uint64_t pol_ent = a.decode ? pol_once : policy_evict_last();
-        const uint64_t pol_win = a.decode ? pol_once : policy_evict_normal();
+        const uint64_t pol_once = policy_evict_first();   // q is read once
+        // per stage (bit st): a load of each kind (window / entry) was issued, and the parity of the
+        // phase the last one completes; used to drain the last loads before exit
+        uint32_t w_issued = 0, w_par = 0, e_issued = 0, e_par = 0;
+        if (lane == 0) {
+            prefetch_tmap(&tm_c);
+            prefetch_tmap(&tm_w);
+        }
         int g = 0;
         for (int64_t n = 0;; ++n) {
             const int64_t u = blockIdx.x + n * gridDim.x;
@@ -511,8 +501,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
             const Plan pl = plans[s];
             const int *elist = elist_all + s * kcap;
             const float *rope_cs = rope_tab + s * ROPE_TAB;
-            const uint16_t *win0 = a.kv_rot + pl.win_row * DD;
-            const uint16_t *ent0 = a.decode && a.C != nullptr ? a.C + pl.row * a.T * DD : a.C;
+            const int64_t ent_row0 = a.decode ? pl.row * a.T : 0;   // row of entry 0 in the entry tensor map
             bool ok = true;
             for (int b = 0; b <= pl.nb; ++b) {
                 if (b == min(1, pl.nb)) {
@@ -602,38 +591,60 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcArgs a)
                         *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0 + 1)) = o1;
                     }
                     fence_async_smem();
-                    mbar_arrive(&kv_full[st]);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&kv_full[st]);
                     continue;
                 }
-                // lane j < 16 resolves the source row of key 16*lw + j once; the issue loop below
-                // takes it by shuffle, so no copy waits on a shared-memory lookup
-                const uint16_t *base = win ? win0 : ent0;
-                int my_row = -1;
-                if (lane < 16 && lw * 16 + lane < nk) {
-                    const int kk = kbase + lw * 16 + lane;
-                    my_row = (win || a.idx == nullptr) ? kk : elist[kk];
-                }
-                const uint64_t pol = win ? pol_win : pol_ent;
-                const uint32_t sdst = smem_u32(sKV + st * STAGE) + (lane >> 3) * KCHUNK;   // unit lane (chunk lane/8)
+                // Loader warp lw fills key rows 16*lw .. 16*lw+15 of the stage, 16 KB, with one elected lane
+                // issuing: a window block is consecutive kv_rot rows (a [16 x 64] tile per 64-dim chunk);
+                // an entry block is a gather (four rows per gather4, per chunk). Every slot receives a real
+                // row: window slots past the last key read the rows that follow (or the zero fill past the
+                // tensor), entry slots past the last key repeat it, so masked keys always hold finite values.
+                uint8_t *stage = sKV + st * STAGE + lw * 16 * 128;
+                uint64_t *bar = win ? &kv_wfull[st] : &kv_full[st];
+                if (win) {
+                    const int y = (int)(pl.win_row + kbase + lw * 16);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(bar, 16 * 1024);
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int key = lw * 16 + r;
-                    const int row = __shfl_sync(0xffffffffu, my_row, r);
-                    const bool valid = row >= 0;
-                    // padding rows: zero-filled, 0 bytes read from any mapped address
-                    const uint16_t *rowp = valid ? base + (int64_t)row * DD + lane * 8 : a.q;
-                    const uint32_t d = sdst + sw128(key, lane & 7);
-                    cp_async16_hint(d, rowp, valid ? 16u : 0u, pol);                        // dims 8*lane ..
-                    cp_async16_hint(d + 4 * KCHUNK, valid ? rowp + 256 : a.q, valid ? 16u : 0u, pol);   // 256 + 8*lane ..
+                        for (int dc = 0; dc < NCH; ++dc) tma_load_2d(stage + dc * KCHUNK, &tm_w, bar, dc * 64, y);
+                    }
+                    w_par = (w_issued >> st) & 1u ? w_par ^ (1u << st) : w_par;
+                    w_issued |= 1u << st;
+                } else {
+                    int my_row = 0;
+                    if (lane < 16) {
+                        const int kk = kbase + min(lw * 16 + lane, nk - 1);
+                        my_row = (int)(ent_row0 + (a.idx != nullptr ? elist[kk] : kk));
+                    }
+                    int r4[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) r4[i] = __shfl_sync(0xffffffffu, my_row, i);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(bar, 16 * 1024);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+                            for (int dc = 0; dc < NCH; ++dc)
+                                tma_gather4(stage + dc * KCHUNK + q4 * 512, &tm_c, bar, dc * 64, r4[4 * q4], r4[4 * q4 + 1],
+                                            r4[4 * q4 + 2], r4[4 * q4 + 3]);
+                    }
+                    e_par = (e_issued >> st) & 1u ? e_par ^ (1u << st) : e_par;
+                    e_issued |= 1u << st;
                 }
-                cp_async_arrive_noinc(win ? &kv_wfull[st] : &kv_full[st]);
+                __syncwarp();
             }
             if (!ok) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(&plan_free[s]);
             g += pl.nb;
         }
-        cp_async_wait_all();   // never leave with copies in flight into this CTA's shared memory
+        // never leave with copies in flight into this CTA's shared memory (after an abort some loads
+        // may not have been consumed): wait, bounded, for the last load of each kind into each stage
+        for (int i = 0; i < NSTAGE; ++i) {
+            if ((w_issued >> i) & 1u) mbar_drain(&kv_wfull[i], (w_par >> i) & 1u);
+            if ((e_issued >> i) & 1u) mbar_drain(&kv_full[i], (e_par >> i) & 1u);
+        }
     } else if (warp == MMA_WARP) {
         // =============== MMA issuer: event loop per query ===============
         // The whole warp runs the loop (every decision is made warp-uniform with a vote) and one
@@ -816,8 +827,22 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     a.log2_theta_tok = x.log2_theta_tok;
     a.log2_theta_cmp = x.log2_theta_cmp;
     const size_t smem = 1024 + OFF_LIST + 2 * sizeof(int) * (size_t)((std::max(a.k, 1) + 3) & ~3);
-    CUtensorMap tq;
+    CUtensorMap tq, tc, tw;
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
+    // entry rows (gather4: one-row boxes) and window rows (16-row tiles); row coordinates are int32
+    const uint64_t c_rows = x.decode ? (uint64_t)x.R * x.T : (uint64_t)x.T;
+    const uint64_t w_rows = x.decode ? (uint64_t)x.R * x.W : (uint64_t)x.R;
+    if (c_rows >= (1ull << 31) || w_rows >= (1ull << 31)) return cudaErrorInvalidValue;
+    if (x.C != nullptr && c_rows > 0) {
+        if (!make_tmap_bf16_sw128(&tc, x.C, c_rows, DD, 1)) return cudaErrorInvalidValue;
+    } else {
+        tc = tq;   // FP8 cache (converted by the loader warps) or no entries: never used
+    }
+    if (w_rows > 0) {
+        if (!make_tmap_bf16_sw128(&tw, x.win, w_rows, DD, 16)) return cudaErrorInvalidValue;
+    } else {
+        tw = tq;   // no window rows: never used
+    }
     a.o = out_rows;   // final rows, or the split partials
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -827,7 +852,7 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int64_t units = x.R * nsplit;
     const unsigned grid = (unsigned)std::min<int64_t>(units, std::max(sms, 1));
-    attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, a);
+    attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tc, tw, a);
     return cudaGetLastError();
 }
 
