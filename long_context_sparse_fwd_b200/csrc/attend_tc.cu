@@ -650,6 +650,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // The whole warp runs the loop (every decision is made warp-uniform with a vote) and one
         // elected lane issues the MMAs and commits: with warp-uniform control flow the descriptors
         // stay in uniform registers and each tcgen05.mma issues without per-instruction overhead.
+        // The loop polls with test_wait: a failing try_wait may park the warp until that barrier
+        // completes, which would hold back an S whose keys are ready behind a softmax still running.
         const uint32_t idS = idesc_bf16(64, 64);
         const uint32_t idPV = idesc_bf16(64, 256, true);
         // descriptors are formed once; a tile / k-step offset is added to the start-address field
@@ -679,8 +681,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int sst = gs % NSTAGE;
                 const bool swin = gb0 + nS < nbw;   // window block: wait until its rope slice is turned
                 if (nS < nb && nS <= nPV + 1 &&
-                    __all_sync(0xffffffffu, swin ? mbar_try_wait(&kv_rdy[sst], (wpar >> sst) & 1u)
-                                                 : mbar_try_wait(&kv_full[sst], (epar >> sst) & 1u))) {
+                    __all_sync(0xffffffffu, swin ? mbar_test_wait(&kv_rdy[sst], (wpar >> sst) & 1u)
+                                                 : mbar_test_wait(&kv_full[sst], (epar >> sst) & 1u))) {
                     if (swin) wpar ^= 1u << sst;
                     else epar ^= 1u << sst;
                     fence_async_smem();   // keys were written by cp.async (generic proxy); the MMA reads via the async proxy
@@ -701,10 +703,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     ++nS;
                     progressed = true;
                 }
-                if (!ofree && nPV < nS) ofree = __all_sync(0xffffffffu, mbar_try_wait(o_free, (uint32_t)((n - 1) & 1)));
+                if (!ofree && nPV < nS) ofree = __all_sync(0xffffffffu, mbar_test_wait(o_free, (uint32_t)((n - 1) & 1)));
                 // PV(nPV) needs the softmax of block nPV (and, for the first, O of the previous query read out)
                 const int gp = g + nPV;
-                if (ofree && nPV < nS && __all_sync(0xffffffffu, mbar_try_wait(&p_ready[gp & 1], (uint32_t)((gp >> 1) & 1)))) {
+                if (ofree && nPV < nS && __all_sync(0xffffffffu, mbar_test_wait(&p_ready[gp & 1], (uint32_t)((gp >> 1) & 1)))) {
                     tc_fence_after();
                     const int b = nPV, st = gp % NSTAGE;
                     if (elect_one()) {

@@ -60,6 +60,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of the phase with `parity` (test_wait never suspends the thread, unlike a
+// failing try_wait, which may park it until the phase completes): for event loops that poll
+// several barriers in turn.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with `parity` of `bar`. Gives up when *abort is set by another role or
 // after `limit_ns` of waiting; on a timeout it sets *abort and records CSA_ERR_TIMEOUT in the
 // status word. Returns false when it gave up.
