@@ -14,9 +14,10 @@
 // entry stay in shared memory; after the last entry tile each epilogue warp runs an exact radix
 // select for one query and writes the kept indices in ascending order.
 //
-// Roles (6 warps): warp 0 issues TMA loads (q^I block once, k^I tiles through a ring of stages),
+// Roles (10 warps): warp 0 issues TMA loads (q^I block once, k^I tiles through a ring of stages),
 // warp 1 owns TMEM (2 x 256 columns, double-buffered accumulators) and issues tcgen05.mma, warps
-// 2-5 read TMEM, score, and select. Every wait is bounded; a timeout sets CSA_ERR_TIMEOUT.
+// 2-9 read TMEM and score (two warps per lane quarter, each half of the queries), then select.
+// Every wait is bounded; a timeout sets CSA_ERR_TIMEOUT.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -30,8 +31,8 @@ namespace {
 
 constexpr int BM = 128;          // entries per tile = TMEM lanes
 constexpr int BN = 256;          // (query, head) columns
-constexpr int NUM_THREADS = 192;
-constexpr int EPI_THREADS = 128;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_THREADS = 256;       // warps 2-9: two warps per TMEM lane quarter, each half of the queries
 constexpr uint32_t TMEM_COLS = 512;
 
 struct IdxParams {
@@ -147,8 +148,8 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint8_t *sA = sB + b_bytes;
     float *scores = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [Q][T_cap]
     float *sw = scores + (size_t)p.Q * p.T_cap;                                  // [BN]
-    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                      // [4][256]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 4 * 256);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                      // [8][256]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 8 * 256);
     uint64_t *full = bars;                   // [stages]
     uint64_t *empty = bars + 8;              // [stages]
     uint64_t *tfull = bars + 16;             // [2]
@@ -243,33 +244,51 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
     } else if (warp >= 2) {
         // ---------------- epilogue: scores into shared memory ----------------
-        const int quarter = warp & 3;              // TMEM lanes this warp may read
+        // warp w reads TMEM lane quarter w % 4 (entries 32*(w%4) .. +31 of the tile); warps 2-5 take
+        // the first half of the block's queries, warps 6-9 the second half
+        const int quarter = warp & 3;
+        const int qhalf = (warp - 2) >> 2;
+        const int qlo = qhalf * (p.Q >> 1), qhi = qlo + (p.Q >> 1);   // Q = 256 / HI is even
         for (int i = 0; i < ntiles; ++i) {
             const int buf = i & 1;
             if (!mbar_wait(&tfull[buf], (i >> 1) & 1, abort, p.status)) break;
             tc_fence_after();
             const int s = i * BM + quarter * 32 + lane;
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-            for (int q = 0; q < p.Q; ++q) {
-                float acc = 0.f;
+            for (int q = qlo; q < qhi; ++q) {
+                // four independent partial sums break the dependent multiply-add chain
+                float acc4[4] = {0.f, 0.f, 0.f, 0.f};
                 // columns [q*HI, (q+1)*HI) of this buffer; never read past them (HI = 16 uses x16 loads)
                 for (int h0 = 0; h0 < p.HI; h0 += 16) {
-                    const float *wq = sw + q * p.HI + h0;
+                    const float4 *wq4 = reinterpret_cast<const float4 *>(sw + q * p.HI + h0);
                     if (h0 + 32 <= p.HI) {
                         float v[32];
                         tmem_ld32(taddr + q * p.HI + h0, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 32; ++j) acc = fmaf(wq[j], fmaxf(v[j], 0.f), acc);
+                        for (int j = 0; j < 8; ++j) {
+                            const float4 w4 = wq4[j];
+                            acc4[0] = fmaf(w4.x, fmaxf(v[4 * j], 0.f), acc4[0]);
+                            acc4[1] = fmaf(w4.y, fmaxf(v[4 * j + 1], 0.f), acc4[1]);
+                            acc4[2] = fmaf(w4.z, fmaxf(v[4 * j + 2], 0.f), acc4[2]);
+                            acc4[3] = fmaf(w4.w, fmaxf(v[4 * j + 3], 0.f), acc4[3]);
+                        }
                         h0 += 16;
                     } else {
                         float v[16];
                         tmem_ld16(taddr + q * p.HI + h0, v);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) acc = fmaf(wq[j], fmaxf(v[j], 0.f), acc);
+                        for (int j = 0; j < 4; ++j) {
+                            const float4 w4 = wq4[j];
+                            acc4[0] = fmaf(w4.x, fmaxf(v[4 * j], 0.f), acc4[0]);
+                            acc4[1] = fmaf(w4.y, fmaxf(v[4 * j + 1], 0.f), acc4[1]);
+                            acc4[2] = fmaf(w4.z, fmaxf(v[4 * j + 2], 0.f), acc4[2]);
+                            acc4[3] = fmaf(w4.w, fmaxf(v[4 * j + 3], 0.f), acc4[3]);
+                        }
                     }
                 }
+                const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
                 if (s < p.T_cap) scores[q * p.T_cap + s] = acc + 0.0f;
             }
             tc_fence_before();
@@ -278,7 +297,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         named_barrier_sync(1, EPI_THREADS);
         // ---------------- exact top-k, one query per warp ----------------
         if (!*abort) {
-            for (int q = warp - 2; q < p.Q; q += 4) {
+            for (int q = warp - 2; q < p.Q; q += 8) {
                 const int64_t t = t0 + q;
                 if (t >= p.S) continue;
                 const int n = (int)visible_entries(t, p.m, p.T);
@@ -365,7 +384,7 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     p.Q = BN / HI;
     p.T_cap = (int)((T + BM - 1) / BM * BM);
     const size_t a_bytes = (size_t)(dI / 64) * BM * 128, b_bytes = (size_t)(dI / 64) * BN * 128;
-    const size_t fixed = 1024 + b_bytes + (size_t)p.Q * p.T_cap * 4 + BN * 4 + 4 * 256 * 4 + 256;
+    const size_t fixed = 1024 + b_bytes + (size_t)p.Q * p.T_cap * 4 + BN * 4 + 8 * 256 * 4 + 256;
     const size_t budget = 227 * 1024;
     p.stages = (int)std::min<size_t>(4, (budget - fixed) / a_bytes);
     if (p.stages < 2) return cudaErrorInvalidValue;
