@@ -556,39 +556,59 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int nk = win ? min(KB, pl.nw - kbase) : min(KB, pl.ne - kbase);
                 if (!win && a.C == nullptr) {
                     // FP8 entry cache: codes * per-entry scale on channels [0,448), bf16 rope on [448,512),
-                    // converted to bf16 here and stored into the swizzled stage
+                    // converted to bf16 here and stored into the swizzled stage. Lane j < 28 handles
+                    // channels [16j, 16j+16) of each row, lanes 28..31 the rope channels 448 + 16*(lane-28).
+                    // The loads of 8 rows are issued together before any is converted.
                     uint8_t *stage = sKV + st * STAGE;
-#pragma unroll 2
-                    for (int r = 0; r < 16; ++r) {
-                        const int key = lw * 16 + r;
-                        uint4 o0 = make_uint4(0u, 0u, 0u, 0u), o1 = o0;
-                        if (key < nk) {
-                            const int64_t e = pl.row * a.T + (a.idx != nullptr ? elist[kbase + key] : kbase + key);
+                    const int d0 = lane < 28 ? 16 * lane : 448 + 16 * (lane - 28);
+                    const int dc = d0 >> 6, u0 = (d0 & 63) >> 3;
+                    int my_e = 0;   // entry (row of the flattened cache) of key 16*lw + lane, lanes < 16
+                    if (lane < 16) {
+                        const int kk = kbase + min(lw * 16 + lane, nk - 1);
+                        my_e = (int)(pl.row * a.T + (a.idx != nullptr ? elist[kk] : kk));
+                    }
+#pragma unroll 1
+                    for (int r0 = 0; r0 < 16; r0 += 8) {
+                        uint4 raw[8], rope1[8];
+                        float sc[8];
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const int64_t e = __shfl_sync(0xffffffffu, my_e, r0 + r);
                             if (lane < 28) {
-                                const float sc = __ldg(a.c8_scale + e);
-                                const uint4 cv = __ldg(reinterpret_cast<const uint4 *>(a.c8 + e * 448) + lane);
-                                const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+                                sc[r] = __ldg(a.c8_scale + e);
+                                raw[r] = __ldg(reinterpret_cast<const uint4 *>(a.c8 + e * 448) + lane);
+                            } else {
+                                const uint4 *rr = reinterpret_cast<const uint4 *>(a.c_rope + e * 64);
+                                raw[r] = __ldg(rr + 2 * (lane - 28));
+                                rope1[r] = __ldg(rr + 2 * (lane - 28) + 1);
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < 8; ++r) {
+                            const int key = lw * 16 + r0 + r;
+                            uint4 o0, o1;
+                            if (key >= nk) {   // padding keys hold zeros
+                                o0 = make_uint4(0u, 0u, 0u, 0u);
+                                o1 = o0;
+                            } else if (lane < 28) {
+                                const uint32_t cw[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
                                 uint32_t ow[8];
 #pragma unroll
                                 for (int q2 = 0; q2 < 8; ++q2) {
                                     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(
                                         (__nv_fp8x2_storage_t)((cw[q2 >> 1] >> ((q2 & 1) * 16)) & 0xffffu), __NV_E4M3);
                                     const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&hr));
-                                    ow[q2] = pack_bf2(f.x * sc, f.y * sc);
+                                    ow[q2] = pack_bf2(f.x * sc[r], f.y * sc[r]);
                                 }
                                 o0 = make_uint4(ow[0], ow[1], ow[2], ow[3]);
                                 o1 = make_uint4(ow[4], ow[5], ow[6], ow[7]);
                             } else {
-                                const uint4 *rr = reinterpret_cast<const uint4 *>(a.c_rope + e * 64);
-                                o0 = __ldg(rr + 2 * (lane - 28));
-                                o1 = __ldg(rr + 2 * (lane - 28) + 1);
+                                o0 = raw[r];
+                                o1 = rope1[r];
                             }
+                            *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0)) = o0;
+                            *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0 + 1)) = o1;
                         }
-                        // lane < 28: dims [16*lane, 16*lane+16); lanes 28..31: rope dims 448 + 16*(lane-28)
-                        const int d0 = lane < 28 ? 16 * lane : 448 + 16 * (lane - 28);
-                        const int dc = d0 >> 6, u0 = (d0 & 63) >> 3;
-                        *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0)) = o0;
-                        *reinterpret_cast<uint4 *>(stage + dc * KCHUNK + sw128(key, u0 + 1)) = o1;
                     }
                     fence_async_smem();
                     __syncwarp();
