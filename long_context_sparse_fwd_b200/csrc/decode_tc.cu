@@ -10,10 +10,10 @@
 // D[s,h] = kI[s,:] . qI[b,h,:] (entries on TMEM lanes, M=128 x N=HI), and each epilogue thread
 // reduces its entry's HI heads in registers and writes one fp32 score.
 //
-// Top-k is exact and deterministic in two stages: every chunk of CHUNK scores keeps its own top-k
-// (any entry of the global top-k is in its chunk's top-k under the same order), then one CTA per
-// sequence selects the final k from the chunk candidates. Both stages are radix selects over
-// order-preserving uint32 keys with ties to the smaller entry index; indices come out ascending.
+// Top-k is exact and deterministic: the scan also records each sequence's key range; a histogram of
+// the leading differing key bits over all of a sequence's scores finds the threshold bin; the
+// entries above it are marked in a bitmap and those in it collected; one CTA per sequence ranks the
+// collected ones and writes the selection in ascending index order (ties to the smaller index).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -30,13 +30,12 @@ constexpr int NUM_THREADS = 192;
 constexpr int EPI_THREADS = 128;
 constexpr int MAX_STAGES = 6;
 constexpr int NACC = 4;                // TMEM accumulators (each HI columns) in flight
-constexpr int SEL_CHUNK = 8192;        // scores per first-stage select CTA
-constexpr int SEL_THREADS = 512;
-constexpr int MERGE_THREADS = 1024;
 
 struct ScoreParams {
     const float *w;      // [B, HI]
     float *scores;       // [B, T]
+    uint32_t *keymax;    // [B] largest order-preserving score key (zero before the scan)
+    uint32_t *nkeymin;   // [B] largest complemented key, i.e. ~(smallest key) (zero before the scan)
     int32_t *status;
     int64_t T, G;        // entries per sequence; total tiles (B * tiles per sequence)
     int HI, dI, stages, tps;
@@ -162,9 +161,30 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         const int quarter = warp & 3, etid = threadIdx.x - 64;
         const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
         float wr[64];   // index weights of the current sequence (HI == 64 keeps them in registers)
+        // range of the score keys of the current sequence seen by this thread, merged into the
+        // sequence's global range (for the top-k's histogram) whenever the sequence changes
+        uint32_t kmax = 0u, knmin = 0u;
+        int64_t b_cur = -1;
+        auto flush_range = [&]() {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+                knmin = max(knmin, __shfl_xor_sync(0xffffffffu, knmin, o));
+            }
+            if (lane == 0 && b_cur >= 0) {
+                atomicMax(p.keymax + b_cur, kmax);
+                atomicMax(p.nkeymin + b_cur, knmin);
+            }
+            kmax = 0u;
+            knmin = 0u;
+        };
         for (int i = 0; i < ntiles; ++i) {
             const int64_t g = g_lo + i, b = g / p.tps;
             const int it = (int)(g - b * p.tps);
+            if (b != b_cur) {
+                flush_range();
+                b_cur = b;
+            }
             if (i == 0 || it == 0) {   // index weights of the new sequence
                 named_barrier_sync(1, EPI_THREADS);
                 for (int h = etid; h < p.HI; h += EPI_THREADS) sw[h] = p.w[b * p.HI + h];
@@ -211,8 +231,14 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 mbar_arrive(&tempty[buf]);
             }
             const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
-            if (s < p.T) p.scores[b * p.T + s] = acc + 0.0f;
+            if (s < p.T) {
+                p.scores[b * p.T + s] = acc + 0.0f;
+                const uint32_t key = score_key(acc);
+                kmax = max(kmax, key);
+                knmin = max(knmin, ~key);
+            }
         }
+        flush_range();
     }
     tc_fence_before();
     __syncthreads();
@@ -222,7 +248,160 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     }
 }
 
-// ---- block-level exact selection over keys in shared memory ------------------------------------------
+// ---- exact top-k by a histogram of the leading differing key bits ----------------------------------
+//
+// Keys are the order-preserving uint32 images of the scores. Over a sequence the keys share every bit
+// above `top` (the highest bit where its smallest and largest key differ); the histogram digit is the
+// (up to) 11 bits [shift, top] below them, so a larger digit means a larger key. The threshold digit
+// d* is the largest one whose suffix count reaches k: every key with a larger digit is selected
+// outright (a bitmap bit per entry), the keys with digit d* are collected as candidates, and the
+// final kernel ranks the candidates (key descending, then entry index ascending) to take the rest.
+// Indices come out ascending from the bitmap; ties go to the smaller index.
+
+constexpr int HBINS = 2048;
+constexpr int TK_CHUNK = 8192;         // entries per histogram / collect CTA
+constexpr int TK_THREADS = 512;
+constexpr int FIN_THREADS = 1024;
+constexpr int CAND_CAP = 2048;         // candidates ranked directly; more take the exact fallback
+
+struct KeyRange {
+    uint32_t prefix_hi;   // the common high bits (bits above top), as in every key
+    int shift;            // digit = (key >> shift) & dmask
+    uint32_t dmask;
+};
+
+__device__ __forceinline__ KeyRange key_range(uint32_t kmax, uint32_t knmin)
+{
+    const uint32_t lo = ~knmin, hi = kmax;
+    KeyRange r;
+    const uint32_t diff = lo ^ hi;
+    if (diff == 0u) {   // one key value: a single bin
+        r.shift = 0;
+        r.dmask = 0u;
+        r.prefix_hi = hi;
+        return r;
+    }
+    const int top = 31 - __clz(diff);
+    r.shift = max(0, top - 10);
+    r.dmask = (2u << (top - r.shift)) - 1u;
+    r.prefix_hi = top == 31 ? 0u : (hi & ~((2u << top) - 1u));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t key_digit(uint32_t key, const KeyRange &r) { return (key >> r.shift) & r.dmask; }
+
+// Threshold digit of a sequence from its histogram (block of `nthreads` >= HBINS / 4 threads; every
+// thread gets the result): d* and the number of keys with a larger digit. Needs T > k.
+__device__ void find_threshold(const uint32_t *hist_g, int k, uint32_t *sh_hist, uint32_t *sh_sums, int *dstar,
+                               uint32_t *above)
+{
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int i = tid; i < HBINS; i += nt) sh_hist[i] = hist_g[i];
+    __syncthreads();
+    // thread t < 512 owns bins [4t, 4t+4); suffix sums over the owners from the top
+    uint32_t own = 0;
+    if (tid < HBINS / 4)
+        own = sh_hist[4 * tid] + sh_hist[4 * tid + 1] + sh_hist[4 * tid + 2] + sh_hist[4 * tid + 3];
+    if (tid < HBINS / 4) sh_sums[tid] = own;
+    __syncthreads();
+    if (tid < 32) {   // warp 0: suffix scan of the 512 owner sums (16 per lane)
+        uint32_t v[16], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) { v[j] = sh_sums[tid * 16 + j]; tot += v[j]; }
+        uint32_t after = tot;   // sums held by higher lanes
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_down_sync(0xffffffffu, after, o);
+            if (tid + o < 32) after += x;
+        }
+        after -= tot;
+        uint32_t run = after;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) {   // exclusive suffix: keys in owners above owner 16*lane+j
+            const uint32_t vj = v[j];
+            sh_sums[tid * 16 + j] = run;
+            run += vj;
+        }
+    }
+    __syncthreads();
+    if (tid < HBINS / 4) {
+        uint32_t run = sh_sums[tid];   // keys in bins >= 4*tid + 4
+        for (int j = 3; j >= 0; --j) {
+            const uint32_t c = sh_hist[4 * tid + j];
+            if (run < (uint32_t)k && run + c >= (uint32_t)k) {
+                sh_sums[HBINS / 4] = (uint32_t)(4 * tid + j);
+                sh_sums[HBINS / 4 + 1] = run;
+            }
+            run += c;
+        }
+    }
+    __syncthreads();
+    *dstar = (int)sh_sums[HBINS / 4];
+    *above = sh_sums[HBINS / 4 + 1];
+    __syncthreads();
+}
+
+// Histogram of the digits of one chunk of one sequence's scores, added into the sequence's histogram.
+__global__ void __launch_bounds__(TK_THREADS)
+topk_hist_kernel(const float *__restrict__ scores, int64_t T, const uint32_t *__restrict__ keymax,
+                 const uint32_t *__restrict__ nkeymin, uint32_t *__restrict__ hist)
+{
+    __shared__ uint32_t sh[HBINS];
+    const int b = blockIdx.y;
+    const KeyRange r = key_range(keymax[b], nkeymin[b]);
+    for (int i = threadIdx.x; i < HBINS; i += TK_THREADS) sh[i] = 0;
+    __syncthreads();
+    const int64_t s0 = (int64_t)blockIdx.x * TK_CHUNK;
+    const int n = (int)min((int64_t)TK_CHUNK, T - s0);
+    const float *sc = scores + b * T + s0;
+    for (int i = threadIdx.x; i < n; i += TK_THREADS) atomicAdd(&sh[key_digit(score_key(sc[i]), r)], 1u);
+    __syncthreads();
+    uint32_t *hg = hist + (int64_t)b * HBINS;
+    for (int i = threadIdx.x; i < HBINS; i += TK_THREADS)
+        if (sh[i] != 0u) atomicAdd(hg + i, sh[i]);
+}
+
+// Entries with a digit above d* set their bitmap bit (one ballot word per warp and 32 entries);
+// entries with digit d* are appended to the sequence's candidate list.
+__global__ void __launch_bounds__(TK_THREADS)
+topk_collect_kernel(const float *__restrict__ scores, int64_t T, int k, const uint32_t *__restrict__ keymax,
+                    const uint32_t *__restrict__ nkeymin, const uint32_t *__restrict__ hist, uint32_t *__restrict__ bitmap,
+                    uint32_t *__restrict__ ncand, uint2 *__restrict__ cand)
+{
+    __shared__ uint32_t sh_hist[HBINS];
+    __shared__ uint32_t sh_sums[HBINS / 4 + 2];
+    const int b = blockIdx.y;
+    const KeyRange r = key_range(keymax[b], nkeymin[b]);
+    int dstar;
+    uint32_t above;
+    find_threshold(hist + (int64_t)b * HBINS, k, sh_hist, sh_sums, &dstar, &above);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t s0 = (int64_t)blockIdx.x * TK_CHUNK;
+    const int64_t nw = (T + 31) >> 5;
+    uint32_t *bm = bitmap + b * nw;
+    uint2 *cb = cand + (int64_t)b * CAND_CAP;
+    for (int base = warp * 32; base < TK_CHUNK; base += TK_THREADS) {
+        const int64_t s = s0 + base + lane;
+        bool take = false, isc = false;
+        uint32_t key = 0u;
+        if (s < T) {
+            key = score_key(scores[b * T + s]);
+            const int d = (int)key_digit(key, r);
+            take = d > dstar;
+            isc = d == dstar;
+        }
+        const unsigned tb = __ballot_sync(0xffffffffu, take);
+        if (s0 + base < T && lane == 0) bm[(s0 + base) >> 5] = tb;
+        const unsigned cb_mask = __ballot_sync(0xffffffffu, isc);
+        if (cb_mask != 0u) {
+            uint32_t pos0 = 0;
+            if (lane == 0) pos0 = atomicAdd(ncand + b, (uint32_t)__popc(cb_mask));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            const uint32_t pos = pos0 + __popc(cb_mask & ((1u << lane) - 1u));
+            if (isc && pos < (uint32_t)CAND_CAP) cb[pos] = make_uint2(key, (uint32_t)s);
+        }
+    }
+}
 
 // inclusive scan of one int per thread over the block; *total receives the block sum
 __device__ __forceinline__ int block_incl_scan(int v, int *wsum, int *total)
@@ -251,205 +430,158 @@ __device__ __forceinline__ int block_incl_scan(int v, int *wsum, int *total)
     return v + before;
 }
 
-// Keep the k largest of keys[0..n) (ties: smaller position first). Writes the kept positions in
-// ascending order to pos[0..min(k,n)) and returns that count. hist: 256 words; sh: 40 words.
-// The radix digits start at the highest bit where the keys differ (scores of one query usually
-// share sign and leading exponent bits, which would put every key into one or two bins).
-__device__ int block_select(const uint32_t *keys, int n, int k, int *pos, uint32_t *hist, int *sh)
+// One CTA per sequence: take the `remaining` best candidates of bin d*, then write the selected
+// entries in ascending order from the bitmap (-1 padding when the sequence has fewer than k entries).
+__global__ void __launch_bounds__(FIN_THREADS)
+topk_final_kernel(const float *__restrict__ scores, int64_t T, int k, const uint32_t *__restrict__ keymax,
+                  const uint32_t *__restrict__ nkeymin, const uint32_t *__restrict__ hist, uint32_t *__restrict__ bitmap,
+                  const uint32_t *__restrict__ ncand, const uint2 *__restrict__ cand, int32_t *__restrict__ idx)
 {
-    if (n <= k) {
-        for (int i = threadIdx.x; i < n; i += blockDim.x) pos[i] = i;
-        __syncthreads();
-        return n;
-    }
-    // smallest and largest key
-    uint32_t lo = 0xffffffffu, hi = 0u;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        lo = min(lo, keys[i]);
-        hi = max(hi, keys[i]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
-    }
-    uint32_t *red = reinterpret_cast<uint32_t *>(hist);   // 2 x 32 words of scratch before the passes
-    if ((threadIdx.x & 31) == 0) {
-        red[threadIdx.x >> 5] = lo;
-        red[32 + (threadIdx.x >> 5)] = hi;
-    }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int nw = blockDim.x >> 5;
-        uint32_t l2 = threadIdx.x < nw ? red[threadIdx.x] : 0xffffffffu;
-        uint32_t h2 = threadIdx.x < nw ? red[32 + threadIdx.x] : 0u;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            l2 = min(l2, __shfl_xor_sync(0xffffffffu, l2, o));
-            h2 = max(h2, __shfl_xor_sync(0xffffffffu, h2, o));
-        }
-        if (threadIdx.x == 0) {
-            sh[35] = (int)l2;
-            sh[36] = (int)h2;
-        }
-    }
-    __syncthreads();
-    lo = (uint32_t)sh[35];
-    hi = (uint32_t)sh[36];
-    __syncthreads();
-    uint32_t prefix, mask, remaining = (uint32_t)k;
-    int lowbit;   // bits [0, lowbit) are still undecided
-    if (lo == hi) {
-        prefix = hi;
-        mask = 0xffffffffu;
-        lowbit = 0;
-    } else {
-        const int top = 31 - __clz(lo ^ hi);   // highest differing bit; bits above it are common
-        mask = top == 31 ? 0u : ~((2u << top) - 1u);
-        prefix = hi & mask;
-        lowbit = top + 1;
-    }
-    while (lowbit > 0) {
-        const int width = min(8, lowbit), shift = lowbit - width;
-        const uint32_t dm = (1u << width) - 1u;
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const uint32_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dm], 1u);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
-            uint32_t c[8], tot = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) { c[j] = hist[lane * 8 + j]; tot += c[j]; }
-            uint32_t above = tot;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t v = __shfl_down_sync(0xffffffffu, above, o);
-                if (lane + o < 32) above += v;
-            }
-            above -= tot;
-            int found = -1;
-            uint32_t above_d = 0, cnt_d = 0, run = above;
-#pragma unroll
-            for (int j = 7; j >= 0; --j) {
-                if (found < 0 && run + c[j] >= remaining) { found = lane * 8 + j; above_d = run; cnt_d = c[j]; }
-                run += c[j];
-            }
-            if (found >= 0 && above < remaining) {
-                sh[32] = found;
-                sh[33] = (int)above_d;
-                sh[34] = (int)cnt_d;
-            }
-        }
-        __syncthreads();
-        prefix |= (uint32_t)sh[32] << shift;
-        mask |= dm << shift;
-        remaining -= (uint32_t)sh[33];
-        const bool whole_bucket = (uint32_t)sh[34] == remaining;
-        lowbit = shift;
-        __syncthreads();
-        if (whole_bucket) break;
-    }
-    // ordered compaction: each thread owns a contiguous run of positions; two block scans place the
-    // kept positions (keys above the threshold, and the first `remaining` equal ones) in order
-    const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
-    const int b0 = min(n, (int)threadIdx.x * per), b1 = min(n, b0 + per);
-    int ngt = 0, neq = 0;
-    for (int i = b0; i < b1; ++i) {
-        const uint32_t key = keys[i] & mask;
-        ngt += key > prefix;
-        neq += key == prefix;
-    }
-    int eq_tot;
-    const int eq_before = block_incl_scan(neq, sh, &eq_tot) - neq;
-    int take_eq = min(max((int)remaining - eq_before, 0), neq);
-    const int cnt = ngt + take_eq;
-    int total;
-    int off = block_incl_scan(cnt, sh, &total) - cnt;
-    for (int i = b0; i < b1; ++i) {
-        const uint32_t key = keys[i] & mask;
-        if (key > prefix || (key == prefix && take_eq-- > 0)) pos[off++] = i;
-    }
-    __syncthreads();
-    return min(total, k);
-}
-
-// Stage 1: per (chunk of SEL_CHUNK scores, sequence) keep the chunk's top-k.
-// cand_idx / cand_key: [B, nchunks, k] (entry index, key); unused slots hold -1 / 0.
-__global__ void __launch_bounds__(SEL_THREADS)
-topk_chunk_kernel(const float *__restrict__ scores, int64_t T, int k, int32_t *__restrict__ cand_idx,
-                  uint32_t *__restrict__ cand_key)
-{
-    extern __shared__ uint32_t csm[];
-    uint32_t *keys = csm;                                          // [SEL_CHUNK]
-    int *pos = reinterpret_cast<int *>(csm + SEL_CHUNK);           // [SEL_CHUNK]
-    __shared__ uint32_t hist[256];
-    __shared__ int sh[40];
-    const int b = blockIdx.y, nchunks = gridDim.x;
-    const int64_t s0 = (int64_t)blockIdx.x * SEL_CHUNK;
-    const int n = (int)min((int64_t)SEL_CHUNK, T - s0);
-    const float *sc = scores + (int64_t)b * T + s0;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = score_key(sc[i]);
-    __syncthreads();
-    const int kk = min(k, SEL_CHUNK);
-    const int cnt = block_select(keys, n, kk, pos, hist, sh);
-    int32_t *oi = cand_idx + ((int64_t)b * nchunks + blockIdx.x) * k;
-    uint32_t *ok = cand_key + ((int64_t)b * nchunks + blockIdx.x) * k;
-    for (int j = threadIdx.x; j < k; j += blockDim.x) {
-        if (j < cnt) {
-            oi[j] = (int32_t)(s0 + pos[j]);
-            ok[j] = keys[pos[j]];
-        } else {
-            oi[j] = -1;
-            ok[j] = 0u;
-        }
-    }
-}
-
-// Stage 2: per sequence, the final top-k among the chunk candidates. Every chunk but the last
-// holds exactly k candidates (k <= SEL_CHUNK), so the valid candidates are a prefix of the array,
-// already in ascending entry order.
-__global__ void __launch_bounds__(MERGE_THREADS)
-topk_merge_kernel(const int32_t *__restrict__ cand_idx, const uint32_t *__restrict__ cand_key, int64_t T, int nchunks,
-                  int k, int32_t *__restrict__ idx)
-{
-    extern __shared__ uint32_t msm[];
-    __shared__ uint32_t hist[256];
-    __shared__ int sh[40];
-    const int b = blockIdx.x;
-    const int total_max = nchunks * k;
-    const int total = (nchunks - 1) * k + (int)min((int64_t)k, T - (int64_t)(nchunks - 1) * SEL_CHUNK);
-    uint32_t *keys = msm;                                         // [total_max]
-    int *ids = reinterpret_cast<int *>(msm + total_max);          // [total_max]
-    int *pos = ids + total_max;                                   // [total_max]
-    const int32_t *ci = cand_idx + (int64_t)b * total_max;
-    const uint32_t *ck = cand_key + (int64_t)b * total_max;
-    for (int j = threadIdx.x; j < total; j += blockDim.x) {
-        keys[j] = ck[j];
-        ids[j] = ci[j];
-    }
-    __syncthreads();
-    const int cnt = block_select(keys, total, k, pos, hist, sh);
+    __shared__ uint32_t sh_hist[HBINS];
+    __shared__ uint32_t sh_sums[HBINS / 4 + 2];
+    __shared__ uint2 sc[CAND_CAP];
+    __shared__ int wsum[32];
+    __shared__ uint32_t sh_sel[4];
+    const int b = blockIdx.x, tid = threadIdx.x;
     int32_t *out = idx + (int64_t)b * k;
-    for (int j = threadIdx.x; j < k; j += blockDim.x) out[j] = j < cnt ? ids[pos[j]] : -1;
+    if (T <= k) {   // every entry is selected
+        for (int j = tid; j < k; j += FIN_THREADS) out[j] = j < T ? j : -1;
+        return;
+    }
+    const KeyRange r = key_range(keymax[b], nkeymin[b]);
+    int dstar;
+    uint32_t above;
+    find_threshold(hist + (int64_t)b * HBINS, k, sh_hist, sh_sums, &dstar, &above);
+    const uint32_t remaining = (uint32_t)k - above;
+    const int64_t nw = (T + 31) >> 5;
+    uint32_t *bm = bitmap + b * nw;
+    const uint32_t n = ncand[b];
+    if (n <= (uint32_t)CAND_CAP) {
+        const uint2 *cb = cand + (int64_t)b * CAND_CAP;
+        for (uint32_t i = tid; i < n; i += FIN_THREADS) sc[i] = cb[i];
+        __syncthreads();
+        for (uint32_t i = tid; i < n; i += FIN_THREADS) {
+            const uint2 me = sc[i];
+            uint32_t rank = 0;
+            for (uint32_t j = 0; j < n; ++j) {
+                const uint2 o = sc[j];
+                rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+            }
+            if (rank < remaining) atomicOr(bm + (me.y >> 5), 1u << (me.y & 31));
+        }
+    } else {
+        // Exact fallback for a crowded threshold bin: radix passes (8 bits) over the keys of bin d*,
+        // read from the scores, below the digit; then the keys above the final threshold and the
+        // first `remaining` equal ones in index order.
+        const float *sq = scores + b * T;
+        uint32_t mask = r.dmask == 0u ? 0xffffffffu : ~((1u << r.shift) - 1u);
+        uint32_t prefix = r.prefix_hi | ((uint32_t)dstar << r.shift);
+        uint32_t rem = remaining;
+        int lowbit = r.dmask == 0u ? 0 : r.shift;
+        uint32_t *h256 = sh_hist;   // 256 bins
+        while (lowbit > 0) {
+            const int width = min(8, lowbit), shf = lowbit - width;
+            const uint32_t dm = (1u << width) - 1u;
+            for (int i = tid; i < 256; i += FIN_THREADS) h256[i] = 0;
+            __syncthreads();
+            for (int64_t i = tid; i < T; i += FIN_THREADS) {
+                const uint32_t key = score_key(sq[i]);
+                if ((key & mask) == prefix) atomicAdd(&h256[(key >> shf) & dm], 1u);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t run = 0;
+                int d = 255;
+                for (; d > 0; --d) {
+                    if (run + h256[d] >= rem) break;
+                    run += h256[d];
+                }
+                sh_sel[0] = (uint32_t)d;
+                sh_sel[1] = run;
+                sh_sel[2] = h256[d];
+            }
+            __syncthreads();
+            prefix |= sh_sel[0] << shf;
+            mask |= dm << shf;
+            rem -= sh_sel[1];
+            lowbit = shf;
+            const bool whole = sh_sel[2] == rem;
+            __syncthreads();
+            if (whole) break;
+        }
+        // selection in index order, 1024 entries per round
+        int eq_seen = 0;
+        for (int64_t base = 0; base < T; base += FIN_THREADS) {
+            const int64_t i = base + tid;
+            uint32_t key = 0u;
+            bool gt = false, eq = false;
+            if (i < T) {
+                key = score_key(sq[i]);
+                gt = (key & mask) > prefix;   // keys of bin d* above the threshold (higher bins are set already)
+                eq = (key & mask) == prefix;
+            }
+            int tot;
+            const int rank = block_incl_scan(eq ? 1 : 0, wsum, &tot) - (eq ? 1 : 0);
+            const bool sel = gt || (eq && (uint32_t)(eq_seen + rank) < rem);
+            if (sel) atomicOr(bm + (i >> 5), 1u << (i & 31));
+            eq_seen += tot;
+        }
+    }
+    __syncthreads();
+    // write the selected entries in ascending order: each thread a contiguous run of bitmap words
+    const int64_t per = (nw + FIN_THREADS - 1) / FIN_THREADS;
+    const int64_t w0 = min(nw, (int64_t)tid * per), w1 = min(nw, w0 + per);
+    int cnt = 0;
+    for (int64_t w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+    int total;
+    int off = block_incl_scan(cnt, wsum, &total) - cnt;
+    for (int64_t w = w0; w < w1; ++w) {
+        uint32_t bits = bm[w];
+        while (bits != 0u && off < k) {
+            const int bit = __ffs(bits) - 1;
+            out[off++] = (int32_t)(w * 32 + bit);
+            bits &= bits - 1u;
+        }
+    }
+    for (int j = total + tid; j < k; j += FIN_THREADS) out[j] = -1;
 }
 
 }  // namespace
 
+// Workspace of the decode index step (256-byte aligned pieces): scores [B, T] fp32, then a region
+// zeroed at the start of every call (keymax [B], nkeymin [B], ncand [B], hist [B, 2048], bitmap
+// [B, ceil(T/32)]), then the candidates [B, 2048] (key, index).
+struct DecodeIndexLayout {
+    size_t scores, zero, zero_bytes, keymax, nkeymin, ncand, hist, bitmap, cand, total;
+};
+
+static DecodeIndexLayout decode_index_layout(int64_t B, int64_t T)
+{
+    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    DecodeIndexLayout L;
+    L.scores = 0;
+    L.zero = al((size_t)B * T * 4);
+    L.keymax = L.zero;
+    L.nkeymin = L.keymax + (size_t)B * 4;
+    L.ncand = L.nkeymin + (size_t)B * 4;
+    L.hist = al(L.ncand + (size_t)B * 4);
+    L.bitmap = L.hist + (size_t)B * HBINS * 4;
+    L.zero_bytes = al(L.bitmap + (size_t)B * ((T + 31) / 32) * 4) - L.zero;
+    L.cand = L.zero + L.zero_bytes;
+    L.total = L.cand + (size_t)B * CAND_CAP * 8;
+    return L;
+}
+
 size_t decode_index_workspace(int64_t B, int64_t T, int k)
 {
-    const int64_t nchunks = (T + SEL_CHUNK - 1) / SEL_CHUNK;
-    return (size_t)B * T * 4 + 2 * (size_t)B * nchunks * k * 4 + 1024;
+    (void)k;
+    return decode_index_layout(B, T).total + 1024;
 }
 
 bool decode_index_tc_supported(int64_t T, int HI, int dI, int k)
 {
-    const int64_t nchunks = (T + SEL_CHUNK - 1) / SEL_CHUNK;
     return (dI == 64 || dI == 128) && (HI == 16 || HI == 32 || HI == 64 || HI == 128) && T >= 1 && k >= 1 &&
-           k <= SEL_CHUNK && nchunks * k * 12 <= 200 * 1024 && T <= (1ll << 26);
+           T <= (1ll << 26);
 }
 
 // scores/candidates live in `ws` (decode_index_workspace bytes, 256-byte aligned)
@@ -458,11 +590,16 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
 {
     if (B == 0) return cudaSuccess;
     char *p8 = static_cast<char *>(ws);
-    float *scores = reinterpret_cast<float *>(p8);
-    const int64_t nchunks = (T + SEL_CHUNK - 1) / SEL_CHUNK;
-    const size_t sbytes = ((size_t)B * T * 4 + 255) & ~(size_t)255;
-    int32_t *cand_idx = reinterpret_cast<int32_t *>(p8 + sbytes);
-    uint32_t *cand_key = reinterpret_cast<uint32_t *>(p8 + sbytes + (size_t)B * nchunks * k * 4);
+    const DecodeIndexLayout L = decode_index_layout(B, T);
+    float *scores = reinterpret_cast<float *>(p8 + L.scores);
+    uint32_t *keymax = reinterpret_cast<uint32_t *>(p8 + L.keymax);
+    uint32_t *nkeymin = reinterpret_cast<uint32_t *>(p8 + L.nkeymin);
+    uint32_t *ncand = reinterpret_cast<uint32_t *>(p8 + L.ncand);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(p8 + L.hist);
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(p8 + L.bitmap);
+    uint2 *cand = reinterpret_cast<uint2 *>(p8 + L.cand);
+    cudaError_t e = cudaMemsetAsync(p8 + L.zero, 0, L.zero_bytes, stream);
+    if (e != cudaSuccess) return e;
 
     CUtensorMap tq, tk;
     if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)B * HI, dI, HI)) return cudaErrorInvalidValue;
@@ -470,6 +607,8 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     ScoreParams sp;
     sp.w = w;
     sp.scores = scores;
+    sp.keymax = keymax;
+    sp.nkeymin = nkeymin;
     sp.status = status;
     sp.T = T;
     sp.HI = HI;
@@ -480,7 +619,7 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     const size_t fixed = 1024 + 2 * (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
     sp.stages = (int)std::min<size_t>(MAX_STAGES, (227 * 1024 - fixed) / a_bytes);
     const size_t smem = fixed + (size_t)sp.stages * a_bytes;
-    cudaError_t e = cudaFuncSetAttribute(decode_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(decode_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     cudaGetDevice(&dev);
@@ -488,16 +627,15 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
     decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dim3 g2((unsigned)nchunks, (unsigned)B);
-    const size_t csmem = (size_t)SEL_CHUNK * 8;
-    e = cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)csmem);
-    if (e != cudaSuccess) return e;
-    topk_chunk_kernel<<<g2, SEL_THREADS, csmem, stream>>>(scores, T, k, cand_idx, cand_key);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const size_t msmem = (size_t)nchunks * k * 12;
-    e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    if (e != cudaSuccess) return e;
-    topk_merge_kernel<<<(unsigned)B, MERGE_THREADS, msmem, stream>>>(cand_idx, cand_key, T, (int)nchunks, k, idx);
+    if (T > k) {
+        const dim3 g2((unsigned)((T + TK_CHUNK - 1) / TK_CHUNK), (unsigned)B);
+        topk_hist_kernel<<<g2, TK_THREADS, 0, stream>>>(scores, T, keymax, nkeymin, hist);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        topk_collect_kernel<<<g2, TK_THREADS, 0, stream>>>(scores, T, k, keymax, nkeymin, hist, bitmap, ncand, cand);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    topk_final_kernel<<<(unsigned)B, FIN_THREADS, 0, stream>>>(scores, T, k, keymax, nkeymin, hist, bitmap, ncand, cand,
+                                                               idx);
     return cudaGetLastError();
 }
 

@@ -243,3 +243,44 @@ def test_decode_short_history():
     """P < W-1: window rows at negative positions are ignored; k > T pads with -1."""
     wl = WORKLOADS[3].with_(ctx=40, topk=16, W=128)
     _decode_check(wl, batch=2, seqs=[0, 1])
+
+
+def _decode_index_only(y, wl):
+    """Run csa_decode and return the selected indices (attention output unused)."""
+    P = wl.ctx - 1
+    kw = dict(C=y["C"]) if wl.cache == "bf16" else dict(c8=y["c8"], c8_scale=y["scale"], c_rope=y["rope"])
+    _, idx = csa.decode(y["q"], y["qI"], y["w"], y["kI"], y["win"], y["sinks"], P, wl.topk, wl.r, wl.theta_tok,
+                        wl.theta_cmp, **kw)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy()
+
+
+def test_decode_topk_all_scores_tied():
+    """Index weights of zero make every score +0: the top-k is the k smallest indices (ties go to the
+    smaller index), taken through the crowded-bin path since T far exceeds the candidate capacity."""
+    wl = WORKLOADS[3].with_(ctx=4 * 20000, topk=1024)
+    y = decode_inputs(wl, device=DEV, batch=2)
+    y["w"] = torch.zeros_like(y["w"])
+    idx = _decode_index_only(y, wl)
+    want = np.arange(wl.topk, dtype=np.int32)
+    for b in range(2):
+        assert np.array_equal(idx[b], want)
+
+
+@pytest.mark.parametrize("ctx,classes", [(4 * 8192, 5), (4 * 40000, 7)])
+def test_decode_topk_few_distinct_scores(ctx, classes):
+    """k^I rows repeat a few distinct vectors, so scores take `classes` values and the threshold value
+    is shared by many entries (directly ranked, or the crowded-bin fallback past its capacity): the
+    selection must equal the oracle's exactly, in ascending order."""
+    wl = WORKLOADS[3].with_(ctx=ctx, topk=1024)
+    y = decode_inputs(wl, device=DEV, batch=2)
+    kI = y["kI"]
+    base = kI[:, :classes].clone()
+    pattern = torch.arange(wl.T, device=kI.device) % classes
+    y["kI"] = base[:, pattern].contiguous()
+    idx = _decode_index_only(y, wl)
+    h = {k: v.cpu() for k, v in y.items()}
+    ridx, _ = oracle.decode_index_topk(h["qI"], h["w"], h["kI"], wl.topk)
+    for b in range(2):
+        assert np.array_equal(idx[b], np.asarray(ridx[b], np.int32)), b
+        assert np.all(np.diff(idx[b][idx[b] >= 0]) > 0)
