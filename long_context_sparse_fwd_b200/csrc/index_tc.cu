@@ -135,6 +135,300 @@ __device__ __forceinline__ void topk_warp(const float *sc, int n, int k, uint32_
     for (int i = written + lane; i < k; i += 32) out[i] = -1;
 }
 
+
+// Exact top-k of one query's scores by a pair of warps (64 threads, named barrier `bar`), ties to the
+// smaller index, indices written in ascending order. A histogram of the (up to) 10 key bits below
+// the highest bit where the query's keys differ gives the threshold bin; its entries are ranked
+// (key descending, index ascending) to find the last selected (key, index); one ordered pass then
+// writes every entry that beats or equals it. A threshold bin of more than 512 entries falls back to
+// the single-warp radix select. `scratch`: 4 KB (histogram, then the bin's entries) + 80 words.
+constexpr int PBINS = 1024;
+constexpr int PCAND = 512;
+
+__device__ __forceinline__ void pair_sync(int bar) { named_barrier_sync(bar, 64); }
+
+__device__ void topk_pair(const float *sc, int n, int k, uint32_t *scratch, int bar, int32_t *out)
+{
+    const int pt = threadIdx.x & 63, lane = threadIdx.x & 31, pw = pt >> 5;
+    uint32_t *hist = scratch;                                  // [PBINS]
+    uint2 *cand = reinterpret_cast<uint2 *>(scratch);          // [PCAND] after the threshold is known
+    uint32_t *vars = scratch + PBINS;                          // [16]
+    if (n <= k) {
+        for (int i = pt; i < k; i += 64) out[i] = i < n ? i : -1;
+        return;
+    }
+    // key range
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (int i = pt; i < n; i += 64) {
+        const uint32_t key = score_key(sc[i]);
+        lo = min(lo, key);
+        hi = max(hi, key);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    for (int i = pt; i < PBINS; i += 64) hist[i] = 0u;
+    if (lane == 0) {
+        vars[2 * pw] = lo;
+        vars[2 * pw + 1] = hi;
+    }
+    pair_sync(bar);
+    lo = min(vars[0], vars[2]);
+    hi = max(vars[1], vars[3]);
+    const uint32_t diff = lo ^ hi;
+    int shift = 0;
+    uint32_t dmask = 0u;
+    if (diff != 0u) {
+        const int top = 31 - __clz(diff);
+        shift = max(0, top - 9);
+        dmask = (2u << (top - shift)) - 1u;
+    }
+    for (int i = pt; i < n; i += 64) atomicAdd(&hist[(score_key(sc[i]) >> shift) & dmask], 1u);
+    pair_sync(bar);
+    // threshold bin: thread pt owns bins [16 pt, 16 pt + 16); suffix sums over the owners
+    uint32_t own = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) own += hist[16 * pt + j];
+    uint32_t after = own;   // owners above this one, within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_down_sync(0xffffffffu, after, o);
+        if (lane + o < 32) after += x;
+    }
+    after -= own;
+    if (lane == 0) vars[4 + pw] = after + own;   // this warp's total
+    pair_sync(bar);
+    if (pw == 0) after += vars[5];               // warp 1 owns the higher bins
+    {
+        uint32_t run = after;
+        for (int j = 15; j >= 0; --j) {
+            const uint32_t c = hist[16 * pt + j];
+            if (run < (uint32_t)k && run + c >= (uint32_t)k) {
+                vars[6] = (uint32_t)(16 * pt + j);   // d*
+                vars[7] = run;                       // entries in higher bins
+            }
+            run += c;
+        }
+    }
+    if (pt == 0) vars[8] = 0u;   // candidate count
+    pair_sync(bar);
+    const uint32_t dstar = vars[6], above = vars[7], remaining = (uint32_t)k - above;
+    // entries of the threshold bin
+    for (int base = pw * 32; base < n; base += 64) {
+        const int i = base + lane;
+        uint32_t key = 0u;
+        bool isc = false;
+        if (i < n) {
+            key = score_key(sc[i]);
+            isc = ((key >> shift) & dmask) == dstar;
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, isc);
+        if (m != 0u) {
+            uint32_t pos0 = 0;
+            if (lane == 0) pos0 = atomicAdd(&vars[8], (uint32_t)__popc(m));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            const uint32_t pos = pos0 + __popc(m & ((1u << lane) - 1u));
+            if (isc && pos < (uint32_t)PCAND) cand[pos] = make_uint2(key, (uint32_t)i);
+        }
+    }
+    pair_sync(bar);
+    const uint32_t nc = vars[8];
+    if (nc > (uint32_t)PCAND) {   // crowded bin: the single-warp radix select (exact)
+        if (pw == 0) topk_warp(sc, n, k, scratch, out);
+        pair_sync(bar);            // the scratch is free again for the pair's next query
+        return;
+    }
+    // the remaining-th best entry of the bin: rank = number of entries that beat it
+    for (uint32_t c = pt; c < nc; c += 64) {
+        const uint2 me = cand[c];
+        uint32_t rank = 0;
+        for (uint32_t j = 0; j < nc; ++j) {
+            const uint2 o = cand[j];
+            rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        }
+        if (rank == remaining - 1u) {
+            vars[9] = me.x;
+            vars[10] = me.y;
+        }
+    }
+    pair_sync(bar);
+    const uint32_t tkey = vars[9], tidx = vars[10];
+    // ordered output: warp 0 takes entries [0, half), warp 1 [half, n); warp 1 starts after warp 0's count
+    const int half = (((n + 1) >> 1) + 31) & ~31;
+    const int b0 = pw == 0 ? 0 : min(half, n), b1 = pw == 0 ? min(half, n) : n;
+    const unsigned lt = (1u << lane) - 1u;
+    int cnt = 0;
+    for (int base = b0; base < b1; base += 32) {
+        const int i = base + lane;
+        bool sel = false;
+        if (i < b1) {
+            const uint32_t key = score_key(sc[i]);
+            sel = key > tkey || (key == tkey && (uint32_t)i <= tidx);
+        }
+        cnt += __popc(__ballot_sync(0xffffffffu, sel));
+    }
+    if (pw == 0 && lane == 0) vars[11] = (uint32_t)cnt;
+    pair_sync(bar);
+    int written = pw == 0 ? 0 : (int)vars[11];
+    for (int base = b0; base < b1; base += 32) {
+        const int i = base + lane;
+        bool sel = false;
+        if (i < b1) {
+            const uint32_t key = score_key(sc[i]);
+            sel = key > tkey || (key == tkey && (uint32_t)i <= tidx);
+        }
+        const unsigned sb = __ballot_sync(0xffffffffu, sel);
+        if (sel) out[written + __popc(sb & lt)] = i;
+        written += __popc(sb);
+    }
+    pair_sync(bar);
+}
+
+// As topk_pair for n <= 2048 with the keys held in registers: thread pt of the pair holds entries
+// pt + 64 j (j < 32), so every pass is an unrolled loop over registers, and warp pw holds the
+// 32-entry groups g = 2 j + pw in index order for the ordered output.
+__device__ void topk_pair_reg(const float *sc, int n, int k, uint32_t *scratch, int bar, int32_t *out)
+{
+    constexpr int KPT = 32;
+    const int pt = threadIdx.x & 63, lane = threadIdx.x & 31, pw = pt >> 5;
+    uint32_t *hist = scratch;                                  // [PBINS]
+    uint2 *cand = reinterpret_cast<uint2 *>(scratch);          // [PCAND] after the threshold is known
+    uint32_t *vars = scratch + PBINS;                          // [16]
+    uint32_t key[KPT];
+    uint32_t lo = 0xffffffffu, hi = 0u;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int i = pt + 64 * j;
+        key[j] = i < n ? score_key(sc[i]) : 0u;
+        if (i < n) {
+            lo = min(lo, key[j]);
+            hi = max(hi, key[j]);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    for (int i = pt; i < PBINS; i += 64) hist[i] = 0u;
+    if (lane == 0) {
+        vars[2 * pw] = lo;
+        vars[2 * pw + 1] = hi;
+    }
+    pair_sync(bar);
+    lo = min(vars[0], vars[2]);
+    hi = max(vars[1], vars[3]);
+    const uint32_t diff = lo ^ hi;
+    int shift = 0;
+    uint32_t dmask = 0u;
+    if (diff != 0u) {
+        const int top = 31 - __clz(diff);
+        shift = max(0, top - 9);
+        dmask = (2u << (top - shift)) - 1u;
+    }
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+        if (pt + 64 * j < n) atomicAdd(&hist[(key[j] >> shift) & dmask], 1u);
+    pair_sync(bar);
+    uint32_t hv[16], own = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        hv[j] = hist[16 * pt + j];
+        own += hv[j];
+    }
+    uint32_t after = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_down_sync(0xffffffffu, after, o);
+        if (lane + o < 32) after += x;
+    }
+    after -= own;
+    if (lane == 0) vars[4 + pw] = after + own;
+    pair_sync(bar);
+    if (pw == 0) after += vars[5];
+    {
+        uint32_t run = after;
+#pragma unroll
+        for (int j = 15; j >= 0; --j) {
+            if (run < (uint32_t)k && run + hv[j] >= (uint32_t)k) {
+                vars[6] = (uint32_t)(16 * pt + j);
+                vars[7] = run;
+            }
+            run += hv[j];
+        }
+    }
+    if (pt == 0) vars[8] = 0u;
+    pair_sync(bar);
+    const uint32_t dstar = vars[6], remaining = (uint32_t)k - vars[7];
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int i = pt + 64 * j;
+        const bool isc = i < n && ((key[j] >> shift) & dmask) == dstar;
+        const unsigned m = __ballot_sync(0xffffffffu, isc);
+        if (m != 0u) {
+            uint32_t pos0 = 0;
+            if (lane == 0) pos0 = atomicAdd(&vars[8], (uint32_t)__popc(m));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            const uint32_t pos = pos0 + __popc(m & ((1u << lane) - 1u));
+            if (isc && pos < (uint32_t)PCAND) cand[pos] = make_uint2(key[j], (uint32_t)i);
+        }
+    }
+    pair_sync(bar);
+    const uint32_t nc = vars[8];
+    if (nc > (uint32_t)PCAND) {   // crowded bin: the single-warp radix select (exact)
+        if (pw == 0) topk_warp(sc, n, k, scratch, out);
+        pair_sync(bar);
+        return;
+    }
+    for (uint32_t c = pt; c < nc; c += 64) {
+        const uint2 me = cand[c];
+        uint32_t rank = 0;
+        for (uint32_t j = 0; j < nc; ++j) {
+            const uint2 o = cand[j];
+            rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        }
+        if (rank == remaining - 1u) {
+            vars[9] = me.x;
+            vars[10] = me.y;
+        }
+    }
+    pair_sync(bar);
+    const uint32_t tkey = vars[9], tidx = vars[10];
+    // ordered output: group counts of this warp's groups (g = 2 j + pw), exclusive scan over all 64
+    uint32_t *gcnt = scratch + PBINS + 16;   // [64] (scratch tail, past vars)
+    unsigned selm[KPT];
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int i = pt + 64 * j;
+        const bool sel = i < n && (key[j] > tkey || (key[j] == tkey && (uint32_t)i <= tidx));
+        selm[j] = __ballot_sync(0xffffffffu, sel);
+        if (lane == 0) gcnt[2 * j + pw] = (uint32_t)__popc(selm[j]);
+    }
+    pair_sync(bar);
+    if (pw == 0) {   // exclusive scan of the 64 group counts (two per lane)
+        const uint32_t c0 = gcnt[2 * lane], c1 = gcnt[2 * lane + 1];
+        uint32_t incl = c0 + c1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += x;
+        }
+        const uint32_t excl = incl - (c0 + c1);
+        gcnt[2 * lane] = excl;
+        gcnt[2 * lane + 1] = excl + c0;
+    }
+    pair_sync(bar);
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+        const int i = pt + 64 * j;
+        if ((selm[j] >> lane) & 1u) out[gcnt[2 * j + pw] + __popc(selm[j] & lt)] = i;
+    }
+    pair_sync(bar);
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      IdxParams p)
@@ -148,8 +442,8 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     uint8_t *sA = sB + b_bytes;
     float *scores = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [Q][T_cap]
     float *sw = scores + (size_t)p.Q * p.T_cap;                                  // [BN]
-    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                      // [8][256]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 8 * 256);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                      // [4 pairs][PBINS + 80]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 4 * (PBINS + 80));
     uint64_t *full = bars;                   // [stages]
     uint64_t *empty = bars + 8;              // [stages]
     uint64_t *tfull = bars + 16;             // [2]
@@ -295,13 +589,19 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             mbar_arrive(&tempty[buf]);
         }
         named_barrier_sync(1, EPI_THREADS);
-        // ---------------- exact top-k, one query per warp ----------------
-        if (!*abort) {
-            for (int q = warp - 2; q < p.Q; q += 8) {
+        // ---------------- exact top-k, one query per pair of warps ----------------
+        {
+            const int pair = (warp - 2) >> 1;
+            for (int q = pair; q < p.Q; q += 4) {
                 const int64_t t = t0 + q;
                 if (t >= p.S) continue;
                 const int n = (int)visible_entries(t, p.m, p.T);
-                topk_warp(scores + (size_t)q * p.T_cap, n, p.k, hist + (warp - 2) * 256, p.idx + t * (int64_t)p.k);
+                if (n > p.k && n <= 2048)
+                    topk_pair_reg(scores + (size_t)q * p.T_cap, n, p.k, hist + pair * (PBINS + 80), 2 + pair,
+                                  p.idx + t * (int64_t)p.k);
+                else
+                    topk_pair(scores + (size_t)q * p.T_cap, n, p.k, hist + pair * (PBINS + 80), 2 + pair,
+                              p.idx + t * (int64_t)p.k);
             }
         }
     }
@@ -384,7 +684,7 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     p.Q = BN / HI;
     p.T_cap = (int)((T + BM - 1) / BM * BM);
     const size_t a_bytes = (size_t)(dI / 64) * BM * 128, b_bytes = (size_t)(dI / 64) * BN * 128;
-    const size_t fixed = 1024 + b_bytes + (size_t)p.Q * p.T_cap * 4 + BN * 4 + 8 * 256 * 4 + 256;
+    const size_t fixed = 1024 + b_bytes + (size_t)p.Q * p.T_cap * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + 256;
     const size_t budget = 227 * 1024;
     p.stages = (int)std::min<size_t>(4, (budget - fixed) / a_bytes);
     if (p.stages < 2) return cudaErrorInvalidValue;

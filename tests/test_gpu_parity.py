@@ -108,6 +108,36 @@ def test_index_topk_all_zero_ties():
         assert idx[t][:n].tolist() == list(range(n)) and (idx[t][n:] == -1).all()
 
 
+
+def test_index_topk_tc_all_zero_ties():
+    """Tensor-core indexer with weights 0: every score is exactly 0, so each query keeps its k smallest
+    visible indices; vis(t) from below k to far above the ranked-bin capacity (the crowded-bin path)."""
+    wl = WORKLOADS[1].with_(S=3000, HI=64, dI=128, topk=64)
+    g, x = gen(prefill_inputs, wl, need_q=False)
+    g["w"] = torch.zeros_like(g["w"])
+    idx = csa.index_topk(g["qI"], g["kI"], g["w"], wl.m, wl.topk).cpu().numpy()
+    for t in [0, 3, 100, 255, 256, 260, 1000, 2047, 2048, 2100, 2999]:
+        n = min(wl.topk, (t + 1) // wl.m)
+        assert idx[t][:n].tolist() == list(range(n)) and (idx[t][n:] == -1).all(), t
+
+
+@pytest.mark.parametrize("classes,k", [(6, 128), (2, 300)])
+def test_index_topk_tc_few_distinct_scores(classes, k):
+    """Tensor-core indexer with k^I rows repeating `classes` vectors: each query's scores take only
+    that many values, so its threshold value is shared by many entries (ranked directly, or the
+    crowded-bin path past 512). The selection must equal the oracle's exactly."""
+    wl = WORKLOADS[1].with_(S=4100, HI=64, dI=128, topk=k)
+    g, x = gen(prefill_inputs, wl, need_q=False)
+    pattern = torch.arange(wl.T) % classes
+    kI = x["kI"][:classes][pattern].contiguous()
+    x["kI"] = kI
+    g["kI"] = kI.to(DEV)
+    idx = csa.index_topk(g["qI"], g["kI"], g["w"], wl.m, wl.topk).cpu().numpy()
+    rows = sample_rows(wl.S, 48, 5, must=[0, 7, 1023, 2047, 2048, 4095, 4099])
+    ridx, _ = oracle.index_topk(x["qI"], x["kI"], x["w"], wl.m, wl.topk, rows=rows)
+    for i, t in enumerate(rows):
+        assert np.array_equal(idx[t], np.asarray(ridx[i], np.int32)), t
+
 # ---- 3. CSA attention (oracle indices fed to the GPU) -----------------------------------------------------
 
 @pytest.mark.parametrize("wid,S,nrows", [(0, 1024, None), (0, 1030, None), (0, 5, None), (1, 8192, 48)])
