@@ -32,7 +32,7 @@ if ROOT not in sys.path:
 
 from workloads import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
 
-WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4}
+WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4, "hca_decode1m": 5}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -88,9 +88,11 @@ def attention_bytes(wl):
 
 
 def decode_bytes(wl, B):
-    """k^I stream + selected entries + window rows + q + o per step."""
+    """k^I stream + selected entries + window rows + q + o per step (HCA decode: every entry, no indexer)."""
     T, D, r = wl.T, wl.D, wl.r
     ent = (D - r) + 4 + 2 * r if wl.cache == "fp8" else 2 * D
+    if wl.kind == "hca_decode":
+        return float(B * (T * ent + wl.W * D * 2 + wl.H * D * 2 + wl.H * D * 4))
     per_seq = T * wl.dI * 2 + wl.topk * ent + wl.W * D * 2 + wl.H * D * 2 + wl.H * D * 4 + wl.HI * (wl.dI * 2 + 4)
     return float(B * per_seq)
 
@@ -156,14 +158,18 @@ class Step:
     def __init__(self, name, wl, csa, dev):
         self.name, self.wl, self.csa, self.dev = name, wl, csa, dev
         self.stream = torch.cuda.current_stream()
-        if wl.kind == "csa_decode":
+        if wl.kind in ("csa_decode", "hca_decode"):
             self.B = wl.B
             self.x = decode_inputs(wl, device=dev)
             self.P = wl.ctx - 1
             self.o = torch.empty(self.B, wl.H, wl.D, dtype=torch.float32, device=dev)
-            self.idx = torch.empty(self.B, wl.topk, dtype=torch.int32, device=dev)
-            self.ws = torch.empty(csa.workspace_size("decode", B=self.B, T=wl.T, k=wl.topk), dtype=torch.uint8,
-                                  device=dev)
+            if wl.kind == "csa_decode":
+                self.idx = torch.empty(self.B, wl.topk, dtype=torch.int32, device=dev)
+                self.ws = torch.empty(csa.workspace_size("decode", B=self.B, T=wl.T, k=wl.topk), dtype=torch.uint8,
+                                      device=dev)
+            else:
+                self.ws = torch.empty(csa.workspace_size("hca_decode", B=self.B, T=wl.T, W=wl.W), dtype=torch.uint8,
+                                      device=dev)
             self.phases = ["decode"]
             self.units = self.B
         else:
@@ -186,17 +192,23 @@ class Step:
         # library kernels per step on the tensor-core paths these workloads take:
         # prefill: compress_entries + rotate_rows, fused index/top-k (CSA), attention;
         # decode: index scan, chunk top-k, merge, split attention, combine
-        return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 5}[self.wl.kind]
+        # decode: index scan, three top-k kernels, split attention, combine (plus one memset); HCA
+        # decode: split attention and combine
+        return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 6, "hca_decode": 2}[self.wl.kind]
 
     def run(self, timed: bool):
         wl, x, csa = self.wl, self.x, self.csa
         ev = self.events
         if timed:
             ev[0].record(self.stream)
-        if wl.kind == "csa_decode":
+        if wl.kind in ("csa_decode", "hca_decode"):
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
-            csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], self.P, wl.topk, wl.r, wl.theta_tok,
-                       wl.theta_cmp, o=self.o, idx=self.idx, workspace=self.ws, **kw)
+            if wl.kind == "csa_decode":
+                csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], self.P, wl.topk, wl.r,
+                           wl.theta_tok, wl.theta_cmp, o=self.o, idx=self.idx, workspace=self.ws, **kw)
+            else:
+                csa.hca_decode(x["q"], x["win"], x["sinks"], self.P, wl.r, wl.theta_tok, wl.theta_cmp, o=self.o,
+                               workspace=self.ws, **kw)
             if timed:
                 ev[1].record(self.stream)
             return
@@ -244,6 +256,10 @@ def e2e_run(step, steps, warmup):
         elif wl.kind == "hca_prefill":
             o, _, _ = csa.hca_forward(x["q"], x["kv"], x["gate"], x["pos_bias"], x["sinks"], wl.m, wl.L, wl.W, wl.r,
                                       wl.theta_tok, wl.theta_cmp, out=(step.o, step.C, step.kv_rot), workspace=step.ws)
+        elif wl.kind == "hca_decode":
+            kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
+            o = csa.hca_decode(x["q"], x["win"], x["sinks"], step.P, wl.r, wl.theta_tok, wl.theta_cmp, o=step.o,
+                               workspace=step.ws, **kw)
         else:
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
             o, _ = csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], step.P, wl.topk, wl.r,
@@ -279,7 +295,7 @@ class OracleStep:
     def __init__(self, wl, target_s=4.0):
         import oracle
         self.oracle, self.wl = oracle, wl
-        if wl.kind == "csa_decode":
+        if wl.kind in ("csa_decode", "hca_decode"):
             self.x = decode_inputs(wl, device="cpu", batch=1)
             self.P = wl.ctx - 1
         else:
@@ -309,8 +325,11 @@ class OracleStep:
         wl, o, x = self.wl, self.oracle, self.x
         self.calls += 1
         t0 = time.perf_counter()
-        if wl.kind == "csa_decode":
-            ridx, _ = o.decode_index_topk(x["qI"], x["w"], x["kI"], wl.topk)
+        if wl.kind in ("csa_decode", "hca_decode"):
+            if wl.kind == "csa_decode":
+                ridx, _ = o.decode_index_topk(x["qI"], x["w"], x["kI"], wl.topk)
+            else:
+                ridx = np.arange(wl.T, dtype=np.int32)[None]
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
             o.decode_attend(x["q"], x["win"], ridx, x["sinks"], self.P, wl.r, wl.theta_tok, wl.theta_cmp, **kw)
             return 1, time.perf_counter() - t0
@@ -322,17 +341,19 @@ class OracleStep:
     def sample_desc(self):
         if self.wl.kind == "csa_decode":
             return f"1 of {self.wl.B} sequences per step (full index scan over T={self.wl.T} + attention)"
+        if self.wl.kind == "hca_decode":
+            return f"1 of {self.wl.B} sequences per step (attention over all T={self.wl.T} entries + window)"
         return (f"{self.n} random query rows of S={self.wl.S} per step (index + top-k + attention per row) "
                 f"plus the full pooling amortised per token")
 
 
 def unit_name(wl):
-    return "queries/s" if wl.kind == "csa_decode" else "tokens/s"
+    return "queries/s" if wl.kind in ("csa_decode", "hca_decode") else "tokens/s"
 
 
 def metric_name(wl):
     return {"csa_prefill": "csa_prefill_tokens_per_s", "hca_prefill": "hca_prefill_tokens_per_s",
-            "csa_decode": "csa_decode_queries_per_s"}[wl.kind]
+            "csa_decode": "csa_decode_queries_per_s", "hca_decode": "hca_decode_queries_per_s"}[wl.kind]
 
 
 def config_of(wl, n_gpus):
@@ -342,6 +363,9 @@ def config_of(wl, n_gpus):
     if wl.kind == "csa_decode":
         c.update({"B": wl.B, "ctx": wl.ctx, "T": wl.T, "topk": wl.topk, "index": f"{wl.HI}x{wl.dI}",
                   "cache": wl.cache})
+        del c["S"]
+    elif wl.kind == "hca_decode":
+        c.update({"B": wl.B, "ctx": wl.ctx, "T": wl.T, "cache": wl.cache})
         del c["S"]
     elif wl.kind == "csa_prefill":
         c.update({"topk": wl.topk, "index": f"{wl.HI}x{wl.dI}", "T": wl.T})
@@ -456,9 +480,10 @@ def main():
     mean_phase = phase_ms.mean(0)
     dom = int(np.argmax(mean_phase))
     dom_name = step.phases[dom]
-    if wl.kind == "csa_decode":
+    if wl.kind in ("csa_decode", "hca_decode"):
         alg = decode_bytes(wl, step.B)
-        roof = {"bound": "hbm", "kernel": "csa_decode (index scan + top-k + attention)",
+        roof = {"bound": "hbm", "kernel": "csa_decode (index scan + top-k + attention)" if wl.kind == "csa_decode"
+                else "hca_decode (split attention + combine)",
                 "achieved": alg / (mean_phase[dom] / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     elif dom_name == "attend":
         alg = csa_attention_flops(wl)

@@ -65,7 +65,8 @@ typedef enum csa_op {
     CSA_OP_ATTEND = 2,        /* csa_attend and hca_attend */
     CSA_OP_CSA_FORWARD = 3,
     CSA_OP_HCA_FORWARD = 4,
-    CSA_OP_DECODE = 5
+    CSA_OP_DECODE = 5,
+    CSA_OP_HCA_DECODE = 6     /* hca_decode (B, T, W) */
 } csa_op;
 
 typedef struct csa_dims {
@@ -177,9 +178,9 @@ CSA_API csa_status csa_decode(const void *q, const void *qI, const float *w, con
  * library holds that array until the process exits. Arguments and results are those of
  * csa_decode, without workspace and workspace_bytes. It allocates nothing.
  *   - Returns CSA_ERR_WORKSPACE, launching nothing, when the problem needs more scratch than the
- *     array holds: the index scores and candidates plus the selected indices, about
- *     B*T*4 + 2*B*ceil(T/8192)*k*4 + B*k*4 bytes (e.g. B=64 sequences of T=32768 entries, or
- *     B=8 of T=262144, fit). Whatever the array has left is used for attention splits.
+ *     array holds: the index scores, the top-k histograms, bitmap and candidates, and the selected
+ *     indices, about B*(4*T + T/8 + 24 KB + 4*k) bytes (e.g. B=64 sequences of T=32768 entries,
+ *     or B=8 of T=262144, fit). Whatever the array has left is used for attention splits.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
  *     that device current; make that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the last call's contents: calls that
@@ -194,6 +195,30 @@ CSA_API csa_status csa_decode_noalloc(const void *q, const void *qI, const float
                       int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W, int32_t rope_dim,
                       int64_t P, double theta_tok, double theta_cmp, float softmax_scale,
                       int32_t *idx_out, float *o, void *stream);
+
+/* ---- 8. HCA decode, and the sliding-window-only layer --------------------------------------------
+ * [HF-V4 "Hybrid attention", HCA (dense attention over all pooled entries); "Attention mask layout",
+ * HCA layer and sliding-window layer; "Cache layers"].
+ * hca_decode: one new query per sequence at position P; keys = every one of the T cached entries
+ * (all visible at decode) plus the window rows win[b] (positions P-W+1 .. P), one softmax with the
+ * sink; no indexer. Entry caches, window, q, sinks and o as in csa_decode (bf16 C, or the FP8
+ * triplet when C == NULL). T = 0 is the decode step of a sliding-window-only layer (window rows and
+ * sink only; C may be NULL).
+ * csa_workspace_size(CSA_OP_HCA_DECODE) is the recommended workspace (split-K partials over the
+ * B*(T+W) keys); any workspace down to 256 bytes is accepted and uses fewer splits. */
+CSA_API csa_status hca_decode(const void *q, const void *C, const uint8_t *c8, const float *c8_scale,
+                      const void *c_rope, const void *win, const float *sinks, int32_t B, int32_t H,
+                      int32_t D, int64_t T, int32_t W, int32_t rope_dim, int64_t P, double theta_tok,
+                      double theta_cmp, float softmax_scale, float *o, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/* swa_attend: prefill of a sliding-window-only layer. For query t, head h: keys kv_rot[j] for
+ * j in [t-W+1, t] (post-RoPE at theta_tok), one softmax with exp(sinks[h]), K = V, the output rope
+ * slice rotated back by -t with theta_tok; no compressed entries. Arguments as hca_attend without
+ * C, T, m and theta_cmp. Workspace: 256 bytes (the status word). */
+CSA_API csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int64_t S, int32_t H,
+                      int32_t D, int32_t W, int32_t rope_dim, double theta_tok, float softmax_scale,
+                      float *o, void *workspace, size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

@@ -15,14 +15,14 @@ import torch
 
 __all__ = [
     "CSAError", "lib", "library_path", "compress", "index_topk", "attend", "hca_attend", "csa_forward",
-    "hca_forward", "decode", "workspace_size", "get_device_status", "OP",
+    "hca_forward", "decode", "hca_decode", "swa_attend", "workspace_size", "get_device_status", "OP",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libcsa.so")
 _lib = None
 
-OP = {"index_topk": 1, "attend": 2, "csa_forward": 3, "hca_forward": 4, "decode": 5}
+OP = {"index_topk": 1, "attend": 2, "csa_forward": 3, "hca_forward": 4, "decode": 5, "hca_decode": 6}
 _STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
            4: "CSA_ERR_TIMEOUT", 5: "CSA_ERR_WORKSPACE"}
 
@@ -68,6 +68,8 @@ def lib():
                                   SZ, P]),
             "csa_decode": (I32, [P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, I32, I64,
                                  F64, F64, F32, P, P, P, SZ, P]),
+            "hca_decode": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I64, F64, F64, F32, P, P, SZ, P]),
+            "swa_attend": (I32, [P, P, P, I64, I32, I32, I32, I32, F64, F32, P, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -264,3 +266,47 @@ def decode(q, qI, w, kI, win, sinks, P: int, k: int, rope_dim: int, theta_tok: f
                                           int(P), float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(idx),
                                           _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
     return o, idx
+
+
+def hca_decode(q, win, sinks, P: int, rope_dim: int, theta_tok: float, theta_cmp: float, C=None, c8=None,
+               c8_scale=None, c_rope=None, T: Optional[int] = None, softmax_scale: float = 0.0, o=None,
+               workspace=None, stream=None) -> torch.Tensor:
+    """HCA decode: every cached entry (bf16 C [B,T,D], or the FP8 triplet) plus the window rows
+    win [B,W,D] and the sink. With no entry cache (T = 0) it is the sliding-window-only decode.
+    Returns o [B,H,D] fp32."""
+    B, H, D = q.shape
+    W = win.shape[1]
+    _dev(q, torch.bfloat16, "q")
+    _dev(win, torch.bfloat16, "win", (B, W, D))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    if C is not None:
+        T = C.shape[1]
+        _dev(C, torch.bfloat16, "C", (B, T, D))
+    elif c8 is not None:
+        T = c8.shape[1]
+        _dev(c8, torch.uint8, "c8", (B, T, D - rope_dim))
+        _dev(c8_scale, torch.float32, "c8_scale", (B, T))
+        _dev(c_rope, torch.bfloat16, "c_rope", (B, T, rope_dim))
+    else:
+        T = 0
+    o = torch.empty(B, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (B, H, D))
+    ws = _workspace("hca_decode", q.device, workspace, B=B, T=T, W=W)
+    _check("hca_decode", lib().hca_decode(_ptr(q), _ptr(C), _ptr(c8), _ptr(c8_scale), _ptr(c_rope), _ptr(win),
+                                          _ptr(sinks), B, H, D, T, W, rope_dim, int(P), float(theta_tok),
+                                          float(theta_cmp), float(softmax_scale), _ptr(o), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
+    return o
+
+
+def swa_attend(q, kv_rot, sinks, W: int, rope_dim: int, theta_tok: float, softmax_scale: float = 0.0, o=None,
+               workspace=None, stream=None) -> torch.Tensor:
+    """Sliding-window-only layer prefill: window rows kv_rot [S,D] and the sink. Returns o [S,H,D] fp32."""
+    S, H, D = q.shape
+    _dev(q, torch.bfloat16, "q")
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
+    ws = _workspace("attend", q.device, workspace)
+    _check("swa_attend", lib().swa_attend(_ptr(q), _ptr(kv_rot), _ptr(sinks), S, H, D, W, rope_dim, float(theta_tok),
+                                          float(softmax_scale), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o

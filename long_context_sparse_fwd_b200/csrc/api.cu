@@ -126,6 +126,14 @@ int decode_splits_preferred(int64_t B)
     return (int)std::min<int64_t>(8, std::max<int64_t>(1, 148 / std::max<int64_t>(B, 1)));
 }
 
+// HCA decode: up to 16 splits per sequence (about one wave of CTAs), never more than its key blocks
+int hca_decode_splits_preferred(int64_t B, int64_t T, int32_t W)
+{
+    const int64_t blocks = (T + 63) / 64 + ((int64_t)std::max(W, 0) + 63) / 64;
+    const int64_t by_sm = std::max<int64_t>(1, 148 / std::max<int64_t>(B, 1));
+    return (int)std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(16, by_sm), std::max<int64_t>(blocks, 1)));
+}
+
 }  // namespace
 
 namespace csa {
@@ -191,6 +199,8 @@ size_t csa_workspace_size(csa_op op, const csa_dims *d)
     case CSA_OP_DECODE:
         return decode_workspace_min(d->B, d->T, d->k) +
                align256(attend_tc_decode_partials(d->B, decode_splits_preferred(d->B)));
+    case CSA_OP_HCA_DECODE:
+        return kStatusBytes + align256(attend_tc_decode_partials(d->B, hca_decode_splits_preferred(d->B, d->T, d->W)));
     }
     return 0;
 }
@@ -394,6 +404,67 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
         return from_cuda(launch_attend_tc_decode(a, nsplit, reinterpret_cast<float *>(base + used), st));
     }
     return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status hca_decode(const void *q, const void *C, const uint8_t *c8, const float *c8_scale, const void *c_rope,
+                      const void *win, const float *sinks, int32_t B, int32_t H, int32_t D, int64_t T, int32_t W,
+                      int32_t rope_dim, int64_t P, double theta_tok, double theta_cmp, float softmax_scale, float *o,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && W >= 0 && P >= 0);
+    CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
+    CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_ARG(B == 0 || (q != nullptr && sinks != nullptr && o != nullptr));
+    CSA_CHECK_ARG(B == 0 || W == 0 || win != nullptr);
+    const bool fp8 = C == nullptr;
+    CSA_CHECK_ARG(B == 0 || T == 0 || !fp8 || (c8 != nullptr && c8_scale != nullptr && c_rope != nullptr));
+    CSA_CHECK_SUP(D == 64 || D == 128 || D == 256 || D == 512);
+    CSA_CHECK_SUP(rope_dim % 8 == 0);
+    CSA_CHECK_ARG(aligned16(q) && aligned16(C) && aligned16(c8) && aligned16(c_rope) && aligned16(win) && aligned16(o));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    AttnArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = static_cast<const uint16_t *>(q);
+    a.win = static_cast<const uint16_t *>(win);
+    a.C = static_cast<const uint16_t *>(C);
+    a.c8 = c8;
+    a.c8_scale = c8_scale;
+    a.c_rope = static_cast<const uint16_t *>(c_rope);
+    a.idx = nullptr;   // every cached entry
+    a.sinks = sinks;
+    a.o = o;
+    a.status = static_cast<int32_t *>(workspace);
+    a.R = B;
+    a.T = T;
+    a.P = P;
+    a.H = H;
+    a.D = D;
+    a.k = 0;
+    a.W = W;
+    a.r = rope_dim;
+    a.m = 1;
+    a.decode = 1;
+    a.scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / sqrt((double)D));
+    a.log2_theta_tok = rope_dim > 0 ? log2(theta_tok) : 0.0;
+    a.log2_theta_cmp = rope_dim > 0 ? log2(theta_cmp) : 0.0;
+    if (attend_tc_supported(H, D, rope_dim, 0)) {
+        int nsplit = hca_decode_splits_preferred(B, T, W);
+        while (nsplit > 1 && kStatusBytes + align256(attend_tc_decode_partials(B, nsplit)) > workspace_bytes) --nsplit;
+        return from_cuda(launch_attend_tc_decode(a, nsplit,
+                                                 reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes), st));
+    }
+    return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int64_t S, int32_t H, int32_t D, int32_t W,
+                      int32_t rope_dim, double theta_tok, float softmax_scale, float *o, void *workspace,
+                      size_t workspace_bytes, void *stream)
+{
+    // the HCA attention with no compressed entries (both rope branches at theta_tok)
+    return hca_attend(q, nullptr, kv_rot, sinks, S, H, D, 0, W, rope_dim, 1, theta_tok, theta_tok, softmax_scale, o,
+                      workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

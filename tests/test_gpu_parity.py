@@ -314,3 +314,69 @@ def test_decode_topk_few_distinct_scores(ctx, classes):
     for b in range(2):
         assert np.array_equal(idx[b], np.asarray(ridx[b], np.int32)), b
         assert np.all(np.diff(idx[b][idx[b] >= 0]) > 0)
+
+
+# ---- 7. HCA decode and the sliding-window-only layer ----------------------------------------------------
+
+# HCA at 1M context: m' = 128 pools 1,048,576 tokens into T = 8192 entries, all attended densely
+HCA_DEC = WORKLOADS[3].with_(name="hca_decode_b8_ctx1m", m=128, L=128, ctx=1 << 20, B=8, topk=0, seed=5)
+
+
+def _hca_decode_check(wl, batch, seqs, entries=True):
+    y = decode_inputs(wl, device=DEV, batch=batch)
+    P = wl.ctx - 1
+    if not entries:
+        kw, T = {}, 0
+    elif wl.cache == "bf16":
+        kw, T = dict(C=y["C"]), wl.T
+    else:
+        kw, T = dict(c8=y["c8"], c8_scale=y["scale"], c_rope=y["rope"]), wl.T
+    o = csa.hca_decode(y["q"], y["win"], y["sinks"], P, wl.r, wl.theta_tok, wl.theta_cmp, **kw)
+    torch.cuda.synchronize()
+    seqs = np.asarray(seqs, np.int64)
+    h = {k: v[seqs].cpu() if v.dim() > 1 else v.cpu() for k, v in y.items()}
+    idx = np.tile(np.arange(T, dtype=np.int32), (len(seqs), 1))
+    if not entries:
+        kwr = dict(C=h["C"][:, :0]) if "C" in h else dict(c8=h["c8"][:, :0], c8_scale=h["scale"][:, :0],
+                                                          c_rope=h["rope"][:, :0])
+    elif wl.cache == "bf16":
+        kwr = dict(C=h["C"])
+    else:
+        kwr = dict(c8=h["c8"], c8_scale=h["scale"], c_rope=h["rope"])
+    ref = oracle.decode_attend(h["q"], h["win"], idx, h["sinks"], P, wl.r, wl.theta_tok, wl.theta_cmp, **kwr)
+    check_close(o.cpu()[seqs], ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
+def test_hca_decode_bf16_ctx1m():
+    _hca_decode_check(HCA_DEC, batch=None, seqs=[0, 5])
+
+
+def test_hca_decode_fp8_ctx1m():
+    _hca_decode_check(HCA_DEC.with_(cache="fp8"), batch=4, seqs=[1, 3])
+
+
+def test_hca_decode_short_history():
+    """Three pooled entries and a window reaching below position 0."""
+    _hca_decode_check(HCA_DEC.with_(ctx=128 * 3 + 50), batch=3, seqs=[0, 1, 2])
+
+
+def test_swa_decode():
+    """The sliding-window-only layer's decode: hca_decode with no entry cache."""
+    _hca_decode_check(HCA_DEC.with_(ctx=5000), batch=4, seqs=[0, 3], entries=False)
+
+
+@pytest.mark.parametrize("wid,S,nrows", [(0, 1030, None), (1, 4096, 64)])
+def test_swa_attend(wid, S, nrows):
+    """Sliding-window-only prefill (no compressed entries): the general path (tiny heads) and the
+    tensor-core path (64 heads x 512), against the oracle's attention with an empty entry set."""
+    wl = WORKLOADS[wid].with_(S=S)
+    g, x = gen(prefill_inputs, wl, need_index=False)
+    a = attend_inputs(wl, device=DEV)
+    o = csa.swa_attend(g["q"], a["kv_rot"], g["sinks"], wl.W, wl.r, wl.theta_tok)
+    torch.cuda.synchronize()
+    rows = None if nrows is None else sample_rows(S, nrows, 11, must=[0, 1, 127, 128, S - 1])
+    ah = host(a)
+    ref = oracle.attend(x["q"], ah["C"][:0], ah["kv_rot"], None, x["sinks"], 1, wl.W, wl.r, wl.theta_tok,
+                        wl.theta_tok, rows=rows)
+    got = o.cpu() if rows is None else o.cpu()[rows]
+    check_close(got, ref, O_MAX_ABS, O_MEAN_ABS, what="o")

@@ -467,6 +467,25 @@ def test_decode_equals_last_prefill_row(cache):
     np.testing.assert_allclose(dec, pre, atol=1e-13)
 
 
+
+def test_hca_decode_equals_last_prefill_row():
+    """HCA decode reading: decode at P over every cached entry plus the window equals row P of the HCA
+    prefill (all entries w < floor((P+1)/m) visible); with no entries it equals the window-only prefill."""
+    wl = WORKLOADS[0].with_(S=96, H=3, D=32, r=8, m=16, L=16, W=10, theta_cmp=160000.0)
+    x = prefill_inputs(wl, need_index=False)
+    C, kvr = oracle.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok)
+    Cb, kvrb = torch.tensor(C).to(torch.bfloat16), torch.tensor(kvr).to(torch.bfloat16)
+    P, T = wl.S - 1, wl.T
+    assert T == 6
+    pre = oracle.attend(x["q"], Cb, kvrb, None, x["sinks"], wl.m, wl.W, wl.r, wl.theta_tok, wl.theta_cmp, rows=[P])
+    dec = oracle.decode_attend(x["q"][P:P + 1], kvrb[P - wl.W + 1: P + 1][None], np.arange(T, dtype=np.int32)[None],
+                               x["sinks"], P, wl.r, wl.theta_tok, wl.theta_cmp, C=Cb[None])
+    np.testing.assert_allclose(dec, pre, atol=1e-13)
+    pre0 = oracle.attend(x["q"], Cb[:0], kvrb, None, x["sinks"], 1, wl.W, wl.r, wl.theta_tok, wl.theta_tok, rows=[P])
+    dec0 = oracle.decode_attend(x["q"][P:P + 1], kvrb[P - wl.W + 1: P + 1][None], np.zeros((1, 0), np.int32),
+                                x["sinks"], P, wl.r, wl.theta_tok, wl.theta_tok, C=Cb[None, :0])
+    np.testing.assert_allclose(dec0, pre0, atol=1e-13)
+
 # ---- P-k>=vis: CSA with a covering top-k equals HCA-style dense over visible entries -------------------
 
 def test_csa_full_topk_equals_dense_entries():

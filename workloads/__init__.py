@@ -28,7 +28,7 @@ __all__ = ["Workload", "WORKLOADS", "prefill_inputs", "attend_inputs", "decode_i
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "csa_prefill" | "hca_prefill" | "csa_decode"
+    kind: str                 # "csa_prefill" | "hca_prefill" | "csa_decode" | "hca_decode"
     S: int = 0                # prefill tokens
     H: int = 64
     D: int = 512
@@ -50,7 +50,7 @@ class Workload:
 
     @property
     def T(self) -> int:
-        return (self.ctx if self.kind == "csa_decode" else self.S) // self.m
+        return (self.ctx if self.kind in ("csa_decode", "hca_decode") else self.S) // self.m
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -66,6 +66,8 @@ WORKLOADS: Dict[int, Workload] = {
                 topk=0, seed=2),
     3: Workload("csa_decode_b64_ctx128k", "csa_decode", B=64, ctx=131072, topk=1024, seed=3),
     4: Workload("csa_decode_b8_ctx1m_fp8", "csa_decode", B=8, ctx=1048576, topk=512, cache="fp8", seed=4),
+    # beyond the five: HCA decode at 1M context (m' = 128: 8192 pooled entries per sequence, all attended)
+    5: Workload("hca_decode_b8_ctx1m", "hca_decode", B=8, ctx=1048576, m=128, L=128, topk=0, seed=5),
 }
 
 
