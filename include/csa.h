@@ -220,6 +220,28 @@ CSA_API csa_status swa_attend(const void *q, const void *kv_rot, const float *si
                       int32_t D, int32_t W, int32_t rope_dim, double theta_tok, float softmax_scale,
                       float *o, void *workspace, size_t workspace_bytes, void *stream);
 
+/* ---- 9. the compressor's decode step --------------------------------------------------------------
+ * [HF-V4 "Hybrid attention" (CSA m-token pooling over overlapping windows, HCA over m'-token
+ * windows), "Cache layers" (the compressed buffers carry the tokens of the window still open);
+ * digest: softmax gate with a learned position bias, FP8 entries with BF16 rope channels].
+ * One new token per sequence at position P (the same P for every sequence; positions start at 0):
+ *   x_new [B, D] bf16 (un-rotated kv, or per-token index keys with rope_dim = 0), g_new [B, D] bf16
+ *   gate logits, pos_bias [L] fp32. state_x, state_g [B, L, D] bf16 hold the last L tokens
+ *   (slot = position mod L); the caller zero-fills nothing: a slot is read only after it was written.
+ * The token is written into the state; when (P+1) is a multiple of m, entry w = (P+1)/m - 1 pools
+ * positions [(w+1)m - L, (w+1)m) exactly as csa_compress, is rotated at w*m with theta_cmp, and is
+ * written to the entry cache: C [B, Tcap, D] bf16, or (C == NULL) the FP8 triplet of csa_decode:
+ * c8 [B, Tcap, D - rope_dim] E4M3 codes (8-byte aligned), c8_scale [B, Tcap] = amax/448 over the
+ * non-rope channels (1 when they are all zero), c_rope [B, Tcap, rope_dim] bf16. An entry index
+ * w >= Tcap is CSA_ERR_INVALID_ARG. With W > 0 the token's row rotated at P with theta_tok is written
+ * to win [B, W, D] at slot (W-1-P) mod W, which csa_decode / hca_decode read as the window rows of P.
+ * Requires D % 8 == 0, D <= 512. No workspace; stream-ordered. */
+CSA_API csa_status csa_compress_append(const void *x_new, const void *g_new, const float *pos_bias,
+                      void *state_x, void *state_g, int32_t B, int32_t D, int32_t m, int32_t L,
+                      int32_t rope_dim, int64_t P, double theta_cmp, double theta_tok, void *C,
+                      uint8_t *c8, float *c8_scale, void *c_rope, int64_t Tcap, void *win, int32_t W,
+                      void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,7 +15,8 @@ import torch
 
 __all__ = [
     "CSAError", "lib", "library_path", "compress", "index_topk", "attend", "hca_attend", "csa_forward",
-    "hca_forward", "decode", "hca_decode", "swa_attend", "workspace_size", "get_device_status", "OP",
+    "hca_forward", "decode", "hca_decode", "swa_attend", "compress_append", "workspace_size", "get_device_status",
+    "OP",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +71,8 @@ def lib():
                                  F64, F64, F32, P, P, P, SZ, P]),
             "hca_decode": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I64, F64, F64, F32, P, P, SZ, P]),
             "swa_attend": (I32, [P, P, P, I64, I32, I32, I32, I32, F64, F32, P, P, SZ, P]),
+            "csa_compress_append": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I64, F64, F64, P, P, P, P, I64, P,
+                                          I32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -310,3 +313,35 @@ def swa_attend(q, kv_rot, sinks, W: int, rope_dim: int, theta_tok: float, softma
     _check("swa_attend", lib().swa_attend(_ptr(q), _ptr(kv_rot), _ptr(sinks), S, H, D, W, rope_dim, float(theta_tok),
                                           float(softmax_scale), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
     return o
+
+
+def compress_append(x_new, g_new, pos_bias, state_x, state_g, P: int, m: int, rope_dim: int, theta_cmp: float,
+                    theta_tok: float, C=None, c8=None, c8_scale=None, c_rope=None, win=None, stream=None) -> None:
+    """The compressor's decode step for the token at position P (the same for every sequence): writes
+    it into the state rings [B,L,D], emits entry (P+1)/m - 1 into the bf16 cache C [B,Tcap,D] (or the
+    FP8 triplet) when (P+1) % m == 0, and writes its rotated window row into win [B,W,D] at slot
+    (W-1-P) mod W."""
+    B, D = x_new.shape
+    L = state_x.shape[1]
+    _dev(x_new, torch.bfloat16, "x_new")
+    _dev(g_new, torch.bfloat16, "g_new", (B, D))
+    _dev(pos_bias, torch.float32, "pos_bias", (L,))
+    _dev(state_x, torch.bfloat16, "state_x", (B, L, D))
+    _dev(state_g, torch.bfloat16, "state_g", (B, L, D))
+    if C is not None:
+        Tcap = C.shape[1]
+        _dev(C, torch.bfloat16, "C", (B, Tcap, D))
+    else:
+        Tcap = c8.shape[1]
+        _dev(c8, torch.uint8, "c8", (B, Tcap, D - rope_dim))
+        _dev(c8_scale, torch.float32, "c8_scale", (B, Tcap))
+        if rope_dim > 0:
+            _dev(c_rope, torch.bfloat16, "c_rope", (B, Tcap, rope_dim))
+    W = 0
+    if win is not None:
+        W = win.shape[1]
+        _dev(win, torch.bfloat16, "win", (B, W, D))
+    _check("csa_compress_append", lib().csa_compress_append(
+        _ptr(x_new), _ptr(g_new), _ptr(pos_bias), _ptr(state_x), _ptr(state_g), B, D, m, L, rope_dim, int(P),
+        float(theta_cmp), float(theta_tok), _ptr(C), _ptr(c8), _ptr(c8_scale), _ptr(c_rope), Tcap, _ptr(win), W,
+        _stream(stream)))

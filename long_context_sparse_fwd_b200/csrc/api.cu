@@ -467,4 +467,50 @@ csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int
                       workspace, workspace_bytes, stream);
 }
 
+csa_status csa_compress_append(const void *x_new, const void *g_new, const float *pos_bias, void *state_x,
+                               void *state_g, int32_t B, int32_t D, int32_t m, int32_t L, int32_t rope_dim, int64_t P,
+                               double theta_cmp, double theta_tok, void *C, uint8_t *c8, float *c8_scale, void *c_rope,
+                               int64_t Tcap, void *win, int32_t W, void *stream)
+{
+    CSA_CHECK_ARG(B >= 0 && D > 0 && m >= 1 && L >= m && P >= 0 && Tcap >= 0 && W >= 0);
+    CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
+    CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_SUP(D % 8 == 0 && D <= 512 && rope_dim % 8 == 0);
+    CSA_CHECK_ARG(B == 0 || (x_new != nullptr && g_new != nullptr && pos_bias != nullptr && state_x != nullptr &&
+                             state_g != nullptr));
+    CSA_CHECK_ARG(W == 0 || B == 0 || win != nullptr);
+    const bool emits = (P + 1) % m == 0;
+    const bool fp8 = C == nullptr;
+    // an entry closing at P must fit the caller's cache, in one of the two formats
+    CSA_CHECK_ARG(!emits || B == 0 || ((P + 1) / m - 1 < Tcap &&
+                                       (!fp8 || (c8 != nullptr && c8_scale != nullptr &&
+                                                 (rope_dim == 0 || c_rope != nullptr)))));
+    CSA_CHECK_ARG(aligned16(x_new) && aligned16(g_new) && aligned16(state_x) && aligned16(state_g) && aligned16(C) &&
+                  aligned16(c_rope) && aligned16(win));
+    CSA_CHECK_ARG(fp8 == false || c8 == nullptr || ((reinterpret_cast<uintptr_t>(c8) & 7u) == 0 && (D - rope_dim) % 8 == 0));
+    AppendArgs a;
+    memset(&a, 0, sizeof a);
+    a.x_new = static_cast<const uint16_t *>(x_new);
+    a.g_new = static_cast<const uint16_t *>(g_new);
+    a.bias = pos_bias;
+    a.state_x = static_cast<uint16_t *>(state_x);
+    a.state_g = static_cast<uint16_t *>(state_g);
+    a.C = static_cast<uint16_t *>(C);
+    a.c8 = c8;
+    a.c8_scale = c8_scale;
+    a.c_rope = static_cast<uint16_t *>(c_rope);
+    a.win = W > 0 ? static_cast<uint16_t *>(win) : nullptr;
+    a.P = P;
+    a.Tcap = Tcap;
+    a.B = B;
+    a.D = D;
+    a.m = m;
+    a.L = L;
+    a.r = rope_dim;
+    a.W = W;
+    a.log2_theta_cmp = rope_dim > 0 ? log2(theta_cmp) : 0.0;
+    a.log2_theta_tok = rope_dim > 0 ? log2(theta_tok) : 0.0;
+    return from_cuda(launch_compress_append(a, as_stream(stream)));
+}
+
 }  // extern "C"

@@ -46,6 +46,22 @@ bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uin
 // 2-D fp32 tensor map, box [box_rows, 32], 128-byte swizzle
 bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
+// append.cu: the compressor's decode step (one token per sequence; emits an entry when a window closes)
+struct AppendArgs {
+    const uint16_t *x_new, *g_new;   // [B, D] bf16 token at position P and its gate logits
+    const float *bias;               // [L] position bias of the pooling window
+    uint16_t *state_x, *state_g;     // [B, L, D] bf16 rings of the last L tokens (slot = position mod L)
+    uint16_t *C;                     // [B, Tcap, D] bf16 entry cache, or null for the FP8 cache:
+    uint8_t *c8;                     //   [B, Tcap, D - r] E4M3 codes
+    float *c8_scale;                 //   [B, Tcap]
+    uint16_t *c_rope;                //   [B, Tcap, r] bf16 rope channels
+    uint16_t *win;                   // [B, W, D] window ring (slot (W-1-P) mod W), or null
+    int64_t P, Tcap;
+    int B, D, m, L, r, W;
+    double log2_theta_cmp, log2_theta_tok;
+};
+cudaError_t launch_compress_append(const AppendArgs &a, cudaStream_t stream);
+
 // api.cu: smallest workspace csa_decode accepts (no attention split partials)
 size_t decode_workspace_min(int64_t B, int64_t T, int32_t k);
 

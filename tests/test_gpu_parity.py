@@ -380,3 +380,84 @@ def test_swa_attend(wid, S, nrows):
                         wl.theta_tok, rows=rows)
     got = o.cpu() if rows is None else o.cpu()[rows]
     check_close(got, ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
+# ---- 8. the compressor's decode step ------------------------------------------------------------------
+
+def _append_history(wl, B, S, fp8=False):
+    """B independent histories of S tokens appended one position at a time; returns host inputs and
+    the device caches."""
+    xs = [prefill_inputs(wl.with_(S=S, seed=wl.seed + 100 * b), need_index=False, need_q=False) for b in range(B)]
+    kv = torch.stack([x["kv"] for x in xs])
+    gate = torch.stack([x["gate"] for x in xs])
+    bias = xs[0]["pos_bias"]
+    T, D, r, L, W = S // wl.m, wl.D, wl.r, wl.L, wl.W
+    kv_d, gate_d, bias_d = kv.to(DEV), gate.to(DEV), bias.to(DEV)
+    state_x = torch.empty(B, L, D, dtype=torch.bfloat16, device=DEV)
+    state_g = torch.empty(B, L, D, dtype=torch.bfloat16, device=DEV)
+    win = torch.zeros(B, W, D, dtype=torch.bfloat16, device=DEV)
+    cache = {}
+    if fp8:
+        cache = dict(c8=torch.zeros(B, T, D - r, dtype=torch.uint8, device=DEV),
+                     c8_scale=torch.zeros(B, T, dtype=torch.float32, device=DEV),
+                     c_rope=torch.zeros(B, T, r, dtype=torch.bfloat16, device=DEV))
+    else:
+        cache = dict(C=torch.zeros(B, T, D, dtype=torch.bfloat16, device=DEV))
+    for P in range(S):
+        csa.compress_append(kv_d[:, P].contiguous(), gate_d[:, P].contiguous(), bias_d, state_x, state_g, P, wl.m,
+                            r, wl.theta_cmp, wl.theta_tok, win=win, **cache)
+    torch.cuda.synchronize()
+    refs = [oracle.compress(kv[b], gate[b], bias, wl.m, wl.L, r, wl.theta_cmp, wl.theta_tok) for b in range(B)]
+    return kv, gate, bias, win, cache, refs
+
+
+@pytest.mark.parametrize("m,L,S,B", [(4, 8, 70, 3), (128, 128, 300, 2)])
+def test_compress_append_matches_prefill_compressor(m, L, S, B):
+    """Token-by-token decode steps leave in the cache exactly the prefill compressor's entries over the
+    same history (CSA overlapping windows, HCA non-overlapping), and in the window ring the rows of the
+    last W positions rotated at their own positions."""
+    wl = WORKLOADS[1].with_(m=m, L=L)
+    kv, gate, bias, win, cache, refs = _append_history(wl, B, S)
+    T, W = S // m, wl.W
+    for b in range(B):
+        Cr, kvr = refs[b]
+        check_close(cache["C"][b].float().cpu(), Cr[:T], C_MAX_ABS, what="C")
+        bf16_rel_close(cache["C"][b].float().cpu(), Cr[:T], "C")
+        for pos in range(max(0, S - W), S):
+            bf16_rel_close(win[b, (W - 1 - pos) % W].float().cpu(), kvr[pos], "window row")
+
+
+def test_compress_append_fp8_cache():
+    """FP8 entry cache: rope channels in bf16, the rest E4M3 codes x (amax / 448) of the entry."""
+    wl = WORKLOADS[1].with_(m=4, L=8)
+    S, B, D, r = 41, 2, wl.D, wl.r
+    _, _, _, _, cache, refs = _append_history(wl, B, S, fp8=True)
+    T = S // wl.m
+    for b in range(B):
+        Cr = refs[b][0][:T]
+        nope, rope = Cr[:, : D - r], Cr[:, D - r:]
+        scale = cache["c8_scale"][b].double().cpu().numpy()
+        np.testing.assert_allclose(scale, np.abs(nope).max(1) / 448.0, rtol=1e-3)
+        codes = cache["c8"][b].cpu().view(torch.float8_e4m3fn).double().numpy()
+        deq = codes * scale[:, None]
+        assert (np.abs(deq - nope) <= 0.0625 * np.abs(nope) + 0.002 * scale[:, None] + 1e-4).all()
+        bf16_rel_close(cache["c_rope"][b].float().cpu(), rope, "rope channels")
+
+
+def test_compress_append_feeds_decode():
+    """The caches written by the decode step serve the decode attention directly: hca_decode on the
+    entry cache and the window ring equals the oracle's decode on the prefill compressor's entries and
+    the window rows in position order (the ring order does not matter to the attention)."""
+    wl = WORKLOADS[1].with_(m=4, L=8)
+    S, B = 300, 2
+    _, _, _, win, cache, refs = _append_history(wl, B, S)
+    T, W, P = S // wl.m, wl.W, S - 1
+    q = torch.randn(B, wl.H, wl.D, generator=torch.Generator().manual_seed(7)).mul_(wl.q_std).to(torch.bfloat16)
+    sinks = torch.randn(wl.H, generator=torch.Generator().manual_seed(8))
+    o = csa.hca_decode(q.to(DEV), win, sinks.to(DEV), P, wl.r, wl.theta_tok, wl.theta_cmp, C=cache["C"])
+    torch.cuda.synchronize()
+    Cb = torch.stack([torch.tensor(refs[b][0][:T]) for b in range(B)]).to(torch.bfloat16)
+    winb = torch.stack([torch.tensor(refs[b][1][P - W + 1:P + 1]) for b in range(B)]).to(torch.bfloat16)
+    ref = oracle.decode_attend(q, winb, np.tile(np.arange(T, dtype=np.int32), (B, 1)), sinks, P, wl.r, wl.theta_tok,
+                               wl.theta_cmp, C=Cb)
+    check_close(o.cpu(), ref, O_MAX_ABS, O_MEAN_ABS, what="o")
