@@ -32,7 +32,8 @@ if ROOT not in sys.path:
 
 from workloads import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
 
-WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4, "hca_decode1m": 5}
+WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4, "hca_decode1m": 5,
+                "append128k": 6}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -85,6 +86,14 @@ def index_flops(wl):
 def attention_bytes(wl):
     """Each tensor once: q in, o out (fp32), entries and window rows once."""
     return wl.S * wl.H * wl.D * 2 + wl.S * wl.H * wl.D * 4 + wl.T * wl.D * 2 + wl.S * wl.D * 2
+
+
+def append_bytes(wl, B):
+    """m decode-step appends per sequence: read the token and gate, write both into the state and the
+    rotated row into the window ring; the closing append reads the L-token window and writes the entry."""
+    D = wl.D
+    per_seq = wl.m * (4 * D + 4 * D + 2 * D) + wl.L * 4 * D + 2 * D
+    return float(B * per_seq)
 
 
 def decode_bytes(wl, B):
@@ -158,7 +167,23 @@ class Step:
     def __init__(self, name, wl, csa, dev):
         self.name, self.wl, self.csa, self.dev = name, wl, csa, dev
         self.stream = torch.cuda.current_stream()
-        if wl.kind in ("csa_decode", "hca_decode"):
+        if wl.kind == "compress_append":
+            # m consecutive decode-step appends (positions P0 .. P0+m-1, the last closes an entry) for B
+            # sequences whose histories already fill the pooling state and the window ring
+            self.B, D, L, W = wl.B, wl.D, wl.L, wl.W
+            g = torch.Generator(device=dev)
+            g.manual_seed(wl.seed)
+            self.x = {"kv": torch.randn(wl.m, self.B, D, generator=g, device=dev).to(torch.bfloat16),   # [position, seq, D]
+                      "gate": torch.randn(wl.m, self.B, D, generator=g, device=dev).to(torch.bfloat16),
+                      "pos_bias": torch.randn(L, generator=g, device=dev) * 0.02}
+            self.state_x = torch.randn(self.B, L, D, generator=g, device=dev).to(torch.bfloat16)
+            self.state_g = torch.randn(self.B, L, D, generator=g, device=dev).to(torch.bfloat16)
+            self.C = torch.empty(self.B, wl.T, D, dtype=torch.bfloat16, device=dev)
+            self.win = torch.empty(self.B, W, D, dtype=torch.bfloat16, device=dev)
+            self.P0 = wl.ctx - wl.m
+            self.phases = ["append"]
+            self.units = self.B * wl.m
+        elif wl.kind in ("csa_decode", "hca_decode"):
             self.B = wl.B
             self.x = decode_inputs(wl, device=dev)
             self.P = wl.ctx - 1
@@ -194,13 +219,21 @@ class Step:
         # decode: index scan, chunk top-k, merge, split attention, combine
         # decode: index scan, three top-k kernels, split attention, combine (plus one memset); HCA
         # decode: split attention and combine
-        return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 6, "hca_decode": 2}[self.wl.kind]
+        return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 6, "hca_decode": 2,
+                "compress_append": self.wl.m}[self.wl.kind]
 
     def run(self, timed: bool):
         wl, x, csa = self.wl, self.x, self.csa
         ev = self.events
         if timed:
             ev[0].record(self.stream)
+        if wl.kind == "compress_append":
+            for i in range(wl.m):
+                csa.compress_append(x["kv"][i], x["gate"][i], x["pos_bias"], self.state_x, self.state_g,
+                                    self.P0 + i, wl.m, wl.r, wl.theta_cmp, wl.theta_tok, C=self.C, win=self.win)
+            if timed:
+                ev[1].record(self.stream)
+            return
         if wl.kind in ("csa_decode", "hca_decode"):
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
             if wl.kind == "csa_decode":
@@ -240,7 +273,9 @@ def e2e_run(step, steps, warmup):
     csa, wl, dev = step.csa, step.wl, step.dev
     host = {k: v.cpu().pin_memory() for k, v in step.x.items()}
     devbuf = {k: torch.empty_like(v) for k, v in step.x.items()}
-    o_host = torch.empty(step.o.shape, dtype=step.o.dtype).pin_memory()
+    out_shape = (step.B, wl.D) if wl.kind == "compress_append" else step.o.shape
+    out_dtype = torch.bfloat16 if wl.kind == "compress_append" else step.o.dtype
+    o_host = torch.empty(out_shape, dtype=out_dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = o_host.numel() * o_host.element_size()
     s = torch.cuda.current_stream()
@@ -249,7 +284,12 @@ def e2e_run(step, steps, warmup):
         for k in host:
             devbuf[k].copy_(host[k], non_blocking=True)
         x = devbuf
-        if wl.kind == "csa_prefill":
+        if wl.kind == "compress_append":
+            for i in range(wl.m):
+                csa.compress_append(x["kv"][i], x["gate"][i], x["pos_bias"], step.state_x, step.state_g,
+                                    step.P0 + i, wl.m, wl.r, wl.theta_cmp, wl.theta_tok, C=step.C, win=step.win)
+            o = step.C[:, (step.P0 + wl.m) // wl.m - 1]   # the entry the last append closed
+        elif wl.kind == "csa_prefill":
             o, _, _, _ = csa.csa_forward(x["q"], x["kv"], x["gate"], x["pos_bias"], x["qI"], x["kI"], x["w"],
                                          x["sinks"], wl.m, wl.L, wl.topk, wl.W, wl.r, wl.theta_tok, wl.theta_cmp,
                                          out=(step.o, step.C, step.kv_rot, step.idx), workspace=step.ws)
@@ -295,7 +335,12 @@ class OracleStep:
     def __init__(self, wl, target_s=4.0):
         import oracle
         self.oracle, self.wl = oracle, wl
-        if wl.kind in ("csa_decode", "hca_decode"):
+        if wl.kind == "compress_append":
+            g = torch.Generator().manual_seed(wl.seed)
+            self.x = {"kv": torch.randn(wl.L, wl.D, generator=g).to(torch.bfloat16),
+                      "gate": torch.randn(wl.L, wl.D, generator=g).to(torch.bfloat16),
+                      "pos_bias": torch.randn(wl.L, generator=g) * 0.02}
+        elif wl.kind in ("csa_decode", "hca_decode"):
             self.x = decode_inputs(wl, device="cpu", batch=1)
             self.P = wl.ctx - 1
         else:
@@ -325,6 +370,9 @@ class OracleStep:
         wl, o, x = self.wl, self.oracle, self.x
         self.calls += 1
         t0 = time.perf_counter()
+        if wl.kind == "compress_append":   # the entries of the last L tokens of one sequence (m appends' work)
+            o.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok)
+            return wl.m, time.perf_counter() - t0
         if wl.kind in ("csa_decode", "hca_decode"):
             if wl.kind == "csa_decode":
                 ridx, _ = o.decode_index_topk(x["qI"], x["w"], x["kI"], wl.topk)
@@ -341,6 +389,8 @@ class OracleStep:
     def sample_desc(self):
         if self.wl.kind == "csa_decode":
             return f"1 of {self.wl.B} sequences per step (full index scan over T={self.wl.T} + attention)"
+        if self.wl.kind == "compress_append":
+            return f"the pooling of the last L={self.wl.L} tokens of 1 of {self.wl.B} sequences per step"
         if self.wl.kind == "hca_decode":
             return f"1 of {self.wl.B} sequences per step (attention over all T={self.wl.T} entries + window)"
         return (f"{self.n} random query rows of S={self.wl.S} per step (index + top-k + attention per row) "
@@ -353,7 +403,8 @@ def unit_name(wl):
 
 def metric_name(wl):
     return {"csa_prefill": "csa_prefill_tokens_per_s", "hca_prefill": "hca_prefill_tokens_per_s",
-            "csa_decode": "csa_decode_queries_per_s", "hca_decode": "hca_decode_queries_per_s"}[wl.kind]
+            "csa_decode": "csa_decode_queries_per_s", "hca_decode": "hca_decode_queries_per_s",
+            "compress_append": "csa_append_tokens_per_s"}[wl.kind]
 
 
 def config_of(wl, n_gpus):
@@ -366,6 +417,9 @@ def config_of(wl, n_gpus):
         del c["S"]
     elif wl.kind == "hca_decode":
         c.update({"B": wl.B, "ctx": wl.ctx, "T": wl.T, "cache": wl.cache})
+        del c["S"]
+    elif wl.kind == "compress_append":
+        c.update({"B": wl.B, "ctx": wl.ctx, "appends_per_step": wl.m})
         del c["S"]
     elif wl.kind == "csa_prefill":
         c.update({"topk": wl.topk, "index": f"{wl.HI}x{wl.dI}", "T": wl.T})
@@ -480,7 +534,11 @@ def main():
     mean_phase = phase_ms.mean(0)
     dom = int(np.argmax(mean_phase))
     dom_name = step.phases[dom]
-    if wl.kind in ("csa_decode", "hca_decode"):
+    if wl.kind == "compress_append":
+        alg = append_bytes(wl, step.B)
+        roof = {"bound": "hbm", "kernel": "compress_append (m launches, latency-bound)",
+                "achieved": alg / (mean_phase[dom] / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    elif wl.kind in ("csa_decode", "hca_decode"):
         alg = decode_bytes(wl, step.B)
         roof = {"bound": "hbm", "kernel": "csa_decode (index scan + top-k + attention)" if wl.kind == "csa_decode"
                 else "hca_decode (split attention + combine)",

@@ -28,7 +28,7 @@ __all__ = ["Workload", "WORKLOADS", "prefill_inputs", "attend_inputs", "decode_i
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "csa_prefill" | "hca_prefill" | "csa_decode" | "hca_decode"
+    kind: str                 # "csa_prefill" | "hca_prefill" | "csa_decode" | "hca_decode" | "compress_append"
     S: int = 0                # prefill tokens
     H: int = 64
     D: int = 512
@@ -50,7 +50,7 @@ class Workload:
 
     @property
     def T(self) -> int:
-        return (self.ctx if self.kind in ("csa_decode", "hca_decode") else self.S) // self.m
+        return (self.ctx if self.kind in ("csa_decode", "hca_decode", "compress_append") else self.S) // self.m
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -68,6 +68,8 @@ WORKLOADS: Dict[int, Workload] = {
     4: Workload("csa_decode_b8_ctx1m_fp8", "csa_decode", B=8, ctx=1048576, topk=512, cache="fp8", seed=4),
     # beyond the five: HCA decode at 1M context (m' = 128: 8192 pooled entries per sequence, all attended)
     5: Workload("hca_decode_b8_ctx1m", "hca_decode", B=8, ctx=1048576, m=128, L=128, topk=0, seed=5),
+    # the CSA compressor's decode step for 64 sequences at 128K context (m = 4 appends close one entry)
+    6: Workload("csa_append_b64_ctx128k", "compress_append", B=64, ctx=131072, m=4, L=8, topk=0, seed=6),
 }
 
 
