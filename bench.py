@@ -30,10 +30,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, decode_inputs, prefill_inputs  # noqa: E402
+from workloads import WORKLOADS, decode_inputs, prefill_inputs, proj_inputs  # noqa: E402
 
 WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4, "hca_decode1m": 5,
-                "append128k": 6}
+                "append128k": 6, "out_proj": 7}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -86,6 +86,12 @@ def index_flops(wl):
 def attention_bytes(wl):
     """Each tensor once: q in, o out (fp32), entries and window rows once."""
     return wl.S * wl.H * wl.D * 2 + wl.S * wl.H * wl.D * 4 + wl.T * wl.D * 2 + wl.S * wl.D * 2
+
+
+def proj_flops(wl):
+    """Two GEMMs per token: G groups of (H/G)*D -> R, then G*R -> hidden."""
+    K = wl.H // wl.o_groups * wl.D
+    return 2.0 * wl.S * (wl.o_groups * K * wl.o_rank + wl.o_groups * wl.o_rank * wl.hidden)
 
 
 def append_bytes(wl, B):
@@ -167,7 +173,14 @@ class Step:
     def __init__(self, name, wl, csa, dev):
         self.name, self.wl, self.csa, self.dev = name, wl, csa, dev
         self.stream = torch.cuda.current_stream()
-        if wl.kind == "compress_append":
+        if wl.kind == "out_proj":
+            self.x = proj_inputs(wl, device=dev)
+            self.z = torch.empty(wl.S, wl.o_groups * wl.o_rank, dtype=torch.bfloat16, device=dev)
+            self.o = torch.empty(wl.S, wl.hidden, dtype=torch.bfloat16, device=dev)
+            self.ws = torch.empty(csa.workspace_size("out_proj"), dtype=torch.uint8, device=dev)
+            self.phases = ["out_proj"]
+            self.units = wl.S
+        elif wl.kind == "compress_append":
             # m consecutive decode-step appends (positions P0 .. P0+m-1, the last closes an entry) for B
             # sequences whose histories already fill the pooling state and the window ring
             self.B, D, L, W = wl.B, wl.D, wl.L, wl.W
@@ -220,13 +233,18 @@ class Step:
         # decode: index scan, three top-k kernels, split attention, combine (plus one memset); HCA
         # decode: split attention and combine
         return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 6, "hca_decode": 2,
-                "compress_append": self.wl.m}[self.wl.kind]
+                "compress_append": self.wl.m, "out_proj": 2}[self.wl.kind]
 
     def run(self, timed: bool):
         wl, x, csa = self.wl, self.x, self.csa
         ev = self.events
         if timed:
             ev[0].record(self.stream)
+        if wl.kind == "out_proj":
+            csa.out_proj(x["o"], x["wa"], x["wb"], z=self.z, out=self.o, workspace=self.ws)
+            if timed:
+                ev[1].record(self.stream)
+            return
         if wl.kind == "compress_append":
             for i in range(wl.m):
                 csa.compress_append(x["kv"][i], x["gate"][i], x["pos_bias"], self.state_x, self.state_g,
@@ -284,7 +302,9 @@ def e2e_run(step, steps, warmup):
         for k in host:
             devbuf[k].copy_(host[k], non_blocking=True)
         x = devbuf
-        if wl.kind == "compress_append":
+        if wl.kind == "out_proj":
+            _, o = csa.out_proj(x["o"], x["wa"], x["wb"], z=step.z, out=step.o, workspace=step.ws)
+        elif wl.kind == "compress_append":
             for i in range(wl.m):
                 csa.compress_append(x["kv"][i], x["gate"][i], x["pos_bias"], step.state_x, step.state_g,
                                     step.P0 + i, wl.m, wl.r, wl.theta_cmp, wl.theta_tok, C=step.C, win=step.win)
@@ -335,7 +355,10 @@ class OracleStep:
     def __init__(self, wl, target_s=4.0):
         import oracle
         self.oracle, self.wl = oracle, wl
-        if wl.kind == "compress_append":
+        if wl.kind == "out_proj":
+            self.x = proj_inputs(wl, device="cpu")
+            self.n = 64
+        elif wl.kind == "compress_append":
             g = torch.Generator().manual_seed(wl.seed)
             self.x = {"kv": torch.randn(wl.L, wl.D, generator=g).to(torch.bfloat16),
                       "gate": torch.randn(wl.L, wl.D, generator=g).to(torch.bfloat16),
@@ -370,6 +393,10 @@ class OracleStep:
         wl, o, x = self.wl, self.oracle, self.x
         self.calls += 1
         t0 = time.perf_counter()
+        if wl.kind == "out_proj":   # a sample of token rows (rows are independent)
+            rows = oracle_sample_rows(wl, self.n, seed=self.calls)
+            o.out_proj(x["o"][rows], x["wa"], x["wb"])
+            return self.n, time.perf_counter() - t0
         if wl.kind == "compress_append":   # the entries of the last L tokens of one sequence (m appends' work)
             o.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok)
             return wl.m, time.perf_counter() - t0
@@ -389,6 +416,8 @@ class OracleStep:
     def sample_desc(self):
         if self.wl.kind == "csa_decode":
             return f"1 of {self.wl.B} sequences per step (full index scan over T={self.wl.T} + attention)"
+        if self.wl.kind == "out_proj":
+            return f"{self.n} random token rows of S={self.wl.S} per step (both projections in fp64)"
         if self.wl.kind == "compress_append":
             return f"the pooling of the last L={self.wl.L} tokens of 1 of {self.wl.B} sequences per step"
         if self.wl.kind == "hca_decode":
@@ -404,7 +433,7 @@ def unit_name(wl):
 def metric_name(wl):
     return {"csa_prefill": "csa_prefill_tokens_per_s", "hca_prefill": "hca_prefill_tokens_per_s",
             "csa_decode": "csa_decode_queries_per_s", "hca_decode": "hca_decode_queries_per_s",
-            "compress_append": "csa_append_tokens_per_s"}[wl.kind]
+            "compress_append": "csa_append_tokens_per_s", "out_proj": "out_proj_tokens_per_s"}[wl.kind]
 
 
 def config_of(wl, n_gpus):
@@ -421,6 +450,10 @@ def config_of(wl, n_gpus):
     elif wl.kind == "compress_append":
         c.update({"B": wl.B, "ctx": wl.ctx, "appends_per_step": wl.m})
         del c["S"]
+    elif wl.kind == "out_proj":
+        c = {"workload": wl.name, "S": wl.S, "H": wl.H, "D": wl.D, "o_groups": wl.o_groups, "o_lora_rank": wl.o_rank,
+             "hidden": wl.hidden, "parallelism": f"replicas{n_gpus}",
+             "l2": "flushed between steps (256 MiB write outside the timed events)"}
     elif wl.kind == "csa_prefill":
         c.update({"topk": wl.topk, "index": f"{wl.HI}x{wl.dI}", "T": wl.T})
     else:
@@ -534,7 +567,11 @@ def main():
     mean_phase = phase_ms.mean(0)
     dom = int(np.argmax(mean_phase))
     dom_name = step.phases[dom]
-    if wl.kind == "compress_append":
+    if wl.kind == "out_proj":
+        alg = proj_flops(wl)
+        roof = {"bound": "tensor", "kernel": "proj_gemm_tc (o_a_proj + o_b_proj)",
+                "achieved": alg / (mean_phase[dom] / 1e3) / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    elif wl.kind == "compress_append":
         alg = append_bytes(wl, step.B)
         roof = {"bound": "hbm", "kernel": "compress_append (m launches, latency-bound)",
                 "achieved": alg / (mean_phase[dom] / 1e3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}

@@ -66,7 +66,8 @@ typedef enum csa_op {
     CSA_OP_CSA_FORWARD = 3,
     CSA_OP_HCA_FORWARD = 4,
     CSA_OP_DECODE = 5,
-    CSA_OP_HCA_DECODE = 6     /* hca_decode (B, T, W) */
+    CSA_OP_HCA_DECODE = 6,    /* hca_decode (B, T, W) */
+    CSA_OP_OUT_PROJ = 7       /* csa_out_proj */
 } csa_op;
 
 typedef struct csa_dims {
@@ -241,6 +242,22 @@ CSA_API csa_status csa_compress_append(const void *x_new, const void *g_new, con
                       int32_t rope_dim, int64_t P, double theta_cmp, double theta_tok, void *C,
                       uint8_t *c8, float *c8_scale, void *c_rope, int64_t Tcap, void *win, int32_t W,
                       void *stream);
+
+/* ---- 10. grouped low-rank output projection ----------------------------------------------------------
+ * [HF-V4 "Hybrid attention", grouped output projection: o_groups head groups, o_lora_rank per group,
+ * then hidden_size (o_a_proj as a grouped linear, then o_b_proj); Atlas config: o_groups 8,
+ * o_lora_rank 1024, hidden_size 4096].
+ *   o   [S, H*D] bf16: the attention output of each token, heads in order (group g = heads
+ *       [g H/G, (g+1) H/G), i.e. columns [g K, (g+1) K) with K = (H/G) D)
+ *   wa  [G, R, K] bf16: o_a_proj, one [R x K] matrix per group (row = output channel)
+ *   wb  [hidden, G*R] bf16: o_b_proj
+ *   z   [S, G*R] bf16 (out): z[:, g R + j] = sum_c o[:, g K + c] * wa[g, j, c]
+ *   out [S, hidden] bf16 (out): out[:, i] = sum_c z[:, c] * wb[i, c]
+ * fp32 accumulation; z is rounded to bf16 before o_b_proj. Requires H % G == 0, R and hidden
+ * multiples of 256, K and G*R multiples of 64. Workspace: 256 bytes (the status word). */
+CSA_API csa_status csa_out_proj(const void *o, const void *wa, const void *wb, int64_t S, int32_t H, int32_t D,
+                      int32_t G, int32_t R, int32_t hidden, void *z, void *out, void *workspace,
+                      size_t workspace_bytes, void *stream);
 
 #ifdef __cplusplus
 }

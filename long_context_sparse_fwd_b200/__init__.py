@@ -15,15 +15,16 @@ import torch
 
 __all__ = [
     "CSAError", "lib", "library_path", "compress", "index_topk", "attend", "hca_attend", "csa_forward",
-    "hca_forward", "decode", "hca_decode", "swa_attend", "compress_append", "workspace_size", "get_device_status",
-    "OP",
+    "hca_forward", "decode", "hca_decode", "swa_attend", "compress_append", "out_proj", "workspace_size",
+    "get_device_status", "OP",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libcsa.so")
 _lib = None
 
-OP = {"index_topk": 1, "attend": 2, "csa_forward": 3, "hca_forward": 4, "decode": 5, "hca_decode": 6}
+OP = {"index_topk": 1, "attend": 2, "csa_forward": 3, "hca_forward": 4, "decode": 5, "hca_decode": 6,
+      "out_proj": 7}
 _STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
            4: "CSA_ERR_TIMEOUT", 5: "CSA_ERR_WORKSPACE"}
 
@@ -73,6 +74,7 @@ def lib():
             "swa_attend": (I32, [P, P, P, I64, I32, I32, I32, I32, F64, F32, P, P, SZ, P]),
             "csa_compress_append": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I64, F64, F64, P, P, P, P, I64, P,
                                           I32, P]),
+            "csa_out_proj": (I32, [P, P, P, I64, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -345,3 +347,28 @@ def compress_append(x_new, g_new, pos_bias, state_x, state_g, P: int, m: int, ro
         _ptr(x_new), _ptr(g_new), _ptr(pos_bias), _ptr(state_x), _ptr(state_g), B, D, m, L, rope_dim, int(P),
         float(theta_cmp), float(theta_tok), _ptr(C), _ptr(c8), _ptr(c8_scale), _ptr(c_rope), Tcap, _ptr(win), W,
         _stream(stream)))
+
+
+def out_proj(o, wa, wb, z=None, out=None, workspace=None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Grouped low-rank output projection: o [S,H,D] (or [S,H*D]) bf16, wa [G,R,(H/G)*D] bf16,
+    wb [hidden,G*R] bf16. Returns (z [S,G*R] bf16, out [S,hidden] bf16)."""
+    S = o.shape[0]
+    G, R, K = wa.shape
+    hidden = wb.shape[0]
+    if o.dim() == 3:
+        H, D = o.shape[1], o.shape[2]
+    else:   # [S, H*D]: only the per-group width K and the row length matter
+        H, D = G, o.shape[1] // G
+    HD = H * D
+    _dev(o, torch.bfloat16, "o")
+    _dev(wa, torch.bfloat16, "wa", (G, R, K))
+    _dev(wb, torch.bfloat16, "wb", (hidden, G * R))
+    if HD != G * K:
+        raise ValueError(f"o has {HD} channels per token; wa expects {G} groups of {K}")
+    z = torch.empty(S, G * R, dtype=torch.bfloat16, device=o.device) if z is None else _dev(z, torch.bfloat16, "z", (S, G * R))
+    out = torch.empty(S, hidden, dtype=torch.bfloat16, device=o.device) if out is None else \
+        _dev(out, torch.bfloat16, "out", (S, hidden))
+    ws = _workspace("out_proj", o.device, workspace)
+    _check("csa_out_proj", lib().csa_out_proj(_ptr(o), _ptr(wa), _ptr(wb), S, H, D, G, R, hidden, _ptr(z), _ptr(out),
+                                              _ptr(ws), ws.numel(), _stream(stream)))
+    return z, out

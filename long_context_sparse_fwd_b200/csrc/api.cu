@@ -201,6 +201,8 @@ size_t csa_workspace_size(csa_op op, const csa_dims *d)
                align256(attend_tc_decode_partials(d->B, decode_splits_preferred(d->B)));
     case CSA_OP_HCA_DECODE:
         return kStatusBytes + align256(attend_tc_decode_partials(d->B, hca_decode_splits_preferred(d->B, d->T, d->W)));
+    case CSA_OP_OUT_PROJ:
+        return kStatusBytes;
     }
     return 0;
 }
@@ -511,6 +513,28 @@ csa_status csa_compress_append(const void *x_new, const void *g_new, const float
     a.log2_theta_cmp = rope_dim > 0 ? log2(theta_cmp) : 0.0;
     a.log2_theta_tok = rope_dim > 0 ? log2(theta_tok) : 0.0;
     return from_cuda(launch_compress_append(a, as_stream(stream)));
+}
+
+csa_status csa_out_proj(const void *o, const void *wa, const void *wb, int64_t S, int32_t H, int32_t D, int32_t G,
+                        int32_t R, int32_t hidden, void *z, void *out, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    CSA_CHECK_ARG(S >= 0 && H > 0 && D > 0 && G > 0 && R > 0 && hidden > 0 && H % G == 0);
+    CSA_CHECK_ARG(S == 0 || (o != nullptr && wa != nullptr && wb != nullptr && z != nullptr && out != nullptr));
+    CSA_CHECK_ARG(aligned16(o) && aligned16(wa) && aligned16(wb) && aligned16(z) && aligned16(out));
+    const int64_t K = (int64_t)(H / G) * D;
+    CSA_CHECK_SUP(K <= (1 << 30) && (int64_t)G * R <= (1 << 30));
+    CSA_CHECK_SUP(csa::proj_gemm_tc_supported(std::max<int64_t>(S, 1), R, (int)K, G) &&
+                  csa::proj_gemm_tc_supported(std::max<int64_t>(S, 1), hidden, G * R, 1));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    int32_t *status = static_cast<int32_t *>(workspace);
+    CSA_CUDA(csa::launch_proj_gemm_tc(static_cast<const uint16_t *>(o), (int64_t)H * D, static_cast<const uint16_t *>(wa),
+                                      static_cast<uint16_t *>(z), (int64_t)G * R, S, R, (int)K, G, status, st));
+    return from_cuda(csa::launch_proj_gemm_tc(static_cast<const uint16_t *>(z), (int64_t)G * R,
+                                              static_cast<const uint16_t *>(wb), static_cast<uint16_t *>(out), hidden, S,
+                                              hidden, G * R, 1, status, st));
 }
 
 }  // extern "C"

@@ -62,6 +62,11 @@ struct AppendArgs {
 };
 cudaError_t launch_compress_append(const AppendArgs &a, cudaStream_t stream);
 
+// proj.cu: grouped GEMM C[:, gN:(g+1)N] = A[:, gK:(g+1)K] . B[gN:(g+1)N, :]^T (bf16, fp32 accumulate)
+bool proj_gemm_tc_supported(int64_t M, int N, int K, int G);
+cudaError_t launch_proj_gemm_tc(const uint16_t *A, int64_t lda, const uint16_t *B, uint16_t *C, int64_t ldc, int64_t M,
+                                int N, int K, int G, int32_t *status, cudaStream_t stream);
+
 // api.cu: smallest workspace csa_decode accepts (no attention split partials)
 size_t decode_workspace_min(int64_t B, int64_t T, int32_t k);
 

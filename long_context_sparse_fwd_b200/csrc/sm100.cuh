@@ -178,6 +178,12 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // wait until every committed bulk store has finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// wait until at most the most recent committed bulk group may still be reading shared memory
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+// wait until every committed bulk group has completed (writes visible in global memory)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Bring one box of a 2-D tensor into L2 (no shared memory, no completion tracking).
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, int y)
 {

@@ -5,7 +5,8 @@ package. The product path (the CUDA library and its binding) never does, and the
 imports the product path.
 
 The arithmetic lives in ``csa_oracle.c`` (plain C, double precision, OpenMP over query rows);
-this module compiles it with gcc and marshals numpy arrays into it. bf16 arrays are passed as
+this module compiles it with gcc and marshals numpy arrays into it. The grouped output projection
+(``out_proj``) is two fp64 matrix products, done with numpy's. bf16 arrays are passed as
 their raw uint16 bit patterns, FP8 E4M3 caches as raw bytes, so the oracle reads exactly the
 values the GPU reads.
 """
@@ -239,3 +240,28 @@ def _as_f64(x) -> np.ndarray:
     except ImportError:  # pragma: no cover
         pass
     return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (8 significant bits, ties to even), as float64.
+    Finite, normal-range values only (what the projection produces)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def out_proj(o, wa, wb):
+    """Grouped low-rank output projection (Hugging Face Transformers docs "DeepSeek-V4", section
+    "Hybrid attention", grouped output projection; llm-atlas "DeepSeek-V4-Flash" config: o_groups,
+    o_lora_rank, hidden_size). The heads are split into G consecutive groups; group g's concatenated
+    head outputs (K = (H/G) D channels) go through wa[g] ([R, K]) to R channels; the G*R channels,
+    stored in bf16, go through wb ([hidden, G*R]). fp64 from the bf16 inputs.
+    Returns (z before its bf16 rounding [S, G*R], out [S, hidden]), both float64."""
+    o_ = _as_f64(o)
+    o_ = o_.reshape(o_.shape[0], -1)
+    wa_, wb_ = _as_f64(wa), _as_f64(wb)
+    G, R, K = wa_.shape
+    assert o_.shape[1] == G * K and wb_.shape[1] == G * R
+    z = np.concatenate([o_[:, g * K:(g + 1) * K] @ wa_[g].T for g in range(G)], axis=1)
+    out = round_bf16(z) @ wb_.T
+    return z, out

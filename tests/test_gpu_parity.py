@@ -461,3 +461,40 @@ def test_compress_append_feeds_decode():
     ref = oracle.decode_attend(q, winb, np.tile(np.arange(T, dtype=np.int32), (B, 1)), sinks, P, wl.r, wl.theta_tok,
                                wl.theta_cmp, C=Cb)
     check_close(o.cpu(), ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
+# ---- 9. grouped output projection --------------------------------------------------------------------
+
+def _proj_close(got, ref, what):
+    got = got.float().cpu().double().numpy()
+    ref = np.asarray(ref)
+    rms = float(np.sqrt((ref ** 2).mean()))
+    bad = np.abs(got - ref) > 2.0 ** -8 * np.abs(ref) + 2e-3 * rms
+    assert not bad.any(), f"{what}: {int(bad.sum())} values beyond bf16 rounding (rms {rms:.3g})"
+
+
+@pytest.mark.parametrize("S", [300, 130])
+def test_out_proj(S):
+    """V4-Flash shapes (8 groups of 8 heads x 512 -> 1024 each -> 4096); S=130 leaves a ragged row tile."""
+    from workloads import proj_inputs
+    wl = WORKLOADS[7].with_(S=S)
+    g = proj_inputs(wl, device=DEV)
+    z, out = csa.out_proj(g["o"], g["wa"], g["wb"])
+    torch.cuda.synchronize()
+    h = host(g)
+    zr, outr = oracle.out_proj(h["o"], h["wa"], h["wb"])
+    _proj_close(z, zr, "z")
+    _proj_close(out, outr, "out")
+
+
+def test_out_proj_full_size_sampled():
+    """S=8192 as the benchmark runs it, checked on sampled rows (rows are independent)."""
+    from workloads import proj_inputs
+    wl = WORKLOADS[7]
+    g = proj_inputs(wl, device=DEV)
+    z, out = csa.out_proj(g["o"], g["wa"], g["wb"])
+    torch.cuda.synchronize()
+    rows = sample_rows(wl.S, 24, 17, must=[0, 127, 128, wl.S - 1])
+    zr, outr = oracle.out_proj(g["o"][rows].cpu(), g["wa"].cpu(), g["wb"].cpu())
+    _proj_close(z[rows], zr, "z")
+    _proj_close(out[rows], outr, "out")

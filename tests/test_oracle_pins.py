@@ -516,3 +516,72 @@ def test_bf16_decode_matches_torch():
     ref = torch.tensor(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
     got = np.array([oracle.bf16_to_f64(int(b)) for b in bits])
     np.testing.assert_array_equal(got, ref)
+
+
+# ---- grouped output projection ---------------------------------------------------------------------
+
+def _bf(x):
+    return torch.tensor(np.asarray(x, np.float64), dtype=torch.float32).to(torch.bfloat16)
+
+
+def test_round_bf16_matches_torch():
+    x = np.random.default_rng(21).standard_normal(20000).astype(np.float32) * np.float32(3.0)
+    got = oracle.round_bf16(x.astype(np.float64))
+    ref = torch.tensor(x).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_out_proj_identity_weights():
+    """wa[g] = I and wb = I: the projection returns the attention output unchanged."""
+    S, G, K = 5, 2, 8
+    o = _bf(np.random.default_rng(1).standard_normal((S, G * K)))
+    wa = _bf(np.stack([np.eye(K)] * G))
+    wb = _bf(np.eye(G * K))
+    z, out = oracle.out_proj(o, wa, wb)
+    np.testing.assert_array_equal(z, o.double().numpy())
+    np.testing.assert_array_equal(out, o.double().numpy())
+
+
+def test_out_proj_groups_are_separate():
+    """The channels of group g depend only on the heads of group g."""
+    rng = np.random.default_rng(2)
+    S, G, K, R, hid = 4, 3, 6, 5, 7
+    o = rng.standard_normal((S, G * K))
+    wa, wb = _bf(rng.standard_normal((G, R, K))), _bf(rng.standard_normal((hid, G * R)))
+    z, _ = oracle.out_proj(_bf(o), wa, wb)
+    o2 = o.copy()
+    o2[:, K:2 * K] = 0.0
+    z2, _ = oracle.out_proj(_bf(o2), wa, wb)
+    np.testing.assert_array_equal(z2[:, R:2 * R], 0.0)
+    np.testing.assert_array_equal(z2[:, :R], z[:, :R])
+    np.testing.assert_array_equal(z2[:, 2 * R:], z[:, 2 * R:])
+
+
+def test_out_proj_permutation_weights():
+    """A permutation wb reorders the bf16-rounded low-rank channels."""
+    rng = np.random.default_rng(3)
+    S, G, K, R = 3, 2, 4, 4
+    o, wa = _bf(rng.standard_normal((S, G * K))), _bf(rng.standard_normal((G, R, K)))
+    perm = rng.permutation(G * R)
+    z, out = oracle.out_proj(o, wa, _bf(np.eye(G * R)[perm]))
+    np.testing.assert_array_equal(out, oracle.round_bf16(z)[:, perm])
+
+
+def test_out_proj_brute_force_tiny():
+    rng = np.random.default_rng(4)
+    S, G, K, R, hid = 2, 2, 3, 2, 3
+    o, wa, wb = (_bf(rng.standard_normal(sh)) for sh in [(S, G * K), (G, R, K), (hid, G * R)])
+    z, out = oracle.out_proj(o, wa, wb)
+    od, wad, wbd = o.double().numpy(), wa.double().numpy(), wb.double().numpy()
+    for t in range(S):
+        zt = []
+        for g in range(G):
+            for j in range(R):
+                acc = 0.0
+                for c in range(K):
+                    acc += od[t, g * K + c] * wad[g, j, c]
+                zt.append(acc)
+        np.testing.assert_allclose(z[t], zt, rtol=1e-15, atol=1e-15)
+        zb = oracle.round_bf16(np.array(zt))
+        for i in range(hid):
+            np.testing.assert_allclose(out[t, i], sum(zb[c] * wbd[i, c] for c in range(G * R)), rtol=1e-14)

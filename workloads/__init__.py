@@ -22,7 +22,7 @@ from typing import Dict, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "prefill_inputs", "attend_inputs", "decode_inputs", "tensor_gen"]
+__all__ = ["Workload", "WORKLOADS", "prefill_inputs", "attend_inputs", "decode_inputs", "proj_inputs", "tensor_gen"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -47,6 +47,10 @@ class Workload:
     B: int = 0
     ctx: int = 0              # tokens of history per sequence
     cache: str = "bf16"       # "bf16" | "fp8"
+    # grouped output projection (o_groups, o_lora_rank, hidden_size of the V4-Flash config)
+    o_groups: int = 8
+    o_rank: int = 1024
+    hidden: int = 4096
 
     @property
     def T(self) -> int:
@@ -70,6 +74,8 @@ WORKLOADS: Dict[int, Workload] = {
     5: Workload("hca_decode_b8_ctx1m", "hca_decode", B=8, ctx=1048576, m=128, L=128, topk=0, seed=5),
     # the CSA compressor's decode step for 64 sequences at 128K context (m = 4 appends close one entry)
     6: Workload("csa_append_b64_ctx128k", "compress_append", B=64, ctx=131072, m=4, L=8, topk=0, seed=6),
+    # the grouped output projection after the V4-Flash attention, S=8192
+    7: Workload("v4flash_out_proj_s8192", "out_proj", S=8192, seed=7),
 }
 
 
@@ -93,7 +99,7 @@ def _uniform(shape, seed, tid, device):
 
 
 # tensor ids (stable: changing one changes that tensor only)
-_Q, _KV, _GATE, _BIAS, _QI, _KI, _WI, _SINK, _C, _KVROT, _WIN = range(11)
+_Q, _KV, _GATE, _BIAS, _QI, _KI, _WI, _SINK, _C, _KVROT, _WIN, _O, _WA, _WB = range(14)
 
 
 def prefill_inputs(wl: Workload, device="cpu", need_index: Optional[bool] = None,
@@ -157,3 +163,15 @@ def decode_inputs(wl: Workload, device="cpu", batch: Optional[int] = None) -> Di
     else:
         out["C"] = _normal((B, T, D), 1.0, wl.seed, _C, device)
     return out
+
+
+def proj_inputs(wl: Workload, device="cpu") -> Dict[str, torch.Tensor]:
+    """Grouped output projection inputs: the attention output o [S, H*D] bf16 ~ N(0, 0.25^2) and
+    synthetic weights wa [G, R, (H/G)*D], wb [hidden, G*R] bf16 ~ N(0, 1/fan_in)."""
+    G, R, hid = wl.o_groups, wl.o_rank, wl.hidden
+    K = wl.H // G * wl.D
+    return {
+        "o": _normal((wl.S, wl.H * wl.D), 0.25, wl.seed, _O, device),
+        "wa": _normal((G, R, K), 1.0 / math.sqrt(K), wl.seed, _WA, device),
+        "wb": _normal((hid, G * R), 1.0 / math.sqrt(G * R), wl.seed, _WB, device),
+    }
