@@ -79,6 +79,99 @@ compress_entries_kernel(const uint16_t *__restrict__ kv, const uint16_t *__restr
     *reinterpret_cast<uint4 *>(C + w * D + d0) = o;
 }
 
+// Long windows (HCA: L = 128): the window of one (entry, 8-channel group) is split across G = 8
+// neighbouring lanes, each walking L/G consecutive positions with its own online softmax; the G
+// partial (max, sum, weighted sum) states are then merged by shuffles. Lane j of a group of 8 lanes
+// takes positions j*L/8 ..; the 4 groups of a warp take 4 consecutive channel groups (64 contiguous
+// bytes of each row).
+__global__ void __launch_bounds__(256)
+compress_entries_split_kernel(const uint16_t *__restrict__ kv, const uint16_t *__restrict__ gate,
+                              const float *__restrict__ bias, int64_t T, int D, int m, int L, int r,
+                              double log2_theta_cmp, uint16_t *__restrict__ C)
+{
+    constexpr int G = 8;
+    const int chunks = D >> 3;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int sub = threadIdx.x & (G - 1);
+    const int64_t item = gid / G;   // (entry, channel group)
+    const bool valid = item < T * chunks;
+    const int64_t w = valid ? item / chunks : 0;
+    const int d0 = valid ? (int)(item - w * chunks) << 3 : 0;
+    const int64_t start = (w + 1) * (int64_t)m - L;
+    const int64_t end = (w + 1) * (int64_t)m;
+    const int per = (L + G - 1) / G;
+    int64_t j0 = start + (int64_t)sub * per, j1 = j0 + per;
+    if (j0 < 0) j0 = 0;
+    if (j1 > end) j1 = end;
+
+    float mx[8], l[8], acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; l[e] = 0.f; acc[e] = 0.f; }
+    if (valid) {
+#pragma unroll 4
+        for (int64_t j = j0; j < j1; ++j) {
+            const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gate + j * D + d0));
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(kv + j * D + d0));
+            const float b = __ldg(bias + (j - start));
+            const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float a = ((e & 1) ? bf_hi(gw[e >> 1]) : bf_lo(gw[e >> 1])) + b;
+                const float x = (e & 1) ? bf_hi(vw[e >> 1]) : bf_lo(vw[e >> 1]);
+                if (a > mx[e]) {
+                    const float corr = expf(mx[e] - a);
+                    l[e] = l[e] * corr + 1.f;
+                    acc[e] = acc[e] * corr + x;
+                    mx[e] = a;
+                } else {
+                    const float pe = expf(a - mx[e]);
+                    l[e] += pe;
+                    acc[e] += pe * x;
+                }
+            }
+        }
+    }
+    // merge the G partial states of this (entry, channel group): lanes differing in the low 3 bits
+#pragma unroll
+    for (int o = 1; o < G; o <<= 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, mx[e], o);
+            const float l2 = __shfl_xor_sync(0xffffffffu, l[e], o);
+            const float a2 = __shfl_xor_sync(0xffffffffu, acc[e], o);
+            const float mm = fmaxf(mx[e], m2);
+            const float c1 = mx[e] == -INFINITY ? 0.f : expf(mx[e] - mm);
+            const float c2 = m2 == -INFINITY ? 0.f : expf(m2 - mm);
+            l[e] = l[e] * c1 + l2 * c2;
+            acc[e] = acc[e] * c1 + a2 * c2;
+            mx[e] = mm;
+        }
+    }
+    if (!valid || sub != 0) return;
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = acc[e] / l[e];
+    if (d0 >= D - r) {
+        const double pos = (double)(w * (int64_t)m);
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const int pp = (d0 + e - (D - r)) >> 1;
+            float c, sn;
+            rope_cos_sin(pos, pp, r, log2_theta_cmp, &c, &sn);
+            const float x0 = out[e], x1 = out[e + 1];
+            out[e] = x0 * c - x1 * sn;
+            out[e + 1] = x0 * sn + x1 * c;
+        }
+    }
+    uint4 o4;
+    o4.x = pack_bf2(out[0], out[1]);
+    o4.y = pack_bf2(out[2], out[3]);
+    o4.z = pack_bf2(out[4], out[5]);
+    o4.w = pack_bf2(out[6], out[7]);
+    *reinterpret_cast<uint4 *>(C + w * D + d0) = o4;
+}
+
 __global__ void __launch_bounds__(256)
 rotate_rows_kernel(const uint16_t *__restrict__ kv, int64_t S, int D, int r, double log2_theta_tok,
                    uint16_t *__restrict__ kv_rot)
@@ -112,8 +205,14 @@ cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const floa
     const int chunks = D / 8;
     if (T > 0 && C != nullptr) {
         const int64_t n = T * chunks;
-        compress_entries_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(kv, gate, bias, T, D, m, L, r,
-                                                                                  log2(theta_cmp), C);
+        if (L >= 64) {   // long windows: split each window across 8 lanes
+            const int64_t nt = n * 8;
+            compress_entries_split_kernel<<<(unsigned)((nt + 255) / 256), 256, 0, stream>>>(kv, gate, bias, T, D, m, L,
+                                                                                             r, log2(theta_cmp), C);
+        } else {
+            compress_entries_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(kv, gate, bias, T, D, m, L, r,
+                                                                                      log2(theta_cmp), C);
+        }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
