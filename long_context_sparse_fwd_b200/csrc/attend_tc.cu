@@ -866,12 +866,11 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
         tw = tq;   // no window rows: never used
     }
     a.o = out_rows;   // final rows, or the split partials
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(attend_tc_kernel), smem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM walks the units (query rows, or sequence splits) with stride grid
     int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
     const int64_t units = x.R * nsplit;
     const unsigned grid = (unsigned)std::min<int64_t>(units, std::max(sms, 1));
     attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tc, tw, a);

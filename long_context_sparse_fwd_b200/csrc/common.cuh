@@ -5,6 +5,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "../../include/csa.h"
 
 namespace csa {
@@ -48,6 +51,45 @@ __device__ __forceinline__ uint32_t score_key(float x)
 {
     uint32_t u = __float_as_uint(x + 0.0f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---- host: per-device settings done once -------------------------------------------------------
+
+constexpr int kMaxDevices = 64;
+
+// Device index and SM count of the current device (the count is queried once per device).
+inline cudaError_t current_device_sms(int *dev, int *sms)
+{
+    static int cached[kMaxDevices];
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return e;
+    if (*dev < 0 || *dev >= kMaxDevices) return cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, *dev);
+    if (cached[*dev] == 0) {
+        int n = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, *dev)) != cudaSuccess) return e;
+        cached[*dev] = n;
+    }
+    *sms = cached[*dev];
+    return cudaSuccess;
+}
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once per (device, kernel) and
+// only when a larger size than before is asked for.
+inline cudaError_t ensure_smem_limit(const void *kernel, size_t bytes)
+{
+    static std::mutex mu;
+    static std::unordered_map<const void *, int> done[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done[dev].find(kernel);
+    if (it != done[dev].end() && it->second >= (int)bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done[dev][kernel] = (int)bytes;
+    return e;
 }
 
 __device__ __forceinline__ int64_t visible_entries(int64_t t, int m, int64_t T)

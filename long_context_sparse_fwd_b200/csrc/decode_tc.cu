@@ -619,11 +619,10 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     const size_t fixed = 1024 + 2 * (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
     sp.stages = (int)std::min<size_t>(MAX_STAGES, (227 * 1024 - fixed) / a_bytes);
     const size_t smem = fixed + (size_t)sp.stages * a_bytes;
-    e = cudaFuncSetAttribute(decode_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_tc_kernel), smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
     const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
     decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -692,7 +692,7 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     CUtensorMap tq, tk;
     if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)S * HI, dI, BN)) return cudaErrorInvalidValue;
     if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)T, dI, BM)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(index_topk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(index_topk_tc_kernel), smem);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((S + p.Q - 1) / p.Q);
     index_topk_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tk, p);

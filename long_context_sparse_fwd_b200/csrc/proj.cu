@@ -234,11 +234,10 @@ cudaError_t launch_proj_gemm_tc(const uint16_t *A, int64_t lda, const uint16_t *
     p.G = G;
     p.mt = (int)((M + TM - 1) / TM);
     p.nt = N / TN;
-    cudaError_t e = cudaFuncSetAttribute(proj_gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(proj_gemm_tc_kernel), SMEM);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
     const int64_t tiles = (int64_t)G * p.mt * p.nt;
     const unsigned grid = (unsigned)std::min<int64_t>(tiles, sms);
     proj_gemm_tc_kernel<<<grid, NUM_THREADS, SMEM, stream>>>(ta, tb, tcm, p);

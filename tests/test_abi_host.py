@@ -133,3 +133,36 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises(ValueError):
         csa.compress(torch.zeros(8, 8, dtype=torch.bfloat16), torch.zeros(8, 8, dtype=torch.bfloat16),
                      torch.zeros(8), 4, 8, 0, 1e4, 1e4)
+
+
+@no_gpu
+def test_later_calls_reject_bad_arguments():
+    """hca_decode, swa_attend, csa_compress_append and csa_out_proj check their arguments on the host."""
+    L = csa.lib()
+
+    def hd(C=FAKE, B=2, D=512, T=100, P=1000, wsb=1 << 20):
+        return L.hca_decode(FAKE, C, None, None, None, FAKE, FAKE, B, 64, D, T, 128, 64, P, 1e4, 1.6e5, 0.0, FAKE,
+                            FAKE, wsb, None)
+    assert hd(T=-1) == INVALID
+    assert hd(P=-5) == INVALID
+    assert hd(C=None) == INVALID                # entries but neither a bf16 nor an FP8 cache
+    assert hd(D=96) == UNSUP
+    assert hd(wsb=16) == WS
+
+    assert L.swa_attend(FAKE, FAKE, FAKE, 64, 8, 96, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == UNSUP
+    assert L.swa_attend(FAKE, None, FAKE, 64, 8, 128, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == INVALID
+
+    def ca(C=FAKE, D=512, Lw=8, P=7, Tcap=2):
+        return L.csa_compress_append(FAKE, FAKE, FAKE, FAKE, FAKE, 2, D, 4, Lw, 64, P, 1.6e5, 1e4, C, None, None,
+                                     None, Tcap, FAKE, 128, None)
+    assert ca(Lw=2) == INVALID                  # pooling window shorter than the stride
+    assert ca(P=11, Tcap=2) == INVALID          # entry 2 closes at P=11 but the cache holds two entries
+    assert ca(C=None) == INVALID                # an entry closes and there is no cache to take it
+    assert ca(D=520) == UNSUP
+
+    def op(G=8, R=1024, hid=4096, wsb=256):
+        return L.csa_out_proj(FAKE, FAKE, FAKE, 128, 64, 512, G, R, hid, FAKE, FAKE, FAKE, wsb, None)
+    assert op(G=7) == INVALID                   # 64 heads do not split into 7 groups
+    assert op(R=1000) == UNSUP                  # o_lora_rank not a multiple of 256
+    assert op(hid=100) == UNSUP
+    assert op(wsb=16) == WS

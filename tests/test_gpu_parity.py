@@ -498,3 +498,30 @@ def test_out_proj_full_size_sampled():
     zr, outr = oracle.out_proj(g["o"][rows].cpu(), g["wa"].cpu(), g["wb"].cpu())
     _proj_close(z[rows], zr, "z")
     _proj_close(out[rows], outr, "out")
+
+
+# ---- 10. empty inputs --------------------------------------------------------------------------------
+
+def test_empty_inputs():
+    """Zero tokens or zero sequences: every call succeeds and returns empty outputs."""
+    from workloads import proj_inputs
+    wl = WORKLOADS[1].with_(S=0)
+    g = prefill_inputs(wl, device=DEV)
+    o, C, kv_rot, idx = csa.csa_forward(g["q"], g["kv"], g["gate"], g["pos_bias"], g["qI"], g["kI"], g["w"],
+                                        g["sinks"], wl.m, wl.L, wl.topk, wl.W, wl.r, wl.theta_tok, wl.theta_cmp)
+    assert o.shape == (0, wl.H, wl.D) and C.shape[0] == 0 and idx.shape[0] == 0
+    h = prefill_inputs(WORKLOADS[2].with_(S=0), device=DEV)
+    o, C, _ = csa.hca_forward(h["q"], h["kv"], h["gate"], h["pos_bias"], h["sinks"], 128, 128, wl.W, wl.r,
+                              wl.theta_tok, wl.theta_cmp)
+    assert o.shape == (0, wl.H, wl.D)
+    dw = WORKLOADS[3].with_(ctx=4096)
+    y = decode_inputs(dw, device=DEV, batch=0)
+    o, idx = csa.decode(y["q"], y["qI"], y["w"], y["kI"], y["win"], y["sinks"], dw.ctx - 1, dw.topk, dw.r,
+                        dw.theta_tok, dw.theta_cmp, C=y["C"])
+    assert o.shape == (0, dw.H, dw.D) and idx.shape == (0, dw.topk)
+    o = csa.hca_decode(y["q"], y["win"], y["sinks"], dw.ctx - 1, dw.r, dw.theta_tok, dw.theta_cmp, C=y["C"])
+    assert o.shape == (0, dw.H, dw.D)
+    p = proj_inputs(WORKLOADS[7].with_(S=0), device=DEV)
+    z, out = csa.out_proj(p["o"], p["wa"], p["wb"])
+    assert z.shape == (0, 8 * 1024) and out.shape == (0, 4096)
+    torch.cuda.synchronize()
