@@ -360,16 +360,18 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
     dims.k = k;
     CSA_TRY(check_workspace(workspace, workspace_bytes, decode_workspace_min(B, T, k)));
     cudaStream_t st = as_stream(stream);
-    CSA_TRY(reset_status(workspace, st));
     char *base = static_cast<char *>(workspace);
     float *scores = reinterpret_cast<float *>(base + kStatusBytes);
     const size_t index_ws = decode_index_bytes(B, T, k);
     int32_t *idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t *>(base + kStatusBytes + index_ws);
     const size_t used = decode_workspace_min(B, T, k);
     if (T > 0 && decode_index_tc_supported(T, HI, dI, k)) {
+        // one clear: the status word and the head of the index workspace that follows it
+        CSA_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + decode_index_head_bytes(B), st));
         CSA_CUDA(launch_decode_index_tc(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
                                         HI, dI, k, idx, scores, static_cast<int32_t *>(workspace), st));
     } else {
+        CSA_TRY(reset_status(workspace, st));
         CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
                                      HI, dI, 1, 1, scores, st));
         CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
@@ -396,6 +398,7 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
     a.r = rope_dim;
     a.m = 1;
     a.decode = 1;
+    a.after_kernel = 1;   // the top-k kernel precedes it on the stream
     a.scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / sqrt((double)D));
     a.log2_theta_tok = rope_dim > 0 ? log2(theta_tok) : 0.0;
     a.log2_theta_cmp = rope_dim > 0 ? log2(theta_cmp) : 0.0;

@@ -221,6 +221,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
+    grid_dependency_wait();   // the index lists (decode: written by the top-k kernel just before)
+    grid_launch_dependents();
 
     if (warp == PLAN_WARP) {
         // ====== planner: index list, block split and rope tables of each query; window rope turn ======
@@ -799,6 +801,7 @@ combine_splits_kernel(const float *__restrict__ part_o, const float *__restrict_
 {
     const int64_t b = blockIdx.x / HH;
     const int h = blockIdx.x % HH;
+    grid_dependency_wait();   // the split partials
     const float z = sinks[h] * 1.4426950408889634f;
     float M = z;
     for (int i = 0; i < nsplit; ++i) {
@@ -873,6 +876,7 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
     const int64_t units = x.R * nsplit;
     const unsigned grid = (unsigned)std::min<int64_t>(units, std::max(sms, 1));
+    if (x.after_kernel) return launch_dependent(attend_tc_kernel, dim3(grid), dim3(NUM_THREADS), smem, stream, tq, tc, tw, a);
     attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tc, tw, a);
     return cudaGetLastError();
 }
@@ -898,8 +902,8 @@ cudaError_t launch_attend_tc_decode(const AttnArgs &x, int nsplit, float *part, 
     float *part_ml = part + (size_t)x.R * nsplit * HH * DD;
     cudaError_t e = launch_tc(x, nsplit, part_o, part_ml, stream);
     if (e != cudaSuccess) return e;
-    combine_splits_kernel<<<(unsigned)(x.R * HH), 128, 0, stream>>>(part_o, part_ml, x.sinks, nsplit, x.o);
-    return cudaGetLastError();
+    return launch_dependent(combine_splits_kernel, dim3((unsigned)(x.R * HH)), dim3(128), 0, stream,
+                            (const float *)part_o, (const float *)part_ml, x.sinks, nsplit, x.o);
 }
 
 }  // namespace csa

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 #include <unordered_map>
 
 #include "../../include/csa.h"
@@ -90,6 +91,37 @@ inline cudaError_t ensure_smem_limit(const void *kernel, size_t bytes)
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e == cudaSuccess) done[dev][kernel] = (int)bytes;
     return e;
+}
+
+// ---- programmatic dependent launch ---------------------------------------------------------------
+//
+// A kernel launched with launch_dependent() may be scheduled while the kernel before it in the stream
+// is still running: it runs its prologue, then grid_dependency_wait() blocks until that kernel has
+// completed and its memory is visible. Every such kernel calls grid_dependency_wait() before it
+// touches memory written earlier in the chain and before it can exit, so that its own completion still
+// implies the completion of everything before it. Both device calls are no-ops when the kernel was
+// launched the ordinary way.
+
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel in the stream (if launched with launch_dependent) start being scheduled.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                                    Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 __device__ __forceinline__ int64_t visible_entries(int64_t t, int m, int64_t T)

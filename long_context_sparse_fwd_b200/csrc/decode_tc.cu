@@ -37,6 +37,8 @@ struct ScoreParams {
     uint32_t *keymax;    // [B] largest order-preserving score key (zero before the scan)
     uint32_t *nkeymin;   // [B] largest complemented key, i.e. ~(smallest key) (zero before the scan)
     int32_t *status;
+    uint4 *zero;         // top-k counters, histograms and bitmaps: cleared here for the kernels after
+    int64_t zero_n16;    // (16-byte words)
     int64_t T, G;        // entries per sequence; total tiles (B * tiles per sequence)
     int HI, dI, stages, tps;
 };
@@ -90,6 +92,7 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
+    grid_launch_dependents();   // the top-k kernels may be scheduled as this grid's CTAs finish
 
     if (warp == 0) {
         if (ntiles > 0) {
@@ -160,6 +163,8 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     } else {
         const int quarter = warp & 3, etid = threadIdx.x - 64;
         const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
+        for (int64_t i = (int64_t)blockIdx.x * EPI_THREADS + etid; i < p.zero_n16; i += (int64_t)gridDim.x * EPI_THREADS)
+            p.zero[i] = make_uint4(0u, 0u, 0u, 0u);
         float wr[64];   // index weights of the current sequence (HI == 64 keeps them in registers)
         // range of the score keys of the current sequence seen by this thread, merged into the
         // sequence's global range (for the top-k's histogram) whenever the sequence changes
@@ -263,6 +268,7 @@ constexpr int TK_CHUNK = 8192;         // entries per histogram / collect CTA
 constexpr int TK_THREADS = 512;
 constexpr int FIN_THREADS = 1024;
 constexpr int CAND_CAP = 2048;         // candidates ranked directly; more take the exact fallback
+constexpr int TK_PER = TK_CHUNK / TK_THREADS;   // scores per thread: all loaded before any is used
 
 struct KeyRange {
     uint32_t prefix_hi;   // the common high bits (bits above top), as in every key
@@ -348,13 +354,23 @@ topk_hist_kernel(const float *__restrict__ scores, int64_t T, const uint32_t *__
 {
     __shared__ uint32_t sh[HBINS];
     const int b = blockIdx.y;
-    const KeyRange r = key_range(keymax[b], nkeymin[b]);
     for (int i = threadIdx.x; i < HBINS; i += TK_THREADS) sh[i] = 0;
+    grid_dependency_wait();   // the scores and key ranges of the scan
+    grid_launch_dependents();
+    const KeyRange r = key_range(keymax[b], nkeymin[b]);
     __syncthreads();
     const int64_t s0 = (int64_t)blockIdx.x * TK_CHUNK;
     const int n = (int)min((int64_t)TK_CHUNK, T - s0);
     const float *sc = scores + b * T + s0;
-    for (int i = threadIdx.x; i < n; i += TK_THREADS) atomicAdd(&sh[key_digit(score_key(sc[i]), r)], 1u);
+    float v[TK_PER];
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j) {
+        const int i = j * TK_THREADS + threadIdx.x;
+        v[j] = i < n ? sc[i] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j)
+        if (j * TK_THREADS + (int)threadIdx.x < n) atomicAdd(&sh[key_digit(score_key(v[j]), r)], 1u);
     __syncthreads();
     uint32_t *hg = hist + (int64_t)b * HBINS;
     for (int i = threadIdx.x; i < HBINS; i += TK_THREADS)
@@ -371,21 +387,31 @@ topk_collect_kernel(const float *__restrict__ scores, int64_t T, int k, const ui
     __shared__ uint32_t sh_hist[HBINS];
     __shared__ uint32_t sh_sums[HBINS / 4 + 2];
     const int b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t s0 = (int64_t)blockIdx.x * TK_CHUNK;
+    grid_dependency_wait();   // the histograms
+    grid_launch_dependents();
+    float v[TK_PER];          // this chunk's scores, in flight while the threshold is found
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j) {
+        const int64_t s = s0 + warp * 32 + j * TK_THREADS + lane;
+        v[j] = s < T ? scores[b * T + s] : 0.f;
+    }
     const KeyRange r = key_range(keymax[b], nkeymin[b]);
     int dstar;
     uint32_t above;
     find_threshold(hist + (int64_t)b * HBINS, k, sh_hist, sh_sums, &dstar, &above);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t s0 = (int64_t)blockIdx.x * TK_CHUNK;
     const int64_t nw = (T + 31) >> 5;
     uint32_t *bm = bitmap + b * nw;
     uint2 *cb = cand + (int64_t)b * CAND_CAP;
-    for (int base = warp * 32; base < TK_CHUNK; base += TK_THREADS) {
+#pragma unroll
+    for (int j = 0; j < TK_PER; ++j) {
+        const int base = warp * 32 + j * TK_THREADS;
         const int64_t s = s0 + base + lane;
         bool take = false, isc = false;
         uint32_t key = 0u;
         if (s < T) {
-            key = score_key(scores[b * T + s]);
+            key = score_key(v[j]);
             const int d = (int)key_digit(key, r);
             take = d > dstar;
             isc = d == dstar;
@@ -444,6 +470,8 @@ topk_final_kernel(const float *__restrict__ scores, int64_t T, int k, const uint
     __shared__ uint32_t sh_sel[4];
     const int b = blockIdx.x, tid = threadIdx.x;
     int32_t *out = idx + (int64_t)b * k;
+    grid_dependency_wait();   // the candidates and bitmaps (or, without them, the scan)
+    grid_launch_dependents();
     if (T <= k) {   // every entry is selected
         for (int j = tid; j < k; j += FIN_THREADS) out[j] = j < T ? j : -1;
         return;
@@ -548,25 +576,28 @@ topk_final_kernel(const float *__restrict__ scores, int64_t T, int k, const uint
 
 }  // namespace
 
-// Workspace of the decode index step (256-byte aligned pieces): scores [B, T] fp32, then a region
-// zeroed at the start of every call (keymax [B], nkeymin [B], ncand [B], hist [B, 2048], bitmap
-// [B, ceil(T/32)]), then the candidates [B, 2048] (key, index).
+// Workspace of the decode index step (256-byte aligned pieces): the head (keymax [B], nkeymin [B]),
+// which the caller zeroes before the call; scores [B, T] fp32; a region the scan kernel zeroes (ncand
+// [B], hist [B, 2048], bitmap [B, ceil(T/32)]); the candidates [B, 2048] (key, index).
 struct DecodeIndexLayout {
-    size_t scores, zero, zero_bytes, keymax, nkeymin, ncand, hist, bitmap, cand, total;
+    size_t keymax, nkeymin, scores, zero, zero_bytes, ncand, hist, bitmap, cand, total;
 };
+
+static size_t al256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t decode_index_head_bytes(int64_t B) { return al256((size_t)B * 8); }
 
 static DecodeIndexLayout decode_index_layout(int64_t B, int64_t T)
 {
-    auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
     DecodeIndexLayout L;
-    L.scores = 0;
-    L.zero = al((size_t)B * T * 4);
-    L.keymax = L.zero;
-    L.nkeymin = L.keymax + (size_t)B * 4;
-    L.ncand = L.nkeymin + (size_t)B * 4;
-    L.hist = al(L.ncand + (size_t)B * 4);
+    L.keymax = 0;
+    L.nkeymin = (size_t)B * 4;
+    L.scores = decode_index_head_bytes(B);
+    L.zero = al256(L.scores + (size_t)B * T * 4);
+    L.ncand = L.zero;
+    L.hist = al256(L.ncand + (size_t)B * 4);
     L.bitmap = L.hist + (size_t)B * HBINS * 4;
-    L.zero_bytes = al(L.bitmap + (size_t)B * ((T + 31) / 32) * 4) - L.zero;
+    L.zero_bytes = al256(L.bitmap + (size_t)B * ((T + 31) / 32) * 4) - L.zero;
     L.cand = L.zero + L.zero_bytes;
     L.total = L.cand + (size_t)B * CAND_CAP * 8;
     return L;
@@ -584,7 +615,9 @@ bool decode_index_tc_supported(int64_t T, int HI, int dI, int k)
            T <= (1ll << 26);
 }
 
-// scores/candidates live in `ws` (decode_index_workspace bytes, 256-byte aligned)
+// scores/candidates live in `ws` (decode_index_workspace bytes, 256-byte aligned), whose first
+// decode_index_head_bytes(B) bytes the caller has zeroed on this stream. The kernels after the scan
+// are launched as programmatic dependents, each one scheduled while the one before it finishes.
 cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t B, int64_t T, int HI,
                                    int dI, int k, int32_t *idx, void *ws, int32_t *status, cudaStream_t stream)
 {
@@ -598,8 +631,7 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     uint32_t *hist = reinterpret_cast<uint32_t *>(p8 + L.hist);
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(p8 + L.bitmap);
     uint2 *cand = reinterpret_cast<uint2 *>(p8 + L.cand);
-    cudaError_t e = cudaMemsetAsync(p8 + L.zero, 0, L.zero_bytes, stream);
-    if (e != cudaSuccess) return e;
+    cudaError_t e;
 
     CUtensorMap tq, tk;
     if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)B * HI, dI, HI)) return cudaErrorInvalidValue;
@@ -610,6 +642,8 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     sp.keymax = keymax;
     sp.nkeymin = nkeymin;
     sp.status = status;
+    sp.zero = reinterpret_cast<uint4 *>(p8 + L.zero);
+    sp.zero_n16 = (int64_t)(L.zero_bytes / 16);
     sp.T = T;
     sp.HI = HI;
     sp.dI = dI;
@@ -628,14 +662,17 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (T > k) {
         const dim3 g2((unsigned)((T + TK_CHUNK - 1) / TK_CHUNK), (unsigned)B);
-        topk_hist_kernel<<<g2, TK_THREADS, 0, stream>>>(scores, T, keymax, nkeymin, hist);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        topk_collect_kernel<<<g2, TK_THREADS, 0, stream>>>(scores, T, k, keymax, nkeymin, hist, bitmap, ncand, cand);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_dependent(topk_hist_kernel, g2, dim3(TK_THREADS), 0, stream, (const float *)scores, T,
+                             (const uint32_t *)keymax, (const uint32_t *)nkeymin, hist);
+        if (e != cudaSuccess) return e;
+        e = launch_dependent(topk_collect_kernel, g2, dim3(TK_THREADS), 0, stream, (const float *)scores, T, k,
+                             (const uint32_t *)keymax, (const uint32_t *)nkeymin, (const uint32_t *)hist, bitmap, ncand,
+                             cand);
+        if (e != cudaSuccess) return e;
     }
-    topk_final_kernel<<<(unsigned)B, FIN_THREADS, 0, stream>>>(scores, T, k, keymax, nkeymin, hist, bitmap, ncand, cand,
-                                                               idx);
-    return cudaGetLastError();
+    return launch_dependent(topk_final_kernel, dim3((unsigned)B), dim3(FIN_THREADS), 0, stream, (const float *)scores, T,
+                            k, (const uint32_t *)keymax, (const uint32_t *)nkeymin, (const uint32_t *)hist, bitmap,
+                            (const uint32_t *)ncand, (const uint2 *)cand, idx);
 }
 
 }  // namespace csa

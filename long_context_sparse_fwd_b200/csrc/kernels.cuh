@@ -21,6 +21,7 @@ struct AttnArgs {
     int32_t *status;           // workspace status word
     int64_t R, T, P;           // rows, entries (per row for decode), decode position
     int H, D, k, W, r, m, decode;
+    int after_kernel;          // launch as a programmatic dependent of the kernel before it in the stream
     float scale;
     double log2_theta_tok, log2_theta_cmp;
 };
@@ -72,6 +73,7 @@ size_t decode_workspace_min(int64_t B, int64_t T, int32_t k);
 
 // decode_tc.cu: decode index scan (tcgen05, HBM streaming) + two-stage exact top-k
 size_t decode_index_workspace(int64_t B, int64_t T, int k);
+size_t decode_index_head_bytes(int64_t B);   // leading bytes of its workspace the caller zeroes
 bool decode_index_tc_supported(int64_t T, int HI, int dI, int k);
 cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t B, int64_t T, int HI,
                                    int dI, int k, int32_t *idx, void *ws, int32_t *status, cudaStream_t stream);
