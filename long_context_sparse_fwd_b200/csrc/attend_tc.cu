@@ -184,6 +184,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint64_t *kv_wfull = bars + 25;    // [stage] loader arrivals, window blocks
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 28);
     volatile int *abort = reinterpret_cast<volatile int *>(bars + 29);
+    uint64_t *tab_ready = bars + 30;   // single use: the first query's rope tables are written
     int *elist_all = reinterpret_cast<int *>(smem + OFF_LIST);    // [slot][kcap]
     const int kcap = (max(a.k, 1) + 3) & ~3;
 
@@ -210,6 +211,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_init(q_free, 1);
         mbar_init(q_ready, LOAD_THREADS);
         mbar_init(drain, 1);
+        mbar_init(tab_ready, 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -221,13 +223,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_ptr;
-    grid_dependency_wait();   // the index lists (decode: written by the top-k kernel just before)
+    // Launched as a programmatic dependent (decode), this grid may start before the top-k kernel
+    // that writes the index lists has finished: only the planner waits for it, right before it
+    // reads the first list, so the rope tables and the first query's Q load overlap that kernel.
     grid_launch_dependents();
 
     if (warp == PLAN_WARP) {
         // ====== planner: index list, block split and rope tables of each query; window rope turn ======
         int g = 0;           // key blocks of this CTA's earlier queries
         uint32_t wpar = 0;   // per stage: parity of the next kv_wfull completion
+        bool dep_waited = false;
         for (int64_t n = 0;; ++n) {
             const int64_t u = blockIdx.x + n * gridDim.x;
             if (u >= units) break;
@@ -243,6 +248,29 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int64_t vis = a.decode ? a.T : visible_entries(t, a.m, a.T);
             const int64_t wpos0 = max((int64_t)0, t - a.W + 1);
             const int nw = (int)(t - wpos0 + 1);
+            {   // rope tables: angle t * f_p (f_p = theta^(-2p/64)) for both thetas, and their difference
+                float *rt = rope_tab + s * ROPE_TAB;
+                float c, sn;
+                rope_cos_sin((double)t, lane, RR, a.log2_theta_tok, &c, &sn);
+                rt[lane * 2] = c;
+                rt[lane * 2 + 1] = sn;
+                rope_cos_sin((double)t, lane, RR, a.log2_theta_cmp, &c, &sn);
+                rt[64 + lane * 2] = c;
+                rt[64 + lane * 2 + 1] = sn;
+                const double e = -(2.0 * lane / (double)RR);
+                const double dang = (double)t * (exp2(e * a.log2_theta_cmp) - exp2(e * a.log2_theta_tok));
+                double sd, cd;
+                sincos(dang, &sd, &cd);
+                rt[128 + lane * 2] = (float)cd;
+                rt[128 + lane * 2 + 1] = (float)sd;
+            }
+            if (n == 0) {   // the loaders write this query's Q into TMEM as soon as its tables exist
+                __threadfence_block();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tab_ready);
+                grid_dependency_wait();   // the index lists
+                dep_waited = true;
+            }
             int *elist = elist_all + s * kcap;
             int ne;
             if (a.idx != nullptr) {   // compacted entry list (CSA); HCA uses entries 0..vis-1 directly
@@ -264,22 +292,6 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             } else {
                 ne = (int)vis;
             }
-            {   // rope tables: angle t * f_p (f_p = theta^(-2p/64)) for both thetas, and their difference
-                float *rt = rope_tab + s * ROPE_TAB;
-                float c, sn;
-                rope_cos_sin((double)t, lane, RR, a.log2_theta_tok, &c, &sn);
-                rt[lane * 2] = c;
-                rt[lane * 2 + 1] = sn;
-                rope_cos_sin((double)t, lane, RR, a.log2_theta_cmp, &c, &sn);
-                rt[64 + lane * 2] = c;
-                rt[64 + lane * 2 + 1] = sn;
-                const double e = -(2.0 * lane / (double)RR);
-                const double dang = (double)t * (exp2(e * a.log2_theta_cmp) - exp2(e * a.log2_theta_tok));
-                double sd, cd;
-                sincos(dang, &sd, &cd);
-                rt[128 + lane * 2] = (float)cd;
-                rt[128 + lane * 2 + 1] = (float)sd;
-            }
             if (lane == 0) {
                 const int nbw = (nw + KB - 1) / KB, nb_all = nbw + (ne + KB - 1) / KB;
                 Plan p;
@@ -298,9 +310,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&plan_ready[s]);
 
+            const Plan pl = plans[s];
             // Turn the rope slice of this unit's window keys (see the header) once each window
             // block has landed; the MMA waits for kv_rdy on window blocks.
-            const Plan pl = plans[s];
             const float *dt = rope_tab + s * ROPE_TAB + 128;
             bool ok = true;
             for (int b = 0; b < pl.nb && pl.gb0 + b < pl.nbw; ++b) {
@@ -334,6 +346,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (!ok) break;
             g += pl.nb;
         }
+        if (!dep_waited) grid_dependency_wait();   // never finish before the kernel this one depends on
     } else if (warp < 4) {
         // =============== softmax + epilogue (warp w owns TMEM quarter w: heads 16w..16w+15) ===============
         const int hl = lane & 15, hf = lane >> 4;   // head of this thread, which half of the columns
@@ -494,8 +507,52 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             prefetch_tmap(&tm_c);
             prefetch_tmap(&tm_w);
         }
+        // Q of a query into TMEM: thread (hl, hf) writes head 16*lw+hl, dims 64c + 32hf .. +31 of each
+        // chunk c. Chunks 0-3 are loaded before `ready` (every S of the previous query has completed)
+        // is awaited, 4-7 (L2 hits after the planner's prefetch) once the first half is in TMEM.
+        auto load_q = [&](int64_t row, const float *rope_cs, uint64_t *ready, uint32_t ready_par) -> bool {
+            const uint4 *qsrc = reinterpret_cast<const uint4 *>(a.q + (row * HH + lw * 16 + hl) * (int64_t)DD + hf * 32);
+            uint4 x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + (i >> 2) * 8 + (i & 3), pol_once);
+            if (!__all_sync(0xffffffffu, mbar_wait(ready, ready_par, abort, a.status))) return false;
+            tc_fence_after();
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                if (half == 1) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + 32 + (i >> 2) * 8 + (i & 3), pol_once);
+                }
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int c = half * 4 + cc;
+                    const uint32_t wq[16] = {x[4 * cc].x,     x[4 * cc].y,     x[4 * cc].z,     x[4 * cc].w,
+                                             x[4 * cc + 1].x, x[4 * cc + 1].y, x[4 * cc + 1].z, x[4 * cc + 1].w,
+                                             x[4 * cc + 2].x, x[4 * cc + 2].y, x[4 * cc + 2].z, x[4 * cc + 2].w,
+                                             x[4 * cc + 3].x, x[4 * cc + 3].y, x[4 * cc + 3].z, x[4 * cc + 3].w};
+                    if (c < NCH - 1) {
+                        tmem_st_half16u(tqq + c * 32, wq);
+                    } else {   // rope dims: rotated with theta_cmp
+                        uint32_t r[16];
+                        rotate16(wq, rope_cs + 64, hf * 16, r);
+                        tmem_st_half16u(tqq + 7 * 32, r);
+                    }
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(q_ready);
+            return true;
+        };
+        // The first query's Q needs no plan: it is written as soon as the planner's rope tables exist
+        // (before the index lists are awaited), while its first keys are being planned.
+        bool run = true;
+        if ((int64_t)blockIdx.x < units) {
+            const int64_t u0 = blockIdx.x;
+            run = load_q(a.decode ? u0 / a.nsplit : a.S - 1 - u0, rope_tab, tab_ready, 0u);
+        }
         int g = 0;
-        for (int64_t n = 0;; ++n) {
+        for (int64_t n = 0; run; ++n) {
             const int64_t u = blockIdx.x + n * gridDim.x;
             if (u >= units) break;
             const int s = (int)(n & 1);
@@ -506,45 +563,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int64_t ent_row0 = a.decode ? pl.row * a.T : 0;   // row of entry 0 in the entry tensor map
             bool ok = true;
             for (int b = 0; b <= pl.nb; ++b) {
-                if (b == min(1, pl.nb)) {
-                    // Q of this query into TMEM, once every S of the previous query has completed:
-                    // thread (hl, hf) writes head 16*lw+hl, dims 64c + 32hf .. +31 of each chunk c
-                    const uint4 *qsrc = reinterpret_cast<const uint4 *>(a.q + (pl.row * HH + lw * 16 + hl) * (int64_t)DD + hf * 32);
-                    // chunks 0-3 are loaded before the wait, 4-7 (L2 hits after the planner's
-                    // prefetch) once the first half is in TMEM
-                    uint4 x[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + (i >> 2) * 8 + (i & 3), pol_once);
-                    if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(q_free, (uint32_t)((n - 1) & 1), abort, a.status))) {
+                if (n > 0 && b == min(1, pl.nb)) {
+                    // Q of this query, once every S of the previous query has completed
+                    if (!load_q(pl.row, rope_cs, q_free, (uint32_t)((n - 1) & 1))) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int half = 0; half < 2; ++half) {
-                        if (half == 1) {
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + 32 + (i >> 2) * 8 + (i & 3), pol_once);
-                        }
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int c = half * 4 + cc;
-                            const uint32_t wq[16] = {x[4 * cc].x,     x[4 * cc].y,     x[4 * cc].z,     x[4 * cc].w,
-                                                     x[4 * cc + 1].x, x[4 * cc + 1].y, x[4 * cc + 1].z, x[4 * cc + 1].w,
-                                                     x[4 * cc + 2].x, x[4 * cc + 2].y, x[4 * cc + 2].z, x[4 * cc + 2].w,
-                                                     x[4 * cc + 3].x, x[4 * cc + 3].y, x[4 * cc + 3].z, x[4 * cc + 3].w};
-                            if (c < NCH - 1) {
-                                tmem_st_half16u(tqq + c * 32, wq);
-                            } else {   // rope dims: rotated with theta_cmp
-                                uint32_t r[16];
-                                rotate16(wq, rope_cs + 64, hf * 16, r);
-                                tmem_st_half16u(tqq + 7 * 32, r);
-                            }
-                        }
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    mbar_arrive(q_ready);
                 }
                 if (b == pl.nb) break;
                 const int gg = g + b;
