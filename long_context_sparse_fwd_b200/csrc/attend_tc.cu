@@ -19,8 +19,10 @@
 //   TMEM (M=64 uses 16 lanes of each 32-lane quarter, "half 0" = lanes +0..15, "half 1" = +16..31):
 //     half 0: S_b   cols [0,64), [64,128)   double-buffered logits (on the lanes of Q, as the
 //                                  A-from-TMEM MMA requires)
-//             Q     cols [128,384) 8 chunks of 64 dims (32 columns, 2 bf16 each), the rope chunk
-//                                  rotated with theta_cmp
+//             Q     cols [128,512) a ring of 12 chunk slots (32 columns each: 64 dims as bf16
+//                                  pairs); query n puts its chunk c (the rope chunk rotated
+//                                  with theta_cmp) in slot (8n + c) mod 12, so the next query's
+//                                  chunks 0-3 are written while the current one still computes
 //     half 1: O     cols [0,512)   output dims 0..511
 // The two branches rotate their rope slices with different thetas. Once a window block has
 // landed, the planner turns the rope slice of each window key by t * (f_cmp - f_tok) per pair
@@ -73,6 +75,11 @@ constexpr int PLAN_CONSUMERS = 4 + 1 + 4;       // loader warps, MMA warp (one a
 constexpr float TAU = 8.f;
 constexpr uint32_t LANE16 = 16u << 16;
 constexpr uint32_t COL_S = 0, COL_Q = 128;   // half 0
+constexpr int QSLOTS = 12;                   // Q chunk slots (32 columns each) from COL_Q
+
+// TMEM slot of chunk c of the CTA's n-th query: consecutive queries share no slot of their first
+// four chunks with the query before, so those are written before that query's last S completes.
+__device__ __forceinline__ uint32_t q_slot(int64_t n, int c) { return (uint32_t)((8 * (int)(n % 3) + c) % QSLOTS); }
 constexpr uint32_t COL_O2 = 256;             // half 1: O dims 256..511 (dims 0..255 at column 0)
 constexpr int ROPE_TAB = 3 * 32 * 2;         // floats per slot: [tok, cmp, cmp - tok][pair][cos, sin]
 constexpr uint32_t TMEM_COLS = 512;
@@ -125,6 +132,14 @@ __device__ __forceinline__ uint4 ldg_hint(const uint4 *p, uint64_t policy)
     return v;
 }
 
+// Registers written by a tcgen05.ld are read only after tcgen05.wait::ld: this empty asm, placed
+// after the wait, keeps the compiler from moving their uses above it.
+__device__ __forceinline__ void reg_fence(float (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 32; ++i) asm volatile("" : "+f"(v[i]));
+}
+
 // Wait (at most 100 ms) for a phase regardless of the abort flag: used before exit so that no
 // copy or MMA is still writing this CTA's shared memory or TMEM.
 __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
@@ -153,7 +168,7 @@ __device__ __forceinline__ void rotate16(const uint32_t (&w)[16], const float *c
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
-                 const __grid_constant__ CUtensorMap tm_w, TcArgs a)
+                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_o, TcArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -313,7 +328,16 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const Plan pl = plans[s];
             // Turn the rope slice of this unit's window keys (see the header) once each window
             // block has landed; the MMA waits for kv_rdy on window blocks.
-            const float *dt = rope_tab + s * ROPE_TAB + 128;
+            // lane l always turns 16-byte unit (l & 7) of a key row: pairs 4(l & 7) .. +3
+            float tc4[4], ts4[4];
+            {
+                const float *dt = rope_tab + s * ROPE_TAB + 128;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    tc4[e] = dt[((lane & 7) * 4 + e) * 2];
+                    ts4[e] = dt[((lane & 7) * 4 + e) * 2 + 1];
+                }
+            }
             bool ok = true;
             for (int b = 0; b < pl.nb && pl.gb0 + b < pl.nbw; ++b) {
                 const int gg = g + b, st = gg % NSTAGE;
@@ -323,21 +347,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 wpar ^= 1u << st;
                 uint8_t *rope_rows = sKV + st * STAGE + (NCH - 1) * KCHUNK;   // dims 448..511 of each key
-#pragma unroll 4
-                for (int i = lane; i < KB * 8; i += 32) {
-                    const int key = i >> 3, uu = i & 7;   // 16-byte unit uu: pairs 4uu .. 4uu+3
-                    uint4 *ptr = reinterpret_cast<uint4 *>(rope_rows + sw128(key, uu));
-                    const uint4 v = *ptr;
-                    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+                uint4 v[16];   // all 16 of this lane's units (rows 4j + lane/8) loaded before any is turned
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    v[j] = *reinterpret_cast<const uint4 *>(rope_rows + sw128(j * 4 + (lane >> 3), lane & 7));
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
                     uint32_t o4[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int pp = uu * 4 + e;
                         const float x0 = bf_lo(w4[e]), x1 = bf_hi(w4[e]);
-                        const float c = dt[pp * 2], sn = dt[pp * 2 + 1];
-                        o4[e] = pack_bf2(x0 * c - x1 * sn, x0 * sn + x1 * c);
+                        o4[e] = pack_bf2(x0 * tc4[e] - x1 * ts4[e], x0 * ts4[e] + x1 * tc4[e]);
                     }
-                    *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                    *reinterpret_cast<uint4 *>(rope_rows + sw128(j * 4 + (lane >> 3), lane & 7)) =
+                        make_uint4(o4[0], o4[1], o4[2], o4[3]);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -355,6 +379,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const uint32_t tq1 = tq0 + LANE16;                            // half 1
         // the sink seeds the running max and sum; split partials leave it to the combine step
         const float zl = partial ? -INFINITY : a.sinks[h] * 1.4426950408889634f;
+        if (threadIdx.x == 0) prefetch_tmap(&tm_o);
         int g = 0;   // key blocks of this CTA's earlier queries
         bool ok = true;
         for (int64_t n = 0;; ++n) {
@@ -443,13 +468,40 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 // leaves as whole 128-byte row segments, 8 lanes per segment.
                 uint8_t *stage0 = sP + warp * 2048, *stage1 = sP + PBUF + warp * 2048;
                 uint8_t *mine = (hf ? stage1 : stage0) + hl * 128;
-                float *obase = a.o + (orow * HH + warp * 16) * (int64_t)DD;
+                // Each staged piece leaves as two TMA tensor stores ([16 heads x 32 dims] each) issued by
+                // lane 0, which also waits for the engine to have read the staging before it is reused.
+                const int orow0 = (int)(orow * HH + warp * 16);
+                auto emit = [&](float (&v)[32], int c) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] *= inv;
+                    if (lane == 0) bulk_wait_read_all();
+                    __syncwarp();
+#pragma unroll
+                    for (int uq = 0; uq < 8; ++uq)
+                        *reinterpret_cast<float4 *>(mine + ((uq ^ (hl & 7)) << 4)) =
+                            make_float4(v[4 * uq], v[4 * uq + 1], v[4 * uq + 2], v[4 * uq + 3]);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_o, stage0, c, orow0);
+                        tma_store_2d(&tm_o, stage1, c + 32, orow0);
+                        bulk_commit();
+                    }
+                };
+                // The TMEM load of the next piece is in flight while the current one is written out.
+                float va[32], vb[32];
+                tmem_ld_half32(tq1, va);
 #pragma unroll 1
-                for (int c = 0; c < DD; c += 64) {
-                    float v[32];
-                    tmem_ld_half32(tq1 + (uint32_t)c, v);
+                for (int c = 0; c < DD; c += 128) {
                     tmem_wait_ld();
-                    if (c == DD - 64) {
+                    reg_fence(va);
+                    tmem_ld_half32(tq1 + (uint32_t)(c + 64), vb);
+                    emit(va, c);
+                    tmem_wait_ld();
+                    reg_fence(vb);
+                    if (c + 128 < DD) {
+                        tmem_ld_half32(tq1 + (uint32_t)(c + 128), va);
+                    } else {
                         tc_fence_before();
                         mbar_arrive(o_free);   // O has been read: the next query's P V may overwrite it
                         // rope dims 448..511: rotated back by -t * f_cmp (window keys were turned to match)
@@ -457,26 +509,15 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         for (int j = 0; j < 32; j += 2) {
                             const int p = hf * 16 + (j >> 1);
                             const float cc = rope_cmp[p * 2], sc = rope_cmp[p * 2 + 1];
-                            const float e0 = v[j], e1 = v[j + 1];
-                            v[j] = e0 * cc + e1 * sc;
-                            v[j + 1] = -e0 * sc + e1 * cc;
+                            const float e0 = vb[j], e1 = vb[j + 1];
+                            vb[j] = e0 * cc + e1 * sc;
+                            vb[j + 1] = -e0 * sc + e1 * cc;
                         }
                     }
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) v[j] *= inv;
-#pragma unroll
-                    for (int uq = 0; uq < 8; ++uq)
-                        *reinterpret_cast<float4 *>(mine + ((uq ^ (hl & 7)) << 4)) =
-                            make_float4(v[4 * uq], v[4 * uq + 1], v[4 * uq + 2], v[4 * uq + 3]);
-                    __syncwarp();
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int rr = i * 4 + (lane >> 3), uq = lane & 7;   // staged row rr
-                        const float4 x = *reinterpret_cast<const float4 *>((rr >= 16 ? stage1 : stage0) + sw128(rr & 15, uq));
-                        __stcs(reinterpret_cast<float4 *>(obase + (rr & 15) * (int64_t)DD + c + (rr >> 4) * 32 + uq * 4), x);
-                    }
-                    __syncwarp();
+                    emit(vb, c + 64);
                 }
+                if (lane == 0) bulk_wait_read_all();   // the P buffers are written again by the next query
+                __syncwarp();
             } else {
                 tc_fence_before();
                 mbar_arrive(o_free);
@@ -494,6 +535,8 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (lane == 0) mbar_arrive(&plan_free[s]);
             g += nb;
         }
+        if (lane == 0) bulk_wait_all();   // every output store of this warp has completed
+        __syncwarp();
     } else if (warp >= LOAD_WARP0 && warp < MMA_WARP) {
         // ===== key loads (TMA into the swizzled stages) and Q into TMEM quarter lw =====
         const int lw = warp - LOAD_WARP0;        // key rows 16*lw .. 16*lw+15 of each block; heads 16*lw..
@@ -507,21 +550,21 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             prefetch_tmap(&tm_c);
             prefetch_tmap(&tm_w);
         }
-        // Q of a query into TMEM: thread (hl, hf) writes head 16*lw+hl, dims 64c + 32hf .. +31 of each
-        // chunk c. Chunks 0-3 are loaded before `ready` (every S of the previous query has completed)
-        // is awaited, 4-7 (L2 hits after the planner's prefetch) once the first half is in TMEM.
-        auto load_q = [&](int64_t row, const float *rope_cs, uint64_t *ready, uint32_t ready_par) -> bool {
+        // Q of the CTA's query qn into TMEM: thread (hl, hf) writes head 16*lw+hl, dims 64c + 32hf .. +31
+        // of each chunk c. Chunks 0-3 go to slots that no S in flight reads (the query before last
+        // has completed, which the previous call awaited), so they are written at once; chunks 4-7,
+        // whose slots held chunks 0-3 of the previous query, once `ready` (every S of the previous
+        // query has completed; for the first query, the rope tables exist) has completed.
+        auto load_q = [&](int64_t qn, int64_t row, const float *rope_cs, uint64_t *ready, uint32_t ready_par) -> bool {
             const uint4 *qsrc = reinterpret_cast<const uint4 *>(a.q + (row * HH + lw * 16 + hl) * (int64_t)DD + hf * 32);
             uint4 x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + (i >> 2) * 8 + (i & 3), pol_once);
-            if (!__all_sync(0xffffffffu, mbar_wait(ready, ready_par, abort, a.status))) return false;
-            tc_fence_after();
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
-                if (half == 1) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + 32 + (i >> 2) * 8 + (i & 3), pol_once);
+                for (int i = 0; i < 16; ++i) x[i] = ldg_hint(qsrc + half * 32 + (i >> 2) * 8 + (i & 3), pol_once);
+                if (half == 1) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(ready, ready_par, abort, a.status))) return false;
+                    tc_fence_after();
                 }
 #pragma unroll
                 for (int cc = 0; cc < 4; ++cc) {
@@ -530,12 +573,13 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                              x[4 * cc + 1].x, x[4 * cc + 1].y, x[4 * cc + 1].z, x[4 * cc + 1].w,
                                              x[4 * cc + 2].x, x[4 * cc + 2].y, x[4 * cc + 2].z, x[4 * cc + 2].w,
                                              x[4 * cc + 3].x, x[4 * cc + 3].y, x[4 * cc + 3].z, x[4 * cc + 3].w};
+                    const uint32_t ta = tqq + q_slot(qn, c) * 32;
                     if (c < NCH - 1) {
-                        tmem_st_half16u(tqq + c * 32, wq);
+                        tmem_st_half16u(ta, wq);
                     } else {   // rope dims: rotated with theta_cmp
                         uint32_t r[16];
                         rotate16(wq, rope_cs + 64, hf * 16, r);
-                        tmem_st_half16u(tqq + 7 * 32, r);
+                        tmem_st_half16u(ta, r);
                     }
                 }
             }
@@ -549,7 +593,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool run = true;
         if ((int64_t)blockIdx.x < units) {
             const int64_t u0 = blockIdx.x;
-            run = load_q(a.decode ? u0 / a.nsplit : a.S - 1 - u0, rope_tab, tab_ready, 0u);
+            run = load_q(0, a.decode ? u0 / a.nsplit : a.S - 1 - u0, rope_tab, tab_ready, 0u);
         }
         int g = 0;
         for (int64_t n = 0; run; ++n) {
@@ -565,7 +609,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int b = 0; b <= pl.nb; ++b) {
                 if (n > 0 && b == min(1, pl.nb)) {
                     // Q of this query, once every S of the previous query has completed
-                    if (!load_q(pl.row, rope_cs, q_free, (uint32_t)((n - 1) & 1))) {
+                    if (!load_q(n, pl.row, rope_cs, q_free, (uint32_t)((n - 1) & 1))) {
                         ok = false;
                         break;
                     }
@@ -737,7 +781,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         const uint32_t d = tmem + COL_S + (uint32_t)(gs & 1) * 64;
 #pragma unroll
                         for (int dc = 0; dc < NCH; ++dc) {
-                            const uint32_t qa = tmem + COL_Q + (uint32_t)dc * 32;
+                            const uint32_t qa = tmem + COL_Q + q_slot(n, dc) * 32;
                             const uint64_t kb = dK + ((sst * STAGE + dc * KCHUNK) >> 4);
 #pragma unroll
                             for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(d, qa + ks * 8, kb + 2 * ks, idS, (dc | ks) != 0);
@@ -893,6 +937,9 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
         tw = tq;   // no window rows: never used
     }
     a.o = out_rows;   // final rows, or the split partials
+    CUtensorMap to;   // output rows [R * 64 (or R * nsplit * 64), 512] fp32, stored as [16 x 32] boxes
+    const uint64_t o_rows = (uint64_t)x.R * (uint64_t)nsplit * HH;
+    if (o_rows >= (1ull << 31) || !make_tmap_f32_sw128(&to, out_rows, o_rows, DD, 16)) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(attend_tc_kernel), smem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM walks the units (query rows, or sequence splits) with stride grid
@@ -900,8 +947,9 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     if ((e = current_device_sms(&dev, &sms)) != cudaSuccess) return e;
     const int64_t units = x.R * nsplit;
     const unsigned grid = (unsigned)std::min<int64_t>(units, std::max(sms, 1));
-    if (x.after_kernel) return launch_dependent(attend_tc_kernel, dim3(grid), dim3(NUM_THREADS), smem, stream, tq, tc, tw, a);
-    attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tc, tw, a);
+    if (x.after_kernel)
+        return launch_dependent(attend_tc_kernel, dim3(grid), dim3(NUM_THREADS), smem, stream, tq, tc, tw, to, a);
+    attend_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tc, tw, to, a);
     return cudaGetLastError();
 }
 
