@@ -31,8 +31,9 @@ namespace {
 
 constexpr int BM = 128;          // entries per tile = TMEM lanes
 constexpr int BN = 256;          // (query, head) columns
-constexpr int NUM_THREADS = 320;
 constexpr int EPI_THREADS = 256;       // warps 2-9: two warps per TMEM lane quarter, each half of the queries
+constexpr int TOPK_THREADS = 256;      // warps 10-17: four pairs, one query each at a time
+constexpr int NUM_THREADS = 64 + EPI_THREADS + TOPK_THREADS;
 constexpr uint32_t TMEM_COLS = 512;
 
 struct IdxParams {
@@ -40,7 +41,9 @@ struct IdxParams {
     int32_t *idx;        // [S, k]
     int32_t *status;
     int64_t S, T;
+    int64_t ngroups;     // groups of Q consecutive queries
     int HI, dI, m, k, Q, stages, T_cap;
+    int nsb;             // scores buffers (2: the top-k of a group overlaps the next group's scoring)
 };
 
 // Exact top-k of one query's scores by one warp: radix select over order-preserving keys, starting
@@ -440,28 +443,42 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t a_bytes = (uint32_t)kchunks * BM * 128;
     uint8_t *sB = smem;
     uint8_t *sA = sB + b_bytes;
-    float *scores = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [Q][T_cap]
-    float *sw = scores + (size_t)p.Q * p.T_cap;                                  // [BN]
-    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                      // [4 pairs][PBINS + 80]
+    float *scores_all = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [nsb][Q][T_cap]
+    float *sw = scores_all + (size_t)p.nsb * p.Q * p.T_cap;                          // [BN]
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                          // [4 pairs][PBINS + 80]
     uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 4 * (PBINS + 80));
-    uint64_t *full = bars;                   // [stages]
-    uint64_t *empty = bars + 8;              // [stages]
-    uint64_t *tfull = bars + 16;             // [2]
-    uint64_t *tempty = bars + 18;            // [2]
-    uint64_t *qfull = bars + 20;
-    uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(bars + 21);
-    volatile int *abort = reinterpret_cast<volatile int *>(bars + 22);
+    uint64_t *full = bars;                   // [stages] k^I tile landed
+    uint64_t *empty = bars + 8;              // [stages] its MMAs completed
+    uint64_t *tfull = bars + 16;             // [2] accumulator written
+    uint64_t *tempty = bars + 18;            // [2] accumulator read by the 256 epilogue threads
+    uint64_t *qfull = bars + 20;             // q^I of the group landed
+    uint64_t *qempty = bars + 21;            // every MMA of the group completed: q^I may be replaced
+    uint64_t *sfull = bars + 22;             // [2] scores buffer complete (8 epilogue warps)
+    uint64_t *sempty = bars + 24;            // [2] scores buffer consumed by the top-k (8 warps)
+    uint32_t *tmem_base_ptr = reinterpret_cast<uint32_t *>(bars + 26);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 27);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t0 = (int64_t)blockIdx.x * p.Q;
-    const int64_t t_last = min(t0 + p.Q - 1, p.S - 1);
-    const int64_t vis_max = visible_entries(t_last, p.m, p.T);
-    const int ntiles = (int)((vis_max + BM - 1) / BM);
+    // Groups of Q consecutive queries, the ones that see the most entries first, dealt round-robin.
+    auto group_of = [&](int64_t gi, int64_t *t0, int *ntiles) -> bool {
+        const int64_t G = blockIdx.x + gi * gridDim.x;
+        if (G >= p.ngroups) return false;
+        *t0 = (p.ngroups - 1 - G) * p.Q;
+        const int64_t t_last = min(*t0 + p.Q - 1, p.S - 1);
+        *ntiles = (int)((visible_entries(t_last, p.m, p.T) + BM - 1) / BM);
+        return true;
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < p.stages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], EPI_THREADS); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], EPI_THREADS);
+            mbar_init(&sfull[i], EPI_THREADS / 32);
+            mbar_init(&sempty[i], TOPK_THREADS / 32);
+        }
         mbar_init(qfull, 1);
+        mbar_init(qempty, 1);
         *abort = 0;
         fence_barrier_init();
     }
@@ -469,129 +486,191 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tmem_alloc(tmem_base_ptr, TMEM_COLS);
         tmem_relinquish();
     }
-    if (warp >= 2) {   // index weights of this block's queries
-        for (int i = threadIdx.x - 64; i < p.Q * p.HI; i += EPI_THREADS) {
-            const int64_t t = t0 + i / p.HI;
-            sw[i] = t < p.S ? p.w[t * p.HI + (i % p.HI)] : 0.f;
-        }
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_base_ptr;
 
-    if (warp == 0 && ntiles > 0) {
+    if (warp == 0) {
         // ---------------- TMA producer (warp-wide loop, one elected lane issues) ----------------
         if (elect_one()) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
-            mbar_arrive_expect_tx(qfull, b_bytes);
-            for (int c = 0; c < kchunks; ++c)
-                tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
         }
         __syncwarp();
-        int issued = 0;
-        for (int i = 0; i < ntiles; ++i) {
-            const int st = i % p.stages;
-            if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((i / p.stages) & 1) ^ 1, abort, p.status))) break;
+        int tile = 0, issued = 0;
+        int64_t ngr = 0;
+        bool ok = true;
+        int64_t t0;
+        int ntiles;
+        for (int64_t gi = 0; ok && group_of(gi, &t0, &ntiles); ++gi) {
+            // q^I of this group once every MMA of the previous group has completed
+            if (gi > 0 && !__all_sync(0xffffffffu, mbar_wait(qempty, (uint32_t)((gi - 1) & 1), abort, p.status))) break;
             if (elect_one()) {
-                mbar_arrive_expect_tx(&full[st], a_bytes);
+                mbar_arrive_expect_tx(qfull, b_bytes);
                 for (int c = 0; c < kchunks; ++c)
-                    tma_load_2d(sA + (size_t)st * a_bytes + (size_t)c * BM * 128, &tm_k, &full[st], c * 64, i * BM);
+                    tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
             }
             __syncwarp();
-            issued = i + 1;
+            ngr = gi + 1;
+            for (int i = 0; i < ntiles; ++i, ++tile) {
+                const int st = tile % p.stages;
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((tile / p.stages) & 1) ^ 1, abort, p.status))) {
+                    ok = false;
+                    break;
+                }
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[st], a_bytes);
+                    for (int c = 0; c < kchunks; ++c)
+                        tma_load_2d(sA + (size_t)st * a_bytes + (size_t)c * BM * 128, &tm_k, &full[st], c * 64, i * BM);
+                }
+                __syncwarp();
+                issued = tile + 1;
+            }
         }
         // never leave with copies in flight into this CTA's shared memory
-        mbar_wait(qfull, 0, abort, p.status, 100000000ull);
+        if (ngr > 0) mbar_wait(qfull, (uint32_t)((ngr - 1) & 1), abort, p.status, 100000000ull);
         for (int i = max(0, issued - p.stages); i < issued; ++i)
             mbar_wait(&full[i % p.stages], (i / p.stages) & 1, abort, p.status, 100000000ull);
-    } else if (warp == 1 && ntiles > 0) {
+    } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         const uint32_t idesc = idesc_bf16(BM, BN);
-        bool ok = mbar_wait(qfull, 0, abort, p.status);
-        int issued = 0;
-        for (int i = 0; ok && i < ntiles; ++i) {
-            const int st = i % p.stages, buf = i & 1;
-            if (!mbar_wait(&tempty[buf], ((i >> 1) & 1) ^ 1, abort, p.status)) break;
-            if (!mbar_wait(&full[st], (i / p.stages) & 1, abort, p.status)) break;
-            tc_fence_after();
-            if (elect_one()) {
-                const uint32_t a0 = smem_u32(sA + (size_t)st * a_bytes), b0 = smem_u32(sB);
-                for (int c = 0; c < kchunks; ++c) {
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = sdesc_sw128(a0 + c * BM * 128 + ks * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(b0 + c * BN * 128 + ks * 32, 16, 1024);
-                        mma_bf16(tmem_base + buf * BN, ad, bd, idesc, (c | ks) != 0);
-                    }
+        int tile = 0;
+        bool ok = true;
+        int64_t t0;
+        int ntiles;
+        for (int64_t gi = 0; ok && group_of(gi, &t0, &ntiles); ++gi) {
+            if (!__all_sync(0xffffffffu, mbar_wait(qfull, (uint32_t)(gi & 1), abort, p.status))) break;
+            for (int i = 0; i < ntiles; ++i, ++tile) {
+                const int st = tile % p.stages, buf = tile & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((tile >> 1) & 1) ^ 1, abort, p.status)) ||
+                    !__all_sync(0xffffffffu, mbar_wait(&full[st], (tile / p.stages) & 1, abort, p.status))) {
+                    ok = false;
+                    break;
                 }
-                mma_commit(&empty[st]);
-                mma_commit(&tfull[buf]);
+                tc_fence_after();
+                if (elect_one()) {
+                    const uint32_t a0 = smem_u32(sA + (size_t)st * a_bytes), b0 = smem_u32(sB);
+                    for (int c = 0; c < kchunks; ++c) {
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad = sdesc_sw128(a0 + c * BM * 128 + ks * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(b0 + c * BN * 128 + ks * 32, 16, 1024);
+                            mma_bf16(tmem_base + buf * BN, ad, bd, idesc, (c | ks) != 0);
+                        }
+                    }
+                    mma_commit(&empty[st]);
+                    mma_commit(&tfull[buf]);
+                }
+                __syncwarp();
             }
+            if (!ok) break;
+            if (elect_one()) mma_commit(qempty);   // q^I is free once this group's MMAs complete
             __syncwarp();
-            issued = i + 1;
         }
-        if (issued > 0) {   // the last accumulator must be complete before TMEM is released
-            const int i = issued - 1;
-            mbar_wait(&tfull[i & 1], (i >> 1) & 1, abort, p.status, 100000000ull);
-        }
-    } else if (warp >= 2) {
+        // every MMA issued must be complete before TMEM is released: the last accumulator's commit
+        // arrives once it and every earlier MMA have completed
+        if (tile > 0) mbar_wait(&tfull[(tile - 1) & 1], ((tile - 1) >> 1) & 1, abort, p.status, 100000000ull);
+    } else if (warp < 2 + EPI_THREADS / 32) {
         // ---------------- epilogue: scores into shared memory ----------------
         // warp w reads TMEM lane quarter w % 4 (entries 32*(w%4) .. +31 of the tile); warps 2-5 take
-        // the first half of the block's queries, warps 6-9 the second half
+        // the first half of the group's queries, warps 6-9 the second half
         const int quarter = warp & 3;
         const int qhalf = (warp - 2) >> 2;
         const int qlo = qhalf * (p.Q >> 1), qhi = qlo + (p.Q >> 1);   // Q = 256 / HI is even
-        for (int i = 0; i < ntiles; ++i) {
-            const int buf = i & 1;
-            if (!mbar_wait(&tfull[buf], (i >> 1) & 1, abort, p.status)) break;
-            tc_fence_after();
-            const int s = i * BM + quarter * 32 + lane;
-            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
-            for (int q = qlo; q < qhi; ++q) {
-                // four independent partial sums break the dependent multiply-add chain
-                float acc4[4] = {0.f, 0.f, 0.f, 0.f};
-                // columns [q*HI, (q+1)*HI) of this buffer; never read past them (HI = 16 uses x16 loads)
-                for (int h0 = 0; h0 < p.HI; h0 += 16) {
-                    const float4 *wq4 = reinterpret_cast<const float4 *>(sw + q * p.HI + h0);
-                    if (h0 + 32 <= p.HI) {
-                        float v[32];
-                        tmem_ld32(taddr + q * p.HI + h0, v);
-                        tmem_wait_ld();
+        const int etid = threadIdx.x - 64;
+        int tile = 0;
+        bool ok = true;
+        int64_t t0;
+        int ntiles;
+        for (int64_t gi = 0; ok && group_of(gi, &t0, &ntiles); ++gi) {
+            const int sb = (int)(gi % p.nsb);
+            const int64_t use = gi / p.nsb;   // earlier uses of this scores buffer
+            if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sempty[sb], (uint32_t)((use - 1) & 1), abort, p.status)))
+                break;
+            float *scores = scores_all + (size_t)sb * p.Q * p.T_cap;
+            named_barrier_sync(1, EPI_THREADS);   // every epilogue thread is done with the previous weights
+            for (int i = etid; i < p.Q * p.HI; i += EPI_THREADS) {
+                const int64_t t = t0 + i / p.HI;
+                sw[i] = t < p.S ? p.w[t * p.HI + (i % p.HI)] : 0.f;
+            }
+            named_barrier_sync(1, EPI_THREADS);
+            for (int i = 0; i < ntiles; ++i, ++tile) {
+                const int buf = tile & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (tile >> 1) & 1, abort, p.status))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const int s = i * BM + quarter * 32 + lane;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+                for (int q = qlo; q < qhi; ++q) {
+                    // four independent partial sums break the dependent multiply-add chain
+                    float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+                    // columns [q*HI, (q+1)*HI) of this buffer; never read past them (HI = 16 uses x16 loads)
+                    for (int h0 = 0; h0 < p.HI; h0 += 16) {
+                        const float4 *wq4 = reinterpret_cast<const float4 *>(sw + q * p.HI + h0);
+                        if (h0 + 64 <= p.HI) {   // 64 heads: both loads in flight, one wait
+                            float v0[32], v1[32];
+                            tmem_ld32(taddr + q * p.HI + h0, v0);
+                            tmem_ld32(taddr + q * p.HI + h0 + 32, v1);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 w4 = wq4[j];
-                            acc4[0] = fmaf(w4.x, fmaxf(v[4 * j], 0.f), acc4[0]);
-                            acc4[1] = fmaf(w4.y, fmaxf(v[4 * j + 1], 0.f), acc4[1]);
-                            acc4[2] = fmaf(w4.z, fmaxf(v[4 * j + 2], 0.f), acc4[2]);
-                            acc4[3] = fmaf(w4.w, fmaxf(v[4 * j + 3], 0.f), acc4[3]);
-                        }
-                        h0 += 16;
-                    } else {
-                        float v[16];
-                        tmem_ld16(taddr + q * p.HI + h0, v);
-                        tmem_wait_ld();
+                            for (int j = 0; j < 16; ++j) {
+                                const float4 w4 = wq4[j];
+                                const float *vv = (j < 8 ? v0 : v1) + 4 * (j & 7);
+                                acc4[0] = fmaf(w4.x, fmaxf(vv[0], 0.f), acc4[0]);
+                                acc4[1] = fmaf(w4.y, fmaxf(vv[1], 0.f), acc4[1]);
+                                acc4[2] = fmaf(w4.z, fmaxf(vv[2], 0.f), acc4[2]);
+                                acc4[3] = fmaf(w4.w, fmaxf(vv[3], 0.f), acc4[3]);
+                            }
+                            h0 += 48;
+                        } else if (h0 + 32 <= p.HI) {
+                            float v[32];
+                            tmem_ld32(taddr + q * p.HI + h0, v);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float4 w4 = wq4[j];
-                            acc4[0] = fmaf(w4.x, fmaxf(v[4 * j], 0.f), acc4[0]);
-                            acc4[1] = fmaf(w4.y, fmaxf(v[4 * j + 1], 0.f), acc4[1]);
-                            acc4[2] = fmaf(w4.z, fmaxf(v[4 * j + 2], 0.f), acc4[2]);
-                            acc4[3] = fmaf(w4.w, fmaxf(v[4 * j + 3], 0.f), acc4[3]);
+                            for (int j = 0; j < 8; ++j) {
+                                const float4 w4 = wq4[j];
+                                acc4[0] = fmaf(w4.x, fmaxf(v[4 * j], 0.f), acc4[0]);
+                                acc4[1] = fmaf(w4.y, fmaxf(v[4 * j + 1], 0.f), acc4[1]);
+                                acc4[2] = fmaf(w4.z, fmaxf(v[4 * j + 2], 0.f), acc4[2]);
+                                acc4[3] = fmaf(w4.w, fmaxf(v[4 * j + 3], 0.f), acc4[3]);
+                            }
+                            h0 += 16;
+                        } else {
+                            float v[16];
+                            tmem_ld16(taddr + q * p.HI + h0, v);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float4 w4 = wq4[j];
+                                acc4[0] = fmaf(w4.x, fmaxf(v[4 * j], 0.f), acc4[0]);
+                                acc4[1] = fmaf(w4.y, fmaxf(v[4 * j + 1], 0.f), acc4[1]);
+                                acc4[2] = fmaf(w4.z, fmaxf(v[4 * j + 2], 0.f), acc4[2]);
+                                acc4[3] = fmaf(w4.w, fmaxf(v[4 * j + 3], 0.f), acc4[3]);
+                            }
                         }
                     }
+                    const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
+                    if (s < p.T_cap) scores[q * p.T_cap + s] = acc + 0.0f;
                 }
-                const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                if (s < p.T_cap) scores[q * p.T_cap + s] = acc + 0.0f;
+                tc_fence_before();
+                mbar_arrive(&tempty[buf]);
             }
-            tc_fence_before();
-            mbar_arrive(&tempty[buf]);
+            if (!ok) break;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfull[sb]);   // this warp's scores of the group are in place
         }
-        named_barrier_sync(1, EPI_THREADS);
-        // ---------------- exact top-k, one query per pair of warps ----------------
-        {
-            const int pair = (warp - 2) >> 1;
+    } else {
+        // ---------------- exact top-k of the previous group's queries, one query per pair of warps ----
+        const int pair = (warp - 2 - EPI_THREADS / 32) >> 1;
+        int64_t t0;
+        int ntiles;
+        for (int64_t gi = 0; group_of(gi, &t0, &ntiles); ++gi) {
+            const int sb = (int)(gi % p.nsb);
+            if (!__all_sync(0xffffffffu, mbar_wait(&sfull[sb], (uint32_t)((gi / p.nsb) & 1), abort, p.status))) break;
+            const float *scores = scores_all + (size_t)sb * p.Q * p.T_cap;
             for (int q = pair; q < p.Q; q += 4) {
                 const int64_t t = t0 + q;
                 if (t >= p.S) continue;
@@ -603,6 +682,8 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     topk_pair(scores + (size_t)q * p.T_cap, n, p.k, hist + pair * (PBINS + 80), 2 + pair,
                               p.idx + t * (int64_t)p.k);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[sb]);   // the buffer may take a later group's scores
         }
     }
     tc_fence_before();
@@ -683,9 +764,15 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     p.k = k;
     p.Q = BN / HI;
     p.T_cap = (int)((T + BM - 1) / BM * BM);
+    p.ngroups = (S + p.Q - 1) / p.Q;
     const size_t a_bytes = (size_t)(dI / 64) * BM * 128, b_bytes = (size_t)(dI / 64) * BN * 128;
-    const size_t fixed = 1024 + b_bytes + (size_t)p.Q * p.T_cap * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + 256;
     const size_t budget = 227 * 1024;
+    size_t fixed = 0;
+    for (p.nsb = 2; p.nsb >= 1; --p.nsb) {   // two scores buffers when three key stages still fit
+        fixed = 1024 + b_bytes + (size_t)p.nsb * p.Q * p.T_cap * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + 256;
+        if (fixed + 2 * a_bytes <= budget) break;
+    }
+    if (p.nsb < 1) return cudaErrorInvalidValue;
     p.stages = (int)std::min<size_t>(4, (budget - fixed) / a_bytes);
     if (p.stages < 2) return cudaErrorInvalidValue;
     const size_t smem = fixed + (size_t)p.stages * a_bytes;
@@ -694,7 +781,9 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)T, dI, BM)) return cudaErrorInvalidValue;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(index_topk_tc_kernel), smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)((S + p.Q - 1) / p.Q);
+    int dev = 0, nsm = 148;
+    if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
+    const unsigned grid = (unsigned)std::min<int64_t>(nsm, p.ngroups);   // persistent
     index_topk_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tk, p);
     return cudaGetLastError();
 }
