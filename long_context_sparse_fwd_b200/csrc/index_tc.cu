@@ -510,6 +510,10 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 mbar_arrive_expect_tx(qfull, b_bytes);
                 for (int c = 0; c < kchunks; ++c)
                     tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
+                int64_t t1;
+                int n1;
+                if (group_of(gi + 1, &t1, &n1))   // the next group's q^I into L2 while this group computes
+                    for (int c = 0; c < kchunks; ++c) tma_prefetch_2d(&tm_q, c * 64, (int)(t1 * p.HI));
             }
             __syncwarp();
             ngr = gi + 1;
@@ -610,22 +614,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     // columns [q*HI, (q+1)*HI) of this buffer; never read past them (HI = 16 uses x16 loads)
                     for (int h0 = 0; h0 < p.HI; h0 += 16) {
                         const float4 *wq4 = reinterpret_cast<const float4 *>(sw + q * p.HI + h0);
-                        if (h0 + 64 <= p.HI) {   // 64 heads: both loads in flight, one wait
-                            float v0[32], v1[32];
-                            tmem_ld32(taddr + q * p.HI + h0, v0);
-                            tmem_ld32(taddr + q * p.HI + h0 + 32, v1);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int j = 0; j < 16; ++j) {
-                                const float4 w4 = wq4[j];
-                                const float *vv = (j < 8 ? v0 : v1) + 4 * (j & 7);
-                                acc4[0] = fmaf(w4.x, fmaxf(vv[0], 0.f), acc4[0]);
-                                acc4[1] = fmaf(w4.y, fmaxf(vv[1], 0.f), acc4[1]);
-                                acc4[2] = fmaf(w4.z, fmaxf(vv[2], 0.f), acc4[2]);
-                                acc4[3] = fmaf(w4.w, fmaxf(vv[3], 0.f), acc4[3]);
-                            }
-                            h0 += 48;
-                        } else if (h0 + 32 <= p.HI) {
+                        if (h0 + 32 <= p.HI) {
                             float v[32];
                             tmem_ld32(taddr + q * p.HI + h0, v);
                             tmem_wait_ld();
