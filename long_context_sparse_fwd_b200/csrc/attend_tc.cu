@@ -687,9 +687,10 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 // Loader warp lw fills key rows 16*lw .. 16*lw+15 of the stage, 16 KB, with one elected lane
                 // issuing: a window block is consecutive kv_rot rows (a [16 x 64] tile per 64-dim chunk);
-                // an entry block is a gather (four rows per gather4, per chunk). Every slot receives a real
-                // row: window slots past the last key read the rows that follow (or the zero fill past the
-                // tensor), entry slots past the last key repeat it, so masked keys always hold finite values.
+                // a selected-entry block is a gather (four rows per gather4, per chunk), an all-entries block
+                // (HCA) consecutive tiles. Every slot receives a real row: window and HCA slots past the last
+                // key read the rows that follow (or the zero fill past the tensor), selected-entry slots past
+                // the last key repeat it, so masked keys always hold finite values.
                 uint8_t *stage = sKV + st * STAGE + lw * 16 * 128;
                 uint64_t *bar = win ? &kv_wfull[st] : &kv_full[st];
                 if (win) {
@@ -701,11 +702,22 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     w_par = (w_issued >> st) & 1u ? w_par ^ (1u << st) : w_par;
                     w_issued |= 1u << st;
+                } else if (a.idx == nullptr) {
+                    // every visible entry (HCA): the block's rows are consecutive, one [16 x 64] tile per
+                    // chunk as for the window; rows past the last key are later entries or the zero fill
+                    const int y = (int)(ent_row0 + kbase + lw * 16);
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(bar, 16 * 1024);
+#pragma unroll
+                        for (int dc = 0; dc < NCH; ++dc) tma_load_2d(stage + dc * KCHUNK, &tm_c, bar, dc * 64, y);
+                    }
+                    e_par = (e_issued >> st) & 1u ? e_par ^ (1u << st) : e_par;
+                    e_issued |= 1u << st;
                 } else {
                     int my_row = 0;
                     if (lane < 16) {
                         const int kk = kbase + min(lw * 16 + lane, nk - 1);
-                        my_row = (int)(ent_row0 + (a.idx != nullptr ? elist[kk] : kk));
+                        my_row = (int)(ent_row0 + elist[kk]);
                     }
                     int r4[16];
 #pragma unroll
@@ -927,7 +939,9 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     const uint64_t w_rows = x.decode ? (uint64_t)x.R * x.W : (uint64_t)x.R;
     if (c_rows >= (1ull << 31) || w_rows >= (1ull << 31)) return cudaErrorInvalidValue;
     if (x.C != nullptr && c_rows > 0) {
-        if (!make_tmap_bf16_sw128(&tc, x.C, c_rows, DD, 1)) return cudaErrorInvalidValue;
+        // selected entries (CSA) are gathered four one-row boxes at a time; every visible entry (HCA)
+        // is read as consecutive 16-row tiles
+        if (!make_tmap_bf16_sw128(&tc, x.C, c_rows, DD, x.idx != nullptr ? 1 : 16)) return cudaErrorInvalidValue;
     } else {
         tc = tq;   // FP8 cache (converted by the loader warps) or no entries: never used
     }
