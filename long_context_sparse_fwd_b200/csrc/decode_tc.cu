@@ -574,6 +574,179 @@ topk_final_kernel(const float *__restrict__ scores, int64_t T, int k, const uint
     for (int j = total + tid; j < k; j += FIN_THREADS) out[j] = -1;
 }
 
+// ---- the whole top-k of one sequence in one CTA (T <= SEQ_T_MAX) ------------------------------------
+//
+// The same selection as the three kernels above, on chip: the sequence's keys stay in shared memory,
+// so the histogram, the threshold, the collection, the ranking of the threshold bin and the ordered
+// output need no global atomics and no further launches.
+
+constexpr int SEQ_T_MAX = 32768;       // 128 KB of keys
+constexpr int SEQ_THREADS = 1024;
+constexpr int SEQ_SUMS = HBINS / 4 + 4;
+constexpr size_t SEQ_SMEM = (size_t)(SEQ_T_MAX + HBINS + SEQ_SUMS + SEQ_T_MAX / 32) * 4 + (size_t)CAND_CAP * 8;
+
+__global__ void __launch_bounds__(SEQ_THREADS, 1)
+topk_seq_kernel(const float *__restrict__ scores, int64_t T64, int k, const uint32_t *__restrict__ keymax,
+                const uint32_t *__restrict__ nkeymin, int32_t *__restrict__ idx)
+{
+    extern __shared__ __align__(16) uint32_t seq_sm[];
+    uint32_t *skey = seq_sm;                       // [T]
+    uint32_t *hist = skey + SEQ_T_MAX;             // [HBINS]
+    uint32_t *sums = hist + HBINS;                 // [SEQ_SUMS]
+    uint32_t *bm = sums + SEQ_SUMS;                // [T / 32] selection bitmap
+    uint2 *cand = reinterpret_cast<uint2 *>(bm + SEQ_T_MAX / 32);   // [CAND_CAP] (key, index)
+    __shared__ int wsum[32];
+    __shared__ uint32_t sh_sel[4];
+    __shared__ uint32_t ncand;
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int T = (int)T64;
+    int32_t *out = idx + (int64_t)b * k;
+    grid_dependency_wait();   // the scores and key ranges of the scan
+    grid_launch_dependents();
+    if (T <= k) {   // every entry is selected
+        for (int j = tid; j < k; j += SEQ_THREADS) out[j] = j < T ? j : -1;
+        return;
+    }
+    const KeyRange r = key_range(keymax[b], nkeymin[b]);
+    const int nw = (T + 31) >> 5;
+    for (int i = tid; i < HBINS; i += SEQ_THREADS) hist[i] = 0u;
+    for (int i = tid; i < nw; i += SEQ_THREADS) bm[i] = 0u;
+    if (tid == 0) ncand = 0u;
+    __syncthreads();
+    // keys into shared memory and the histogram of their digits, eight loads in flight per thread
+    const float *sc = scores + (int64_t)b * T;
+    for (int base = 0; base < T; base += SEQ_THREADS * 8) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + j * SEQ_THREADS + tid;
+            v[j] = i < T ? sc[i] : 0.f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = base + j * SEQ_THREADS + tid;
+            if (i < T) {
+                const uint32_t key = score_key(v[j]);
+                skey[i] = key;
+                atomicAdd(&hist[key_digit(key, r)], 1u);
+            }
+        }
+    }
+    __syncthreads();
+    int dstar;
+    uint32_t above;
+    find_threshold(hist, k, hist, sums, &dstar, &above);   // its copy-in reads the histogram in place
+    const uint32_t remaining = (uint32_t)k - above;
+    // digits above d* are selected (one ballot word per warp and 32 entries); digit d* is a candidate
+    for (int base = 0; base < T; base += SEQ_THREADS) {
+        const int i = base + tid;
+        bool take = false, isc = false;
+        uint32_t key = 0u;
+        if (i < T) {
+            key = skey[i];
+            const int d = (int)key_digit(key, r);
+            take = d > dstar;
+            isc = d == dstar;
+        }
+        const unsigned tb = __ballot_sync(0xffffffffu, take);
+        const int w0 = base + (tid & ~31);
+        if (lane == 0 && w0 < T) bm[w0 >> 5] = tb;
+        const unsigned cm = __ballot_sync(0xffffffffu, isc);
+        if (cm != 0u) {
+            uint32_t pos0 = 0;
+            if (lane == 0) pos0 = atomicAdd(&ncand, (uint32_t)__popc(cm));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            const uint32_t pos = pos0 + __popc(cm & ((1u << lane) - 1u));
+            if (isc && pos < (uint32_t)CAND_CAP) cand[pos] = make_uint2(key, (uint32_t)i);
+        }
+    }
+    __syncthreads();
+    const uint32_t n = ncand;
+    if (n <= (uint32_t)CAND_CAP) {
+        for (uint32_t c = tid; c < n; c += SEQ_THREADS) {
+            const uint2 me = cand[c];
+            uint32_t rank = 0;
+            for (uint32_t j = 0; j < n; ++j) {
+                const uint2 o = cand[j];
+                rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+            }
+            if (rank < remaining) atomicOr(bm + (me.y >> 5), 1u << (me.y & 31));
+        }
+    } else {
+        // Exact fallback for a crowded threshold bin: radix passes (8 bits) over the keys of bin d*
+        // below the digit, then the keys above the final threshold and the first `remaining` equal
+        // ones in index order.
+        uint32_t mask = r.dmask == 0u ? 0xffffffffu : ~((1u << r.shift) - 1u);
+        uint32_t prefix = r.prefix_hi | ((uint32_t)dstar << r.shift);
+        uint32_t rem = remaining;
+        int lowbit = r.dmask == 0u ? 0 : r.shift;
+        uint32_t *h256 = hist;
+        while (lowbit > 0) {
+            const int width = min(8, lowbit), shf = lowbit - width;
+            const uint32_t dm = (1u << width) - 1u;
+            for (int i = tid; i < 256; i += SEQ_THREADS) h256[i] = 0u;
+            __syncthreads();
+            for (int i = tid; i < T; i += SEQ_THREADS) {
+                const uint32_t key = skey[i];
+                if ((key & mask) == prefix) atomicAdd(&h256[(key >> shf) & dm], 1u);
+            }
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t run = 0;
+                int d = 255;
+                for (; d > 0; --d) {
+                    if (run + h256[d] >= rem) break;
+                    run += h256[d];
+                }
+                sh_sel[0] = (uint32_t)d;
+                sh_sel[1] = run;
+                sh_sel[2] = h256[d];
+            }
+            __syncthreads();
+            prefix |= sh_sel[0] << shf;
+            mask |= dm << shf;
+            rem -= sh_sel[1];
+            lowbit = shf;
+            const bool whole = sh_sel[2] == rem;
+            __syncthreads();
+            if (whole) break;
+        }
+        int eq_seen = 0;
+        for (int base = 0; base < T; base += SEQ_THREADS) {
+            const int i = base + tid;
+            uint32_t key = 0u;
+            bool gt = false, eq = false;
+            if (i < T) {
+                key = skey[i];
+                gt = (key & mask) > prefix;   // keys of bin d* above the threshold (higher bins are set already)
+                eq = (key & mask) == prefix;
+            }
+            int tot;
+            const int rank = block_incl_scan(eq ? 1 : 0, wsum, &tot) - (eq ? 1 : 0);
+            const bool sel = gt || (eq && (uint32_t)(eq_seen + rank) < rem);
+            if (sel) atomicOr(bm + (i >> 5), 1u << (i & 31));
+            eq_seen += tot;
+        }
+    }
+    __syncthreads();
+    // the selected entries in ascending order: each thread a contiguous run of bitmap words
+    const int per = (nw + SEQ_THREADS - 1) / SEQ_THREADS;
+    const int w0 = min(nw, tid * per), w1 = min(nw, w0 + per);
+    int cnt = 0;
+    for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+    int total;
+    int off = block_incl_scan(cnt, wsum, &total) - cnt;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t bits = bm[w];
+        while (bits != 0u && off < k) {
+            const int bit = __ffs(bits) - 1;
+            out[off++] = w * 32 + bit;
+            bits &= bits - 1u;
+        }
+    }
+    for (int j = total + tid; j < k; j += SEQ_THREADS) out[j] = -1;
+}
+
 }  // namespace
 
 // Workspace of the decode index step (256-byte aligned pieces): the head (keymax [B], nkeymin [B]),
@@ -642,8 +815,9 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     sp.keymax = keymax;
     sp.nkeymin = nkeymin;
     sp.status = status;
+    const bool seq_topk = T <= SEQ_T_MAX;   // the top-k on chip, one CTA per sequence
     sp.zero = reinterpret_cast<uint4 *>(p8 + L.zero);
-    sp.zero_n16 = (int64_t)(L.zero_bytes / 16);
+    sp.zero_n16 = seq_topk ? 0 : (int64_t)(L.zero_bytes / 16);   // counters of the three-kernel top-k
     sp.T = T;
     sp.HI = HI;
     sp.dI = dI;
@@ -660,6 +834,11 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
     decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (seq_topk) {
+        if ((e = ensure_smem_limit(reinterpret_cast<const void *>(topk_seq_kernel), SEQ_SMEM)) != cudaSuccess) return e;
+        return launch_dependent(topk_seq_kernel, dim3((unsigned)B), dim3(SEQ_THREADS), SEQ_SMEM, stream, (const float *)scores,
+                                T, k, (const uint32_t *)keymax, (const uint32_t *)nkeymin, idx);
+    }
     if (T > k) {
         const dim3 g2((unsigned)((T + TK_CHUNK - 1) / TK_CHUNK), (unsigned)B);
         e = launch_dependent(topk_hist_kernel, g2, dim3(TK_THREADS), 0, stream, (const float *)scores, T,
