@@ -613,9 +613,28 @@ topk_seq_kernel(const float *__restrict__ scores, int64_t T64, int k, const uint
     for (int i = tid; i < nw; i += SEQ_THREADS) bm[i] = 0u;
     if (tid == 0) ncand = 0u;
     __syncthreads();
-    // keys into shared memory and the histogram of their digits, eight loads in flight per thread
+    // keys into shared memory and the histogram of their digits
     const float *sc = scores + (int64_t)b * T;
-    for (int base = 0; base < T; base += SEQ_THREADS * 8) {
+    if ((T & 3) == 0) {   // rows 16-byte aligned: all of a thread's scores (up to 32) in flight at once
+        float4 v[SEQ_T_MAX / (4 * SEQ_THREADS)];
+#pragma unroll
+        for (int j = 0; j < SEQ_T_MAX / (4 * SEQ_THREADS); ++j) {
+            const int i4 = j * SEQ_THREADS + tid;
+            v[j] = 4 * i4 < T ? reinterpret_cast<const float4 *>(sc)[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < SEQ_T_MAX / (4 * SEQ_THREADS); ++j) {
+            const int i4 = j * SEQ_THREADS + tid;
+            if (4 * i4 < T) {
+                const uint32_t k0 = score_key(v[j].x), k1 = score_key(v[j].y), k2 = score_key(v[j].z), k3 = score_key(v[j].w);
+                reinterpret_cast<uint4 *>(skey)[i4] = make_uint4(k0, k1, k2, k3);
+                atomicAdd(&hist[key_digit(k0, r)], 1u);
+                atomicAdd(&hist[key_digit(k1, r)], 1u);
+                atomicAdd(&hist[key_digit(k2, r)], 1u);
+                atomicAdd(&hist[key_digit(k3, r)], 1u);
+            }
+        }
+    } else for (int base = 0; base < T; base += SEQ_THREADS * 8) {
         float v[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -637,8 +656,35 @@ topk_seq_kernel(const float *__restrict__ scores, int64_t T64, int k, const uint
     uint32_t above;
     find_threshold(hist, k, hist, sums, &dstar, &above);   // its copy-in reads the histogram in place
     const uint32_t remaining = (uint32_t)k - above;
-    // digits above d* are selected (one ballot word per warp and 32 entries); digit d* is a candidate
-    for (int base = 0; base < T; base += SEQ_THREADS) {
+    // digits above d* are selected (a bitmap bit per entry); digit d* is a candidate
+    if ((T & 127) == 0) {
+        // four consecutive keys per lane: its nibble of the bitmap, eight lanes per 32-entry word
+        for (int i4 = tid; 4 * i4 < T; i4 += SEQ_THREADS) {
+            const uint4 kv = reinterpret_cast<const uint4 *>(skey)[i4];
+            const uint32_t kk[4] = {kv.x, kv.y, kv.z, kv.w};
+            uint32_t nib = 0u;
+            bool anyc = false;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int d = (int)key_digit(kk[e], r);
+                nib |= (d > dstar ? 1u : 0u) << e;
+                anyc |= d == dstar;
+            }
+            uint32_t word = nib << (4 * (lane & 7));
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            word |= __shfl_xor_sync(0xffffffffu, word, 2);
+            word |= __shfl_xor_sync(0xffffffffu, word, 4);
+            if ((lane & 7) == 0) bm[i4 >> 3] = word;
+            if (__any_sync(0xffffffffu, anyc) && anyc) {   // rare: the threshold bin holds few entries
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if ((int)key_digit(kk[e], r) == dstar) {
+                        const uint32_t pos = atomicAdd(&ncand, 1u);
+                        if (pos < (uint32_t)CAND_CAP) cand[pos] = make_uint2(kk[e], (uint32_t)(4 * i4 + e));
+                    }
+            }
+        }
+    } else for (int base = 0; base < T; base += SEQ_THREADS) {
         const int i = base + tid;
         bool take = false, isc = false;
         uint32_t key = 0u;
