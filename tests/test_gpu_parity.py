@@ -285,10 +285,12 @@ def _decode_index_only(y, wl):
     return idx.cpu().numpy()
 
 
-def test_decode_topk_all_scores_tied():
+@pytest.mark.parametrize("ctx", [4 * 20000, 4 * 40000])
+def test_decode_topk_all_scores_tied(ctx):
     """Index weights of zero make every score +0: the top-k is the k smallest indices (ties go to the
-    smaller index), taken through the crowded-bin path since T far exceeds the candidate capacity."""
-    wl = WORKLOADS[3].with_(ctx=4 * 20000, topk=1024)
+    smaller index), taken through the crowded-bin path since T far exceeds the candidate capacity.
+    T = 20000 selects within one CTA per sequence, T = 40000 through the chunked kernels."""
+    wl = WORKLOADS[3].with_(ctx=ctx, topk=1024)
     y = decode_inputs(wl, device=DEV, batch=2)
     y["w"] = torch.zeros_like(y["w"])
     idx = _decode_index_only(y, wl)
