@@ -12,8 +12,10 @@
 //
 // Top-k is exact and deterministic: the scan also records each sequence's key range; a histogram of
 // the leading differing key bits over all of a sequence's scores finds the threshold bin; the
-// entries above it are marked in a bitmap and those in it collected; one CTA per sequence ranks the
-// collected ones and writes the selection in ascending index order (ties to the smaller index).
+// entries above it are marked in a bitmap and those in it collected and ranked, and the selection
+// is written in ascending index order (ties to the smaller index). Up to 32768 entries per sequence
+// one CTA does all of it with the sequence's keys in shared memory; past that, chunks of 8192
+// entries are histogrammed and collected by many CTAs and one CTA per sequence ranks and writes.
 #include <algorithm>
 
 #include "kernels.cuh"

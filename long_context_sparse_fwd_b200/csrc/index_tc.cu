@@ -11,13 +11,15 @@
 //     D[s, (q,h)] = kI[s,:] . qI[q,h,:]          M = 128 entries, N = 256, K = dI
 // Each epilogue thread then owns one entry and reduces a query's HI columns in registers
 // (w-weighted ReLU sum): no cross-lane reduction. The scores of the Q queries for every visible
-// entry stay in shared memory; after the last entry tile each epilogue warp runs an exact radix
-// select for one query and writes the kept indices in ascending order.
+// entry stay in shared memory; once a group's last entry tile is scored, a pair of warps per query
+// runs the exact selection and writes the kept indices in ascending order.
 //
-// Roles (10 warps): warp 0 issues TMA loads (q^I block once, k^I tiles through a ring of stages),
-// warp 1 owns TMEM (2 x 256 columns, double-buffered accumulators) and issues tcgen05.mma, warps
-// 2-9 read TMEM and score (two warps per lane quarter, each half of the queries), then select.
-// Every wait is bounded; a timeout sets CSA_ERR_TIMEOUT.
+// Persistent: one CTA per SM walks groups of Q queries, the groups that see the most entries first.
+// Roles (18 warps): warp 0 issues TMA loads (a group's q^I block, then its k^I tiles through a ring
+// of stages), warp 1 owns TMEM (2 x 256 columns, double-buffered accumulators) and issues
+// tcgen05.mma, warps 2-9 read TMEM and score (two warps per lane quarter, each half of the
+// queries), warps 10-17 (four pairs) select the previous group's top-k from a second scores buffer
+// while the next group is scored. Every wait is bounded; a timeout sets CSA_ERR_TIMEOUT.
 #include <algorithm>
 
 #include "kernels.cuh"
