@@ -265,3 +265,76 @@ def out_proj(o, wa, wb):
     z = np.concatenate([o_[:, g * K:(g + 1) * K] @ wa_[g].T for g in range(G)], axis=1)
     out = round_bf16(z) @ wb_.T
     return z, out
+
+
+# ---- MXFP4 lightning-indexer operands (axbrief digest "Compressed attention and a new optimizer":
+# MXFP4 on the indexer's query-key path; insight.ai.kr digest of the HF blog: the indexer is
+# stored in FP4). The format is the OCP Microscaling one: blocks of 32 consecutive channels share
+# an E8M0 scale 2^(e-127); elements are E2M1. Quantisation and packing are fixed by DEFINITION's
+# reading for the FP4 indexer.
+
+MXFP4_BLOCK = 32
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])   # magnitude code 0..7
+
+
+def _e2m1_round(q: np.ndarray) -> np.ndarray:
+    """Magnitude codes (0..7) of |q| rounded to the nearest E2M1 value, ties to the even code,
+    saturating at 6."""
+    a = np.abs(q)
+    code = np.zeros(a.shape, np.int64)
+    for c in range(1, 8):   # walk up the grid: past the midpoint, or on it with an even upper code
+        lo, hi = E2M1_VALUES[c - 1], E2M1_VALUES[c]
+        mid = 0.5 * (lo + hi)
+        up = (a > mid) | ((a == mid) & (c % 2 == 0))
+        code = np.where(up & (code == c - 1), c, code)
+    return code
+
+
+def mxfp4_quantize(x):
+    """x [..., d] (d a multiple of 32; bf16 or float values) -> (codes uint8 [..., d/2],
+    scales uint8 [..., d/32]). Per block: amax = max |x|; e = 0 for amax = 0, else
+    e = clamp(floor(log2 amax) - 2 + 127, 0, 254); element = E2M1 rounding of x / 2^(e-127), sign
+    in bit 3 (never on a zero); channel 2i in the low nibble of byte i."""
+    v = _as_f64(x)
+    d = v.shape[-1]
+    assert d % MXFP4_BLOCK == 0
+    blocks = v.reshape(v.shape[:-1] + (d // MXFP4_BLOCK, MXFP4_BLOCK))
+    amax = np.abs(blocks).max(axis=-1)
+    with np.errstate(divide="ignore"):
+        ex = np.floor(np.log2(np.where(amax > 0, amax, 1.0))).astype(np.int64)
+    e = np.where(amax > 0, np.clip(ex - 2 + 127, 0, 254), 0)
+    q = blocks / np.ldexp(1.0, e - 127)[..., None]
+    mag = _e2m1_round(q)
+    sign = (q < 0) & (mag > 0)
+    nib = (mag | (sign.astype(np.int64) << 3)).reshape(v.shape)
+    codes = (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+    return codes, e.astype(np.uint8)
+
+
+def mxfp4_dequantize(codes, scales) -> np.ndarray:
+    """Inverse of the packing: values [..., 2 * codes.shape[-1]] float64 (exact)."""
+    c = _np(codes, np.uint8).astype(np.int64)
+    s = _np(scales, np.uint8).astype(np.int64)
+    nib = np.stack([c & 15, c >> 4], axis=-1).reshape(c.shape[:-1] + (2 * c.shape[-1],))
+    val = E2M1_VALUES[nib & 7] * np.where(nib & 8, -1.0, 1.0)
+    d = val.shape[-1]
+    blocks = val.reshape(val.shape[:-1] + (d // MXFP4_BLOCK, MXFP4_BLOCK))
+    return (blocks * np.ldexp(1.0, s - 127)[..., None]).reshape(val.shape)
+
+
+def _bf16_bits_exact(x: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of float64 values that bf16 represents exactly (checked)."""
+    f = np.ascontiguousarray(x.astype(np.float32))
+    assert np.array_equal(f.astype(np.float64), x), "value not representable in fp32"
+    bits = f.view(np.uint32)
+    assert not np.any(bits & 0xFFFF), "value not representable in bf16"
+    return (bits >> 16).astype(np.uint16)
+
+
+def decode_index_topk_fp4(qc, qs, w, kc, ks, k: int, rows=None):
+    """Decode indexer + top-k on MXFP4 operands: the indexer formula on the dequantised q^I
+    [B, HI, dI] and k^I [B, T, dI] (every E2M1 value times a power of two is exact in bf16, so the
+    bf16 oracle receives exactly these values)."""
+    qv = _bf16_bits_exact(mxfp4_dequantize(qc, qs))
+    kv = _bf16_bits_exact(mxfp4_dequantize(kc, ks))
+    return decode_index_topk(qv, w, kv, k, rows=rows)

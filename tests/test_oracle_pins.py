@@ -585,3 +585,75 @@ def test_out_proj_brute_force_tiny():
         zb = oracle.round_bf16(np.array(zt))
         for i in range(hid):
             np.testing.assert_allclose(out[t, i], sum(zb[c] * wbd[i, c] for c in range(G * R)), rtol=1e-14)
+
+
+# ---- MXFP4 indexer operands (OCP Microscaling format; DEFINITION reading R24) ------------------
+
+def test_mxfp4_e2m1_table():
+    """The sixteen E2M1 codes decode to the OCP table (sign in bit 3) at scale 2^0 (E8M0 127)."""
+    codes = np.array([[c | (c + 1) << 4 for c in range(0, 16, 2)] * 2], np.uint8)   # 16 bytes = 32 values
+    vals = oracle.mxfp4_dequantize(codes, np.array([[127]], np.uint8))[0, :16]
+    want = [0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6]
+    assert vals.tolist() == want
+
+
+def test_mxfp4_rounding_worked_example():
+    """amax 7 gives the shared exponent floor(log2 7) - 2 = 0; each value then rounds to the nearest
+    E2M1 value, ties to the even code, saturating at 6 (hand-worked)."""
+    x = np.zeros((1, 32))
+    x[0, :12] = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, -0.25, -0.3, -2.9, 0.5]
+    codes, scales = oracle.mxfp4_quantize(x)
+    assert scales.tolist() == [[127]]
+    nib = [(b >> (4 * h)) & 15 for b in codes[0].tolist() for h in (0, 1)]
+    #          0.25 0.75 1.25 1.75 2.5 3.5 5.0 7.0 -0.25 -0.3  -2.9    0.5
+    assert nib[:12] == [0, 2, 2, 4, 4, 6, 6, 7, 0, 8 | 1, 8 | 5, 1]
+    assert all(v == 0 for v in nib[12:])
+
+
+def test_mxfp4_shared_exponent_and_zero_block():
+    """The scale exponent follows floor(log2 amax) - 2 across magnitudes; an all-zero block takes
+    E8M0 0 and zero codes; the element reaching amax lands in [4, 8) before rounding."""
+    for amax, e in [(1.0, 125), (0.75, 124), (4.0, 127), (6.5, 127), (1024.0, 135), (2.0 ** -100, 25)]:
+        x = np.zeros((1, 32))
+        x[0, 3] = amax
+        codes, scales = oracle.mxfp4_quantize(x)
+        assert int(scales[0, 0]) == e, (amax, scales)
+        assert 4.0 <= amax / 2.0 ** (e - 127) < 8.0
+    codes, scales = oracle.mxfp4_quantize(np.zeros((2, 64)))
+    assert not codes.any() and not scales.any()
+
+
+def test_mxfp4_round_trip_on_representable_blocks():
+    """Blocks whose values are E2M1 values times 2^(e-127), with at least one magnitude 4 or 6 (so
+    the block maximum selects exponent e), quantise back to the same codes and scales."""
+    rng = np.random.default_rng(3)
+    n = 200
+    mag = rng.integers(0, 8, size=(n, 32))
+    mag[np.arange(n), rng.integers(0, 32, n)] = rng.choice([6, 7], n)
+    sign = rng.integers(0, 2, size=(n, 32)) & (mag > 0)
+    e = rng.integers(60, 200, size=n)
+    vals = (oracle.E2M1_VALUES[mag] * np.where(sign, -1.0, 1.0)) * np.ldexp(1.0, e - 127)[:, None]
+    codes, scales = oracle.mxfp4_quantize(vals)
+    assert scales[:, 0].tolist() == e.tolist()
+    back = oracle.mxfp4_dequantize(codes, scales)
+    assert np.array_equal(back, vals)
+
+
+def test_fp4_indexer_equals_bf16_indexer_on_fp4_values():
+    """With q^I and k^I already MXFP4 values, the FP4 decode indexer selects exactly what the bf16
+    indexer selects on the same (exact) values."""
+    rng = np.random.default_rng(4)
+    B, HI, dI, T, k = 2, 8, 64, 300, 40
+    qc, qs = oracle.mxfp4_quantize(rng.standard_normal((B, HI, dI)))
+    kc, ks = oracle.mxfp4_quantize(rng.standard_normal((B, T, dI)))
+    w = rng.random((B, HI)).astype(np.float32)
+    idx4, sc4 = oracle.decode_index_topk_fp4(qc, qs, w, kc, ks, k)
+    qv = oracle.mxfp4_dequantize(qc, qs)
+    kv = oracle.mxfp4_dequantize(kc, ks)
+    # the scores by hand, in fp64, on the dequantised values
+    ref = np.einsum("bhd,btd->bht", qv, kv)
+    ref = np.einsum("bh,bht->bt", w.astype(np.float64), np.maximum(ref, 0.0))
+    assert np.allclose(sc4, ref, rtol=1e-12, atol=1e-12)
+    for b in range(B):
+        want = np.sort(np.argsort(-ref[b], kind="stable")[:k])
+        assert np.array_equal(np.sort(idx4[b][idx4[b] >= 0]), want)
