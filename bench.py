@@ -33,6 +33,7 @@ if ROOT not in sys.path:
 from workloads import WORKLOADS, decode_inputs, prefill_inputs, proj_inputs  # noqa: E402
 
 WORKLOAD_IDS = {"csa_prefill": 1, "hca_prefill": 2, "decode128k": 3, "decode1m": 4, "hca_decode1m": 5,
+                "decode128k_fp4": 8,
                 "append128k": 6, "out_proj": 7}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -108,7 +109,13 @@ def decode_bytes(wl, B):
     ent = (D - r) + 4 + 2 * r if wl.cache == "fp8" else 2 * D
     if wl.kind == "hca_decode":
         return float(B * (T * ent + wl.W * D * 2 + wl.H * D * 2 + wl.H * D * 4))
-    per_seq = T * wl.dI * 2 + wl.topk * ent + wl.W * D * 2 + wl.H * D * 2 + wl.H * D * 4 + wl.HI * (wl.dI * 2 + 4)
+    if wl.index_fmt == "fp4":   # MXFP4 k^I (codes + E8M0 scales); q^I quantised each step
+        ki = T * (wl.dI // 2 + wl.dI // 32)
+        qi = wl.HI * (wl.dI * 2 + 2 * (wl.dI // 2 + wl.dI // 32) + 4)
+    else:
+        ki = T * wl.dI * 2
+        qi = wl.HI * (wl.dI * 2 + 4)
+    per_seq = ki + wl.topk * ent + wl.W * D * 2 + wl.H * D * 2 + wl.H * D * 4 + qi
     return float(B * per_seq)
 
 
@@ -203,6 +210,11 @@ class Step:
             self.o = torch.empty(self.B, wl.H, wl.D, dtype=torch.float32, device=dev)
             if wl.kind == "csa_decode":
                 self.idx = torch.empty(self.B, wl.topk, dtype=torch.int32, device=dev)
+                if wl.index_fmt == "fp4":   # the cache holds k^I as MXFP4; q^I is quantised every step
+                    self.x["kc"], self.x["ks"] = csa.quantize_mxfp4(self.x["kI"])
+                    del self.x["kI"]
+                    self.qc = torch.empty(self.B, wl.HI, wl.dI // 2, dtype=torch.uint8, device=dev)
+                    self.qs = torch.empty(self.B, wl.HI, wl.dI // 32, dtype=torch.uint8, device=dev)
                 self.ws = torch.empty(csa.workspace_size("decode", B=self.B, T=wl.T, k=wl.topk), dtype=torch.uint8,
                                       device=dev)
             else:
@@ -232,7 +244,11 @@ class Step:
         # decode: index scan, chunk top-k, merge, split attention, combine
         # decode: index scan, three top-k kernels, split attention, combine (plus one memset); HCA
         # decode: split attention and combine
-        return {"csa_prefill": 4, "hca_prefill": 3, "csa_decode": 6, "hca_decode": 2,
+        # CSA decode: index scan, top-k (one kernel up to 32768 entries per sequence, else three), split
+        # attention, combine; the FP4 indexer adds the quantisation of q^I
+        if self.wl.kind == "csa_decode":
+            return (4 if self.wl.T <= 32768 else 6) + (1 if self.wl.index_fmt == "fp4" else 0)
+        return {"csa_prefill": 4, "hca_prefill": 3, "hca_decode": 2,
                 "compress_append": self.wl.m, "out_proj": 2}[self.wl.kind]
 
     def run(self, timed: bool):
@@ -254,7 +270,12 @@ class Step:
             return
         if wl.kind in ("csa_decode", "hca_decode"):
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
-            if wl.kind == "csa_decode":
+            if wl.kind == "csa_decode" and wl.index_fmt == "fp4":
+                csa.quantize_mxfp4(x["qI"], codes=self.qc, scales=self.qs)
+                csa.decode_fp4(x["q"], self.qc, self.qs, x["w"], x["kc"], x["ks"], x["win"], x["sinks"], self.P,
+                               wl.topk, wl.r, wl.theta_tok, wl.theta_cmp, o=self.o, idx=self.idx, workspace=self.ws,
+                               **kw)
+            elif wl.kind == "csa_decode":
                 csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], self.P, wl.topk, wl.r,
                            wl.theta_tok, wl.theta_cmp, o=self.o, idx=self.idx, workspace=self.ws, **kw)
             else:
@@ -320,6 +341,12 @@ def e2e_run(step, steps, warmup):
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
             o = csa.hca_decode(x["q"], x["win"], x["sinks"], step.P, wl.r, wl.theta_tok, wl.theta_cmp, o=step.o,
                                workspace=step.ws, **kw)
+        elif wl.index_fmt == "fp4":
+            kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
+            csa.quantize_mxfp4(x["qI"], codes=step.qc, scales=step.qs)
+            o, _ = csa.decode_fp4(x["q"], step.qc, step.qs, x["w"], x["kc"], x["ks"], x["win"], x["sinks"], step.P,
+                                  wl.topk, wl.r, wl.theta_tok, wl.theta_cmp, o=step.o, idx=step.idx,
+                                  workspace=step.ws, **kw)
         else:
             kw = dict(C=x["C"]) if wl.cache == "bf16" else dict(c8=x["c8"], c8_scale=x["scale"], c_rope=x["rope"])
             o, _ = csa.decode(x["q"], x["qI"], x["w"], x["kI"], x["win"], x["sinks"], step.P, wl.topk, wl.r,
@@ -366,6 +393,8 @@ class OracleStep:
         elif wl.kind in ("csa_decode", "hca_decode"):
             self.x = decode_inputs(wl, device="cpu", batch=1)
             self.P = wl.ctx - 1
+            if wl.index_fmt == "fp4":   # the MXFP4 cache is built once, outside the timed steps
+                self.kq = oracle.mxfp4_quantize(self.x["kI"])
         else:
             self.x = prefill_inputs(wl, device="cpu")
             t0 = time.perf_counter()
@@ -401,7 +430,10 @@ class OracleStep:
             o.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok)
             return wl.m, time.perf_counter() - t0
         if wl.kind in ("csa_decode", "hca_decode"):
-            if wl.kind == "csa_decode":
+            if wl.kind == "csa_decode" and wl.index_fmt == "fp4":
+                qc, qs = o.mxfp4_quantize(x["qI"])
+                ridx, _ = o.decode_index_topk_fp4(qc, qs, x["w"], self.kq[0], self.kq[1], wl.topk)
+            elif wl.kind == "csa_decode":
                 ridx, _ = o.decode_index_topk(x["qI"], x["w"], x["kI"], wl.topk)
             else:
                 ridx = np.arange(wl.T, dtype=np.int32)[None]
@@ -442,7 +474,7 @@ def config_of(wl, n_gpus):
          "l2": "flushed between steps (256 MiB write outside the timed events)"}
     if wl.kind == "csa_decode":
         c.update({"B": wl.B, "ctx": wl.ctx, "T": wl.T, "topk": wl.topk, "index": f"{wl.HI}x{wl.dI}",
-                  "cache": wl.cache})
+                  "cache": wl.cache, "index_format": "mxfp4" if wl.index_fmt == "fp4" else "bf16"})
         del c["S"]
     elif wl.kind == "hca_decode":
         c.update({"B": wl.B, "ctx": wl.ctx, "T": wl.T, "cache": wl.cache})

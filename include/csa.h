@@ -259,6 +259,32 @@ CSA_API csa_status csa_out_proj(const void *o, const void *wa, const void *wb, i
                       int32_t G, int32_t R, int32_t hidden, void *z, void *out, void *workspace,
                       size_t workspace_bytes, void *stream);
 
+/* ---- 11. FP4 (MXFP4) lightning indexer, decode -----------------------------------------------------
+ * [Axbrief "Compressed attention and a new optimizer": MXFP4 on the lightning indexer's query-key
+ * path; HF-blog digest: the indexer stored in FP4]. MXFP4 is the OCP Microscaling format: blocks of
+ * 32 consecutive channels share an E8M0 scale 2^(e-127) (one byte); elements are E2M1 codes (values
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6, sign in bit 3), two per byte, channel 2i in the low nibble.
+ *
+ * csa_quantize_mxfp4: x [rows, cols] bf16 -> codes [rows, cols/2] uint8, scales [rows, cols/32] uint8.
+ *   Per block: amax = max |x|; e = 0 for amax = 0, else clamp(floor(log2 amax) - 2 + 127, 0, 254);
+ *   element = x / 2^(e-127) rounded to the nearest E2M1 value, ties to the even code, saturating at 6;
+ *   a value that rounds to zero is stored as +0. Requires cols % 32 == 0 and 16-byte aligned x, codes.
+ *
+ * csa_decode_fp4: csa_decode with the indexer's operands in MXFP4:
+ *   qI_codes [B, HI, dI/2], qI_scales [B, HI, dI/32], kI_codes [B, T, dI/2], kI_scales [B, T, dI/32];
+ *   the index scores are the indexer formula on the dequantised values (exact products, fp32
+ *   accumulation); everything else is csa_decode's. Requires dI of 64 or 128 and HI of 16, 32, 64 or
+ *   128; workspace as csa_decode (csa_workspace_size(CSA_OP_DECODE)). */
+CSA_API csa_status csa_quantize_mxfp4(const void *x, int64_t rows, int32_t cols, uint8_t *codes, uint8_t *scales,
+                              void *stream);
+
+CSA_API csa_status csa_decode_fp4(const void *q, const uint8_t *qI_codes, const uint8_t *qI_scales, const float *w,
+                      const uint8_t *kI_codes, const uint8_t *kI_scales, const void *C, const uint8_t *c8,
+                      const float *c8_scale, const void *c_rope, const void *win, const float *sinks, int32_t B,
+                      int32_t H, int32_t D, int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W,
+                      int32_t rope_dim, int64_t P, double theta_tok, double theta_cmp, float softmax_scale,
+                      int32_t *idx_out, float *o, void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -16,6 +16,7 @@ import torch
 __all__ = [
     "CSAError", "lib", "library_path", "compress", "index_topk", "attend", "hca_attend", "csa_forward",
     "hca_forward", "decode", "hca_decode", "swa_attend", "compress_append", "out_proj", "workspace_size",
+    "quantize_mxfp4", "decode_fp4",
     "get_device_status", "OP",
 ]
 
@@ -75,6 +76,9 @@ def lib():
             "csa_compress_append": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I64, F64, F64, P, P, P, P, I64, P,
                                           I32, P]),
             "csa_out_proj": (I32, [P, P, P, I64, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
+            "csa_quantize_mxfp4": (I32, [P, I64, I32, P, P, P]),
+            "csa_decode_fp4": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, I32,
+                                     I64, F64, F64, F32, P, P, P, SZ, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -270,6 +274,57 @@ def decode(q, qI, w, kI, win, sinks, P: int, k: int, rope_dim: int, theta_tok: f
                                           _ptr(c_rope), _ptr(win), _ptr(sinks), B, H, D, T, HI, dI, k, W, rope_dim,
                                           int(P), float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(idx),
                                           _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, idx
+
+
+def quantize_mxfp4(x, codes=None, scales=None, stream=None):
+    """MXFP4 (OCP Microscaling) of bf16 rows x [..., d] (d a multiple of 32): returns
+    (codes [..., d/2] uint8, two E2M1 codes per byte with channel 2i in the low nibble,
+    scales [..., d/32] uint8 E8M0)."""
+    _dev(x, torch.bfloat16, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    shape = tuple(x.shape[:-1])
+    codes = torch.empty(shape + (d // 2,), dtype=torch.uint8, device=x.device) if codes is None else \
+        _dev(codes, torch.uint8, "codes", shape + (d // 2,))
+    scales = torch.empty(shape + (d // 32,), dtype=torch.uint8, device=x.device) if scales is None else \
+        _dev(scales, torch.uint8, "scales", shape + (d // 32,))
+    _check("csa_quantize_mxfp4", lib().csa_quantize_mxfp4(_ptr(x), rows, d, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def decode_fp4(q, qI_codes, qI_scales, w, kI_codes, kI_scales, win, sinks, P: int, k: int, rope_dim: int,
+               theta_tok: float, theta_cmp: float, C=None, c8=None, c8_scale=None, c_rope=None,
+               softmax_scale: float = 0.0, o=None, idx=None, workspace=None, stream=None):
+    """csa_decode with the indexer's q^I and k^I in MXFP4 (codes and scales as quantize_mxfp4 returns
+    them: qI [B,HI,dI/2] + [B,HI,dI/32], kI [B,T,dI/2] + [B,T,dI/32]). Returns (o [B,H,D] fp32,
+    idx [B,k] int32)."""
+    B, H, D = q.shape
+    HI, dI = qI_codes.shape[1], 2 * qI_codes.shape[2]
+    T = kI_codes.shape[1]
+    W = win.shape[1]
+    _dev(q, torch.bfloat16, "q")
+    _dev(qI_codes, torch.uint8, "qI_codes", (B, HI, dI // 2))
+    _dev(qI_scales, torch.uint8, "qI_scales", (B, HI, dI // 32))
+    _dev(w, torch.float32, "w", (B, HI))
+    _dev(kI_codes, torch.uint8, "kI_codes", (B, T, dI // 2))
+    _dev(kI_scales, torch.uint8, "kI_scales", (B, T, dI // 32))
+    _dev(win, torch.bfloat16, "win", (B, W, D))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    if C is not None:
+        _dev(C, torch.bfloat16, "C", (B, T, D))
+    else:
+        _dev(c8, torch.uint8, "c8", (B, T, D - rope_dim))
+        _dev(c8_scale, torch.float32, "c8_scale", (B, T))
+        _dev(c_rope, torch.bfloat16, "c_rope", (B, T, rope_dim))
+    o = torch.empty(B, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (B, H, D))
+    idx = torch.empty(B, k, dtype=torch.int32, device=q.device) if idx is None else _dev(idx, torch.int32, "idx", (B, k))
+    ws = _workspace("decode", q.device, workspace, B=B, T=T, k=k)
+    _check("csa_decode_fp4", lib().csa_decode_fp4(
+        _ptr(q), _ptr(qI_codes), _ptr(qI_scales), _ptr(w), _ptr(kI_codes), _ptr(kI_scales), _ptr(C), _ptr(c8),
+        _ptr(c8_scale), _ptr(c_rope), _ptr(win), _ptr(sinks), B, H, D, T, HI, dI, k, W, rope_dim, int(P),
+        float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(idx), _ptr(o), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return o, idx
 
 

@@ -15,7 +15,7 @@ SRC_DIR = os.path.join(HERE, "csrc")
 LIB_PATH = os.path.join(HERE, "libcsa.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
-SOURCES = ["api.cu", "compress.cu", "index_topk.cu", "attend_simt.cu", "index_tc.cu", "attend_tc.cu", "decode_tc.cu", "decode_noalloc.cu", "append.cu", "proj.cu"]
+SOURCES = ["api.cu", "compress.cu", "index_topk.cu", "attend_simt.cu", "index_tc.cu", "attend_tc.cu", "decode_tc.cu", "decode_noalloc.cu", "append.cu", "proj.cu", "fp4.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-cudart", "static"]

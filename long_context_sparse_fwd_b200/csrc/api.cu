@@ -333,49 +333,16 @@ csa_status hca_forward(const void *q, const void *kv, const void *gate, const fl
     return from_cuda(attend_any(a, st));
 }
 
-csa_status csa_decode(const void *q, const void *qI, const float *w, const void *kI, const void *C, const uint8_t *c8,
-                      const float *c8_scale, const void *c_rope, const void *win, const float *sinks, int32_t B,
-                      int32_t H, int32_t D, int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W, int32_t rope_dim,
-                      int64_t P, double theta_tok, double theta_cmp, float softmax_scale, int32_t *idx_out, float *o,
-                      void *workspace, size_t workspace_bytes, void *stream)
+// The attention of a decode step once the index lists `idx` are on the stream (shared by csa_decode
+// and csa_decode_fp4).
+static csa_status decode_attention(const void *q, const void *C, const uint8_t *c8, const float *c8_scale,
+                                   const void *c_rope, const void *win, const float *sinks, int32_t B, int32_t H,
+                                   int32_t D, int64_t T, int32_t k, int32_t W, int32_t rope_dim, int64_t P,
+                                   double theta_tok, double theta_cmp, float softmax_scale, int32_t *idx, float *o,
+                                   void *workspace, size_t workspace_bytes, cudaStream_t st)
 {
-    CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && HI > 0 && dI > 0 && k >= 1 && W >= 0 && P >= 0);
-    CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
-    CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
-    CSA_CHECK_ARG(B == 0 || (q != nullptr && qI != nullptr && w != nullptr && sinks != nullptr && o != nullptr));
-    CSA_CHECK_ARG(B == 0 || T == 0 || kI != nullptr);
-    CSA_CHECK_ARG(B == 0 || W == 0 || win != nullptr);
-    const bool fp8 = C == nullptr;
-    CSA_CHECK_ARG(B == 0 || T == 0 || !fp8 || (c8 != nullptr && c8_scale != nullptr && c_rope != nullptr));
-    CSA_CHECK_SUP(D == 64 || D == 128 || D == 256 || D == 512);
-    CSA_CHECK_SUP(rope_dim % 8 == 0 && k <= 4096);
-    CSA_CHECK_SUP(dI == 32 || dI == 64 || dI == 128 || dI == 256);
-    CSA_CHECK_SUP(HI <= 128 && (size_t)HI * dI * 4 <= 160 * 1024);
-    CSA_CHECK_ARG(aligned16(q) && aligned16(qI) && aligned16(kI) && aligned16(C) && aligned16(c8) &&
-                  aligned16(c_rope) && aligned16(win) && aligned16(o));
-    csa_dims dims;
-    memset(&dims, 0, sizeof dims);
-    dims.B = B;
-    dims.T = T;
-    dims.k = k;
-    CSA_TRY(check_workspace(workspace, workspace_bytes, decode_workspace_min(B, T, k)));
-    cudaStream_t st = as_stream(stream);
     char *base = static_cast<char *>(workspace);
-    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
-    const size_t index_ws = decode_index_bytes(B, T, k);
-    int32_t *idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t *>(base + kStatusBytes + index_ws);
     const size_t used = decode_workspace_min(B, T, k);
-    if (T > 0 && decode_index_tc_supported(T, HI, dI, k)) {
-        // one clear: the status word and the head of the index workspace that follows it
-        CSA_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + decode_index_head_bytes(B), st));
-        CSA_CUDA(launch_decode_index_tc(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
-                                        HI, dI, k, idx, scores, static_cast<int32_t *>(workspace), st));
-    } else {
-        CSA_TRY(reset_status(workspace, st));
-        CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
-                                     HI, dI, 1, 1, scores, st));
-        CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
-    }
     AttnArgs a;
     memset(&a, 0, sizeof a);
     a.q = static_cast<const uint16_t *>(q);
@@ -409,6 +376,101 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
         return from_cuda(launch_attend_tc_decode(a, nsplit, reinterpret_cast<float *>(base + used), st));
     }
     return from_cuda(launch_attend_simt(a, st));
+}
+
+csa_status csa_decode(const void *q, const void *qI, const float *w, const void *kI, const void *C, const uint8_t *c8,
+                      const float *c8_scale, const void *c_rope, const void *win, const float *sinks, int32_t B,
+                      int32_t H, int32_t D, int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W, int32_t rope_dim,
+                      int64_t P, double theta_tok, double theta_cmp, float softmax_scale, int32_t *idx_out, float *o,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && HI > 0 && dI > 0 && k >= 1 && W >= 0 && P >= 0);
+    CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
+    CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_ARG(B == 0 || (q != nullptr && qI != nullptr && w != nullptr && sinks != nullptr && o != nullptr));
+    CSA_CHECK_ARG(B == 0 || T == 0 || kI != nullptr);
+    CSA_CHECK_ARG(B == 0 || W == 0 || win != nullptr);
+    const bool fp8 = C == nullptr;
+    CSA_CHECK_ARG(B == 0 || T == 0 || !fp8 || (c8 != nullptr && c8_scale != nullptr && c_rope != nullptr));
+    CSA_CHECK_SUP(D == 64 || D == 128 || D == 256 || D == 512);
+    CSA_CHECK_SUP(rope_dim % 8 == 0 && k <= 4096);
+    CSA_CHECK_SUP(dI == 32 || dI == 64 || dI == 128 || dI == 256);
+    CSA_CHECK_SUP(HI <= 128 && (size_t)HI * dI * 4 <= 160 * 1024);
+    CSA_CHECK_ARG(aligned16(q) && aligned16(qI) && aligned16(kI) && aligned16(C) && aligned16(c8) &&
+                  aligned16(c_rope) && aligned16(win) && aligned16(o));
+    csa_dims dims;
+    memset(&dims, 0, sizeof dims);
+    dims.B = B;
+    dims.T = T;
+    dims.k = k;
+    CSA_TRY(check_workspace(workspace, workspace_bytes, decode_workspace_min(B, T, k)));
+    cudaStream_t st = as_stream(stream);
+    char *base = static_cast<char *>(workspace);
+    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
+    const size_t index_ws = decode_index_bytes(B, T, k);
+    int32_t *idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t *>(base + kStatusBytes + index_ws);
+    if (T > 0 && decode_index_tc_supported(T, HI, dI, k)) {
+        // one clear: the status word and the head of the index workspace that follows it
+        CSA_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + decode_index_head_bytes(B), st));
+        CSA_CUDA(launch_decode_index_tc(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
+                                        HI, dI, k, idx, scores, static_cast<int32_t *>(workspace), st));
+    } else {
+        CSA_TRY(reset_status(workspace, st));
+        CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
+                                     HI, dI, 1, 1, scores, st));
+        CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
+    }
+    return decode_attention(q, C, c8, c8_scale, c_rope, win, sinks, B, H, D, T, k, W, rope_dim, P, theta_tok, theta_cmp,
+                            softmax_scale, idx, o, workspace, workspace_bytes, st);
+}
+
+csa_status csa_quantize_mxfp4(const void *x, int64_t rows, int32_t cols, uint8_t *codes, uint8_t *scales, void *stream)
+{
+    CSA_CHECK_ARG(rows >= 0 && cols > 0 && cols % 32 == 0);
+    CSA_CHECK_ARG(rows == 0 || (x != nullptr && codes != nullptr && scales != nullptr));
+    CSA_CHECK_ARG(aligned16(x) && aligned16(codes));
+    return from_cuda(launch_quantize_mxfp4(static_cast<const uint16_t *>(x), rows, cols, codes, scales,
+                                           as_stream(stream)));
+}
+
+csa_status csa_decode_fp4(const void *q, const uint8_t *qI_codes, const uint8_t *qI_scales, const float *w,
+                          const uint8_t *kI_codes, const uint8_t *kI_scales, const void *C, const uint8_t *c8,
+                          const float *c8_scale, const void *c_rope, const void *win, const float *sinks, int32_t B,
+                          int32_t H, int32_t D, int64_t T, int32_t HI, int32_t dI, int32_t k, int32_t W,
+                          int32_t rope_dim, int64_t P, double theta_tok, double theta_cmp, float softmax_scale,
+                          int32_t *idx_out, float *o, void *workspace, size_t workspace_bytes, void *stream)
+{
+    CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && HI > 0 && dI > 0 && k >= 1 && W >= 0 && P >= 0);
+    CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
+    CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
+    CSA_CHECK_ARG(B == 0 || (q != nullptr && qI_codes != nullptr && qI_scales != nullptr && w != nullptr &&
+                             sinks != nullptr && o != nullptr));
+    CSA_CHECK_ARG(B == 0 || T == 0 || (kI_codes != nullptr && kI_scales != nullptr));
+    CSA_CHECK_ARG(B == 0 || W == 0 || win != nullptr);
+    const bool fp8 = C == nullptr;
+    CSA_CHECK_ARG(B == 0 || T == 0 || !fp8 || (c8 != nullptr && c8_scale != nullptr && c_rope != nullptr));
+    CSA_CHECK_SUP(D == 64 || D == 128 || D == 256 || D == 512);
+    CSA_CHECK_SUP(rope_dim % 8 == 0 && k <= 4096);
+    CSA_CHECK_SUP((dI == 64 || dI == 128) && (HI == 16 || HI == 32 || HI == 64 || HI == 128));
+    CSA_CHECK_SUP(T == 0 || decode_index_fp4_supported(T, HI, dI, k));
+    CSA_CHECK_ARG(aligned16(q) && aligned16(qI_codes) && aligned16(kI_codes) && aligned16(C) && aligned16(c8) &&
+                  aligned16(c_rope) && aligned16(win) && aligned16(o));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, decode_workspace_min(B, T, k)));
+    cudaStream_t st = as_stream(stream);
+    char *base = static_cast<char *>(workspace);
+    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
+    const size_t index_ws = decode_index_bytes(B, T, k);
+    int32_t *idx = idx_out != nullptr ? idx_out : reinterpret_cast<int32_t *>(base + kStatusBytes + index_ws);
+    if (T > 0) {
+        CSA_CUDA(cudaMemsetAsync(workspace, 0, kStatusBytes + decode_index_head_bytes(B), st));
+        CSA_CUDA(launch_decode_index_fp4(qI_codes, qI_scales, w, kI_codes, kI_scales, B, T, HI, dI, k, idx, scores,
+                                         static_cast<int32_t *>(workspace), st));
+    } else {   // no entries: every index slot is -1
+        CSA_TRY(reset_status(workspace, st));
+        CSA_CUDA(launch_topk_rows(scores, B, 0, 1, 1, k, idx, st));
+    }
+    return decode_attention(q, C, c8, c8_scale, c_rope, win, sinks, B, H, D, T, k, W, rope_dim, P, theta_tok, theta_cmp,
+                            softmax_scale, idx, o, workspace, workspace_bytes, st);
 }
 
 csa_status hca_decode(const void *q, const void *C, const uint8_t *c8, const float *c8_scale, const void *c_rope,

@@ -17,6 +17,7 @@
 // one CTA does all of it with the sequence's keys in shared memory; past that, chunks of 8192
 // entries are histogrammed and collected by many CTAs and one CTA per sequence ranks and writes.
 #include <algorithm>
+#include <cstring>
 
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -26,6 +27,8 @@ namespace csa {
 using namespace sm100;
 
 namespace {
+
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 constexpr int BM = 128;
 constexpr int NUM_THREADS = 192;
@@ -44,6 +47,98 @@ struct ScoreParams {
     int64_t T, G;        // entries per sequence; total tiles (B * tiles per sequence)
     int HI, dI, stages, tps;
 };
+
+// Epilogue of the scan (four warps, 128 threads, one TMEM lane quarter each): each thread owns one entry
+// of the tile, reduces its HI heads (w-weighted ReLU) in registers and writes one fp32 score; it also
+// tracks the sequence's key range for the top-k and clears the chunked top-k's counters.
+__device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tmem, uint64_t *tfull, uint64_t *tempty,
+                                              volatile int *abort, float *sw, int64_t g_lo, int ntiles, int warp,
+                                              int lane, int etid)
+{
+    const int quarter = warp & 3;
+    const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
+    for (int64_t i = (int64_t)blockIdx.x * EPI_THREADS + etid; i < p.zero_n16; i += (int64_t)gridDim.x * EPI_THREADS)
+        p.zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    float wr[64];   // index weights of the current sequence (HI == 64 keeps them in registers)
+    // range of the score keys of the current sequence seen by this thread, merged into the
+    // sequence's global range (for the top-k's histogram) whenever the sequence changes
+    uint32_t kmax = 0u, knmin = 0u;
+    int64_t b_cur = -1;
+    auto flush_range = [&]() {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+            knmin = max(knmin, __shfl_xor_sync(0xffffffffu, knmin, o));
+        }
+        if (lane == 0 && b_cur >= 0) {
+            atomicMax(p.keymax + b_cur, kmax);
+            atomicMax(p.nkeymin + b_cur, knmin);
+        }
+        kmax = 0u;
+        knmin = 0u;
+    };
+    for (int i = 0; i < ntiles; ++i) {
+        const int64_t g = g_lo + i, b = g / p.tps;
+        const int it = (int)(g - b * p.tps);
+        if (b != b_cur) {
+            flush_range();
+            b_cur = b;
+        }
+        if (i == 0 || it == 0) {   // index weights of the new sequence
+            named_barrier_sync(1, EPI_THREADS);
+            for (int h = etid; h < p.HI; h += EPI_THREADS) sw[h] = p.w[b * p.HI + h];
+            named_barrier_sync(1, EPI_THREADS);
+            if (p.HI == 64) {
+#pragma unroll
+                for (int h = 0; h < 64; ++h) wr[h] = sw[h];
+            }
+        }
+        const int buf = i % NACC;
+        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i / NACC) & 1, abort, p.status))) break;
+        tc_fence_after();
+        float acc = 0.f;
+        if (p.HI == 64) {
+            float v0[32], v1[32];
+            tmem_ld32(taddr0 + buf * 64, v0);        // both loads in flight, one wait
+            tmem_ld32(taddr0 + buf * 64 + 32, v1);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);               // the accumulator may be reused from here
+#pragma unroll
+            for (int jj = 0; jj < 32; ++jj) {
+                acc = fmaf(wr[jj], fmaxf(v0[jj], 0.f), acc);
+                acc = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), acc);
+            }
+        } else {
+            for (int h0 = 0; h0 < p.HI; h0 += 16) {
+                if (h0 + 32 <= p.HI) {
+                    float v[32];
+                    tmem_ld32(taddr0 + buf * p.HI + h0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
+                    h0 += 16;
+                } else {
+                    float v[16];
+                    tmem_ld16(taddr0 + buf * p.HI + h0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[buf]);
+        }
+        const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
+        if (s < p.T) {
+            p.scores[b * p.T + s] = acc + 0.0f;
+            const uint32_t key = score_key(acc);
+            kmax = max(kmax, key);
+            knmin = max(knmin, ~key);
+        }
+    }
+    flush_range();
+}
 
 // Persistent: CTA c takes the contiguous tile range [c*G/n, (c+1)*G/n) of the flat list
 // (sequence-major, 128 entries per tile), so the HBM stream never idles on a wave tail. q^I of the
@@ -163,89 +258,252 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
         }
     } else {
-        const int quarter = warp & 3, etid = threadIdx.x - 64;
-        const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
-        for (int64_t i = (int64_t)blockIdx.x * EPI_THREADS + etid; i < p.zero_n16; i += (int64_t)gridDim.x * EPI_THREADS)
-            p.zero[i] = make_uint4(0u, 0u, 0u, 0u);
-        float wr[64];   // index weights of the current sequence (HI == 64 keeps them in registers)
-        // range of the score keys of the current sequence seen by this thread, merged into the
-        // sequence's global range (for the top-k's histogram) whenever the sequence changes
-        uint32_t kmax = 0u, knmin = 0u;
-        int64_t b_cur = -1;
-        auto flush_range = [&]() {
+        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, tcols);
+    }
+}
+
+// ---- the same scan on MXFP4 operands ------------------------------------------------------------------
+//
+// q^I and k^I arrive as MXFP4 (E2M1 codes, two per byte, and one E8M0 scale per 32 channels). A
+// producer warp brings each 128-entry tile of k^I codes (dI/2 bytes per entry) into a ring of staging
+// buffers by TMA; four converter warps (one entry row per thread) dequantise it into the bf16
+// 128-byte-swizzled A tile the MMA reads, and at each new sequence dequantise its q^I into the B
+// operand. Every E2M1 value times a power of two is exact in bf16, so the bf16 MMA with fp32
+// accumulation computes the scores of the dequantised operands. The epilogue is the bf16 scan's.
+
+constexpr int F4_THREADS = 320;        // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue, warps 6-9 convert
+constexpr int F4_CONV0 = 6;
+constexpr int F4_CST = 6;              // code staging buffers
+
+struct Fp4Params {
+    ScoreParams sp;
+    const uint8_t *qc, *qs;            // q^I codes [B, HI, dI/2], scales [B, HI, dI/32]
+    const uint8_t *ks;                 // k^I scales [B*T, dI/32]
+    int64_t rows;                      // B*T
+};
+
+// The two dequantised values of a code byte (channel 2i in the low half) as a bf16 pair, unscaled.
+__device__ __forceinline__ uint32_t e2m1_pair_bits(uint32_t byte)
+{
+    auto one = [](uint32_t n) -> uint32_t {
+        const uint32_t m = n & 7u;
+        uint32_t f;   // fp32 bits of the magnitude
+        if (m == 0u) f = 0u;
+        else if (m == 1u) f = 126u << 23;                                   // 0.5
+        else f = (((m >> 1) + 126u) << 23) | ((m & 1u) << 22);              // (1 + mant/2) 2^(exp-1)
+        f |= (n & 8u) && m != 0u ? 0x80000000u : 0u;
+        return f >> 16;                                                     // exact: bf16 keeps the top half
+    };
+    return one(byte & 15u) | (one(byte >> 4) << 16);
+}
+
+// 2^(e-127) as a bf16 pair (exact for every E8M0 value below 255; e = 0 is the subnormal 2^-127)
+__device__ __forceinline__ __nv_bfloat162 e8m0_scale2(uint32_t e)
+{
+    const uint32_t f = e != 0u ? (e << 23) : 0x00400000u;
+    const uint32_t h2 = (f >> 16) | (f & 0xffff0000u);
+    __nv_bfloat162 r;
+    memcpy(&r, &h2, 4);
+    return r;
+}
+
+__global__ void __launch_bounds__(F4_THREADS, 1)
+decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
+{
+    const ScoreParams &p = f.sp;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int kchunks = p.dI / 64;
+    const uint32_t a_bytes = (uint32_t)kchunks * BM * 128;   // bf16 A tile
+    const uint32_t b_bytes = (uint32_t)kchunks * p.HI * 128; // bf16 q^I
+    const uint32_t c_row = (uint32_t)p.dI / 2;               // code bytes per entry
+    const uint32_t c_bytes = c_row * BM;
+    uint8_t *sA = smem;                                      // [2][a_bytes]
+    uint8_t *sB = sA + 2 * a_bytes;                          // [2][b_bytes]
+    uint8_t *sC = sB + 2 * b_bytes;                          // [F4_CST][c_bytes]
+    float *sw = reinterpret_cast<float *>(sC + F4_CST * c_bytes);   // [256]
+    uint32_t *lut = reinterpret_cast<uint32_t *>(sw + 256);         // [256] code byte -> bf16 pair
+    uint64_t *bars = reinterpret_cast<uint64_t *>(lut + 256);
+    uint64_t *cfull = bars, *cempty = bars + 8;              // [F4_CST]
+    uint64_t *afull = bars + 16, *aempty = bars + 18;        // [2]
+    uint64_t *qfull = bars + 20, *qempty = bars + 22;        // [2]
+    uint64_t *tfull = bars + 24, *tempty = bars + 28;        // [NACC]
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(bars + 32);
+    volatile int *abort = reinterpret_cast<volatile int *>(bars + 33);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t g_lo = (int64_t)blockIdx.x * p.G / gridDim.x;
+    const int64_t g_hi = (int64_t)(blockIdx.x + 1) * p.G / gridDim.x;
+    const int ntiles = (int)(g_hi - g_lo);
+    const int64_t b_first = g_lo / p.tps;
+    const uint32_t tcols = p.HI * NACC <= 32 ? 32 : (p.HI * NACC <= 64 ? 64 : (p.HI * NACC <= 128 ? 128 : (p.HI * NACC <= 256 ? 256 : 512)));
+    const int ctid = threadIdx.x - F4_CONV0 * 32;            // converter thread: entry row of the tile
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < F4_CST; ++i) { mbar_init(&cfull[i], 1); mbar_init(&cempty[i], 128); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&afull[i], 128);
+            mbar_init(&aempty[i], 1);
+            mbar_init(&qfull[i], 128);
+            mbar_init(&qempty[i], 1);
+        }
+        for (int i = 0; i < NACC; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], EPI_THREADS);
+        }
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (ctid >= 0) {
+        lut[ctid] = e2m1_pair_bits((uint32_t)ctid);
+        lut[ctid + 128] = e2m1_pair_bits((uint32_t)ctid + 128u);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_ptr, tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    grid_launch_dependents();   // the top-k may be scheduled as this grid's CTAs finish
+
+    if (warp == 0) {
+        // ---------------- TMA producer: k^I code tiles ----------------
+        if (ntiles > 0) {
+            if (elect_one()) prefetch_tmap(&tm_kc);
+            __syncwarp();
+            const uint64_t pol_stream = policy_evict_first();
+            int issued = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int64_t g = g_lo + i, b = g / p.tps;
+                const int it = (int)(g - b * p.tps), st = i % F4_CST;
+                if (!__all_sync(0xffffffffu, mbar_wait(&cempty[st], ((i / F4_CST) & 1) ^ 1, abort, p.status))) break;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&cfull[st], c_bytes);
+                    tma_load_2d_hint(sC + st * c_bytes, &tm_kc, &cfull[st], 0, (int)(b * p.T + (int64_t)it * BM), pol_stream);
+                }
+                __syncwarp();
+                issued = i + 1;
+            }
+            for (int i = max(0, issued - F4_CST); i < issued; ++i)   // no copy in flight at exit
+                mbar_wait(&cfull[i % F4_CST], (i / F4_CST) & 1, abort, p.status, 100000000ull);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (ntiles > 0) {
+            const uint32_t idesc = idesc_bf16(BM, p.HI);
+            const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
+            int issued = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int64_t g = g_lo + i, b = g / p.tps;
+                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+                if (i == 0 || it == 0)
+                    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status))) break;
+                const int buf = i % NACC, ab = i & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((i / NACC) & 1) ^ 1, abort, p.status))) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&afull[ab], (i >> 1) & 1, abort, p.status))) break;
+                tc_fence_after();
+                const uint64_t dBj = dB + (((j & 1) * b_bytes) >> 4);
+                if (elect_one()) {
+                    for (int c = 0; c < kchunks; ++c)
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-                knmin = max(knmin, __shfl_xor_sync(0xffffffffu, knmin, o));
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tmem + buf * p.HI, dA + ((ab * a_bytes + c * BM * 128 + ks * 32) >> 4),
+                                     dBj + ((c * p.HI * 128 + ks * 32) >> 4), idesc, (c | ks) != 0);
+                    mma_commit(&aempty[ab]);
+                    mma_commit(&tfull[buf]);
+                    if (i + 1 == ntiles || it + 1 == p.tps) mma_commit(&qempty[j & 1]);
+                }
+                __syncwarp();
+                issued = i + 1;
             }
-            if (lane == 0 && b_cur >= 0) {
-                atomicMax(p.keymax + b_cur, kmax);
-                atomicMax(p.nkeymin + b_cur, knmin);
-            }
-            kmax = 0u;
-            knmin = 0u;
-        };
+            if (issued > 0)
+                mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
+        }
+    } else if (warp < F4_CONV0) {
+        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
+    } else {
+        // ---------------- converters: thread ctid dequantises entry row ctid of each tile ----------------
+        const int nblk = p.dI / 32;                           // scale blocks per row
         for (int i = 0; i < ntiles; ++i) {
             const int64_t g = g_lo + i, b = g / p.tps;
-            const int it = (int)(g - b * p.tps);
-            if (b != b_cur) {
-                flush_range();
-                b_cur = b;
-            }
-            if (i == 0 || it == 0) {   // index weights of the new sequence
-                named_barrier_sync(1, EPI_THREADS);
-                for (int h = etid; h < p.HI; h += EPI_THREADS) sw[h] = p.w[b * p.HI + h];
-                named_barrier_sync(1, EPI_THREADS);
-                if (p.HI == 64) {
+            const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+            if (i == 0 || it == 0) {
+                // q^I of the new sequence into B operand buffer j & 1 (HI rows x dI), once the MMAs
+                // of the sequence two back are done with it
+                if (!__all_sync(0xffffffffu, mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status))) break;
+                uint8_t *dst = sB + (j & 1) * b_bytes;
+                for (int q = ctid; q < p.HI * nblk; q += 128) {   // one 32-channel block each
+                    const int h = q / nblk, blk = q % nblk;
+                    const int64_t rq = b * p.HI + h;
+                    const uint4 cv = *reinterpret_cast<const uint4 *>(f.qc + rq * (p.dI / 2) + blk * 16);
+                    const __nv_bfloat162 sc2 = e8m0_scale2(f.qs[rq * nblk + blk]);
+                    const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-                    for (int h = 0; h < 64; ++h) wr[h] = sw[h];
-                }
-            }
-            const int buf = i % NACC;
-            if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i / NACC) & 1, abort, p.status))) break;
-            tc_fence_after();
-            float acc = 0.f;
-            if (p.HI == 64) {
-                float v0[32], v1[32];
-                tmem_ld32(taddr0 + buf * 64, v0);        // both loads in flight, one wait
-                tmem_ld32(taddr0 + buf * 64 + 32, v1);
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&tempty[buf]);               // the accumulator may be reused from here
+                    for (int u = 0; u < 4; ++u) {   // 8 channels per 16-byte unit
+                        uint32_t o[4];
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    acc = fmaf(wr[jj], fmaxf(v0[jj], 0.f), acc);
-                    acc = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), acc);
-                }
-            } else {
-                for (int h0 = 0; h0 < p.HI; h0 += 16) {
-                    if (h0 + 32 <= p.HI) {
-                        float v[32];
-                        tmem_ld32(taddr0 + buf * p.HI + h0, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int jj = 0; jj < 32; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
-                        h0 += 16;
-                    } else {
-                        float v[16];
-                        tmem_ld16(taddr0 + buf * p.HI + h0, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int jj = 0; jj < 16; ++jj) acc = fmaf(sw[h0 + jj], fmaxf(v[jj], 0.f), acc);
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t pr = lut[(cw[u] >> (8 * e)) & 255u];
+                            const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&pr), sc2);
+                            o[e] = *reinterpret_cast<const uint32_t *>(&v);
+                        }
+                        const int ch = blk * 32 + u * 8, c = ch >> 6, uu = (ch & 63) >> 3;
+                        *reinterpret_cast<uint4 *>(dst + c * p.HI * 128 + h * 128 + ((uu ^ (h & 7)) << 4)) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&tempty[buf]);
+                fence_async_smem();
+                mbar_arrive(&qfull[j & 1]);
             }
-            const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
-            if (s < p.T) {
-                p.scores[b * p.T + s] = acc + 0.0f;
-                const uint32_t key = score_key(acc);
-                kmax = max(kmax, key);
-                knmin = max(knmin, ~key);
+            const int st = i % F4_CST, ab = i & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&cfull[st], (i / F4_CST) & 1, abort, p.status))) break;
+            // Thread ctid takes 32-channel block u = ctid % nblk of rows ctid / nblk + k * (128 / nblk),
+            // k < nblk: a warp reads 512 contiguous staging bytes per pass.
+            const int rpp = 128 / nblk, u = ctid % nblk;
+            uint4 cv[4];
+            uint32_t sb[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (k >= nblk) break;
+                const int r = k * rpp + ctid / nblk;
+                cv[k] = *reinterpret_cast<const uint4 *>(sC + st * c_bytes + r * c_row + u * 16);
+                const int64_t grow = b * p.T + (int64_t)it * BM + r;
+                sb[k] = grow < f.rows ? (uint32_t)f.ks[grow * nblk + u] : 0u;
             }
+            mbar_arrive(&cempty[st]);   // the staging buffer may be refilled
+            if (!__all_sync(0xffffffffu, mbar_wait(&aempty[ab], ((i >> 1) & 1) ^ 1, abort, p.status))) break;
+            uint8_t *dst = sA + ab * a_bytes;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (k >= nblk) break;
+                const int r = k * rpp + ctid / nblk;
+                const __nv_bfloat162 sc2 = e8m0_scale2(sb[k]);
+                const uint32_t cw[4] = {cv[k].x, cv[k].y, cv[k].z, cv[k].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {   // channels 32u + 8q .. +7: bytes 4q .. 4q+3 of the block
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint32_t pr = lut[(cw[q] >> (8 * e)) & 255u];
+                        const __nv_bfloat162 v = __hmul2(*reinterpret_cast<const __nv_bfloat162 *>(&pr), sc2);
+                        o[e] = *reinterpret_cast<const uint32_t *>(&v);
+                    }
+                    const int ch = u * 32 + q * 8, c = ch >> 6, uu = (ch & 63) >> 3;
+                    *reinterpret_cast<uint4 *>(dst + c * BM * 128 + r * 128 + ((uu ^ (r & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            fence_async_smem();   // generic-proxy writes, read by the MMA through the async proxy
+            mbar_arrive(&afull[ab]);
         }
-        flush_range();
     }
     tc_fence_before();
     __syncthreads();
@@ -836,15 +1094,11 @@ bool decode_index_tc_supported(int64_t T, int HI, int dI, int k)
            T <= (1ll << 26);
 }
 
-// scores/candidates live in `ws` (decode_index_workspace bytes, 256-byte aligned), whose first
-// decode_index_head_bytes(B) bytes the caller has zeroed on this stream. The kernels after the scan
-// are launched as programmatic dependents, each one scheduled while the one before it finishes.
-cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t B, int64_t T, int HI,
-                                   int dI, int k, int32_t *idx, void *ws, int32_t *status, cudaStream_t stream)
+// The top-k after a scan: one CTA per sequence up to SEQ_T_MAX entries, else the chunked kernels;
+// each launched as a programmatic dependent of the kernel before it.
+static cudaError_t launch_topk_after_scan(char *p8, const DecodeIndexLayout &L, int64_t B, int64_t T, int k, int32_t *idx,
+                                          cudaStream_t stream)
 {
-    if (B == 0) return cudaSuccess;
-    char *p8 = static_cast<char *>(ws);
-    const DecodeIndexLayout L = decode_index_layout(B, T);
     float *scores = reinterpret_cast<float *>(p8 + L.scores);
     uint32_t *keymax = reinterpret_cast<uint32_t *>(p8 + L.keymax);
     uint32_t *nkeymin = reinterpret_cast<uint32_t *>(p8 + L.nkeymin);
@@ -853,36 +1107,7 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(p8 + L.bitmap);
     uint2 *cand = reinterpret_cast<uint2 *>(p8 + L.cand);
     cudaError_t e;
-
-    CUtensorMap tq, tk;
-    if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)B * HI, dI, HI)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)(B * T), dI, BM)) return cudaErrorInvalidValue;
-    ScoreParams sp;
-    sp.w = w;
-    sp.scores = scores;
-    sp.keymax = keymax;
-    sp.nkeymin = nkeymin;
-    sp.status = status;
-    const bool seq_topk = T <= SEQ_T_MAX;   // the top-k on chip, one CTA per sequence
-    sp.zero = reinterpret_cast<uint4 *>(p8 + L.zero);
-    sp.zero_n16 = seq_topk ? 0 : (int64_t)(L.zero_bytes / 16);   // counters of the three-kernel top-k
-    sp.T = T;
-    sp.HI = HI;
-    sp.dI = dI;
-    sp.tps = (int)((T + BM - 1) / BM);
-    sp.G = (int64_t)B * sp.tps;
-    const size_t a_bytes = (size_t)(dI / 64) * BM * 128;
-    const size_t fixed = 1024 + 2 * (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
-    sp.stages = (int)std::min<size_t>(MAX_STAGES, (227 * 1024 - fixed) / a_bytes);
-    const size_t smem = fixed + (size_t)sp.stages * a_bytes;
-    e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_tc_kernel), smem);
-    if (e != cudaSuccess) return e;
-    int dev = 0, nsm = 148;
-    if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
-    const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
-    decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (seq_topk) {
+    if (T <= SEQ_T_MAX) {   // the top-k on chip, one CTA per sequence
         if ((e = ensure_smem_limit(reinterpret_cast<const void *>(topk_seq_kernel), SEQ_SMEM)) != cudaSuccess) return e;
         return launch_dependent(topk_seq_kernel, dim3((unsigned)B), dim3(SEQ_THREADS), SEQ_SMEM, stream, (const float *)scores,
                                 T, k, (const uint32_t *)keymax, (const uint32_t *)nkeymin, idx);
@@ -900,6 +1125,88 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     return launch_dependent(topk_final_kernel, dim3((unsigned)B), dim3(FIN_THREADS), 0, stream, (const float *)scores, T,
                             k, (const uint32_t *)keymax, (const uint32_t *)nkeymin, (const uint32_t *)hist, bitmap,
                             (const uint32_t *)ncand, (const uint2 *)cand, idx);
+}
+
+// scores/candidates live in `ws` (decode_index_workspace bytes, 256-byte aligned), whose first
+// decode_index_head_bytes(B) bytes the caller has zeroed on this stream. The kernels after the scan
+// are launched as programmatic dependents, each one scheduled while the one before it finishes.
+// Score parameters shared by the bf16 and MXFP4 scans.
+static ScoreParams score_params(char *p8, const DecodeIndexLayout &L, const float *w, int64_t B, int64_t T, int HI,
+                                int dI, int32_t *status)
+{
+    ScoreParams sp;
+    sp.w = w;
+    sp.scores = reinterpret_cast<float *>(p8 + L.scores);
+    sp.keymax = reinterpret_cast<uint32_t *>(p8 + L.keymax);
+    sp.nkeymin = reinterpret_cast<uint32_t *>(p8 + L.nkeymin);
+    sp.status = status;
+    sp.zero = reinterpret_cast<uint4 *>(p8 + L.zero);
+    sp.zero_n16 = T <= SEQ_T_MAX ? 0 : (int64_t)(L.zero_bytes / 16);   // counters of the chunked top-k
+    sp.T = T;
+    sp.HI = HI;
+    sp.dI = dI;
+    sp.tps = (int)((T + BM - 1) / BM);
+    sp.G = (int64_t)B * sp.tps;
+    sp.stages = 0;
+    return sp;
+}
+
+cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t B, int64_t T, int HI,
+                                   int dI, int k, int32_t *idx, void *ws, int32_t *status, cudaStream_t stream)
+{
+    if (B == 0) return cudaSuccess;
+    char *p8 = static_cast<char *>(ws);
+    const DecodeIndexLayout L = decode_index_layout(B, T);
+    CUtensorMap tq, tk;
+    if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)B * HI, dI, HI)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)(B * T), dI, BM)) return cudaErrorInvalidValue;
+    ScoreParams sp = score_params(p8, L, w, B, T, HI, dI, status);
+    const size_t a_bytes = (size_t)(dI / 64) * BM * 128;
+    const size_t fixed = 1024 + 2 * (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
+    sp.stages = (int)std::min<size_t>(MAX_STAGES, (227 * 1024 - fixed) / a_bytes);
+    const size_t smem = fixed + (size_t)sp.stages * a_bytes;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_tc_kernel), smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 148;
+    if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
+    const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
+    decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_topk_after_scan(p8, L, B, T, k, idx, stream);
+}
+
+bool decode_index_fp4_supported(int64_t T, int HI, int dI, int k)
+{
+    return decode_index_tc_supported(T, HI, dI, k) && (int64_t)T * 4 < (1ll << 31);
+}
+
+// MXFP4 operands: codes two per byte (channel 2i in the low nibble), one E8M0 scale per 32 channels.
+cudaError_t launch_decode_index_fp4(const uint8_t *qc, const uint8_t *qs, const float *w, const uint8_t *kc,
+                                    const uint8_t *ks, int64_t B, int64_t T, int HI, int dI, int k, int32_t *idx,
+                                    void *ws, int32_t *status, cudaStream_t stream)
+{
+    if (B == 0) return cudaSuccess;
+    char *p8 = static_cast<char *>(ws);
+    const DecodeIndexLayout L = decode_index_layout(B, T);
+    CUtensorMap tkc;   // k^I codes as rows of dI/2 bytes, 128-row boxes
+    if (!make_tmap_u8_rows(&tkc, kc, (uint64_t)(B * T), (uint64_t)dI / 2, BM)) return cudaErrorInvalidValue;
+    Fp4Params f;
+    f.sp = score_params(p8, L, w, B, T, HI, dI, status);
+    f.qc = qc;
+    f.qs = qs;
+    f.ks = ks;
+    f.rows = B * T;
+    const size_t a_bytes = (size_t)(dI / 64) * BM * 128, b_bytes = (size_t)(dI / 64) * HI * 128;
+    const size_t c_bytes = (size_t)dI / 2 * BM;
+    const size_t smem = 1024 + 2 * a_bytes + 2 * b_bytes + F4_CST * c_bytes + 256 * 4 + 256 * 4 + 34 * 8;
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_fp4_kernel), smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, nsm = 148;
+    if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
+    const unsigned g1 = (unsigned)std::min<int64_t>(nsm, f.sp.G);
+    decode_scores_fp4_kernel<<<g1, F4_THREADS, smem, stream>>>(tkc, f);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_topk_after_scan(p8, L, B, T, k, idx, stream);
 }
 
 }  // namespace csa

@@ -732,6 +732,19 @@ bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint
     return make_tmap_sw128(map, base, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, rows, cols, box_rows);
 }
 
+bool make_tmap_u8_rows(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr || cols % 16 != 0 || cols > 256) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols};
+    cuuint32_t box[2] = {(cuuint32_t)cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)
 {
     (void)k;

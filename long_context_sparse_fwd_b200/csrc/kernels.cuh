@@ -46,6 +46,8 @@ cudaError_t launch_attend_tc_decode(const AttnArgs &a, int nsplit, float *part, 
 bool make_tmap_bf16_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // 2-D fp32 tensor map, box [box_rows, 32], 128-byte swizzle
 bool make_tmap_f32_sw128(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// 2-D byte tensor map over [rows, cols] (cols a multiple of 16, at most 256), box [box_rows, cols], no swizzle
+bool make_tmap_u8_rows(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // append.cu: the compressor's decode step (one token per sequence; emits an entry when a window closes)
 struct AppendArgs {
@@ -77,6 +79,14 @@ size_t decode_index_head_bytes(int64_t B);   // leading bytes of its workspace t
 bool decode_index_tc_supported(int64_t T, int HI, int dI, int k);
 cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t B, int64_t T, int HI,
                                    int dI, int k, int32_t *idx, void *ws, int32_t *status, cudaStream_t stream);
+// the same on MXFP4 q^I and k^I (codes two per byte, one E8M0 scale per 32 channels)
+bool decode_index_fp4_supported(int64_t T, int HI, int dI, int k);
+cudaError_t launch_decode_index_fp4(const uint8_t *qc, const uint8_t *qs, const float *w, const uint8_t *kc,
+                                    const uint8_t *ks, int64_t B, int64_t T, int HI, int dI, int k, int32_t *idx,
+                                    void *ws, int32_t *status, cudaStream_t stream);
+// fp4.cu: bf16 rows -> MXFP4 codes and scales
+cudaError_t launch_quantize_mxfp4(const uint16_t *x, int64_t rows, int cols, uint8_t *codes, uint8_t *scales,
+                                  cudaStream_t stream);
 
 // index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);

@@ -318,6 +318,65 @@ def test_decode_topk_few_distinct_scores(ctx, classes):
         assert np.all(np.diff(idx[b][idx[b] >= 0]) > 0)
 
 
+# ---- FP4 (MXFP4) lightning indexer, decode --------------------------------------------------------------
+
+def test_quantize_mxfp4_matches_oracle():
+    """bf16 rows of mixed magnitudes (row scales 2^-40 .. 2^40), an all-zero block and exact E2M1
+    midpoints: codes and scales bit-exact with the oracle."""
+    g = torch.Generator().manual_seed(11)
+    x = torch.randn(300, 128, generator=g, dtype=torch.float64)
+    x *= torch.pow(2.0, torch.randint(-40, 41, (300, 1), generator=g).double())
+    x[5, 32:64] = 0.0
+    x[6, :8] = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0], dtype=torch.float64)
+    x[6, 8:32] = 0.0
+    xb = x.to(torch.bfloat16)
+    codes, scales = csa.quantize_mxfp4(xb.to(DEV))
+    torch.cuda.synchronize()
+    rc, rs = oracle.mxfp4_quantize(xb)
+    assert np.array_equal(scales.cpu().numpy(), rs)
+    assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+def _decode_fp4_check(wl, batch, seqs):
+    y = decode_inputs(wl, device=DEV, batch=batch)
+    P = wl.ctx - 1
+    qc, qs = csa.quantize_mxfp4(y["qI"])
+    kc, ks = csa.quantize_mxfp4(y["kI"])
+    kw = dict(C=y["C"]) if wl.cache == "bf16" else dict(c8=y["c8"], c8_scale=y["scale"], c_rope=y["rope"])
+    o, idx = csa.decode_fp4(y["q"], qc, qs, y["w"], kc, ks, y["win"], y["sinks"], P, wl.topk, wl.r, wl.theta_tok,
+                            wl.theta_cmp, **kw)
+    torch.cuda.synchronize()
+    seqs = np.asarray(seqs, np.int64)
+    h = {k: v[seqs].cpu() if v.dim() > 1 else v.cpu() for k, v in y.items()}
+    rq = oracle.mxfp4_quantize(h["qI"])
+    rk = oracle.mxfp4_quantize(h["kI"])
+    assert np.array_equal(qc.cpu().numpy()[seqs], rq[0]) and np.array_equal(kc.cpu().numpy()[seqs], rk[0])
+    ridx, sc = oracle.decode_index_topk_fp4(rq[0], rq[1], h["w"], rk[0], rk[1], wl.topk)
+    gidx = idx.cpu().numpy()[seqs]
+    exc = check_topk_sets(gidx, ridx, sc, [wl.T] * len(seqs), wl.topk)
+    assert len(exc) <= 1, f"near-tie exceptions in {len(exc)} sequences"
+    assert all(np.all(np.diff(r[r >= 0]) > 0) for r in gidx)
+    # the attention over the selection the GPU made (its sets are the oracle's up to near-ties)
+    kwr = dict(C=h["C"]) if wl.cache == "bf16" else dict(c8=h["c8"], c8_scale=h["scale"], c_rope=h["rope"])
+    ref = oracle.decode_attend(h["q"], h["win"], gidx, h["sinks"], P, wl.r, wl.theta_tok, wl.theta_cmp, **kwr)
+    check_close(o.cpu()[seqs], ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
+def test_decode_fp4_small():
+    """MXFP4 indexer, ragged last tile (T = 2049), one CTA per sequence for the top-k."""
+    _decode_fp4_check(WORKLOADS[3].with_(ctx=4 * 2049 + 3), batch=3, seqs=[0, 1, 2])
+
+
+def test_decode_fp4_ctx128k():
+    """MXFP4 indexer at the 128K decode size (64 sequences of 32768 entries), sampled sequences."""
+    _decode_fp4_check(WORKLOADS[3], batch=None, seqs=[0, 41, 63])
+
+
+def test_decode_fp4_chunked_topk_fp8_cache():
+    """MXFP4 indexer past 32768 entries (chunked top-k) with the FP8 entry cache."""
+    _decode_fp4_check(WORKLOADS[4].with_(ctx=4 * 40000 + 1, B=2), batch=None, seqs=[0, 1])
+
+
 # ---- 7. HCA decode and the sliding-window-only layer ----------------------------------------------------
 
 # HCA at 1M context: m' = 128 pools 1,048,576 tokens into T = 8192 entries, all attended densely

@@ -47,6 +47,7 @@ class Workload:
     B: int = 0
     ctx: int = 0              # tokens of history per sequence
     cache: str = "bf16"       # "bf16" | "fp8"
+    index_fmt: str = "bf16"   # indexer operands q^I, k^I: "bf16" | "fp4" (MXFP4)
     # grouped output projection (o_groups, o_lora_rank, hidden_size of the V4-Flash config)
     o_groups: int = 8
     o_rank: int = 1024
@@ -76,6 +77,8 @@ WORKLOADS: Dict[int, Workload] = {
     6: Workload("csa_append_b64_ctx128k", "compress_append", B=64, ctx=131072, m=4, L=8, topk=0, seed=6),
     # the grouped output projection after the V4-Flash attention, S=8192
     7: Workload("v4flash_out_proj_s8192", "out_proj", S=8192, seed=7),
+    # CSA decode at 128K context with the FP4 (MXFP4) lightning indexer: k^I cached as MXFP4
+    8: Workload("csa_decode_b64_ctx128k_fp4idx", "csa_decode", B=64, ctx=131072, topk=1024, seed=3, index_fmt="fp4"),
 }
 
 
