@@ -1,6 +1,8 @@
 """Benchmark of the CSA / HCA attention forward on B200 (one JSON line on stdout).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload csa_prefill|hca_prefill|decode128k|decode1m]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+        NAME: csa_prefill (default) | hca_prefill | decode128k | decode1m | decode128k_fp4 (MXFP4 indexer)
+              | hca_decode1m | append128k (compressor decode step) | out_proj (grouped output projection)
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed on this host's cores
 
 A step is one full pass of the layer forward over one batch of synthetic inputs already resident

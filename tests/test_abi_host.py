@@ -166,3 +166,23 @@ def test_later_calls_reject_bad_arguments():
     assert op(R=1000) == UNSUP                  # o_lora_rank not a multiple of 256
     assert op(hid=100) == UNSUP
     assert op(wsb=16) == WS
+
+
+def test_fp4_calls_reject_bad_arguments():
+    """csa_quantize_mxfp4 and csa_decode_fp4 check their arguments on the host, before any launch."""
+    L = csa.lib()
+    assert L.csa_quantize_mxfp4(FAKE, 4, 48, FAKE, FAKE, None) == INVALID     # 48 channels: not whole blocks
+    assert L.csa_quantize_mxfp4(FAKE, -1, 64, FAKE, FAKE, None) == INVALID
+    assert L.csa_quantize_mxfp4(None, 4, 64, FAKE, FAKE, None) == INVALID     # rows but no input
+    assert L.csa_quantize_mxfp4(FAKE, 0, 64, None, None, None) == 0           # nothing to do
+
+    def df(qc=FAKE, kc=FAKE, C=FAKE, B=2, T=100, HI=64, dI=128, k=64, wsb=1 << 24):
+        return L.csa_decode_fp4(FAKE, qc, FAKE, FAKE, kc, FAKE, C, None, None, None, FAKE, FAKE, B, 64, 512, T, HI, dI,
+                                k, 128, 64, 1000, 1e4, 1.6e5, 0.0, None, FAKE, FAKE, wsb, None)
+    assert df(T=-1) == INVALID
+    assert df(qc=None) == INVALID               # index query codes missing
+    assert df(kc=None) == INVALID               # entries but no index key codes
+    assert df(C=None) == INVALID                # entries but neither a bf16 nor an FP8 cache
+    assert df(dI=96) == UNSUP                   # MXFP4 scan: d_I of 64 or 128
+    assert df(HI=48) == UNSUP
+    assert df(wsb=16) == WS
