@@ -5,8 +5,10 @@
               | hca_decode1m | append128k (compressor decode step) | out_proj (grouped output projection)
     python bench.py --impl reference ...   # the fp64 CPU oracle, timed on this host's cores
 
-A step is one full pass of the layer forward over one batch of synthetic inputs already resident
-in HBM: compress -> lightning indexer + top-k -> sparse + window attention for CSA prefill
+The default line (the V4-Flash CSA prefill layer) carries a "side" object with the V4-Flash HCA
+prefill layer and the two CSA decode batches (128K context, and 1M context with the FP8 cache), each
+timed the same way. A step is one full pass of the layer forward over one batch of synthetic inputs
+already resident in HBM: compress -> lightning indexer + top-k -> sparse + window attention for CSA prefill
 (the V4-Flash layer, S=8192), compress -> dense attention for HCA prefill (S=65536), and
 indexer + top-k -> attention for decode. Per-step CUDA events on the launching stream time
 every kernel phase; L2 is flushed (a 256 MiB write) between steps, outside the timed events.
@@ -540,6 +542,55 @@ def cpu_baseline(wl):
             "sample": st.sample_desc() + f"; {st.calls} steps"}
 
 
+SIDE_WORKLOADS = ("hca_prefill", "decode128k", "decode1m")
+
+
+def side_runs(csa, dev, steps, flush, reduce_max):
+    """The other headline configurations, each timed as the main line is (device events around each
+    step, L2 flushed between steps, max over ranks): the V4-Flash HCA prefill layer and the two CSA
+    decode batches. Returns {workload: summary}; each workload's buffers are freed before the next."""
+    peaks, peak_src = load_peaks()
+    out = {}
+    for name in SIDE_WORKLOADS:
+        wl = WORKLOADS[WORKLOAD_IDS[name]]
+        step = Step(name, wl, csa, dev)
+        for _ in range(3):
+            step.run(False)
+        torch.cuda.synchronize()
+        ph = []
+        for _ in range(steps):
+            flush.fill_(1)
+            step.run(True)
+            torch.cuda.synchronize()
+            ph.append(step.phase_ms())
+        ph = np.array(ph)
+        total = reduce_max(float(ph.sum()))
+        mean_phase = ph.mean(0)
+        d = {"metric": metric_name(wl), "value": step.units * steps / (total / 1e3), "unit": unit_name(wl),
+             "ms_per_step": total / steps, "steps": steps, "config": config_of(wl, 1),
+             "phases_ms": {n: float(v) for n, v in zip(step.phases, mean_phase)}}
+        if wl.kind == "hca_prefill":
+            t_att = float(mean_phase[step.phases.index("attend")]) / 1e3
+            fl, by = csa_attention_flops(wl), attention_bytes(wl)
+            d["roofline"] = {"kernel": "attention", "bound": "tensor and hbm (ridge)",
+                             "achieved_tflops": fl / t_att / 1e12, "peak_tflops": peaks["bf16_tflops"],
+                             "frac_tensor": fl / t_att / 1e12 / peaks["bf16_tflops"],
+                             "achieved_gbs": by / t_att / 1e9, "peak_gbs": peaks["hbm_gbs"],
+                             "frac_hbm": by / t_att / 1e9 / peaks["hbm_gbs"], "peak_source": peak_src}
+        else:
+            by = decode_bytes(wl, step.B)
+            t = total / steps / 1e3
+            d["roofline"] = {"kernel": "whole decode step (index scan + top-k + attention + combine)",
+                             "bound": "hbm", "algorithmic_bytes": by, "achieved": by / t / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": by / t / 1e9 / peaks["hbm_gbs"],
+                             "peak_source": peak_src}
+        d["gpu_launches"] = step.launches_per_step() * steps
+        out[name] = d
+        del step
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -549,6 +600,7 @@ def main():
     ap.add_argument("--workload", default="csa_prefill", choices=sorted(WORKLOAD_IDS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side", action="store_true", help="skip the HCA prefill and decode objects of the default line")
     args = ap.parse_args()
     wl = WORKLOADS[WORKLOAD_IDS[args.workload]]
     rank = int(os.environ.get("RANK", "0"))
@@ -631,6 +683,16 @@ def main():
     roof["traffic"] = recorded_traffic(args.workload)   # ncu DRAM bytes per launch (profiles/traffic.txt)
     roof["ms_per_launch"] = float(mean_phase[dom])
 
+    def reduce_max(v):
+        tv = torch.tensor([v], dtype=torch.float64, device=dev)
+        if dist is not None:
+            dist.all_reduce(tv, op=dist.ReduceOp.MAX)
+        return float(tv.item())
+
+    side = None
+    if args.workload == "csa_prefill" and not args.no_side:
+        side = side_runs(csa, dev, max(3, min(args.steps, 10)), flush, reduce_max)
+
     e2e = None
     if not args.no_e2e:
         ms, h2d, d2h = e2e_run(step, max(2, args.steps // 2), 1)
@@ -650,6 +712,8 @@ def main():
         "roofline": roof, "e2e": e2e, "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clk.summary(),
     }
+    if side is not None:
+        line["side"] = side
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if dist is not None:

@@ -183,7 +183,10 @@ CSA_API csa_status csa_decode(const void *q, const void *qI, const float *w, con
  *     indices, about B*(4*T + T/8 + 24 KB + 4*k) bytes (e.g. B=64 sequences of T=32768 entries,
  *     or B=8 of T=262144, fit). Whatever the array has left is used for attention splits.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *     that device current; make that first call before any stream capture.
+ *     that device current; make that first call before any stream capture. The address is kept per
+ *     device together with the CUDA context it belongs to and looked up again when a different
+ *     context is current (after cudaDeviceReset, or under a context the caller created).
+ *   - B, T and k so large that a scratch size would overflow are CSA_ERR_INVALID_ARG.
  *   - All calls on a device share the one array and it keeps the last call's contents: calls that
  *     overlap on the GPU (different streams, or different host threads) race and must be
  *     serialised by the caller. The device status word of the last call is not readable through

@@ -137,6 +137,15 @@ int hca_decode_splits_preferred(int64_t B, int64_t T, int32_t W)
 }  // namespace
 
 namespace csa {
+// Every decode workspace term is at most a few times 4*B*T or 4*B*k bytes: with T <= 2^40 entries
+// per sequence and B*T, B*k below 2^56 none of them can overflow a 64-bit size.
+bool decode_sizes_representable(int64_t B, int64_t T, int32_t k)
+{
+    if (B < 0 || T < 0 || k < 0 || T > ((int64_t)1 << 40)) return false;
+    const uint64_t lim = (uint64_t)1 << 56;
+    return B == 0 || ((uint64_t)T <= lim / (uint64_t)B && (uint64_t)k <= lim / (uint64_t)B);
+}
+
 size_t decode_workspace_min(int64_t B, int64_t T, int32_t k)
 {
     return kStatusBytes + decode_index_bytes(B, T, k) + align256(sizeof(int32_t) * (size_t)B * (size_t)k);
@@ -385,6 +394,7 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
                       void *workspace, size_t workspace_bytes, void *stream)
 {
     CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && HI > 0 && dI > 0 && k >= 1 && W >= 0 && P >= 0);
+    CSA_CHECK_ARG(decode_sizes_representable(B, T, k));
     CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
     CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
     CSA_CHECK_ARG(B == 0 || (q != nullptr && qI != nullptr && w != nullptr && sinks != nullptr && o != nullptr));
@@ -441,6 +451,7 @@ csa_status csa_decode_fp4(const void *q, const uint8_t *qI_codes, const uint8_t 
                           int32_t *idx_out, float *o, void *workspace, size_t workspace_bytes, void *stream)
 {
     CSA_CHECK_ARG(B >= 0 && H > 0 && D > 0 && T >= 0 && HI > 0 && dI > 0 && k >= 1 && W >= 0 && P >= 0);
+    CSA_CHECK_ARG(decode_sizes_representable(B, T, k));
     CSA_CHECK_ARG(rope_dim >= 0 && rope_dim <= D && (rope_dim % 2) == 0);
     CSA_CHECK_ARG(rope_dim == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
     CSA_CHECK_ARG(B == 0 || (q != nullptr && qI_codes != nullptr && qI_scales != nullptr && w != nullptr &&

@@ -9,8 +9,11 @@
 //
 // The array is a file-scope __device__ variable: each GPU that loads the library holds one copy
 // of it until the process exits. Host code cannot use the array's name as a device address (it is
-// a host-side stand-in), so the device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and cached.
+// a host-side stand-in), so the device address is looked up with cudaGetSymbolAddress, with the
+// device current, the first time a CUDA context uses this entry point. The address belongs to that
+// context: it is cached per device together with the context it was taken in (the driver's current
+// context), and taken again when another context is current (after cudaDeviceReset, or under a
+// caller that made its own context current).
 #include <mutex>
 
 #include "kernels.cuh"
@@ -22,23 +25,51 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-void *g_scratch_addr[kMaxDevices];
+struct ScratchAddr {
+    void *ctx;    // the driver context the address was taken in
+    void *addr;
+};
+ScratchAddr g_scratch[kMaxDevices];
 std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device (looked up on first use per device).
+typedef int (*CtxGetCurrentFn)(void **);
+
+// cuCtxGetCurrent through the runtime's driver entry point table (the library links no libcuda).
+CtxGetCurrentFn ctx_get_current_fn()
+{
+    static CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<CtxGetCurrentFn>(p);
+        return nullptr;
+    }();
+    return fn;
+}
+
+// Device address of the scratch array in the current device's current context.
 csa_status scratch_on_current_device(void **out)
 {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return CSA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return CSA_ERR_UNSUPPORTED;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (get_ctx == nullptr) return CSA_ERR_CUDA;
+    void *ctx = nullptr;
+    if (get_ctx(&ctx) != 0) return CSA_ERR_CUDA;   // null while no context is current on this thread yet
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (ctx == nullptr || g_scratch[dev].addr == nullptr || g_scratch[dev].ctx != ctx) {
         void *p = nullptr;
+        // looks the symbol up in the current context, making the device's primary context current
+        // first when none is
         const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
         if (e != cudaSuccess || p == nullptr) return CSA_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+        if (get_ctx(&ctx) != 0 || ctx == nullptr) return CSA_ERR_CUDA;
+        g_scratch[dev].ctx = ctx;
+        g_scratch[dev].addr = p;
     }
-    *out = g_scratch_addr[dev];
+    *out = g_scratch[dev].addr;
     return CSA_OK;
 }
 
@@ -55,6 +86,8 @@ csa_status csa_decode_noalloc(const void *q, const void *qI, const float *w, con
                               float softmax_scale, int32_t *idx_out, float *o, void *stream)
 {
     if (B < 0 || T < 0 || k < 1) return CSA_ERR_INVALID_ARG;
+    // sizes whose byte counts would overflow are refused before any size is computed
+    if (!csa::decode_sizes_representable(B, T, k)) return CSA_ERR_INVALID_ARG;
     if (csa::decode_workspace_min(B, T, k) > kNoAllocScratchBytes) return CSA_ERR_WORKSPACE;
     void *scratch = nullptr;
     const csa_status s = scratch_on_current_device(&scratch);

@@ -72,6 +72,8 @@ cudaError_t launch_proj_gemm_tc(const uint16_t *A, int64_t lda, const uint16_t *
 
 // api.cu: smallest workspace csa_decode accepts (no attention split partials)
 size_t decode_workspace_min(int64_t B, int64_t T, int32_t k);
+// api.cu: false when B, T or k are so large that a decode workspace size would overflow size_t
+bool decode_sizes_representable(int64_t B, int64_t T, int32_t k);
 
 // decode_tc.cu: decode index scan (tcgen05, HBM streaming) + two-stage exact top-k
 size_t decode_index_workspace(int64_t B, int64_t T, int k);

@@ -49,6 +49,12 @@ def lib():
         L.orc_bf16_to_f64.argtypes = [ctypes.c_uint16]
         L.orc_e4m3_to_f64.restype = _F64
         L.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_from_f32.restype = ctypes.c_uint8
+        L.orc_e4m3_from_f32.argtypes = [ctypes.c_float]
+        L.orc_e4m3_from_f32_array.restype = None
+        L.orc_e4m3_from_f32_array.argtypes = [_P, _I64, _P]
+        L.orc_fp8_entry_rows.restype = None
+        L.orc_fp8_entry_rows.argtypes = [_P, _I64, _I32, _P, _P]
         L.orc_rope.restype = None
         L.orc_rope.argtypes = [_P, _I32, _I32, _F64, _F64]
         L.orc_compress.restype = _I64
@@ -101,6 +107,27 @@ def _ptr(a: Optional[np.ndarray]):
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes (uint8, same shape) of binary32 values: nearest, ties to the even code, finite
+    overflow saturating to +-448, NaN -> 0x7F (the OCP FP8 definition's saturating conversion)."""
+    x_ = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    out = np.empty(x_.shape, np.uint8)
+    lib().orc_e4m3_from_f32_array(_ptr(x_), x_.size, _ptr(out))
+    return out
+
+
+def fp8_entry_rows(x):
+    """FP8 form of entry rows x [n, c] (binary32 values of the non-rope channels): per row
+    scale = amax / 448 in binary32 (1 for an all-zero row) and codes = E4M3 of x / scale.
+    Returns (codes uint8 [n, c], scale float32 [n])."""
+    x_ = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    n, c = x_.shape
+    codes = np.empty((n, c), np.uint8)
+    scale = np.empty(n, np.float32)
+    lib().orc_fp8_entry_rows(_ptr(x_), n, c, _ptr(codes), _ptr(scale))
+    return codes, scale
 
 
 def bf16_to_f64(bits: int) -> float:
@@ -269,9 +296,9 @@ def out_proj(o, wa, wb):
 
 # ---- MXFP4 lightning-indexer operands (axbrief digest "Compressed attention and a new optimizer":
 # MXFP4 on the indexer's query-key path; insight.ai.kr digest of the HF blog: the indexer is
-# stored in FP4). The format is the OCP Microscaling one: blocks of 32 consecutive channels share
-# an E8M0 scale 2^(e-127); elements are E2M1. Quantisation and packing are fixed by DEFINITION's
-# reading for the FP4 indexer.
+# stored in FP4). The pages name the format without its details; it is taken as the OCP
+# Microscaling one: blocks of 32 consecutive channels share an E8M0 scale 2^(e-127); elements are
+# E2M1, rounded to nearest with ties to the even code and saturating at 6.
 
 MXFP4_BLOCK = 32
 E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])   # magnitude code 0..7

@@ -58,6 +58,57 @@ double orc_e4m3_to_f64(uint8_t v)
     return sign ? -mag : mag;
 }
 
+/* The E4M3 code nearest to a binary32 value, as the OCP definition's saturating conversion
+ * rounds it: round to nearest, ties to the code with an even mantissa (its lowest bit 0); finite
+ * values beyond the largest magnitude (448) saturate to +-448; NaN gives the NaN code 0x7F. The sign
+ * bit is kept, also on a result of zero. The nearest magnitude is found by comparing |x| with every
+ * finite non-negative code in turn (codes 0x00..0x7E increase with their value). */
+uint8_t orc_e4m3_from_f32(float x)
+{
+    if (isnan(x))
+        return 0x7F;
+    int sign = signbit(x) ? 1 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0)
+        return (uint8_t)(0x7E | (sign << 7));
+    int best = 0;
+    double best_err = INFINITY;
+    for (int c = 0; c <= 0x7E; ++c) {
+        double err = fabs(a - orc_e4m3_to_f64((uint8_t)c));
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint8_t)(best | (sign << 7));
+}
+
+void orc_e4m3_from_f32_array(const float *x, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = orc_e4m3_from_f32(x[i]);
+}
+
+/* FP8 form of entry rows (the FP8 KV cache of the insight.ai.kr digest: most of each entry in FP8,
+ * the rope channels kept in BF16; the per-entry scale reading): per row of `cols` binary32 values,
+ * scale = amax / 448 rounded to binary32 (1 when the row is all zero), each code the E4M3 encoding
+ * of x / scale rounded to binary32. Both roundings are single roundings of the exact quotient:
+ * a quotient of two binary32 values never lies closer to a binary32 rounding boundary than the
+ * binary64 rounding error, so rounding through binary64 first changes nothing. */
+void orc_fp8_entry_rows(const float *x, int64_t rows, int cols, uint8_t *codes, float *scale)
+{
+    for (int64_t i = 0; i < rows; ++i) {
+        const float *xr = x + i * (int64_t)cols;
+        double amax = 0.0;
+        for (int c = 0; c < cols; ++c)
+            if (fabs((double)xr[c]) > amax) amax = fabs((double)xr[c]);
+        float s = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+        scale[i] = s;
+        for (int c = 0; c < cols; ++c)
+            codes[i * (int64_t)cols + c] = orc_e4m3_from_f32((float)((double)xr[c] / (double)s));
+    }
+}
+
 void orc_bf16_array_to_f64(const uint16_t *x, int64_t n, double *out)
 {
     for (int64_t i = 0; i < n; ++i)

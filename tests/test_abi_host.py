@@ -118,14 +118,16 @@ def test_index_topk_rejects_bad_arguments():
 def test_decode_rejects_bad_arguments():
     L = csa.lib()
 
-    def f(C=FAKE, c8=None, B=2, D=512, k=64, P=100, dI=128, wsb=1 << 24):
-        return L.csa_decode(FAKE, FAKE, FAKE, FAKE, C, c8, None, None, FAKE, FAKE, B, 8, D, 256, 4, dI, k, 8, 64,
+    def f(C=FAKE, c8=None, B=2, D=512, k=64, P=100, dI=128, wsb=1 << 24, T=256):
+        return L.csa_decode(FAKE, FAKE, FAKE, FAKE, C, c8, None, None, FAKE, FAKE, B, 8, D, T, 4, dI, k, 8, 64,
                             P, 1e4, 1.6e5, 0.0, None, FAKE, FAKE, wsb, None)
     assert f(C=None) == INVALID                 # neither bf16 entries nor an FP8 cache
     assert f(P=-1) == INVALID
     assert f(D=96) == UNSUP
     assert f(dI=40) == UNSUP
     assert f(wsb=64) == WS
+    assert f(T=1 << 41) == INVALID               # sizes that would overflow the workspace arithmetic
+    assert f(B=1 << 30, T=1 << 30) == INVALID
 
 
 def test_binding_refuses_cpu_tensors():

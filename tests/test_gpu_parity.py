@@ -227,6 +227,28 @@ def test_hca_forward_end_to_end():
     check_close(o.cpu()[rows], ref, O_MAX_ABS, O_MEAN_ABS, what="o")
 
 
+@pytest.mark.parametrize("S", [65536, 16384 + 77])
+def test_hca_forward_full_size(S):
+    """The V4-Flash HCA prefill layer at its own size (65536 tokens: up to 512 pooled entries, eight
+    64-key entry blocks per query) and at 16461 tokens (a ragged last entry block), in the launch
+    configuration the benchmark times, on sampled rows: the last 64, both sides of window closes
+    (128 j - 1 and 128 j) and random rows. Rows are independent once the entries exist."""
+    wl = WORKLOADS[2].with_(S=S)
+    g, x = gen(prefill_inputs, wl)
+    o, C, kvr = csa.hca_forward(g["q"], g["kv"], g["gate"], g["pos_bias"], g["sinks"], wl.m, wl.L, wl.W, wl.r,
+                                wl.theta_tok, wl.theta_cmp)
+    torch.cuda.synchronize()
+    must = list(range(S - 64, S)) + [128 * j - 1 for j in (1, 2, 3, 64, 128, 255, 256, 511)] + \
+        [128 * j for j in (1, 2, 64, 128, 256, 500)]
+    rows = sample_rows(S, 64, 21, must=must)
+    Cr, kvrr = oracle.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok)
+    check_close(C, Cr, C_MAX_ABS, what="C")
+    bf16_rel_close(kvr[torch.as_tensor(rows, device=DEV)], kvrr[rows], "kv_rot")
+    ref = oracle.attend(x["q"], Cr, kvrr, None, x["sinks"], wl.m, wl.W, wl.r, wl.theta_tok, wl.theta_cmp, rows=rows)
+    got = o[torch.as_tensor(rows, device=DEV)].cpu()
+    check_close(got, ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
 def test_forward_is_deterministic():
     wl = WORKLOADS[0]
     g = prefill_inputs(wl, device=DEV)
@@ -488,8 +510,59 @@ def test_compress_append_matches_prefill_compressor(m, L, S, B):
             bf16_rel_close(win[b, (W - 1 - pos) % W].float().cpu(), kvr[pos], "window row")
 
 
+def _fp8_codes_match(codes, ref_nope, scale, what, max_ties):
+    """GPU codes against the oracle's E4M3 encoding of ref / scale (the GPU's own scale, so both take
+    the rounding decision on the same quotient). Where the quotient lies within 1e-5 relative of a
+    rounding boundary between two codes the two sides' pooled values (fp32 against fp64) may fall on
+    different sides: either neighbouring code is accepted there, and such ties are counted."""
+    q = np.asarray(ref_nope, np.float64) / np.asarray(scale, np.float64)[:, None]
+    lo = oracle.e4m3_encode((q * (1 - 1e-5)).astype(np.float32))
+    hi = oracle.e4m3_encode((q * (1 + 1e-5)).astype(np.float32))
+    want = oracle.e4m3_encode(q.astype(np.float32))
+    tie = lo != hi
+    ok = (codes == want) | (tie & ((codes == lo) | (codes == hi)))
+    assert ok.all(), f"{what}: {int((~ok).sum())} codes differ from the oracle's encoding"
+    assert int(tie.sum()) <= max_ties, f"{what}: {int(tie.sum())} near-boundary quotients"
+
+
+def test_compress_append_fp8_codes_exact():
+    """With m = L = 1 an entry is its token exactly (a one-position softmax has weight 1), so the FP8
+    codes and scales must equal the oracle's bit for bit: scale = amax/448 in binary32, codes the
+    nearest E4M3 value of x / scale with ties to the even code. Row 0 of each sequence is crafted so
+    its scale is exactly 1 and its elements sit on E4M3 rounding midpoints."""
+    wl = WORKLOADS[1].with_(m=1, L=1)
+    B, S, D, r = 2, 6, wl.D, wl.r
+    xs = [prefill_inputs(wl.with_(S=S, seed=wl.seed + 100 * b), need_index=False, need_q=False) for b in range(B)]
+    kv = torch.stack([x["kv"] for x in xs]).float()
+    mids = [448.0, 1.0625, 1.1875, -1.0625, -1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 0.0, 13.0, 15.0, 240.0, -416.0]
+    for b in range(B):
+        kv[b, 0, :D - r] = torch.tensor(mids * ((D - r) // len(mids)) + mids[:(D - r) % len(mids)])
+    kv = kv.to(torch.bfloat16)
+    gate = torch.stack([x["gate"] for x in xs])
+    bias = xs[0]["pos_bias"]
+    state_x = torch.empty(B, 1, D, dtype=torch.bfloat16, device=DEV)
+    state_g = torch.empty(B, 1, D, dtype=torch.bfloat16, device=DEV)
+    c8 = torch.zeros(B, S, D - r, dtype=torch.uint8, device=DEV)
+    c8s = torch.zeros(B, S, dtype=torch.float32, device=DEV)
+    crope = torch.zeros(B, S, r, dtype=torch.bfloat16, device=DEV)
+    kv_d, gate_d = kv.to(DEV), gate.to(DEV)
+    for P in range(S):
+        csa.compress_append(kv_d[:, P].contiguous(), gate_d[:, P].contiguous(), bias.to(DEV), state_x, state_g, P,
+                            1, r, wl.theta_cmp, wl.theta_tok, c8=c8, c8_scale=c8s, c_rope=crope)
+    torch.cuda.synchronize()
+    for b in range(B):
+        rc, rs = oracle.fp8_entry_rows(kv[b, :, :D - r].float().numpy())
+        assert np.array_equal(c8s[b].cpu().numpy(), rs), "scales"
+        assert np.array_equal(c8[b].cpu().numpy(), rc), "codes"
+        Cr, _ = oracle.compress(kv[b], gate[b], bias, 1, 1, r, wl.theta_cmp, wl.theta_tok)
+        bf16_rel_close(crope[b].float().cpu(), Cr[:, D - r:], "rope channels")
+    assert c8s[0, 0].item() == 1.0
+
+
 def test_compress_append_fp8_cache():
-    """FP8 entry cache: rope channels in bf16, the rest E4M3 codes x (amax / 448) of the entry."""
+    """FP8 entry cache of the CSA compressor (m = 4, L = 8): rope channels in bf16; scales equal the
+    oracle's amax/448 to binary32 rounding of the pooled values; codes equal the oracle's encoding of
+    the oracle's pooled value over the GPU's scale, apart from counted near-boundary quotients."""
     wl = WORKLOADS[1].with_(m=4, L=8)
     S, B, D, r = 41, 2, wl.D, wl.r
     _, _, _, _, cache, refs = _append_history(wl, B, S, fp8=True)
@@ -497,11 +570,10 @@ def test_compress_append_fp8_cache():
     for b in range(B):
         Cr = refs[b][0][:T]
         nope, rope = Cr[:, : D - r], Cr[:, D - r:]
-        scale = cache["c8_scale"][b].double().cpu().numpy()
-        np.testing.assert_allclose(scale, np.abs(nope).max(1) / 448.0, rtol=1e-3)
-        codes = cache["c8"][b].cpu().view(torch.float8_e4m3fn).double().numpy()
-        deq = codes * scale[:, None]
-        assert (np.abs(deq - nope) <= 0.0625 * np.abs(nope) + 0.002 * scale[:, None] + 1e-4).all()
+        scale = cache["c8_scale"][b].cpu().numpy()
+        _, rs = oracle.fp8_entry_rows(nope)
+        np.testing.assert_allclose(scale, rs, rtol=2.0 ** -20, atol=0)
+        _fp8_codes_match(cache["c8"][b].cpu().numpy(), nope, scale, "codes", max_ties=8)
         bf16_rel_close(cache["c_rope"][b].float().cpu(), rope, "rope channels")
 
 

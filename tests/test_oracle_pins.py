@@ -510,6 +510,76 @@ def test_fp8_e4m3_all_codes():
     assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
 
 
+def _e4m3_value(c):
+    """E4M3 value of a code from the OCP layout (sign, 4 exponent bits with bias 7, 3 mantissa bits),
+    written out here independently of the oracle's decoder."""
+    s, e, f = (c >> 7) & 1, (c >> 3) & 15, c & 7
+    v = (f / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + f / 8.0) * 2.0 ** (e - 7)
+    return -v if s else v
+
+
+def test_fp8_encode_every_code_round_trips():
+    """Every finite code's own value encodes back to that code (both zeros keep their sign)."""
+    codes = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    vals = np.array([_e4m3_value(c) for c in codes], np.float64)
+    vals[codes.index(0x80)] = -0.0
+    got = oracle.e4m3_encode(vals.astype(np.float32))
+    np.testing.assert_array_equal(got, np.array(codes, np.uint8))
+
+
+def test_fp8_encode_midpoints_round_to_even_code():
+    """Halfway between neighbouring codes the even code wins; just above or below the midpoint the
+    nearer code does. Covers the subnormal range, the subnormal/normal seam and every binade."""
+    for c in range(0, 0x7E):
+        lo, hi = _e4m3_value(c), _e4m3_value(c + 1)
+        mid = np.float32((lo + hi) / 2.0)
+        assert float(mid) == (lo + hi) / 2.0            # exactly representable in binary32
+        even = c if c % 2 == 0 else c + 1
+        assert oracle.e4m3_encode(np.array([mid]))[0] == even, hex(c)
+        assert oracle.e4m3_encode(np.array([-mid]))[0] == even | 0x80, hex(c)
+        up, down = np.nextafter(mid, np.float32(np.inf)), np.nextafter(mid, np.float32(0))
+        assert oracle.e4m3_encode(np.array([up]))[0] == c + 1
+        assert oracle.e4m3_encode(np.array([down]))[0] == c
+
+
+def test_fp8_encode_saturates_and_keeps_nan():
+    x = np.array([448.0, 449.0, 463.9, 464.0, 1e30, np.inf, -500.0, -np.inf, np.nan, 2.0 ** -11, -2.0 ** -11],
+                 np.float32)
+    got = oracle.e4m3_encode(x)
+    np.testing.assert_array_equal(got, np.array([0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F, 0x00, 0x80],
+                                                np.uint8))
+
+
+def test_fp8_encode_matches_torch_cast_in_range():
+    """torch's float8_e4m3fn cast rounds to nearest even; within +-448 it must agree code for code."""
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal(200000) * np.exp2(rng.integers(-12, 9, 200000))).astype(np.float32)
+    x = x[np.abs(x) <= 448.0]
+    ref = torch.tensor(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.e4m3_encode(x), ref)
+
+
+def test_fp8_entry_rows_scale_and_codes():
+    """Per-row scale amax/448: the largest element becomes code 448, an all-zero row keeps scale 1
+    and zero codes, and every decoded element is within half a code step of x / scale."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((40, 448)).astype(np.float32) * np.float32(3.0)
+    x[7] = 0.0
+    codes, scale = oracle.fp8_entry_rows(x)
+    assert scale[7] == 1.0 and not codes[7].any()
+    for i in range(40):
+        if i == 7:
+            continue
+        assert scale[i] == np.float32(np.abs(x[i]).max() / 448.0)
+        j = int(np.abs(x[i]).argmax())
+        assert codes[i, j] & 0x7F == 0x7E
+        q = x[i].astype(np.float64) / float(scale[i])
+        dec = np.array([_e4m3_value(int(c)) for c in codes[i]])
+        # half the spacing of the binade holding q (3 mantissa bits; subnormal spacing 2^-9)
+        half_step = np.exp2(np.maximum(np.floor(np.log2(np.maximum(np.abs(q), 2.0 ** -6))), -6) - 3) / 2
+        assert (np.abs(dec - q) <= half_step * (1 + 1e-12)).all()
+
+
 def test_bf16_decode_matches_torch():
     bits = np.random.default_rng(12).integers(0, 2 ** 16, size=4000, dtype=np.uint16)
     bits = bits[((bits >> 7) & 0xFF) != 0xFF]                                 # finite values
@@ -587,7 +657,7 @@ def test_out_proj_brute_force_tiny():
             np.testing.assert_allclose(out[t, i], sum(zb[c] * wbd[i, c] for c in range(G * R)), rtol=1e-14)
 
 
-# ---- MXFP4 indexer operands (OCP Microscaling format; DEFINITION reading R24) ------------------
+# ---- MXFP4 indexer operands (the OCP Microscaling format, which the pages name for the indexer) ----
 
 def test_mxfp4_e2m1_table():
     """The sixteen E2M1 codes decode to the OCP table (sign in bit 3) at scale 2^0 (E8M0 127)."""

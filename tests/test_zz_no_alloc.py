@@ -39,22 +39,26 @@ def call_noalloc(y, wl, B, P, o, idx, cache):
              wl.theta_cmp, 0.0, ptr(idx), ptr(o), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("wid,ctx,B", [(3, 65536, 8), (4, 131072, 4)])
-def test_noalloc_decode_matches_decode(wid, ctx, B):
-    wl = WORKLOADS[wid].with_(ctx=ctx)
-    y = decode_inputs(wl, device="cuda", batch=B)
-    P = wl.ctx - 1
-    kw = dict(C=y["C"]) if wl.cache == "bf16" else dict(c8=y["c8"], c8_scale=y["scale"], c_rope=y["rope"])
-    ref_o, ref_idx = csa.decode(y["q"], y["qI"], y["w"], y["kI"], y["win"], y["sinks"], P, wl.topk, wl.r,
-                                wl.theta_tok, wl.theta_cmp, **kw)
-    torch.cuda.synchronize()
-    for _ in range(2):
+@pytest.mark.parametrize("wid,ctx,B,B2", [(3, 65536, 8, 6), (4, 131072, 4, 3), (3, 262144, 2, 1)])
+def test_noalloc_decode_matches_decode(wid, ctx, B, B2):
+    """Two calls in a row on different inputs (another seed and batch): each must equal csa_decode on
+    the same inputs, so nothing the first call left in the shared array leaks into the second. The
+    last case has 65536 entries per sequence, past the single-CTA top-k, so the chunked top-k's
+    histograms, bitmap and candidates live in the shared array too."""
+    for call, (seed_add, batch) in enumerate([(0, B), (17, B2)]):
+        wl = WORKLOADS[wid].with_(ctx=ctx, seed=WORKLOADS[wid].seed + seed_add)
+        y = decode_inputs(wl, device="cuda", batch=batch)
+        P = wl.ctx - 1
+        kw = dict(C=y["C"]) if wl.cache == "bf16" else dict(c8=y["c8"], c8_scale=y["scale"], c_rope=y["rope"])
+        ref_o, ref_idx = csa.decode(y["q"], y["qI"], y["w"], y["kI"], y["win"], y["sinks"], P, wl.topk, wl.r,
+                                    wl.theta_tok, wl.theta_cmp, **kw)
+        torch.cuda.synchronize()
         o = torch.full_like(ref_o, float("nan"))
         idx = torch.full_like(ref_idx, -7)
-        assert call_noalloc(y, wl, B, P, o, idx, wl.cache) == 0
+        assert call_noalloc(y, wl, batch, P, o, idx, wl.cache) == 0, call
         torch.cuda.synchronize()
-        check_close(o, ref_o.cpu().double().numpy(), O_MAX_ABS, O_MEAN_ABS, what="o")
-        assert torch.equal(idx, ref_idx)
+        check_close(o, ref_o.cpu().double().numpy(), O_MAX_ABS, O_MEAN_ABS, what=f"o (call {call})")
+        assert torch.equal(idx, ref_idx), call
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
@@ -71,3 +75,8 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
            ptr(y["sinks"]), 64, wl.H, wl.D, 1 << 20, wl.HI, wl.dI, wl.topk, wl.W, wl.r, wl.ctx - 1, wl.theta_tok,
            wl.theta_cmp, 0.0, ptr(idx), ptr(o), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == 5   # CSA_ERR_WORKSPACE
+    # sizes whose byte counts would overflow are refused as invalid, also before anything is launched
+    rc = f(ptr(y["q"]), ptr(y["qI"]), ptr(y["w"]), ptr(y["kI"]), ptr(y["C"]), None, None, None, ptr(y["win"]),
+           ptr(y["sinks"]), 1 << 30, wl.H, wl.D, 1 << 40, wl.HI, wl.dI, wl.topk, wl.W, wl.r, wl.ctx - 1, wl.theta_tok,
+           wl.theta_cmp, 0.0, ptr(idx), ptr(o), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 1   # CSA_ERR_INVALID_ARG
