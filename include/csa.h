@@ -26,6 +26,11 @@
  *     key is skipped). Read it with csa_get_device_status after the call.
  *   - Calls on the same workspace must not overlap on the GPU.
  *   - Nothing here aborts, traps or asserts on the device.
+ *   - Prefill calls (1-5) take a chunk of S tokens at positions pos0 .. pos0+S-1 ([HF-V4 "Cache
+ *     layers"]: the compressor and indexer state carries over between forward calls). Per-query
+ *     tensors (q, qI, w, idx, o) hold the chunk's S rows; tensors of the whole history (kv, gate,
+ *     kv_rot, C, kI) are indexed by absolute position or entry. A chunk's results equal rows
+ *     pos0 .. pos0+S-1 of one prefill over positions 0 .. pos0+S-1. pos0 = 0 is a whole prefill.
  */
 #ifndef CSA_B200_H
 #define CSA_B200_H
@@ -87,67 +92,79 @@ CSA_API size_t csa_workspace_size(csa_op op, const csa_dims *dims);
 CSA_API csa_status csa_get_device_status(const void *workspace, int32_t *status, void *stream);
 
 /* ---- 1. compressor ------------------------------------------------------------------------------
- * [HF-V4 "Hybrid attention"; digest]. Entry w (0 <= w < T = floor(S/m)) pools the window
- * [(w+1)m - L, (w+1)m) clipped to [0,S): per channel d, softmax over positions j of
- * gate[j,d] + pos_bias[j - ((w+1)m - L)], weights applied to kv[j,d]. CSA: L = 2m (overlapping),
- * HCA: L = m. The entry is then RoPE-rotated at position w*m with theta_cmp on its last rope_dim
- * channels (interleaved pairs). kv_rot[j] = kv[j] rotated at position j with theta_tok.
- *   kv, gate   [S, D] bf16            pos_bias [L] fp32
- *   C          [T, D] bf16 (out)      kv_rot   [S, D] bf16 (out, may be NULL)
- * Requires D % 8 == 0, rope_dim even, rope_dim % 8 == 0, rope_dim <= D, 1 <= m <= L <= 4096. */
+ * [HF-V4 "Hybrid attention"; digest]. Entry w pools the window [(w+1)m - L, (w+1)m) clipped at
+ * position 0: per channel d, softmax over positions j of gate[j,d] + pos_bias[j - ((w+1)m - L)],
+ * weights applied to kv[j,d]. CSA: L = 2m (overlapping), HCA: L = m. The entry is then
+ * RoPE-rotated at position w*m with theta_cmp on its last rope_dim channels (interleaved pairs).
+ * kv_rot[j] = kv[j] rotated at position j with theta_tok. A chunk at pos0 writes the entries whose
+ * window closes inside it, w in [floor(pos0/m), floor((pos0+S)/m)), and kv_rot rows [pos0, pos0+S).
+ *   kv, gate   [pos0 + S, D] bf16 by position; rows before max(0, floor(pos0/m)*m + m - L) are not
+ *              read (an entry closing in the chunk may pool positions before pos0)
+ *   pos_bias   [L] fp32
+ *   C          [floor((pos0+S)/m), D] bf16 (out: the chunk's entries; earlier rows untouched)
+ *   kv_rot     [pos0 + S, D] bf16 (out: rows [pos0, pos0+S); may be NULL)
+ * Requires D % 8 == 0, rope_dim even, rope_dim % 8 == 0, rope_dim <= D, 1 <= m <= L <= 4096,
+ * 0 <= pos0 <= 2^40. */
 CSA_API csa_status csa_compress(const void *kv, const void *gate, const float *pos_bias,
-                        int64_t S, int32_t D, int32_t m, int32_t L, int32_t rope_dim,
+                        int64_t S, int64_t pos0, int32_t D, int32_t m, int32_t L, int32_t rope_dim,
                         double theta_cmp, double theta_tok,
                         void *C, void *kv_rot, void *stream);
 
 /* ---- 2. lightning indexer + top-k (prefill) ----------------------------------------------------
  * [HF-V4 "Hybrid attention", CSA; "Attention mask layout", CSA layer; digest].
- * I[t,s] = sum_h w[t,h] * ReLU(qI[t,h,:] . kI[s,:]) for visible entries s < floor((t+1)/m);
- * idx[t] = the min(k, vis) largest, ties to the smaller s, written in ascending index order,
+ * For the query at position t = pos0 + i (row i of the chunk):
+ * I[t,s] = sum_h w[i,h] * ReLU(qI[i,h,:] . kI[s,:]) for visible entries s < vis(t) = min(T, floor((t+1)/m));
+ * idx[i] = the min(k, vis) largest, ties to the smaller s, written in ascending index order,
  * remaining slots -1.
- *   qI [S, HI, dI] bf16   kI [T, dI] bf16   w [S, HI] fp32   idx [S, k] int32 (out)
+ *   qI [S, HI, dI] bf16   kI [T, dI] bf16 (every entry so far, T <= floor((pos0+S)/m))
+ *   w [S, HI] fp32        idx [S, k] int32 (out)
  * Requires dI % 8 == 0, 1 <= k. */
 CSA_API csa_status csa_index_topk(const void *qI, const void *kI, const float *w,
-                          int64_t S, int64_t T, int32_t HI, int32_t dI, int32_t m, int32_t k,
+                          int64_t S, int64_t pos0, int64_t T, int32_t HI, int32_t dI, int32_t m, int32_t k,
                           int32_t *idx, void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---- 3. sparse + window attention (CSA prefill) ---------------------------------------------
  * [HF-V4 "Hybrid attention": shared K=V MQA, partial interleaved RoPE, output rope slice rotated
  * at -i (eq. 26), per-head sink (eq. 27), sliding-window branch; "Attention mask layout"].
- * For query t, head h: keys = kv_rot[j] for j in [t-W+1, t] (window) plus C[s] for s in idx[t]
- * (s != -1). Logits lambda*(R_tok(t) q).kv_rot[j] and lambda*(R_cmp(t) q).C[s]; one softmax over
- * all keys plus exp(sinks[h]); K = V; each branch's rope slice rotated back by -t with its theta.
- *   q [S, H, D] bf16 (un-rotated)   C [T, D] bf16 (post-RoPE)   kv_rot [S, D] bf16 (post-RoPE)
+ * For the query at position t = pos0 + i (row i), head h: keys = kv_rot[j] for j in [t-W+1, t]
+ * (window) plus C[s] for s in idx[i] (s != -1). Logits lambda*(R_tok(t) q).kv_rot[j] and
+ * lambda*(R_cmp(t) q).C[s]; one softmax over all keys plus exp(sinks[h]); K = V; each branch's
+ * rope slice rotated back by -t with its theta.
+ *   q [S, H, D] bf16 (un-rotated)   C [T, D] bf16 (post-RoPE, T <= floor((pos0+S)/m))
+ *   kv_rot [pos0 + S, D] bf16 (post-RoPE, by position)
  *   idx [S, k] int32                sinks [H] fp32               o [S, H, D] fp32 (out)
- * softmax_scale <= 0 selects 1/sqrt(D). Index values >= floor((t+1)/m) are skipped and reported
- * as CSA_ERR_INVALID_ARG in the workspace status. */
+ * softmax_scale <= 0 selects 1/sqrt(D). Index values >= vis(t) are skipped and reported as
+ * CSA_ERR_INVALID_ARG in the workspace status. */
 CSA_API csa_status csa_attend(const void *q, const void *C, const void *kv_rot, const int32_t *idx,
-                      const float *sinks, int64_t S, int32_t H, int32_t D, int64_t T, int32_t k,
+                      const float *sinks, int64_t S, int64_t pos0, int32_t H, int32_t D, int64_t T, int32_t k,
                       int32_t W, int32_t rope_dim, int32_t m, double theta_tok, double theta_cmp,
                       float softmax_scale, float *o, void *workspace, size_t workspace_bytes,
                       void *stream);
 
 /* ---- 4. dense compressed + window attention (HCA prefill) --------------------------------------
  * [HF-V4 "Hybrid attention", HCA; "Attention mask layout", HCA layer]. As csa_attend with the
- * entry branch = every visible entry C[w], w < floor((t+1)/m). */
+ * entry branch = every visible entry C[w], w < vis(t), t = pos0 + i. */
 CSA_API csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const float *sinks,
-                      int64_t S, int32_t H, int32_t D, int64_t T, int32_t W, int32_t rope_dim,
+                      int64_t S, int64_t pos0, int32_t H, int32_t D, int64_t T, int32_t W, int32_t rope_dim,
                       int32_t m, double theta_tok, double theta_cmp, float softmax_scale, float *o,
                       void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---- 5. fused layer forward ----------------------------------------------------------------------
  * csa_forward = csa_compress (L = 2m) -> csa_index_topk -> csa_attend, in stream order.
  * hca_forward = csa_compress (L = m)  -> hca_attend. Intermediates C, kv_rot, idx are
- * caller-provided outputs (kv_rot and C are needed by later decode steps as cache). */
+ * caller-provided outputs (kv_rot and C are needed by later decode steps as cache). For a chunk at
+ * pos0, kv, gate and kv_rot are [pos0 + S, D] by position, C is [floor((pos0+S)/m), D] holding the
+ * earlier chunks' entries, kI [floor((pos0+S)/m), dI] every entry's index key; the rest are the
+ * chunk's S rows. */
 CSA_API csa_status csa_forward(const void *q, const void *kv, const void *gate, const float *pos_bias,
                        const void *qI, const void *kI, const float *w, const float *sinks,
-                       int64_t S, int32_t H, int32_t D, int32_t HI, int32_t dI, int32_t m, int32_t L,
+                       int64_t S, int64_t pos0, int32_t H, int32_t D, int32_t HI, int32_t dI, int32_t m, int32_t L,
                        int32_t k, int32_t W, int32_t rope_dim, double theta_tok, double theta_cmp,
                        float softmax_scale, void *C, void *kv_rot, int32_t *idx, float *o,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 CSA_API csa_status hca_forward(const void *q, const void *kv, const void *gate, const float *pos_bias,
-                       const float *sinks, int64_t S, int32_t H, int32_t D, int32_t m, int32_t L,
+                       const float *sinks, int64_t S, int64_t pos0, int32_t H, int32_t D, int32_t m, int32_t L,
                        int32_t W, int32_t rope_dim, double theta_tok, double theta_cmp,
                        float softmax_scale, void *C, void *kv_rot, float *o,
                        void *workspace, size_t workspace_bytes, void *stream);
@@ -216,11 +233,11 @@ CSA_API csa_status hca_decode(const void *q, const void *C, const uint8_t *c8, c
                       double theta_cmp, float softmax_scale, float *o, void *workspace,
                       size_t workspace_bytes, void *stream);
 
-/* swa_attend: prefill of a sliding-window-only layer. For query t, head h: keys kv_rot[j] for
- * j in [t-W+1, t] (post-RoPE at theta_tok), one softmax with exp(sinks[h]), K = V, the output rope
- * slice rotated back by -t with theta_tok; no compressed entries. Arguments as hca_attend without
- * C, T, m and theta_cmp. Workspace: 256 bytes (the status word). */
-CSA_API csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int64_t S, int32_t H,
+/* swa_attend: prefill of a sliding-window-only layer. For the query at position t = pos0 + i, head h:
+ * keys kv_rot[j] for j in [t-W+1, t] (post-RoPE at theta_tok), one softmax with exp(sinks[h]),
+ * K = V, the output rope slice rotated back by -t with theta_tok; no compressed entries. Arguments
+ * as hca_attend without C, T, m and theta_cmp. Workspace: 256 bytes (the status word). */
+CSA_API csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int64_t S, int64_t pos0, int32_t H,
                       int32_t D, int32_t W, int32_t rope_dim, double theta_tok, float softmax_scale,
                       float *o, void *workspace, size_t workspace_bytes, void *stream);
 

@@ -60,19 +60,19 @@ def lib():
             "csa_version": (ctypes.c_char_p, []),
             "csa_workspace_size": (SZ, [I32, ctypes.POINTER(_Dims)]),
             "csa_get_device_status": (I32, [P, ctypes.POINTER(ctypes.c_int32), P]),
-            "csa_compress": (I32, [P, P, P, I64, I32, I32, I32, I32, F64, F64, P, P, P]),
-            "csa_index_topk": (I32, [P, P, P, I64, I64, I32, I32, I32, I32, P, P, SZ, P]),
-            "csa_attend": (I32, [P, P, P, P, P, I64, I32, I32, I64, I32, I32, I32, I32, F64, F64, F32, P, P,
+            "csa_compress": (I32, [P, P, P, I64, I64, I32, I32, I32, I32, F64, F64, P, P, P]),
+            "csa_index_topk": (I32, [P, P, P, I64, I64, I64, I32, I32, I32, I32, P, P, SZ, P]),
+            "csa_attend": (I32, [P, P, P, P, P, I64, I64, I32, I32, I64, I32, I32, I32, I32, F64, F64, F32, P, P,
                                  SZ, P]),
-            "hca_attend": (I32, [P, P, P, P, I64, I32, I32, I64, I32, I32, I32, F64, F64, F32, P, P, SZ, P]),
-            "csa_forward": (I32, [P, P, P, P, P, P, P, P, I64, I32, I32, I32, I32, I32, I32, I32, I32, I32, F64,
-                                  F64, F32, P, P, P, P, P, SZ, P]),
-            "hca_forward": (I32, [P, P, P, P, P, I64, I32, I32, I32, I32, I32, I32, F64, F64, F32, P, P, P, P,
+            "hca_attend": (I32, [P, P, P, P, I64, I64, I32, I32, I64, I32, I32, I32, F64, F64, F32, P, P, SZ, P]),
+            "csa_forward": (I32, [P, P, P, P, P, P, P, P, I64, I64, I32, I32, I32, I32, I32, I32, I32, I32, I32,
+                                  F64, F64, F32, P, P, P, P, P, SZ, P]),
+            "hca_forward": (I32, [P, P, P, P, P, I64, I64, I32, I32, I32, I32, I32, I32, F64, F64, F32, P, P, P, P,
                                   SZ, P]),
             "csa_decode": (I32, [P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, I32, I64,
                                  F64, F64, F32, P, P, P, SZ, P]),
             "hca_decode": (I32, [P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I64, F64, F64, F32, P, P, SZ, P]),
-            "swa_attend": (I32, [P, P, P, I64, I32, I32, I32, I32, F64, F32, P, P, SZ, P]),
+            "swa_attend": (I32, [P, P, P, I64, I64, I32, I32, I32, I32, F64, F32, P, P, SZ, P]),
             "csa_compress_append": (I32, [P, P, P, P, P, I32, I32, I32, I32, I32, I64, F64, F64, P, P, P, P, I64, P,
                                           I32, P]),
             "csa_out_proj": (I32, [P, P, P, I64, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
@@ -139,111 +139,143 @@ def get_device_status(ws: torch.Tensor, stream=None) -> int:
 # ---- the calls ----------------------------------------------------------------------------------------
 
 def compress(kv, gate, pos_bias, m: int, L: int, rope_dim: int, theta_cmp: float, theta_tok: float,
-             C=None, kv_rot=None, want_kv_rot: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
-    S, D = kv.shape
-    T = S // m
-    _dev(kv, torch.bfloat16, "kv", (S, D))
-    _dev(gate, torch.bfloat16, "gate", (S, D))
+             C=None, kv_rot=None, want_kv_rot: bool = True, pos0: int = 0,
+             stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kv, gate [N, D] by position (N = pos0 + S). Writes the entries closing in the chunk
+    [pos0, N) into C [N // m, D] and rows [pos0, N) into kv_rot [N, D]; with pos0 > 0 pass the
+    caches (C, kv_rot) holding the earlier chunks."""
+    N, D = kv.shape
+    S = N - int(pos0)
+    if S < 0:
+        raise ValueError("kv holds fewer rows than pos0")
+    T = N // m
+    _dev(kv, torch.bfloat16, "kv", (N, D))
+    _dev(gate, torch.bfloat16, "gate", (N, D))
     _dev(pos_bias, torch.float32, "pos_bias", (L,))
+    if pos0 > 0 and (C is None or (want_kv_rot and kv_rot is None)):
+        raise ValueError("a chunk at pos0 > 0 needs the caches C and kv_rot of the earlier chunks")
     C = torch.empty(T, D, dtype=torch.bfloat16, device=kv.device) if C is None else _dev(C, torch.bfloat16, "C", (T, D))
     if want_kv_rot:
-        kv_rot = torch.empty_like(kv) if kv_rot is None else _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+        kv_rot = torch.empty_like(kv) if kv_rot is None else _dev(kv_rot, torch.bfloat16, "kv_rot", (N, D))
     else:
         kv_rot = None
-    _check("csa_compress", lib().csa_compress(_ptr(kv), _ptr(gate), _ptr(pos_bias), S, D, m, L, rope_dim,
+    _check("csa_compress", lib().csa_compress(_ptr(kv), _ptr(gate), _ptr(pos_bias), S, int(pos0), D, m, L, rope_dim,
                                               float(theta_cmp), float(theta_tok), _ptr(C), _ptr(kv_rot),
                                               _stream(stream)))
     return C, kv_rot
 
 
-def index_topk(qI, kI, w, m: int, k: int, idx=None, workspace=None, stream=None) -> torch.Tensor:
+def index_topk(qI, kI, w, m: int, k: int, idx=None, workspace=None, pos0: int = 0, stream=None) -> torch.Tensor:
+    """qI [S, HI, dI], w [S, HI] of the queries at positions pos0 .. pos0+S-1; kI [T, dI] every entry
+    so far. Returns idx [S, k]."""
     S, HI, dI = qI.shape
     T = kI.shape[0]
     _dev(qI, torch.bfloat16, "qI")
     _dev(kI, torch.bfloat16, "kI", (T, dI))
     _dev(w, torch.float32, "w", (S, HI))
     idx = torch.empty(S, k, dtype=torch.int32, device=qI.device) if idx is None else _dev(idx, torch.int32, "idx", (S, k))
-    ws = _workspace("index_topk", qI.device, workspace, S=S, T=T)
-    _check("csa_index_topk", lib().csa_index_topk(_ptr(qI), _ptr(kI), _ptr(w), S, T, HI, dI, m, k, _ptr(idx),
-                                                  _ptr(ws), ws.numel(), _stream(stream)))
+    ws = _workspace("index_topk", qI.device, workspace, S=S, T=T, HI=HI, dI=dI, k=k)
+    _check("csa_index_topk", lib().csa_index_topk(_ptr(qI), _ptr(kI), _ptr(w), S, int(pos0), T, HI, dI, m, k,
+                                                  _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
     return idx
 
 
 def attend(q, C, kv_rot, idx, sinks, m: int, W: int, rope_dim: int, theta_tok: float, theta_cmp: float,
-           softmax_scale: float = 0.0, o=None, workspace=None, stream=None) -> torch.Tensor:
+           softmax_scale: float = 0.0, o=None, workspace=None, pos0: int = 0, stream=None) -> torch.Tensor:
+    """q [S, H, D] and idx [S, k] of the queries at positions pos0 .. pos0+S-1; C [T, D]; kv_rot
+    [pos0 + S, D] by position. Returns o [S, H, D] fp32."""
     S, H, D = q.shape
     T = C.shape[0]
     k = idx.shape[1]
     _dev(q, torch.bfloat16, "q")
     _dev(C, torch.bfloat16, "C", (T, D))
-    _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (int(pos0) + S, D))
     _dev(idx, torch.int32, "idx", (S, k))
     _dev(sinks, torch.float32, "sinks", (H,))
     o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
     ws = _workspace("attend", q.device, workspace)
-    _check("csa_attend", lib().csa_attend(_ptr(q), _ptr(C), _ptr(kv_rot), _ptr(idx), _ptr(sinks), S, H, D, T, k, W,
+    _check("csa_attend", lib().csa_attend(_ptr(q), _ptr(C), _ptr(kv_rot), _ptr(idx), _ptr(sinks), S, int(pos0), H, D,
+                                          T, k, W, rope_dim, m, float(theta_tok), float(theta_cmp),
+                                          float(softmax_scale), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def hca_attend(q, C, kv_rot, sinks, m: int, W: int, rope_dim: int, theta_tok: float, theta_cmp: float,
+               softmax_scale: float = 0.0, o=None, workspace=None, pos0: int = 0, stream=None) -> torch.Tensor:
+    S, H, D = q.shape
+    T = C.shape[0]
+    _dev(q, torch.bfloat16, "q")
+    _dev(C, torch.bfloat16, "C", (T, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (int(pos0) + S, D))
+    _dev(sinks, torch.float32, "sinks", (H,))
+    o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
+    ws = _workspace("attend", q.device, workspace)
+    _check("hca_attend", lib().hca_attend(_ptr(q), _ptr(C), _ptr(kv_rot), _ptr(sinks), S, int(pos0), H, D, T, W,
                                           rope_dim, m, float(theta_tok), float(theta_cmp), float(softmax_scale),
                                           _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
     return o
 
 
-def hca_attend(q, C, kv_rot, sinks, m: int, W: int, rope_dim: int, theta_tok: float, theta_cmp: float,
-               softmax_scale: float = 0.0, o=None, workspace=None, stream=None) -> torch.Tensor:
-    S, H, D = q.shape
-    T = C.shape[0]
-    _dev(q, torch.bfloat16, "q")
-    _dev(C, torch.bfloat16, "C", (T, D))
-    _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
-    _dev(sinks, torch.float32, "sinks", (H,))
-    o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
-    ws = _workspace("attend", q.device, workspace)
-    _check("hca_attend", lib().hca_attend(_ptr(q), _ptr(C), _ptr(kv_rot), _ptr(sinks), S, H, D, T, W, rope_dim, m,
-                                          float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(o),
-                                          _ptr(ws), ws.numel(), _stream(stream)))
-    return o
-
-
 def csa_forward(q, kv, gate, pos_bias, qI, kI, w, sinks, m: int, L: int, k: int, W: int, rope_dim: int,
                 theta_tok: float, theta_cmp: float, softmax_scale: float = 0.0, out=None, workspace=None,
-                stream=None):
-    """Returns (o, C, kv_rot, idx). `out` may pass preallocated (o, C, kv_rot, idx)."""
+                pos0: int = 0, stream=None):
+    """Returns (o, C, kv_rot, idx). `out` may pass preallocated (o, C, kv_rot, idx). For a chunk at
+    pos0 > 0, kv and gate are [pos0 + S, D] by position, kI [(pos0 + S) // m, dI] holds every entry's
+    index key, and `out` must carry the caches C [(pos0 + S) // m, D] and kv_rot [pos0 + S, D] of the
+    earlier chunks; q, qI, w, o and idx hold the chunk's S rows."""
     S, H, D = q.shape
     HI, dI = qI.shape[1], qI.shape[2]
-    T = S // m
-    for t, n, dt in ((q, "q", torch.bfloat16), (kv, "kv", torch.bfloat16), (gate, "gate", torch.bfloat16),
-                     (pos_bias, "pos_bias", torch.float32), (qI, "qI", torch.bfloat16), (kI, "kI", torch.bfloat16),
-                     (w, "w", torch.float32), (sinks, "sinks", torch.float32)):
-        _dev(t, dt, n)
+    N = int(pos0) + S
+    T = N // m
+    for t, n, dt, shp in ((q, "q", torch.bfloat16, None), (kv, "kv", torch.bfloat16, (N, D)),
+                          (gate, "gate", torch.bfloat16, (N, D)), (pos_bias, "pos_bias", torch.float32, None),
+                          (qI, "qI", torch.bfloat16, (S, HI, dI)), (kI, "kI", torch.bfloat16, (T, dI)),
+                          (w, "w", torch.float32, (S, HI)), (sinks, "sinks", torch.float32, None)):
+        _dev(t, dt, n, shp)
     if out is None:
+        if pos0 > 0:
+            raise ValueError("a chunk at pos0 > 0 needs out=(o, C, kv_rot, idx) with the earlier chunks' caches")
         dev = q.device
         out = (torch.empty(S, H, D, dtype=torch.float32, device=dev), torch.empty(T, D, dtype=torch.bfloat16, device=dev),
-               torch.empty(S, D, dtype=torch.bfloat16, device=dev), torch.empty(S, k, dtype=torch.int32, device=dev))
+               torch.empty(N, D, dtype=torch.bfloat16, device=dev), torch.empty(S, k, dtype=torch.int32, device=dev))
     o, C, kv_rot, idx = out
-    ws = _workspace("csa_forward", q.device, workspace, S=S, T=T)
+    _dev(o, torch.float32, "o", (S, H, D))
+    _dev(C, torch.bfloat16, "C", (T, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (N, D))
+    _dev(idx, torch.int32, "idx", (S, k))
+    ws = _workspace("csa_forward", q.device, workspace, S=S, T=T, HI=HI, dI=dI, k=k)
     _check("csa_forward", lib().csa_forward(_ptr(q), _ptr(kv), _ptr(gate), _ptr(pos_bias), _ptr(qI), _ptr(kI), _ptr(w),
-                                            _ptr(sinks), S, H, D, HI, dI, m, L, k, W, rope_dim, float(theta_tok),
-                                            float(theta_cmp), float(softmax_scale), _ptr(C), _ptr(kv_rot), _ptr(idx),
-                                            _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+                                            _ptr(sinks), S, int(pos0), H, D, HI, dI, m, L, k, W, rope_dim,
+                                            float(theta_tok), float(theta_cmp), float(softmax_scale), _ptr(C),
+                                            _ptr(kv_rot), _ptr(idx), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
     return o, C, kv_rot, idx
 
 
 def hca_forward(q, kv, gate, pos_bias, sinks, m: int, L: int, W: int, rope_dim: int, theta_tok: float,
-                theta_cmp: float, softmax_scale: float = 0.0, out=None, workspace=None, stream=None):
-    """Returns (o, C, kv_rot)."""
+                theta_cmp: float, softmax_scale: float = 0.0, out=None, workspace=None, pos0: int = 0, stream=None):
+    """Returns (o, C, kv_rot). For a chunk at pos0 > 0 see csa_forward (out = (o, C, kv_rot))."""
     S, H, D = q.shape
-    T = S // m
-    for t, n, dt in ((q, "q", torch.bfloat16), (kv, "kv", torch.bfloat16), (gate, "gate", torch.bfloat16),
-                     (pos_bias, "pos_bias", torch.float32), (sinks, "sinks", torch.float32)):
-        _dev(t, dt, n)
+    N = int(pos0) + S
+    T = N // m
+    for t, n, dt, shp in ((q, "q", torch.bfloat16, None), (kv, "kv", torch.bfloat16, (N, D)),
+                          (gate, "gate", torch.bfloat16, (N, D)), (pos_bias, "pos_bias", torch.float32, None),
+                          (sinks, "sinks", torch.float32, None)):
+        _dev(t, dt, n, shp)
     if out is None:
+        if pos0 > 0:
+            raise ValueError("a chunk at pos0 > 0 needs out=(o, C, kv_rot) with the earlier chunks' caches")
         dev = q.device
         out = (torch.empty(S, H, D, dtype=torch.float32, device=dev), torch.empty(T, D, dtype=torch.bfloat16, device=dev),
-               torch.empty(S, D, dtype=torch.bfloat16, device=dev))
+               torch.empty(N, D, dtype=torch.bfloat16, device=dev))
     o, C, kv_rot = out
+    _dev(o, torch.float32, "o", (S, H, D))
+    _dev(C, torch.bfloat16, "C", (T, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (N, D))
     ws = _workspace("hca_forward", q.device, workspace)
-    _check("hca_forward", lib().hca_forward(_ptr(q), _ptr(kv), _ptr(gate), _ptr(pos_bias), _ptr(sinks), S, H, D, m, L,
-                                            W, rope_dim, float(theta_tok), float(theta_cmp), float(softmax_scale),
-                                            _ptr(C), _ptr(kv_rot), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    _check("hca_forward", lib().hca_forward(_ptr(q), _ptr(kv), _ptr(gate), _ptr(pos_bias), _ptr(sinks), S, int(pos0),
+                                            H, D, m, L, W, rope_dim, float(theta_tok), float(theta_cmp),
+                                            float(softmax_scale), _ptr(C), _ptr(kv_rot), _ptr(o), _ptr(ws),
+                                            ws.numel(), _stream(stream)))
     return o, C, kv_rot
 
 
@@ -359,16 +391,18 @@ def hca_decode(q, win, sinks, P: int, rope_dim: int, theta_tok: float, theta_cmp
 
 
 def swa_attend(q, kv_rot, sinks, W: int, rope_dim: int, theta_tok: float, softmax_scale: float = 0.0, o=None,
-               workspace=None, stream=None) -> torch.Tensor:
-    """Sliding-window-only layer prefill: window rows kv_rot [S,D] and the sink. Returns o [S,H,D] fp32."""
+               workspace=None, pos0: int = 0, stream=None) -> torch.Tensor:
+    """Sliding-window-only layer prefill of the queries at positions pos0 .. pos0+S-1: window rows
+    kv_rot [pos0 + S, D] by position and the sink. Returns o [S,H,D] fp32."""
     S, H, D = q.shape
     _dev(q, torch.bfloat16, "q")
-    _dev(kv_rot, torch.bfloat16, "kv_rot", (S, D))
+    _dev(kv_rot, torch.bfloat16, "kv_rot", (int(pos0) + S, D))
     _dev(sinks, torch.float32, "sinks", (H,))
     o = torch.empty(S, H, D, dtype=torch.float32, device=q.device) if o is None else _dev(o, torch.float32, "o", (S, H, D))
     ws = _workspace("attend", q.device, workspace)
-    _check("swa_attend", lib().swa_attend(_ptr(q), _ptr(kv_rot), _ptr(sinks), S, H, D, W, rope_dim, float(theta_tok),
-                                          float(softmax_scale), _ptr(o), _ptr(ws), ws.numel(), _stream(stream)))
+    _check("swa_attend", lib().swa_attend(_ptr(q), _ptr(kv_rot), _ptr(sinks), S, int(pos0), H, D, W, rope_dim,
+                                          float(theta_tok), float(softmax_scale), _ptr(o), _ptr(ws), ws.numel(),
+                                          _stream(stream)))
     return o
 
 

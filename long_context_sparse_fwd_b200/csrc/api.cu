@@ -58,12 +58,13 @@ csa_status reset_status(void *ws, cudaStream_t stream)
     return CSA_OK;
 }
 
-csa_status check_compress(const void *kv, const void *gate, const float *pos_bias, int64_t S, int32_t D, int32_t m,
-                          int32_t L, int32_t r, double theta_cmp, double theta_tok, const void *C)
+csa_status check_compress(const void *kv, const void *gate, const float *pos_bias, int64_t S, int64_t pos0,
+                          int32_t D, int32_t m, int32_t L, int32_t r, double theta_cmp, double theta_tok, const void *C)
 {
-    CSA_CHECK_ARG(S >= 0 && D > 0 && m >= 1 && L >= m && r >= 0 && r <= D && (r % 2) == 0);
+    CSA_CHECK_ARG(S >= 0 && pos0 >= 0 && pos0 <= ((int64_t)1 << 40) && D > 0 && m >= 1 && L >= m && r >= 0 &&
+                  r <= D && (r % 2) == 0);
     CSA_CHECK_ARG(S == 0 || (kv != nullptr && gate != nullptr && pos_bias != nullptr));
-    CSA_CHECK_ARG(S / m == 0 || C != nullptr);
+    CSA_CHECK_ARG((pos0 + S) / m == pos0 / m || C != nullptr);   // entries close in this chunk
     CSA_CHECK_ARG(r == 0 || (theta_ok(theta_cmp) && theta_ok(theta_tok)));
     CSA_CHECK_SUP(D % 8 == 0 && r % 8 == 0 && L <= 4096);
     CSA_CHECK_ARG(aligned16(kv) && aligned16(gate) && aligned16(C));
@@ -71,11 +72,12 @@ csa_status check_compress(const void *kv, const void *gate, const float *pos_bia
 }
 
 csa_status check_attend_common(const void *q, const void *C, const void *kv_rot, const float *sinks, int64_t S,
-                               int32_t H, int32_t D, int64_t T, int32_t W, int32_t r, int32_t m, double theta_tok,
-                               double theta_cmp, const float *o)
+                               int64_t pos0, int32_t H, int32_t D, int64_t T, int32_t W, int32_t r, int32_t m,
+                               double theta_tok, double theta_cmp, const float *o)
 {
-    CSA_CHECK_ARG(S >= 0 && H > 0 && D > 0 && T >= 0 && W >= 0 && m >= 1 && r >= 0 && r <= D && (r % 2) == 0);
-    CSA_CHECK_ARG(T <= S / m);
+    CSA_CHECK_ARG(S >= 0 && pos0 >= 0 && pos0 <= ((int64_t)1 << 40) && H > 0 && D > 0 && T >= 0 && W >= 0 &&
+                  m >= 1 && r >= 0 && r <= D && (r % 2) == 0);
+    CSA_CHECK_ARG(T <= (pos0 + S) / m);
     CSA_CHECK_ARG(S == 0 || (q != nullptr && sinks != nullptr && o != nullptr));
     CSA_CHECK_ARG(S == 0 || W == 0 || kv_rot != nullptr);
     CSA_CHECK_ARG(T == 0 || C != nullptr);
@@ -87,8 +89,8 @@ csa_status check_attend_common(const void *q, const void *C, const void *kv_rot,
 }
 
 AttnArgs prefill_args(const void *q, const void *C, const void *kv_rot, const int32_t *idx, const float *sinks,
-                      int64_t S, int32_t H, int32_t D, int64_t T, int32_t k, int32_t W, int32_t r, int32_t m,
-                      double theta_tok, double theta_cmp, float scale, float *o, void *ws)
+                      int64_t S, int64_t pos0, int32_t H, int32_t D, int64_t T, int32_t k, int32_t W, int32_t r,
+                      int32_t m, double theta_tok, double theta_cmp, float scale, float *o, void *ws)
 {
     AttnArgs a;
     memset(&a, 0, sizeof a);
@@ -100,6 +102,7 @@ AttnArgs prefill_args(const void *q, const void *C, const void *kv_rot, const in
     a.o = o;
     a.status = static_cast<int32_t *>(ws);
     a.R = S;
+    a.pos0 = pos0;
     a.T = T;
     a.H = H;
     a.D = D;
@@ -164,16 +167,16 @@ cudaError_t attend_any(const AttnArgs &a, cudaStream_t st)
 
 // Prefill indexer + top-k: the tcgen05 kernel with on-chip scores where it applies, else the
 // general path (scores through the workspace, then a radix select per row).
-cudaError_t index_topk_any(const void *qI, const void *kI, const float *w, int64_t S, int64_t T, int32_t HI,
-                           int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace, cudaStream_t st)
+cudaError_t index_topk_any(const void *qI, const void *kI, const float *w, int64_t S, int64_t pos0, int64_t T,
+                           int32_t HI, int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace, cudaStream_t st)
 {
     const uint16_t *q16 = static_cast<const uint16_t *>(qI), *k16 = static_cast<const uint16_t *>(kI);
     if (T > 0 && index_topk_tc_supported(T, HI, dI, k))
-        return launch_index_topk_tc(q16, k16, w, S, T, HI, dI, m, k, idx, static_cast<int32_t *>(workspace), st);
+        return launch_index_topk_tc(q16, k16, w, S, pos0, T, HI, dI, m, k, idx, static_cast<int32_t *>(workspace), st);
     float *scores = reinterpret_cast<float *>(static_cast<char *>(workspace) + kStatusBytes);
-    cudaError_t e = launch_index_scores(q16, w, k16, S, T, HI, dI, m, 0, scores, st);
+    cudaError_t e = launch_index_scores(q16, w, k16, S, pos0, T, HI, dI, m, 0, scores, st);
     if (e != cudaSuccess) return e;
-    return launch_topk_rows(scores, S, T, m, 0, k, idx, st);
+    return launch_topk_rows(scores, S, pos0, T, m, 0, k, idx, st);
 }
 
 }  // namespace
@@ -201,6 +204,9 @@ size_t csa_workspace_size(csa_op op, const csa_dims *d)
     switch (op) {
     case CSA_OP_INDEX_TOPK:
     case CSA_OP_CSA_FORWARD:
+        // the tensor-core indexer keeps its scores on chip; the general path stages S x T scores.
+        // Without the index shape (HI = 0) the general path's size is returned.
+        if (d->HI > 0 && d->T > 0 && index_topk_tc_supported(d->T, d->HI, d->dI, std::max(d->k, 1))) return kStatusBytes;
         return kStatusBytes + scores_bytes(d->S, d->T);
     case CSA_OP_ATTEND:
     case CSA_OP_HCA_FORWARD:
@@ -226,23 +232,23 @@ csa_status csa_get_device_status(const void *workspace, int32_t *status, void *s
     return CSA_OK;
 }
 
-csa_status csa_compress(const void *kv, const void *gate, const float *pos_bias, int64_t S, int32_t D, int32_t m,
-                        int32_t L, int32_t rope_dim, double theta_cmp, double theta_tok, void *C, void *kv_rot,
-                        void *stream)
+csa_status csa_compress(const void *kv, const void *gate, const float *pos_bias, int64_t S, int64_t pos0, int32_t D,
+                        int32_t m, int32_t L, int32_t rope_dim, double theta_cmp, double theta_tok, void *C,
+                        void *kv_rot, void *stream)
 {
-    CSA_TRY(check_compress(kv, gate, pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    CSA_TRY(check_compress(kv, gate, pos_bias, S, pos0, D, m, L, rope_dim, theta_cmp, theta_tok, C));
     CSA_CHECK_ARG(aligned16(kv_rot));
     return from_cuda(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate),
-                                     pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok,
+                                     pos_bias, S, pos0, D, m, L, rope_dim, theta_cmp, theta_tok,
                                      static_cast<uint16_t *>(C), static_cast<uint16_t *>(kv_rot), as_stream(stream)));
 }
 
-csa_status csa_index_topk(const void *qI, const void *kI, const float *w, int64_t S, int64_t T, int32_t HI,
-                          int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace, size_t workspace_bytes,
-                          void *stream)
+csa_status csa_index_topk(const void *qI, const void *kI, const float *w, int64_t S, int64_t pos0, int64_t T,
+                          int32_t HI, int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace,
+                          size_t workspace_bytes, void *stream)
 {
-    CSA_CHECK_ARG(S >= 0 && T >= 0 && HI > 0 && dI > 0 && m >= 1 && k >= 1);
-    CSA_CHECK_ARG(T <= S / m);
+    CSA_CHECK_ARG(S >= 0 && pos0 >= 0 && pos0 <= ((int64_t)1 << 40) && T >= 0 && HI > 0 && dI > 0 && m >= 1 && k >= 1);
+    CSA_CHECK_ARG(T <= (pos0 + S) / m);
     CSA_CHECK_ARG(S == 0 || (qI != nullptr && w != nullptr && idx != nullptr));
     CSA_CHECK_ARG(T == 0 || kI != nullptr);
     CSA_CHECK_SUP(dI == 32 || dI == 64 || dI == 128 || dI == 256);
@@ -252,53 +258,56 @@ csa_status csa_index_topk(const void *qI, const void *kI, const float *w, int64_
     memset(&dims, 0, sizeof dims);
     dims.S = S;
     dims.T = T;
+    dims.HI = HI;
+    dims.dI = dI;
+    dims.k = k;
     CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_INDEX_TOPK, &dims)));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
-    CSA_CUDA(index_topk_any(qI, kI, w, S, T, HI, dI, m, k, idx, workspace, st));
+    CSA_CUDA(index_topk_any(qI, kI, w, S, pos0, T, HI, dI, m, k, idx, workspace, st));
     return CSA_OK;
 }
 
 csa_status csa_attend(const void *q, const void *C, const void *kv_rot, const int32_t *idx, const float *sinks,
-                      int64_t S, int32_t H, int32_t D, int64_t T, int32_t k, int32_t W, int32_t rope_dim, int32_t m,
-                      double theta_tok, double theta_cmp, float softmax_scale, float *o, void *workspace,
+                      int64_t S, int64_t pos0, int32_t H, int32_t D, int64_t T, int32_t k, int32_t W, int32_t rope_dim,
+                      int32_t m, double theta_tok, double theta_cmp, float softmax_scale, float *o, void *workspace,
                       size_t workspace_bytes, void *stream)
 {
-    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, pos0, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
     CSA_CHECK_ARG(k >= 1 && (S == 0 || idx != nullptr));
     CSA_CHECK_SUP(k <= 4096);
     CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
-    AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
+    AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, pos0, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
     return from_cuda(attend_any(a, st));
 }
 
-csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const float *sinks, int64_t S, int32_t H,
-                      int32_t D, int64_t T, int32_t W, int32_t rope_dim, int32_t m, double theta_tok,
+csa_status hca_attend(const void *q, const void *C, const void *kv_rot, const float *sinks, int64_t S, int64_t pos0,
+                      int32_t H, int32_t D, int64_t T, int32_t W, int32_t rope_dim, int32_t m, double theta_tok,
                       double theta_cmp, float softmax_scale, float *o, void *workspace, size_t workspace_bytes,
                       void *stream)
 {
-    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, pos0, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
     CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
-    AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
+    AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, pos0, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
     return from_cuda(attend_any(a, st));
 }
 
 csa_status csa_forward(const void *q, const void *kv, const void *gate, const float *pos_bias, const void *qI,
-                       const void *kI, const float *w, const float *sinks, int64_t S, int32_t H, int32_t D,
-                       int32_t HI, int32_t dI, int32_t m, int32_t L, int32_t k, int32_t W, int32_t rope_dim,
+                       const void *kI, const float *w, const float *sinks, int64_t S, int64_t pos0, int32_t H,
+                       int32_t D, int32_t HI, int32_t dI, int32_t m, int32_t L, int32_t k, int32_t W, int32_t rope_dim,
                        double theta_tok, double theta_cmp, float softmax_scale, void *C, void *kv_rot, int32_t *idx,
                        float *o, void *workspace, size_t workspace_bytes, void *stream)
 {
-    const int64_t T = m >= 1 ? S / m : 0;
-    CSA_TRY(check_compress(kv, gate, pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    CSA_TRY(check_compress(kv, gate, pos_bias, S, pos0, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    const int64_t T = (pos0 + S) / m;
     CSA_CHECK_ARG(kv_rot != nullptr || S == 0);
-    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, pos0, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
     CSA_CHECK_ARG(k >= 1 && (S == 0 || idx != nullptr));
     CSA_CHECK_SUP(k <= 4096);
     CSA_CHECK_ARG(HI > 0 && dI > 0 && (S == 0 || (qI != nullptr && w != nullptr)) && (T == 0 || kI != nullptr));
@@ -309,35 +318,38 @@ csa_status csa_forward(const void *q, const void *kv, const void *gate, const fl
     memset(&dims, 0, sizeof dims);
     dims.S = S;
     dims.T = T;
+    dims.HI = HI;
+    dims.dI = dI;
+    dims.k = k;
     CSA_TRY(check_workspace(workspace, workspace_bytes, csa_workspace_size(CSA_OP_CSA_FORWARD, &dims)));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
-    CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, D,
-                             m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
+    CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, pos0,
+                             D, m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
                              static_cast<uint16_t *>(kv_rot), st));
-    CSA_CUDA(index_topk_any(qI, kI, w, S, T, HI, dI, m, k, idx, workspace, st));
-    AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
+    CSA_CUDA(index_topk_any(qI, kI, w, S, pos0, T, HI, dI, m, k, idx, workspace, st));
+    AttnArgs a = prefill_args(q, C, kv_rot, idx, sinks, S, pos0, H, D, T, k, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
     return from_cuda(attend_any(a, st));
 }
 
 csa_status hca_forward(const void *q, const void *kv, const void *gate, const float *pos_bias, const float *sinks,
-                       int64_t S, int32_t H, int32_t D, int32_t m, int32_t L, int32_t W, int32_t rope_dim,
-                       double theta_tok, double theta_cmp, float softmax_scale, void *C, void *kv_rot, float *o,
-                       void *workspace, size_t workspace_bytes, void *stream)
+                       int64_t S, int64_t pos0, int32_t H, int32_t D, int32_t m, int32_t L, int32_t W,
+                       int32_t rope_dim, double theta_tok, double theta_cmp, float softmax_scale, void *C, void *kv_rot,
+                       float *o, void *workspace, size_t workspace_bytes, void *stream)
 {
-    const int64_t T = m >= 1 ? S / m : 0;
-    CSA_TRY(check_compress(kv, gate, pos_bias, S, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    CSA_TRY(check_compress(kv, gate, pos_bias, S, pos0, D, m, L, rope_dim, theta_cmp, theta_tok, C));
+    const int64_t T = (pos0 + S) / m;
     CSA_CHECK_ARG(kv_rot != nullptr || S == 0);
-    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
+    CSA_TRY(check_attend_common(q, C, kv_rot, sinks, S, pos0, H, D, T, W, rope_dim, m, theta_tok, theta_cmp, o));
     CSA_CHECK_ARG(aligned16(kv_rot));
     CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
     cudaStream_t st = as_stream(stream);
     CSA_TRY(reset_status(workspace, st));
-    CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, D,
-                             m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
+    CSA_CUDA(launch_compress(static_cast<const uint16_t *>(kv), static_cast<const uint16_t *>(gate), pos_bias, S, pos0,
+                             D, m, L, rope_dim, theta_cmp, theta_tok, static_cast<uint16_t *>(C),
                              static_cast<uint16_t *>(kv_rot), st));
-    AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
+    AttnArgs a = prefill_args(q, C, kv_rot, nullptr, sinks, S, pos0, H, D, T, 0, W, rope_dim, m, theta_tok, theta_cmp,
                               softmax_scale, o, workspace);
     return from_cuda(attend_any(a, st));
 }
@@ -426,9 +438,9 @@ csa_status csa_decode(const void *q, const void *qI, const float *w, const void 
                                         HI, dI, k, idx, scores, static_cast<int32_t *>(workspace), st));
     } else {
         CSA_TRY(reset_status(workspace, st));
-        CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, T,
+        CSA_CUDA(launch_index_scores(static_cast<const uint16_t *>(qI), w, static_cast<const uint16_t *>(kI), B, 0, T,
                                      HI, dI, 1, 1, scores, st));
-        CSA_CUDA(launch_topk_rows(scores, B, T, 1, 1, k, idx, st));
+        CSA_CUDA(launch_topk_rows(scores, B, 0, T, 1, 1, k, idx, st));
     }
     return decode_attention(q, C, c8, c8_scale, c_rope, win, sinks, B, H, D, T, k, W, rope_dim, P, theta_tok, theta_cmp,
                             softmax_scale, idx, o, workspace, workspace_bytes, st);
@@ -478,7 +490,7 @@ csa_status csa_decode_fp4(const void *q, const uint8_t *qI_codes, const uint8_t 
                                          static_cast<int32_t *>(workspace), st));
     } else {   // no entries: every index slot is -1
         CSA_TRY(reset_status(workspace, st));
-        CSA_CUDA(launch_topk_rows(scores, B, 0, 1, 1, k, idx, st));
+        CSA_CUDA(launch_topk_rows(scores, B, 0, 0, 1, 1, k, idx, st));
     }
     return decode_attention(q, C, c8, c8_scale, c_rope, win, sinks, B, H, D, T, k, W, rope_dim, P, theta_tok, theta_cmp,
                             softmax_scale, idx, o, workspace, workspace_bytes, st);
@@ -536,13 +548,13 @@ csa_status hca_decode(const void *q, const void *C, const uint8_t *c8, const flo
     return from_cuda(launch_attend_simt(a, st));
 }
 
-csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int64_t S, int32_t H, int32_t D, int32_t W,
-                      int32_t rope_dim, double theta_tok, float softmax_scale, float *o, void *workspace,
-                      size_t workspace_bytes, void *stream)
+csa_status swa_attend(const void *q, const void *kv_rot, const float *sinks, int64_t S, int64_t pos0, int32_t H,
+                      int32_t D, int32_t W, int32_t rope_dim, double theta_tok, float softmax_scale, float *o,
+                      void *workspace, size_t workspace_bytes, void *stream)
 {
     // the HCA attention with no compressed entries (both rope branches at theta_tok)
-    return hca_attend(q, nullptr, kv_rot, sinks, S, H, D, 0, W, rope_dim, 1, theta_tok, theta_tok, softmax_scale, o,
-                      workspace, workspace_bytes, stream);
+    return hca_attend(q, nullptr, kv_rot, sinks, S, pos0, H, D, 0, W, rope_dim, 1, theta_tok, theta_tok, softmax_scale,
+                      o, workspace, workspace_bytes, stream);
 }
 
 csa_status csa_compress_append(const void *x_new, const void *g_new, const float *pos_bias, void *state_x,

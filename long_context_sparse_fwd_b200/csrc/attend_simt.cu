@@ -43,7 +43,7 @@ attend_simt_kernel(AttnArgs a)
     const int h0 = blockIdx.y * HG;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = h0 + warp;
-    const int64_t t = a.decode ? a.P : row;
+    const int64_t t = a.decode ? a.P : a.pos0 + row;
     const int r = a.r;
 
     // ---- rotated query copies ----

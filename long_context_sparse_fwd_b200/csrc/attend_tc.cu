@@ -104,6 +104,7 @@ struct TcArgs {
     float *part_ml;           // split partials: [R*nsplit, 64, 2] (log2-domain reference max, sum)
     int32_t *status;
     int64_t S, T, P;          // S: prefill rows; P: decode position
+    int64_t pos0;             // prefill: position of row 0 (window rows indexed by position)
     int k, W, m, decode, nsplit;
     float scale_log2;         // softmax scale * log2(e)
     double log2_theta_tok, log2_theta_cmp;
@@ -259,7 +260,7 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int split = a.decode ? (int)(u % a.nsplit) : 0;
             if (lane == 0 && (!a.decode || split == 0))   // bring this query's Q into L2 ahead of its use
                 for (int dc = 0; dc < NCH; ++dc) tma_prefetch_2d(&tm_q, dc * 64, (int)(row * HH));
-            const int64_t t = a.decode ? a.P : row;                   // position of the query
+            const int64_t t = a.decode ? a.P : a.pos0 + row;          // position of the query
             const int64_t vis = a.decode ? a.T : visible_entries(t, a.m, a.T);
             const int64_t wpos0 = max((int64_t)0, t - a.W + 1);
             const int nw = (int)(t - wpos0 + 1);
@@ -774,7 +775,9 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             int nS = 0, nPV = 0;
             bool ofree = n == 0;      // O of the previous query has been read out
             bool ok = true;
-            uint64_t t_progress = __shfl_sync(0xffffffffu, globaltimer(), 0);
+            // The timeout clock is read only while the loop is idle (every 256 polls without
+            // progress): a read of the global timer is slow and would delay the next issue.
+            uint64_t t_idle = 0;
             uint32_t polls = 0;
             while (nPV < nb) {
                 bool progressed = false;
@@ -828,10 +831,12 @@ attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     progressed = true;
                 }
                 if (progressed) {
-                    t_progress = __shfl_sync(0xffffffffu, globaltimer(), 0);
+                    polls = 0;
                 } else if ((++polls & 255u) == 0) {
                     if (__any_sync(0xffffffffu, *abort != 0)) { ok = false; break; }
-                    if (__shfl_sync(0xffffffffu, globaltimer(), 0) - t_progress > 2000000000ull) {
+                    const uint64_t now = __shfl_sync(0xffffffffu, globaltimer(), 0);
+                    if (polls == 256u) t_idle = now;   // first idle check since the last progress
+                    if (now - t_idle > 2000000000ull) {
                         if (lane == 0) {
                             *abort = 1;
                             report(a.status, CSA_ERR_TIMEOUT);
@@ -923,6 +928,7 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     a.S = x.R;
     a.T = x.T;
     a.P = x.P;
+    a.pos0 = x.decode ? 0 : x.pos0;
     a.k = x.idx != nullptr ? x.k : 0;
     a.W = x.W;
     a.m = x.m;
@@ -936,7 +942,7 @@ static cudaError_t launch_tc(const AttnArgs &x, int nsplit, float *out_rows, flo
     if (!make_tmap_bf16_sw128(&tq, x.q, (uint64_t)x.R * HH, DD, 64)) return cudaErrorInvalidValue;
     // entry rows (gather4: one-row boxes) and window rows (16-row tiles); row coordinates are int32
     const uint64_t c_rows = x.decode ? (uint64_t)x.R * x.T : (uint64_t)x.T;
-    const uint64_t w_rows = x.decode ? (uint64_t)x.R * x.W : (uint64_t)x.R;
+    const uint64_t w_rows = x.decode ? (uint64_t)x.R * x.W : (uint64_t)(x.pos0 + x.R);
     if (c_rows >= (1ull << 31) || w_rows >= (1ull << 31)) return cudaErrorInvalidValue;
     if (x.C != nullptr && c_rows > 0) {
         // selected entries (CSA) are gathered four one-row boxes at a time; every visible entry (HCA)

@@ -1,61 +1,69 @@
-// compress.cu -- softmax-gated KV compressor (CSA m=4 / window 2m; HCA m'=128 / window m') and
-// the RoPE'd raw-row copy for the sliding-window branch.
+// compress.cu -- softmax-gated KV compressor (CSA m=4 / window 2m; HCA m'=128 / window m') fused with
+// the RoPE'd raw-row copy for the sliding-window branch, for a prefill chunk at positions
+// pos0 .. pos0+S-1 (pos0 = 0 for a whole prefill).
 //
 // Hugging Face Transformers docs "DeepSeek-V4", section "Hybrid attention": CSA pools every m
 // tokens into one entry over overlapping windows, HCA over non-overlapping windows of m'; the
 // insight.ai.kr digest of the HF blog: the pooling is a softmax gate with a learned position
-// bias. Entry w pools [(w+1)m - L, (w+1)m) clipped to [0,S); per channel the weights are a
-// softmax over positions of gate + bias[offset]; the entry is rotated at position w*m with
-// compress_rope_theta (llm-atlas "DeepSeek-V4-Flash", config.json table).
+// bias; section "Cache layers": state carries over between forward calls. Entry w pools
+// [(w+1)m - L, (w+1)m) clipped at position 0; per channel the weights are a softmax over positions of
+// gate + bias[offset]; the entry is rotated at position w*m with compress_rope_theta (llm-atlas
+// "DeepSeek-V4-Flash", config.json table). A chunk writes the entries whose window closes inside it,
+// w in [floor(pos0/m), floor((pos0+S)/m)), and the window rows of its own positions.
 //
-// HBM-bound streaming: each thread owns 8 channels (one 16-byte vector) of one entry and walks
-// the window with an online softmax in fp32; overlapping CSA windows re-read the previous block
-// from L2. The raw-row kernel reads each kv row once and writes it rotated at its own position.
+// HBM-bound streaming, one launch with two roles: the first CTAs write the chunk's rows rotated at
+// their own position with theta_tok (one thread per row and 8-channel group, 16-byte vectors); the
+// rest pool the entries (one thread per entry and 8-channel group walking the window with an online
+// softmax in fp32, whose rows the row role has just brought into L2). Long windows (HCA, L >= 64)
+// split each entry's window across 8 lanes whose online-softmax states are merged by shuffles.
 #include "kernels.cuh"
 
 namespace csa {
 
-__global__ void __launch_bounds__(256)
-compress_entries_kernel(const uint16_t *__restrict__ kv, const uint16_t *__restrict__ gate,
-                        const float *__restrict__ bias, int64_t T, int D, int m, int L, int r,
-                        double log2_theta_cmp, uint16_t *__restrict__ C)
+namespace {
+
+// Row j of kv rotated at position j with theta_tok on the rope channels this 8-channel group holds.
+__device__ __forceinline__ uint4 rotate_row8(uint4 v, int64_t j, int d0, int D, int r, double log2_theta_tok)
 {
-    const int chunks = D >> 3;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= T * chunks) return;
-    const int64_t w = gid / chunks;
-    const int d0 = (int)(gid - w * chunks) << 3;
-    const int64_t start = (w + 1) * (int64_t)m - L;
-    const int64_t end = (w + 1) * (int64_t)m;
-    const int64_t lo = start < 0 ? 0 : start;
-
-    float mx[8], l[8], acc[8];
+    if (d0 < D - r) return v;
+    uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; l[e] = 0.f; acc[e] = 0.f; }
+    for (int e = 0; e < 4; ++e) {
+        const int p = (d0 + 2 * e - (D - r)) >> 1;
+        float c, s;
+        rope_cos_sin((double)j, p, r, log2_theta_tok, &c, &s);
+        const float x0 = bf_lo(vw[e]), x1 = bf_hi(vw[e]);
+        vw[e] = pack_bf2(x0 * c - x1 * s, x0 * s + x1 * c);
+    }
+    return make_uint4(vw[0], vw[1], vw[2], vw[3]);
+}
 
-#pragma unroll 4
-    for (int64_t j = lo; j < end; ++j) {
-        const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gate + j * D + d0));
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(kv + j * D + d0));
-        const float b = __ldg(bias + (j - start));
-        const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
-        const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+// One online-softmax step over the 8 channels of a row: gate logits g (+ bias b), values v.
+__device__ __forceinline__ void pool_step(uint4 g, uint4 v, float b, float (&mx)[8], float (&l)[8], float (&acc)[8])
+{
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const float a = ((e & 1) ? bf_hi(gw[e >> 1]) : bf_lo(gw[e >> 1])) + b;
-            const float x = (e & 1) ? bf_hi(vw[e >> 1]) : bf_lo(vw[e >> 1]);
-            if (a > mx[e]) {
-                const float corr = expf(mx[e] - a);
-                l[e] = l[e] * corr + 1.f;
-                acc[e] = acc[e] * corr + x;
-                mx[e] = a;
-            } else {
-                const float p = expf(a - mx[e]);
-                l[e] += p;
-                acc[e] += p * x;
-            }
+    for (int e = 0; e < 8; ++e) {
+        const float a = ((e & 1) ? bf_hi(gw[e >> 1]) : bf_lo(gw[e >> 1])) + b;
+        const float x = (e & 1) ? bf_hi(vw[e >> 1]) : bf_lo(vw[e >> 1]);
+        if (a > mx[e]) {
+            const float corr = expf(mx[e] - a);
+            l[e] = l[e] * corr + 1.f;
+            acc[e] = acc[e] * corr + x;
+            mx[e] = a;
+        } else {
+            const float pe = expf(a - mx[e]);
+            l[e] += pe;
+            acc[e] += pe * x;
         }
     }
+}
+
+// Normalise, rotate at the entry position w*m with theta_cmp and store entry w's 8 channels.
+__device__ __forceinline__ void store_entry8(const float (&l)[8], const float (&acc)[8], int64_t w, int m, int d0, int D,
+                                             int r, double log2_theta_cmp, uint16_t *C)
+{
     float out[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) out[e] = acc[e] / l[e];
@@ -63,12 +71,12 @@ compress_entries_kernel(const uint16_t *__restrict__ kv, const uint16_t *__restr
         const double pos = (double)(w * (int64_t)m);
 #pragma unroll
         for (int e = 0; e < 8; e += 2) {
-            const int p = (d0 + e - (D - r)) >> 1;
-            float c, s;
-            rope_cos_sin(pos, p, r, log2_theta_cmp, &c, &s);
+            const int pp = (d0 + e - (D - r)) >> 1;
+            float c, sn;
+            rope_cos_sin(pos, pp, r, log2_theta_cmp, &c, &sn);
             const float x0 = out[e], x1 = out[e + 1];
-            out[e] = x0 * c - x1 * s;
-            out[e + 1] = x0 * s + x1 * c;
+            out[e] = x0 * c - x1 * sn;
+            out[e + 1] = x0 * sn + x1 * c;
         }
     }
     uint4 o;
@@ -79,27 +87,78 @@ compress_entries_kernel(const uint16_t *__restrict__ kv, const uint16_t *__restr
     *reinterpret_cast<uint4 *>(C + w * D + d0) = o;
 }
 
-// Long windows (HCA: L = 128): the window of one (entry, 8-channel group) is split across G = 8
-// neighbouring lanes, each walking L/G consecutive positions with its own online softmax; the G
-// partial (max, sum, weighted sum) states are then merged by shuffles. Lane j of a group of 8 lanes
+struct CompressArgs {
+    const uint16_t *kv, *gate;   // [pos0 + S, D] by absolute position
+    const float *bias;           // [L]
+    uint16_t *C;                 // [T1, D] (entries [T0, T1) written)
+    uint16_t *kv_rot;            // [pos0 + S, D] (rows [pos0, pos0 + S) written) or null
+    int64_t pos0, end;           // chunk positions [pos0, end)
+    int64_t T0, T1;              // entries [T0, T1) close inside the chunk
+    int64_t rot_blocks;          // CTAs of the row role (the rest of the grid pools entries)
+    int D, m, L, r;
+    double log2_theta_cmp, log2_theta_tok;
+};
+
+// Row role: one thread per (row, 8-channel group) of the chunk writes the row rotated at its position.
+__device__ __forceinline__ void rotate_role(const CompressArgs &a, int64_t gid)
+{
+    const int chunks = a.D >> 3;
+    const int64_t j = a.pos0 + gid / chunks;
+    if (j >= a.end) return;
+    const int d0 = (int)(gid % chunks) << 3;
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.kv + j * a.D + d0));
+    *reinterpret_cast<uint4 *>(a.kv_rot + j * a.D + d0) = rotate_row8(v, j, d0, a.D, a.r, a.log2_theta_tok);
+}
+
+// Short windows (CSA, L = 2m): the row role, then one thread per (entry, 8-channel group) walking the
+// entry's window with an online softmax.
+__global__ void __launch_bounds__(256)
+compress_fused_kernel(CompressArgs a)
+{
+    if (blockIdx.x < a.rot_blocks) {
+        rotate_role(a, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+        return;
+    }
+    const int chunks = a.D >> 3;
+    const int64_t gid = (int64_t)(blockIdx.x - a.rot_blocks) * blockDim.x + threadIdx.x;
+    const int64_t w = a.T0 + gid / chunks;
+    if (w >= a.T1) return;
+    const int d0 = (int)(gid % chunks) << 3;
+    const int64_t start = (w + 1) * (int64_t)a.m - a.L, end = (w + 1) * (int64_t)a.m;
+    float mx[8], l[8], acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { mx[e] = -INFINITY; l[e] = 0.f; acc[e] = 0.f; }
+#pragma unroll 4
+    for (int64_t j = start < 0 ? 0 : start; j < end; ++j) {
+        const uint4 g = __ldg(reinterpret_cast<const uint4 *>(a.gate + j * a.D + d0));
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.kv + j * a.D + d0));
+        pool_step(g, v, __ldg(a.bias + (j - start)), mx, l, acc);
+    }
+    store_entry8(l, acc, w, a.m, d0, a.D, a.r, a.log2_theta_cmp, a.C);
+}
+
+// Long windows (HCA: L = 128): the row role, then the window of one (entry, 8-channel group) split
+// across G = 8 neighbouring lanes, each walking L/G consecutive positions with its own online softmax;
+// the G partial (max, sum, weighted sum) states are merged by shuffles. Lane j of a group of 8 lanes
 // takes positions j*L/8 ..; the 4 groups of a warp take 4 consecutive channel groups (64 contiguous
 // bytes of each row).
 __global__ void __launch_bounds__(256)
-compress_entries_split_kernel(const uint16_t *__restrict__ kv, const uint16_t *__restrict__ gate,
-                              const float *__restrict__ bias, int64_t T, int D, int m, int L, int r,
-                              double log2_theta_cmp, uint16_t *__restrict__ C)
+compress_fused_split_kernel(CompressArgs a)
 {
+    if (blockIdx.x < a.rot_blocks) {
+        rotate_role(a, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+        return;
+    }
     constexpr int G = 8;
-    const int chunks = D >> 3;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int chunks = a.D >> 3;
+    const int64_t gid = (int64_t)(blockIdx.x - a.rot_blocks) * blockDim.x + threadIdx.x;
     const int sub = threadIdx.x & (G - 1);
     const int64_t item = gid / G;   // (entry, channel group)
-    const bool valid = item < T * chunks;
-    const int64_t w = valid ? item / chunks : 0;
-    const int d0 = valid ? (int)(item - w * chunks) << 3 : 0;
-    const int64_t start = (w + 1) * (int64_t)m - L;
-    const int64_t end = (w + 1) * (int64_t)m;
-    const int per = (L + G - 1) / G;
+    const bool valid = item < (a.T1 - a.T0) * chunks;
+    const int64_t w = a.T0 + (valid ? item / chunks : 0);
+    const int d0 = valid ? (int)(item % chunks) << 3 : 0;
+    const int64_t start = (w + 1) * (int64_t)a.m - a.L, end = (w + 1) * (int64_t)a.m;
+    const int per = (a.L + G - 1) / G;
     int64_t j0 = start + (int64_t)sub * per, j1 = j0 + per;
     if (j0 < 0) j0 = 0;
     if (j1 > end) j1 = end;
@@ -110,26 +169,9 @@ compress_entries_split_kernel(const uint16_t *__restrict__ kv, const uint16_t *_
     if (valid) {
 #pragma unroll 4
         for (int64_t j = j0; j < j1; ++j) {
-            const uint4 g = __ldg(reinterpret_cast<const uint4 *>(gate + j * D + d0));
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(kv + j * D + d0));
-            const float b = __ldg(bias + (j - start));
-            const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
-            const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float a = ((e & 1) ? bf_hi(gw[e >> 1]) : bf_lo(gw[e >> 1])) + b;
-                const float x = (e & 1) ? bf_hi(vw[e >> 1]) : bf_lo(vw[e >> 1]);
-                if (a > mx[e]) {
-                    const float corr = expf(mx[e] - a);
-                    l[e] = l[e] * corr + 1.f;
-                    acc[e] = acc[e] * corr + x;
-                    mx[e] = a;
-                } else {
-                    const float pe = expf(a - mx[e]);
-                    l[e] += pe;
-                    acc[e] += pe * x;
-                }
-            }
+            const uint4 g = __ldg(reinterpret_cast<const uint4 *>(a.gate + j * a.D + d0));
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(a.kv + j * a.D + d0));
+            pool_step(g, v, __ldg(a.bias + (j - start)), mx, l, acc);
         }
     }
     // merge the G partial states of this (entry, channel group): lanes differing in the low 3 bits
@@ -149,79 +191,42 @@ compress_entries_split_kernel(const uint16_t *__restrict__ kv, const uint16_t *_
         }
     }
     if (!valid || sub != 0) return;
-    float out[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = acc[e] / l[e];
-    if (d0 >= D - r) {
-        const double pos = (double)(w * (int64_t)m);
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-            const int pp = (d0 + e - (D - r)) >> 1;
-            float c, sn;
-            rope_cos_sin(pos, pp, r, log2_theta_cmp, &c, &sn);
-            const float x0 = out[e], x1 = out[e + 1];
-            out[e] = x0 * c - x1 * sn;
-            out[e + 1] = x0 * sn + x1 * c;
-        }
-    }
-    uint4 o4;
-    o4.x = pack_bf2(out[0], out[1]);
-    o4.y = pack_bf2(out[2], out[3]);
-    o4.z = pack_bf2(out[4], out[5]);
-    o4.w = pack_bf2(out[6], out[7]);
-    *reinterpret_cast<uint4 *>(C + w * D + d0) = o4;
+    store_entry8(l, acc, w, a.m, d0, a.D, a.r, a.log2_theta_cmp, a.C);
 }
 
-__global__ void __launch_bounds__(256)
-rotate_rows_kernel(const uint16_t *__restrict__ kv, int64_t S, int D, int r, double log2_theta_tok,
-                   uint16_t *__restrict__ kv_rot)
-{
-    const int chunks = D >> 3;
-    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= S * chunks) return;
-    const int64_t j = gid / chunks;
-    const int d0 = (int)(gid - j * chunks) << 3;
-    uint4 v = __ldg(reinterpret_cast<const uint4 *>(kv + j * D + d0));
-    if (d0 >= D - r) {
-        uint32_t vw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int p = (d0 + 2 * e - (D - r)) >> 1;
-            float c, s;
-            rope_cos_sin((double)j, p, r, log2_theta_tok, &c, &s);
-            const float x0 = bf_lo(vw[e]), x1 = bf_hi(vw[e]);
-            vw[e] = pack_bf2(x0 * c - x1 * s, x0 * s + x1 * c);
-        }
-        v.x = vw[0]; v.y = vw[1]; v.z = vw[2]; v.w = vw[3];
-    }
-    *reinterpret_cast<uint4 *>(kv_rot + j * D + d0) = v;
-}
+}  // namespace
 
-cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const float *bias, int64_t S, int D,
-                            int m, int L, int r, double theta_cmp, double theta_tok, uint16_t *C,
+cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const float *bias, int64_t S, int64_t pos0,
+                            int D, int m, int L, int r, double theta_cmp, double theta_tok, uint16_t *C,
                             uint16_t *kv_rot, cudaStream_t stream)
 {
-    const int64_t T = S / m;
-    const int chunks = D / 8;
-    if (T > 0 && C != nullptr) {
-        const int64_t n = T * chunks;
-        if (L >= 64) {   // long windows: split each window across 8 lanes
-            const int64_t nt = n * 8;
-            compress_entries_split_kernel<<<(unsigned)((nt + 255) / 256), 256, 0, stream>>>(kv, gate, bias, T, D, m, L,
-                                                                                             r, log2(theta_cmp), C);
-        } else {
-            compress_entries_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(kv, gate, bias, T, D, m, L, r,
-                                                                                      log2(theta_cmp), C);
-        }
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    if (S > 0 && kv_rot != nullptr) {
-        const int64_t n = S * chunks;
-        rotate_rows_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(kv, S, D, r, log2(theta_tok), kv_rot);
-        return cudaGetLastError();
-    }
-    return cudaSuccess;
+    if (S <= 0) return cudaSuccess;
+    CompressArgs a;
+    a.kv = kv;
+    a.gate = gate;
+    a.bias = bias;
+    a.C = C;
+    a.kv_rot = kv_rot;
+    a.pos0 = pos0;
+    a.end = pos0 + S;
+    a.T0 = pos0 / m;
+    a.T1 = C != nullptr ? a.end / m : a.T0;   // no entry cache: rows only
+    a.D = D;
+    a.m = m;
+    a.L = L;
+    a.r = r;
+    a.log2_theta_cmp = r > 0 ? log2(theta_cmp) : 0.0;
+    a.log2_theta_tok = r > 0 ? log2(theta_tok) : 0.0;
+    const int64_t chunks = D / 8;
+    a.rot_blocks = kv_rot != nullptr ? (S * chunks + 255) / 256 : 0;
+    const int64_t items = (a.T1 - a.T0) * chunks * (L >= 64 ? 8 : 1);   // long windows: 8 lanes per item
+    const int64_t grid = a.rot_blocks + (items + 255) / 256;
+    if (grid == 0) return cudaSuccess;
+    if (L >= 64)
+        compress_fused_split_kernel<<<(unsigned)grid, 256, 0, stream>>>(a);
+    else
+        compress_fused_kernel<<<(unsigned)grid, 256, 0, stream>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace csa

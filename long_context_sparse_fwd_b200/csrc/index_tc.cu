@@ -43,6 +43,7 @@ struct IdxParams {
     int32_t *idx;        // [S, k]
     int32_t *status;
     int64_t S, T;
+    int64_t pos0;        // position of query row 0
     int64_t ngroups;     // groups of Q consecutive queries
     int HI, dI, m, k, Q, stages, T_cap;
     int nsb;             // scores buffers (2: the top-k of a group overlaps the next group's scoring)
@@ -467,7 +468,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         if (G >= p.ngroups) return false;
         *t0 = (p.ngroups - 1 - G) * p.Q;
         const int64_t t_last = min(*t0 + p.Q - 1, p.S - 1);
-        *ntiles = (int)((visible_entries(t_last, p.m, p.T) + BM - 1) / BM);
+        *ntiles = (int)((visible_entries(p.pos0 + t_last, p.m, p.T) + BM - 1) / BM);
         return true;
     };
 
@@ -665,7 +666,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             for (int q = pair; q < p.Q; q += 4) {
                 const int64_t t = t0 + q;
                 if (t >= p.S) continue;
-                const int n = (int)visible_entries(t, p.m, p.T);
+                const int n = (int)visible_entries(p.pos0 + t, p.m, p.T);
                 if (n > p.k && n <= 2048)
                     topk_pair_reg(scores + (size_t)q * p.T_cap, n, p.k, hist + pair * (PBINS + 80), 2 + pair,
                                   p.idx + t * (int64_t)p.k);
@@ -752,8 +753,9 @@ bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)
            encode_fn() != nullptr;
 }
 
-cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t T, int HI,
-                                 int dI, int m, int k, int32_t *idx, int32_t *status, cudaStream_t stream)
+cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t pos0,
+                                 int64_t T, int HI, int dI, int m, int k, int32_t *idx, int32_t *status,
+                                 cudaStream_t stream)
 {
     if (S == 0) return cudaSuccess;
     IdxParams p;
@@ -761,6 +763,7 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     p.idx = idx;
     p.status = status;
     p.S = S;
+    p.pos0 = pos0;
     p.T = T;
     p.HI = HI;
     p.dI = dI;

@@ -18,13 +18,13 @@ namespace csa {
 template <int DI>
 __global__ void __launch_bounds__(256)
 index_scores_kernel(const uint16_t *__restrict__ qI, const float *__restrict__ w, const uint16_t *__restrict__ kI,
-                    int64_t T, int HI, int m, int decode, float *__restrict__ scores)
+                    int64_t pos0, int64_t T, int HI, int m, int decode, float *__restrict__ scores)
 {
     extern __shared__ float smem[];
     float *qs = smem;              // [HI][DI]
     float *ws = smem + HI * DI;    // [HI]
     const int64_t row = blockIdx.x;
-    const int64_t vis = decode ? T : visible_entries(row, m, T);
+    const int64_t vis = decode ? T : visible_entries(pos0 + row, m, T);
     const int64_t s0 = (int64_t)blockIdx.y * 256;
     if (s0 >= vis) return;
     const uint16_t *qrow = qI + row * (int64_t)HI * DI;
@@ -89,13 +89,14 @@ __device__ __forceinline__ int block_scan_incl(int v, int *warp_sums, int *total
 }
 
 __global__ void __launch_bounds__(TOPK_THREADS)
-topk_rows_kernel(const float *__restrict__ scores, int64_t T, int m, int decode, int k, int32_t *__restrict__ idx)
+topk_rows_kernel(const float *__restrict__ scores, int64_t pos0, int64_t T, int m, int decode, int k,
+                 int32_t *__restrict__ idx)
 {
     __shared__ uint32_t hist[256];
     __shared__ int warp_sums[32];
     __shared__ uint32_t sh_prefix, sh_remaining;
     const int64_t row = blockIdx.x;
-    const int64_t n = decode ? T : visible_entries(row, m, T);
+    const int64_t n = decode ? T : visible_entries(pos0 + row, m, T);
     const float *sc = scores + row * T;
     int32_t *out = idx + row * (int64_t)k;
 
@@ -150,8 +151,8 @@ topk_rows_kernel(const float *__restrict__ scores, int64_t T, int m, int decode,
     }
 }
 
-cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t R, int64_t T,
-                                int HI, int dI, int m, int decode, float *scores, cudaStream_t stream)
+cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t R, int64_t pos0,
+                                int64_t T, int HI, int dI, int m, int decode, float *scores, cudaStream_t stream)
 {
     if (R == 0 || T == 0) return cudaSuccess;
     dim3 grid((unsigned)R, (unsigned)((T + 255) / 256));
@@ -162,7 +163,7 @@ cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16
         if (smem > 48 * 1024)                                                                         \
             cudaFuncSetAttribute(index_scores_kernel<DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                  (int)smem);                                                          \
-        index_scores_kernel<DV><<<grid, 256, smem, stream>>>(qI, w, kI, T, HI, m, decode, scores);    \
+        index_scores_kernel<DV><<<grid, 256, smem, stream>>>(qI, w, kI, pos0, T, HI, m, decode, scores); \
         break;
         CSA_CASE(32)
         CSA_CASE(64)
@@ -175,11 +176,11 @@ cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t T, int m, int decode, int k, int32_t *idx,
-                             cudaStream_t stream)
+cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t pos0, int64_t T, int m, int decode, int k,
+                             int32_t *idx, cudaStream_t stream)
 {
     if (R == 0) return cudaSuccess;
-    topk_rows_kernel<<<(unsigned)R, TOPK_THREADS, 0, stream>>>(scores, T, m, decode, k, idx);
+    topk_rows_kernel<<<(unsigned)R, TOPK_THREADS, 0, stream>>>(scores, pos0, T, m, decode, k, idx);
     return cudaGetLastError();
 }
 

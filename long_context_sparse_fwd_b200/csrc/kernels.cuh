@@ -20,19 +20,23 @@ struct AttnArgs {
     float *o;                  // [R, H, D] fp32
     int32_t *status;           // workspace status word
     int64_t R, T, P;           // rows, entries (per row for decode), decode position
+    int64_t pos0;              // prefill: position of row 0 (kv_rot rows are absolute positions)
     int H, D, k, W, r, m, decode;
     int after_kernel;          // launch as a programmatic dependent of the kernel before it in the stream
     float scale;
     double log2_theta_tok, log2_theta_cmp;
 };
 
-cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const float *bias, int64_t S, int D, int m,
-                            int L, int r, double theta_cmp, double theta_tok, uint16_t *C, uint16_t *kv_rot,
-                            cudaStream_t stream);
-cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t R, int64_t T,
-                                int HI, int dI, int m, int decode, float *scores, cudaStream_t stream);
-cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t T, int m, int decode, int k, int32_t *idx,
-                             cudaStream_t stream);
+// compress.cu: one prefill chunk at positions [pos0, pos0 + S): entries [floor(pos0/m), floor((pos0+S)/m))
+// into C and rows [pos0, pos0 + S) into kv_rot (either may be null); kv, gate, C, kv_rot by absolute index
+cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const float *bias, int64_t S, int64_t pos0,
+                            int D, int m, int L, int r, double theta_cmp, double theta_tok, uint16_t *C,
+                            uint16_t *kv_rot, cudaStream_t stream);
+// index_topk.cu: general-path scores and top-k; prefill row r is the query at position pos0 + r
+cudaError_t launch_index_scores(const uint16_t *qI, const float *w, const uint16_t *kI, int64_t R, int64_t pos0,
+                                int64_t T, int HI, int dI, int m, int decode, float *scores, cudaStream_t stream);
+cudaError_t launch_topk_rows(const float *scores, int64_t R, int64_t pos0, int64_t T, int m, int decode, int k,
+                             int32_t *idx, cudaStream_t stream);
 cudaError_t launch_attend_simt(const AttnArgs &a, cudaStream_t stream);
 
 // attend_tc.cu: tcgen05 prefill attention for H=64, D=512, rope 64 (CSA when idx != null, else HCA)
@@ -92,7 +96,8 @@ cudaError_t launch_quantize_mxfp4(const uint16_t *x, int64_t rows, int cols, uin
 
 // index_tc.cu: tcgen05 indexer with fused top-k (entries on TMEM lanes, scores kept on chip)
 bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
-cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t T, int HI,
-                                 int dI, int m, int k, int32_t *idx, int32_t *status, cudaStream_t stream);
+cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t pos0,
+                                 int64_t T, int HI, int dI, int m, int k, int32_t *idx, int32_t *status,
+                                 cudaStream_t stream);
 
 }  // namespace csa

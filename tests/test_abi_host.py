@@ -43,7 +43,8 @@ def test_status_strings():
 def test_workspace_sizes():
     assert csa.workspace_size("attend") == 256
     assert csa.workspace_size("hca_forward") == 256
-    assert csa.workspace_size("index_topk", S=8192, T=2048) == 256 + 8192 * 2048 * 4
+    assert csa.workspace_size("index_topk", S=8192, T=2048) == 256 + 8192 * 2048 * 4   # no index shape given
+    assert csa.workspace_size("index_topk", S=8192, T=8192, HI=64, dI=128, k=512) == 256 + 8192 * 8192 * 4
     assert csa.workspace_size("decode", B=64, T=32768, k=1024) >= 256 + 64 * 32768 * 4 + 64 * 1024 * 4
 
 
@@ -56,10 +57,11 @@ MIS = ctypes.c_void_p(0x10002)       # misaligned
 
 
 def compress(**kw):
-    a = dict(kv=FAKE, gate=FAKE, b=FAKE, S=64, D=64, m=4, L=8, r=16, tc=160000.0, tt=10000.0, C=FAKE, kvr=FAKE)
+    a = dict(kv=FAKE, gate=FAKE, b=FAKE, S=64, pos0=0, D=64, m=4, L=8, r=16, tc=160000.0, tt=10000.0, C=FAKE,
+             kvr=FAKE)
     a.update(kw)
-    return csa.lib().csa_compress(a["kv"], a["gate"], a["b"], a["S"], a["D"], a["m"], a["L"], a["r"], a["tc"],
-                                  a["tt"], a["C"], a["kvr"], None)
+    return csa.lib().csa_compress(a["kv"], a["gate"], a["b"], a["S"], a["pos0"], a["D"], a["m"], a["L"], a["r"],
+                                  a["tc"], a["tt"], a["C"], a["kvr"], None)
 
 
 @no_gpu
@@ -76,20 +78,27 @@ def test_compress_rejects_bad_arguments():
     assert compress(D=60) == UNSUP
     assert compress(r=12) == UNSUP
     assert compress(L=8192, m=4096) == UNSUP
+    assert compress(pos0=-1) == INVALID
+    assert compress(pos0=1 << 41) == INVALID
+    assert compress(S=3, pos0=5, C=None) == INVALID   # positions 5..7: entry 1 closes at 7 and there is no cache
+    assert compress(S=2, pos0=4, C=None, kv=MIS) == INVALID
 
 
 def attend(**kw):
-    a = dict(q=FAKE, C=FAKE, kvr=FAKE, idx=FAKE, sinks=FAKE, S=64, H=8, D=128, T=16, k=4, W=8, r=32, m=4,
+    a = dict(q=FAKE, C=FAKE, kvr=FAKE, idx=FAKE, sinks=FAKE, S=64, pos0=0, H=8, D=128, T=16, k=4, W=8, r=32, m=4,
              tt=1e4, tc=1.6e5, sc=0.0, o=FAKE, ws=FAKE, wsb=256)
     a.update(kw)
-    return csa.lib().csa_attend(a["q"], a["C"], a["kvr"], a["idx"], a["sinks"], a["S"], a["H"], a["D"], a["T"],
-                                a["k"], a["W"], a["r"], a["m"], a["tt"], a["tc"], a["sc"], a["o"], a["ws"],
+    return csa.lib().csa_attend(a["q"], a["C"], a["kvr"], a["idx"], a["sinks"], a["S"], a["pos0"], a["H"], a["D"],
+                                a["T"], a["k"], a["W"], a["r"], a["m"], a["tt"], a["tc"], a["sc"], a["o"], a["ws"],
                                 a["wsb"], None)
 
 
 @no_gpu
 def test_attend_rejects_bad_arguments():
     assert attend(T=17) == INVALID             # more entries than floor(S/m)
+    assert attend(T=17, pos0=4, D=96) == UNSUP  # 17 entries exist after a chunk at pos0 = 4: only D is wrong
+    assert attend(T=18, pos0=4) == INVALID      # but not 18
+    assert attend(pos0=-3) == INVALID
     assert attend(H=0) == INVALID
     assert attend(W=-1) == INVALID
     assert attend(k=0) == INVALID
@@ -105,9 +114,12 @@ def test_attend_rejects_bad_arguments():
 @no_gpu
 def test_index_topk_rejects_bad_arguments():
     L = csa.lib()
-    f = lambda S=64, T=16, HI=4, dI=64, m=4, k=8, ws=FAKE, wsb=1 << 20, q=FAKE: L.csa_index_topk(
-        q, FAKE, FAKE, S, T, HI, dI, m, k, FAKE, ws, wsb, None)
+    f = lambda S=64, T=16, HI=4, dI=64, m=4, k=8, ws=FAKE, wsb=1 << 20, q=FAKE, pos0=0: L.csa_index_topk(
+        q, FAKE, FAKE, S, pos0, T, HI, dI, m, k, FAKE, ws, wsb, None)
     assert f(T=17) == INVALID
+    assert f(T=20, pos0=16, dI=48) == UNSUP     # 20 entries exist after a chunk at pos0 = 16: only dI is wrong
+    assert f(T=21, pos0=16) == INVALID
+    assert f(pos0=-1) == INVALID
     assert f(k=0) == INVALID
     assert f(q=None) == INVALID
     assert f(dI=48) == UNSUP
@@ -151,8 +163,9 @@ def test_later_calls_reject_bad_arguments():
     assert hd(D=96) == UNSUP
     assert hd(wsb=16) == WS
 
-    assert L.swa_attend(FAKE, FAKE, FAKE, 64, 8, 96, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == UNSUP
-    assert L.swa_attend(FAKE, None, FAKE, 64, 8, 128, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == INVALID
+    assert L.swa_attend(FAKE, FAKE, FAKE, 64, 0, 8, 96, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == UNSUP
+    assert L.swa_attend(FAKE, None, FAKE, 64, 0, 8, 128, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == INVALID
+    assert L.swa_attend(FAKE, FAKE, FAKE, 64, -1, 8, 128, 128, 32, 1e4, 0.0, FAKE, FAKE, 256, None) == INVALID
 
     def ca(C=FAKE, D=512, Lw=8, P=7, Tcap=2):
         return L.csa_compress_append(FAKE, FAKE, FAKE, FAKE, FAKE, 2, D, 4, Lw, 64, P, 1.6e5, 1e4, C, None, None,

@@ -249,6 +249,77 @@ def test_hca_forward_full_size(S):
     check_close(got, ref, O_MAX_ABS, O_MEAN_ABS, what="o")
 
 
+# ---- 5b. prefill in chunks (state carried across calls: pos0) -------------------------------------------
+
+def _chunked_csa(wl, g, bounds):
+    """csa_forward over the chunks [bounds[i], bounds[i+1]) of one sequence, the caches (C, kv_rot)
+    carried from chunk to chunk; returns (o, C, kv_rot, idx) over all positions."""
+    S, D, m = wl.S, wl.D, wl.m
+    C = torch.full((S // m, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    kvr = torch.full((S, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    o = torch.empty(S, wl.H, D, dtype=torch.float32, device=DEV)
+    idx = torch.empty(S, wl.topk, dtype=torch.int32, device=DEV)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        n = b
+        csa.csa_forward(g["q"][a:b], g["kv"][:n], g["gate"][:n], g["pos_bias"], g["qI"][a:b], g["kI"][:n // m],
+                        g["w"][a:b], g["sinks"], m, wl.L, wl.topk, wl.W, wl.r, wl.theta_tok, wl.theta_cmp,
+                        out=(o[a:b], C[:n // m], kvr[:n], idx[a:b]), pos0=a)
+    torch.cuda.synchronize()
+    return o, C, kvr, idx
+
+
+@pytest.mark.parametrize("wid,bounds,nrows", [(1, (0, 4096, 8192), 24), (0, (0, 333, 601, 1030), None)])
+def test_csa_forward_chunked_equals_one_shot(wid, bounds, nrows):
+    """A prefill split into chunks (V4-Flash shapes 4096 + 4096 on the tensor-core kernels; the tiny
+    layer in chunks starting inside stride blocks on the general kernels) gives bit for bit the
+    one-shot results: entries, window rows, top-k sets and outputs; the last chunk's rows also match
+    the oracle's one-shot prefill."""
+    wl = WORKLOADS[wid].with_(S=bounds[-1])
+    g, x = gen(prefill_inputs, wl)
+    o1, C1, kvr1, idx1 = csa.csa_forward(g["q"], g["kv"], g["gate"], g["pos_bias"], g["qI"], g["kI"], g["w"],
+                                         g["sinks"], wl.m, wl.L, wl.topk, wl.W, wl.r, wl.theta_tok, wl.theta_cmp)
+    o, C, kvr, idx = _chunked_csa(wl, g, bounds)
+    assert torch.equal(C, C1) and torch.equal(kvr, kvr1)
+    assert torch.equal(idx, idx1)
+    assert torch.equal(o, o1)
+    a = bounds[-2]
+    rows = np.arange(a, wl.S) if nrows is None else sample_rows(wl.S - a, nrows, 19, must=[0, wl.S - a - 1]) + a
+    ridx, sc = oracle.index_topk(x["qI"], x["kI"], x["w"], wl.m, wl.topk, rows=rows)
+    vis = [oracle.visible(t, wl.m, wl.T) for t in rows]
+    exc = check_topk_sets(idx.cpu().numpy()[rows], ridx, sc, vis, wl.topk)
+    keep = np.array([t for i, t in enumerate(rows) if i not in {e[0] for e in exc}])
+    Cr, kvrr = oracle.compress(x["kv"], x["gate"], x["pos_bias"], wl.m, wl.L, wl.r, wl.theta_cmp, wl.theta_tok)
+    idx_full = np.full((wl.S, wl.topk), -1, np.int32)
+    idx_full[rows] = ridx
+    ref = oracle.attend(x["q"], Cr, kvrr, idx_full, x["sinks"], wl.m, wl.W, wl.r, wl.theta_tok, wl.theta_cmp,
+                        rows=keep)
+    check_close(o.cpu()[keep], ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
+def test_hca_forward_chunked_equals_one_shot():
+    """HCA prefill in two chunks, the second starting inside a 128-token window (entry 7 pools positions
+    896..1023, 104 of them from the first chunk): bit for bit the one-shot results."""
+    wl = WORKLOADS[2].with_(S=4096 + 77)
+    g, _ = gen(prefill_inputs, wl)
+    o1, C1, kvr1 = csa.hca_forward(g["q"], g["kv"], g["gate"], g["pos_bias"], g["sinks"], wl.m, wl.L, wl.W, wl.r,
+                                   wl.theta_tok, wl.theta_cmp)
+    S, D, m = wl.S, wl.D, wl.m
+    C = torch.full((S // m, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    kvr = torch.full((S, D), float("nan"), dtype=torch.bfloat16, device=DEV)
+    o = torch.empty(S, wl.H, D, dtype=torch.float32, device=DEV)
+    for a, b in ((0, 1000), (1000, S)):
+        csa.hca_forward(g["q"][a:b], g["kv"][:b], g["gate"][:b], g["pos_bias"], g["sinks"], m, wl.L, wl.W, wl.r,
+                        wl.theta_tok, wl.theta_cmp, out=(o[a:b], C[:b // m], kvr[:b]), pos0=a)
+    torch.cuda.synchronize()
+    assert torch.equal(C, C1) and torch.equal(kvr, kvr1) and torch.equal(o, o1)
+
+
+def test_index_topk_workspace_is_status_word_on_the_tensor_core_path():
+    """The fused tensor-core indexer keeps its scores on chip: its workspace is the status word only."""
+    assert csa.workspace_size("index_topk", S=8192, T=2048, HI=64, dI=128, k=512) == 256
+    assert csa.workspace_size("csa_forward", S=8192, T=2048, HI=64, dI=128, k=512) == 256
+
+
 def test_forward_is_deterministic():
     wl = WORKLOADS[0]
     g = prefill_inputs(wl, device=DEV)
