@@ -11,11 +11,11 @@
 // "DeepSeek-V4-Flash", config.json table). A chunk writes the entries whose window closes inside it,
 // w in [floor(pos0/m), floor((pos0+S)/m)), and the window rows of its own positions.
 //
-// HBM-bound streaming, one launch with two roles: the first CTAs write the chunk's rows rotated at
-// their own position with theta_tok (one thread per row and 8-channel group, 16-byte vectors); the
-// rest pool the entries (one thread per entry and 8-channel group walking the window with an online
-// softmax in fp32, whose rows the row role has just brought into L2). Long windows (HCA, L >= 64)
-// split each entry's window across 8 lanes whose online-softmax states are merged by shuffles.
+// HBM-bound streaming, one launch with two roles: the first CTAs pool the entries (one thread per entry
+// and 8-channel group walking the window with an online softmax in fp32, 16-byte vectors; these are
+// the longer dependency chains, so they start first); the rest write the chunk's rows rotated at
+// their own position with theta_tok (one thread per row and 8-channel group). Long windows (HCA,
+// L >= 64) split each entry's window across 8 lanes whose online-softmax states are merged by shuffles.
 #include "kernels.cuh"
 
 namespace csa {
@@ -94,7 +94,7 @@ struct CompressArgs {
     uint16_t *kv_rot;            // [pos0 + S, D] (rows [pos0, pos0 + S) written) or null
     int64_t pos0, end;           // chunk positions [pos0, end)
     int64_t T0, T1;              // entries [T0, T1) close inside the chunk
-    int64_t rot_blocks;          // CTAs of the row role (the rest of the grid pools entries)
+    int64_t pool_blocks;         // CTAs of the pooling role (the rest of the grid rotates rows)
     int D, m, L, r;
     double log2_theta_cmp, log2_theta_tok;
 };
@@ -115,12 +115,12 @@ __device__ __forceinline__ void rotate_role(const CompressArgs &a, int64_t gid)
 __global__ void __launch_bounds__(256)
 compress_fused_kernel(CompressArgs a)
 {
-    if (blockIdx.x < a.rot_blocks) {
-        rotate_role(a, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    if (blockIdx.x >= a.pool_blocks) {
+        rotate_role(a, (int64_t)(blockIdx.x - a.pool_blocks) * blockDim.x + threadIdx.x);
         return;
     }
     const int chunks = a.D >> 3;
-    const int64_t gid = (int64_t)(blockIdx.x - a.rot_blocks) * blockDim.x + threadIdx.x;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t w = a.T0 + gid / chunks;
     if (w >= a.T1) return;
     const int d0 = (int)(gid % chunks) << 3;
@@ -145,13 +145,13 @@ compress_fused_kernel(CompressArgs a)
 __global__ void __launch_bounds__(256)
 compress_fused_split_kernel(CompressArgs a)
 {
-    if (blockIdx.x < a.rot_blocks) {
-        rotate_role(a, (int64_t)blockIdx.x * blockDim.x + threadIdx.x);
+    if (blockIdx.x >= a.pool_blocks) {
+        rotate_role(a, (int64_t)(blockIdx.x - a.pool_blocks) * blockDim.x + threadIdx.x);
         return;
     }
     constexpr int G = 8;
     const int chunks = a.D >> 3;
-    const int64_t gid = (int64_t)(blockIdx.x - a.rot_blocks) * blockDim.x + threadIdx.x;
+    const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int sub = threadIdx.x & (G - 1);
     const int64_t item = gid / G;   // (entry, channel group)
     const bool valid = item < (a.T1 - a.T0) * chunks;
@@ -218,9 +218,9 @@ cudaError_t launch_compress(const uint16_t *kv, const uint16_t *gate, const floa
     a.log2_theta_cmp = r > 0 ? log2(theta_cmp) : 0.0;
     a.log2_theta_tok = r > 0 ? log2(theta_tok) : 0.0;
     const int64_t chunks = D / 8;
-    a.rot_blocks = kv_rot != nullptr ? (S * chunks + 255) / 256 : 0;
     const int64_t items = (a.T1 - a.T0) * chunks * (L >= 64 ? 8 : 1);   // long windows: 8 lanes per item
-    const int64_t grid = a.rot_blocks + (items + 255) / 256;
+    a.pool_blocks = (items + 255) / 256;                                 // the longer chains start first
+    const int64_t grid = a.pool_blocks + (kv_rot != nullptr ? (S * chunks + 255) / 256 : 0);
     if (grid == 0) return cudaSuccess;
     if (L >= 64)
         compress_fused_split_kernel<<<(unsigned)grid, 256, 0, stream>>>(a);

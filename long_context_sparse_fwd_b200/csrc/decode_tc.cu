@@ -51,9 +51,10 @@ struct ScoreParams {
 // Epilogue of the scan (four warps, 128 threads, one TMEM lane quarter each): each thread owns one entry
 // of the tile, reduces its HI heads (w-weighted ReLU) in registers and writes one fp32 score; it also
 // tracks the sequence's key range for the top-k and clears the chunked top-k's counters.
+// With perm4, accumulator row 32 j + r holds entry 4 r + j of the tile (the block-scaled MXFP4 scan).
 __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tmem, uint64_t *tfull, uint64_t *tempty,
                                               volatile int *abort, float *sw, int64_t g_lo, int ntiles, int warp,
-                                              int lane, int etid)
+                                              int lane, int etid, bool perm4 = false)
 {
     const int quarter = warp & 3;
     const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -129,7 +130,7 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
             tc_fence_before();
             mbar_arrive(&tempty[buf]);
         }
-        const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
+        const int64_t s = (int64_t)it * BM + (perm4 ? 4 * lane + quarter : quarter * 32 + lane);
         if (s < p.T) {
             p.scores[b * p.T + s] = acc + 0.0f;
             const uint32_t key = score_key(acc);
@@ -504,6 +505,184 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
             fence_async_smem();   // generic-proxy writes, read by the MMA through the async proxy
             mbar_arrive(&afull[ab]);
         }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, tcols);
+    }
+}
+
+// ---- the MXFP4 scan on the block-scaled tensor-core MMA ---------------------------------------------
+//
+// The same scan with the MXFP4 operands fed to tcgen05.mma kind::mxf4 directly: packed E2M1 codes in
+// shared memory (64-byte rows, 64-byte swizzle, K = 64 channels per instruction) and one E8M0 scale per
+// 32 channels in TMEM, so nothing is converted and the k^I stream is 68 bytes per entry (64 code bytes,
+// 4 scale bytes). In TMEM the scales of matrix row 32 j + r (r < 32) sit in lane r of every lane
+// quarter, column j, one byte per 32-channel block. The k^I code tile is brought by a three-dimensional
+// tensor map that stores entry 4 r + j of the tile at row 32 j + r; the tile's scales, contiguous in
+// memory (4 bytes per entry), then form the [32 x 16 bytes] matrix that tcgen05.cp replicates into the
+// four quarters as they are. The q^I scales of a sequence (row = head) are gathered by the producer warp
+// into the same arrangement (lane r, column j: head r + 32 j). dI = 128 (two instructions per tile),
+// HI <= 64 (N <= 64), T a multiple of 4.
+
+constexpr int X4_THREADS = 192;        // warp 0 TMA and q^I scales, warp 1 MMA and scale copies, warps 2-5 epilogue
+constexpr int X4_STAGES = 12;
+constexpr uint32_t X4_A_BYTES = BM * 64;          // 128 entries x 64 code bytes
+constexpr uint32_t X4_SF_BYTES = 512;             // [32 x 16 bytes] of scales
+constexpr uint32_t X4_SFA_COL = 256, X4_SFB_COL = 272;   // TMEM columns of the scale slots (4 each)
+
+struct Mxf4Params {
+    ScoreParams sp;
+    const uint8_t *qs;                 // q^I scales [B, HI, 4]
+};
+
+__global__ void __launch_bounds__(X4_THREADS, 1)
+decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_kc,
+                          const __grid_constant__ CUtensorMap tm_ks, Mxf4Params f)
+{
+    const ScoreParams &p = f.sp;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t b_bytes = (uint32_t)p.HI * 64;
+    uint8_t *sA = smem;                                           // [X4_STAGES][X4_A_BYTES]
+    uint8_t *sB = sA + X4_STAGES * X4_A_BYTES;                    // [2][4 KB]
+    uint8_t *sSFA = sB + 2 * 4096;                                // [X4_STAGES][X4_SF_BYTES]
+    uint8_t *sSFB = sSFA + X4_STAGES * X4_SF_BYTES;               // [2][X4_SF_BYTES]
+    float *sw = reinterpret_cast<float *>(sSFB + 2 * X4_SF_BYTES);   // [256]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 256);
+    uint64_t *full = bars, *empty = bars + X4_STAGES;             // [X4_STAGES]
+    uint64_t *tfull = bars + 2 * X4_STAGES, *tempty = tfull + NACC;   // [NACC]
+    uint64_t *qfull = tempty + NACC, *qempty = qfull + 2;         // [2]
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(qempty + 2);
+    volatile int *abort = reinterpret_cast<volatile int *>(qempty + 3);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t g_lo = (int64_t)blockIdx.x * p.G / gridDim.x;
+    const int64_t g_hi = (int64_t)(blockIdx.x + 1) * p.G / gridDim.x;
+    const int ntiles = (int)(g_hi - g_lo);
+    const int64_t b_first = g_lo / p.tps;
+    constexpr uint32_t tcols = 512;   // accumulators NACC x HI (<= 256) and the scale slots
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < X4_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < NACC; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], EPI_THREADS);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&qfull[i], 2);   // the q^I code load (with its bytes) and the gathered scales
+            mbar_init(&qempty[i], 1);
+        }
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_ptr, tcols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_ptr;
+    grid_launch_dependents();   // the top-k may be scheduled as this grid's CTAs finish
+
+    if (warp == 0) {
+        // ---------------- producer: code and scale tiles by TMA; q^I and its scales per sequence ----------
+        if (ntiles > 0) {
+            if (elect_one()) {
+                prefetch_tmap(&tm_qc);
+                prefetch_tmap(&tm_kc);
+                prefetch_tmap(&tm_ks);
+            }
+            __syncwarp();
+            const uint64_t pol_stream = policy_evict_first();   // k^I is read once per step
+            int issued = 0, nseg = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int64_t g = g_lo + i, b = g / p.tps;
+                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+                if (i == 0 || it == 0) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status))) break;
+                    if (elect_one()) {
+                        mbar_arrive_expect_tx(&qfull[j & 1], b_bytes);
+                        tma_load_2d(sB + (j & 1) * 4096, &tm_qc, &qfull[j & 1], 0, (int)(b * p.HI));
+                    }
+                    // scales of q^I: lane r writes row r = the 4-byte scale words of heads r + 32 c
+                    uint32_t wq[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int h = lane + 32 * c;
+                        wq[c] = h < p.HI ? *reinterpret_cast<const uint32_t *>(f.qs + (b * p.HI + h) * 4) : 0u;
+                    }
+                    *reinterpret_cast<uint4 *>(sSFB + (j & 1) * X4_SF_BYTES + lane * 16) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&qfull[j & 1]);
+                    nseg = j + 1;
+                }
+                const int st = i % X4_STAGES;
+                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((i / X4_STAGES) & 1) ^ 1, abort, p.status))) break;
+                const int r0 = (int)((b * p.T + (int64_t)it * BM) / 4);   // T % 4 == 0: tiles start on a group of 4
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(&full[st], X4_A_BYTES + X4_SF_BYTES);
+                    asm volatile(
+                        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+                        "[%0], [%1, {%2, %3, %4}], [%5], %6;"
+                        ::"r"(smem_u32(sA + st * X4_A_BYTES)), "l"(reinterpret_cast<uint64_t>(&tm_kc)), "r"(0), "r"(r0),
+                        "r"(0), "r"(smem_u32(&full[st])), "l"(pol_stream)
+                        : "memory");
+                    tma_load_2d_hint(sSFA + st * X4_SF_BYTES, &tm_ks, &full[st], 0, r0, pol_stream);
+                }
+                __syncwarp();
+                issued = i + 1;
+            }
+            // never leave with copies in flight into this CTA's shared memory
+            for (int j = max(0, nseg - 2); j < nseg; ++j)
+                mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status, 100000000ull);
+            for (int i = max(0, issued - X4_STAGES); i < issued; ++i)
+                mbar_wait(&full[i % X4_STAGES], (i / X4_STAGES) & 1, abort, p.status, 100000000ull);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer: scale copies into TMEM, then two block-scaled MMAs per tile ----------
+        if (ntiles > 0) {
+            const uint32_t id0 = idesc_mxf4(BM, p.HI, 0), id2 = idesc_mxf4(BM, p.HI, 2);
+            const uint64_t dA = sdesc_sw64(smem_u32(sA), 512), dB = sdesc_sw64(smem_u32(sB), 512);
+            int issued = 0;
+            for (int i = 0; i < ntiles; ++i) {
+                const int64_t g = g_lo + i, b = g / p.tps;
+                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+                const uint32_t sfb = tmem + X4_SFB_COL + (uint32_t)(j & 1) * 4;
+                if (i == 0 || it == 0) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status))) break;
+                    tc_fence_after();
+                    if (elect_one()) tmem_cp_32x128b_x4(sfb, sdesc_plain(smem_u32(sSFB + (j & 1) * X4_SF_BYTES), 16, 128));
+                    __syncwarp();
+                }
+                const int st = i % X4_STAGES, buf = i % NACC;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((i / NACC) & 1) ^ 1, abort, p.status))) break;
+                if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / X4_STAGES) & 1, abort, p.status))) break;
+                tc_fence_after();
+                const uint32_t sfa = tmem + X4_SFA_COL + (uint32_t)buf * 4;
+                if (elect_one()) {
+                    tmem_cp_32x128b_x4(sfa, sdesc_plain(smem_u32(sSFA + st * X4_SF_BYTES), 16, 128));
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)   // channels 64 ks .. 64 ks + 63: scale bytes 2 ks, 2 ks + 1
+                        mma_mxf4(tmem + buf * p.HI, dA + ((st * X4_A_BYTES + ks * 32) >> 4),
+                                 dB + (((j & 1) * 4096 + ks * 32) >> 4), ks ? id2 : id0,
+                                 sfa | ((uint32_t)(2 * ks) << 30), sfb | ((uint32_t)(2 * ks) << 30), ks != 0);
+                    mma_commit(&empty[st]);
+                    mma_commit(&tfull[buf]);
+                    if (i + 1 == ntiles || it + 1 == p.tps) mma_commit(&qempty[j & 1]);   // done with this q^I
+                }
+                __syncwarp();
+                issued = i + 1;
+            }
+            if (issued > 0)
+                mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
+        }
+    } else {
+        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64, true);
     }
     tc_fence_before();
     __syncthreads();
@@ -1190,6 +1369,27 @@ cudaError_t launch_decode_index_fp4(const uint8_t *qc, const uint8_t *qs, const 
     const DecodeIndexLayout L = decode_index_layout(B, T);
     CUtensorMap tkc;   // k^I codes as rows of dI/2 bytes, 128-row boxes
     if (!make_tmap_u8_rows(&tkc, kc, (uint64_t)(B * T), (uint64_t)dI / 2, BM)) return cudaErrorInvalidValue;
+    if (dI == 128 && HI <= 64 && T % 4 == 0 && (reinterpret_cast<uintptr_t>(qs) & 3u) == 0 &&
+        (reinterpret_cast<uintptr_t>(ks) & 15u) == 0) {
+        // block-scaled MMA on the MXFP4 operands as they are
+        CUtensorMap tqc, tkc3, tks;
+        if (!make_tmap_u8_sw64(&tqc, qc, (uint64_t)B * HI, (uint32_t)HI)) return cudaErrorInvalidValue;
+        if (!make_tmap_u8_sw64_perm4(&tkc3, kc, (uint64_t)(B * T))) return cudaErrorInvalidValue;
+        if (!make_tmap_u8_rows(&tks, ks, (uint64_t)(B * T) / 4, 16, 32)) return cudaErrorInvalidValue;
+        Mxf4Params x;
+        x.sp = score_params(p8, L, w, B, T, HI, dI, status);
+        x.qs = qs;
+        const size_t smem = 1024 + X4_STAGES * (size_t)X4_A_BYTES + 2 * 4096 + (X4_STAGES + 2) * (size_t)X4_SF_BYTES +
+                            256 * 4 + (2 * X4_STAGES + 2 * NACC + 4 + 2) * 8;
+        cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_mxf4_kernel), smem);
+        if (e != cudaSuccess) return e;
+        int dev = 0, nsm = 148;
+        if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
+        const unsigned g1 = (unsigned)std::min<int64_t>(nsm, x.sp.G);
+        decode_scores_mxf4_kernel<<<g1, X4_THREADS, smem, stream>>>(tqc, tkc3, tks, x);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        return launch_topk_after_scan(p8, L, B, T, k, idx, stream);
+    }
     Fp4Params f;
     f.sp = score_params(p8, L, w, B, T, HI, dI, status);
     f.qc = qc;

@@ -328,6 +328,54 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Shared-memory matrix descriptor, 64-byte swizzle, K-major: 64-byte rows, 8-row groups `sbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
+           (1ull << 46) | (4ull << 61);
+}
+
+// Shared-memory matrix descriptor without swizzle: 8-row core matrices of 16-byte rows, `sbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_plain(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor of the block-scaled MXFP4 MMA (kind::mxf4, 32-element scale blocks): A and B
+// E2M1, K-major, E8M0 scales, D fp32, shape M x N, K = 64 per instruction; sf_id selects the first scale
+// byte of each row's 32-bit scale word (0 for channels 0..63, 2 for 64..127).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, int sf_id)
+{
+    return ((uint32_t)sf_id << 4)           // B scale factor id
+         | (1u << 7)                        // A format: E2M1
+         | (1u << 10)                       // B format: E2M1
+         | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | (1u << 23)                       // scale format: E8M0
+         | ((uint32_t)(M >> 4) << 24)       // M / 16
+         | ((uint32_t)sf_id << 29);         // A scale factor id
+}
+
+// D[tmem] (+)= (A * sfa) (B * sfb)^T on MXFP4 operands in shared memory, scales in TMEM (the scale
+// address carries the scale byte in its top two bits, matching the descriptor's sf_id), one thread.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, bool accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Copy a [32 rows x 16 bytes] shared-memory matrix into TMEM at `taddr` (4 columns), replicated into the
+// 32-lane group of each of the four warp quarters; ordered with the MMAs this thread issues after it.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          bool accumulate)

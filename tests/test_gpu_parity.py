@@ -470,6 +470,41 @@ def test_decode_fp4_chunked_topk_fp8_cache():
     _decode_fp4_check(WORKLOADS[4].with_(ctx=4 * 40000 + 1, B=2), batch=None, seqs=[0, 1])
 
 
+@pytest.mark.parametrize("HI,ctx,spread", [(64, 4 * 2052, 0), (16, 4 * 4100, 0), (32, 4 * 1000 + 2, 0),
+                                             (64, 4 * 8192, 40)])
+def test_decode_fp4_block_scaled_mma(HI, ctx, spread):
+    """The MXFP4 scan on the block-scaled MMA (d_I = 128, HI <= 64, T a multiple of 4): a ragged last
+    tile, N = 16 and 32 query-head columns, and k^I rows whose magnitudes span 2^-spread .. 2^spread so
+    the E8M0 scales cover a wide range; selections equal the oracle's on the dequantised operands."""
+    wl = WORKLOADS[3].with_(ctx=ctx, HI=HI, topk=256)
+    assert wl.T % 4 == 0
+    y = decode_inputs(wl, device=DEV, batch=3)
+    if spread:
+        g = torch.Generator(device=DEV).manual_seed(23)
+        mag = torch.pow(2.0, torch.randint(-spread, spread + 1, (3, wl.T, 1), generator=g, device=DEV).float())
+        y["kI"] = (y["kI"].float() * mag).to(torch.bfloat16)
+    _decode_fp4_from(wl, y, seqs=[0, 1, 2])
+
+
+def _decode_fp4_from(wl, y, seqs):
+    P = wl.ctx - 1
+    qc, qs = csa.quantize_mxfp4(y["qI"])
+    kc, ks = csa.quantize_mxfp4(y["kI"])
+    o, idx = csa.decode_fp4(y["q"], qc, qs, y["w"], kc, ks, y["win"], y["sinks"], P, wl.topk, wl.r, wl.theta_tok,
+                            wl.theta_cmp, C=y["C"])
+    torch.cuda.synchronize()
+    seqs = np.asarray(seqs, np.int64)
+    h = {k: v[seqs].cpu() if v.dim() > 1 else v.cpu() for k, v in y.items()}
+    rq = oracle.mxfp4_quantize(h["qI"])
+    rk = oracle.mxfp4_quantize(h["kI"])
+    ridx, sc = oracle.decode_index_topk_fp4(rq[0], rq[1], h["w"], rk[0], rk[1], wl.topk)
+    gidx = idx.cpu().numpy()[seqs]
+    exc = check_topk_sets(gidx, ridx, sc, [wl.T] * len(seqs), wl.topk)
+    assert len(exc) <= 1, f"near-tie exceptions in {len(exc)} sequences"
+    ref = oracle.decode_attend(h["q"], h["win"], gidx, h["sinks"], P, wl.r, wl.theta_tok, wl.theta_cmp, C=h["C"])
+    check_close(o.cpu()[seqs], ref, O_MAX_ABS, O_MEAN_ABS, what="o")
+
+
 # ---- 7. HCA decode and the sliding-window-only layer ----------------------------------------------------
 
 # HCA at 1M context: m' = 128 pools 1,048,576 tokens into T = 8192 entries, all attended densely
