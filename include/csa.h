@@ -279,7 +279,7 @@ CSA_API csa_status csa_out_proj(const void *o, const void *wa, const void *wb, i
                       int32_t G, int32_t R, int32_t hidden, void *z, void *out, void *workspace,
                       size_t workspace_bytes, void *stream);
 
-/* ---- 11. FP4 (MXFP4) lightning indexer, decode -----------------------------------------------------
+/* ---- 11. FP4 (MXFP4) lightning indexer, prefill and decode ------------------------------------------
  * [Axbrief "Compressed attention and a new optimizer": MXFP4 on the lightning indexer's query-key
  * path; HF-blog digest: the indexer stored in FP4]. MXFP4 is the OCP Microscaling format: blocks of
  * 32 consecutive channels share an E8M0 scale 2^(e-127) (one byte); elements are E2M1 codes (values
@@ -297,6 +297,18 @@ CSA_API csa_status csa_out_proj(const void *o, const void *wa, const void *wb, i
  *   128; workspace as csa_decode (csa_workspace_size(CSA_OP_DECODE)). */
 CSA_API csa_status csa_quantize_mxfp4(const void *x, int64_t rows, int32_t cols, uint8_t *codes, uint8_t *scales,
                               void *stream);
+
+/* csa_index_topk_fp4: csa_index_topk (prefill, chunk at pos0) with the indexer's operands in MXFP4:
+ *   qI_codes [S, HI, dI/2], qI_scales [S, HI, dI/32], kI_codes [T, dI/2], kI_scales [T, dI/32]
+ *   (layout of csa_quantize_mxfp4); w [S, HI] fp32; idx [S, k] int32 (out).
+ * The scores are the indexer formula on the dequantised values (exact products, fp32 accumulation),
+ * computed by the block-scaled tensor-core MMA; the top-k is csa_index_topk's. Requires dI = 128,
+ * HI of 16, 32 or 64, T <= 4096, 16-byte aligned codes and 4-byte aligned scales. Workspace: 256 bytes
+ * (the status word). */
+CSA_API csa_status csa_index_topk_fp4(const uint8_t *qI_codes, const uint8_t *qI_scales, const float *w,
+                              const uint8_t *kI_codes, const uint8_t *kI_scales, int64_t S, int64_t pos0, int64_t T,
+                              int32_t HI, int32_t dI, int32_t m, int32_t k, int32_t *idx, void *workspace,
+                              size_t workspace_bytes, void *stream);
 
 CSA_API csa_status csa_decode_fp4(const void *q, const uint8_t *qI_codes, const uint8_t *qI_scales, const float *w,
                       const uint8_t *kI_codes, const uint8_t *kI_scales, const void *C, const uint8_t *c8,

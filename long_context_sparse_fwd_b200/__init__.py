@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "CSAError", "lib", "library_path", "compress", "index_topk", "attend", "hca_attend", "csa_forward",
     "hca_forward", "decode", "hca_decode", "swa_attend", "compress_append", "out_proj", "workspace_size",
-    "quantize_mxfp4", "decode_fp4",
+    "quantize_mxfp4", "decode_fp4", "index_topk_fp4",
     "get_device_status", "OP",
 ]
 
@@ -77,6 +77,7 @@ def lib():
                                           I32, P]),
             "csa_out_proj": (I32, [P, P, P, I64, I32, I32, I32, I32, I32, P, P, P, SZ, P]),
             "csa_quantize_mxfp4": (I32, [P, I64, I32, P, P, P]),
+            "csa_index_topk_fp4": (I32, [P, P, P, P, P, I64, I64, I64, I32, I32, I32, I32, P, P, SZ, P]),
             "csa_decode_fp4": (I32, [P, P, P, P, P, P, P, P, P, P, P, P, I32, I32, I32, I64, I32, I32, I32, I32, I32,
                                      I64, F64, F64, F32, P, P, P, SZ, P]),
         }
@@ -323,6 +324,26 @@ def quantize_mxfp4(x, codes=None, scales=None, stream=None):
         _dev(scales, torch.uint8, "scales", shape + (d // 32,))
     _check("csa_quantize_mxfp4", lib().csa_quantize_mxfp4(_ptr(x), rows, d, _ptr(codes), _ptr(scales), _stream(stream)))
     return codes, scales
+
+
+def index_topk_fp4(qc, qs, w, kc, ks, m: int, k: int, idx=None, workspace=None, pos0: int = 0,
+                   stream=None) -> torch.Tensor:
+    """Prefill lightning indexer + top-k on MXFP4 operands (csa_quantize_mxfp4 layout): qc [S, HI, dI/2],
+    qs [S, HI, dI/32], kc [T, dI/2], ks [T, dI/32] uint8; w [S, HI] fp32. Returns idx [S, k] int32."""
+    S, HI, half = qc.shape
+    dI = 2 * half
+    T = kc.shape[0]
+    _dev(qc, torch.uint8, "qI codes")
+    _dev(qs, torch.uint8, "qI scales", (S, HI, dI // 32))
+    _dev(kc, torch.uint8, "kI codes", (T, dI // 2))
+    _dev(ks, torch.uint8, "kI scales", (T, dI // 32))
+    _dev(w, torch.float32, "w", (S, HI))
+    idx = torch.empty(S, k, dtype=torch.int32, device=qc.device) if idx is None else _dev(idx, torch.int32, "idx", (S, k))
+    ws = _workspace("attend", qc.device, workspace)
+    _check("csa_index_topk_fp4", lib().csa_index_topk_fp4(_ptr(qc), _ptr(qs), _ptr(w), _ptr(kc), _ptr(ks), S, int(pos0),
+                                                          T, HI, dI, m, k, _ptr(idx), _ptr(ws), ws.numel(),
+                                                          _stream(stream)))
+    return idx
 
 
 def decode_fp4(q, qI_codes, qI_scales, w, kI_codes, kI_scales, win, sinks, P: int, k: int, rope_dim: int,

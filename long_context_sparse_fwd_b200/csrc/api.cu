@@ -455,6 +455,31 @@ csa_status csa_quantize_mxfp4(const void *x, int64_t rows, int32_t cols, uint8_t
                                            as_stream(stream)));
 }
 
+csa_status csa_index_topk_fp4(const uint8_t *qI_codes, const uint8_t *qI_scales, const float *w, const uint8_t *kI_codes,
+                              const uint8_t *kI_scales, int64_t S, int64_t pos0, int64_t T, int32_t HI, int32_t dI,
+                              int32_t m, int32_t k, int32_t *idx, void *workspace, size_t workspace_bytes, void *stream)
+{
+    CSA_CHECK_ARG(S >= 0 && pos0 >= 0 && pos0 <= ((int64_t)1 << 40) && T >= 0 && HI > 0 && dI > 0 && m >= 1 && k >= 1);
+    CSA_CHECK_ARG(T <= (pos0 + S) / m);
+    CSA_CHECK_ARG(S == 0 || (qI_codes != nullptr && qI_scales != nullptr && w != nullptr && idx != nullptr));
+    CSA_CHECK_ARG(T == 0 || (kI_codes != nullptr && kI_scales != nullptr));
+    CSA_CHECK_ARG(aligned16(qI_codes) && aligned16(kI_codes) && (reinterpret_cast<uintptr_t>(qI_scales) & 3u) == 0 &&
+                  (reinterpret_cast<uintptr_t>(kI_scales) & 3u) == 0);
+    CSA_CHECK_SUP(dI == 128 && (HI == 16 || HI == 32 || HI == 64) && T <= 4096);
+    CSA_CHECK_SUP(T == 0 || index_topk_fp4_supported(T, HI, dI, k));
+    CSA_TRY(check_workspace(workspace, workspace_bytes, kStatusBytes));
+    cudaStream_t st = as_stream(stream);
+    CSA_TRY(reset_status(workspace, st));
+    if (T == 0) {   // nothing visible yet: every slot is -1
+        float *none = nullptr;
+        CSA_CUDA(launch_topk_rows(none, S, pos0, 0, m, 0, k, idx, st));
+        return CSA_OK;
+    }
+    CSA_CUDA(launch_index_topk_fp4(qI_codes, qI_scales, w, kI_codes, kI_scales, S, pos0, T, HI, dI, m, k, idx,
+                                   static_cast<int32_t *>(workspace), st));
+    return CSA_OK;
+}
+
 csa_status csa_decode_fp4(const void *q, const uint8_t *qI_codes, const uint8_t *qI_scales, const float *w,
                           const uint8_t *kI_codes, const uint8_t *kI_scales, const void *C, const uint8_t *c8,
                           const float *c8_scale, const void *c_rope, const void *win, const float *sinks, int32_t B,

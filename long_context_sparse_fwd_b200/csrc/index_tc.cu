@@ -31,6 +31,8 @@ using namespace sm100;
 
 namespace {
 
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 constexpr int BM = 128;          // entries per tile = TMEM lanes
 constexpr int BN = 256;          // (query, head) columns
 constexpr int EPI_THREADS = 256;       // warps 2-9: two warps per TMEM lane quarter, each half of the queries
@@ -47,7 +49,16 @@ struct IdxParams {
     int64_t ngroups;     // groups of Q consecutive queries
     int HI, dI, m, k, Q, stages, T_cap;
     int nsb;             // scores buffers (2: the top-k of a group overlaps the next group's scoring)
+    int bn;              // (query, head) columns per group: 256 (bf16), 128 (MXFP4)
+    // MXFP4 operands (fp4 != 0): q^I and k^I as packed E2M1 codes (the tensor maps) with one E8M0
+    // scale per 32 channels: qs [S, HI, 4], ks [T, 4] (d_I = 128)
+    int fp4;
+    const uint8_t *qs, *ks;
 };
+
+// Scale-factor columns of the MXFP4 mode (after the two 128-column accumulators): per accumulator
+// buffer a k^I slot, per group parity a q^I slot, 4 columns each.
+constexpr uint32_t F4_SFA_COL = 256, F4_SFB_COL = 264;
 
 // Exact top-k of one query's scores by one warp: radix select over order-preserving keys, starting
 // at the highest bit where the keys differ (one query's scores usually share their leading bits), then
@@ -441,15 +452,20 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const int kchunks = p.dI / 64;                      // 128-byte swizzle atoms along K
-    const uint32_t b_bytes = (uint32_t)kchunks * BN * 128;
-    const uint32_t a_bytes = (uint32_t)kchunks * BM * 128;
+    const int kchunks = p.dI / 64;                      // 128-byte swizzle atoms along K (bf16)
+    // bf16: 128-byte swizzled rows of 64 channels; MXFP4: one 64-byte swizzled row of 128 packed codes
+    const uint32_t b_bytes = p.fp4 ? (uint32_t)p.bn * 64 : (uint32_t)kchunks * BN * 128;
+    const uint32_t a_bytes = p.fp4 ? (uint32_t)BM * 64 : (uint32_t)kchunks * BM * 128;
     uint8_t *sB = smem;
     uint8_t *sA = sB + b_bytes;
     float *scores_all = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [nsb][Q][T_cap]
     float *sw = scores_all + (size_t)p.nsb * p.Q * p.T_cap;                          // [BN]
     uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                          // [4 pairs][PBINS + 80]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(hist + 4 * (PBINS + 80));
+    // MXFP4: k^I scales of every tile [T_cap / 128][32 x 16 bytes] and the group's q^I scales [2][32 x 16]
+    // in the arrangement the scale copy into TMEM takes (row r: the scale words of rows r + 32 j)
+    uint8_t *sSFA = reinterpret_cast<uint8_t *>(hist + 4 * (PBINS + 80));
+    uint8_t *sSFB = sSFA + (p.fp4 ? (size_t)(p.T_cap / BM) * 512 : 0);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sSFB + (p.fp4 ? 1024 : 0));
     uint64_t *full = bars;                   // [stages] k^I tile landed
     uint64_t *empty = bars + 8;              // [stages] its MMAs completed
     uint64_t *tfull = bars + 16;             // [2] accumulator written
@@ -480,10 +496,19 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             mbar_init(&sfull[i], EPI_THREADS / 32);
             mbar_init(&sempty[i], TOPK_THREADS / 32);
         }
-        mbar_init(qfull, 1);
+        mbar_init(qfull, p.fp4 ? 2 : 1);   // MXFP4: the code load and the gathered q^I scales
         mbar_init(qempty, 1);
         *abort = 0;
         fence_barrier_init();
+    }
+    if (p.fp4) {   // every tile's k^I scales, once: tile t, row r, word j = the scale word of entry 128 t + r + 32 j
+        const int nwords = p.T_cap;
+        for (int e = threadIdx.x; e < nwords; e += NUM_THREADS) {
+            const uint32_t v = e < p.T ? *reinterpret_cast<const uint32_t *>(p.ks + (int64_t)e * 4) : 0u;
+            const int t = e / BM, rr = e % BM;
+            *reinterpret_cast<uint32_t *>(sSFA + t * 512 + (rr & 31) * 16 + (rr >> 5) * 4) = v;
+        }
+        fence_async_smem();   // read by tcgen05.cp through the async proxy
     }
     if (warp == 1) {
         tmem_alloc(tmem_base_ptr, TMEM_COLS);
@@ -511,12 +536,28 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             if (gi > 0 && !__all_sync(0xffffffffu, mbar_wait(qempty, (uint32_t)((gi - 1) & 1), abort, p.status))) break;
             if (elect_one()) {
                 mbar_arrive_expect_tx(qfull, b_bytes);
-                for (int c = 0; c < kchunks; ++c)
-                    tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
+                if (p.fp4) {
+                    tma_load_2d(sB, &tm_q, qfull, 0, (int)(t0 * p.HI));
+                } else {
+                    for (int c = 0; c < kchunks; ++c)
+                        tma_load_2d(sB + (size_t)c * BN * 128, &tm_q, qfull, c * 64, (int)(t0 * p.HI));
+                }
                 int64_t t1;
                 int n1;
                 if (group_of(gi + 1, &t1, &n1))   // the next group's q^I into L2 while this group computes
-                    for (int c = 0; c < kchunks; ++c) tma_prefetch_2d(&tm_q, c * 64, (int)(t1 * p.HI));
+                    for (int c = 0; c < (p.fp4 ? 1 : kchunks); ++c) tma_prefetch_2d(&tm_q, c * 64, (int)(t1 * p.HI));
+            }
+            if (p.fp4) {   // the group's q^I scales: lane r writes row r = the scale words of rows r + 32 j
+                uint32_t wq[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t row = t0 * p.HI + lane + 32 * j;   // (query, head) row of q^I
+                    wq[j] = lane + 32 * j < p.bn && row < p.S * p.HI ? *reinterpret_cast<const uint32_t *>(p.qs + row * 4) : 0u;
+                }
+                *reinterpret_cast<uint4 *>(sSFB + (gi & 1) * 512 + lane * 16) = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(qfull);
             }
             __syncwarp();
             ngr = gi + 1;
@@ -528,8 +569,12 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&full[st], a_bytes);
-                    for (int c = 0; c < kchunks; ++c)
-                        tma_load_2d(sA + (size_t)st * a_bytes + (size_t)c * BM * 128, &tm_k, &full[st], c * 64, i * BM);
+                    if (p.fp4) {
+                        tma_load_2d(sA + (size_t)st * a_bytes, &tm_k, &full[st], 0, i * BM);
+                    } else {
+                        for (int c = 0; c < kchunks; ++c)
+                            tma_load_2d(sA + (size_t)st * a_bytes + (size_t)c * BM * 128, &tm_k, &full[st], c * 64, i * BM);
+                    }
                 }
                 __syncwarp();
                 issued = tile + 1;
@@ -542,12 +587,19 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         const uint32_t idesc = idesc_bf16(BM, BN);
+        const uint32_t idf0 = idesc_mxf4(BM, p.bn, 0), idf2 = idesc_mxf4(BM, p.bn, 2);
         int tile = 0;
         bool ok = true;
         int64_t t0;
         int ntiles;
         for (int64_t gi = 0; ok && group_of(gi, &t0, &ntiles); ++gi) {
             if (!__all_sync(0xffffffffu, mbar_wait(qfull, (uint32_t)(gi & 1), abort, p.status))) break;
+            const uint32_t sfb = tmem_base + F4_SFB_COL + (uint32_t)(gi & 1) * 4;
+            if (p.fp4) {   // the group's q^I scales into TMEM (ordered before this thread's later MMAs)
+                tc_fence_after();
+                if (elect_one()) tmem_cp_32x128b_x4(sfb, sdesc_plain(smem_u32(sSFB + (gi & 1) * 512), 16, 128));
+                __syncwarp();
+            }
             for (int i = 0; i < ntiles; ++i, ++tile) {
                 const int st = tile % p.stages, buf = tile & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((tile >> 1) & 1) ^ 1, abort, p.status)) ||
@@ -556,6 +608,22 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     break;
                 }
                 tc_fence_after();
+                if (p.fp4) {
+                    if (elect_one()) {
+                        const uint32_t sfa = tmem_base + F4_SFA_COL + (uint32_t)buf * 4;
+                        tmem_cp_32x128b_x4(sfa, sdesc_plain(smem_u32(sSFA + i * 512), 16, 128));
+                        const uint32_t a0 = smem_u32(sA + (size_t)st * a_bytes), b0 = smem_u32(sB);
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks)   // channels 64 ks .. +63: scale bytes 2 ks, 2 ks + 1
+                            mma_mxf4(tmem_base + buf * p.bn, sdesc_sw64(a0 + ks * 32, 512), sdesc_sw64(b0 + ks * 32, 512),
+                                     ks ? idf2 : idf0, sfa | ((uint32_t)(2 * ks) << 30), sfb | ((uint32_t)(2 * ks) << 30),
+                                     ks != 0);
+                        mma_commit(&empty[st]);
+                        mma_commit(&tfull[buf]);
+                    }
+                    __syncwarp();
+                    continue;
+                }
                 if (elect_one()) {
                     const uint32_t a0 = smem_u32(sA + (size_t)st * a_bytes), b0 = smem_u32(sB);
                     for (int c = 0; c < kchunks; ++c) {
@@ -610,7 +678,7 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 }
                 tc_fence_after();
                 const int s = i * BM + quarter * 32 + lane;
-                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * BN;
+                const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * p.bn;
                 for (int q = qlo; q < qhi; ++q) {
                     // four independent partial sums break the dependent multiply-add chain
                     float acc4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -784,9 +852,10 @@ bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)
            encode_fn() != nullptr;
 }
 
-cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t pos0,
-                                 int64_t T, int HI, int dI, int m, int k, int32_t *idx, int32_t *status,
-                                 cudaStream_t stream)
+// Shared-memory plan and launch of the fused indexer for either operand format.
+static cudaError_t launch_index_topk(const void *qI, const void *kI, const uint8_t *qs, const uint8_t *ks, bool fp4,
+                                     const float *w, int64_t S, int64_t pos0, int64_t T, int HI, int dI, int m, int k,
+                                     int32_t *idx, int32_t *status, cudaStream_t stream)
 {
     if (S == 0) return cudaSuccess;
     IdxParams p;
@@ -800,23 +869,34 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     p.dI = dI;
     p.m = m;
     p.k = k;
-    p.Q = BN / HI;
+    p.fp4 = fp4 ? 1 : 0;
+    p.qs = qs;
+    p.ks = ks;
+    p.bn = fp4 ? 128 : BN;   // MXFP4: two 128-column accumulators leave TMEM room for the scales
+    p.Q = p.bn / HI;
     p.T_cap = (int)((T + BM - 1) / BM * BM);
     p.ngroups = (S + p.Q - 1) / p.Q;
-    const size_t a_bytes = (size_t)(dI / 64) * BM * 128, b_bytes = (size_t)(dI / 64) * BN * 128;
+    const size_t a_bytes = fp4 ? (size_t)BM * 64 : (size_t)(dI / 64) * BM * 128;
+    const size_t b_bytes = fp4 ? (size_t)p.bn * 64 : (size_t)(dI / 64) * BN * 128;
+    const size_t sf_bytes = fp4 ? (size_t)(p.T_cap / BM) * 512 + 1024 : 0;
     const size_t budget = 227 * 1024;
     size_t fixed = 0;
     for (p.nsb = 2; p.nsb >= 1; --p.nsb) {   // two scores buffers when three key stages still fit
-        fixed = 1024 + b_bytes + (size_t)p.nsb * p.Q * p.T_cap * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + 256;
+        fixed = 1024 + b_bytes + (size_t)p.nsb * p.Q * p.T_cap * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + sf_bytes + 256;
         if (fixed + 2 * a_bytes <= budget) break;
     }
     if (p.nsb < 1) return cudaErrorInvalidValue;
-    p.stages = (int)std::min<size_t>(4, (budget - fixed) / a_bytes);
+    p.stages = (int)std::min<size_t>(fp4 ? 8 : 4, (budget - fixed) / a_bytes);
     if (p.stages < 2) return cudaErrorInvalidValue;
     const size_t smem = fixed + (size_t)p.stages * a_bytes;
     CUtensorMap tq, tk;
-    if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)S * HI, dI, BN)) return cudaErrorInvalidValue;
-    if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)T, dI, BM)) return cudaErrorInvalidValue;
+    if (fp4) {
+        if (!make_tmap_u8_sw64(&tq, qI, (uint64_t)S * HI, (uint32_t)p.bn)) return cudaErrorInvalidValue;
+        if (!make_tmap_u8_sw64(&tk, kI, (uint64_t)T, BM)) return cudaErrorInvalidValue;
+    } else {
+        if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)S * HI, dI, BN)) return cudaErrorInvalidValue;
+        if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)T, dI, BM)) return cudaErrorInvalidValue;
+    }
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(index_topk_tc_kernel), smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
@@ -824,6 +904,26 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
     const unsigned grid = (unsigned)std::min<int64_t>(nsm, p.ngroups);   // persistent
     index_topk_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tk, p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t pos0,
+                                 int64_t T, int HI, int dI, int m, int k, int32_t *idx, int32_t *status,
+                                 cudaStream_t stream)
+{
+    return launch_index_topk(qI, kI, nullptr, nullptr, false, w, S, pos0, T, HI, dI, m, k, idx, status, stream);
+}
+
+bool index_topk_fp4_supported(int64_t T, int HI, int dI, int k)
+{
+    (void)k;
+    return dI == 128 && (HI == 16 || HI == 32 || HI == 64) && T >= 1 && T <= 4096 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_index_topk_fp4(const uint8_t *qc, const uint8_t *qs, const float *w, const uint8_t *kc,
+                                  const uint8_t *ks, int64_t S, int64_t pos0, int64_t T, int HI, int dI, int m, int k,
+                                  int32_t *idx, int32_t *status, cudaStream_t stream)
+{
+    return launch_index_topk(qc, kc, qs, ks, true, w, S, pos0, T, HI, dI, m, k, idx, status, stream);
 }
 
 }  // namespace csa

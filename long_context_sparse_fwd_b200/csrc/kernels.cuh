@@ -103,5 +103,10 @@ bool index_topk_tc_supported(int64_t T, int HI, int dI, int k);
 cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t pos0,
                                  int64_t T, int HI, int dI, int m, int k, int32_t *idx, int32_t *status,
                                  cudaStream_t stream);
+// the same on MXFP4 q^I and k^I (d_I = 128, HI <= 64): block-scaled MMA, fused top-k
+bool index_topk_fp4_supported(int64_t T, int HI, int dI, int k);
+cudaError_t launch_index_topk_fp4(const uint8_t *qc, const uint8_t *qs, const float *w, const uint8_t *kc,
+                                  const uint8_t *ks, int64_t S, int64_t pos0, int64_t T, int HI, int dI, int m, int k,
+                                  int32_t *idx, int32_t *status, cudaStream_t stream);
 
 }  // namespace csa

@@ -365,3 +365,11 @@ def decode_index_topk_fp4(qc, qs, w, kc, ks, k: int, rows=None):
     qv = _bf16_bits_exact(mxfp4_dequantize(qc, qs))
     kv = _bf16_bits_exact(mxfp4_dequantize(kc, ks))
     return decode_index_topk(qv, w, kv, k, rows=rows)
+
+
+def index_topk_fp4(qc, qs, w, kc, ks, m: int, k: int, rows=None):
+    """Prefill indexer + top-k on MXFP4 operands: the indexer formula on the dequantised q^I [S, HI, dI]
+    and k^I [T, dI] (exact in bf16, see decode_index_topk_fp4)."""
+    qv = _bf16_bits_exact(mxfp4_dequantize(qc, qs))
+    kv = _bf16_bits_exact(mxfp4_dequantize(kc, ks))
+    return index_topk(qv, kv, w, m, k, rows=rows)

@@ -199,5 +199,13 @@ def test_fp4_calls_reject_bad_arguments():
     assert df(kc=None) == INVALID               # entries but no index key codes
     assert df(C=None) == INVALID                # entries but neither a bf16 nor an FP8 cache
     assert df(dI=96) == UNSUP                   # MXFP4 scan: d_I of 64 or 128
+
+    def pf(qc=FAKE, kc=FAKE, S=64, pos0=0, T=16, HI=64, dI=128, k=8, qs=FAKE):
+        return L.csa_index_topk_fp4(qc, qs, FAKE, kc, FAKE, S, pos0, T, HI, dI, 4, k, FAKE, FAKE, 256, None)
+    assert pf(T=17) == INVALID                  # more entries than floor((pos0 + S) / m)
+    assert pf(qc=None) == INVALID
+    assert pf(qs=ctypes.c_void_p(0x10002)) == INVALID   # scales must be 4-byte aligned
+    assert pf(dI=64) == UNSUP                   # the block-scaled prefill path takes d_I = 128
+    assert pf(HI=128) == UNSUP
     assert df(HI=48) == UNSUP
     assert df(wsb=16) == WS

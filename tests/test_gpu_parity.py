@@ -505,6 +505,28 @@ def _decode_fp4_from(wl, y, seqs):
     check_close(o.cpu()[seqs], ref, O_MAX_ABS, O_MEAN_ABS, what="o")
 
 
+@pytest.mark.parametrize("HI,S,k,pos0,nrows", [(64, 8192, 512, 0, 160), (16, 1030, 64, 0, None),
+                                                (32, 2048 + 37, 128, 0, 96), (64, 3000, 256, 1000, 96)])
+def test_index_topk_fp4_prefill(HI, S, k, pos0, nrows):
+    """Prefill lightning indexer on MXFP4 operands (block-scaled MMA, fused top-k): V4-Flash shapes at
+    S = 8192 (sampled rows), N = 16 and 32 head columns with ragged entry tiles, and a chunk at pos0 > 0
+    against the whole sequence's entries; sets equal the oracle's on the dequantised operands."""
+    wl = WORKLOADS[1].with_(S=S, HI=HI, topk=k)
+    g, x = gen(prefill_inputs, wl, need_q=False)
+    qc, qs = csa.quantize_mxfp4(g["qI"].reshape(S * HI, wl.dI))
+    kc, ks = csa.quantize_mxfp4(g["kI"])
+    qc, qs = qc.reshape(S, HI, wl.dI // 2), qs.reshape(S, HI, wl.dI // 32)
+    a = pos0
+    idx = csa.index_topk_fp4(qc[a:], qs[a:], g["w"][a:], kc, ks, wl.m, k, pos0=a)
+    torch.cuda.synchronize()
+    rows = np.arange(a, S) if nrows is None else sample_rows(S - a, nrows, 29, must=[0, 1, S - a - 1]) + a
+    hq, hk = (qc.cpu(), qs.cpu()), (kc.cpu(), ks.cpu())
+    ridx, sc = oracle.index_topk_fp4(hq[0], hq[1], x["w"], hk[0], hk[1], wl.m, k, rows=rows)
+    vis = [oracle.visible(t, wl.m, wl.T) for t in rows]
+    exc = check_topk_sets(idx.cpu().numpy()[rows - a], ridx, sc, vis, k)
+    assert len(exc) <= max(2, len(rows) // 50), f"too many near-tie exceptions: {exc[:5]}"
+
+
 # ---- 7. HCA decode and the sliding-window-only layer ----------------------------------------------------
 
 # HCA at 1M context: m' = 128 pools 1,048,576 tokens into T = 8192 entries, all attended densely
