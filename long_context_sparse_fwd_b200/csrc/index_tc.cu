@@ -50,6 +50,11 @@ struct IdxParams {
     int HI, dI, m, k, Q, stages, T_cap;
     int nsb;             // scores buffers (2: the top-k of a group overlaps the next group's scoring)
     int bn;              // (query, head) columns per group: 256 (bf16), 128 (MXFP4)
+    // Entries are scored in chunks of `chunk` (a multiple of 128). One chunk covering every entry
+    // (kcap = 0) is ranked in place. Otherwise each query's scores buffer holds its running top-k
+    // (up to kcap scores) right before the chunk's scores, so the ranking of [running set, chunk]
+    // keeps the running set exact; qstride = kcap + chunk floats per query.
+    int chunk, kcap, qstride;
     // MXFP4 operands (fp4 != 0): q^I and k^I as packed E2M1 codes (the tensor maps) with one E8M0
     // scale per 32 channels: qs [S, HI, 4], ks [T, 4] (d_I = 128)
     int fp4;
@@ -458,12 +463,18 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t a_bytes = p.fp4 ? (uint32_t)BM * 64 : (uint32_t)kchunks * BM * 128;
     uint8_t *sB = smem;
     uint8_t *sA = sB + b_bytes;
-    float *scores_all = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [nsb][Q][T_cap]
-    float *sw = scores_all + (size_t)p.nsb * p.Q * p.T_cap;                          // [BN]
+    float *scores_all = reinterpret_cast<float *>(sA + (size_t)p.stages * a_bytes);   // [nsb][Q][qstride]
+    float *sw = scores_all + (size_t)p.nsb * p.Q * p.qstride;                        // [BN]
     uint32_t *hist = reinterpret_cast<uint32_t *>(sw + BN);                          // [4 pairs][PBINS + 80]
     // MXFP4: k^I scales of every tile [T_cap / 128][32 x 16 bytes] and the group's q^I scales [2][32 x 16]
     // in the arrangement the scale copy into TMEM takes (row r: the scale words of rows r + 32 j)
-    uint8_t *sSFA = reinterpret_cast<uint8_t *>(hist + 4 * (PBINS + 80));
+    // chunked ranking: running top-k of each query (scores, entry indices, count) and each pair's
+    // selected positions
+    float *run_sc = reinterpret_cast<float *>(hist + 4 * (PBINS + 80));              // [Q][kcap]
+    int32_t *run_idx = reinterpret_cast<int32_t *>(run_sc + (size_t)p.Q * p.kcap);     // [Q][kcap]
+    int32_t *run_cnt = run_idx + (size_t)p.Q * p.kcap;                                 // [Q] (16-aligned)
+    int32_t *sel_all = run_cnt + ((p.kcap > 0 ? p.Q : 0) + 3) / 4 * 4;                 // [4 pairs][kcap]
+    uint8_t *sSFA = reinterpret_cast<uint8_t *>(sel_all + 4 * (size_t)p.kcap);
     uint8_t *sSFB = sSFA + (p.fp4 ? (size_t)(p.T_cap / BM) * 512 : 0);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sSFB + (p.fp4 ? 1024 : 0));
     uint64_t *full = bars;                   // [stages] k^I tile landed
@@ -658,26 +669,47 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         bool ok = true;
         int64_t t0;
         int ntiles;
+        const int ct = p.chunk / BM;   // tiles per chunk
+        int64_t unit = 0;              // (group, chunk) units so far: the scores buffers go round by unit
+        float *scores = scores_all;
+        int sb = 0;
         for (int64_t gi = 0; ok && group_of(gi, &t0, &ntiles); ++gi) {
-            const int sb = (int)(gi % p.nsb);
-            const int64_t use = gi / p.nsb;   // earlier uses of this scores buffer
-            if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(&sempty[sb], (uint32_t)((use - 1) & 1), abort, p.status)))
-                break;
-            float *scores = scores_all + (size_t)sb * p.Q * p.T_cap;
             named_barrier_sync(1, EPI_THREADS);   // every epilogue thread is done with the previous weights
             for (int i = etid; i < p.Q * p.HI; i += EPI_THREADS) {
                 const int64_t t = t0 + i / p.HI;
                 sw[i] = t < p.S ? p.w[t * p.HI + (i % p.HI)] : 0.f;
             }
             named_barrier_sync(1, EPI_THREADS);
+            if (ntiles == 0) {   // nothing visible to the group yet: one empty chunk, so its rows get -1
+                sb = (int)(unit % p.nsb);
+                const int64_t use = unit / p.nsb;
+                if (use > 0 &&
+                    !__all_sync(0xffffffffu, mbar_wait(&sempty[sb], (uint32_t)((use - 1) & 1), abort, p.status))) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfull[sb]);
+                ++unit;
+            }
             for (int i = 0; i < ntiles; ++i, ++tile) {
+                if (i % ct == 0) {   // a new chunk: its scores buffer once the top-k is done with it
+                    sb = (int)(unit % p.nsb);
+                    const int64_t use = unit / p.nsb;   // earlier uses of this scores buffer
+                    if (use > 0 &&
+                        !__all_sync(0xffffffffu, mbar_wait(&sempty[sb], (uint32_t)((use - 1) & 1), abort, p.status))) {
+                        ok = false;
+                        break;
+                    }
+                    scores = scores_all + (size_t)sb * p.Q * p.qstride + p.kcap;
+                }
                 const int buf = tile & 1;
                 if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (tile >> 1) & 1, abort, p.status))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int s = i * BM + quarter * 32 + lane;
+                const int s = (i % ct) * BM + quarter * 32 + lane;   // entry within the chunk
                 const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + buf * p.bn;
                 for (int q = qlo; q < qhi; ++q) {
                     // four independent partial sums break the dependent multiply-add chain
@@ -713,37 +745,85 @@ index_topk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         }
                     }
                     const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-                    if (s < p.T_cap) scores[q * p.T_cap + s] = acc + 0.0f;
+                    scores[q * p.qstride + s] = acc + 0.0f;
                 }
                 tc_fence_before();
                 mbar_arrive(&tempty[buf]);
+                if (i % ct == ct - 1 || i + 1 == ntiles) {   // this warp's scores of the chunk are in place
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sfull[sb]);
+                    ++unit;
+                }
             }
             if (!ok) break;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sfull[sb]);   // this warp's scores of the group are in place
         }
     } else {
         // ---------------- exact top-k of the previous group's queries, one query per pair of warps ----
         const int pair = (warp - 2 - EPI_THREADS / 32) >> 1;
+        const int pt = threadIdx.x & 63;
+        const int bar = 2 + pair;
+        uint32_t *scratch = hist + pair * (PBINS + 80);
+        int32_t *sel = sel_all + pair * p.kcap;
+        const int ct = p.chunk / BM;
+        int64_t unit = 0;
         int64_t t0;
         int ntiles;
-        for (int64_t gi = 0; group_of(gi, &t0, &ntiles); ++gi) {
-            const int sb = (int)(gi % p.nsb);
-            if (!__all_sync(0xffffffffu, mbar_wait(&sfull[sb], (uint32_t)((gi / p.nsb) & 1), abort, p.status))) break;
-            const float *scores = scores_all + (size_t)sb * p.Q * p.T_cap;
-            for (int q = pair; q < p.Q; q += 4) {
-                const int64_t t = t0 + q;
-                if (t >= p.S) continue;
-                const int n = (int)visible_entries(p.pos0 + t, p.m, p.T);
-                if (n > p.k && n <= 2048)
-                    topk_pair_reg(scores + (size_t)q * p.T_cap, n, p.k, hist + pair * (PBINS + 80), 2 + pair,
-                                  p.idx + t * (int64_t)p.k);
-                else
-                    topk_pair(scores + (size_t)q * p.T_cap, n, p.k, hist + pair * (PBINS + 80), 2 + pair,
-                              p.idx + t * (int64_t)p.k);
+        bool ok = true;
+        for (int64_t gi = 0; ok && group_of(gi, &t0, &ntiles); ++gi) {
+            const int nch = max(1, (ntiles + ct - 1) / ct);   // a group with no entries yet: one empty chunk
+            for (int c = 0; c < nch; ++c, ++unit) {
+                const int sb = (int)(unit % p.nsb);
+                if (!__all_sync(0xffffffffu, mbar_wait(&sfull[sb], (uint32_t)((unit / p.nsb) & 1), abort, p.status))) {
+                    ok = false;
+                    break;
+                }
+                float *scores = scores_all + (size_t)sb * p.Q * p.qstride;
+                for (int q = pair; q < p.Q; q += 4) {
+                    const int64_t t = t0 + q;
+                    if (t >= p.S) continue;
+                    const int n = (int)visible_entries(p.pos0 + t, p.m, p.T);
+                    int32_t *orow = p.idx + t * (int64_t)p.k;
+                    float *sq = scores + (size_t)q * p.qstride + p.kcap;   // the chunk's scores of query q
+                    if (p.kcap == 0) {   // every entry in one chunk: rank it in place
+                        if (n > p.k && n <= 2048)
+                            topk_pair_reg(sq, n, p.k, scratch, bar, orow);
+                        else
+                            topk_pair(sq, n, p.k, scratch, bar, orow);
+                        continue;
+                    }
+                    const int nc = min(max(n - c * p.chunk, 0), p.chunk);   // this query's entries in the chunk
+                    if (nc == 0) {
+                        if (c == 0)   // nothing visible yet: every slot is -1
+                            for (int j = pt; j < p.k; j += 64) orow[j] = -1;
+                        continue;
+                    }
+                    const int r = c == 0 ? 0 : run_cnt[q];
+                    for (int j = pt; j < r; j += 64) sq[j - r] = run_sc[q * p.kcap + j];   // running set first
+                    pair_sync(bar);
+                    const int nn = r + nc;
+                    if (nn > p.k && nn <= 2048)
+                        topk_pair_reg(sq - r, nn, p.k, scratch, bar, sel);
+                    else
+                        topk_pair(sq - r, nn, p.k, scratch, bar, sel);
+                    // the new running set: positions below r are running entries, the rest chunk entries. Its
+                    // scores are read from the ranked buffer (the running scores were copied there), its
+                    // entry indices replace the positions in `sel` (each slot by its own thread), then move.
+                    const int r2 = min(p.k, nn);
+                    for (int j = pt; j < r2; j += 64) {
+                        const int pos = sel[j];
+                        run_sc[q * p.kcap + j] = sq[pos - r];
+                        sel[j] = pos < r ? run_idx[q * p.kcap + pos] : c * p.chunk + (pos - r);
+                    }
+                    pair_sync(bar);
+                    for (int j = pt; j < r2; j += 64) run_idx[q * p.kcap + j] = sel[j];
+                    if (pt == 0) run_cnt[q] = r2;
+                    pair_sync(bar);
+                    if ((c + 1) * p.chunk >= n)   // the query's last chunk: its selection, ascending
+                        for (int j = pt; j < p.k; j += 64) orow[j] = j < r2 ? run_idx[q * p.kcap + j] : -1;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sempty[sb]);   // the buffer may take a later chunk's scores
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sempty[sb]);   // the buffer may take a later group's scores
         }
     }
     tc_fence_before();
@@ -845,19 +925,61 @@ bool make_tmap_u8_sw64_perm4(CUtensorMap *map, const void *base, uint64_t rows)
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)
+
+// Shared-memory plan of the fused indexer: every entry in one chunk when the scores of a group's
+// queries fit (two scores buffers when three key stages still fit), else (bf16, k <= 1024) chunks of
+// entries with a running top-k per query, one scores buffer, the chunk as long as shared memory allows.
+struct IdxPlan {
+    int bn, Q, T_cap, nsb, stages, chunk, kcap, qstride;
+    size_t smem;
+};
+
+static bool plan_index_topk(int64_t T, int HI, int dI, int k, bool fp4, IdxPlan *pl)
 {
-    (void)k;
-    return (dI == 64 || dI == 128) && (HI == 16 || HI == 32 || HI == 64 || HI == 128) && T <= 4096 && T >= 1 &&
-           encode_fn() != nullptr;
+    if (T < 1 || T > (1ll << 24) || !(dI == 64 || dI == 128) || !(HI == 16 || HI == 32 || HI == 64 || HI == 128))
+        return false;
+    if (fp4 && (dI != 128 || HI > 64 || T > 4096)) return false;
+    pl->bn = fp4 ? 128 : BN;   // MXFP4: two 128-column accumulators leave TMEM room for the scales
+    pl->Q = pl->bn / HI;
+    pl->T_cap = (int)((T + BM - 1) / BM * BM);
+    const size_t a_bytes = fp4 ? (size_t)BM * 64 : (size_t)(dI / 64) * BM * 128;
+    const size_t b_bytes = fp4 ? (size_t)pl->bn * 64 : (size_t)(dI / 64) * BN * 128;
+    const size_t sf_bytes = fp4 ? (size_t)(pl->T_cap / BM) * 512 + 1024 : 0;
+    const size_t budget = 227 * 1024;
+    auto fixed_of = [&](int nsb, int qstride, int kcap) {
+        const size_t run = kcap > 0 ? (size_t)pl->Q * kcap * 8 + (size_t)(pl->Q + 3) / 4 * 16 + 4 * (size_t)kcap * 4 : 0;
+        return 1024 + b_bytes + (size_t)nsb * pl->Q * qstride * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + run + sf_bytes + 256;
+    };
+    pl->kcap = 0;
+    pl->chunk = pl->qstride = pl->T_cap;
+    for (pl->nsb = 2; pl->nsb >= 1; --pl->nsb)
+        if (fixed_of(pl->nsb, pl->qstride, 0) + 2 * a_bytes <= budget) break;
+    if (pl->nsb < 1) {   // chunks of entries with a running top-k
+        if (fp4 || k > 1024) return false;
+        pl->nsb = 1;
+        pl->kcap = (k + 3) & ~3;
+        const size_t base = fixed_of(1, 0, pl->kcap) + 2 * a_bytes;
+        if (base >= budget) return false;
+        const int64_t room = (int64_t)((budget - base) / ((size_t)pl->Q * 4)) - pl->kcap;   // floats per query
+        pl->chunk = (int)std::min<int64_t>(room / BM * BM, pl->T_cap);
+        if (pl->chunk < 4 * BM) return false;
+        pl->qstride = pl->kcap + pl->chunk;
+    }
+    const size_t fixed = fixed_of(pl->nsb, pl->qstride, pl->kcap);
+    pl->stages = (int)std::min<size_t>(fp4 ? 8 : 4, (budget - fixed) / a_bytes);
+    if (pl->stages < 2) return false;
+    pl->smem = fixed + (size_t)pl->stages * a_bytes;
+    return true;
 }
 
-// Shared-memory plan and launch of the fused indexer for either operand format.
+// Launch of the fused indexer for either operand format.
 static cudaError_t launch_index_topk(const void *qI, const void *kI, const uint8_t *qs, const uint8_t *ks, bool fp4,
                                      const float *w, int64_t S, int64_t pos0, int64_t T, int HI, int dI, int m, int k,
                                      int32_t *idx, int32_t *status, cudaStream_t stream)
 {
     if (S == 0) return cudaSuccess;
+    IdxPlan pl;
+    if (!plan_index_topk(T, HI, dI, k, fp4, &pl)) return cudaErrorInvalidValue;
     IdxParams p;
     p.w = w;
     p.idx = idx;
@@ -872,23 +994,15 @@ static cudaError_t launch_index_topk(const void *qI, const void *kI, const uint8
     p.fp4 = fp4 ? 1 : 0;
     p.qs = qs;
     p.ks = ks;
-    p.bn = fp4 ? 128 : BN;   // MXFP4: two 128-column accumulators leave TMEM room for the scales
-    p.Q = p.bn / HI;
-    p.T_cap = (int)((T + BM - 1) / BM * BM);
+    p.bn = pl.bn;
+    p.Q = pl.Q;
+    p.T_cap = pl.T_cap;
+    p.nsb = pl.nsb;
+    p.stages = pl.stages;
+    p.chunk = pl.chunk;
+    p.kcap = pl.kcap;
+    p.qstride = pl.qstride;
     p.ngroups = (S + p.Q - 1) / p.Q;
-    const size_t a_bytes = fp4 ? (size_t)BM * 64 : (size_t)(dI / 64) * BM * 128;
-    const size_t b_bytes = fp4 ? (size_t)p.bn * 64 : (size_t)(dI / 64) * BN * 128;
-    const size_t sf_bytes = fp4 ? (size_t)(p.T_cap / BM) * 512 + 1024 : 0;
-    const size_t budget = 227 * 1024;
-    size_t fixed = 0;
-    for (p.nsb = 2; p.nsb >= 1; --p.nsb) {   // two scores buffers when three key stages still fit
-        fixed = 1024 + b_bytes + (size_t)p.nsb * p.Q * p.T_cap * 4 + BN * 4 + 4 * (PBINS + 80) * 4 + sf_bytes + 256;
-        if (fixed + 2 * a_bytes <= budget) break;
-    }
-    if (p.nsb < 1) return cudaErrorInvalidValue;
-    p.stages = (int)std::min<size_t>(fp4 ? 8 : 4, (budget - fixed) / a_bytes);
-    if (p.stages < 2) return cudaErrorInvalidValue;
-    const size_t smem = fixed + (size_t)p.stages * a_bytes;
     CUtensorMap tq, tk;
     if (fp4) {
         if (!make_tmap_u8_sw64(&tq, qI, (uint64_t)S * HI, (uint32_t)p.bn)) return cudaErrorInvalidValue;
@@ -897,13 +1011,19 @@ static cudaError_t launch_index_topk(const void *qI, const void *kI, const uint8
         if (!make_tmap_bf16_sw128(&tq, qI, (uint64_t)S * HI, dI, BN)) return cudaErrorInvalidValue;
         if (!make_tmap_bf16_sw128(&tk, kI, (uint64_t)T, dI, BM)) return cudaErrorInvalidValue;
     }
-    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(index_topk_tc_kernel), smem);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(index_topk_tc_kernel), pl.smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<int64_t>(nsm, p.ngroups);   // persistent
-    index_topk_tc_kernel<<<grid, NUM_THREADS, smem, stream>>>(tq, tk, p);
+    index_topk_tc_kernel<<<grid, NUM_THREADS, pl.smem, stream>>>(tq, tk, p);
     return cudaGetLastError();
+}
+
+bool index_topk_tc_supported(int64_t T, int HI, int dI, int k)
+{
+    IdxPlan pl;
+    return encode_fn() != nullptr && plan_index_topk(T, HI, dI, k, false, &pl);
 }
 
 cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const float *w, int64_t S, int64_t pos0,
@@ -915,8 +1035,8 @@ cudaError_t launch_index_topk_tc(const uint16_t *qI, const uint16_t *kI, const f
 
 bool index_topk_fp4_supported(int64_t T, int HI, int dI, int k)
 {
-    (void)k;
-    return dI == 128 && (HI == 16 || HI == 32 || HI == 64) && T >= 1 && T <= 4096 && encode_fn() != nullptr;
+    IdxPlan pl;
+    return encode_fn() != nullptr && plan_index_topk(T, HI, dI, k, true, &pl);
 }
 
 cudaError_t launch_index_topk_fp4(const uint8_t *qc, const uint8_t *qs, const float *w, const uint8_t *kc,

@@ -81,10 +81,12 @@ def test_index_topk(wid, S, nrows):
 
 
 @pytest.mark.parametrize("HI,dI,S,k", [(64, 128, 1030, 16), (32, 64, 777, 40), (128, 128, 600, 8),
-                                        (16, 64, 5000, 300), (64, 128, 16384, 512), (64, 128, 20000, 512)])
+                                        (16, 64, 5000, 300), (64, 128, 16384, 512), (64, 128, 20000, 512),
+                                        (16, 64, 30000, 300), (64, 128, 40000, 1024), (64, 128, 65536, 512)])
 def test_index_topk_shapes(HI, dI, S, k):
-    """Tensor-core path shapes (N = 256 query-head columns, T up to 4096 on chip), ragged query
-    blocks and entry tiles, k above and below vis(t); S=20000 (T > 4096) takes the general path."""
+    """Tensor-core path shapes (N = 256 query-head columns), ragged query blocks and entry tiles, k above
+    and below vis(t). Up to 4096 entries the scores of a group stay on chip whole; past that (S = 20000
+    and up, to 16384 entries at S = 65536) they are ranked chunk by chunk against a running top-k."""
     wl = WORKLOADS[1].with_(S=S, HI=HI, dI=dI, topk=k)
     g, x = gen(prefill_inputs, wl, need_q=False)
     idx = csa.index_topk(g["qI"], g["kI"], g["w"], wl.m, wl.topk)
@@ -121,19 +123,31 @@ def test_index_topk_tc_all_zero_ties():
         assert idx[t][:n].tolist() == list(range(n)) and (idx[t][n:] == -1).all(), t
 
 
-@pytest.mark.parametrize("classes,k", [(6, 128), (2, 300)])
-def test_index_topk_tc_few_distinct_scores(classes, k):
+def test_index_topk_tc_chunked_all_zero_ties():
+    """Past 4096 entries (chunked ranking) with weights 0: every score is exactly 0 and each query keeps
+    its k smallest visible indices, so ties across chunk boundaries go to the smaller index."""
+    wl = WORKLOADS[1].with_(S=24000, HI=64, dI=128, topk=512)
+    g, _ = gen(prefill_inputs, wl, need_q=False)
+    g["w"] = torch.zeros_like(g["w"])
+    idx = csa.index_topk(g["qI"], g["kI"], g["w"], wl.m, wl.topk).cpu().numpy()
+    for t in [0, 2, 3, 2047, 2048, 11775, 11776, 12000, 16383, 23999]:
+        n = min(wl.topk, (t + 1) // wl.m)
+        assert idx[t][:n].tolist() == list(range(n)) and (idx[t][n:] == -1).all(), t
+
+
+@pytest.mark.parametrize("classes,k,S", [(6, 128, 4100), (2, 300, 4100), (3, 256, 20004)])
+def test_index_topk_tc_few_distinct_scores(classes, k, S):
     """Tensor-core indexer with k^I rows repeating `classes` vectors: each query's scores take only
     that many values, so its threshold value is shared by many entries (ranked directly, or the
     crowded-bin path past 512). The selection must equal the oracle's exactly."""
-    wl = WORKLOADS[1].with_(S=4100, HI=64, dI=128, topk=k)
+    wl = WORKLOADS[1].with_(S=S, HI=64, dI=128, topk=k)
     g, x = gen(prefill_inputs, wl, need_q=False)
     pattern = torch.arange(wl.T) % classes
     kI = x["kI"][:classes][pattern].contiguous()
     x["kI"] = kI
     g["kI"] = kI.to(DEV)
     idx = csa.index_topk(g["qI"], g["kI"], g["w"], wl.m, wl.topk).cpu().numpy()
-    rows = sample_rows(wl.S, 48, 5, must=[0, 7, 1023, 2047, 2048, 4095, 4099])
+    rows = sample_rows(wl.S, 48, 5, must=[0, 7, 1023, 2047, 2048, 4095, 4099, S - 1])
     ridx, _ = oracle.index_topk(x["qI"], x["kI"], x["w"], wl.m, wl.topk, rows=rows)
     for i, t in enumerate(rows):
         assert np.array_equal(idx[t], np.asarray(ridx[i], np.int32)), t
@@ -318,6 +332,8 @@ def test_index_topk_workspace_is_status_word_on_the_tensor_core_path():
     """The fused tensor-core indexer keeps its scores on chip: its workspace is the status word only."""
     assert csa.workspace_size("index_topk", S=8192, T=2048, HI=64, dI=128, k=512) == 256
     assert csa.workspace_size("csa_forward", S=8192, T=2048, HI=64, dI=128, k=512) == 256
+    # past 4096 entries as well: ranked chunk by chunk on chip, no S x T scores
+    assert csa.workspace_size("index_topk", S=65536, T=16384, HI=64, dI=128, k=512) == 256
 
 
 def test_forward_is_deterministic():
