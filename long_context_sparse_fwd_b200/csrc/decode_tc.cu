@@ -48,13 +48,27 @@ struct ScoreParams {
     int HI, dI, stages, tps;
 };
 
+// (sequence, tile within the sequence) of a CTA's consecutive tiles, advanced without a 64-bit division
+// per tile (one costs some 450 cycles of a role's per-tile loop).
+struct TileCursor {
+    int64_t b;
+    int it, tps;
+    __device__ TileCursor(int64_t g0, int tps_) : b(g0 / tps_), it((int)(g0 - (g0 / tps_) * tps_)), tps(tps_) {}
+    __device__ __forceinline__ void next()
+    {
+        if (++it == tps) {
+            it = 0;
+            ++b;
+        }
+    }
+};
+
 // Epilogue of the scan (four warps, 128 threads, one TMEM lane quarter each): each thread owns one entry
 // of the tile, reduces its HI heads (w-weighted ReLU) in registers and writes one fp32 score; it also
 // tracks the sequence's key range for the top-k and clears the chunked top-k's counters.
-// With perm4, accumulator row 32 j + r holds entry 4 r + j of the tile (the block-scaled MXFP4 scan).
 __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tmem, uint64_t *tfull, uint64_t *tempty,
                                               volatile int *abort, float *sw, int64_t g_lo, int ntiles, int warp,
-                                              int lane, int etid, bool perm4 = false)
+                                              int lane, int etid)
 {
     const int quarter = warp & 3;
     const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -78,9 +92,10 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
         kmax = 0u;
         knmin = 0u;
     };
-    for (int i = 0; i < ntiles; ++i) {
-        const int64_t g = g_lo + i, b = g / p.tps;
-        const int it = (int)(g - b * p.tps);
+    TileCursor cur(g_lo, p.tps);
+    for (int i = 0; i < ntiles; ++i, cur.next()) {
+        const int64_t b = cur.b;
+        const int it = cur.it;
         if (b != b_cur) {
             flush_range();
             b_cur = b;
@@ -105,11 +120,15 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&tempty[buf]);               // the accumulator may be reused from here
+            float a1 = 0.f, a2 = 0.f, a3 = 0.f;   // four independent chains: the sum is latency-bound otherwise
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
+            for (int jj = 0; jj < 32; jj += 2) {
                 acc = fmaf(wr[jj], fmaxf(v0[jj], 0.f), acc);
-                acc = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), acc);
+                a1 = fmaf(wr[jj + 1], fmaxf(v0[jj + 1], 0.f), a1);
+                a2 = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), a2);
+                a3 = fmaf(wr[33 + jj], fmaxf(v1[jj + 1], 0.f), a3);
             }
+            acc = (acc + a1) + (a2 + a3);
         } else {
             for (int h0 = 0; h0 < p.HI; h0 += 16) {
                 if (h0 + 32 <= p.HI) {
@@ -130,7 +149,7 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
             tc_fence_before();
             mbar_arrive(&tempty[buf]);
         }
-        const int64_t s = (int64_t)it * BM + (perm4 ? 4 * lane + quarter : quarter * 32 + lane);
+        const int64_t s = (int64_t)it * BM + quarter * 32 + lane;
         if (s < p.T) {
             p.scores[b * p.T + s] = acc + 0.0f;
             const uint32_t key = score_key(acc);
@@ -196,9 +215,10 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (ntiles > 0) {
             const uint64_t pol_stream = policy_evict_first();   // k^I is read once per step
             int issued = 0, nseg = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int64_t g = g_lo + i, b = g / p.tps;
-                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+            TileCursor cur(g_lo, p.tps);
+            for (int i = 0; i < ntiles; ++i, cur.next()) {
+                const int64_t b = cur.b;
+                const int it = cur.it, j = (int)(b - b_first);
                 if (i == 0 || it == 0) {   // a new sequence: its q^I into buffer j & 1
                     if (!__all_sync(0xffffffffu, mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status))) break;
                     if (elect_one()) {
@@ -232,9 +252,10 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
             const uint32_t idesc = idesc_bf16(BM, p.HI);
             const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
             int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int64_t g = g_lo + i, b = g / p.tps;
-                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+            TileCursor cur(g_lo, p.tps);
+            for (int i = 0; i < ntiles; ++i, cur.next()) {
+                const int64_t b = cur.b;
+                const int it = cur.it, j = (int)(b - b_first);
                 if (i == 0 || it == 0)
                     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status))) break;
                 const int st = i % p.stages, buf = i % NACC;
@@ -382,9 +403,10 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
             __syncwarp();
             const uint64_t pol_stream = policy_evict_first();
             int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int64_t g = g_lo + i, b = g / p.tps;
-                const int it = (int)(g - b * p.tps), st = i % F4_CST;
+            TileCursor cur(g_lo, p.tps);
+            for (int i = 0; i < ntiles; ++i, cur.next()) {
+                const int64_t b = cur.b;
+                const int it = cur.it, st = i % F4_CST;
                 if (!__all_sync(0xffffffffu, mbar_wait(&cempty[st], ((i / F4_CST) & 1) ^ 1, abort, p.status))) break;
                 if (elect_one()) {
                     mbar_arrive_expect_tx(&cfull[st], c_bytes);
@@ -402,9 +424,10 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
             const uint32_t idesc = idesc_bf16(BM, p.HI);
             const uint64_t dA = sdesc_sw128(smem_u32(sA), 16, 1024), dB = sdesc_sw128(smem_u32(sB), 16, 1024);
             int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int64_t g = g_lo + i, b = g / p.tps;
-                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+            TileCursor cur(g_lo, p.tps);
+            for (int i = 0; i < ntiles; ++i, cur.next()) {
+                const int64_t b = cur.b;
+                const int it = cur.it, j = (int)(b - b_first);
                 if (i == 0 || it == 0)
                     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status))) break;
                 const int buf = i % NACC, ab = i & 1;
@@ -433,9 +456,10 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
     } else {
         // ---------------- converters: thread ctid dequantises entry row ctid of each tile ----------------
         const int nblk = p.dI / 32;                           // scale blocks per row
-        for (int i = 0; i < ntiles; ++i) {
-            const int64_t g = g_lo + i, b = g / p.tps;
-            const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+        TileCursor cur(g_lo, p.tps);
+        for (int i = 0; i < ntiles; ++i, cur.next()) {
+            const int64_t b = cur.b;
+            const int it = cur.it, j = (int)(b - b_first);
             if (i == 0 || it == 0) {
                 // q^I of the new sequence into B operand buffer j & 1 (HI rows x dI), once the MMAs
                 // of the sequence two back are done with it
@@ -520,14 +544,20 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
 // shared memory (64-byte rows, 64-byte swizzle, K = 64 channels per instruction) and one E8M0 scale per
 // 32 channels in TMEM, so nothing is converted and the k^I stream is 68 bytes per entry (64 code bytes,
 // 4 scale bytes). In TMEM the scales of matrix row 32 j + r (r < 32) sit in lane r of every lane
-// quarter, column j, one byte per 32-channel block. The k^I code tile is brought by a three-dimensional
-// tensor map that stores entry 4 r + j of the tile at row 32 j + r; the tile's scales, contiguous in
-// memory (4 bytes per entry), then form the [32 x 16 bytes] matrix that tcgen05.cp replicates into the
-// four quarters as they are. The q^I scales of a sequence (row = head) are gathered by the producer warp
-// into the same arrangement (lane r, column j: head r + 32 j). dI = 128 (two instructions per tile),
-// HI <= 64 (N <= 64), T a multiple of 4.
+// quarter, column j, one byte per 32-channel block: tcgen05.cp replicates a [32 x 16 bytes] matrix whose
+// row r holds the scale words of entries r, r + 32, r + 64, r + 96 into the four quarters.
+// A tile's codes (128 entries x 64 bytes) and scales (4 bytes per entry) are brought by four loader warps
+// with 16- and 4-byte cp.async copies written straight into the MMA's layout: code row t's four 16-byte
+// units at u ^ ((t >> 1) & 3) (the 64-byte swizzle), scale word of entry r + 32 j at row r, column j.
+// The load path keeps many more bytes in flight per SM than the copy engine does for this stream (with
+// tensor-map or bulk copies a tile's issue alone took ~700 cycles and one or two tiles were in flight,
+// about a third of the HBM rate). The q^I scales of a sequence (row = head) are
+// gathered by the producer warp into the same arrangement (lane r, column j: head r + 32 j). dI = 128 (two
+// instructions per tile), HI <= 64 (N <= 64), T a multiple of 4.
 
-constexpr int X4_THREADS = 192;        // warp 0 TMA and q^I scales, warp 1 MMA and scale copies, warps 2-5 epilogue
+constexpr int X4_THREADS = 320;        // warp 0 q^I and its scales, warp 1 MMA and scale copies, warps 2-5
+                                       // epilogue, warps 6-9 k^I loads
+constexpr int X4_INFLIGHT = 8;         // tiles of copies in flight per loader thread (<= X4_STAGES)
 constexpr int X4_STAGES = 12;
 constexpr uint32_t X4_A_BYTES = BM * 64;          // 128 entries x 64 code bytes
 constexpr uint32_t X4_SF_BYTES = 512;             // [32 x 16 bytes] of scales
@@ -536,11 +566,25 @@ constexpr uint32_t X4_SFA_COL = 256, X4_SFB_COL = 272;   // TMEM columns of the 
 struct Mxf4Params {
     ScoreParams sp;
     const uint8_t *qs;                 // q^I scales [B, HI, 4]
+    const uint8_t *kc;                 // k^I codes [B*T, 64], 16-byte aligned
+    const uint8_t *ks;                 // k^I scales [B*T, 4], 16-byte aligned
 };
 
+// Asynchronous global -> shared copies through the load path (cp.async), grouped per commit.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint64_t policy)
+{
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(policy) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __global__ void __launch_bounds__(X4_THREADS, 1)
-decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __grid_constant__ CUtensorMap tm_kc,
-                          const __grid_constant__ CUtensorMap tm_ks, Mxf4Params f)
+decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params f)
 {
     const ScoreParams &p = f.sp;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -566,7 +610,10 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __gri
     constexpr uint32_t tcols = 512;   // accumulators NACC x HI (<= 256) and the scale slots
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < X4_STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < X4_STAGES; ++i) {
+            mbar_init(&full[i], 128);   // every loader thread, once its copies of the tile have landed
+            mbar_init(&empty[i], 1);
+        }
         for (int i = 0; i < NACC; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], EPI_THREADS);
@@ -589,19 +636,15 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __gri
     grid_launch_dependents();   // the top-k may be scheduled as this grid's CTAs finish
 
     if (warp == 0) {
-        // ---------------- producer: code and scale tiles by TMA; q^I and its scales per sequence ----------
+        // ---------------- q^I and its scales, per sequence ----------------
         if (ntiles > 0) {
-            if (elect_one()) {
-                prefetch_tmap(&tm_qc);
-                prefetch_tmap(&tm_kc);
-                prefetch_tmap(&tm_ks);
-            }
+            if (elect_one()) prefetch_tmap(&tm_qc);
             __syncwarp();
-            const uint64_t pol_stream = policy_evict_first();   // k^I is read once per step
-            int issued = 0, nseg = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int64_t g = g_lo + i, b = g / p.tps;
-                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+            int nseg = 0;
+            TileCursor cur(g_lo, p.tps);
+            for (int i = 0; i < ntiles; ++i, cur.next()) {
+                const int64_t b = cur.b;
+                const int it = cur.it, j = (int)(b - b_first);
                 if (i == 0 || it == 0) {
                     if (!__all_sync(0xffffffffu, mbar_wait(&qempty[j & 1], ((j >> 1) & 1) ^ 1, abort, p.status))) break;
                     if (elect_one()) {
@@ -621,27 +664,10 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __gri
                     if (lane == 0) mbar_arrive(&qfull[j & 1]);
                     nseg = j + 1;
                 }
-                const int st = i % X4_STAGES;
-                if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((i / X4_STAGES) & 1) ^ 1, abort, p.status))) break;
-                const int r0 = (int)((b * p.T + (int64_t)it * BM) / 4);   // T % 4 == 0: tiles start on a group of 4
-                if (elect_one()) {
-                    mbar_arrive_expect_tx(&full[st], X4_A_BYTES + X4_SF_BYTES);
-                    asm volatile(
-                        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
-                        "[%0], [%1, {%2, %3, %4}], [%5], %6;"
-                        ::"r"(smem_u32(sA + st * X4_A_BYTES)), "l"(reinterpret_cast<uint64_t>(&tm_kc)), "r"(0), "r"(r0),
-                        "r"(0), "r"(smem_u32(&full[st])), "l"(pol_stream)
-                        : "memory");
-                    tma_load_2d_hint(sSFA + st * X4_SF_BYTES, &tm_ks, &full[st], 0, r0, pol_stream);
-                }
-                __syncwarp();
-                issued = i + 1;
             }
             // never leave with copies in flight into this CTA's shared memory
             for (int j = max(0, nseg - 2); j < nseg; ++j)
                 mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status, 100000000ull);
-            for (int i = max(0, issued - X4_STAGES); i < issued; ++i)
-                mbar_wait(&full[i % X4_STAGES], (i / X4_STAGES) & 1, abort, p.status, 100000000ull);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer: scale copies into TMEM, then two block-scaled MMAs per tile ----------
@@ -649,9 +675,10 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __gri
             const uint32_t id0 = idesc_mxf4(BM, p.HI, 0), id2 = idesc_mxf4(BM, p.HI, 2);
             const uint64_t dA = sdesc_sw64(smem_u32(sA), 512), dB = sdesc_sw64(smem_u32(sB), 512);
             int issued = 0;
-            for (int i = 0; i < ntiles; ++i) {
-                const int64_t g = g_lo + i, b = g / p.tps;
-                const int it = (int)(g - b * p.tps), j = (int)(b - b_first);
+            TileCursor cur(g_lo, p.tps);
+            for (int i = 0; i < ntiles; ++i, cur.next()) {
+                const int64_t b = cur.b;
+                const int it = cur.it, j = (int)(b - b_first);
                 const uint32_t sfb = tmem + X4_SFB_COL + (uint32_t)(j & 1) * 4;
                 if (i == 0 || it == 0) {
                     if (!__all_sync(0xffffffffu, mbar_wait(&qfull[j & 1], (j >> 1) & 1, abort, p.status))) break;
@@ -681,8 +708,51 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, const __gri
             if (issued > 0)
                 mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
         }
+    } else if (warp < 6) {
+        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
     } else {
-        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64, true);
+        // ---------------- loads: each thread one code row of every tile, straight into the swizzled layout ----
+        // Row t's four 16-byte units land at u ^ ((t >> 1) & 3) (the 64-byte swizzle); warp 6 also brings
+        // the scale words, entry r + 32 j to row r, column j. A thread keeps X4_INFLIGHT tiles of its copies in
+        // flight: once the copies of tile i - X4_INFLIGHT + 1 have landed it makes them visible to the tensor
+        // core (proxy fence) and arrives on that tile's barrier. Only the tile's own rows are read (T % 4 == 0),
+        // rows past the sequence's end keep older contents and their scores are not stored.
+        const int t = threadIdx.x - 192;                      // code row = entry of the tile
+        const int rot = (t >> 1) & 3;
+        const uint64_t pol_stream = policy_evict_first();    // k^I is read once per step
+        int issued = 0;
+        TileCursor cur(g_lo, p.tps);
+        for (int i = 0; i < ntiles; ++i, cur.next()) {
+            const int st = i % X4_STAGES;
+            const int64_t b = cur.b;
+            const int it = cur.it;
+            if (!__all_sync(0xffffffffu, mbar_wait(&empty[st], ((i / X4_STAGES) & 1) ^ 1, abort, p.status))) break;
+            const int64_t e0 = b * p.T + (int64_t)it * BM;    // first entry of the tile
+            const int64_t left = p.T - (int64_t)it * BM;
+            const int rows = (int)(left < BM ? left : BM);
+            if (t < rows) {
+                const uint8_t *src = f.kc + (e0 + t) * 64;
+                const uint32_t dst = smem_u32(sA + st * X4_A_BYTES + t * 64);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) cp_async16(dst + (uint32_t)((u ^ rot) << 4), src + u * 16, pol_stream);
+            }
+            if (warp == 6) {
+                const uint32_t dst = smem_u32(sSFA + st * X4_SF_BYTES + lane * 16);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    if (lane + 32 * jj < rows) cp_async4(dst + 4 * jj, f.ks + (e0 + lane + 32 * jj) * 4);
+            }
+            cp_async_commit();
+            issued = i + 1;
+            if (i >= X4_INFLIGHT - 1) {
+                cp_async_wait<X4_INFLIGHT - 1>();
+                fence_async_smem();   // generic-proxy writes, read next by tcgen05.cp / tcgen05.mma
+                mbar_arrive(&full[(i - X4_INFLIGHT + 1) % X4_STAGES]);
+            }
+        }
+        cp_async_wait<0>();   // never leave with copies in flight into this CTA's shared memory
+        fence_async_smem();
+        for (int i = max(0, issued - (X4_INFLIGHT - 1)); i < issued; ++i) mbar_arrive(&full[i % X4_STAGES]);
     }
     tc_fence_before();
     __syncthreads();
@@ -1370,15 +1440,15 @@ cudaError_t launch_decode_index_fp4(const uint8_t *qc, const uint8_t *qs, const 
     CUtensorMap tkc;   // k^I codes as rows of dI/2 bytes, 128-row boxes
     if (!make_tmap_u8_rows(&tkc, kc, (uint64_t)(B * T), (uint64_t)dI / 2, BM)) return cudaErrorInvalidValue;
     if (dI == 128 && HI <= 64 && T % 4 == 0 && (reinterpret_cast<uintptr_t>(qs) & 3u) == 0 &&
-        (reinterpret_cast<uintptr_t>(ks) & 15u) == 0) {
+        (reinterpret_cast<uintptr_t>(ks) & 15u) == 0 && (reinterpret_cast<uintptr_t>(kc) & 15u) == 0) {
         // block-scaled MMA on the MXFP4 operands as they are
-        CUtensorMap tqc, tkc3, tks;
+        CUtensorMap tqc;
         if (!make_tmap_u8_sw64(&tqc, qc, (uint64_t)B * HI, (uint32_t)HI)) return cudaErrorInvalidValue;
-        if (!make_tmap_u8_sw64_perm4(&tkc3, kc, (uint64_t)(B * T))) return cudaErrorInvalidValue;
-        if (!make_tmap_u8_rows(&tks, ks, (uint64_t)(B * T) / 4, 16, 32)) return cudaErrorInvalidValue;
         Mxf4Params x;
         x.sp = score_params(p8, L, w, B, T, HI, dI, status);
         x.qs = qs;
+        x.kc = kc;
+        x.ks = ks;
         const size_t smem = 1024 + X4_STAGES * (size_t)X4_A_BYTES + 2 * 4096 + (X4_STAGES + 2) * (size_t)X4_SF_BYTES +
                             256 * 4 + (2 * X4_STAGES + 2 * NACC + 4 + 2) * 8;
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_mxf4_kernel), smem);
@@ -1386,7 +1456,7 @@ cudaError_t launch_decode_index_fp4(const uint8_t *qc, const uint8_t *qs, const 
         int dev = 0, nsm = 148;
         if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
         const unsigned g1 = (unsigned)std::min<int64_t>(nsm, x.sp.G);
-        decode_scores_mxf4_kernel<<<g1, X4_THREADS, smem, stream>>>(tqc, tkc3, tks, x);
+        decode_scores_mxf4_kernel<<<g1, X4_THREADS, smem, stream>>>(tqc, x);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         return launch_topk_after_scan(p8, L, B, T, k, idx, stream);
     }

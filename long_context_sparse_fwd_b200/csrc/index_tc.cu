@@ -909,23 +909,6 @@ bool make_tmap_u8_sw64(CUtensorMap *map, const void *base, uint64_t rows, uint32
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Three-dimensional view of [rows, 64] bytes (rows a multiple of 4) whose 128-row box lands in shared
-// memory permuted: box row 32 j + r holds source row 4 r + j (r < 32, j < 4) of the tile, with a
-// 64-byte swizzle. Dimensions: bytes (64), r (stride 256 B), j (stride 64 B).
-bool make_tmap_u8_sw64_perm4(CUtensorMap *map, const void *base, uint64_t rows)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (fn == nullptr || rows % 4 != 0) return false;
-    cuuint64_t dims[3] = {64, rows / 4, 4};
-    cuuint64_t strides[2] = {256, 64};
-    cuuint32_t box[3] = {64, 32, 4};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-
 // Shared-memory plan of the fused indexer: every entry in one chunk when the scores of a group's
 // queries fit (two scores buffers when three key stages still fit), else (bf16, k <= 1024) chunks of
 // entries with a running top-k per query, one scores buffer, the chunk as long as shared memory allows.

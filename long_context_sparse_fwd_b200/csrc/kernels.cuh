@@ -55,7 +55,6 @@ bool make_tmap_u8_rows(CUtensorMap *map, const void *base, uint64_t rows, uint64
 // 2-D byte tensor map over [rows, 64], box [box_rows, 64], 64-byte swizzle
 bool make_tmap_u8_sw64(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows);
 // [rows, 64] bytes as 128-row boxes whose shared-memory row 32 j + r is source row 4 r + j, 64-byte swizzle
-bool make_tmap_u8_sw64_perm4(CUtensorMap *map, const void *base, uint64_t rows);
 
 // append.cu: the compressor's decode step (one token per sequence; emits an entry when a window closes)
 struct AppendArgs {

@@ -78,17 +78,21 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
 
 // Bounded wait for the phase with `parity` of `bar`. Gives up when *abort is set by another role or
 // after `limit_ns` of waiting; on a timeout it sets *abort and records CSA_ERR_TIMEOUT in the
-// status word. Returns false when it gave up.
+// status word. Returns false when it gave up. The global timer is first read after 256 failed polls
+// (a read of it is slow, and a wait that ends soon should not pay for one), so the limit counts
+// from there.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *status,
                                           uint64_t limit_ns = 2000000000ull)
 {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+    uint64_t t0 = 0;
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((n & 255u) == 0) {
             if (*abort) return false;
-            if (globaltimer() - t0 > limit_ns) {
+            const uint64_t now = globaltimer();
+            if (n == 256u) {
+                t0 = now;
+            } else if (now - t0 > limit_ns) {
                 *abort = 1;
                 report(status, CSA_ERR_TIMEOUT);
                 return false;
