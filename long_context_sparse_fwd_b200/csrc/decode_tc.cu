@@ -66,6 +66,9 @@ struct TileCursor {
 // Epilogue of the scan (four warps, 128 threads, one TMEM lane quarter each): each thread owns one entry
 // of the tile, reduces its HI heads (w-weighted ReLU) in registers and writes one fp32 score; it also
 // tracks the sequence's key range for the top-k and clears the chunked top-k's counters.
+// NA accumulators in TMEM (tile i in accumulator i % NA); WREG: the index weights of the current sequence
+// are held in registers (else read from shared memory, for a kernel that runs two CTAs per SM).
+template <int NA, bool WREG>
 __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tmem, uint64_t *tfull, uint64_t *tempty,
                                               volatile int *abort, float *sw, int64_t g_lo, int ntiles, int warp,
                                               int lane, int etid)
@@ -74,7 +77,7 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
     const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16);
     for (int64_t i = (int64_t)blockIdx.x * EPI_THREADS + etid; i < p.zero_n16; i += (int64_t)gridDim.x * EPI_THREADS)
         p.zero[i] = make_uint4(0u, 0u, 0u, 0u);
-    float wr[64];   // index weights of the current sequence (HI == 64 keeps them in registers)
+    float wr[WREG ? 64 : 1];   // index weights of the current sequence (HI == 64 keeps them in registers)
     // range of the score keys of the current sequence seen by this thread, merged into the
     // sequence's global range (for the top-k's histogram) whenever the sequence changes
     uint32_t kmax = 0u, knmin = 0u;
@@ -104,13 +107,13 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
             named_barrier_sync(1, EPI_THREADS);
             for (int h = etid; h < p.HI; h += EPI_THREADS) sw[h] = p.w[b * p.HI + h];
             named_barrier_sync(1, EPI_THREADS);
-            if (p.HI == 64) {
+            if (WREG && p.HI == 64) {
 #pragma unroll
-                for (int h = 0; h < 64; ++h) wr[h] = sw[h];
+                for (int h = 0; h < (WREG ? 64 : 1); ++h) wr[h] = sw[h];
             }
         }
-        const int buf = i % NACC;
-        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i / NACC) & 1, abort, p.status))) break;
+        const int buf = i % NA;
+        if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], (i / NA) & 1, abort, p.status))) break;
         tc_fence_after();
         float acc = 0.f;
         if (p.HI == 64) {
@@ -121,12 +124,24 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
             tc_fence_before();
             mbar_arrive(&tempty[buf]);               // the accumulator may be reused from here
             float a1 = 0.f, a2 = 0.f, a3 = 0.f;   // four independent chains: the sum is latency-bound otherwise
+            if constexpr (WREG) {
 #pragma unroll
-            for (int jj = 0; jj < 32; jj += 2) {
-                acc = fmaf(wr[jj], fmaxf(v0[jj], 0.f), acc);
-                a1 = fmaf(wr[jj + 1], fmaxf(v0[jj + 1], 0.f), a1);
-                a2 = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), a2);
-                a3 = fmaf(wr[33 + jj], fmaxf(v1[jj + 1], 0.f), a3);
+                for (int jj = 0; jj < 32; jj += 2) {
+                    acc = fmaf(wr[jj], fmaxf(v0[jj], 0.f), acc);
+                    a1 = fmaf(wr[jj + 1], fmaxf(v0[jj + 1], 0.f), a1);
+                    a2 = fmaf(wr[32 + jj], fmaxf(v1[jj], 0.f), a2);
+                    a3 = fmaf(wr[33 + jj], fmaxf(v1[jj + 1], 0.f), a3);
+                }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 32; jj += 2) {
+                    const float2 w0 = *reinterpret_cast<const float2 *>(sw + jj);
+                    const float2 w1 = *reinterpret_cast<const float2 *>(sw + 32 + jj);
+                    acc = fmaf(w0.x, fmaxf(v0[jj], 0.f), acc);
+                    a1 = fmaf(w0.y, fmaxf(v0[jj + 1], 0.f), a1);
+                    a2 = fmaf(w1.x, fmaxf(v1[jj], 0.f), a2);
+                    a3 = fmaf(w1.y, fmaxf(v1[jj + 1], 0.f), a3);
+                }
             }
             acc = (acc + a1) + (a2 + a3);
         } else {
@@ -163,7 +178,7 @@ __device__ __forceinline__ void scan_epilogue(const ScoreParams &p, uint32_t tme
 // Persistent: CTA c takes the contiguous tile range [c*G/n, (c+1)*G/n) of the flat list
 // (sequence-major, 128 entries per tile), so the HBM stream never idles on a wave tail. q^I of the
 // current sequence is double-buffered; a range crosses at most a few sequence boundaries.
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, 2)
 decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         ScoreParams p)
 {
@@ -280,7 +295,7 @@ decode_scores_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
                 mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
         }
     } else {
-        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
+        scan_epilogue<NACC, false>(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
     }
     tc_fence_before();
     __syncthreads();
@@ -452,7 +467,7 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
                 mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
         }
     } else if (warp < F4_CONV0) {
-        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
+        scan_epilogue<NACC, true>(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
     } else {
         // ---------------- converters: thread ctid dequantises entry row ctid of each tile ----------------
         const int nblk = p.dI / 32;                           // scale blocks per row
@@ -555,13 +570,18 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
 // gathered by the producer warp into the same arrangement (lane r, column j: head r + 32 j). dI = 128 (two
 // instructions per tile), HI <= 64 (N <= 64), T a multiple of 4.
 
-constexpr int X4_THREADS = 320;        // warp 0 q^I and its scales, warp 1 MMA and scale copies, warps 2-5
-                                       // epilogue, warps 6-9 k^I loads
-constexpr int X4_INFLIGHT = 8;         // tiles of copies in flight per loader thread (<= X4_STAGES)
-constexpr int X4_STAGES = 12;
+// Two CTAs per SM (two independent tile pipelines): 256 threads and at most 128 registers each, about 96 KB
+// of shared memory and 256 TMEM columns per CTA.
+constexpr int X4_THREADS = 256;        // warp 0 q^I and its scales, warp 1 MMA and scale copies, warps 2-5
+                                       // epilogue, warps 6-7 k^I loads (two code rows per thread)
+constexpr int X4_LOADERS = 64;
+constexpr int X4_INFLIGHT = 7;         // tiles of copies in flight per loader thread (<= X4_STAGES)
+constexpr int X4_STAGES = 10;
+constexpr int X4_NACC = 3;             // TMEM accumulators (64 columns each)
 constexpr uint32_t X4_A_BYTES = BM * 64;          // 128 entries x 64 code bytes
 constexpr uint32_t X4_SF_BYTES = 512;             // [32 x 16 bytes] of scales
-constexpr uint32_t X4_SFA_COL = 256, X4_SFB_COL = 272;   // TMEM columns of the scale slots (4 each)
+constexpr uint32_t X4_SFA_COL = 192, X4_SFB_COL = 208;   // TMEM columns of the scale slots (4 each)
+constexpr uint32_t X4_TMEM_COLS = 256;
 
 struct Mxf4Params {
     ScoreParams sp;
@@ -583,7 +603,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(X4_THREADS, 1)
+__global__ void __launch_bounds__(X4_THREADS, 2)
 decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params f)
 {
     const ScoreParams &p = f.sp;
@@ -597,8 +617,8 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params 
     float *sw = reinterpret_cast<float *>(sSFB + 2 * X4_SF_BYTES);   // [256]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sw + 256);
     uint64_t *full = bars, *empty = bars + X4_STAGES;             // [X4_STAGES]
-    uint64_t *tfull = bars + 2 * X4_STAGES, *tempty = tfull + NACC;   // [NACC]
-    uint64_t *qfull = tempty + NACC, *qempty = qfull + 2;         // [2]
+    uint64_t *tfull = bars + 2 * X4_STAGES, *tempty = tfull + X4_NACC;   // [X4_NACC]
+    uint64_t *qfull = tempty + X4_NACC, *qempty = qfull + 2;      // [2]
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(qempty + 2);
     volatile int *abort = reinterpret_cast<volatile int *>(qempty + 3);
 
@@ -607,14 +627,14 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params 
     const int64_t g_hi = (int64_t)(blockIdx.x + 1) * p.G / gridDim.x;
     const int ntiles = (int)(g_hi - g_lo);
     const int64_t b_first = g_lo / p.tps;
-    constexpr uint32_t tcols = 512;   // accumulators NACC x HI (<= 256) and the scale slots
+    constexpr uint32_t tcols = X4_TMEM_COLS;   // accumulators X4_NACC x HI (HI <= 64) and the scale slots
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < X4_STAGES; ++i) {
-            mbar_init(&full[i], 128);   // every loader thread, once its copies of the tile have landed
+            mbar_init(&full[i], X4_LOADERS);   // every loader thread, once its copies of the tile have landed
             mbar_init(&empty[i], 1);
         }
-        for (int i = 0; i < NACC; ++i) {
+        for (int i = 0; i < X4_NACC; ++i) {
             mbar_init(&tfull[i], 1);
             mbar_init(&tempty[i], EPI_THREADS);
         }
@@ -686,8 +706,8 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params 
                     if (elect_one()) tmem_cp_32x128b_x4(sfb, sdesc_plain(smem_u32(sSFB + (j & 1) * X4_SF_BYTES), 16, 128));
                     __syncwarp();
                 }
-                const int st = i % X4_STAGES, buf = i % NACC;
-                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((i / NACC) & 1) ^ 1, abort, p.status))) break;
+                const int st = i % X4_STAGES, buf = i % X4_NACC;
+                if (!__all_sync(0xffffffffu, mbar_wait(&tempty[buf], ((i / X4_NACC) & 1) ^ 1, abort, p.status))) break;
                 if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / X4_STAGES) & 1, abort, p.status))) break;
                 tc_fence_after();
                 const uint32_t sfa = tmem + X4_SFA_COL + (uint32_t)buf * 4;
@@ -706,19 +726,18 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params 
                 issued = i + 1;
             }
             if (issued > 0)
-                mbar_wait(&tfull[(issued - 1) % NACC], ((issued - 1) / NACC) & 1, abort, p.status, 100000000ull);
+                mbar_wait(&tfull[(issued - 1) % X4_NACC], ((issued - 1) / X4_NACC) & 1, abort, p.status, 100000000ull);
         }
     } else if (warp < 6) {
-        scan_epilogue(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
+        scan_epilogue<X4_NACC, false>(p, tmem, tfull, tempty, abort, sw, g_lo, ntiles, warp, lane, threadIdx.x - 64);
     } else {
-        // ---------------- loads: each thread one code row of every tile, straight into the swizzled layout ----
-        // Row t's four 16-byte units land at u ^ ((t >> 1) & 3) (the 64-byte swizzle); warp 6 also brings
+        // ---------------- loads: each thread two code rows of every tile, straight into the swizzled layout ---
+        // Row r's four 16-byte units land at u ^ ((r >> 1) & 3) (the 64-byte swizzle); warp 6 also brings
         // the scale words, entry r + 32 j to row r, column j. A thread keeps X4_INFLIGHT tiles of its copies in
         // flight: once the copies of tile i - X4_INFLIGHT + 1 have landed it makes them visible to the tensor
         // core (proxy fence) and arrives on that tile's barrier. Only the tile's own rows are read (T % 4 == 0),
         // rows past the sequence's end keep older contents and their scores are not stored.
-        const int t = threadIdx.x - 192;                      // code row = entry of the tile
-        const int rot = (t >> 1) & 3;
+        const int t = threadIdx.x - 192;                      // code rows t and t + 64 (= entries of the tile)
         const uint64_t pol_stream = policy_evict_first();    // k^I is read once per step
         int issued = 0;
         TileCursor cur(g_lo, p.tps);
@@ -730,11 +749,15 @@ decode_scores_mxf4_kernel(const __grid_constant__ CUtensorMap tm_qc, Mxf4Params 
             const int64_t e0 = b * p.T + (int64_t)it * BM;    // first entry of the tile
             const int64_t left = p.T - (int64_t)it * BM;
             const int rows = (int)(left < BM ? left : BM);
-            if (t < rows) {
-                const uint8_t *src = f.kc + (e0 + t) * 64;
-                const uint32_t dst = smem_u32(sA + st * X4_A_BYTES + t * 64);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) cp_async16(dst + (uint32_t)((u ^ rot) << 4), src + u * 16, pol_stream);
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = t + rr * X4_LOADERS, rot = (r >> 1) & 3;
+                if (r < rows) {
+                    const uint8_t *src = f.kc + (e0 + r) * 64;
+                    const uint32_t dst = smem_u32(sA + st * X4_A_BYTES + r * 64);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) cp_async16(dst + (uint32_t)((u ^ rot) << 4), src + u * 16, pol_stream);
+                }
             }
             if (warp == 6) {
                 const uint32_t dst = smem_u32(sSFA + st * X4_SF_BYTES + lane * 16);
@@ -1412,13 +1435,17 @@ cudaError_t launch_decode_index_tc(const uint16_t *qI, const float *w, const uin
     ScoreParams sp = score_params(p8, L, w, B, T, HI, dI, status);
     const size_t a_bytes = (size_t)(dI / 64) * BM * 128;
     const size_t fixed = 1024 + 2 * (size_t)(dI / 64) * HI * 128 + 256 * 4 + 256;
-    sp.stages = (int)std::min<size_t>(MAX_STAGES, (227 * 1024 - fixed) / a_bytes);
+    // Two CTAs per SM (two independent tile pipelines) when two stages of each still fit in half of
+    // shared memory and the accumulators in half of TMEM; else one CTA with as many stages as fit.
+    const size_t half_smem = 113 * 1024;
+    const bool two = (int64_t)HI * NACC <= 256 && fixed + 2 * a_bytes <= half_smem;
+    sp.stages = (int)std::min<size_t>(MAX_STAGES, ((two ? half_smem : 227 * 1024) - fixed) / a_bytes);
     const size_t smem = fixed + (size_t)sp.stages * a_bytes;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_tc_kernel), smem);
     if (e != cudaSuccess) return e;
     int dev = 0, nsm = 148;
     if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
-    const unsigned g1 = (unsigned)std::min<int64_t>(nsm, sp.G);
+    const unsigned g1 = (unsigned)std::min<int64_t>((two ? 2 : 1) * (int64_t)nsm, sp.G);
     decode_scores_tc_kernel<<<g1, NUM_THREADS, smem, stream>>>(tq, tk, sp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return launch_topk_after_scan(p8, L, B, T, k, idx, stream);
@@ -1450,12 +1477,12 @@ cudaError_t launch_decode_index_fp4(const uint8_t *qc, const uint8_t *qs, const 
         x.kc = kc;
         x.ks = ks;
         const size_t smem = 1024 + X4_STAGES * (size_t)X4_A_BYTES + 2 * 4096 + (X4_STAGES + 2) * (size_t)X4_SF_BYTES +
-                            256 * 4 + (2 * X4_STAGES + 2 * NACC + 4 + 2) * 8;
+                            256 * 4 + (2 * X4_STAGES + 2 * X4_NACC + 4 + 2) * 8;
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void *>(decode_scores_mxf4_kernel), smem);
         if (e != cudaSuccess) return e;
         int dev = 0, nsm = 148;
         if ((e = current_device_sms(&dev, &nsm)) != cudaSuccess) return e;
-        const unsigned g1 = (unsigned)std::min<int64_t>(nsm, x.sp.G);
+        const unsigned g1 = (unsigned)std::min<int64_t>(2 * (int64_t)nsm, x.sp.G);   // two CTAs per SM
         decode_scores_mxf4_kernel<<<g1, X4_THREADS, smem, stream>>>(tqc, x);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         return launch_topk_after_scan(p8, L, B, T, k, idx, stream);
