@@ -880,32 +880,45 @@ bool attend_tc_supported(int H, int D, int r, int k)
 // Combine the split partials of decode: per (sequence, head), o = sum_i 2^(m_i - M) O_i / L with
 // L = 2^(z - M) + sum_i 2^(m_i - M) l_i and M the largest of the split maxima and the sink z (all in
 // the log2 domain). The sink enters here exactly once.
+constexpr int COMBINE_MAX = 16;   // the most splits a decode call uses (HCA decode)
+
 __global__ void __launch_bounds__(128)
 combine_splits_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml, const float *__restrict__ sinks,
                       int nsplit, float *__restrict__ o)
 {
     const int64_t b = blockIdx.x / HH;
     const int h = blockIdx.x % HH;
-    grid_dependency_wait();   // the split partials
     const float z = sinks[h] * 1.4426950408889634f;
-    float M = z;
-    for (int i = 0; i < nsplit; ++i) {
-        const float mi = part_ml[((b * nsplit + i) * HH + h) * 2];
-        M = fmaxf(M, mi);
+    grid_dependency_wait();   // the split partials
+    // Every split's (max, sum) and partial row are loaded at once (at most COMBINE_MAX splits). An empty split's
+    // row was never written: it is left out by a select, so whatever the memory holds never reaches the sum.
+    float mi[COMBINE_MAX], li[COMBINE_MAX];
+    float4 v[COMBINE_MAX];
+#pragma unroll
+    for (int i = 0; i < COMBINE_MAX; ++i) {
+        if (i < nsplit) {
+            const int64_t r = (b * nsplit + i) * HH + h;
+            mi[i] = part_ml[r * 2];
+            li[i] = part_ml[r * 2 + 1];
+            v[i] = reinterpret_cast<const float4 *>(part_o + r * (int64_t)DD)[threadIdx.x];
+        }
     }
+    float M = z;
+#pragma unroll
+    for (int i = 0; i < COMBINE_MAX; ++i)
+        if (i < nsplit) M = fmaxf(M, mi[i]);
     float L = (z == -INFINITY) ? 0.f : exp2f(z - M);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < nsplit; ++i) {
-        const float mi = part_ml[((b * nsplit + i) * HH + h) * 2];
-        const float li = part_ml[((b * nsplit + i) * HH + h) * 2 + 1];
-        if (mi == -INFINITY || li == 0.f) continue;   // empty split: its O was never written
-        const float wgt = exp2f(mi - M);
-        L += wgt * li;
-        const float4 v = reinterpret_cast<const float4 *>(part_o + ((b * nsplit + i) * HH + h) * (int64_t)DD)[threadIdx.x];
-        acc.x += wgt * v.x;
-        acc.y += wgt * v.y;
-        acc.z += wgt * v.z;
-        acc.w += wgt * v.w;
+#pragma unroll
+    for (int i = 0; i < COMBINE_MAX; ++i) {
+        if (i < nsplit && mi[i] != -INFINITY && li[i] != 0.f) {
+            const float wgt = exp2f(mi[i] - M);
+            L += wgt * li[i];
+            acc.x += wgt * v[i].x;
+            acc.y += wgt * v[i].y;
+            acc.z += wgt * v[i].z;
+            acc.w += wgt * v[i].w;
+        }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
     reinterpret_cast<float4 *>(o + (b * HH + h) * (int64_t)DD)[threadIdx.x] =
@@ -990,6 +1003,7 @@ cudaError_t launch_attend_tc_decode(const AttnArgs &x, int nsplit, float *part, 
 {
     if (x.R == 0) return cudaSuccess;
     if (nsplit <= 1) return launch_tc(x, 1, x.o, nullptr, stream);
+    if (nsplit > COMBINE_MAX) return cudaErrorInvalidValue;
     float *part_o = part;
     float *part_ml = part + (size_t)x.R * nsplit * HH * DD;
     cudaError_t e = launch_tc(x, nsplit, part_o, part_ml, stream);
