@@ -882,6 +882,8 @@ bool attend_tc_supported(int H, int D, int r, int k)
 // the log2 domain). The sink enters here exactly once.
 constexpr int COMBINE_MAX = 16;   // the most splits a decode call uses (HCA decode)
 
+// NMAX: the most splits this instance takes (its registers hold one row of each).
+template <int NMAX>
 __global__ void __launch_bounds__(128)
 combine_splits_kernel(const float *__restrict__ part_o, const float *__restrict__ part_ml, const float *__restrict__ sinks,
                       int nsplit, float *__restrict__ o)
@@ -890,12 +892,12 @@ combine_splits_kernel(const float *__restrict__ part_o, const float *__restrict_
     const int h = blockIdx.x % HH;
     const float z = sinks[h] * 1.4426950408889634f;
     grid_dependency_wait();   // the split partials
-    // Every split's (max, sum) and partial row are loaded at once (at most COMBINE_MAX splits). An empty split's
+    // Every split's (max, sum) and partial row are loaded at once (at most NMAX splits). An empty split's
     // row was never written: it is left out by a select, so whatever the memory holds never reaches the sum.
-    float mi[COMBINE_MAX], li[COMBINE_MAX];
-    float4 v[COMBINE_MAX];
+    float mi[NMAX], li[NMAX];
+    float4 v[NMAX];
 #pragma unroll
-    for (int i = 0; i < COMBINE_MAX; ++i) {
+    for (int i = 0; i < NMAX; ++i) {
         if (i < nsplit) {
             const int64_t r = (b * nsplit + i) * HH + h;
             mi[i] = part_ml[r * 2];
@@ -905,12 +907,12 @@ combine_splits_kernel(const float *__restrict__ part_o, const float *__restrict_
     }
     float M = z;
 #pragma unroll
-    for (int i = 0; i < COMBINE_MAX; ++i)
+    for (int i = 0; i < NMAX; ++i)
         if (i < nsplit) M = fmaxf(M, mi[i]);
     float L = (z == -INFINITY) ? 0.f : exp2f(z - M);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < COMBINE_MAX; ++i) {
+    for (int i = 0; i < NMAX; ++i) {
         if (i < nsplit && mi[i] != -INFINITY && li[i] != 0.f) {
             const float wgt = exp2f(mi[i] - M);
             L += wgt * li[i];
@@ -1008,8 +1010,14 @@ cudaError_t launch_attend_tc_decode(const AttnArgs &x, int nsplit, float *part, 
     float *part_ml = part + (size_t)x.R * nsplit * HH * DD;
     cudaError_t e = launch_tc(x, nsplit, part_o, part_ml, stream);
     if (e != cudaSuccess) return e;
-    return launch_dependent(combine_splits_kernel, dim3((unsigned)(x.R * HH)), dim3(128), 0, stream,
-                            (const float *)part_o, (const float *)part_ml, x.sinks, nsplit, x.o);
+    auto combine = [&](auto kern) {
+        return launch_dependent(kern, dim3((unsigned)(x.R * HH)), dim3(128), 0, stream, (const float *)part_o,
+                                (const float *)part_ml, x.sinks, nsplit, x.o);
+    };
+    if (nsplit <= 2) return combine(combine_splits_kernel<2>);
+    if (nsplit <= 4) return combine(combine_splits_kernel<4>);
+    if (nsplit <= 8) return combine(combine_splits_kernel<8>);
+    return combine(combine_splits_kernel<COMBINE_MAX>);
 }
 
 }  // namespace csa
