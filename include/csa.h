@@ -294,7 +294,10 @@ CSA_API csa_status csa_out_proj(const void *o, const void *wa, const void *wb, i
  *   qI_codes [B, HI, dI/2], qI_scales [B, HI, dI/32], kI_codes [B, T, dI/2], kI_scales [B, T, dI/32];
  *   the index scores are the indexer formula on the dequantised values (exact products, fp32
  *   accumulation); everything else is csa_decode's. Requires dI of 64 or 128 and HI of 16, 32, 64 or
- *   128; workspace as csa_decode (csa_workspace_size(CSA_OP_DECODE)). */
+ *   128; workspace as csa_decode (csa_workspace_size(CSA_OP_DECODE)). With dI = 128, HI <= 64, T a
+ *   multiple of 4, 16-byte aligned kI_codes and kI_scales and 4-byte aligned qI_scales the scores come
+ *   from the block-scaled tensor-core MMA on the codes as stored; other shapes dequantise each tile to
+ *   bf16 in shared memory first (the same scores). */
 CSA_API csa_status csa_quantize_mxfp4(const void *x, int64_t rows, int32_t cols, uint8_t *codes, uint8_t *scales,
                               void *stream);
 

@@ -561,14 +561,13 @@ decode_scores_fp4_kernel(const __grid_constant__ CUtensorMap tm_kc, Fp4Params f)
 // 4 scale bytes). In TMEM the scales of matrix row 32 j + r (r < 32) sit in lane r of every lane
 // quarter, column j, one byte per 32-channel block: tcgen05.cp replicates a [32 x 16 bytes] matrix whose
 // row r holds the scale words of entries r, r + 32, r + 64, r + 96 into the four quarters.
-// A tile's codes (128 entries x 64 bytes) and scales (4 bytes per entry) are brought by four loader warps
+// A tile's codes (128 entries x 64 bytes) and scales (4 bytes per entry) are brought by two loader warps
 // with 16- and 4-byte cp.async copies written straight into the MMA's layout: code row t's four 16-byte
 // units at u ^ ((t >> 1) & 3) (the 64-byte swizzle), scale word of entry r + 32 j at row r, column j.
-// The load path keeps many more bytes in flight per SM than the copy engine does for this stream (with
-// tensor-map or bulk copies a tile's issue alone took ~700 cycles and one or two tiles were in flight,
-// about a third of the HBM rate). The q^I scales of a sequence (row = head) are
-// gathered by the producer warp into the same arrangement (lane r, column j: head r + 32 j). dI = 128 (two
-// instructions per tile), HI <= 64 (N <= 64), T a multiple of 4.
+// The roles hand each tile over through mbarriers, and with one CTA per SM every role advanced at the pace
+// of those handovers rather than of the stream: two CTAs run on each SM, each a pipeline of its own. The q^I
+// scales of a sequence (row = head) are gathered by the producer warp into the same arrangement (lane r,
+// column j: head r + 32 j). dI = 128 (two instructions per tile), HI <= 64 (N <= 64), T a multiple of 4.
 
 // Two CTAs per SM (two independent tile pipelines): 256 threads and at most 128 registers each, about 96 KB
 // of shared memory and 256 TMEM columns per CTA.
