@@ -378,6 +378,13 @@ def test_decode_fp8_ctx1m():
     _decode_check(WORKLOADS[4], batch=None, seqs=[0, 7])
 
 
+@pytest.mark.parametrize("batch", [37, 20])
+def test_decode_split_counts(batch):
+    """Batches that spread each sequence's key blocks over 4 and 7 CTAs (148 / B splits), so the split combine
+    runs its 4- and 8-row instances; selections and outputs against the oracle on sampled sequences."""
+    _decode_check(WORKLOADS[3].with_(ctx=4 * 4096 + 3), batch=batch, seqs=[0, batch // 2, batch - 1])
+
+
 def test_decode_short_history():
     """P < W-1: window rows at negative positions are ignored; k > T pads with -1."""
     wl = WORKLOADS[3].with_(ctx=40, topk=16, W=128)
